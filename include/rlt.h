@@ -1,0 +1,246 @@
+/*
+ * rlt.h -- C ABI of the B200 (sm_100a) Recurrent Looped Transformer decoder.
+ *
+ * Page key used in the citations below:
+ *   [RLT-96] "RLT Runs 96 Blocks Per Token With Recurrent State, No Resets"
+ *            (aimastery.page)
+ *   [RLT-TC] "Recurrent Looped Transformer (RLT): prompts in parallel, depth in
+ *            sequence" (thakicloud.com)
+ *   [RLT-FT] "Recurrent Looped Transformer debunked" (flowtivity.ai)
+ *   [RLT-PV] "Per-token recurrence, no quality gain" (news.promtvault.app)
+ *
+ * The model: a causal encoder turns every known token into e_t and projects
+ * the prefix-restricted key/value memory M<=t, shared by all decoder layers
+ * (G = 1) or one per decoder layer (G = L_D) ([RLT-96] "Architecture: encoder
+ * memory meets recurrent decoder"). A recurrent decoder carries the state
+ * H_t = (s_t, C_t^D): s_t the final decoder output vector, C_t^D the retained
+ * sliding-window keys/values of every decoder layer, W - 1 of them since the
+ * window W includes the current token. Each transition H_{t-1} -> H_t runs a
+ * gated merge of e_t with s_{t-1} (feedback scale alpha), then per decoder
+ * block causal SWA, cross-attention to M<=t and an FFN (same section). The
+ * state starts from the learned s* and an empty cache and is never reset at
+ * the prompt/response boundary ([RLT-TC] "What is this technology").
+ * Independent sequences share one batched step ([RLT-96] "Three design
+ * principles and their caveats", model-hardware co-design).
+ *
+ * Conventions for every call:
+ *   - Every call returns an rlt_status (RLT_OK = 0) unless stated otherwise.
+ *   - Arguments are validated completely on the host before anything is
+ *     enqueued: a call that returns an error changed no state.
+ *   - Device work is enqueued asynchronously on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream). Host pointers named h_* are read
+ *     before the call returns.
+ *   - The library allocates no device memory: all device state lives in the
+ *     caller's arena (rlt_arena_bytes), owned by the caller.
+ *   - One model is driven from one host thread at a time.
+ *   - Matrices are row-major [out][in] (y = W x). The q/k/v projection stacks
+ *     rows q | k | v; head h owns entries h*dh .. h*dh + dh - 1 of each.
+ */
+#ifndef RLT_H
+#define RLT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RLT_API __attribute__((visibility("default")))
+#define RLT_MAX_LAYERS 64
+
+typedef struct CUstream_st *rlt_stream; /* the same type as cudaStream_t */
+typedef struct rlt_model rlt_model;     /* opaque; host memory only */
+
+typedef enum rlt_status {
+  RLT_OK = 0,
+  RLT_ERR_INVALID_ARG = 1,  /* null pointer, bad size, id out of range */
+  RLT_ERR_UNSUPPORTED = 2,  /* shape the kernels do not cover */
+  RLT_ERR_NOT_READY = 3,    /* t_dec >= t_enc: e_t / M<=t not produced yet */
+  RLT_ERR_CAPACITY = 4,     /* position or arena capacity exceeded */
+  RLT_ERR_DUPLICATE_ID = 5, /* a sequence listed twice in one batch */
+  RLT_ERR_CUDA = 6,         /* a CUDA runtime call failed */
+  RLT_ERR_TIMEOUT = 7,      /* a bounded device wait gave up */
+  RLT_ERR_DEVICE = 8        /* a kernel's own bounds check fired */
+} rlt_status;
+
+enum { RLT_GELU = 0, RLT_SWIGLU = 1 }; /* FFN form */
+enum { RLT_F32 = 0, RLT_BF16 = 1 };    /* storage of matrices, K/V, e, M */
+
+/* Model shape and capacity. [RLT-96] "Architecture" names d-independent
+ * quantities W (window, includes the current token) and G (memory groups). */
+typedef struct rlt_config {
+  int d;            /* model width; d = n_heads * head_dim */
+  int n_heads;      /* heads of self- and cross-attention */
+  int head_dim;     /* 16, 32, 64 or 128 */
+  int n_enc_layers; /* L_E */
+  int n_dec_layers; /* L_D */
+  int ffn_dim;      /* F */
+  int ffn_kind;     /* RLT_GELU: W2 GELU(W1 u); RLT_SWIGLU: W2 (SiLU(Wa u) * Wb u) */
+  int vocab;        /* V */
+  int window;       /* W >= 1 */
+  int mem_groups;   /* G: 1 or n_dec_layers */
+  int tied;         /* 1: decoder layer l uses encoder layer l's q/k/v, o and
+                       FFN matrices ([RLT-96] "Architecture", tied config) */
+  int dtype;        /* RLT_F32 or RLT_BF16 */
+  int max_seqs;     /* sequence slots in the arena */
+  int max_len;      /* positions per sequence (encoder memory capacity) */
+  int max_prefill_tokens; /* encoder work buffer, tokens; 0 = automatic */
+  float alpha;      /* feedback scale of the gated merge; 0 turns feedback off */
+  float rms_eps;    /* RMSNorm epsilon (1e-6) */
+  float rope_theta; /* rotary base (1e4) */
+} rlt_config;
+
+/* Borrowed device pointers, alive until rlt_destroy. Matrices are in the
+ * model dtype; norm gains, gate bias and s* are always float32.
+ *   embed [V][d]
+ *   enc_ln1/enc_ln2 [d], enc_wqkv [3d][d], enc_wo [d][d],
+ *   enc_w1 [F][d] (GELU W1, or SwiGLU Wa), enc_wb [F][d] (SwiGLU Wb, else
+ *   unused), enc_w2 [d][F], enc_lnf [d]
+ *   mem_wk/mem_wv [d][d] per group
+ *   gate_w [d][2d] (columns 0..d-1 multiply e_t, d..2d-1 multiply s_{t-1}),
+ *   gate_b [d], sstar [d]
+ *   dec_ln1/ln2/ln3 [d], dec_wqkv, dec_wo, dec_wqx [d][d], dec_wox [d][d],
+ *   dec_w1, dec_wb, dec_w2 as in the encoder (ignored when tied), dec_lnf [d]
+ */
+typedef struct rlt_weights {
+  const void *embed;
+  const void *enc_ln1[RLT_MAX_LAYERS], *enc_wqkv[RLT_MAX_LAYERS],
+      *enc_wo[RLT_MAX_LAYERS], *enc_ln2[RLT_MAX_LAYERS],
+      *enc_w1[RLT_MAX_LAYERS], *enc_wb[RLT_MAX_LAYERS], *enc_w2[RLT_MAX_LAYERS];
+  const void *enc_lnf;
+  const void *mem_wk[RLT_MAX_LAYERS], *mem_wv[RLT_MAX_LAYERS];
+  const void *gate_w, *gate_b, *sstar;
+  const void *dec_ln1[RLT_MAX_LAYERS], *dec_wqkv[RLT_MAX_LAYERS],
+      *dec_wo[RLT_MAX_LAYERS], *dec_ln2[RLT_MAX_LAYERS],
+      *dec_wqx[RLT_MAX_LAYERS], *dec_wox[RLT_MAX_LAYERS],
+      *dec_ln3[RLT_MAX_LAYERS], *dec_w1[RLT_MAX_LAYERS],
+      *dec_wb[RLT_MAX_LAYERS], *dec_w2[RLT_MAX_LAYERS];
+  const void *dec_lnf;
+} rlt_weights;
+
+/* Host only. RLT_OK if the kernels cover `cfg`; else why not. */
+RLT_API int rlt_check_config(const rlt_config *cfg);
+
+/* Host only. Bytes of device arena rlt_create needs for `cfg` (0 if the
+ * config is invalid). The arena holds s, the ring KV cache, e, M, positions
+ * and all work buffers. */
+RLT_API size_t rlt_arena_bytes(const rlt_config *cfg);
+
+/* Bind a model to weights and an arena (>= rlt_arena_bytes, 256-byte
+ * aligned device memory owned by the caller). Runs set-up kernels on the
+ * legacy default stream and waits for them; every sequence slot starts reset.
+ * *out receives a host handle released by rlt_destroy. */
+RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *weights,
+                       void *d_arena, size_t arena_bytes, rlt_model **out);
+
+/* Release the host handle (not the arena, not the weights). NULL is a no-op. */
+RLT_API void rlt_destroy(rlt_model *model);
+
+/* Slot `seq`: s <- s*, empty cache, t_dec = t_enc = 0 ([RLT-96]
+ * "Architecture": start state and empty cache before the first token). */
+RLT_API int rlt_reset_seq(rlt_model *model, int seq, rlt_stream stream);
+
+/* Causal encoder + memory projection over whole sequences from position 0
+ * ([RLT-96] "Architecture"; [RLT-TC] "What is this technology": token-
+ * parallel prefill). Sequence h_seq_ids[i] gets tokens
+ * tokens[h_offsets[i] .. h_offsets[i] + h_lengths[i]) (int32; `tokens` may be
+ * a device pointer or pinned host memory). Sets t_enc = length and resets the
+ * decoder state of those slots (s*, empty cache, t_dec = 0).
+ * Errors: INVALID_ARG (ids, offsets, token values are not checked on the host
+ * but out-of-range tokens set RLT_ERR_DEVICE), DUPLICATE_ID, CAPACITY
+ * (length > max_len). */
+RLT_API int rlt_prefill_encoder(rlt_model *model, const int32_t *tokens,
+                                const int32_t *h_seq_ids,
+                                const int32_t *h_offsets,
+                                const int32_t *h_lengths, int n,
+                                rlt_stream stream);
+
+/* One transition H_{t-1} -> H_t for each listed sequence, batched into one
+ * step (t = that sequence's own t_dec). Errors: INVALID_ARG, DUPLICATE_ID,
+ * NOT_READY (t_dec >= t_enc), CAPACITY (t_dec >= max_len). */
+RLT_API int rlt_decoder_step(rlt_model *model, const int32_t *h_ready_ids,
+                             int n_ready, rlt_stream stream);
+
+/* n_steps lock-step transitions of the listed sequences (every sequence must
+ * have n_steps positions ready). Equivalent to n_steps rlt_decoder_step calls
+ * with the same list; a non-NULL stream lets the steps replay as one CUDA
+ * graph. */
+RLT_API int rlt_run_sequence(rlt_model *model, const int32_t *h_seq_ids, int n,
+                             int n_steps, rlt_stream stream);
+
+/* Ready-set scheduler: sequence h_seq_ids[i] still needs h_steps[i]
+ * transitions. Each tick batches every sequence with a pending step into one
+ * decoder step, until none is left (ragged batches: sequences drop out as
+ * they finish). Same errors as rlt_decoder_step, checked for every tick
+ * before any is enqueued. */
+RLT_API int rlt_run_ragged(rlt_model *model, const int32_t *h_seq_ids,
+                           const int32_t *h_steps, int n, rlt_stream stream);
+
+/* Host only: the scheduler's plan. h_tick_sizes[k] = number of sequences in
+ * tick k (k < *n_ticks <= max_ticks); h_order lists the n sequence indices in
+ * the order ticks batch them (ids that finish last first). */
+RLT_API int rlt_plan_ragged(const int32_t *h_steps, int n, int32_t *h_order,
+                            int32_t *h_tick_sizes, int max_ticks, int *n_ticks);
+
+/* Export H_t of slot `seq`: s_out [d] float32; cache_out [L_D][2][W-1][d]
+ * in the model dtype, K rows then V rows, positions t-(W-1) .. t-1 oldest
+ * first with slots of negative positions zero; *t_out = t (number of
+ * transitions taken). Any output may be NULL; outputs may be device or
+ * pinned host memory and are complete when `stream` reaches this point.
+ * K entries are stored with their rotary encoding applied. */
+RLT_API int rlt_get_state(rlt_model *model, int seq, float *s_out,
+                          void *cache_out, int64_t *t_out, rlt_stream stream);
+
+/* Import H_t into slot `seq` (same layouts as rlt_get_state). t must be
+ * <= max_len. Inputs may be device or pinned host memory. */
+RLT_API int rlt_set_state(rlt_model *model, int seq, const float *s_in,
+                          const void *cache_in, int64_t t, rlt_stream stream);
+
+/* Export the encoder output of slot `seq`: e_out [t_enc][d] and mem_out
+ * [G][t_enc][2][d] (K row then V row per position) in the model dtype.
+ * Either may be NULL. */
+RLT_API int rlt_get_encoder_output(rlt_model *model, int seq, void *e_out,
+                                   void *mem_out, int64_t *t_enc_out,
+                                   rlt_stream stream);
+
+/* Kernel classes reported by rlt_get_stats. */
+enum {
+  RLT_K_XATTN = 0, /* decoder cross-attention over M<=t (split-KV + merge) */
+  RLT_K_SWA = 1,   /* decoder sliding-window self-attention over the ring */
+  RLT_K_GEMM = 2,  /* decoder projections / FFN / gate GEMMs */
+  RLT_K_OTHER = 3, /* decoder norms, rotary/ring writes, gather, final norm */
+  RLT_K_ENC = 4,   /* every encoder prefill kernel */
+  RLT_K_COUNT = 5
+};
+
+typedef struct rlt_stats {
+  int64_t launches;                    /* kernels enqueued since rlt_create */
+  int64_t kernel_launches[RLT_K_COUNT]; /* profiled launches per class */
+  double kernel_ms[RLT_K_COUNT];       /* summed CUDA-event time per class */
+  double kernel_bytes[RLT_K_COUNT];    /* algorithmic HBM bytes of those launches */
+  double kernel_flops[RLT_K_COUNT];    /* algorithmic FLOPs of those launches */
+} rlt_stats;
+
+/* Measurement hook (no counterpart in the method): while enabled, every
+ * kernel launch is bracketed by a pair of CUDA events on its own stream and
+ * attributed to a class with the bytes/FLOPs the algorithm must move for it
+ * (weights once per launch; K/V rows actually attended; activations).
+ * Enabling or disabling clears the accumulated per-class figures. */
+RLT_API int rlt_profile(rlt_model *model, int enable);
+
+/* Synchronises the model's last stream, folds every completed event pair
+ * into the per-class sums and copies the counters into *out. */
+RLT_API int rlt_get_stats(rlt_model *model, rlt_stats *out);
+
+/* Synchronises the model's last stream and returns the first device-side
+ * error recorded since the previous poll (RLT_OK if none), then clears it. */
+RLT_API int rlt_poll_device_error(rlt_model *model);
+
+/* Static description of a status code (never NULL). */
+RLT_API const char *rlt_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RLT_H */

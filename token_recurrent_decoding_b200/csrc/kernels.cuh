@@ -1,0 +1,447 @@
+// Non-GEMM kernels of the RLT step and prefill: norms, rotary encoding, ring
+// and memory writes, decode attention (SWA over the ring, split-KV
+// cross-attention over M<=t), encoder causal attention, state import/export.
+//
+// Page key: [RLT-96] "RLT Runs 96 Blocks Per Token With Recurrent State, No
+// Resets" (aimastery.page); [RLT-TC] "Recurrent Looped Transformer (RLT):
+// prompts in parallel, depth in sequence" (thakicloud.com).
+#pragma once
+
+#include "common.cuh"
+
+namespace rlt {
+
+// ------------------------------------------------------------------ tables
+// cos/sin of position p times theta^(-2j/dh), computed in double once.
+__global__ void k_rope_table(float2 *tab, int max_len, int dh, double theta) {
+  int half = dh / 2;
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)max_len * half) return;
+  int p = (int)(i / half), j = (int)(i % half);
+  double ang = (double)p * pow(theta, -2.0 * j / dh);
+  double s, c;
+  sincos(ang, &s, &c);
+  tab[i] = make_float2((float)c, (float)s);
+}
+
+// ------------------------------------------------------------------ norms
+// out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * gamma, one warp per row.
+template <typename T>
+__global__ void k_rmsnorm(int rows, int d, const float *__restrict__ x,
+                          const float *__restrict__ gamma, float eps, T *__restrict__ out) {
+  int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float *xr = x + (size_t)r * d;
+  float ss = 0.f;
+  for (int c = lane * 4; c < d; c += 128) {
+    float4 v = *reinterpret_cast<const float4 *>(xr + c);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  float rs = rsqrtf(ss / d + eps);
+  for (int c = lane * 4; c < d; c += 128) {
+    float4 v = *reinterpret_cast<const float4 *>(xr + c);
+    float4 g = *reinterpret_cast<const float4 *>(gamma + c);
+    T *o = out + (size_t)r * d + c;
+    o[0] = from_f<T>(v.x * rs * g.x);
+    o[1] = from_f<T>(v.y * rs * g.y);
+    o[2] = from_f<T>(v.z * rs * g.z);
+    o[3] = from_f<T>(v.w * rs * g.w);
+  }
+}
+
+// ----------------------------------------------------------- decoder step
+// Step start: position of each ready slot, GEMM input [e_t ; s_{t-1}] and fp32
+// copies for the gated merge. With feedback off the residual is e_t itself.
+template <typename T>
+__global__ void k_step_gather(int n, int d, int max_len, const int *__restrict__ ready,
+                              const int *__restrict__ t_dec, int *__restrict__ pos,
+                              const T *__restrict__ e, const float *__restrict__ s,
+                              T *__restrict__ xin, float *__restrict__ e32,
+                              float *__restrict__ s32, float *__restrict__ h, int alpha_zero) {
+  int i = blockIdx.x;
+  if (i >= n) return;
+  int seq = ready[i];
+  int t = t_dec[seq];
+  if (threadIdx.x == 0) pos[i] = t;
+  const T *er = e + ((size_t)seq * max_len + t) * d;
+  const float *sr = s + (size_t)seq * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    T ev = er[c];
+    float sv = sr[c];
+    float ef = to_f(ev);
+    xin[(size_t)i * 2 * d + c] = ev;
+    xin[(size_t)i * 2 * d + d + c] = from_f<T>(sv);
+    e32[(size_t)i * d + c] = ef;
+    s32[(size_t)i * d + c] = sv;
+    if (alpha_zero) h[(size_t)i * d + c] = ef;
+  }
+}
+
+// After the q/k/v projection: rotary q (fp32, kept for the SWA), rotary k and
+// plain v written into ring slot t mod W of this layer.
+// Ring layout per layer: [max_seqs][H][2][W][dh].
+template <typename T>
+__global__ void k_dec_qkv_post(int n, int H, int dh, int W, const int *__restrict__ ready,
+                               const int *__restrict__ pos, const float *__restrict__ qkv,
+                               const float2 *__restrict__ rope, float *__restrict__ q_out,
+                               T *__restrict__ ring_l) {
+  int half = dh / 2, d = H * dh;
+  long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long)n * H * half) return;
+  int j = (int)(idx % half);
+  int h = (int)((idx / half) % H);
+  int i = (int)(idx / ((long)half * H));
+  int seq = ready[i], t = pos[i];
+  float2 cs = rope[(size_t)t * half + j];
+  const float *row = qkv + (size_t)i * 3 * d;
+  int c1 = h * dh + j, c2 = c1 + half;
+  float q1 = row[c1], q2 = row[c2];
+  q_out[(size_t)i * d + c1] = q1 * cs.x - q2 * cs.y;
+  q_out[(size_t)i * d + c2] = q2 * cs.x + q1 * cs.y;
+  float k1 = row[d + c1], k2 = row[d + c2];
+  float v1 = row[2 * d + c1], v2 = row[2 * d + c2];
+  int slot = t % W;
+  T *kb = ring_l + (((size_t)seq * H + h) * 2 + 0) * W * dh + (size_t)slot * dh;
+  T *vb = kb + (size_t)W * dh;
+  kb[j] = from_f<T>(k1 * cs.x - k2 * cs.y);
+  kb[j + half] = from_f<T>(k2 * cs.x + k1 * cs.y);
+  vb[j] = from_f<T>(v1);
+  vb[j + half] = from_f<T>(v2);
+}
+
+// Online-softmax state of one lane group over the keys it has seen.
+template <int VEC> struct SoftAcc {
+  float m, l, acc[VEC];
+  __device__ void init() {
+    m = -INFINITY; l = 0.f;
+#pragma unroll
+    for (int v = 0; v < VEC; v++) acc[v] = 0.f;
+  }
+  __device__ void add(float s, const float *vv) {
+    float mn = fmaxf(m, s);
+    float c = expf(m - mn), p = expf(s - mn);
+    l = l * c + p;
+#pragma unroll
+    for (int v = 0; v < VEC; v++) acc[v] = acc[v] * c + p * vv[v];
+    m = mn;
+  }
+  // Merge with the lane `off` positions away (another key group).
+  __device__ void merge_xor(int off) {
+    float m2 = __shfl_xor_sync(FULL_MASK, m, off);
+    float l2 = __shfl_xor_sync(FULL_MASK, l, off);
+    float mn = fmaxf(m, m2);
+    float c1 = (m == -INFINITY) ? 0.f : expf(m - mn);
+    float c2 = (m2 == -INFINITY) ? 0.f : expf(m2 - mn);
+    l = l * c1 + l2 * c2;
+#pragma unroll
+    for (int v = 0; v < VEC; v++) {
+      float a2 = __shfl_xor_sync(FULL_MASK, acc[v], off);
+      acc[v] = acc[v] * c1 + a2 * c2;
+    }
+    m = mn;
+  }
+};
+
+// One warp attends one query over keys p in [p_lo, p_hi] whose rows sit at
+// K + row(p) * DH (row(p) = p mod ring for the ring, p for the memory).
+// LPK lanes share a key (VEC elements each, one 16-byte load); the warp covers
+// KPP keys per pass. Returns the warp-merged state in every lane.
+template <typename T, int DH, bool RING>
+__device__ __forceinline__ void warp_attend(const float *qr, const T *__restrict__ K,
+                                            const T *__restrict__ V, int p_lo, int p_hi,
+                                            int ring, int lane, SoftAcc<V16<T>::N> &st) {
+  constexpr int VEC = V16<T>::N;
+  constexpr int LPK = DH / VEC;
+  constexpr int KPP = 32 / LPK;
+  const int sub = lane % LPK, grp = lane / LPK;
+  st.init();
+  int p = p_lo + grp;
+#pragma unroll 2
+  for (; p - grp <= p_hi; p += KPP) {
+    bool valid = p <= p_hi;
+    float kf[VEC], vf[VEC];
+    if (valid) {
+      int row = RING ? (p % ring) : p;
+      ld16(K + (size_t)row * DH + sub * VEC, kf);
+      ld16(V + (size_t)row * DH + sub * VEC, vf);
+    } else {
+#pragma unroll
+      for (int v = 0; v < VEC; v++) kf[v] = vf[v] = 0.f;
+    }
+    float sdot = 0.f;
+#pragma unroll
+    for (int v = 0; v < VEC; v++) sdot = fmaf(qr[v], kf[v], sdot);
+#pragma unroll
+    for (int o = 1; o < LPK; o <<= 1) sdot += __shfl_xor_sync(FULL_MASK, sdot, o);
+    if (valid) st.add(sdot, vf);
+  }
+#pragma unroll
+  for (int o = LPK; o < 32; o <<= 1) st.merge_xor(o);
+}
+
+// Decoder SWA: slot i, head h attends positions max(0, t-W+1) .. t of its ring.
+template <typename T, int DH>
+__global__ void k_swa_decode(int n, int H, int W, const int *__restrict__ ready,
+                             const int *__restrict__ pos, const float *__restrict__ q,
+                             const T *__restrict__ ring_l, T *__restrict__ out, float scale) {
+  constexpr int VEC = V16<T>::N, LPK = DH / VEC;
+  int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= n * H) return;
+  int i = gw / H, h = gw % H, d = H * DH;
+  int seq = ready[i], t = pos[i];
+  int sub = lane % LPK;
+  float qr[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; v++) qr[v] = q[(size_t)i * d + h * DH + sub * VEC + v] * scale;
+  const T *K = ring_l + (((size_t)seq * H + h) * 2) * W * DH;
+  const T *V = K + (size_t)W * DH;
+  SoftAcc<VEC> st;
+  int p_lo = t - W + 1 > 0 ? t - W + 1 : 0;
+  warp_attend<T, DH, true>(qr, K, V, p_lo, t, W, lane, st);
+  if (lane < LPK) {
+    float inv = 1.f / st.l;
+#pragma unroll
+    for (int v = 0; v < VEC; v++)
+      out[(size_t)i * d + h * DH + sub * VEC + v] = from_f<T>(st.acc[v] * inv);
+  }
+}
+
+// Cross-attention, split over chunks of CH memory positions: item (i, h, c)
+// covers positions [c*CH, min(t+1, (c+1)*CH)) and writes its partial
+// (acc[DH], m, l). Memory layout per group: [max_seqs][H][2][max_len][dh].
+// The grid covers `xchunks` splits per (i, h); the partial buffer is laid out
+// with `max_chunks` per (i, h).
+template <typename T, int DH>
+__global__ void k_xattn_partial(int n, int H, int CH, int xchunks, int max_chunks, int max_len,
+                                const int *__restrict__ ready, const int *__restrict__ pos,
+                                const float *__restrict__ q, const T *__restrict__ mem_g,
+                                float *__restrict__ part, float scale) {
+  constexpr int VEC = V16<T>::N, LPK = DH / VEC;
+  int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= n * H * xchunks) return;
+  int c = gw % xchunks, ih = gw / xchunks;
+  int i = ih / H, h = ih % H, d = H * DH;
+  int t = pos[i];
+  int p_lo = c * CH;
+  if (p_lo > t) return;
+  int p_hi = min(t, p_lo + CH - 1);
+  int seq = ready[i];
+  int sub = lane % LPK;
+  float qr[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; v++) qr[v] = q[(size_t)i * d + h * DH + sub * VEC + v] * scale;
+  const T *K = mem_g + (((size_t)seq * H + h) * 2) * max_len * DH;
+  const T *V = K + (size_t)max_len * DH;
+  SoftAcc<VEC> st;
+  warp_attend<T, DH, false>(qr, K, V, p_lo, p_hi, 0, lane, st);
+  float *pp = part + ((size_t)ih * max_chunks + c) * (DH + 2);
+  if (lane < LPK) {
+#pragma unroll
+    for (int v = 0; v < VEC; v++) pp[sub * VEC + v] = st.acc[v];
+  }
+  if (lane == 0) {
+    pp[DH] = st.m;
+    pp[DH + 1] = st.l;
+  }
+}
+
+// Merge the chunk partials of (i, h) in chunk order.
+template <typename T, int DH>
+__global__ void k_xattn_combine(int n, int H, int CH, int max_chunks, const int *__restrict__ pos,
+                                const float *__restrict__ part, T *__restrict__ out) {
+  int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= n * H) return;
+  int i = gw / H, h = gw % H, d = H * DH;
+  int nc = pos[i] / CH + 1;
+  const float *pp = part + (size_t)gw * max_chunks * (DH + 2);
+  float mx = -INFINITY;
+  for (int c = 0; c < nc; c++) mx = fmaxf(mx, pp[c * (DH + 2) + DH]);
+  float L = 0.f;
+  for (int c = 0; c < nc; c++) L += expf(pp[c * (DH + 2) + DH] - mx) * pp[c * (DH + 2) + DH + 1];
+  float inv = 1.f / L;
+  for (int j = lane; j < DH; j += 32) {
+    float o = 0.f;
+    for (int c = 0; c < nc; c++) o += expf(pp[c * (DH + 2) + DH] - mx) * pp[c * (DH + 2) + j];
+    out[(size_t)i * d + h * DH + j] = from_f<T>(o * inv);
+  }
+}
+
+// Step end: s_t = RMSNorm_f(h) and t_dec += 1 ([RLT-96] "Architecture": s_t is
+// the final decoder output vector). One warp per slot.
+__global__ void k_step_final(int n, int d, const int *__restrict__ ready, int *__restrict__ t_dec,
+                             const float *__restrict__ h, const float *__restrict__ gamma,
+                             float eps, float *__restrict__ s) {
+  int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (i >= n) return;
+  int seq = ready[i];
+  const float *hr = h + (size_t)i * d;
+  float ss = 0.f;
+  for (int c = lane; c < d; c += 32) ss += hr[c] * hr[c];
+  ss = warp_sum(ss);
+  float rs = rsqrtf(ss / d + eps);
+  for (int c = lane; c < d; c += 32) s[(size_t)seq * d + c] = hr[c] * rs * gamma[c];
+  if (lane == 0) t_dec[seq] += 1;
+}
+
+// ----------------------------------------------------------------- prefill
+// Token embedding rows into the fp32 residual stream; out-of-range token ids
+// record an error and embed zeros.
+template <typename T>
+__global__ void k_embed(int ntok, int d, int vocab, const int *__restrict__ tok,
+                        const T *__restrict__ E, float *__restrict__ h, int *err) {
+  int m = blockIdx.x;
+  if (m >= ntok) return;
+  int id = tok[m];
+  bool ok = id >= 0 && id < vocab;
+  if (!ok && threadIdx.x == 0) set_error(err, DEV_ERR_TOKEN);
+  for (int c = threadIdx.x; c < d; c += blockDim.x)
+    h[(size_t)m * d + c] = ok ? to_f(E[(size_t)id * d + c]) : 0.f;
+}
+
+// Encoder q/k/v: rotary q, k at each token's position; head-major [H][ntok][dh].
+template <typename T>
+__global__ void k_enc_qkv_post(int ntok, int H, int dh, const int *__restrict__ tok_pos,
+                               const float *__restrict__ qkv, const float2 *__restrict__ rope,
+                               T *__restrict__ Qh, T *__restrict__ Kh, T *__restrict__ Vh) {
+  int half = dh / 2, d = H * dh;
+  long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long)ntok * H * half) return;
+  int j = (int)(idx % half);
+  int h = (int)((idx / half) % H);
+  int m = (int)(idx / ((long)half * H));
+  int p = tok_pos[m];
+  float2 cs = rope[(size_t)p * half + j];
+  const float *row = qkv + (size_t)m * 3 * d;
+  int c1 = h * dh + j, c2 = c1 + half;
+  size_t o = ((size_t)h * ntok + m) * dh;
+  float q1 = row[c1], q2 = row[c2], k1 = row[d + c1], k2 = row[d + c2];
+  Qh[o + j] = from_f<T>(q1 * cs.x - q2 * cs.y);
+  Qh[o + j + half] = from_f<T>(q2 * cs.x + q1 * cs.y);
+  Kh[o + j] = from_f<T>(k1 * cs.x - k2 * cs.y);
+  Kh[o + j + half] = from_f<T>(k2 * cs.x + k1 * cs.y);
+  Vh[o + j] = from_f<T>(row[2 * d + c1]);
+  Vh[o + j + half] = from_f<T>(row[2 * d + c2]);
+}
+
+// Encoder causal attention (SIMT form): one warp per (token, head) attends the
+// keys of positions 0..p of its own sequence ([RLT-96] "Architecture": causal
+// mask over known tokens). Tokens of one sequence are contiguous; tok_start[m]
+// is the chunk row of that sequence's first token.
+template <typename T, int DH>
+__global__ void k_enc_attn_simt(int ntok, int H, const int *__restrict__ tok_pos,
+                                const int *__restrict__ tok_start, const T *__restrict__ Qh,
+                                const T *__restrict__ Kh, const T *__restrict__ Vh,
+                                T *__restrict__ out, float scale) {
+  constexpr int VEC = V16<T>::N, LPK = DH / VEC;
+  int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= ntok * H) return;
+  int m = gw / H, h = gw % H, d = H * DH;
+  int p = tok_pos[m], st0 = tok_start[m];
+  int sub = lane % LPK;
+  float qr[VEC];
+  ld16(Qh + ((size_t)h * ntok + m) * DH + sub * VEC, qr);
+#pragma unroll
+  for (int v = 0; v < VEC; v++) qr[v] *= scale;
+  const T *K = Kh + ((size_t)h * ntok + st0) * DH;
+  const T *V = Vh + ((size_t)h * ntok + st0) * DH;
+  SoftAcc<VEC> st;
+  warp_attend<T, DH, false>(qr, K, V, 0, p, 0, lane, st);
+  if (lane < LPK) {
+    float inv = 1.f / st.l;
+#pragma unroll
+    for (int v = 0; v < VEC; v++)
+      out[(size_t)m * d + h * DH + sub * VEC + v] = from_f<T>(st.acc[v] * inv);
+  }
+}
+
+// Encoder output e_t = RMSNorm_E(h): compact rows for the memory GEMM and the
+// per-sequence e arena [max_seqs][max_len][d]. One warp per token.
+template <typename T>
+__global__ void k_enc_final(int ntok, int d, int max_len, const float *__restrict__ h,
+                            const float *__restrict__ gamma, float eps,
+                            const int *__restrict__ tok_slot, const int *__restrict__ tok_pos,
+                            T *__restrict__ e_tok, T *__restrict__ e_arena) {
+  int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (m >= ntok) return;
+  const float *hr = h + (size_t)m * d;
+  float ss = 0.f;
+  for (int c = lane; c < d; c += 32) ss += hr[c] * hr[c];
+  ss = warp_sum(ss);
+  float rs = rsqrtf(ss / d + eps);
+  T *ea = e_arena + ((size_t)tok_slot[m] * max_len + tok_pos[m]) * d;
+  for (int c = lane; c < d; c += 32) {
+    T v = from_f<T>(hr[c] * rs * gamma[c]);
+    e_tok[(size_t)m * d + c] = v;
+    ea[c] = v;
+  }
+}
+
+// ------------------------------------------------------------ state access
+// Ring (this slot, all layers) -> [L][2][W-1][d] window, oldest first; slots of
+// negative positions are zero.
+template <typename T>
+__global__ void k_get_window(int L, int H, int dh, int W, int max_seqs, int seq, long t,
+                             const T *__restrict__ ring, T *__restrict__ out) {
+  int d = H * dh, Wm1 = W - 1;
+  long total = (long)L * 2 * Wm1 * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    int c = (int)(idx % d);
+    int i = (int)((idx / d) % Wm1);
+    int kv = (int)((idx / ((long)d * Wm1)) % 2);
+    int l = (int)(idx / ((long)d * Wm1 * 2));
+    long p = t - Wm1 + i;
+    T v = from_f<T>(0.f);
+    if (p >= 0) {
+      int h = c / dh, j = c % dh;
+      v = ring[(((((size_t)l * max_seqs + seq) * H + h) * 2 + kv) * W + (p % W)) * dh + j];
+    }
+    out[idx] = v;
+  }
+}
+
+template <typename T>
+__global__ void k_set_window(int L, int H, int dh, int W, int max_seqs, int seq, long t,
+                             const T *__restrict__ in, T *__restrict__ ring) {
+  int d = H * dh, Wm1 = W - 1;
+  long total = (long)L * 2 * Wm1 * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    int c = (int)(idx % d);
+    int i = (int)((idx / d) % Wm1);
+    int kv = (int)((idx / ((long)d * Wm1)) % 2);
+    int l = (int)(idx / ((long)d * Wm1 * 2));
+    long p = t - Wm1 + i;
+    if (p < 0) continue;
+    int h = c / dh, j = c % dh;
+    ring[(((((size_t)l * max_seqs + seq) * H + h) * 2 + kv) * W + (p % W)) * dh + j] = in[idx];
+  }
+}
+
+// Memory (one slot, all groups) -> [G][t_enc][2][d].
+template <typename T>
+__global__ void k_get_memory(int G, int H, int dh, int max_seqs, int max_len, int seq, int T_enc,
+                             const T *__restrict__ mem, T *__restrict__ out) {
+  int d = H * dh;
+  long total = (long)G * T_enc * 2 * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    int c = (int)(idx % d);
+    int kv = (int)((idx / d) % 2);
+    int p = (int)((idx / (2L * d)) % T_enc);
+    int g = (int)(idx / (2L * d * T_enc));
+    int h = c / dh, j = c % dh;
+    out[idx] = mem[(((((size_t)g * max_seqs + seq) * H + h) * 2 + kv) * max_len + p) * dh + j];
+  }
+}
+
+// s <- s* for the listed slots.
+__global__ void k_reset_s(int n, int d, const int *__restrict__ ids, const float *__restrict__ sstar,
+                          float *__restrict__ s) {
+  int i = blockIdx.x;
+  if (i >= n) return;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) s[(size_t)ids[i] * d + c] = sstar[c];
+}
+
+}  // namespace rlt

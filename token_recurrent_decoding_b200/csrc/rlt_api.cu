@@ -1,0 +1,900 @@
+// Host side of the RLT C ABI (include/rlt.h): validation, arena layout, and
+// the launch sequences of the decoder step and the encoder prefill.
+//
+// Page key: [RLT-96] "RLT Runs 96 Blocks Per Token With Recurrent State, No
+// Resets" (aimastery.page); [RLT-TC] "Recurrent Looped Transformer (RLT):
+// prompts in parallel, depth in sequence" (thakicloud.com); [RLT-FT]
+// "Recurrent Looped Transformer debunked" (flowtivity.ai).
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/rlt.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+using namespace rlt;
+
+namespace {
+
+constexpr int XCH = 256;  // memory positions per cross-attention split
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Layout {
+  // persistent state
+  size_t s, t_dec, t_enc, e, mem, ring, rope, err;
+  // decoder step work buffers (max_seqs rows)
+  size_t ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part;
+  // encoder work buffers (ptok rows)
+  size_t tok, tok_slot, tok_pos, tok_start, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
+  size_t staging, staging_bytes;
+  size_t total;
+  int max_chunks, ptok;
+};
+
+int elem_size(const rlt_config *c) { return c->dtype == RLT_BF16 ? 2 : 4; }
+
+int check_config(const rlt_config *c) {
+  if (!c) return RLT_ERR_INVALID_ARG;
+  if (c->d <= 0 || c->n_heads <= 0 || c->head_dim <= 0 || c->d != c->n_heads * c->head_dim)
+    return RLT_ERR_INVALID_ARG;
+  if (c->n_enc_layers < 0 || c->n_enc_layers > RLT_MAX_LAYERS || c->n_dec_layers < 1 ||
+      c->n_dec_layers > RLT_MAX_LAYERS)
+    return RLT_ERR_INVALID_ARG;
+  if (c->ffn_dim <= 0 || c->vocab <= 0 || c->window < 1 || c->max_seqs < 1 || c->max_len < 1)
+    return RLT_ERR_INVALID_ARG;
+  if (c->ffn_kind != RLT_GELU && c->ffn_kind != RLT_SWIGLU) return RLT_ERR_INVALID_ARG;
+  if (c->dtype != RLT_F32 && c->dtype != RLT_BF16) return RLT_ERR_INVALID_ARG;
+  if (c->mem_groups != 1 && c->mem_groups != c->n_dec_layers) return RLT_ERR_UNSUPPORTED;
+  if (c->tied && c->n_dec_layers > c->n_enc_layers) return RLT_ERR_INVALID_ARG;
+  if (!std::isfinite(c->alpha) || !(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f))
+    return RLT_ERR_INVALID_ARG;
+  if (c->max_prefill_tokens < 0) return RLT_ERR_INVALID_ARG;
+  if (c->max_prefill_tokens > 0 && c->max_prefill_tokens < c->max_len) return RLT_ERR_INVALID_ARG;
+  int dh = c->head_dim;
+  if (dh != 16 && dh != 32 && dh != 64 && dh != 128) return RLT_ERR_UNSUPPORTED;
+  if (c->d % 4 || c->ffn_dim % 4) return RLT_ERR_UNSUPPORTED;
+  if (c->dtype == RLT_BF16 && (c->d % 64 || c->ffn_dim % 64)) return RLT_ERR_UNSUPPORTED;
+  if ((long)c->max_seqs * c->max_len > (1L << 31)) return RLT_ERR_UNSUPPORTED;
+  return RLT_OK;
+}
+
+size_t compute_layout(const rlt_config *c, Layout *L) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes ? bytes : 1);
+    return o;
+  };
+  size_t es = elem_size(c);
+  size_t S = c->max_seqs, T = c->max_len, d = c->d, F = c->ffn_dim, H = c->n_heads;
+  size_t G = c->mem_groups, LD = c->n_dec_layers, W = c->window, dh = c->head_dim;
+  long ptok = c->max_prefill_tokens > 0 ? c->max_prefill_tokens
+                                        : std::min<long>((long)S * T, 131072L);
+  ptok = std::max<long>(ptok, c->max_len);
+  L->ptok = (int)ptok;
+  L->max_chunks = (int)((T + XCH - 1) / XCH);
+  L->s = take(S * d * 4);
+  L->t_dec = take(S * 4);
+  L->t_enc = take(S * 4);
+  L->e = take(S * T * d * es);
+  L->mem = take(G * S * H * 2 * T * dh * es);
+  L->ring = take(LD * S * H * 2 * W * dh * es);
+  L->rope = take(T * (dh / 2) * 8);
+  L->err = take(16);
+  L->ready = take(S * 4);
+  L->pos = take(S * 4);
+  L->h = take(S * d * 4);
+  L->xin = take(S * 2 * d * es);
+  L->e32 = take(S * d * 4);
+  L->s32 = take(S * d * 4);
+  L->qkv = take(S * 3 * d * 4);
+  L->q = take(S * d * 4);
+  L->a = take(S * d * es);
+  L->u = take(S * d * es);
+  L->fa = take(c->ffn_kind == RLT_SWIGLU ? S * F * 4 : 0);
+  L->f = take(S * F * es);
+  L->part = take(S * H * L->max_chunks * (dh + 2) * 4);
+  size_t P = (size_t)ptok;
+  L->tok = take(P * 4);
+  L->tok_slot = take(P * 4);
+  L->tok_pos = take(P * 4);
+  L->tok_start = take(P * 4);
+  L->eh = take(P * d * 4);
+  L->eu = take(P * d * es);
+  L->eqkv = take(P * 3 * d * 4);
+  L->Qh = take(P * d * es);
+  L->Kh = take(P * d * es);
+  L->Vh = take(P * d * es);
+  L->ea = take(P * d * es);
+  L->efa = take(c->ffn_kind == RLT_SWIGLU ? P * F * 4 : 0);
+  L->ef = take(P * F * es);
+  L->etok = take(P * d * es);
+  size_t st = std::max(LD * 2 * (W > 1 ? W - 1 : 1) * d * es, G * T * 2 * d * es);
+  L->staging_bytes = st;
+  L->staging = take(st);
+  L->total = off;
+  return off;
+}
+
+}  // namespace
+
+struct StepInfo {
+  int n;            // ready slots
+  int xchunks;      // cross-attention splits to launch (covers max t)
+  double sum_keys;  // sum over slots of (t + 1): memory rows attended
+  double sum_win;   // sum over slots of min(t + 1, W): ring rows attended
+};
+
+struct ProfSpan {
+  int kind;
+  cudaEvent_t a, b;
+  double bytes, flops;
+};
+
+struct rlt_model {
+  rlt_config cfg;
+  rlt_weights w;
+  Layout L;
+  uint8_t *arena = nullptr;
+  int device = 0;
+  std::vector<int> t_dec, t_enc;
+  cudaStream_t last_stream = nullptr;
+  template <typename X> X *at(size_t off) const { return reinterpret_cast<X *>(arena + off); }
+  // dtype/head-dim specialised launch sequences
+  // measurement hook (rlt_profile / rlt_get_stats)
+  bool profiling = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<ProfSpan> pending;
+  rlt_stats stats{};
+  cudaError_t (*step)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
+  cudaError_t (*prefill)(rlt_model *, int, cudaStream_t) = nullptr;
+  cudaError_t (*get_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
+  cudaError_t (*set_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
+  cudaError_t (*get_memory)(rlt_model *, int, int, cudaStream_t) = nullptr;
+};
+
+namespace {
+
+#define RLT_TRY(x)                           \
+  do {                                       \
+    cudaError_t e_ = (x);                    \
+    if (e_ != cudaSuccess) return e_;        \
+  } while (0)
+
+inline int blocks_for(long threads, int bs) { return (int)((threads + bs - 1) / bs); }
+
+cudaEvent_t take_event(rlt_model *M) {
+  if (!M->ev_pool.empty()) {
+    cudaEvent_t e = M->ev_pool.back();
+    M->ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Counts one kernel launch; in profile mode brackets it with CUDA events on
+// the launching stream and records the class and algorithmic bytes / FLOPs.
+struct Span {
+  rlt_model *M;
+  cudaStream_t st;
+  int kind;
+  double bytes, flops;
+  cudaEvent_t a = nullptr;
+  Span(rlt_model *M_, cudaStream_t st_, int kind_, double bytes_ = 0, double flops_ = 0)
+      : M(M_), st(st_), kind(kind_), bytes(bytes_), flops(flops_) {
+    M->stats.launches++;
+    if (M->profiling) {
+      a = take_event(M);
+      if (a) cudaEventRecord(a, st);
+    }
+  }
+  ~Span() {
+    if (!a) return;
+    cudaEvent_t b = take_event(M);
+    if (!b) return;
+    cudaEventRecord(b, st);
+    M->pending.push_back({kind, a, b, bytes, flops});
+  }
+};
+
+// GEMM launch wrapper: class RLT_K_GEMM (or the encoder class) with the
+// algorithmic traffic of one pass over the weights and activations.
+template <typename T, class Epi>
+cudaError_t gemm_k(rlt_model *M, int kind, int m, int n, int k, const T *A, int lda, const T *B,
+                   int ldb, Epi epi, cudaStream_t st) {
+  double es = sizeof(T);
+  Span sp(M, st, kind, (double)n * k * es + (double)m * k * es + (double)m * n * 4.0,
+          2.0 * m * n * k);
+  return gemm(m, n, k, A, lda, B, ldb, epi, st);
+}
+
+template <typename T> struct W_ {
+  // Decoder matrices of layer l, honouring weight tying.
+  static const T *qkv(const rlt_model *M, int l) {
+    return (const T *)(M->cfg.tied ? M->w.enc_wqkv[l] : M->w.dec_wqkv[l]);
+  }
+  static const T *o(const rlt_model *M, int l) {
+    return (const T *)(M->cfg.tied ? M->w.enc_wo[l] : M->w.dec_wo[l]);
+  }
+  static const T *w1(const rlt_model *M, int l) {
+    return (const T *)(M->cfg.tied ? M->w.enc_w1[l] : M->w.dec_w1[l]);
+  }
+  static const T *wb(const rlt_model *M, int l) {
+    return (const T *)(M->cfg.tied ? M->w.enc_wb[l] : M->w.dec_wb[l]);
+  }
+  static const T *w2(const rlt_model *M, int l) {
+    return (const T *)(M->cfg.tied ? M->w.enc_w2[l] : M->w.dec_w2[l]);
+  }
+};
+
+// One batched decoder transition for the n slots listed in the arena's ready
+// list ([RLT-96] "Architecture": gated merge, then per block SWA,
+// cross-attention, FFN; s_t is the final output). `xchunks` bounds the
+// cross-attention splits launched (covers the largest t in the batch).
+template <typename T, int DH>
+cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const int n = si.n, xchunks = si.xchunks;
+  const int d = c.d, H = c.n_heads, F = c.ffn_dim, W = c.window;
+  const float scale = 1.0f / sqrtf((float)DH), eps = c.rms_eps;
+  const double es = sizeof(T);
+  int *ready = M->at<int>(L.ready), *pos = M->at<int>(L.pos), *t_dec = M->at<int>(L.t_dec);
+  float *h = M->at<float>(L.h), *e32 = M->at<float>(L.e32), *s32 = M->at<float>(L.s32);
+  float *qkv = M->at<float>(L.qkv), *q = M->at<float>(L.q), *fa = M->at<float>(L.fa);
+  float *part = M->at<float>(L.part), *s = M->at<float>(L.s);
+  T *xin = M->at<T>(L.xin), *a = M->at<T>(L.a), *u = M->at<T>(L.u), *f = M->at<T>(L.f);
+  T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem);
+  const float2 *rope = M->at<float2>(L.rope);
+  const bool a0 = c.alpha == 0.0f;
+  const size_t ring_layer = (size_t)c.max_seqs * H * 2 * W * DH;
+  const size_t mem_group = (size_t)c.max_seqs * H * 2 * c.max_len * DH;
+  const int rows_blocks = blocks_for((long)n * 32, 256);
+  const double row_bytes = (double)n * d * (4 + es);  // one fp32 read + one T write per row
+
+  {
+    Span sp(M, st, RLT_K_OTHER, (double)n * d * (es + 4) + row_bytes);
+    k_step_gather<T><<<n, 256, 0, st>>>(n, d, c.max_len, ready, t_dec, pos, M->at<T>(L.e), s,
+                                        xin, e32, s32, h, a0);
+  }
+  RLT_TRY(cudaGetLastError());
+  if (!a0)
+    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, 2 * d, xin, 2 * d, (const T *)M->w.gate_w, 2 * d,
+                   EpiGate{e32, s32, (const float *)M->w.gate_b, c.alpha, h, d}, st));
+  for (int l = 0; l < c.n_dec_layers; l++) {
+    T *ring_l = ring + (size_t)l * ring_layer;
+    const T *mem_g = mem + (size_t)(c.mem_groups == 1 ? 0 : l) * mem_group;
+    // sliding-window self-attention sublayer
+    {
+      Span sp(M, st, RLT_K_OTHER, row_bytes);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, d, h, (const float *)M->w.dec_ln1[l], eps, u);
+    }
+    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, 3 * d, d, u, d, W_<T>::qkv(M, l), d,
+                   EpiStoreF32{qkv, 3 * d}, st));
+    {
+      Span sp(M, st, RLT_K_OTHER, (double)n * 3 * d * 4 + (double)n * d * (4 + 2 * es));
+      k_dec_qkv_post<T><<<blocks_for((long)n * H * (DH / 2), 256), 256, 0, st>>>(
+          n, H, DH, W, ready, pos, qkv, rope, q, ring_l);
+    }
+    {
+      Span sp(M, st, RLT_K_SWA, si.sum_win * 2.0 * d * es + (double)n * d * (4 + es),
+              4.0 * d * si.sum_win);
+      k_swa_decode<T, DH><<<blocks_for((long)n * H * 32, 256), 256, 0, st>>>(n, H, W, ready, pos,
+                                                                             q, ring_l, a, scale);
+    }
+    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, d, a, d, W_<T>::o(M, l), d, EpiResid{h, d}, st));
+    // cross-attention sublayer over M<=t
+    {
+      Span sp(M, st, RLT_K_OTHER, row_bytes);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, d, h, (const float *)M->w.dec_ln2[l], eps, u);
+    }
+    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, d, u, d, (const T *)M->w.dec_wqx[l], d,
+                   EpiStoreF32{q, d}, st));
+    {
+      Span sp(M, st, RLT_K_XATTN, si.sum_keys * 2.0 * d * es, 4.0 * d * si.sum_keys);
+      k_xattn_partial<T, DH><<<blocks_for((long)n * H * xchunks * 32, 256), 256, 0, st>>>(
+          n, H, XCH, xchunks, L.max_chunks, c.max_len, ready, pos, q, mem_g, part, scale);
+    }
+    {
+      Span sp(M, st, RLT_K_OTHER, (double)n * H * xchunks * (DH + 2) * 4 + (double)n * d * es);
+      k_xattn_combine<T, DH><<<blocks_for((long)n * H * 32, 256), 256, 0, st>>>(
+          n, H, XCH, L.max_chunks, pos, part, a);
+    }
+    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, d, a, d, (const T *)M->w.dec_wox[l], d, EpiResid{h, d},
+                   st));
+    // FFN sublayer
+    {
+      Span sp(M, st, RLT_K_OTHER, row_bytes);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, d, h, (const float *)M->w.dec_ln3[l], eps, u);
+    }
+    if (c.ffn_kind == RLT_GELU) {
+      RLT_TRY(gemm_k(M, RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiGelu<T>{f, F}, st));
+    } else {
+      RLT_TRY(gemm_k(M, RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiStoreF32{fa, F}, st));
+      RLT_TRY(gemm_k(M, RLT_K_GEMM, n, F, d, u, d, W_<T>::wb(M, l), d, EpiSwiglu<T>{fa, f, F},
+                     st));
+    }
+    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, F, f, F, W_<T>::w2(M, l), F, EpiResid{h, d}, st));
+  }
+  {
+    Span sp(M, st, RLT_K_OTHER, (double)n * d * 8);
+    k_step_final<<<rows_blocks, 256, 0, st>>>(n, d, ready, t_dec, h,
+                                              (const float *)M->w.dec_lnf, eps, s);
+  }
+  return cudaGetLastError();
+}
+
+// Encoder over one chunk of ntok tokens already staged in the arena (token
+// ids, slot, position, sequence start), then the memory projection
+// ([RLT-96] "Architecture"; [RLT-TC] "What is this technology").
+template <typename T, int DH>
+cudaError_t prefill_impl(rlt_model *M, int ntok, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const rlt_weights &w = M->w;
+  const int d = c.d, H = c.n_heads, F = c.ffn_dim;
+  const float scale = 1.0f / sqrtf((float)DH), eps = c.rms_eps;
+  const int K = RLT_K_ENC;
+  int *tok = M->at<int>(L.tok), *tslot = M->at<int>(L.tok_slot), *tpos = M->at<int>(L.tok_pos);
+  int *tstart = M->at<int>(L.tok_start);
+  float *eh = M->at<float>(L.eh), *eqkv = M->at<float>(L.eqkv), *efa = M->at<float>(L.efa);
+  T *eu = M->at<T>(L.eu), *Qh = M->at<T>(L.Qh), *Kh = M->at<T>(L.Kh), *Vh = M->at<T>(L.Vh);
+  T *ea = M->at<T>(L.ea), *ef = M->at<T>(L.ef), *etok = M->at<T>(L.etok);
+  const float2 *rope = M->at<float2>(L.rope);
+  const int rows_blocks = blocks_for((long)ntok * 32, 256);
+
+  {
+    Span sp(M, st, K);
+    k_embed<T><<<ntok, 256, 0, st>>>(ntok, d, c.vocab, tok, (const T *)w.embed, eh,
+                                     M->at<int>(L.err));
+  }
+  RLT_TRY(cudaGetLastError());
+  for (int l = 0; l < c.n_enc_layers; l++) {
+    {
+      Span sp(M, st, K);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, d, eh, (const float *)w.enc_ln1[l], eps, eu);
+    }
+    RLT_TRY(gemm_k(M, K, ntok, 3 * d, d, eu, d, (const T *)w.enc_wqkv[l], d,
+                   EpiStoreF32{eqkv, 3 * d}, st));
+    {
+      Span sp(M, st, K);
+      k_enc_qkv_post<T><<<blocks_for((long)ntok * H * (DH / 2), 256), 256, 0, st>>>(
+          ntok, H, DH, tpos, eqkv, rope, Qh, Kh, Vh);
+    }
+    {
+      Span sp(M, st, K);
+      k_enc_attn_simt<T, DH><<<blocks_for((long)ntok * H * 32, 256), 256, 0, st>>>(
+          ntok, H, tpos, tstart, Qh, Kh, Vh, ea, scale);
+    }
+    RLT_TRY(gemm_k(M, K, ntok, d, d, ea, d, (const T *)w.enc_wo[l], d, EpiResid{eh, d}, st));
+    {
+      Span sp(M, st, K);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, d, eh, (const float *)w.enc_ln2[l], eps, eu);
+    }
+    if (c.ffn_kind == RLT_GELU) {
+      RLT_TRY(gemm_k(M, K, ntok, F, d, eu, d, (const T *)w.enc_w1[l], d, EpiGelu<T>{ef, F}, st));
+    } else {
+      RLT_TRY(gemm_k(M, K, ntok, F, d, eu, d, (const T *)w.enc_w1[l], d, EpiStoreF32{efa, F},
+                     st));
+      RLT_TRY(gemm_k(M, K, ntok, F, d, eu, d, (const T *)w.enc_wb[l], d,
+                     EpiSwiglu<T>{efa, ef, F}, st));
+    }
+    RLT_TRY(gemm_k(M, K, ntok, d, F, ef, F, (const T *)w.enc_w2[l], F, EpiResid{eh, d}, st));
+  }
+  {
+    Span sp(M, st, K);
+    k_enc_final<T><<<rows_blocks, 256, 0, st>>>(ntok, d, c.max_len, eh, (const float *)w.enc_lnf,
+                                                eps, tslot, tpos, etok, M->at<T>(L.e));
+  }
+  RLT_TRY(cudaGetLastError());
+  const size_t mem_group = (size_t)c.max_seqs * H * 2 * c.max_len * DH;
+  for (int g = 0; g < c.mem_groups; g++) {
+    T *mg = M->at<T>(L.mem) + (size_t)g * mem_group;
+    RLT_TRY(gemm_k(M, K, ntok, d, d, etok, d, (const T *)w.mem_wk[g], d,
+                   EpiMem<T>{mg, tslot, tpos, H, DH, c.max_len, 0}, st));
+    RLT_TRY(gemm_k(M, K, ntok, d, d, etok, d, (const T *)w.mem_wv[g], d,
+                   EpiMem<T>{mg, tslot, tpos, H, DH, c.max_len, 1}, st));
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t get_window_impl(rlt_model *M, int seq, long t, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  if (c.window < 2) return cudaSuccess;
+  k_get_window<T><<<256, 256, 0, st>>>(c.n_dec_layers, c.n_heads, c.head_dim, c.window,
+                                       c.max_seqs, seq, t, M->at<T>(M->L.ring),
+                                       M->at<T>(M->L.staging));
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t set_window_impl(rlt_model *M, int seq, long t, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  if (c.window < 2) return cudaSuccess;
+  k_set_window<T><<<256, 256, 0, st>>>(c.n_dec_layers, c.n_heads, c.head_dim, c.window,
+                                       c.max_seqs, seq, t, M->at<T>(M->L.staging),
+                                       M->at<T>(M->L.ring));
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t get_memory_impl(rlt_model *M, int seq, int t_enc, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  if (t_enc == 0) return cudaSuccess;
+  k_get_memory<T><<<512, 256, 0, st>>>(c.mem_groups, c.n_heads, c.head_dim, c.max_seqs,
+                                       c.max_len, seq, t_enc, M->at<T>(M->L.mem),
+                                       M->at<T>(M->L.staging));
+  return cudaGetLastError();
+}
+
+template <typename T, int DH> void bind(rlt_model *M) {
+  M->step = step_impl<T, DH>;
+  M->prefill = prefill_impl<T, DH>;
+  M->get_window = get_window_impl<T>;
+  M->set_window = set_window_impl<T>;
+  M->get_memory = get_memory_impl<T>;
+}
+
+template <typename T> void bind_dh(rlt_model *M) {
+  switch (M->cfg.head_dim) {
+    case 16: bind<T, 16>(M); break;
+    case 32: bind<T, 32>(M); break;
+    case 64: bind<T, 64>(M); break;
+    default: bind<T, 128>(M); break;
+  }
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? RLT_OK : RLT_ERR_CUDA; }
+
+// Host mirrors of t_dec / t_enc -> device (stream ordered).
+cudaError_t push_positions(rlt_model *M, cudaStream_t st) {
+  size_t b = sizeof(int) * M->cfg.max_seqs;
+  RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.t_dec), M->t_dec.data(), b, cudaMemcpyHostToDevice, st));
+  return cudaMemcpyAsync(M->at<int>(M->L.t_enc), M->t_enc.data(), b, cudaMemcpyHostToDevice, st);
+}
+
+// Shared validation of a batch of sequence ids; `need` steps per sequence.
+int check_batch(const rlt_model *M, const int32_t *ids, int n, int need) {
+  if (!M || n < 0 || (n > 0 && !ids)) return RLT_ERR_INVALID_ARG;
+  if (n > M->cfg.max_seqs) return RLT_ERR_CAPACITY;
+  std::vector<char> seen(M->cfg.max_seqs, 0);
+  for (int i = 0; i < n; i++) {
+    int s = ids[i];
+    if (s < 0 || s >= M->cfg.max_seqs) return RLT_ERR_INVALID_ARG;
+    if (seen[s]) return RLT_ERR_DUPLICATE_ID;
+    seen[s] = 1;
+  }
+  for (int i = 0; i < n; i++) {
+    int s = ids[i];
+    if ((long)M->t_dec[s] + need > M->cfg.max_len) return RLT_ERR_CAPACITY;
+    if ((long)M->t_dec[s] + need > M->t_enc[s]) return RLT_ERR_NOT_READY;
+  }
+  return RLT_OK;
+}
+
+// Batch description for one step of the listed slots at their current t.
+StepInfo step_info(const rlt_model *M, const int32_t *ids, int n) {
+  StepInfo si{n, 1, 0.0, 0.0};
+  int tmax = 0;
+  for (int i = 0; i < n; i++) {
+    int t = M->t_dec[ids[i]];
+    tmax = std::max(tmax, t);
+    si.sum_keys += t + 1;
+    si.sum_win += std::min(t + 1, M->cfg.window);
+  }
+  si.xchunks = std::min(M->L.max_chunks, tmax / XCH + 1);
+  return si;
+}
+
+void advance(rlt_model *M, const int32_t *ids, int n) {
+  for (int i = 0; i < n; i++) M->t_dec[ids[i]] += 1;
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+extern "C" {
+
+RLT_API const char *rlt_status_string(int s) {
+  switch (s) {
+    case RLT_OK: return "ok";
+    case RLT_ERR_INVALID_ARG: return "invalid argument";
+    case RLT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RLT_ERR_NOT_READY: return "sequence not ready: encoder output for t_dec not produced";
+    case RLT_ERR_CAPACITY: return "capacity exceeded";
+    case RLT_ERR_DUPLICATE_ID: return "sequence listed twice in one batch";
+    case RLT_ERR_CUDA: return "CUDA runtime error";
+    case RLT_ERR_TIMEOUT: return "bounded device wait timed out";
+    case RLT_ERR_DEVICE: return "device-side check failed (bad token id)";
+    default: return "unknown status";
+  }
+}
+
+RLT_API int rlt_check_config(const rlt_config *cfg) { return check_config(cfg); }
+
+RLT_API size_t rlt_arena_bytes(const rlt_config *cfg) {
+  if (check_config(cfg) != RLT_OK) return 0;
+  Layout L;
+  return compute_layout(cfg, &L);
+}
+
+RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *w, void *d_arena,
+                       size_t arena_bytes, rlt_model **out) {
+  if (!out) return RLT_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = check_config(cfg);
+  if (rc != RLT_OK) return rc;
+  if (!w || !d_arena || ((uintptr_t)d_arena & 255)) return RLT_ERR_INVALID_ARG;
+  Layout L;
+  if (arena_bytes < compute_layout(cfg, &L)) return RLT_ERR_CAPACITY;
+  // every pointer the configuration reads must be present
+  bool ok = w->embed && w->enc_lnf && w->gate_b && w->sstar && w->dec_lnf;
+  if (cfg->alpha != 0.0f) ok = ok && w->gate_w;
+  for (int l = 0; l < cfg->n_enc_layers; l++) {
+    ok = ok && w->enc_ln1[l] && w->enc_wqkv[l] && w->enc_wo[l] && w->enc_ln2[l] && w->enc_w1[l] &&
+         w->enc_w2[l];
+    if (cfg->ffn_kind == RLT_SWIGLU) ok = ok && w->enc_wb[l];
+  }
+  for (int g = 0; g < cfg->mem_groups; g++) ok = ok && w->mem_wk[g] && w->mem_wv[g];
+  for (int l = 0; l < cfg->n_dec_layers; l++) {
+    ok = ok && w->dec_ln1[l] && w->dec_ln2[l] && w->dec_ln3[l] && w->dec_wqx[l] && w->dec_wox[l];
+    if (!cfg->tied) {
+      ok = ok && w->dec_wqkv[l] && w->dec_wo[l] && w->dec_w1[l] && w->dec_w2[l];
+      if (cfg->ffn_kind == RLT_SWIGLU) ok = ok && w->dec_wb[l];
+    }
+  }
+  if (!ok) return RLT_ERR_INVALID_ARG;
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, d_arena) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    return RLT_ERR_INVALID_ARG;
+  }
+  rlt_model *M = new (std::nothrow) rlt_model();
+  if (!M) return RLT_ERR_CAPACITY;
+  M->cfg = *cfg;
+  M->w = *w;
+  M->L = L;
+  M->arena = static_cast<uint8_t *>(d_arena);
+  M->device = pa.device;
+  M->t_dec.assign(cfg->max_seqs, 0);
+  M->t_enc.assign(cfg->max_seqs, 0);
+  if (cfg->dtype == RLT_BF16) bind_dh<bf16>(M); else bind_dh<float>(M);
+  cudaError_t e = cudaSetDevice(M->device);
+  int half = cfg->head_dim / 2;
+  if (e == cudaSuccess) e = cudaMemsetAsync(M->arena, 0, L.total, 0);
+  if (e == cudaSuccess) {
+    k_rope_table<<<blocks_for((long)cfg->max_len * half, 256), 256>>>(
+        M->at<float2>(L.rope), cfg->max_len, cfg->head_dim, (double)cfg->rope_theta);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) {
+    std::vector<int> ids(cfg->max_seqs);
+    for (int i = 0; i < cfg->max_seqs; i++) ids[i] = i;
+    e = cudaMemcpy(M->at<int>(L.ready), ids.data(), sizeof(int) * ids.size(),
+                   cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) {
+      k_reset_s<<<cfg->max_seqs, 128>>>(cfg->max_seqs, cfg->d, M->at<int>(L.ready),
+                                        (const float *)w->sstar, M->at<float>(L.s));
+      e = cudaGetLastError();
+    }
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    delete M;
+    return RLT_ERR_CUDA;
+  }
+  *out = M;
+  return RLT_OK;
+}
+
+RLT_API void rlt_destroy(rlt_model *M) {
+  if (!M) return;
+  cudaStreamSynchronize(M->last_stream);
+  for (auto &p : M->pending) {
+    cudaEventDestroy(p.a);
+    cudaEventDestroy(p.b);
+  }
+  for (auto e : M->ev_pool) cudaEventDestroy(e);
+  delete M;
+}
+
+RLT_API int rlt_reset_seq(rlt_model *M, int seq, rlt_stream stream) {
+  if (!M || seq < 0 || seq >= M->cfg.max_seqs) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->t_dec[seq] = 0;
+  M->t_enc[seq] = 0;
+  M->last_stream = st;
+  cudaError_t e = cudaMemcpyAsync(M->at<float>(M->L.s) + (size_t)seq * M->cfg.d, M->w.sstar,
+                                  sizeof(float) * M->cfg.d, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = push_positions(M, st);
+  return cuda_status(e);
+}
+
+RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32_t *ids,
+                                const int32_t *offsets, const int32_t *lengths, int n,
+                                rlt_stream stream) {
+  if (!M || n < 0 || (n > 0 && (!ids || !offsets || !lengths))) return RLT_ERR_INVALID_ARG;
+  if (n > M->cfg.max_seqs) return RLT_ERR_CAPACITY;
+  std::vector<char> seen(M->cfg.max_seqs, 0);
+  long total = 0;
+  for (int i = 0; i < n; i++) {
+    if (ids[i] < 0 || ids[i] >= M->cfg.max_seqs || offsets[i] < 0 || lengths[i] < 0)
+      return RLT_ERR_INVALID_ARG;
+    if (seen[ids[i]]) return RLT_ERR_DUPLICATE_ID;
+    seen[ids[i]] = 1;
+    if (lengths[i] > M->cfg.max_len) return RLT_ERR_CAPACITY;
+    total += lengths[i];
+  }
+  if (total > 0 && !tokens) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  const Layout &L = M->L;
+  std::vector<int> slot, pos, start;
+  int i = 0;
+  while (i < n) {
+    // pack whole sequences into one chunk of at most ptok tokens
+    int j = i;
+    long ntok = 0;
+    while (j < n && ntok + lengths[j] <= L.ptok) ntok += lengths[j++];
+    slot.assign(ntok, 0);
+    pos.assign(ntok, 0);
+    start.assign(ntok, 0);
+    long m = 0;
+    for (int k = i; k < j; k++) {
+      if (lengths[k] == 0) continue;
+      cudaError_t e = cudaMemcpyAsync(M->at<int>(L.tok) + m, tokens + offsets[k],
+                                      sizeof(int32_t) * lengths[k], cudaMemcpyDefault, st);
+      if (e != cudaSuccess) return RLT_ERR_CUDA;
+      for (int p = 0; p < lengths[k]; p++, m++) {
+        slot[m] = ids[k];
+        pos[m] = p;
+        start[m] = (int)(m - p);
+      }
+    }
+    if (ntok > 0) {
+      cudaError_t e = cudaMemcpyAsync(M->at<int>(L.tok_slot), slot.data(), 4 * ntok,
+                                      cudaMemcpyHostToDevice, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(M->at<int>(L.tok_pos), pos.data(), 4 * ntok, cudaMemcpyHostToDevice, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(M->at<int>(L.tok_start), start.data(), 4 * ntok,
+                            cudaMemcpyHostToDevice, st);
+      if (e == cudaSuccess) e = M->prefill(M, (int)ntok, st);
+      if (e != cudaSuccess) return RLT_ERR_CUDA;
+      // the host vectors are reused next chunk: pageable copies are staged
+      // at enqueue time, so reuse is safe
+    }
+    i = j;
+  }
+  // prefill starts every listed slot afresh: s*, empty cache, t_dec = 0
+  std::vector<int> idv(ids, ids + n);
+  for (int k = 0; k < n; k++) {
+    M->t_enc[ids[k]] = lengths[k];
+    M->t_dec[ids[k]] = 0;
+  }
+  cudaError_t e = cudaSuccess;
+  if (n > 0) {
+    e = cudaMemcpyAsync(M->at<int>(L.ready), idv.data(), 4 * n, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) {
+      k_reset_s<<<n, 128, 0, st>>>(n, M->cfg.d, M->at<int>(L.ready), (const float *)M->w.sstar,
+                                   M->at<float>(L.s));
+      e = cudaGetLastError();
+    }
+  }
+  if (e == cudaSuccess) e = push_positions(M, st);
+  return cuda_status(e);
+}
+
+RLT_API int rlt_decoder_step(rlt_model *M, const int32_t *ids, int n, rlt_stream stream) {
+  int rc = check_batch(M, ids, n, 1);
+  if (rc != RLT_OK || n == 0) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  std::vector<int32_t> idv(ids, ids + n);  // pageable copy: read before return
+  cudaError_t e = cudaMemcpyAsync(M->at<int>(M->L.ready), idv.data(), 4 * n,
+                                  cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = M->step(M, step_info(M, ids, n), st);
+  if (e != cudaSuccess) return RLT_ERR_CUDA;
+  advance(M, ids, n);
+  return RLT_OK;
+}
+
+RLT_API int rlt_run_sequence(rlt_model *M, const int32_t *ids, int n, int n_steps,
+                             rlt_stream stream) {
+  if (n_steps < 0) return RLT_ERR_INVALID_ARG;
+  int rc = check_batch(M, ids, n, n_steps);
+  if (rc != RLT_OK || n == 0 || n_steps == 0) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  std::vector<int32_t> idv(ids, ids + n);
+  cudaError_t e = cudaMemcpyAsync(M->at<int>(M->L.ready), idv.data(), 4 * n,
+                                  cudaMemcpyHostToDevice, st);
+  for (int k = 0; k < n_steps && e == cudaSuccess; k++) {
+    e = M->step(M, step_info(M, idv.data(), n), st);
+    advance(M, idv.data(), n);
+  }
+  return cuda_status(e);
+}
+
+RLT_API int rlt_plan_ragged(const int32_t *steps, int n, int32_t *order, int32_t *tick_sizes,
+                            int max_ticks, int *n_ticks) {
+  if (n < 0 || (n > 0 && (!steps || !order)) || !n_ticks) return RLT_ERR_INVALID_ARG;
+  int tmax = 0;
+  for (int i = 0; i < n; i++) {
+    if (steps[i] < 0) return RLT_ERR_INVALID_ARG;
+    tmax = std::max(tmax, (int)steps[i]);
+  }
+  if (tmax > max_ticks || (tmax > 0 && !tick_sizes)) return RLT_ERR_CAPACITY;
+  std::vector<int> idx(n);
+  for (int i = 0; i < n; i++) idx[i] = i;
+  // longest first: tick k batches the prefix of sequences with steps > k
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return steps[a] > steps[b]; });
+  for (int i = 0; i < n; i++) order[i] = idx[i];
+  int c = n;
+  for (int k = 0; k < tmax; k++) {
+    while (c > 0 && steps[idx[c - 1]] <= k) c--;
+    tick_sizes[k] = c;
+  }
+  *n_ticks = tmax;
+  return RLT_OK;
+}
+
+RLT_API int rlt_run_ragged(rlt_model *M, const int32_t *ids, const int32_t *steps, int n,
+                           rlt_stream stream) {
+  if (!M || n < 0 || (n > 0 && (!ids || !steps))) return RLT_ERR_INVALID_ARG;
+  if (n > M->cfg.max_seqs) return RLT_ERR_CAPACITY;
+  int tmax = 0;
+  for (int i = 0; i < n; i++) {
+    if (steps[i] < 0) return RLT_ERR_INVALID_ARG;
+    tmax = std::max(tmax, (int)steps[i]);
+  }
+  // every tick of every sequence is checked up front (all or nothing)
+  std::vector<char> seen(M->cfg.max_seqs, 0);
+  for (int i = 0; i < n; i++) {
+    int s = ids[i];
+    if (s < 0 || s >= M->cfg.max_seqs) return RLT_ERR_INVALID_ARG;
+    if (seen[s]) return RLT_ERR_DUPLICATE_ID;
+    seen[s] = 1;
+  }
+  for (int i = 0; i < n; i++) {
+    int s = ids[i];
+    if ((long)M->t_dec[s] + steps[i] > M->cfg.max_len) return RLT_ERR_CAPACITY;
+    if ((long)M->t_dec[s] + steps[i] > M->t_enc[s]) return RLT_ERR_NOT_READY;
+  }
+  if (tmax == 0) return RLT_OK;
+  std::vector<int> order(n), sizes(tmax), sorted(n);
+  int nt = 0;
+  rlt_plan_ragged(steps, n, order.data(), sizes.data(), tmax, &nt);
+  for (int i = 0; i < n; i++) sorted[i] = ids[order[i]];
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  cudaError_t e = cudaMemcpyAsync(M->at<int>(M->L.ready), sorted.data(), 4 * n,
+                                  cudaMemcpyHostToDevice, st);
+  for (int k = 0; k < nt && e == cudaSuccess; k++) {
+    int c = sizes[k];
+    e = M->step(M, step_info(M, sorted.data(), c), st);
+    advance(M, sorted.data(), c);
+  }
+  return cuda_status(e);
+}
+
+RLT_API int rlt_get_state(rlt_model *M, int seq, float *s_out, void *cache_out, int64_t *t_out,
+                          rlt_stream stream) {
+  if (!M || seq < 0 || seq >= M->cfg.max_seqs) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  const rlt_config &c = M->cfg;
+  long t = M->t_dec[seq];
+  if (t_out) *t_out = t;
+  cudaError_t e = cudaSuccess;
+  if (s_out)
+    e = cudaMemcpyAsync(s_out, M->at<float>(M->L.s) + (size_t)seq * c.d, sizeof(float) * c.d,
+                        cudaMemcpyDefault, st);
+  if (e == cudaSuccess && cache_out && c.window > 1) {
+    size_t bytes = (size_t)c.n_dec_layers * 2 * (c.window - 1) * c.d * elem_size(&c);
+    e = M->get_window(M, seq, t, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(cache_out, M->at<uint8_t>(M->L.staging), bytes, cudaMemcpyDefault, st);
+  }
+  return cuda_status(e);
+}
+
+RLT_API int rlt_set_state(rlt_model *M, int seq, const float *s_in, const void *cache_in,
+                          int64_t t, rlt_stream stream) {
+  if (!M || seq < 0 || seq >= M->cfg.max_seqs || t < 0 || t > M->cfg.max_len)
+    return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  const rlt_config &c = M->cfg;
+  cudaError_t e = cudaSuccess;
+  if (s_in)
+    e = cudaMemcpyAsync(M->at<float>(M->L.s) + (size_t)seq * c.d, s_in, sizeof(float) * c.d,
+                        cudaMemcpyDefault, st);
+  if (e == cudaSuccess && cache_in && c.window > 1) {
+    size_t bytes = (size_t)c.n_dec_layers * 2 * (c.window - 1) * c.d * elem_size(&c);
+    e = cudaMemcpyAsync(M->at<uint8_t>(M->L.staging), cache_in, bytes, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = M->set_window(M, seq, (long)t, st);
+  }
+  if (e != cudaSuccess) return RLT_ERR_CUDA;
+  M->t_dec[seq] = (int)t;
+  return cuda_status(push_positions(M, st));
+}
+
+RLT_API int rlt_get_encoder_output(rlt_model *M, int seq, void *e_out, void *mem_out,
+                                   int64_t *t_enc_out, rlt_stream stream) {
+  if (!M || seq < 0 || seq >= M->cfg.max_seqs) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  const rlt_config &c = M->cfg;
+  int te = M->t_enc[seq];
+  if (t_enc_out) *t_enc_out = te;
+  size_t es = elem_size(&c);
+  cudaError_t e = cudaSuccess;
+  if (e_out && te > 0)
+    e = cudaMemcpyAsync(e_out, M->at<uint8_t>(M->L.e) + (size_t)seq * c.max_len * c.d * es,
+                        (size_t)te * c.d * es, cudaMemcpyDefault, st);
+  if (e == cudaSuccess && mem_out && te > 0) {
+    e = M->get_memory(M, seq, te, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(mem_out, M->at<uint8_t>(M->L.staging),
+                          (size_t)c.mem_groups * te * 2 * c.d * es, cudaMemcpyDefault, st);
+  }
+  return cuda_status(e);
+}
+
+RLT_API int rlt_profile(rlt_model *M, int enable) {
+  if (!M) return RLT_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(M->last_stream) != cudaSuccess) return RLT_ERR_CUDA;
+  for (auto &p : M->pending) {
+    M->ev_pool.push_back(p.a);
+    M->ev_pool.push_back(p.b);
+  }
+  M->pending.clear();
+  int64_t launches = M->stats.launches;
+  M->stats = rlt_stats{};
+  M->stats.launches = launches;
+  M->profiling = enable != 0;
+  return RLT_OK;
+}
+
+RLT_API int rlt_get_stats(rlt_model *M, rlt_stats *out) {
+  if (!M || !out) return RLT_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(M->last_stream) != cudaSuccess) return RLT_ERR_CUDA;
+  for (auto &p : M->pending) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+      M->stats.kernel_ms[p.kind] += ms;
+      M->stats.kernel_launches[p.kind] += 1;
+      M->stats.kernel_bytes[p.kind] += p.bytes;
+      M->stats.kernel_flops[p.kind] += p.flops;
+    } else {
+      cudaGetLastError();
+    }
+    M->ev_pool.push_back(p.a);
+    M->ev_pool.push_back(p.b);
+  }
+  M->pending.clear();
+  *out = M->stats;
+  return RLT_OK;
+}
+
+RLT_API int rlt_poll_device_error(rlt_model *M) {
+  if (!M) return RLT_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(M->last_stream) != cudaSuccess) return RLT_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, M->at<int>(M->L.err), sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return RLT_ERR_CUDA;
+  if (v != 0 && cudaMemset(M->at<int>(M->L.err), 0, sizeof(int)) != cudaSuccess)
+    return RLT_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,327 @@
+"""Python binding of the RLT C ABI (``include/rlt.h``): argument marshalling only.
+
+Every step of the path runs in ``librlt.so``'s kernels. PyTorch provides the
+device memory (weights, arena, outputs) and the CUDA streams. There is no CPU
+fallback: if the library is missing, importing a model raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+from typing import Dict, Optional
+
+import numpy as np
+
+from .configs import BF16, SWIGLU, RLTConfig
+
+MAX_LAYERS = 64
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librlt.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "rlt.h")
+
+RLT_OK = 0
+STATUS = {0: "RLT_OK", 1: "RLT_ERR_INVALID_ARG", 2: "RLT_ERR_UNSUPPORTED",
+          3: "RLT_ERR_NOT_READY", 4: "RLT_ERR_CAPACITY", 5: "RLT_ERR_DUPLICATE_ID",
+          6: "RLT_ERR_CUDA", 7: "RLT_ERR_TIMEOUT", 8: "RLT_ERR_DEVICE"}
+
+
+class RLTError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} "
+                         f"({_lib().rlt_status_string(status).decode()})")
+
+
+class rlt_config(C.Structure):
+    _fields_ = [(n, C.c_int) for n in (
+        "d", "n_heads", "head_dim", "n_enc_layers", "n_dec_layers", "ffn_dim",
+        "ffn_kind", "vocab", "window", "mem_groups", "tied", "dtype", "max_seqs",
+        "max_len", "max_prefill_tokens")] + [
+        ("alpha", C.c_float), ("rms_eps", C.c_float), ("rope_theta", C.c_float)]
+
+
+_ENC = ("enc_ln1", "enc_wqkv", "enc_wo", "enc_ln2", "enc_w1", "enc_wb", "enc_w2")
+_DEC = ("dec_ln1", "dec_wqkv", "dec_wo", "dec_ln2", "dec_wqx", "dec_wox", "dec_ln3",
+        "dec_w1", "dec_wb", "dec_w2")
+
+
+class rlt_weights(C.Structure):
+    _fields_ = ([("embed", C.c_void_p)]
+                + [(n, C.c_void_p * MAX_LAYERS) for n in _ENC]
+                + [("enc_lnf", C.c_void_p)]
+                + [("mem_wk", C.c_void_p * MAX_LAYERS), ("mem_wv", C.c_void_p * MAX_LAYERS)]
+                + [("gate_w", C.c_void_p), ("gate_b", C.c_void_p), ("sstar", C.c_void_p)]
+                + [(n, C.c_void_p * MAX_LAYERS) for n in _DEC]
+                + [("dec_lnf", C.c_void_p)])
+
+
+K_XATTN, K_SWA, K_GEMM, K_OTHER, K_ENC = range(5)
+K_NAMES = ("xattn", "swa", "gemm", "other", "encoder")
+
+
+class rlt_stats(C.Structure):
+    _fields_ = [("launches", C.c_int64), ("kernel_launches", C.c_int64 * 5),
+                ("kernel_ms", C.c_double * 5), ("kernel_bytes", C.c_double * 5),
+                ("kernel_flops", C.c_double * 5)]
+
+
+_LIB = None
+
+
+def _declare(lib):
+    P, I = C.c_void_p, C.c_int
+    lib.rlt_check_config.argtypes = [P]
+    lib.rlt_arena_bytes.argtypes = [P]
+    lib.rlt_arena_bytes.restype = C.c_size_t
+    lib.rlt_create.argtypes = [P, P, P, C.c_size_t, C.POINTER(P)]
+    lib.rlt_destroy.argtypes = [P]
+    lib.rlt_destroy.restype = None
+    lib.rlt_reset_seq.argtypes = [P, I, P]
+    lib.rlt_prefill_encoder.argtypes = [P, P, P, P, P, I, P]
+    lib.rlt_decoder_step.argtypes = [P, P, I, P]
+    lib.rlt_run_sequence.argtypes = [P, P, I, I, P]
+    lib.rlt_run_ragged.argtypes = [P, P, P, I, P]
+    lib.rlt_plan_ragged.argtypes = [P, I, P, P, I, C.POINTER(I)]
+    lib.rlt_get_state.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
+    lib.rlt_set_state.argtypes = [P, I, P, P, C.c_int64, P]
+    lib.rlt_get_encoder_output.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
+    lib.rlt_poll_device_error.argtypes = [P]
+    lib.rlt_profile.argtypes = [P, I]
+    lib.rlt_get_stats.argtypes = [P, P]
+    lib.rlt_status_string.argtypes = [I]
+    lib.rlt_status_string.restype = C.c_char_p
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"librlt.so not built ({LIB_PATH}); run "
+                               "python -m token_recurrent_decoding_b200.build")
+        lib = C.CDLL(LIB_PATH)
+        _declare(lib)
+        _LIB = lib
+    return _LIB
+
+
+def header_symbols():
+    """Function names the public header declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RLT_API\s+[\w\s\*]+?\b(rlt_\w+)\s*\(", text)))
+
+
+def _check(rc: int, what: str):
+    if rc != RLT_OK:
+        raise RLTError(rc, what)
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def make_config(cfg: RLTConfig, max_seqs: int, max_len: int, max_prefill_tokens: int = 0):
+    return rlt_config(cfg.d, cfg.n_heads, cfg.head_dim, cfg.n_enc, cfg.n_dec, cfg.ffn_dim,
+                      cfg.ffn_kind, cfg.vocab, cfg.window, cfg.mem_groups, int(cfg.tied),
+                      cfg.dtype, max_seqs, max_len, max_prefill_tokens, float(cfg.alpha),
+                      float(cfg.rms_eps), float(cfg.rope_theta))
+
+
+def check_config(cfg: RLTConfig, max_seqs: int, max_len: int) -> int:
+    c = make_config(cfg, max_seqs, max_len)
+    return _lib().rlt_check_config(C.byref(c))
+
+
+def arena_bytes(cfg: RLTConfig, max_seqs: int, max_len: int, max_prefill_tokens: int = 0) -> int:
+    c = make_config(cfg, max_seqs, max_len, max_prefill_tokens)
+    return int(_lib().rlt_arena_bytes(C.byref(c)))
+
+
+def plan_ragged(steps):
+    """Host-only scheduler plan: (order, tick sizes)."""
+    st = _i32(steps)
+    n = st.shape[0]
+    order = np.zeros(max(n, 1), np.int32)
+    tmax = int(st.max()) if n else 0
+    sizes = np.zeros(max(tmax, 1), np.int32)
+    nt = C.c_int(0)
+    _check(_lib().rlt_plan_ragged(_p(st), n, _p(order), _p(sizes), max(tmax, 1), C.byref(nt)),
+           "rlt_plan_ragged")
+    return order[:n], sizes[: nt.value]
+
+
+class Model:
+    """One RLT model bound to device weights and a device arena.
+
+    ``weights`` maps the generator's tensor names to numpy float32 arrays (the
+    bf16 values for bf16 models); they are uploaded once with torch.
+    """
+
+    def __init__(self, cfg: RLTConfig, weights: Dict[str, np.ndarray], max_seqs: int,
+                 max_len: int, device: str = "cuda", max_prefill_tokens: int = 0,
+                 stream=None):
+        import torch
+        self.torch = torch
+        self.cfg = cfg
+        self.max_seqs, self.max_len = max_seqs, max_len
+        self.device = torch.device(device)
+        self.wdtype = torch.bfloat16 if cfg.dtype == BF16 else torch.float32
+        self.stream = stream
+        lib = _lib()
+        self._c = make_config(cfg, max_seqs, max_len, max_prefill_tokens)
+        rc = lib.rlt_check_config(C.byref(self._c))
+        _check(rc, "rlt_check_config")
+        self.arena_bytes = int(lib.rlt_arena_bytes(C.byref(self._c)))
+        self._dev = {}
+        w = rlt_weights()
+
+        def up(name, matrix=True):
+            src = weights[name]
+            key = id(src)
+            if key not in self._dev:  # tied names share one device tensor
+                t = torch.from_numpy(np.ascontiguousarray(src, dtype=np.float32))
+                t = t.to(self.device)
+                if matrix:
+                    t = t.to(self.wdtype)
+                self._dev[key] = t
+            return self._dev[key].data_ptr()
+
+        sw = cfg.ffn_kind == SWIGLU
+        w.embed = up("embed")
+        for l in range(cfg.n_enc):
+            w.enc_ln1[l] = up(f"enc.{l}.ln1", False)
+            w.enc_wqkv[l] = up(f"enc.{l}.wqkv")
+            w.enc_wo[l] = up(f"enc.{l}.wo")
+            w.enc_ln2[l] = up(f"enc.{l}.ln2", False)
+            w.enc_w1[l] = up(f"enc.{l}.wa" if sw else f"enc.{l}.w1")
+            if sw:
+                w.enc_wb[l] = up(f"enc.{l}.wb")
+            w.enc_w2[l] = up(f"enc.{l}.w2")
+        w.enc_lnf = up("enc.lnf", False)
+        for g in range(cfg.mem_groups):
+            w.mem_wk[g] = up(f"mem.{g}.wk")
+            w.mem_wv[g] = up(f"mem.{g}.wv")
+        w.gate_w = up("gate.w")
+        w.gate_b = up("gate.b", False)
+        w.sstar = up("sstar", False)
+        for l in range(cfg.n_dec):
+            w.dec_ln1[l] = up(f"dec.{l}.ln1", False)
+            w.dec_ln2[l] = up(f"dec.{l}.ln2", False)
+            w.dec_ln3[l] = up(f"dec.{l}.ln3", False)
+            w.dec_wqx[l] = up(f"dec.{l}.wqx")
+            w.dec_wox[l] = up(f"dec.{l}.wox")
+            if not cfg.tied:
+                w.dec_wqkv[l] = up(f"dec.{l}.wqkv")
+                w.dec_wo[l] = up(f"dec.{l}.wo")
+                w.dec_w1[l] = up(f"dec.{l}.wa" if sw else f"dec.{l}.w1")
+                if sw:
+                    w.dec_wb[l] = up(f"dec.{l}.wb")
+                w.dec_w2[l] = up(f"dec.{l}.w2")
+        w.dec_lnf = up("dec.lnf", False)
+        self._w = w
+        self.arena = torch.empty(self.arena_bytes, dtype=torch.uint8, device=self.device)
+        torch.cuda.synchronize(self.device)
+        h = C.c_void_p()
+        _check(lib.rlt_create(C.byref(self._c), C.byref(w), C.c_void_p(self.arena.data_ptr()),
+                              self.arena_bytes, C.byref(h)), "rlt_create")
+        self._h = h
+
+    # ------------------------------------------------------------------
+    def _st(self, stream=None):
+        s = stream if stream is not None else self.stream
+        if s is None:
+            s = self.torch.cuda.current_stream(self.device)
+        return C.c_void_p(s.cuda_stream)
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib().rlt_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- the C-ABI calls, same names ------------------------------------
+    def reset_seq(self, seq: int, stream=None):
+        _check(_lib().rlt_reset_seq(self._h, seq, self._st(stream)), "rlt_reset_seq")
+
+    def prefill_encoder(self, tokens, seq_ids, offsets, lengths, stream=None):
+        """tokens: torch int32 tensor (device or pinned host)."""
+        ids, off, lens = _i32(seq_ids), _i32(offsets), _i32(lengths)
+        self._tok_keep = tokens
+        _check(_lib().rlt_prefill_encoder(self._h, C.c_void_p(tokens.data_ptr()), _p(ids),
+                                          _p(off), _p(lens), ids.shape[0], self._st(stream)),
+               "rlt_prefill_encoder")
+
+    def decoder_step(self, ready_ids, stream=None):
+        ids = _i32(ready_ids)
+        _check(_lib().rlt_decoder_step(self._h, _p(ids), ids.shape[0], self._st(stream)),
+               "rlt_decoder_step")
+
+    def run_sequence(self, seq_ids, n_steps: int, stream=None):
+        ids = _i32(seq_ids)
+        _check(_lib().rlt_run_sequence(self._h, _p(ids), ids.shape[0], int(n_steps),
+                                       self._st(stream)), "rlt_run_sequence")
+
+    def run_ragged(self, seq_ids, steps, stream=None):
+        ids, st = _i32(seq_ids), _i32(steps)
+        _check(_lib().rlt_run_ragged(self._h, _p(ids), _p(st), ids.shape[0], self._st(stream)),
+               "rlt_run_ragged")
+
+    def get_state(self, seq: int, stream=None):
+        """(s [d] float32, cache [L_D][2][W-1][d] model dtype, t) as device tensors."""
+        torch = self.torch
+        c = self.cfg
+        s = torch.empty(c.d, dtype=torch.float32, device=self.device)
+        cache = torch.zeros((c.n_dec, 2, max(c.window - 1, 0), c.d), dtype=self.wdtype,
+                            device=self.device)
+        t = C.c_int64(0)
+        _check(_lib().rlt_get_state(self._h, seq, C.c_void_p(s.data_ptr()),
+                                    C.c_void_p(cache.data_ptr()) if cache.numel() else None,
+                                    C.byref(t), self._st(stream)), "rlt_get_state")
+        return s, cache, int(t.value)
+
+    def set_state(self, seq: int, s, cache, t: int, stream=None):
+        self._set_keep = (s, cache)
+        _check(_lib().rlt_set_state(self._h, seq,
+                                    C.c_void_p(s.data_ptr()) if s is not None else None,
+                                    C.c_void_p(cache.data_ptr()) if cache is not None and cache.numel() else None,
+                                    int(t), self._st(stream)), "rlt_set_state")
+
+    def get_encoder_output(self, seq: int, stream=None):
+        """(e [t_enc][d], mem [G][t_enc][2][d]) device tensors in the model dtype."""
+        torch = self.torch
+        c = self.cfg
+        t = C.c_int64(0)
+        _check(_lib().rlt_get_encoder_output(self._h, seq, None, None, C.byref(t),
+                                             self._st(stream)), "rlt_get_encoder_output")
+        te = int(t.value)
+        e = torch.empty((te, c.d), dtype=self.wdtype, device=self.device)
+        mem = torch.empty((c.mem_groups, te, 2, c.d), dtype=self.wdtype, device=self.device)
+        if te:
+            _check(_lib().rlt_get_encoder_output(self._h, seq, C.c_void_p(e.data_ptr()),
+                                                 C.c_void_p(mem.data_ptr()), C.byref(t),
+                                                 self._st(stream)), "rlt_get_encoder_output")
+        return e, mem
+
+    def profile(self, enable: bool):
+        _check(_lib().rlt_profile(self._h, int(bool(enable))), "rlt_profile")
+
+    def get_stats(self) -> dict:
+        st = rlt_stats()
+        _check(_lib().rlt_get_stats(self._h, C.byref(st)), "rlt_get_stats")
+        out = {"launches": int(st.launches)}
+        for k, name in enumerate(K_NAMES):
+            out[name] = {"launches": int(st.kernel_launches[k]), "ms": float(st.kernel_ms[k]),
+                         "bytes": float(st.kernel_bytes[k]), "flops": float(st.kernel_flops[k])}
+        return out
+
+    def poll_device_error(self) -> int:
+        return int(_lib().rlt_poll_device_error(self._h))
