@@ -197,7 +197,7 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    r.m.profile(True)
+    r.m.profile(args.profile_stride)
     launches0 = r.m.get_stats()["launches"]
     clk = ClockSampler(torch.cuda.current_device())
     with clk:
@@ -215,7 +215,7 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
         torch.cuda.synchronize()
         barrier(dist)
     stats = r.m.get_stats()
-    r.m.profile(False)
+    r.m.profile(0)
     total_ms = t0.elapsed_time(t1)
     enc_ms = sum(a.elapsed_time(b) for a, b, _ in evs)
     dec_ms = sum(b.elapsed_time(c) for _, b, c in evs)
@@ -372,6 +372,8 @@ def main():
                     help="one JSON line per workload (not the default contract line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-positions", type=int, default=24)
+    ap.add_argument("--profile-stride", type=int, default=16,
+                    help="event-time every k-th decoder step for the per-kernel roofline")
     args = ap.parse_args()
 
     if args.impl == "reference":

@@ -164,8 +164,10 @@ RLT_API int rlt_decoder_step(rlt_model *model, const int32_t *h_ready_ids,
 
 /* n_steps lock-step transitions of the listed sequences (every sequence must
  * have n_steps positions ready). Equivalent to n_steps rlt_decoder_step calls
- * with the same list; a non-NULL stream lets the steps replay as one CUDA
- * graph. */
+ * with the same list. On a non-NULL stream every step after the first of its
+ * shape replays a captured CUDA graph (the graphs are cached in the model and
+ * keyed by the batch bound and the cross-attention split count), so the first
+ * call on such a stream must not itself be inside a stream capture. */
 RLT_API int rlt_run_sequence(rlt_model *model, const int32_t *h_seq_ids, int n,
                              int n_steps, rlt_stream stream);
 
@@ -222,11 +224,13 @@ typedef struct rlt_stats {
   double kernel_flops[RLT_K_COUNT];    /* algorithmic FLOPs of those launches */
 } rlt_stats;
 
-/* Measurement hook (no counterpart in the method): while enabled, every
- * kernel launch is bracketed by a pair of CUDA events on its own stream and
- * attributed to a class with the bytes/FLOPs the algorithm must move for it
- * (weights once per launch; K/V rows actually attended; activations).
- * Enabling or disabling clears the accumulated per-class figures. */
+/* Measurement hook (no counterpart in the method). enable = k > 0: every
+ * k-th decoder step (and every encoder prefill) runs with each kernel launch
+ * bracketed by a pair of CUDA events on its own stream and attributed to a
+ * class with the bytes/FLOPs the algorithm must move for it (weights once per
+ * launch; K/V rows actually attended; activations). The other steps replay
+ * unprofiled. enable = 0 turns it off. Either call clears the per-class sums
+ * (the launch counter keeps running). Synchronises the model's last stream. */
 RLT_API int rlt_profile(rlt_model *model, int enable);
 
 /* Synchronises the model's last stream, folds every completed event pair

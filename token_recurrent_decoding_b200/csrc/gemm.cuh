@@ -102,8 +102,8 @@ __device__ __forceinline__ int swz(int r, int c) { return r * GEMM_BK + ((c ^ (r
 
 template <int BM, int BN, int WM, int WN, int STAGES, class Epi>
 __global__ void __launch_bounds__(WM *WN * 32)
-    k_gemm_bf16(int M, int N, int K, const bf16 *__restrict__ A, int lda,
-                const bf16 *__restrict__ B, int ldb, Epi epi) {
+    k_gemm_bf16(int M, const int *__restrict__ Mdev, int N, int K, const bf16 *__restrict__ A,
+                int lda, const bf16 *__restrict__ B, int ldb, Epi epi) {
   constexpr int NT = WM * WN * 32;
   constexpr int TM = BM / WM, TN = BN / WN;
   constexpr int FM = TM / 16, FN = TN / 8;
@@ -115,6 +115,8 @@ __global__ void __launch_bounds__(WM *WN * 32)
   const int wm = warp / WN, wn = warp % WN;
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
   const int KT = K / GEMM_BK;
+  if (Mdev) M = *Mdev;  // rows decided on the device (grid sized for an upper bound)
+  if (m0 >= M) return;
 
   auto load_stage = [&](int st, int kt) {
     bf16 *as = As + st * BM * GEMM_BK;
@@ -199,12 +201,14 @@ __global__ void __launch_bounds__(WM *WN * 32)
 // 64x64 output tile, 256 threads, 4x4 outputs per thread, K in steps of 16.
 template <class Epi>
 __global__ void __launch_bounds__(256)
-    k_gemm_f32(int M, int N, int K, const float *__restrict__ A, int lda,
-               const float *__restrict__ B, int ldb, Epi epi) {
+    k_gemm_f32(int M, const int *__restrict__ Mdev, int N, int K, const float *__restrict__ A,
+               int lda, const float *__restrict__ B, int ldb, Epi epi) {
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  if (Mdev) M = *Mdev;
+  if (m0 >= M) return;
   float acc[4][4] = {};
   for (int k0 = 0; k0 < K; k0 += 16) {
     for (int i = tid; i < 64 * 16; i += 256) {
@@ -242,8 +246,8 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------------ launchers
 template <int BM, int BN, int WM, int WN, int STAGES, class Epi>
-cudaError_t launch_gemm_bf16_cfg(int M, int N, int K, const bf16 *A, int lda, const bf16 *B,
-                                 int ldb, Epi epi, cudaStream_t st) {
+cudaError_t launch_gemm_bf16_cfg(int M, const int *Mdev, int N, int K, const bf16 *A, int lda,
+                                 const bf16 *B, int ldb, Epi epi, cudaStream_t st) {
   constexpr int smem = STAGES * (BM + BN) * GEMM_BK * 2;
   auto kern = k_gemm_bf16<BM, BN, WM, WN, STAGES, Epi>;
   static bool attr_set = false;  // per template instance
@@ -253,26 +257,28 @@ cudaError_t launch_gemm_bf16_cfg(int M, int N, int K, const bf16 *A, int lda, co
     attr_set = true;
   }
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-  kern<<<grid, WM * WN * 32, smem, st>>>(M, N, K, A, lda, B, ldb, epi);
+  kern<<<grid, WM * WN * 32, smem, st>>>(M, Mdev, N, K, A, lda, B, ldb, epi);
   return cudaGetLastError();
 }
 
 // Tile choice: large M (encoder) uses 128x128 tiles; the decoder's small
-// batches use 64x64 tiles so more SMs stream the weights.
+// batches use 64x64 tiles so more SMs stream the weights. M is the grid's row
+// bound; Mdev (optional) gives the actual rows at run time (<= M).
 template <class Epi>
-cudaError_t gemm(int M, int N, int K, const bf16 *A, int lda, const bf16 *B, int ldb, Epi epi,
-                 cudaStream_t st) {
+cudaError_t gemm(int M, const int *Mdev, int N, int K, const bf16 *A, int lda, const bf16 *B,
+                 int ldb, Epi epi, cudaStream_t st) {
   if (M <= 0 || N <= 0) return cudaSuccess;
-  if (M >= 1024) return launch_gemm_bf16_cfg<128, 128, 2, 4, 3>(M, N, K, A, lda, B, ldb, epi, st);
-  return launch_gemm_bf16_cfg<64, 64, 2, 2, 4>(M, N, K, A, lda, B, ldb, epi, st);
+  if (M >= 1024)
+    return launch_gemm_bf16_cfg<128, 128, 2, 4, 3>(M, Mdev, N, K, A, lda, B, ldb, epi, st);
+  return launch_gemm_bf16_cfg<64, 64, 2, 2, 4>(M, Mdev, N, K, A, lda, B, ldb, epi, st);
 }
 
 template <class Epi>
-cudaError_t gemm(int M, int N, int K, const float *A, int lda, const float *B, int ldb, Epi epi,
-                 cudaStream_t st) {
+cudaError_t gemm(int M, const int *Mdev, int N, int K, const float *A, int lda, const float *B,
+                 int ldb, Epi epi, cudaStream_t st) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + 63) / 64, (M + 63) / 64);
-  k_gemm_f32<Epi><<<grid, 256, 0, st>>>(M, N, K, A, lda, B, ldb, epi);
+  k_gemm_f32<Epi><<<grid, 256, 0, st>>>(M, Mdev, N, K, A, lda, B, ldb, epi);
   return cudaGetLastError();
 }
 

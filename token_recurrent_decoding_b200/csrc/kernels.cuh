@@ -27,9 +27,11 @@ __global__ void k_rope_table(float2 *tab, int max_len, int dh, double theta) {
 // ------------------------------------------------------------------ norms
 // out[r] = x[r] / sqrt(mean(x[r]^2) + eps) * gamma, one warp per row.
 template <typename T>
-__global__ void k_rmsnorm(int rows, int d, const float *__restrict__ x,
-                          const float *__restrict__ gamma, float eps, T *__restrict__ out) {
+__global__ void k_rmsnorm(int rows, const int *__restrict__ rows_dev, int d,
+                          const float *__restrict__ x, const float *__restrict__ gamma, float eps,
+                          T *__restrict__ out) {
   int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (rows_dev) rows = *rows_dev;
   if (r >= rows) return;
   const float *xr = x + (size_t)r * d;
   float ss = 0.f;
@@ -54,13 +56,14 @@ __global__ void k_rmsnorm(int rows, int d, const float *__restrict__ x,
 // Step start: position of each ready slot, GEMM input [e_t ; s_{t-1}] and fp32
 // copies for the gated merge. With feedback off the residual is e_t itself.
 template <typename T>
-__global__ void k_step_gather(int n, int d, int max_len, const int *__restrict__ ready,
+__global__ void k_step_gather(const int *__restrict__ n_dev, int d, int max_len,
+                              const int *__restrict__ ready,
                               const int *__restrict__ t_dec, int *__restrict__ pos,
                               const T *__restrict__ e, const float *__restrict__ s,
                               T *__restrict__ xin, float *__restrict__ e32,
                               float *__restrict__ s32, float *__restrict__ h, int alpha_zero) {
   int i = blockIdx.x;
-  if (i >= n) return;
+  if (i >= *n_dev) return;
   int seq = ready[i];
   int t = t_dec[seq];
   if (threadIdx.x == 0) pos[i] = t;
@@ -82,13 +85,13 @@ __global__ void k_step_gather(int n, int d, int max_len, const int *__restrict__
 // plain v written into ring slot t mod W of this layer.
 // Ring layout per layer: [max_seqs][H][2][W][dh].
 template <typename T>
-__global__ void k_dec_qkv_post(int n, int H, int dh, int W, const int *__restrict__ ready,
-                               const int *__restrict__ pos, const float *__restrict__ qkv,
-                               const float2 *__restrict__ rope, float *__restrict__ q_out,
-                               T *__restrict__ ring_l) {
+__global__ void k_dec_qkv_post(const int *__restrict__ n_dev, int H, int dh, int W,
+                               const int *__restrict__ ready, const int *__restrict__ pos,
+                               const float *__restrict__ qkv, const float2 *__restrict__ rope,
+                               float *__restrict__ q_out, T *__restrict__ ring_l) {
   int half = dh / 2, d = H * dh;
   long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long)n * H * half) return;
+  if (idx >= (long)(*n_dev) * H * half) return;
   int j = (int)(idx % half);
   int h = (int)((idx / half) % H);
   int i = (int)(idx / ((long)half * H));
@@ -180,100 +183,13 @@ __device__ __forceinline__ void warp_attend(const float *qr, const T *__restrict
   for (int o = LPK; o < 32; o <<= 1) st.merge_xor(o);
 }
 
-// Decoder SWA: slot i, head h attends positions max(0, t-W+1) .. t of its ring.
-template <typename T, int DH>
-__global__ void k_swa_decode(int n, int H, int W, const int *__restrict__ ready,
-                             const int *__restrict__ pos, const float *__restrict__ q,
-                             const T *__restrict__ ring_l, T *__restrict__ out, float scale) {
-  constexpr int VEC = V16<T>::N, LPK = DH / VEC;
-  int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (gw >= n * H) return;
-  int i = gw / H, h = gw % H, d = H * DH;
-  int seq = ready[i], t = pos[i];
-  int sub = lane % LPK;
-  float qr[VEC];
-#pragma unroll
-  for (int v = 0; v < VEC; v++) qr[v] = q[(size_t)i * d + h * DH + sub * VEC + v] * scale;
-  const T *K = ring_l + (((size_t)seq * H + h) * 2) * W * DH;
-  const T *V = K + (size_t)W * DH;
-  SoftAcc<VEC> st;
-  int p_lo = t - W + 1 > 0 ? t - W + 1 : 0;
-  warp_attend<T, DH, true>(qr, K, V, p_lo, t, W, lane, st);
-  if (lane < LPK) {
-    float inv = 1.f / st.l;
-#pragma unroll
-    for (int v = 0; v < VEC; v++)
-      out[(size_t)i * d + h * DH + sub * VEC + v] = from_f<T>(st.acc[v] * inv);
-  }
-}
-
-// Cross-attention, split over chunks of CH memory positions: item (i, h, c)
-// covers positions [c*CH, min(t+1, (c+1)*CH)) and writes its partial
-// (acc[DH], m, l). Memory layout per group: [max_seqs][H][2][max_len][dh].
-// The grid covers `xchunks` splits per (i, h); the partial buffer is laid out
-// with `max_chunks` per (i, h).
-template <typename T, int DH>
-__global__ void k_xattn_partial(int n, int H, int CH, int xchunks, int max_chunks, int max_len,
-                                const int *__restrict__ ready, const int *__restrict__ pos,
-                                const float *__restrict__ q, const T *__restrict__ mem_g,
-                                float *__restrict__ part, float scale) {
-  constexpr int VEC = V16<T>::N, LPK = DH / VEC;
-  int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (gw >= n * H * xchunks) return;
-  int c = gw % xchunks, ih = gw / xchunks;
-  int i = ih / H, h = ih % H, d = H * DH;
-  int t = pos[i];
-  int p_lo = c * CH;
-  if (p_lo > t) return;
-  int p_hi = min(t, p_lo + CH - 1);
-  int seq = ready[i];
-  int sub = lane % LPK;
-  float qr[VEC];
-#pragma unroll
-  for (int v = 0; v < VEC; v++) qr[v] = q[(size_t)i * d + h * DH + sub * VEC + v] * scale;
-  const T *K = mem_g + (((size_t)seq * H + h) * 2) * max_len * DH;
-  const T *V = K + (size_t)max_len * DH;
-  SoftAcc<VEC> st;
-  warp_attend<T, DH, false>(qr, K, V, p_lo, p_hi, 0, lane, st);
-  float *pp = part + ((size_t)ih * max_chunks + c) * (DH + 2);
-  if (lane < LPK) {
-#pragma unroll
-    for (int v = 0; v < VEC; v++) pp[sub * VEC + v] = st.acc[v];
-  }
-  if (lane == 0) {
-    pp[DH] = st.m;
-    pp[DH + 1] = st.l;
-  }
-}
-
-// Merge the chunk partials of (i, h) in chunk order.
-template <typename T, int DH>
-__global__ void k_xattn_combine(int n, int H, int CH, int max_chunks, const int *__restrict__ pos,
-                                const float *__restrict__ part, T *__restrict__ out) {
-  int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (gw >= n * H) return;
-  int i = gw / H, h = gw % H, d = H * DH;
-  int nc = pos[i] / CH + 1;
-  const float *pp = part + (size_t)gw * max_chunks * (DH + 2);
-  float mx = -INFINITY;
-  for (int c = 0; c < nc; c++) mx = fmaxf(mx, pp[c * (DH + 2) + DH]);
-  float L = 0.f;
-  for (int c = 0; c < nc; c++) L += expf(pp[c * (DH + 2) + DH] - mx) * pp[c * (DH + 2) + DH + 1];
-  float inv = 1.f / L;
-  for (int j = lane; j < DH; j += 32) {
-    float o = 0.f;
-    for (int c = 0; c < nc; c++) o += expf(pp[c * (DH + 2) + DH] - mx) * pp[c * (DH + 2) + j];
-    out[(size_t)i * d + h * DH + j] = from_f<T>(o * inv);
-  }
-}
-
 // Step end: s_t = RMSNorm_f(h) and t_dec += 1 ([RLT-96] "Architecture": s_t is
 // the final decoder output vector). One warp per slot.
-__global__ void k_step_final(int n, int d, const int *__restrict__ ready, int *__restrict__ t_dec,
-                             const float *__restrict__ h, const float *__restrict__ gamma,
-                             float eps, float *__restrict__ s) {
+__global__ void k_step_final(const int *__restrict__ n_dev, int d, const int *__restrict__ ready,
+                             int *__restrict__ t_dec, const float *__restrict__ h,
+                             const float *__restrict__ gamma, float eps, float *__restrict__ s) {
   int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (i >= n) return;
+  if (i >= *n_dev) return;
   int seq = ready[i];
   const float *hr = h + (size_t)i * d;
   float ss = 0.f;

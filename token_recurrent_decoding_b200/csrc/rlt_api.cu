@@ -8,13 +8,16 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "../../include/rlt.h"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "kernels.cuh"
+#include "attn.cuh"
 
 using namespace rlt;
 
@@ -28,7 +31,7 @@ struct Layout {
   // persistent state
   size_t s, t_dec, t_enc, e, mem, ring, rope, err;
   // decoder step work buffers (max_seqs rows)
-  size_t ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part;
+  size_t nready, ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part, counters;
   // encoder work buffers (ptok rows)
   size_t tok, tok_slot, tok_pos, tok_start, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
   size_t staging, staging_bytes;
@@ -86,6 +89,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->ring = take(LD * S * H * 2 * W * dh * es);
   L->rope = take(T * (dh / 2) * 8);
   L->err = take(16);
+  L->nready = take(4);
   L->ready = take(S * 4);
   L->pos = take(S * 4);
   L->h = take(S * d * 4);
@@ -99,6 +103,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->fa = take(c->ffn_kind == RLT_SWIGLU ? S * F * 4 : 0);
   L->f = take(S * F * es);
   L->part = take(S * H * L->max_chunks * (dh + 2) * 4);
+  L->counters = take(S * H * 4);
   size_t P = (size_t)ptok;
   L->tok = take(P * 4);
   L->tok_slot = take(P * 4);
@@ -125,6 +130,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
 
 struct StepInfo {
   int n;            // ready slots
+  int n_grid;       // grid row bound (n rounded up; kernels read n on the device)
   int xchunks;      // cross-attention splits to launch (covers max t)
   double sum_keys;  // sum over slots of (t + 1): memory rows attended
   double sum_win;   // sum over slots of min(t + 1, W): ring rows attended
@@ -145,12 +151,19 @@ struct rlt_model {
   std::vector<int> t_dec, t_enc;
   cudaStream_t last_stream = nullptr;
   template <typename X> X *at(size_t off) const { return reinterpret_cast<X *>(arena + off); }
-  // dtype/head-dim specialised launch sequences
   // measurement hook (rlt_profile / rlt_get_stats)
   bool profiling = false;
   std::vector<cudaEvent_t> ev_pool;
   std::vector<ProfSpan> pending;
   rlt_stats stats{};
+  int prof_stride = 0;       // profile every prof_stride-th decoder step (0: off)
+  int64_t step_counter = 0;  // decoder steps enqueued
+  // replayable decoder steps, keyed by (grid row bound, cross-attention splits)
+  struct Graph {
+    cudaGraphExec_t exec;
+    int64_t launches;
+  };
+  std::map<std::pair<int, int>, Graph> graphs;
   cudaError_t (*step)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
   cudaError_t (*prefill)(rlt_model *, int, cudaStream_t) = nullptr;
   cudaError_t (*get_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
@@ -212,7 +225,7 @@ cudaError_t gemm_k(rlt_model *M, int kind, int m, int n, int k, const T *A, int 
   double es = sizeof(T);
   Span sp(M, st, kind, (double)n * k * es + (double)m * k * es + (double)m * n * 4.0,
           2.0 * m * n * k);
-  return gemm(m, n, k, A, lda, B, ldb, epi, st);
+  return gemm(m, nullptr, n, k, A, lda, B, ldb, epi, st);
 }
 
 template <typename T> struct W_ {
@@ -238,18 +251,43 @@ template <typename T> struct W_ {
 // list ([RLT-96] "Architecture": gated merge, then per block SWA,
 // cross-attention, FFN; s_t is the final output). `xchunks` bounds the
 // cross-attention splits launched (covers the largest t in the batch).
+// Decode-attention launch: window > 0 is the SWA over the layer's ring, 0 the
+// cross-attention over the memory group.
+template <typename T, int DH>
+cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunks,
+                        const T *base, long seq_stride, long head_stride, long v_offset,
+                        T *out, cudaStream_t st) {
+  constexpr int STAGES = 4, NW = 4;
+  constexpr int smem = attn_smem_bytes<T, DH, STAGES, NW>();
+  auto kern = k_attn_decode<T, DH, STAGES, NW>;
+  static bool attr = false;
+  if (!attr) {
+    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr = true;
+  }
+  const Layout &L = M->L;
+  const rlt_config &c = M->cfg;
+  kern<<<si.n_grid * c.n_heads * xchunks, NW * 32, smem, st>>>(
+      M->at<int>(L.nready), c.n_heads, window, XCH, xchunks, L.max_chunks, M->at<int>(L.ready),
+      M->at<int>(L.pos), M->at<float>(L.q), base, seq_stride, head_stride, v_offset,
+      M->at<float>(L.part), M->at<int>(L.counters), out, 1.0f / sqrtf((float)DH),
+      M->at<int>(L.err));
+  return cudaGetLastError();
+}
+
 template <typename T, int DH>
 cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   const rlt_config &c = M->cfg;
   const Layout &L = M->L;
-  const int n = si.n, xchunks = si.xchunks;
+  const int n = si.n_grid;  // grid bound; the kernels read the real n on the device
+  const int *nd = M->at<int>(L.nready);
   const int d = c.d, H = c.n_heads, F = c.ffn_dim, W = c.window;
-  const float scale = 1.0f / sqrtf((float)DH), eps = c.rms_eps;
+  const float eps = c.rms_eps;
   const double es = sizeof(T);
   int *ready = M->at<int>(L.ready), *pos = M->at<int>(L.pos), *t_dec = M->at<int>(L.t_dec);
   float *h = M->at<float>(L.h), *e32 = M->at<float>(L.e32), *s32 = M->at<float>(L.s32);
   float *qkv = M->at<float>(L.qkv), *q = M->at<float>(L.q), *fa = M->at<float>(L.fa);
-  float *part = M->at<float>(L.part), *s = M->at<float>(L.s);
+  float *s = M->at<float>(L.s);
   T *xin = M->at<T>(L.xin), *a = M->at<T>(L.a), *u = M->at<T>(L.u), *f = M->at<T>(L.f);
   T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem);
   const float2 *rope = M->at<float2>(L.rope);
@@ -257,75 +295,75 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   const size_t ring_layer = (size_t)c.max_seqs * H * 2 * W * DH;
   const size_t mem_group = (size_t)c.max_seqs * H * 2 * c.max_len * DH;
   const int rows_blocks = blocks_for((long)n * 32, 256);
-  const double row_bytes = (double)n * d * (4 + es);  // one fp32 read + one T write per row
+  const double nr = si.n;  // real rows, for the algorithmic byte counts
+  const double row_bytes = nr * d * (4 + es);
+  auto G = [&](int kind, int m, int nn, int k, const T *A, int lda, const T *B, int ldb,
+               auto epi) {
+    Span sp(M, st, kind, (double)nn * k * es + nr * k * es + nr * nn * 4.0, 2.0 * nr * nn * k);
+    return gemm(m, nd, nn, k, A, lda, B, ldb, epi, st);
+  };
 
   {
-    Span sp(M, st, RLT_K_OTHER, (double)n * d * (es + 4) + row_bytes);
-    k_step_gather<T><<<n, 256, 0, st>>>(n, d, c.max_len, ready, t_dec, pos, M->at<T>(L.e), s,
+    Span sp(M, st, RLT_K_OTHER, nr * d * (es + 4) + row_bytes);
+    k_step_gather<T><<<n, 256, 0, st>>>(nd, d, c.max_len, ready, t_dec, pos, M->at<T>(L.e), s,
                                         xin, e32, s32, h, a0);
   }
   RLT_TRY(cudaGetLastError());
   if (!a0)
-    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, 2 * d, xin, 2 * d, (const T *)M->w.gate_w, 2 * d,
-                   EpiGate{e32, s32, (const float *)M->w.gate_b, c.alpha, h, d}, st));
+    RLT_TRY(G(RLT_K_GEMM, n, d, 2 * d, xin, 2 * d, (const T *)M->w.gate_w, 2 * d,
+              EpiGate{e32, s32, (const float *)M->w.gate_b, c.alpha, h, d}));
   for (int l = 0; l < c.n_dec_layers; l++) {
     T *ring_l = ring + (size_t)l * ring_layer;
     const T *mem_g = mem + (size_t)(c.mem_groups == 1 ? 0 : l) * mem_group;
     // sliding-window self-attention sublayer
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, d, h, (const float *)M->w.dec_ln1[l], eps, u);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln1[l], eps,
+                                                u);
     }
-    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, 3 * d, d, u, d, W_<T>::qkv(M, l), d,
-                   EpiStoreF32{qkv, 3 * d}, st));
+    RLT_TRY(G(RLT_K_GEMM, n, 3 * d, d, u, d, W_<T>::qkv(M, l), d, EpiStoreF32{qkv, 3 * d}));
     {
-      Span sp(M, st, RLT_K_OTHER, (double)n * 3 * d * 4 + (double)n * d * (4 + 2 * es));
+      Span sp(M, st, RLT_K_OTHER, nr * 3 * d * 4 + nr * d * (4 + 2 * es));
       k_dec_qkv_post<T><<<blocks_for((long)n * H * (DH / 2), 256), 256, 0, st>>>(
-          n, H, DH, W, ready, pos, qkv, rope, q, ring_l);
+          nd, H, DH, W, ready, pos, qkv, rope, q, ring_l);
     }
     {
-      Span sp(M, st, RLT_K_SWA, si.sum_win * 2.0 * d * es + (double)n * d * (4 + es),
+      Span sp(M, st, RLT_K_SWA, si.sum_win * 2.0 * d * es + nr * d * (4 + es),
               4.0 * d * si.sum_win);
-      k_swa_decode<T, DH><<<blocks_for((long)n * H * 32, 256), 256, 0, st>>>(n, H, W, ready, pos,
-                                                                             q, ring_l, a, scale);
+      RLT_TRY((launch_attn<T, DH>(M, si, W, 1, ring_l, (long)H * 2 * W * DH, 2L * W * DH,
+                                  (long)W * DH, a, st)));
     }
-    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, d, a, d, W_<T>::o(M, l), d, EpiResid{h, d}, st));
+    RLT_TRY(G(RLT_K_GEMM, n, d, d, a, d, W_<T>::o(M, l), d, EpiResid{h, d}));
     // cross-attention sublayer over M<=t
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, d, h, (const float *)M->w.dec_ln2[l], eps, u);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln2[l], eps,
+                                                u);
     }
-    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, d, u, d, (const T *)M->w.dec_wqx[l], d,
-                   EpiStoreF32{q, d}, st));
+    RLT_TRY(G(RLT_K_GEMM, n, d, d, u, d, (const T *)M->w.dec_wqx[l], d, EpiStoreF32{q, d}));
     {
       Span sp(M, st, RLT_K_XATTN, si.sum_keys * 2.0 * d * es, 4.0 * d * si.sum_keys);
-      k_xattn_partial<T, DH><<<blocks_for((long)n * H * xchunks * 32, 256), 256, 0, st>>>(
-          n, H, XCH, xchunks, L.max_chunks, c.max_len, ready, pos, q, mem_g, part, scale);
+      RLT_TRY((launch_attn<T, DH>(M, si, 0, si.xchunks, mem_g, (long)H * 2 * c.max_len * DH,
+                                  2L * c.max_len * DH, (long)c.max_len * DH, a, st)));
     }
-    {
-      Span sp(M, st, RLT_K_OTHER, (double)n * H * xchunks * (DH + 2) * 4 + (double)n * d * es);
-      k_xattn_combine<T, DH><<<blocks_for((long)n * H * 32, 256), 256, 0, st>>>(
-          n, H, XCH, L.max_chunks, pos, part, a);
-    }
-    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, d, a, d, (const T *)M->w.dec_wox[l], d, EpiResid{h, d},
-                   st));
+    RLT_TRY(G(RLT_K_GEMM, n, d, d, a, d, (const T *)M->w.dec_wox[l], d, EpiResid{h, d}));
     // FFN sublayer
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, d, h, (const float *)M->w.dec_ln3[l], eps, u);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln3[l], eps,
+                                                u);
     }
     if (c.ffn_kind == RLT_GELU) {
-      RLT_TRY(gemm_k(M, RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiGelu<T>{f, F}, st));
+      RLT_TRY(G(RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiGelu<T>{f, F}));
     } else {
-      RLT_TRY(gemm_k(M, RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiStoreF32{fa, F}, st));
-      RLT_TRY(gemm_k(M, RLT_K_GEMM, n, F, d, u, d, W_<T>::wb(M, l), d, EpiSwiglu<T>{fa, f, F},
-                     st));
+      RLT_TRY(G(RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiStoreF32{fa, F}));
+      RLT_TRY(G(RLT_K_GEMM, n, F, d, u, d, W_<T>::wb(M, l), d, EpiSwiglu<T>{fa, f, F}));
     }
-    RLT_TRY(gemm_k(M, RLT_K_GEMM, n, d, F, f, F, W_<T>::w2(M, l), F, EpiResid{h, d}, st));
+    RLT_TRY(G(RLT_K_GEMM, n, d, F, f, F, W_<T>::w2(M, l), F, EpiResid{h, d}));
   }
   {
-    Span sp(M, st, RLT_K_OTHER, (double)n * d * 8);
-    k_step_final<<<rows_blocks, 256, 0, st>>>(n, d, ready, t_dec, h,
+    Span sp(M, st, RLT_K_OTHER, nr * d * 8);
+    k_step_final<<<rows_blocks, 256, 0, st>>>(nd, d, ready, t_dec, h,
                                               (const float *)M->w.dec_lnf, eps, s);
   }
   return cudaGetLastError();
@@ -359,7 +397,8 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, cudaStream_t st) {
   for (int l = 0; l < c.n_enc_layers; l++) {
     {
       Span sp(M, st, K);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, d, eh, (const float *)w.enc_ln1[l], eps, eu);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh, (const float *)w.enc_ln1[l],
+                                                eps, eu);
     }
     RLT_TRY(gemm_k(M, K, ntok, 3 * d, d, eu, d, (const T *)w.enc_wqkv[l], d,
                    EpiStoreF32{eqkv, 3 * d}, st));
@@ -376,7 +415,8 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, cudaStream_t st) {
     RLT_TRY(gemm_k(M, K, ntok, d, d, ea, d, (const T *)w.enc_wo[l], d, EpiResid{eh, d}, st));
     {
       Span sp(M, st, K);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, d, eh, (const float *)w.enc_ln2[l], eps, eu);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh, (const float *)w.enc_ln2[l],
+                                                eps, eu);
     }
     if (c.ffn_kind == RLT_GELU) {
       RLT_TRY(gemm_k(M, K, ntok, F, d, eu, d, (const T *)w.enc_w1[l], d, EpiGelu<T>{ef, F}, st));
@@ -482,7 +522,7 @@ int check_batch(const rlt_model *M, const int32_t *ids, int n, int need) {
 
 // Batch description for one step of the listed slots at their current t.
 StepInfo step_info(const rlt_model *M, const int32_t *ids, int n) {
-  StepInfo si{n, 1, 0.0, 0.0};
+  StepInfo si{n, (n + 63) / 64 * 64, 1, 0.0, 0.0};
   int tmax = 0;
   for (int i = 0; i < n; i++) {
     int t = M->t_dec[ids[i]];
@@ -491,7 +531,51 @@ StepInfo step_info(const rlt_model *M, const int32_t *ids, int n) {
     si.sum_win += std::min(t + 1, M->cfg.window);
   }
   si.xchunks = std::min(M->L.max_chunks, tmax / XCH + 1);
+  si.n_grid = std::min(si.n_grid, M->cfg.max_seqs);
   return si;
+}
+
+// One decoder step of the slots already listed in the arena's ready list:
+// the batch size goes to the device, then the step runs directly (first use,
+// legacy stream, or a profiled sample) or replays its captured graph.
+cudaError_t enqueue_step(rlt_model *M, const StepInfo &si, cudaStream_t st) {
+  int nval = si.n;
+  RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.nready), &nval, sizeof(int), cudaMemcpyHostToDevice,
+                          st));  // pageable source: staged before return
+  const bool prof = M->profiling && M->prof_stride > 0 && (M->step_counter % M->prof_stride == 0);
+  M->step_counter++;
+  auto key = std::make_pair(si.n_grid, si.xchunks);
+  auto it = M->graphs.find(key);
+  if (st == nullptr || prof || it == M->graphs.end()) {
+    const bool saved = M->profiling;
+    M->profiling = prof;
+    cudaError_t e = M->step(M, si, st);
+    M->profiling = saved;
+    RLT_TRY(e);
+    if (st == nullptr || it != M->graphs.end()) return cudaSuccess;
+    // capture this (row bound, splits) once for replay
+    int64_t l0 = M->stats.launches;
+    cudaGraph_t g = nullptr;
+    RLT_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+    M->profiling = false;
+    cudaError_t ec = M->step(M, si, st);
+    M->profiling = saved;
+    cudaError_t ee = cudaStreamEndCapture(st, &g);
+    if (ec != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      return ec;
+    }
+    RLT_TRY(ee);
+    cudaGraphExec_t ge = nullptr;
+    cudaError_t ei = cudaGraphInstantiate(&ge, g, 0);
+    cudaGraphDestroy(g);
+    RLT_TRY(ei);
+    M->graphs[key] = {ge, M->stats.launches - l0};
+    M->stats.launches = l0;  // captured, not launched
+    return cudaSuccess;
+  }
+  M->stats.launches += it->second.launches;
+  return cudaGraphLaunch(it->second.exec, st);
 }
 
 void advance(rlt_model *M, const int32_t *ids, int n) {
@@ -603,6 +687,7 @@ RLT_API void rlt_destroy(rlt_model *M) {
     cudaEventDestroy(p.b);
   }
   for (auto e : M->ev_pool) cudaEventDestroy(e);
+  for (auto &g : M->graphs) cudaGraphExecDestroy(g.second.exec);
   delete M;
 }
 
@@ -701,7 +786,7 @@ RLT_API int rlt_decoder_step(rlt_model *M, const int32_t *ids, int n, rlt_stream
   std::vector<int32_t> idv(ids, ids + n);  // pageable copy: read before return
   cudaError_t e = cudaMemcpyAsync(M->at<int>(M->L.ready), idv.data(), 4 * n,
                                   cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = M->step(M, step_info(M, ids, n), st);
+  if (e == cudaSuccess) e = enqueue_step(M, step_info(M, ids, n), st);
   if (e != cudaSuccess) return RLT_ERR_CUDA;
   advance(M, ids, n);
   return RLT_OK;
@@ -718,7 +803,7 @@ RLT_API int rlt_run_sequence(rlt_model *M, const int32_t *ids, int n, int n_step
   cudaError_t e = cudaMemcpyAsync(M->at<int>(M->L.ready), idv.data(), 4 * n,
                                   cudaMemcpyHostToDevice, st);
   for (int k = 0; k < n_steps && e == cudaSuccess; k++) {
-    e = M->step(M, step_info(M, idv.data(), n), st);
+    e = enqueue_step(M, step_info(M, idv.data(), n), st);
     advance(M, idv.data(), n);
   }
   return cuda_status(e);
@@ -780,7 +865,7 @@ RLT_API int rlt_run_ragged(rlt_model *M, const int32_t *ids, const int32_t *step
                                   cudaMemcpyHostToDevice, st);
   for (int k = 0; k < nt && e == cudaSuccess; k++) {
     int c = sizes[k];
-    e = M->step(M, step_info(M, sorted.data(), c), st);
+    e = enqueue_step(M, step_info(M, sorted.data(), c), st);
     advance(M, sorted.data(), c);
   }
   return cuda_status(e);
@@ -861,7 +946,9 @@ RLT_API int rlt_profile(rlt_model *M, int enable) {
   int64_t launches = M->stats.launches;
   M->stats = rlt_stats{};
   M->stats.launches = launches;
-  M->profiling = enable != 0;
+  M->profiling = enable > 0;
+  M->prof_stride = enable > 0 ? enable : 0;
+  M->step_counter = 0;
   return RLT_OK;
 }
 

@@ -311,8 +311,9 @@ class Model:
                                                  self._st(stream)), "rlt_get_encoder_output")
         return e, mem
 
-    def profile(self, enable: bool):
-        _check(_lib().rlt_profile(self._h, int(bool(enable))), "rlt_profile")
+    def profile(self, stride: int):
+        """stride k > 0: profile every k-th decoder step (and every prefill); 0: off."""
+        _check(_lib().rlt_profile(self._h, int(stride)), "rlt_profile")
 
     def get_stats(self) -> dict:
         st = rlt_stats()
