@@ -24,7 +24,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from token_recurrent_decoding_b200 import configs, inputs, roofline  # noqa: E402
+from token_recurrent_decoding_b200 import configs, inputs, ranks, roofline  # noqa: E402
 
 METRIC = "decoder sequence-steps/s (bf16, B200) and % of step roofline (HBM/tensor)"
 DEFAULT_WORKLOAD = "m140_bf16"
@@ -65,12 +65,7 @@ def dist_setup(n_gpus):
 
 
 def max_over_ranks(x: float, dist) -> float:
-    if dist is None:
-        return x
-    import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return ranks.max_over_ranks(x, dist, device="cuda")
 
 
 def barrier(dist):
@@ -136,7 +131,7 @@ class ClockSampler:
 class Runner:
     """Owns the device model and the seeded inputs of one workload."""
 
-    def __init__(self, wl, device="cuda"):
+    def __init__(self, wl, device="cuda", rank=0, world=1):
         import torch
         from token_recurrent_decoding_b200.rlt import Model
         self.torch = torch
@@ -144,7 +139,10 @@ class Runner:
         cfg = wl.model
         self.stream = torch.cuda.Stream()
         w = inputs.make_weights(cfg)
-        self.tok = inputs.make_tokens(cfg.vocab, wl.lengths)
+        # weak scaling: the job holds world x B sequences; this rank owns a
+        # contiguous shard of them (same lengths, its own tokens)
+        lo, hi = ranks.shard_range(world * wl.batch, rank, world)
+        self.tok = inputs.make_tokens(cfg.vocab, list(wl.lengths) * world)[lo:hi]
         lengths = np.asarray(wl.lengths, np.int32)
         self.lengths = lengths
         flat = np.concatenate([self.tok[i, :L] for i, L in enumerate(lengths)]).astype(np.int32)
@@ -187,7 +185,7 @@ class Runner:
 
 def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
     import torch
-    r = Runner(wl)
+    r = Runner(wl, rank=rank, world=world)
     st = r.stream
     torch.cuda.synchronize()
     for _ in range(args.warmup):

@@ -1,0 +1,215 @@
+// tcgen05 / TMEM GEMM for the large projections of the encoder prefill:
+//   C[m][n] = sum_k A[m][k] * B[n][k],  A = activations [M][K], B = weights
+//   [N][K], both bf16 K-major, fp32 accumulation in tensor memory.
+//
+// One CTA computes a 128 x BN tile. Warp 0 (one lane) streams A and B tiles
+// of 64 K-elements with TMA (cp.async.bulk.tensor, 128-byte swizzle) into a
+// STAGES-deep shared-memory ring; warp 1 owns the TMEM accumulator and one
+// lane issues tcgen05.mma (kind::f16, M = 128, N = BN, K = 16 per
+// instruction), releasing each stage with tcgen05.commit on its "empty"
+// barrier. After the last K block a commit on the accumulator barrier hands
+// the tile to all four warps, which read it back with tcgen05.ld (warp w owns
+// TMEM lanes 32w..32w+31 = tile rows) and apply the epilogue functor two
+// columns at a time. Every mbarrier wait is bounded in device time.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace rlt {
+
+// ---------------------------------------------------------------- PTX pieces
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major tile written by TMA with the
+// 128-byte swizzle (8-row groups of 1024 bytes).
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void *p) {
+  const uint64_t addr = smem_u32(p);
+  uint64_t d = 0;
+  d |= (addr >> 4) & 0x3FFFull;           // start address
+  d |= (uint64_t)1 << 16;                 // leading byte offset (unused for SW128 K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;                 // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                 // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A/B, fp32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4)                        // D format f32
+         | (1u << 7)                      // A format bf16
+         | (1u << 10)                     // B format bf16
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; i++) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+
+constexpr int TC_BM = 128, TC_BK = 64;
+constexpr uint64_t WAIT_LIMIT_NS_TC = 2000000000ull;  // bounded waits: 2 s of device time
+
+template <int BN, int STAGES> struct TcSmem {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  // tiles (1024-byte aligned) + barriers + TMEM address + alignment slack
+  static constexpr int BYTES = STAGES * STAGE + (2 * STAGES + 1) * 8 + 16 + 1024;
+};
+
+template <int BN, int STAGES, class Epi>
+__global__ void __launch_bounds__(128, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              int M, int N, int K, Epi epi, int *err) {
+  static_assert(BN == 64 || BN == 128 || BN == 256, "TMEM columns are a power of two");
+  using SM = TcSmem<BN, STAGES>;
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t *tsm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(tsm + STAGES * SM::STAGE);
+  uint64_t *empty = full + STAGES;
+  uint64_t *accum = empty + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * TC_BM, n0 = blockIdx.x * BN;
+  const int KB = K / TC_BK;
+
+  if (threadIdx.x == 0) {
+    s_fail = 0;
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // producer: TMA into the ring
+    for (int kb = 0; kb < KB; kb++) {
+      const int s = kb % STAGES, u = kb / STAGES;
+      if (u > 0 && !mbar_wait_bounded(&empty[s], (u - 1) & 1, WAIT_LIMIT_NS_TC)) {
+        atomicExch(&s_fail, 1);
+        break;
+      }
+      uint8_t *a = tsm + s * SM::STAGE;
+      uint8_t *b = a + SM::A_BYTES;
+      mbar_expect_tx(&full[s], SM::STAGE);
+      tma_load_2d(a, &tmA, kb * TC_BK, m0, &full[s]);
+      tma_load_2d(b, &tmB, kb * TC_BK, n0, &full[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
+    for (int kb = 0; kb < KB; kb++) {
+      const int s = kb % STAGES, u = kb / STAGES;
+      if (!mbar_wait_bounded(&full[s], u & 1, WAIT_LIMIT_NS_TC)) {
+        atomicExch(&s_fail, 1);
+        break;
+      }
+      tc_fence_after();
+      const uint8_t *a = tsm + s * SM::STAGE;
+      const uint8_t *b = a + SM::A_BYTES;
+      const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(b);
+#pragma unroll
+      for (int k = 0; k < TC_BK / 16; k++) {
+        // advance 16 elements (32 bytes) along K inside the swizzle atom
+        umma_bf16(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc,
+                  (kb > 0 || k > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty[s]);
+    }
+    umma_commit(accum);
+  }
+  __syncwarp();
+  // epilogue: wait for the accumulator, read this warp's 32 rows
+  const bool acc_ok = mbar_wait_bounded(accum, 0, WAIT_LIMIT_NS_TC);
+  tc_fence_after();
+  if (!acc_ok || s_fail) {
+    if (threadIdx.x == 0) set_error(err, DEV_ERR_TIMEOUT);
+  } else {
+    const int row = m0 + warp * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float v[16];
+      tmem_ld16(lane_base + c0, v);
+      if (row < M) {
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          const int col = n0 + c0 + j;
+          if (col < N) epi(row, col, v[j], v[j + 1]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, BN);
+}
+
+}  // namespace rlt

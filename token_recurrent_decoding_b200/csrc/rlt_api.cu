@@ -10,6 +10,8 @@
 #include <cstring>
 #include <map>
 #include <new>
+#include <tuple>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -18,6 +20,8 @@
 #include "gemm.cuh"
 #include "kernels.cuh"
 #include "attn.cuh"
+#include "enc_attn.cuh"
+#include "gemm_tc.cuh"
 
 using namespace rlt;
 
@@ -33,7 +37,7 @@ struct Layout {
   // decoder step work buffers (max_seqs rows)
   size_t nready, ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part, counters;
   // encoder work buffers (ptok rows)
-  size_t tok, tok_slot, tok_pos, tok_start, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
+  size_t tok, tok_slot, tok_pos, tok_start, blk, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
   size_t staging, staging_bytes;
   size_t total;
   int max_chunks, ptok;
@@ -109,6 +113,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->tok_slot = take(P * 4);
   L->tok_pos = take(P * 4);
   L->tok_start = take(P * 4);
+  L->blk = take((P / 64 + S + 1) * 16);
   L->eh = take(P * d * 4);
   L->eu = take(P * d * es);
   L->eqkv = take(P * 3 * d * 4);
@@ -164,8 +169,10 @@ struct rlt_model {
     int64_t launches;
   };
   std::map<std::pair<int, int>, Graph> graphs;
+  // TMA descriptors of bf16 [rows][cols] matrices, keyed by (pointer, rows, cols, box rows)
+  std::map<std::tuple<const void *, uint64_t, uint64_t, uint32_t>, CUtensorMap> tmaps;
   cudaError_t (*step)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
-  cudaError_t (*prefill)(rlt_model *, int, cudaStream_t) = nullptr;
+  cudaError_t (*prefill)(rlt_model *, int, int, cudaStream_t) = nullptr;
   cudaError_t (*get_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
   cudaError_t (*set_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
   cudaError_t (*get_memory)(rlt_model *, int, int, cudaStream_t) = nullptr;
@@ -180,6 +187,71 @@ namespace {
   } while (0)
 
 inline int blocks_for(long threads, int bs) { return (int)((threads + bs - 1) / bs); }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// 2-D TMA map of a row-major bf16 [rows][cols] matrix, box = 64 columns
+// (128 bytes, the swizzle span) x box_rows rows, 128-byte swizzle, zero fill
+// outside the matrix.
+const CUtensorMap *tmap_bf16(rlt_model *M, const void *ptr, uint64_t rows, uint64_t cols,
+                             uint32_t box_rows) {
+  auto key = std::make_tuple(ptr, rows, cols, box_rows);
+  auto it = M->tmaps.find(key);
+  if (it != M->tmaps.end()) return &it->second;
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return nullptr;
+  CUtensorMap m;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return nullptr;
+  return &M->tmaps.emplace(key, m).first->second;
+}
+
+// tcgen05 GEMM of the encoder: A [a_rows][k] activations (only the first m
+// rows are used), B [n][k] weights.
+template <class Epi>
+cudaError_t gemm_tc(rlt_model *M, int m, int a_rows, int n, int k, const bf16 *A, const bf16 *B,
+                    Epi epi, cudaStream_t st) {
+  constexpr int BN = 128, STAGES = 3;
+  constexpr int smem = TcSmem<BN, STAGES>::BYTES;
+  if (m <= 0) return cudaSuccess;
+  const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
+  const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
+  if (!ma || !mb) return cudaErrorInvalidValue;
+  auto kern = k_gemm_tc<BN, STAGES, Epi>;
+  static bool attr = false;
+  if (!attr) {
+    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr = true;
+  }
+  dim3 grid((n + BN - 1) / BN, (m + TC_BM - 1) / TC_BM);
+  kern<<<grid, 128, smem, st>>>(*ma, *mb, m, n, k, epi, M->at<int>(M->L.err));
+  return cudaGetLastError();
+}
 
 cudaEvent_t take_event(rlt_model *M) {
   if (!M->ev_pool.empty()) {
@@ -219,6 +291,20 @@ struct Span {
 
 // GEMM launch wrapper: class RLT_K_GEMM (or the encoder class) with the
 // algorithmic traffic of one pass over the weights and activations.
+// Encoder GEMM: tcgen05 for bf16 models, exact fp32 SIMT for fp32 models.
+// A is an encoder work buffer of ptok rows and k columns (lda = k).
+template <typename T, class Epi>
+cudaError_t gemm_enc(rlt_model *M, int m, int n, int k, const T *A, const T *B, Epi epi,
+                     cudaStream_t st) {
+  double es = sizeof(T);
+  Span sp(M, st, RLT_K_ENC, (double)n * k * es + (double)m * k * es + (double)m * n * 4.0,
+          2.0 * m * n * k);
+  if constexpr (std::is_same<T, bf16>::value)
+    return gemm_tc(M, m, M->L.ptok, n, k, A, B, epi, st);
+  else
+    return gemm(m, nullptr, n, k, A, k, B, k, epi, st);
+}
+
 template <typename T, class Epi>
 cudaError_t gemm_k(rlt_model *M, int kind, int m, int n, int k, const T *A, int lda, const T *B,
                    int ldb, Epi epi, cudaStream_t st) {
@@ -372,8 +458,34 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
 // Encoder over one chunk of ntok tokens already staged in the arena (token
 // ids, slot, position, sequence start), then the memory projection
 // ([RLT-96] "Architecture"; [RLT-TC] "What is this technology").
+// Causal attention of the encoder chunk: tensor-core flash attention for bf16
+// models, the per-query SIMT kernel for fp32 models.
 template <typename T, int DH>
-cudaError_t prefill_impl(rlt_model *M, int ntok, cudaStream_t st) {
+cudaError_t enc_attention(rlt_model *M, int ntok, int nblk, const T *Qh, const T *Kh, const T *Vh,
+                          T *ea, cudaStream_t st) {
+  const Layout &L = M->L;
+  const int H = M->cfg.n_heads;
+  if constexpr (std::is_same<T, bf16>::value && DH >= 32) {
+    constexpr int smem = FaSmem<DH>::BYTES;
+    static bool attr = false;
+    if (!attr) {
+      RLT_TRY(cudaFuncSetAttribute(k_enc_flash<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   smem));
+      attr = true;
+    }
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
+    k_enc_flash<DH><<<dim3(nblk, H), 128, smem, st>>>(ntok, M->at<int>(L.blk), Qh, Kh, Vh, ea, H,
+                                                       scale_log2);
+  } else {
+    k_enc_attn_simt<T, DH><<<blocks_for((long)ntok * H * 32, 256), 256, 0, st>>>(
+        ntok, H, M->at<int>(L.tok_pos), M->at<int>(L.tok_start), Qh, Kh, Vh, ea,
+        1.0f / sqrtf((float)DH));
+  }
+  return cudaGetLastError();
+}
+
+template <typename T, int DH>
+cudaError_t prefill_impl(rlt_model *M, int ntok, int nblk, cudaStream_t st) {
   const rlt_config &c = M->cfg;
   const Layout &L = M->L;
   const rlt_weights &w = M->w;
@@ -400,8 +512,8 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, cudaStream_t st) {
       k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh, (const float *)w.enc_ln1[l],
                                                 eps, eu);
     }
-    RLT_TRY(gemm_k(M, K, ntok, 3 * d, d, eu, d, (const T *)w.enc_wqkv[l], d,
-                   EpiStoreF32{eqkv, 3 * d}, st));
+    RLT_TRY(gemm_enc(M, ntok, 3 * d, d, eu, (const T *)w.enc_wqkv[l], EpiStoreF32{eqkv, 3 * d},
+                     st));
     {
       Span sp(M, st, K);
       k_enc_qkv_post<T><<<blocks_for((long)ntok * H * (DH / 2), 256), 256, 0, st>>>(
@@ -409,24 +521,21 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, cudaStream_t st) {
     }
     {
       Span sp(M, st, K);
-      k_enc_attn_simt<T, DH><<<blocks_for((long)ntok * H * 32, 256), 256, 0, st>>>(
-          ntok, H, tpos, tstart, Qh, Kh, Vh, ea, scale);
+      RLT_TRY((enc_attention<T, DH>(M, ntok, nblk, Qh, Kh, Vh, ea, st)));
     }
-    RLT_TRY(gemm_k(M, K, ntok, d, d, ea, d, (const T *)w.enc_wo[l], d, EpiResid{eh, d}, st));
+    RLT_TRY(gemm_enc(M, ntok, d, d, ea, (const T *)w.enc_wo[l], EpiResid{eh, d}, st));
     {
       Span sp(M, st, K);
       k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh, (const float *)w.enc_ln2[l],
                                                 eps, eu);
     }
     if (c.ffn_kind == RLT_GELU) {
-      RLT_TRY(gemm_k(M, K, ntok, F, d, eu, d, (const T *)w.enc_w1[l], d, EpiGelu<T>{ef, F}, st));
+      RLT_TRY(gemm_enc(M, ntok, F, d, eu, (const T *)w.enc_w1[l], EpiGelu<T>{ef, F}, st));
     } else {
-      RLT_TRY(gemm_k(M, K, ntok, F, d, eu, d, (const T *)w.enc_w1[l], d, EpiStoreF32{efa, F},
-                     st));
-      RLT_TRY(gemm_k(M, K, ntok, F, d, eu, d, (const T *)w.enc_wb[l], d,
-                     EpiSwiglu<T>{efa, ef, F}, st));
+      RLT_TRY(gemm_enc(M, ntok, F, d, eu, (const T *)w.enc_w1[l], EpiStoreF32{efa, F}, st));
+      RLT_TRY(gemm_enc(M, ntok, F, d, eu, (const T *)w.enc_wb[l], EpiSwiglu<T>{efa, ef, F}, st));
     }
-    RLT_TRY(gemm_k(M, K, ntok, d, F, ef, F, (const T *)w.enc_w2[l], F, EpiResid{eh, d}, st));
+    RLT_TRY(gemm_enc(M, ntok, d, F, ef, (const T *)w.enc_w2[l], EpiResid{eh, d}, st));
   }
   {
     Span sp(M, st, K);
@@ -437,10 +546,10 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, cudaStream_t st) {
   const size_t mem_group = (size_t)c.max_seqs * H * 2 * c.max_len * DH;
   for (int g = 0; g < c.mem_groups; g++) {
     T *mg = M->at<T>(L.mem) + (size_t)g * mem_group;
-    RLT_TRY(gemm_k(M, K, ntok, d, d, etok, d, (const T *)w.mem_wk[g], d,
-                   EpiMem<T>{mg, tslot, tpos, H, DH, c.max_len, 0}, st));
-    RLT_TRY(gemm_k(M, K, ntok, d, d, etok, d, (const T *)w.mem_wv[g], d,
-                   EpiMem<T>{mg, tslot, tpos, H, DH, c.max_len, 1}, st));
+    RLT_TRY(gemm_enc(M, ntok, d, d, etok, (const T *)w.mem_wk[g],
+                     EpiMem<T>{mg, tslot, tpos, H, DH, c.max_len, 0}, st));
+    RLT_TRY(gemm_enc(M, ntok, d, d, etok, (const T *)w.mem_wv[g],
+                     EpiMem<T>{mg, tslot, tpos, H, DH, c.max_len, 1}, st));
   }
   return cudaGetLastError();
 }
@@ -722,7 +831,7 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
   cudaStream_t st = (cudaStream_t)stream;
   M->last_stream = st;
   const Layout &L = M->L;
-  std::vector<int> slot, pos, start;
+  std::vector<int> slot, pos, start, blk;
   int i = 0;
   while (i < n) {
     // pack whole sequences into one chunk of at most ptok tokens
@@ -732,9 +841,16 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
     slot.assign(ntok, 0);
     pos.assign(ntok, 0);
     start.assign(ntok, 0);
+    blk.clear();
     long m = 0;
     for (int k = i; k < j; k++) {
       if (lengths[k] == 0) continue;
+      for (int qb = 0; qb * 64 < lengths[k]; qb++) {
+        blk.push_back((int)m);
+        blk.push_back(lengths[k]);
+        blk.push_back(qb);
+        blk.push_back(0);
+      }
       cudaError_t e = cudaMemcpyAsync(M->at<int>(L.tok) + m, tokens + offsets[k],
                                       sizeof(int32_t) * lengths[k], cudaMemcpyDefault, st);
       if (e != cudaSuccess) return RLT_ERR_CUDA;
@@ -752,7 +868,10 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
       if (e == cudaSuccess)
         e = cudaMemcpyAsync(M->at<int>(L.tok_start), start.data(), 4 * ntok,
                             cudaMemcpyHostToDevice, st);
-      if (e == cudaSuccess) e = M->prefill(M, (int)ntok, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(M->at<int>(L.blk), blk.data(), 4 * blk.size(), cudaMemcpyHostToDevice,
+                            st);
+      if (e == cudaSuccess) e = M->prefill(M, (int)ntok, (int)(blk.size() / 4), st);
       if (e != cudaSuccess) return RLT_ERR_CUDA;
       // the host vectors are reused next chunk: pageable copies are staged
       // at enqueue time, so reuse is safe
