@@ -93,7 +93,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->ring = take(LD * S * H * 2 * W * dh * es);
   L->rope = take(T * (dh / 2) * 8);
   L->err = take(16);
-  L->nready = take(4);
+  L->nready = take(2 * 4);
   L->ready = take(S * 4);
   L->pos = take(S * 4);
   L->h = take(S * d * 4);
@@ -133,9 +133,16 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
 
 }  // namespace
 
+// One chain of a decoder step: the ready-list rows [row0, row0 + n) run as
+// one sequence of kernels on one stream. A step is one chain, or two chains
+// over the two halves of the batch on two streams (sequences are independent,
+// so the halves overlap: one half's GEMMs run while the other's attention
+// streams K/V).
 struct StepInfo {
-  int n;            // ready slots
+  int row0;         // first ready-list row of this chain
+  int n;            // rows of this chain
   int n_grid;       // grid row bound (n rounded up; kernels read n on the device)
+  int chain;        // which device batch-size slot (0 or 1) the kernels read
   int xchunks;      // cross-attention splits to launch (covers max t)
   double sum_keys;  // sum over slots of (t + 1): memory rows attended
   double sum_win;   // sum over slots of min(t + 1, W): ring rows attended
@@ -168,7 +175,9 @@ struct rlt_model {
     cudaGraphExec_t exec;
     int64_t launches;
   };
-  std::map<std::pair<int, int>, Graph> graphs;
+  std::map<std::tuple<int, int, int>, Graph> graphs;
+  cudaStream_t side = nullptr;  // second chain of a split step
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   // TMA descriptors of bf16 [rows][cols] matrices, keyed by (pointer, rows, cols, box rows)
   std::map<std::tuple<const void *, uint64_t, uint64_t, uint32_t>, CUtensorMap> tmaps;
   cudaError_t (*step)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
@@ -353,11 +362,12 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
   }
   const Layout &L = M->L;
   const rlt_config &c = M->cfg;
+  const size_t r0 = si.row0, H = c.n_heads;
   kern<<<si.n_grid * c.n_heads * xchunks, NW * 32, smem, st>>>(
-      M->at<int>(L.nready), c.n_heads, window, XCH, xchunks, L.max_chunks, M->at<int>(L.ready),
-      M->at<int>(L.pos), M->at<float>(L.q), base, seq_stride, head_stride, v_offset,
-      M->at<float>(L.part), M->at<int>(L.counters), out, 1.0f / sqrtf((float)DH),
-      M->at<int>(L.err));
+      M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks,
+      M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0, M->at<float>(L.q) + r0 * c.d, base,
+      seq_stride, head_stride, v_offset, M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
+      M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH), M->at<int>(L.err));
   return cudaGetLastError();
 }
 
@@ -366,15 +376,19 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   const rlt_config &c = M->cfg;
   const Layout &L = M->L;
   const int n = si.n_grid;  // grid bound; the kernels read the real n on the device
-  const int *nd = M->at<int>(L.nready);
+  const int *nd = M->at<int>(L.nready) + si.chain;
   const int d = c.d, H = c.n_heads, F = c.ffn_dim, W = c.window;
   const float eps = c.rms_eps;
   const double es = sizeof(T);
-  int *ready = M->at<int>(L.ready), *pos = M->at<int>(L.pos), *t_dec = M->at<int>(L.t_dec);
-  float *h = M->at<float>(L.h), *e32 = M->at<float>(L.e32), *s32 = M->at<float>(L.s32);
-  float *qkv = M->at<float>(L.qkv), *q = M->at<float>(L.q), *fa = M->at<float>(L.fa);
+  const size_t r0 = si.row0;  // this chain's rows of every per-row buffer
+  int *ready = M->at<int>(L.ready) + r0, *pos = M->at<int>(L.pos) + r0;
+  int *t_dec = M->at<int>(L.t_dec);
+  float *h = M->at<float>(L.h) + r0 * d, *e32 = M->at<float>(L.e32) + r0 * d;
+  float *s32 = M->at<float>(L.s32) + r0 * d, *qkv = M->at<float>(L.qkv) + r0 * 3 * d;
+  float *q = M->at<float>(L.q) + r0 * d, *fa = M->at<float>(L.fa) + r0 * F;
   float *s = M->at<float>(L.s);
-  T *xin = M->at<T>(L.xin), *a = M->at<T>(L.a), *u = M->at<T>(L.u), *f = M->at<T>(L.f);
+  T *xin = M->at<T>(L.xin) + r0 * 2 * d, *a = M->at<T>(L.a) + r0 * d, *u = M->at<T>(L.u) + r0 * d;
+  T *f = M->at<T>(L.f) + r0 * F;
   T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem);
   const float2 *rope = M->at<float2>(L.rope);
   const bool a0 = c.alpha == 0.0f;
@@ -631,7 +645,7 @@ int check_batch(const rlt_model *M, const int32_t *ids, int n, int need) {
 
 // Batch description for one step of the listed slots at their current t.
 StepInfo step_info(const rlt_model *M, const int32_t *ids, int n) {
-  StepInfo si{n, (n + 63) / 64 * 64, 1, 0.0, 0.0};
+  StepInfo si{0, n, (n + 63) / 64 * 64, 0, 1, 0.0, 0.0};
   int tmax = 0;
   for (int i = 0; i < n; i++) {
     int t = M->t_dec[ids[i]];
@@ -644,30 +658,66 @@ StepInfo step_info(const rlt_model *M, const int32_t *ids, int n) {
   return si;
 }
 
+// Batches of at least this many rows run as two half-batch chains.
+constexpr int SPLIT_MIN_ROWS = 128;
+
+// Split a whole-batch step into its chains (byte sums shared in proportion).
+int make_chains(const rlt_model *M, const StepInfo &all, StepInfo ch[2]) {
+  if (all.n < SPLIT_MIN_ROWS || !M->side) {
+    ch[0] = all;
+    return 1;
+  }
+  const int na = (all.n + 1) / 2, nb = all.n - na;
+  const double fa = (double)na / all.n;
+  ch[0] = {0, na, std::min((na + 63) / 64 * 64, M->cfg.max_seqs), 0, all.xchunks,
+           all.sum_keys * fa, all.sum_win * fa};
+  ch[1] = {na, nb, std::min((nb + 63) / 64 * 64, M->cfg.max_seqs - na), 1, all.xchunks,
+           all.sum_keys * (1 - fa), all.sum_win * (1 - fa)};
+  return 2;
+}
+
+// Launch the chains of one step on `st` (and the side stream).
+cudaError_t launch_chains(rlt_model *M, const StepInfo *ch, int nch, cudaStream_t st) {
+  if (nch == 1) return M->step(M, ch[0], st);
+  RLT_TRY(cudaEventRecord(M->ev_fork, st));
+  RLT_TRY(cudaStreamWaitEvent(M->side, M->ev_fork, 0));
+  RLT_TRY(M->step(M, ch[0], st));
+  RLT_TRY(M->step(M, ch[1], M->side));
+  RLT_TRY(cudaEventRecord(M->ev_join, M->side));
+  return cudaStreamWaitEvent(st, M->ev_join, 0);
+}
+
 // One decoder step of the slots already listed in the arena's ready list:
-// the batch size goes to the device, then the step runs directly (first use,
-// legacy stream, or a profiled sample) or replays its captured graph.
-cudaError_t enqueue_step(rlt_model *M, const StepInfo &si, cudaStream_t st) {
-  int nval = si.n;
-  RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.nready), &nval, sizeof(int), cudaMemcpyHostToDevice,
-                          st));  // pageable source: staged before return
+// the batch sizes go to the device, then the step runs directly (first use,
+// legacy stream, or a profiled sample, which runs as one unsplit chain so
+// each kernel is timed alone) or replays its captured graph.
+cudaError_t enqueue_step(rlt_model *M, const StepInfo &all, cudaStream_t st) {
+  StepInfo ch[2];
   const bool prof = M->profiling && M->prof_stride > 0 && (M->step_counter % M->prof_stride == 0);
   M->step_counter++;
-  auto key = std::make_pair(si.n_grid, si.xchunks);
+  int nch = 1;
+  if (st == nullptr || prof)
+    ch[0] = all;
+  else
+    nch = make_chains(M, all, ch);
+  int nval[2] = {ch[0].n, nch == 2 ? ch[1].n : 0};
+  RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.nready), nval, sizeof(nval), cudaMemcpyHostToDevice,
+                          st));  // pageable source: staged before return
+  auto key = std::make_tuple(ch[0].n_grid, nch == 2 ? ch[1].n_grid : 0, all.xchunks);
   auto it = M->graphs.find(key);
   if (st == nullptr || prof || it == M->graphs.end()) {
     const bool saved = M->profiling;
     M->profiling = prof;
-    cudaError_t e = M->step(M, si, st);
+    cudaError_t e = launch_chains(M, ch, nch, st);
     M->profiling = saved;
     RLT_TRY(e);
-    if (st == nullptr || it != M->graphs.end()) return cudaSuccess;
-    // capture this (row bound, splits) once for replay
+    if (st == nullptr || prof) return cudaSuccess;
+    // capture this shape once for replay
     int64_t l0 = M->stats.launches;
     cudaGraph_t g = nullptr;
     RLT_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
     M->profiling = false;
-    cudaError_t ec = M->step(M, si, st);
+    cudaError_t ec = launch_chains(M, ch, nch, st);
     M->profiling = saved;
     cudaError_t ee = cudaStreamEndCapture(st, &g);
     if (ec != cudaSuccess) {
@@ -779,9 +829,12 @@ RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *w, void *d_aren
       e = cudaGetLastError();
     }
   }
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&M->side, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&M->ev_fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&M->ev_join, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
-    delete M;
+    rlt_destroy(M);
     return RLT_ERR_CUDA;
   }
   *out = M;
@@ -797,6 +850,12 @@ RLT_API void rlt_destroy(rlt_model *M) {
   }
   for (auto e : M->ev_pool) cudaEventDestroy(e);
   for (auto &g : M->graphs) cudaGraphExecDestroy(g.second.exec);
+  if (M->side) {
+    cudaStreamSynchronize(M->side);
+    cudaStreamDestroy(M->side);
+  }
+  if (M->ev_fork) cudaEventDestroy(M->ev_fork);
+  if (M->ev_join) cudaEventDestroy(M->ev_join);
   delete M;
 }
 
