@@ -206,6 +206,31 @@ RLT_API int rlt_get_encoder_output(rlt_model *model, int seq, void *e_out,
                                    void *mem_out, int64_t *t_enc_out,
                                    rlt_stream stream);
 
+/* Bytes of device workspace rlt_attend needs (0 if the shape is invalid). */
+RLT_API size_t rlt_attend_workspace_bytes(int n, int n_heads, int head_dim, int cap);
+
+/* The decoder's cross-attention kernel as a standalone operation: for every
+ * row i < n and head h, out[i][h] = softmax(q[i][h] . K_j / sqrt(dh)) V_j
+ * over the first h_lengths[i] rows j of that (row, head)'s key and value
+ * blocks -- one query against a prefix-restricted memory M<=t ([RLT-96]
+ * "Architecture": cross-attention to encoder memory; [RLT-TC] "What is this
+ * technology": the prefix-restricted global KV memory).
+ *   q       device, float32 [n][n_heads][head_dim]
+ *   kv      device, dtype, [n][n_heads][2][cap][head_dim]: a key block of
+ *           cap rows, then a value block of cap rows, per (row, head)
+ *   h_lengths host, int32 [n], each in [1, cap]; read before return
+ *   out     device, dtype, [n][n_heads][head_dim]
+ *   workspace device, >= rlt_attend_workspace_bytes(n, n_heads, head_dim,
+ *           cap) bytes, 256-byte aligned, owned by the caller; its first
+ *           int32 is a device error word (0 = ok, RLT_ERR_TIMEOUT if a
+ *           bounded wait gave up). Calls sharing a workspace must not overlap.
+ * Rows are split into chunks of 256 positions merged in chunk order, so a
+ * row's result does not depend on the other rows. Errors: INVALID_ARG,
+ * UNSUPPORTED (head_dim not 16/32/64/128), CAPACITY (workspace too small). */
+RLT_API int rlt_attend(const float *q, const void *kv, const int32_t *h_lengths, int n,
+                       int n_heads, int head_dim, int cap, int dtype, void *out,
+                       void *workspace, size_t workspace_bytes, rlt_stream stream);
+
 /* Kernel classes reported by rlt_get_stats. */
 enum {
   RLT_K_XATTN = 0, /* decoder cross-attention over M<=t (split-KV + merge) */

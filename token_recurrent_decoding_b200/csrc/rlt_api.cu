@@ -741,6 +741,106 @@ void advance(rlt_model *M, const int32_t *ids, int n) {
   for (int i = 0; i < n; i++) M->t_dec[ids[i]] += 1;
 }
 
+// ------------------------------------------------- standalone decode attention
+struct AttendWs {
+  size_t err, ready, pos, counters, part, total;
+};
+
+AttendWs attend_ws_layout(int n, int H, int dh, int cap) {
+  AttendWs w;
+  size_t off = 0;
+  auto take = [&](size_t b) {
+    size_t o = off;
+    off += align256(b ? b : 1);
+    return o;
+  };
+  size_t chunks = ((size_t)cap + XCH - 1) / XCH;
+  w.err = take(2 * 4 + 8);  // error word, then the device batch size
+  w.ready = take((size_t)n * 4);
+  w.pos = take((size_t)n * 4);
+  w.counters = take((size_t)n * H * 4);
+  w.part = take((size_t)n * H * chunks * (dh + 2) * 4);
+  w.total = off;
+  return w;
+}
+
+bool attend_shape_ok(int n, int H, int dh, int cap) {
+  return n > 0 && H > 0 && cap > 0 && (dh == 16 || dh == 32 || dh == 64 || dh == 128) &&
+         (size_t)n * H * cap * dh < (size_t)1 << 40;
+}
+
+__global__ void k_attend_prep(int n, int *ready) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) ready[i] = i;
+}
+
+template <typename T, int DH>
+cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengths, int n, int H,
+                          int cap, void *out, uint8_t *ws, cudaStream_t st) {
+  constexpr int STAGES = 4, NW = 4;
+  constexpr int smem = attn_smem_bytes<T, DH, STAGES, NW>();
+  auto kern = k_attn_decode<T, DH, STAGES, NW>;
+  static bool attr = false;
+  if (!attr) {
+    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr = true;
+  }
+  const AttendWs w = attend_ws_layout(n, H, DH, cap);
+  int lmax = 1;
+  std::vector<int> pos(n), hdr(2, 0);
+  for (int i = 0; i < n; i++) {
+    pos[i] = h_lengths[i] - 1;
+    lmax = std::max(lmax, (int)h_lengths[i]);
+  }
+  hdr[1] = n;
+  // pageable sources are staged before each call returns
+  RLT_TRY(cudaMemcpyAsync(ws + w.err, hdr.data(), 8, cudaMemcpyHostToDevice, st));
+  RLT_TRY(cudaMemcpyAsync(ws + w.pos, pos.data(), 4 * (size_t)n, cudaMemcpyHostToDevice, st));
+  RLT_TRY(cudaMemsetAsync(ws + w.counters, 0, (size_t)n * H * 4, st));
+  k_attend_prep<<<blocks_for(n, 256), 256, 0, st>>>(n, reinterpret_cast<int *>(ws + w.ready));
+  RLT_TRY(cudaGetLastError());
+  const int xchunks = (lmax + XCH - 1) / XCH, max_chunks = (cap + XCH - 1) / XCH;
+  kern<<<n * H * xchunks, NW * 32, smem, st>>>(
+      reinterpret_cast<int *>(ws + w.err) + 1, H, 0, XCH, xchunks, max_chunks,
+      reinterpret_cast<int *>(ws + w.ready), reinterpret_cast<int *>(ws + w.pos), q,
+      static_cast<const T *>(kv), (long)H * 2 * cap * DH, 2L * cap * DH, (long)cap * DH,
+      reinterpret_cast<float *>(ws + w.part), reinterpret_cast<int *>(ws + w.counters),
+      static_cast<T *>(out), 1.0f / sqrtf((float)DH), reinterpret_cast<int *>(ws + w.err));
+  return cudaGetLastError();
+}
+
+// Shared by every entry point that runs the standalone decode attention.
+int attend_run(const float *q, const void *kv, const int32_t *h_lengths, int n, int H, int dh,
+               int cap, int dtype, void *out, void *workspace, size_t workspace_bytes,
+               cudaStream_t st) {
+  if (!q || !kv || !h_lengths || !out || !workspace || ((uintptr_t)workspace & 255))
+    return RLT_ERR_INVALID_ARG;
+  if (dtype != RLT_F32 && dtype != RLT_BF16) return RLT_ERR_INVALID_ARG;
+  if (!(dh == 16 || dh == 32 || dh == 64 || dh == 128)) return RLT_ERR_UNSUPPORTED;
+  if (!attend_shape_ok(n, H, dh, cap)) return RLT_ERR_INVALID_ARG;
+  for (int i = 0; i < n; i++)
+    if (h_lengths[i] < 1 || h_lengths[i] > cap) return RLT_ERR_INVALID_ARG;
+  if (workspace_bytes < attend_ws_layout(n, H, dh, cap).total) return RLT_ERR_CAPACITY;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  cudaError_t e;
+  if (dtype == RLT_BF16) {
+    switch (dh) {
+      case 16: e = attend_launch<bf16, 16>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+      case 32: e = attend_launch<bf16, 32>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+      case 64: e = attend_launch<bf16, 64>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+      default: e = attend_launch<bf16, 128>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+    }
+  } else {
+    switch (dh) {
+      case 16: e = attend_launch<float, 16>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+      case 32: e = attend_launch<float, 32>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+      case 64: e = attend_launch<float, 64>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+      default: e = attend_launch<float, 128>(q, kv, h_lengths, n, H, cap, out, ws, st); break;
+    }
+  }
+  return cuda_status(e);
+}
+
 }  // namespace
 
 // ===================================================================== C ABI
@@ -762,6 +862,18 @@ RLT_API const char *rlt_status_string(int s) {
 }
 
 RLT_API int rlt_check_config(const rlt_config *cfg) { return check_config(cfg); }
+
+RLT_API size_t rlt_attend_workspace_bytes(int n, int n_heads, int head_dim, int cap) {
+  if (!attend_shape_ok(n, n_heads, head_dim, cap)) return 0;
+  return attend_ws_layout(n, n_heads, head_dim, cap).total;
+}
+
+RLT_API int rlt_attend(const float *q, const void *kv, const int32_t *h_lengths, int n,
+                       int n_heads, int head_dim, int cap, int dtype, void *out,
+                       void *workspace, size_t workspace_bytes, rlt_stream stream) {
+  return attend_run(q, kv, h_lengths, n, n_heads, head_dim, cap, dtype, out, workspace,
+                    workspace_bytes, (cudaStream_t)stream);
+}
 
 RLT_API size_t rlt_arena_bytes(const rlt_config *cfg) {
   if (check_config(cfg) != RLT_OK) return 0;

@@ -87,6 +87,9 @@ def _declare(lib):
     lib.rlt_set_state.argtypes = [P, I, P, P, C.c_int64, P]
     lib.rlt_get_encoder_output.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
     lib.rlt_poll_device_error.argtypes = [P]
+    lib.rlt_attend_workspace_bytes.argtypes = [I, I, I, I]
+    lib.rlt_attend_workspace_bytes.restype = C.c_size_t
+    lib.rlt_attend.argtypes = [P, P, P, I, I, I, I, I, P, P, C.c_size_t, P]
     lib.rlt_profile.argtypes = [P, I]
     lib.rlt_get_stats.argtypes = [P, P]
     lib.rlt_status_string.argtypes = [I]
@@ -152,6 +155,30 @@ def plan_ragged(steps):
     _check(_lib().rlt_plan_ragged(_p(st), n, _p(order), _p(sizes), max(tmax, 1), C.byref(nt)),
            "rlt_plan_ragged")
     return order[:n], sizes[: nt.value]
+
+
+def attend_workspace_bytes(n: int, n_heads: int, head_dim: int, cap: int) -> int:
+    return int(_lib().rlt_attend_workspace_bytes(n, n_heads, head_dim, cap))
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def attend(q, kv, lengths, out, workspace, stream=None):
+    """rlt_attend: q [n][H][dh] fp32, kv [n][H][2][cap][dh] (bf16 or fp32),
+    lengths (host ints) -> out [n][H][dh] (kv dtype). Torch tensors on the GPU."""
+    import torch
+    n, H, two, cap, dh = kv.shape
+    assert two == 2 and q.shape == (n, H, dh) and out.shape == (n, H, dh)
+    dtype = BF16 if kv.dtype == torch.bfloat16 else 0
+    lens = _i32(lengths)
+    _check(_lib().rlt_attend(C.c_void_p(q.data_ptr()), C.c_void_p(kv.data_ptr()), _p(lens), n, H,
+                             dh, cap, dtype, C.c_void_p(out.data_ptr()),
+                             C.c_void_p(workspace.data_ptr()), workspace.numel(),
+                             _stream_handle(stream)), "rlt_attend")
 
 
 class Model:
