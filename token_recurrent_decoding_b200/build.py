@@ -13,6 +13,14 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librlt.so")
 MAIN = os.path.join(CSRC, "rlt_api.cu")
+
+
+def units():
+    """Every translation unit of the library (rlt_api.cu first)."""
+    extra = sorted(f for f in os.listdir(CSRC) if f.endswith(".cu") and f != "rlt_api.cu")
+    return [MAIN] + [os.path.join(CSRC, f) for f in extra]
+
+
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -41,7 +49,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not stale():
         return LIB
     tmp = LIB + ".tmp"
-    cmd = [NVCC, *FLAGS, *extra, MAIN, "-o", tmp]
+    cmd = [NVCC, *FLAGS, *extra, *units(), "-o", tmp]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

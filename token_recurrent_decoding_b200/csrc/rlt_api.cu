@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "../../include/rlt.h"
+#include "internal.h"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "kernels.cuh"
@@ -843,6 +844,21 @@ int attend_run(const float *q, const void *kv, const int32_t *h_lengths, int n, 
 
 }  // namespace
 
+namespace rlt {
+
+int attend_run_internal(const float *q, const void *kv, const int32_t *h_lengths, int n, int H,
+                        int dh, int cap, int dtype, void *out, void *workspace,
+                        size_t workspace_bytes, cudaStream_t st) {
+  return attend_run(q, kv, h_lengths, n, H, dh, cap, dtype, out, workspace, workspace_bytes, st);
+}
+
+size_t attend_workspace_internal(int n, int H, int dh, int cap) {
+  if (!attend_shape_ok(n, H, dh, cap)) return 0;
+  return attend_ws_layout(n, H, dh, cap).total;
+}
+
+}  // namespace rlt
+
 // ===================================================================== C ABI
 extern "C" {
 
@@ -864,8 +880,7 @@ RLT_API const char *rlt_status_string(int s) {
 RLT_API int rlt_check_config(const rlt_config *cfg) { return check_config(cfg); }
 
 RLT_API size_t rlt_attend_workspace_bytes(int n, int n_heads, int head_dim, int cap) {
-  if (!attend_shape_ok(n, n_heads, head_dim, cap)) return 0;
-  return attend_ws_layout(n, n_heads, head_dim, cap).total;
+  return rlt::attend_workspace_internal(n, n_heads, head_dim, cap);
 }
 
 RLT_API int rlt_attend(const float *q, const void *kv, const int32_t *h_lengths, int n,
