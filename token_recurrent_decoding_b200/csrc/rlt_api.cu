@@ -177,6 +177,13 @@ struct rlt_model {
     int64_t launches;
   };
   std::map<std::tuple<int, int, int>, Graph> graphs;
+  // profiled steps replay a graph with event-record nodes between kernels
+  struct ProfGraph {
+    cudaGraphExec_t exec;
+    std::vector<ProfSpan> spans;
+    int64_t launches;
+  };
+  std::map<std::tuple<int, int, int>, ProfGraph> prof_graphs;
   cudaStream_t side = nullptr;  // second chain of a split step
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   // TMA descriptors of bf16 [rows][cols] matrices, keyed by (pointer, rows, cols, box rows)
@@ -364,8 +371,10 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
   const Layout &L = M->L;
   const rlt_config &c = M->cfg;
   const size_t r0 = si.row0, H = c.n_heads;
-  kern<<<si.n_grid * c.n_heads * xchunks, NW * 32, smem, st>>>(
-      M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks,
+  const int units = si.n_grid * c.n_heads * xchunks;
+  const int grid = std::min(units, attn_grid_ctas<T, DH, STAGES, NW>());
+  kern<<<grid, NW * 32, smem, st>>>(
+      M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks, si.n_grid,
       M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0, M->at<float>(L.q) + r0 * c.d, base,
       seq_stride, head_stride, v_offset, M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
       M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH), M->at<int>(L.err));
@@ -692,6 +701,55 @@ cudaError_t launch_chains(rlt_model *M, const StepInfo *ch, int nch, cudaStream_
 // the batch sizes go to the device, then the step runs directly (first use,
 // legacy stream, or a profiled sample, which runs as one unsplit chain so
 // each kernel is timed alone) or replays its captured graph.
+// Fold the event pairs of one replayed profiling graph into the class sums;
+// attention bytes/FLOPs follow this step's positions.
+cudaError_t fold_profile(rlt_model *M, const rlt_model::ProfGraph &pg, const StepInfo &si) {
+  const double es = M->cfg.dtype == RLT_BF16 ? 2.0 : 4.0, d = M->cfg.d;
+  for (const ProfSpan &p : pg.spans) {
+    float ms = 0.f;
+    RLT_TRY(cudaEventElapsedTime(&ms, p.a, p.b));
+    double bytes = p.bytes, flops = p.flops;
+    if (p.kind == RLT_K_XATTN) {
+      bytes = si.sum_keys * 2.0 * d * es;
+      flops = 4.0 * d * si.sum_keys;
+    } else if (p.kind == RLT_K_SWA) {
+      bytes = si.sum_win * 2.0 * d * es + (double)si.n * d * (4 + es);
+      flops = 4.0 * d * si.sum_win;
+    }
+    M->stats.kernel_ms[p.kind] += ms;
+    M->stats.kernel_launches[p.kind] += 1;
+    M->stats.kernel_bytes[p.kind] += bytes;
+    M->stats.kernel_flops[p.kind] += flops;
+  }
+  return cudaSuccess;
+}
+
+// Capture `fn` on st into an executable graph; returns the kernels counted.
+template <class Fn>
+cudaError_t capture(rlt_model *M, cudaStream_t st, Fn fn, cudaGraphExec_t *out, int64_t *launches) {
+  const int64_t l0 = M->stats.launches;
+  cudaGraph_t g = nullptr;
+  RLT_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+  cudaError_t ec = fn();
+  cudaError_t ee = cudaStreamEndCapture(st, &g);
+  *launches = M->stats.launches - l0;
+  M->stats.launches = l0;  // captured, not launched
+  if (ec != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    return ec;
+  }
+  RLT_TRY(ee);
+  cudaError_t ei = cudaGraphInstantiate(out, g, 0);
+  cudaGraphDestroy(g);
+  return ei;
+}
+
+// One decoder step of the slots already listed in the arena's ready list:
+// the batch sizes go to the device, then the step runs directly (legacy
+// stream, or the first use of a shape) or replays its captured graph. Every
+// prof_stride-th step, when profiling, runs as one unsplit chain from a graph
+// whose event-record nodes bracket each kernel, so every kernel is timed
+// alone and without host gaps; that step is synchronised and folded.
 cudaError_t enqueue_step(rlt_model *M, const StepInfo &all, cudaStream_t st) {
   StepInfo ch[2];
   const bool prof = M->profiling && M->prof_stride > 0 && (M->step_counter % M->prof_stride == 0);
@@ -705,34 +763,43 @@ cudaError_t enqueue_step(rlt_model *M, const StepInfo &all, cudaStream_t st) {
   RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.nready), nval, sizeof(nval), cudaMemcpyHostToDevice,
                           st));  // pageable source: staged before return
   auto key = std::make_tuple(ch[0].n_grid, nch == 2 ? ch[1].n_grid : 0, all.xchunks);
-  auto it = M->graphs.find(key);
-  if (st == nullptr || prof || it == M->graphs.end()) {
-    const bool saved = M->profiling;
+  const bool saved = M->profiling;
+  if (st == nullptr) {  // legacy stream: cannot capture
     M->profiling = prof;
     cudaError_t e = launch_chains(M, ch, nch, st);
     M->profiling = saved;
-    RLT_TRY(e);
-    if (st == nullptr || prof) return cudaSuccess;
-    // capture this shape once for replay
-    int64_t l0 = M->stats.launches;
-    cudaGraph_t g = nullptr;
-    RLT_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
-    M->profiling = false;
-    cudaError_t ec = launch_chains(M, ch, nch, st);
-    M->profiling = saved;
-    cudaError_t ee = cudaStreamEndCapture(st, &g);
-    if (ec != cudaSuccess) {
-      if (g) cudaGraphDestroy(g);
-      return ec;
+    return e;
+  }
+  if (prof) {
+    auto pit = M->prof_graphs.find(key);
+    if (pit == M->prof_graphs.end()) {
+      rlt_model::ProfGraph pg{};
+      const size_t p0 = M->pending.size();
+      M->profiling = true;
+      cudaError_t e = capture(M, st, [&] { return launch_chains(M, ch, 1, st); }, &pg.exec,
+                              &pg.launches);
+      M->profiling = saved;
+      pg.spans.assign(M->pending.begin() + p0, M->pending.end());
+      M->pending.resize(p0);
+      RLT_TRY(e);
+      pit = M->prof_graphs.emplace(key, pg).first;
     }
-    RLT_TRY(ee);
-    cudaGraphExec_t ge = nullptr;
-    cudaError_t ei = cudaGraphInstantiate(&ge, g, 0);
-    cudaGraphDestroy(g);
-    RLT_TRY(ei);
-    M->graphs[key] = {ge, M->stats.launches - l0};
-    M->stats.launches = l0;  // captured, not launched
-    return cudaSuccess;
+    M->stats.launches += pit->second.launches;
+    RLT_TRY(cudaGraphLaunch(pit->second.exec, st));
+    RLT_TRY(cudaStreamSynchronize(st));
+    return fold_profile(M, pit->second, all);
+  }
+  auto it = M->graphs.find(key);
+  if (it == M->graphs.end()) {
+    M->profiling = false;
+    cudaError_t e = launch_chains(M, ch, nch, st);
+    if (e == cudaSuccess) {
+      rlt_model::Graph g{};
+      e = capture(M, st, [&] { return launch_chains(M, ch, nch, st); }, &g.exec, &g.launches);
+      if (e == cudaSuccess) M->graphs[key] = g;
+    }
+    M->profiling = saved;
+    return e;
   }
   M->stats.launches += it->second.launches;
   return cudaGraphLaunch(it->second.exec, st);
@@ -801,8 +868,9 @@ cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengt
   k_attend_prep<<<blocks_for(n, 256), 256, 0, st>>>(n, reinterpret_cast<int *>(ws + w.ready));
   RLT_TRY(cudaGetLastError());
   const int xchunks = (lmax + XCH - 1) / XCH, max_chunks = (cap + XCH - 1) / XCH;
-  kern<<<n * H * xchunks, NW * 32, smem, st>>>(
-      reinterpret_cast<int *>(ws + w.err) + 1, H, 0, XCH, xchunks, max_chunks,
+  const int grid = std::min(n * H * xchunks, attn_grid_ctas<T, DH, STAGES, NW>());
+  kern<<<grid, NW * 32, smem, st>>>(
+      reinterpret_cast<int *>(ws + w.err) + 1, H, 0, XCH, xchunks, max_chunks, n,
       reinterpret_cast<int *>(ws + w.ready), reinterpret_cast<int *>(ws + w.pos), q,
       static_cast<const T *>(kv), (long)H * 2 * cap * DH, 2L * cap * DH, (long)cap * DH,
       reinterpret_cast<float *>(ws + w.part), reinterpret_cast<int *>(ws + w.counters),
@@ -977,6 +1045,13 @@ RLT_API void rlt_destroy(rlt_model *M) {
   }
   for (auto e : M->ev_pool) cudaEventDestroy(e);
   for (auto &g : M->graphs) cudaGraphExecDestroy(g.second.exec);
+  for (auto &g : M->prof_graphs) {
+    cudaGraphExecDestroy(g.second.exec);
+    for (auto &p : g.second.spans) {
+      cudaEventDestroy(p.a);
+      cudaEventDestroy(p.b);
+    }
+  }
   if (M->side) {
     cudaStreamSynchronize(M->side);
     cudaStreamDestroy(M->side);

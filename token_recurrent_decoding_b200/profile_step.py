@@ -1,0 +1,114 @@
+"""Short runs of the hot path for profilers (few launches, device-timed).
+
+Decoder steps at a chosen position:
+
+    python -m token_recurrent_decoding_b200.profile_step --workload m140_bf16 --t 512 --steps 2
+
+prefills the encoder for the batch, places every sequence at position t with a
+random state imported through rlt_set_state (s and the window of every layer),
+and runs `steps` decoder steps with direct launches on the legacy stream, so a
+profiler sees each kernel once per layer per step. Prints the CUDA-event time
+of each step and its algorithmic bytes.
+
+The decode attention kernel alone, through rlt_attend:
+
+    python -m token_recurrent_decoding_b200.profile_step --attend --n 256 --heads 12 \
+        --dh 64 --cap 1024 --len 1024 --reps 3
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import numpy as np
+
+
+def run_steps(args):
+    import torch
+
+    from . import configs, inputs, roofline
+    from .rlt import Model
+    wl = configs.workloads()[args.workload]
+    cfg = wl.model
+    B = args.batch or wl.batch
+    T = wl.max_len
+    lengths = [T] * B
+    w = inputs.make_weights(cfg)
+    tok = inputs.make_tokens(cfg.vocab, lengths)
+    m = Model(cfg, w, B, T)
+    del w
+    flat = torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda()
+    offsets = np.arange(B, dtype=np.int32) * T
+    m.prefill_encoder(flat, list(range(B)), offsets, lengths)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    s = torch.randn(cfg.d, generator=g, device="cuda")
+    cache = torch.randn((cfg.n_dec, 2, max(cfg.window - 1, 0), cfg.d), generator=g,
+                        device="cuda").to(m.wdtype)
+    for i in range(B):
+        m.set_state(i, s, cache, args.t)
+    torch.cuda.synchronize()
+    ids = list(range(B))
+    times = []
+    for k in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        m.decoder_step(ids)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    assert m.poll_device_error() == 0
+    ts = [np.full(B, args.t + k) for k in range(args.steps)]
+    byts = [roofline.decoder_step_bytes(cfg, x) for x in ts]
+    print(json.dumps({"workload": args.workload, "batch": B, "t": args.t,
+                      "step_ms": times, "step_GB": [x / 1e9 for x in byts],
+                      "GB_s": [x / (ms / 1e3) / 1e9 for x, ms in zip(byts, times)]}))
+
+
+def run_attend(args):
+    import torch
+
+    from . import rlt
+    n, H, dh, cap = args.n, args.heads, args.dh, args.cap
+    L = args.len or cap
+    g = torch.Generator(device="cuda").manual_seed(3)
+    q = torch.randn((n, H, dh), generator=g, device="cuda")
+    kv = torch.randn((n, H, 2, cap, dh), generator=g, device="cuda").to(torch.bfloat16)
+    out = torch.empty((n, H, dh), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(rlt.attend_workspace_bytes(n, H, dh, cap), dtype=torch.uint8,
+                     device="cuda")
+    lengths = [L] * n
+    times = []
+    for _ in range(args.reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        rlt.attend(q, kv, lengths, out, ws)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    byts = n * H * 2 * L * dh * 2
+    print(json.dumps({"attend": [n, H, dh, cap, L], "ms": times, "GB": byts / 1e9,
+                      "GB_s": [byts / (t / 1e3) / 1e9 for t in times]}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="m140_bf16")
+    ap.add_argument("--t", type=int, default=512)
+    ap.add_argument("--steps", type=int, default=2)
+    ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--attend", action="store_true")
+    ap.add_argument("--n", type=int, default=256)
+    ap.add_argument("--heads", type=int, default=12)
+    ap.add_argument("--dh", type=int, default=64)
+    ap.add_argument("--cap", type=int, default=1024)
+    ap.add_argument("--len", type=int, default=0)
+    ap.add_argument("--reps", type=int, default=3)
+    args = ap.parse_args()
+    if args.attend:
+        run_attend(args)
+    else:
+        run_steps(args)
+
+
+if __name__ == "__main__":
+    main()
