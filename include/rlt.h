@@ -231,6 +231,27 @@ RLT_API int rlt_attend(const float *q, const void *kv, const int32_t *h_lengths,
                        int n_heads, int head_dim, int cap, int dtype, void *out,
                        void *workspace, size_t workspace_bytes, rlt_stream stream);
 
+/* Scratch bytes compiled into the library for rlt_attend_noalloc (8 MiB). */
+#define RLT_ATTEND_NOALLOC_BYTES (8u << 20)
+
+/* rlt_attend for callers that cannot allocate device memory (no counterpart
+ * in the paper: a deployment convenience). Same arguments, layouts and
+ * results as rlt_attend, minus the workspace: the scratch lives in a
+ * file-scope device array of RLT_ATTEND_NOALLOC_BYTES that every GPU loading
+ * the library holds until exit. Allocates nothing (no cudaMalloc / cudaFree).
+ *   - Returns RLT_ERR_CAPACITY when rlt_attend_workspace_bytes(n, n_heads,
+ *     head_dim, cap) exceeds RLT_ATTEND_NOALLOC_BYTES.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address once; make that first call before any stream
+ *     capture.
+ *   - All calls on a device share its one array; each call clears what must
+ *     start at zero, but calls that overlap on the GPU (for example on two
+ *     streams) race on the array: serialise them.
+ *   - The device error word of rlt_attend is not reported. */
+RLT_API int rlt_attend_noalloc(const float *q, const void *kv, const int32_t *h_lengths, int n,
+                               int n_heads, int head_dim, int cap, int dtype, void *out,
+                               rlt_stream stream);
+
 /* Kernel classes reported by rlt_get_stats. */
 enum {
   RLT_K_XATTN = 0, /* decoder cross-attention over M<=t (split-KV + merge) */
