@@ -72,5 +72,5 @@ def test_attend_workspace_sizing():
     assert rlt.attend_workspace_bytes(0, 1, 64, 8) == 0
     assert rlt.attend_workspace_bytes(4, 1, 48, 8) == 0
     a = rlt.attend_workspace_bytes(256, 12, 64, 1024)
-    assert a >= 256 * 12 * 4 * 66 * 4
+    assert a > 256 * 12 * 66 * 4  # partials of more than one chunk per (row, head)
     assert rlt.attend_workspace_bytes(256, 12, 64, 2048) > a

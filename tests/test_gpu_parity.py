@@ -22,10 +22,11 @@ ENC_TOL = {configs.F32: (1e-5, 1e-6), configs.BF16: (6e-2, 1.5e-2)}
 CACHE_TOL = {configs.F32: 1e-5, configs.BF16: 5e-2}
 
 
-@pytest.mark.parametrize("name", list(SMALL))
-def test_encoder_and_memory_parity(name):
+@pytest.mark.parametrize("name,lengths", [(n, [37, 70, 5, 1]) for n in SMALL]
+                         + [("m50_like", [300, 257, 128, 1, 64]),
+                            ("tied_like", [200, 129, 63])])
+def test_encoder_and_memory_parity(name, lengths):
     cfg = SMALL[name]
-    lengths = [37, 70, 5, 1]
     m, w, tok = make_model(cfg, lengths)
     o = oracle.Oracle(cfg, w)
     tmax, trel = ENC_TOL[cfg.dtype]
@@ -243,3 +244,25 @@ def test_graph_replay_equals_direct_launches():
         assert sa[2] == sb[2] == lengths[i]
         assert torch.equal(sa[0], sb[0]) and torch.equal(sa[1], sb[1])
     assert a.poll_device_error() == 0 and b.poll_device_error() == 0
+
+
+def test_encoder_is_causal_at_full_size_bitwise():
+    """Changing tokens after position k changes no e_<=k and no memory row
+    <= k, at the ~140M workload's size (256 x 1024 tokens, 131072-row chunks)."""
+    wl = configs.workloads()["m140_bf16"]
+    cfg = wl.model
+    B, T = 8, wl.max_len
+    w = inputs.make_weights(cfg)
+    tok = inputs.make_tokens(cfg.vocab, [T] * B)
+    m = Model(cfg, w, B, T)
+    prefill_all(m, tok, [T] * B)
+    before = [m.get_encoder_output(i) for i in (0, 5)]
+    k = 700
+    tok2 = tok.copy()
+    tok2[:, k + 1:] = (tok2[:, k + 1:] + 7) % cfg.vocab
+    prefill_all(m, tok2, [T] * B)
+    for (e0, m0), i in zip(before, (0, 5)):
+        e1, m1 = m.get_encoder_output(i)
+        assert torch.equal(e0[: k + 1], e1[: k + 1])
+        assert torch.equal(m0[:, : k + 1], m1[:, : k + 1])
+        assert not torch.equal(e0[k + 1:], e1[k + 1:])

@@ -100,10 +100,27 @@ constexpr int GEMM_BK = 64;  // 128-byte rows of bf16, 8 chunks of 16 bytes
 // Shared tile [rows][64] bf16 with chunk c of row r stored at c ^ (r & 7).
 __device__ __forceinline__ int swz(int r, int c) { return r * GEMM_BK + ((c ^ (r & 7)) << 3); }
 
+// Split-K scratch of one GEMM call: `splits` partial tiles [split][M][N] in
+// fp32 and one arrival counter per output tile (zero between calls).
+struct SplitK {
+  int splits;
+  float *part;
+  int *counters;
+};
+
+// K blocks (64 wide) per split, at most 8: the split count depends only on K,
+// never on the batch, so a row's result does not depend on its batch.
+inline int gemm_splits(int K) {
+  const int kt = K / 64;
+  for (int s = 1; s <= kt; s++)
+    if (kt % s == 0 && kt / s <= 8) return s;
+  return 1;
+}
+
 template <int BM, int BN, int WM, int WN, int STAGES, class Epi>
 __global__ void __launch_bounds__(WM *WN * 32)
     k_gemm_bf16(int M, const int *__restrict__ Mdev, int N, int K, const bf16 *__restrict__ A,
-                int lda, const bf16 *__restrict__ B, int ldb, Epi epi) {
+                int lda, const bf16 *__restrict__ B, int ldb, Epi epi, SplitK sk) {
   constexpr int NT = WM * WN * 32;
   constexpr int TM = BM / WM, TN = BN / WN;
   constexpr int FM = TM / 16, FN = TN / 8;
@@ -114,9 +131,14 @@ __global__ void __launch_bounds__(WM *WN * 32)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wm = warp / WN, wn = warp % WN;
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-  const int KT = K / GEMM_BK;
+  const int M_grid = gridDim.y * BM;
+  // this split's K blocks
+  const int kt_all = K / GEMM_BK, z = blockIdx.z;
+  const int kt0 = z * kt_all / sk.splits, KT = (z + 1) * kt_all / sk.splits - kt0;
   if (Mdev) M = *Mdev;  // rows decided on the device (grid sized for an upper bound)
   if (m0 >= M) return;
+  A += (size_t)kt0 * GEMM_BK;
+  B += (size_t)kt0 * GEMM_BK;
 
   auto load_stage = [&](int st, int kt) {
     bf16 *as = As + st * BM * GEMM_BK;
@@ -184,6 +206,54 @@ __global__ void __launch_bounds__(WM *WN * 32)
   }
   cp_async_wait<0>();
 
+  if (sk.splits > 1) {
+    // write this split's partial tile; the last split to arrive sums all of
+    // them in split order and runs the epilogue
+    float *pz = sk.part + (size_t)z * M_grid * N;
+#pragma unroll
+    for (int fm = 0; fm < FM; fm++)
+#pragma unroll
+      for (int fn = 0; fn < FN; fn++) {
+        int r = m0 + wm * TM + fm * 16 + (lane >> 2);
+        int c = n0 + wn * TN + fn * 8 + (lane & 3) * 2;
+        if (c < N) {
+          if (r < M)
+            *reinterpret_cast<float2 *>(pz + (size_t)r * N + c) =
+                make_float2(acc[fm][fn][0], acc[fm][fn][1]);
+          if (r + 8 < M)
+            *reinterpret_cast<float2 *>(pz + (size_t)(r + 8) * N + c) =
+                make_float2(acc[fm][fn][2], acc[fm][fn][3]);
+        }
+      }
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+    if (tid == 0) s_last = (atomicAdd(&sk.counters[tile], 1) == sk.splits - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+#pragma unroll
+    for (int fm = 0; fm < FM; fm++)
+#pragma unroll
+      for (int fn = 0; fn < FN; fn++)
+#pragma unroll
+        for (int hrow = 0; hrow < 2; hrow++) {
+          int r = m0 + wm * TM + fm * 16 + (lane >> 2) + hrow * 8;
+          int c = n0 + wn * TN + fn * 8 + (lane & 3) * 2;
+          if (c >= N || r >= M) continue;
+          float2 v = make_float2(0.f, 0.f);
+          for (int zz = 0; zz < sk.splits; zz++) {
+            float2 p = __ldcg(reinterpret_cast<const float2 *>(
+                sk.part + ((size_t)zz * M_grid + r) * N + c));
+            v.x += p.x;
+            v.y += p.y;
+          }
+          epi(r, c, v.x, v.y);
+        }
+    if (tid == 0) sk.counters[tile] = 0;
+    return;
+  }
 #pragma unroll
   for (int fm = 0; fm < FM; fm++)
 #pragma unroll
@@ -247,7 +317,7 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------ launchers
 template <int BM, int BN, int WM, int WN, int STAGES, class Epi>
 cudaError_t launch_gemm_bf16_cfg(int M, const int *Mdev, int N, int K, const bf16 *A, int lda,
-                                 const bf16 *B, int ldb, Epi epi, cudaStream_t st) {
+                                 const bf16 *B, int ldb, Epi epi, SplitK sk, cudaStream_t st) {
   constexpr int smem = STAGES * (BM + BN) * GEMM_BK * 2;
   auto kern = k_gemm_bf16<BM, BN, WM, WN, STAGES, Epi>;
   static bool attr_set = false;  // per template instance
@@ -256,26 +326,31 @@ cudaError_t launch_gemm_bf16_cfg(int M, const int *Mdev, int N, int K, const bf1
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-  kern<<<grid, WM * WN * 32, smem, st>>>(M, Mdev, N, K, A, lda, B, ldb, epi);
+  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, sk.splits);
+  kern<<<grid, WM * WN * 32, smem, st>>>(M, Mdev, N, K, A, lda, B, ldb, epi, sk);
   return cudaGetLastError();
 }
 
 // Tile choice: large M (encoder) uses 128x128 tiles; the decoder's small
 // batches use 64x64 tiles so more SMs stream the weights. M is the grid's row
 // bound; Mdev (optional) gives the actual rows at run time (<= M).
+// `ws` (optional) enables split-K for the small-batch tiles: part must hold
+// gemm_splits(K) * round_up(M, 64) * N floats, counters one int per 64x64 tile.
 template <class Epi>
 cudaError_t gemm(int M, const int *Mdev, int N, int K, const bf16 *A, int lda, const bf16 *B,
-                 int ldb, Epi epi, cudaStream_t st) {
+                 int ldb, Epi epi, cudaStream_t st, const SplitK *ws = nullptr) {
   if (M <= 0 || N <= 0) return cudaSuccess;
+  SplitK one{1, nullptr, nullptr};
   if (M >= 1024)
-    return launch_gemm_bf16_cfg<128, 128, 2, 4, 3>(M, Mdev, N, K, A, lda, B, ldb, epi, st);
-  return launch_gemm_bf16_cfg<64, 64, 2, 2, 4>(M, Mdev, N, K, A, lda, B, ldb, epi, st);
+    return launch_gemm_bf16_cfg<128, 128, 2, 4, 3>(M, Mdev, N, K, A, lda, B, ldb, epi, one, st);
+  SplitK sk = one;
+  if (ws && ws->part && gemm_splits(K) > 1) sk = {gemm_splits(K), ws->part, ws->counters};
+  return launch_gemm_bf16_cfg<64, 64, 2, 2, 4>(M, Mdev, N, K, A, lda, B, ldb, epi, sk, st);
 }
 
 template <class Epi>
 cudaError_t gemm(int M, const int *Mdev, int N, int K, const float *A, int lda, const float *B,
-                 int ldb, Epi epi, cudaStream_t st) {
+                 int ldb, Epi epi, cudaStream_t st, const SplitK * = nullptr) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + 63) / 64, (M + 63) / 64);
   k_gemm_f32<Epi><<<grid, 256, 0, st>>>(M, Mdev, N, K, A, lda, B, ldb, epi);

@@ -28,7 +28,7 @@ using namespace rlt;
 
 namespace {
 
-constexpr int XCH = 256;  // memory positions per cross-attention split
+constexpr int XCH = 512;  // memory positions per cross-attention split
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -37,6 +37,7 @@ struct Layout {
   size_t s, t_dec, t_enc, e, mem, ring, rope, err;
   // decoder step work buffers (max_seqs rows)
   size_t nready, ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part, counters;
+  size_t gpart[2], gcnt[2];  // split-K scratch of each step chain
   // encoder work buffers (ptok rows)
   size_t tok, tok_slot, tok_pos, tok_start, blk, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
   size_t staging, staging_bytes;
@@ -109,6 +110,17 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->f = take(S * F * es);
   L->part = take(S * H * L->max_chunks * (dh + 2) * 4);
   L->counters = take(S * H * 4);
+  {
+    // split-K scratch: largest splits * N over the decoder GEMMs, per row
+    auto sn = [](size_t n, size_t k) { return (size_t)gemm_splits((int)k) * n; };
+    const size_t per_row = std::max({sn(d, 2 * d), sn(3 * d, d), sn(d, d), sn(F, d), sn(d, F)});
+    const size_t rows = (S + 63) / 64 * 64;
+    const size_t tiles = rows / 64 * ((std::max({3 * d, F, d}) + 63) / 64);
+    for (int ch = 0; ch < 2; ch++) {
+      L->gpart[ch] = take(c->dtype == RLT_BF16 ? per_row * rows * 4 : 0);
+      L->gcnt[ch] = take(tiles * 4);
+    }
+  }
   size_t P = (size_t)ptok;
   L->tok = take(P * 4);
   L->tok_slot = take(P * 4);
@@ -166,6 +178,7 @@ struct rlt_model {
   template <typename X> X *at(size_t off) const { return reinterpret_cast<X *>(arena + off); }
   // measurement hook (rlt_profile / rlt_get_stats)
   bool profiling = false;
+  bool capturing = false;  // inside a stream capture: events become graph record nodes
   std::vector<cudaEvent_t> ev_pool;
   std::vector<ProfSpan> pending;
   rlt_stats stats{};
@@ -294,15 +307,23 @@ struct Span {
     M->stats.launches++;
     if (M->profiling) {
       a = take_event(M);
-      if (a) cudaEventRecord(a, st);
+      if (a) record(a);
     }
   }
   ~Span() {
     if (!a) return;
     cudaEvent_t b = take_event(M);
     if (!b) return;
-    cudaEventRecord(b, st);
+    record(b);
     M->pending.push_back({kind, a, b, bytes, flops});
+  }
+  // Under capture a plain record only orders streams; an external record
+  // becomes a node that records the event each time the graph runs.
+  void record(cudaEvent_t e) {
+    if (M->capturing)
+      cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    else
+      cudaEventRecord(e, st);
   }
 };
 
@@ -360,20 +381,13 @@ template <typename T, int DH>
 cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunks,
                         const T *base, long seq_stride, long head_stride, long v_offset,
                         T *out, cudaStream_t st) {
-  constexpr int STAGES = 4, NW = 4;
-  constexpr int smem = attn_smem_bytes<T, DH, STAGES, NW>();
-  auto kern = k_attn_decode<T, DH, STAGES, NW>;
-  static bool attr = false;
-  if (!attr) {
-    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    attr = true;
-  }
+  constexpr int smem = attn_smem_bytes<T, DH>();
   const Layout &L = M->L;
   const rlt_config &c = M->cfg;
   const size_t r0 = si.row0, H = c.n_heads;
   const int units = si.n_grid * c.n_heads * xchunks;
-  const int grid = std::min(units, attn_grid_ctas<T, DH, STAGES, NW>());
-  kern<<<grid, NW * 32, smem, st>>>(
+  const int grid = std::min(units, attn_grid_ctas<T, DH>());  // also sets the smem limit
+  k_attn_decode<T, DH><<<grid, (ATTN_NC + 1) * 32, smem, st>>>(
       M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks, si.n_grid,
       M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0, M->at<float>(L.q) + r0 * c.d, base,
       seq_stride, head_stride, v_offset, M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
@@ -410,7 +424,8 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   auto G = [&](int kind, int m, int nn, int k, const T *A, int lda, const T *B, int ldb,
                auto epi) {
     Span sp(M, st, kind, (double)nn * k * es + nr * k * es + nr * nn * 4.0, 2.0 * nr * nn * k);
-    return gemm(m, nd, nn, k, A, lda, B, ldb, epi, st);
+    const SplitK sk{0, M->at<float>(L.gpart[si.chain]), M->at<int>(L.gcnt[si.chain])};
+    return gemm(m, nd, nn, k, A, lda, B, ldb, epi, st, &sk);
   };
 
   {
@@ -730,7 +745,9 @@ cudaError_t capture(rlt_model *M, cudaStream_t st, Fn fn, cudaGraphExec_t *out, 
   const int64_t l0 = M->stats.launches;
   cudaGraph_t g = nullptr;
   RLT_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+  M->capturing = true;
   cudaError_t ec = fn();
+  M->capturing = false;
   cudaError_t ee = cudaStreamEndCapture(st, &g);
   *launches = M->stats.launches - l0;
   M->stats.launches = l0;  // captured, not launched
@@ -845,14 +862,8 @@ __global__ void k_attend_prep(int n, int *ready) {
 template <typename T, int DH>
 cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengths, int n, int H,
                           int cap, void *out, uint8_t *ws, cudaStream_t st) {
-  constexpr int STAGES = 4, NW = 4;
-  constexpr int smem = attn_smem_bytes<T, DH, STAGES, NW>();
-  auto kern = k_attn_decode<T, DH, STAGES, NW>;
-  static bool attr = false;
-  if (!attr) {
-    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    attr = true;
-  }
+  constexpr int smem = attn_smem_bytes<T, DH>();
+  const int ctas = attn_grid_ctas<T, DH>();  // also sets the smem limit
   const AttendWs w = attend_ws_layout(n, H, DH, cap);
   int lmax = 1;
   std::vector<int> pos(n), hdr(2, 0);
@@ -868,8 +879,8 @@ cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengt
   k_attend_prep<<<blocks_for(n, 256), 256, 0, st>>>(n, reinterpret_cast<int *>(ws + w.ready));
   RLT_TRY(cudaGetLastError());
   const int xchunks = (lmax + XCH - 1) / XCH, max_chunks = (cap + XCH - 1) / XCH;
-  const int grid = std::min(n * H * xchunks, attn_grid_ctas<T, DH, STAGES, NW>());
-  kern<<<grid, NW * 32, smem, st>>>(
+  const int grid = std::min(n * H * xchunks, ctas);
+  k_attn_decode<T, DH><<<grid, (ATTN_NC + 1) * 32, smem, st>>>(
       reinterpret_cast<int *>(ws + w.err) + 1, H, 0, XCH, xchunks, max_chunks, n,
       reinterpret_cast<int *>(ws + w.ready), reinterpret_cast<int *>(ws + w.pos), q,
       static_cast<const T *>(kv), (long)H * 2 * cap * DH, 2L * cap * DH, (long)cap * DH,
