@@ -7,22 +7,23 @@
 //    max(0, t-W+1)..t. Either way the window is rows 0 .. min(t+1, W)-1.
 //  * cross-attention over the prefix-restricted memory M<=t: rows 0..t.
 //
-// Work is cut into units (slot, head, chunk of CH rows). A persistent grid of
-// (SMs x resident CTAs) walks the units round-robin. Each CTA runs one
-// producer warp and NC consumer warps over a STAGES-deep ring of
-// shared-memory tiles (KT rows of K and of V):
-//   producer: waits for a stage to be released ("empty" mbarrier), then
-//             fills it with two bulk asynchronous copies (cp.async.bulk)
-//             whose completion is counted in bytes on the "full" mbarrier;
-//   consumer warp w: takes tiles j = w, w + NC, ... of each unit, waits on
-//             their "full" barrier, folds them into its own online softmax
-//             (one rescale per group of keys), releases the stage.
-// No CTA-wide barrier sits in the stream; the consumer warps meet once per
-// unit (a named barrier) to merge their states in warp order. A unit of a
-// multi-chunk row writes its partial (acc, m, l); the last unit of that row
-// to finish merges the partials in chunk order. Every merge order depends only
-// on the row's own t, so results never depend on the batch around the row or
-// on which CTA ran which unit. Every wait is bounded in device time.
+// Work is cut into units (slot, head, chunk of CH rows); one warp owns a whole
+// unit. A persistent grid of (SMs x resident CTAs) runs, per CTA, one
+// producer warp and NC consumer warps; consumer warp w of CTA b takes units
+// b*NC + w, then every (grid * NC)-th unit after it. Each consumer warp has
+// its own ring of SW shared-memory stages; a stage holds a header (unit,
+// rows, first/last flags), the query (first tile of a unit) and KT rows of K
+// and of V. The producer lane walks the units of all its warps, and fills a
+// warp's free stage (its "empty" mbarrier completed) with the header written
+// by the producer and three bulk asynchronous copies (cp.async.bulk) whose
+// completion is counted in bytes on the stage's "full" mbarrier. Consumers
+// never read global memory before their result: they wait on "full", fold the
+// tile into an online softmax (base-2 exponent, one rescale per group of
+// keys), and hand the stage back. A unit of a multi-chunk row writes a
+// partial (acc, m, l); the last unit of that row to finish merges the
+// partials in chunk order. Every reduction order depends only on the row's
+// own t, so results never depend on the batch around the row or on which
+// warp ran which unit. Every wait is bounded in device time.
 //
 // Page key: [RLT-96] "RLT Runs 96 Blocks Per Token With Recurrent State, No
 // Resets" (aimastery.page).
@@ -36,8 +37,8 @@ namespace rlt {
 // Bounded device waits give up after this long and report RLT_ERR_TIMEOUT.
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
-constexpr int ATTN_NC = 4;      // consumer warps per CTA
-constexpr int ATTN_STAGES = 8;  // tiles in flight per CTA
+constexpr int ATTN_NC = 4;  // consumer warps per CTA
+constexpr int ATTN_SW = 3;  // stages per consumer warp
 
 template <typename T, int DH> struct AttnShape {
   static constexpr int KT = 4096 / (DH * (int)sizeof(T));  // rows per 4 KB tile
@@ -47,17 +48,24 @@ template <typename T, int DH> struct AttnShape {
   static constexpr int P = KT / KPP;         // passes per tile
   static constexpr int PG = P >= 4 ? 4 : P;  // passes per softmax rescale
   static_assert(KT % KPP == 0 && P % PG == 0, "tile rows split into passes and groups");
+  // stage: header (64 B), query (DH floats), K tile, V tile
+  static constexpr int HDR = 64;
+  static constexpr int QB = DH * 4;
+  static constexpr int TILE = KT * DH * (int)sizeof(T);
+  static constexpr int STAGE = HDR + QB + 2 * TILE;  // multiple of 16
 };
 
 template <typename T, int DH> constexpr int attn_smem_bytes() {
-  return ATTN_STAGES * 2 * AttnShape<T, DH>::KT * DH * (int)sizeof(T)  // tiles
-         + 2 * ATTN_STAGES * 8                                          // full, empty
-         + ATTN_NC * (DH + 2) * 4 + 16;                                 // merge scratch
+  return ATTN_NC * ATTN_SW * AttnShape<T, DH>::STAGE + 2 * ATTN_NC * ATTN_SW * 8 + 16;
 }
 
-struct AttnUnit {
-  int ih, c, r0, r1;  // (slot*H + head), chunk, rows [r0, r1)
-  const void *K;      // key block of this (slot, head)
+// Header the producer writes into a stage for its consumer.
+struct AttnHdr {
+  int ih;     // slot * H + head
+  int c;      // chunk
+  int rows;   // rows in this tile
+  int flags;  // 1: first tile of the unit, 2: last tile of the unit, 4: no more units
+  int nch;    // chunks of this row
 };
 
 // Geometry shared by every thread of the grid.
@@ -68,45 +76,31 @@ struct AttnGeom {
   long seq_stride, head_stride;
 };
 
-// Unit u -> its rows, or false if empty (slot past n, or chunk past the row's end).
-template <typename T>
-__device__ __forceinline__ bool attn_unit(const AttnGeom &g, int u, AttnUnit &out) {
-  const int pairs = g.units / g.xchunks;  // n_grid * H
-  const int c = u / pairs, ih = u % pairs;
-  const int i = ih / g.H, h = ih % g.H;
-  if (i >= g.n) return false;
-  const int t = __ldg(g.pos + i);
-  const int L = g.window > 0 ? min(t + 1, g.window) : t + 1;
-  if (c * g.CH >= L) return false;
-  out.ih = ih;
-  out.c = c;
-  out.r0 = c * g.CH;
-  out.r1 = min(L, out.r0 + g.CH);
-  const int seq = __ldg(g.ready + i);
-  out.K = static_cast<const T *>(g.base) + (size_t)seq * g.seq_stride + (size_t)h * g.head_stride;
-  return true;
-}
-
-// Cursor over the tiles of this CTA's units, in order.
-template <typename T, int KT> struct TileCursor {
-  int u;       // current unit index (grid-strided)
-  int j;       // tile within the unit
-  int ntiles;  // tiles of the current unit (0: exhausted)
-  AttnUnit cur;
-  __device__ void seek(const AttnGeom &g, int stride) {
-    while (u < g.units) {
-      if (attn_unit<T>(g, u, cur)) {
-        ntiles = (cur.r1 - cur.r0 + KT - 1) / KT;
-        j = 0;
-        return;
-      }
-      u += stride;
-    }
-    ntiles = 0;
+// Producer-side walk over one consumer warp's units and their tiles.
+template <typename T, int KT> struct UnitWalk {
+  int u, j, ntiles, nch, ih, c, r0, r1;
+  const T *K;
+  __device__ bool load(const AttnGeom &g) {
+    const int pairs = g.units / g.xchunks;  // n_grid * H
+    c = u / pairs;
+    ih = u % pairs;
+    const int i = ih / g.H, h = ih % g.H;
+    if (i >= g.n) return false;
+    const int t = __ldg(g.pos + i);
+    const int L = g.window > 0 ? min(t + 1, g.window) : t + 1;
+    nch = (L + g.CH - 1) / g.CH;
+    if (c >= nch) return false;
+    r0 = c * g.CH;
+    r1 = min(L, r0 + g.CH);
+    ntiles = (r1 - r0 + KT - 1) / KT;
+    j = 0;
+    const int seq = __ldg(g.ready + i);
+    K = static_cast<const T *>(g.base) + (size_t)seq * g.seq_stride + (size_t)h * g.head_stride;
+    return true;
   }
-  __device__ void start(const AttnGeom &g, int first, int stride) {
-    u = first;
-    seek(g, stride);
+  __device__ void seek(const AttnGeom &g, int stride) {
+    while (u < g.units && !load(g)) u += stride;
+    if (u >= g.units) ntiles = 0;
   }
   __device__ void next(const AttnGeom &g, int stride) {
     if (++j < ntiles) return;
@@ -120,10 +114,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Named barrier among the consumer warps only (the producer never joins).
-__device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, %0;\n" ::"n"(ATTN_NC * 32) : "memory");
+// 16 bytes of shared memory as float (bf16 pairs unpacked with integer ops).
+__device__ __forceinline__ void lds16_fast(const bf16 *p, float *f) {
+  uint4 v = *reinterpret_cast<const uint4 *>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
 }
+__device__ __forceinline__ void lds16_fast(const float *p, float *f) { lds16(p, f); }
 
 template <typename T, int DH>
 __global__ void __launch_bounds__((ATTN_NC + 1) * 32)
@@ -135,21 +136,19 @@ __global__ void __launch_bounds__((ATTN_NC + 1) * 32)
                   float scale, int *err) {
   using S = AttnShape<T, DH>;
   constexpr int KT = S::KT, VEC = S::VEC, LPK = S::LPK, KPP = S::KPP, P = S::P, PG = S::PG;
-  constexpr int STAGES = ATTN_STAGES, NC = ATTN_NC;
+  constexpr int NC = ATTN_NC, SW = ATTN_SW;
   extern __shared__ __align__(128) uint8_t smem[];
-  T *tiles = reinterpret_cast<T *>(smem);  // [STAGES][2][KT * DH]
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * 2 * KT * DH * sizeof(T));
-  uint64_t *empty = full + STAGES;
-  float *red = reinterpret_cast<float *>(empty + STAGES);  // [NC][DH + 2]
-  int *s_abort = reinterpret_cast<int *>(red + NC * (DH + 2));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + NC * SW * S::STAGE);
+  uint64_t *empty = full + NC * SW;
+  int *s_abort = reinterpret_cast<int *>(empty + NC * SW);
 
   const AttnGeom g{*n_dev, H, window, CH, xchunks, n_grid * H * xchunks, ready, pos, base,
                    seq_stride, head_stride};
-  const int stride = gridDim.x;
+  const int stride = gridDim.x * NC;  // consumer warps in the grid
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    for (int s = 0; s < STAGES; s++) {
+    for (int s = 0; s < NC * SW; s++) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -161,177 +160,181 @@ __global__ void __launch_bounds__((ATTN_NC + 1) * 32)
   if (warp == NC) {
     // ---------------------------------------------------------- producer
     if (lane != 0) return;
-    TileCursor<T, KT> pc{};
-    pc.start(g, blockIdx.x, stride);
-    int gidx = 0;
-    for (; !pc.done(); gidx++) {
-      const int s = gidx % STAGES;
-      if (gidx >= STAGES &&
-          !mbar_wait_bounded(&empty[s], (unsigned)((gidx / STAGES - 1) & 1), WAIT_LIMIT_NS)) {
+    UnitWalk<T, KT> wk[NC];
+    int issued[NC];
+    bool ended[NC];
+    int live = NC;  // warps not yet sent their end marker
+    for (int w = 0; w < NC; w++) {
+      wk[w].u = blockIdx.x * NC + w;
+      wk[w].seek(g, stride);
+      issued[w] = 0;
+      ended[w] = false;
+    }
+    uint64_t t0 = globaltimer_ns();
+    while (live > 0) {
+      bool progress = false;
+      for (int w = 0; w < NC; w++) {
+        if (ended[w]) continue;
+        const int k = issued[w], s = w * SW + k % SW;
+        if (k >= SW && !mbar_try_wait(&empty[s], (unsigned)((k / SW - 1) & 1))) continue;
+        UnitWalk<T, KT> &x = wk[w];
+        uint8_t *st = smem + (size_t)s * S::STAGE;
+        progress = true;
+        issued[w]++;
+        if (x.done()) {  // end marker: a header with no copies behind it
+          reinterpret_cast<AttnHdr *>(st)->flags = 4;
+          mbar_arrive(&full[s]);
+          ended[w] = true;
+          live--;
+          continue;
+        }
+        const int row0 = x.r0 + x.j * KT;
+        const int rows = min(KT, x.r1 - row0);
+        const bool first = x.j == 0;
+        AttnHdr *hd = reinterpret_cast<AttnHdr *>(st);
+        hd->ih = x.ih;
+        hd->c = x.c;
+        hd->rows = rows;
+        hd->flags = (first ? 1 : 0) | (x.j + 1 == x.ntiles ? 2 : 0);
+        hd->nch = x.nch;
+        const unsigned bytes = (unsigned)(rows * DH * (int)sizeof(T));
+        // the arrive below releases the header writes to the consumer
+        mbar_expect_tx(&full[s], 2 * bytes + (first ? S::QB : 0));
+        if (first) bulk_g2s(st + S::HDR, q + (size_t)x.ih * DH, S::QB, &full[s]);
+        bulk_g2s(st + S::HDR + S::QB, x.K + (size_t)row0 * DH, bytes, &full[s]);
+        bulk_g2s(st + S::HDR + S::QB + S::TILE, x.K + v_offset + (size_t)row0 * DH, bytes,
+                 &full[s]);
+        x.next(g, stride);
+      }
+      if (progress) {
+        t0 = globaltimer_ns();
+      } else if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
         atomicExch(s_abort, 1);
         set_error(err, DEV_ERR_TIMEOUT);
         break;
       }
-      if (*(volatile int *)s_abort) break;
-      const int row0 = pc.cur.r0 + pc.j * KT;
-      const unsigned bytes = (unsigned)(min(KT, pc.cur.r1 - row0) * DH * (int)sizeof(T));
-      const T *K = static_cast<const T *>(pc.cur.K);
-      T *kt = tiles + (size_t)s * 2 * KT * DH;
-      mbar_expect_tx(&full[s], 2 * bytes);
-      bulk_g2s(kt, K + (size_t)row0 * DH, bytes, &full[s]);
-      bulk_g2s(kt + KT * DH, K + v_offset + (size_t)row0 * DH, bytes, &full[s]);
-      pc.next(g, stride);
     }
     // let every copy this CTA issued land before the CTA may exit
-    for (int k = max(0, gidx - STAGES); k < gidx; k++)
-      mbar_wait_bounded(&full[k % STAGES], (unsigned)((k / STAGES) & 1), WAIT_LIMIT_NS);
+    for (int w = 0; w < NC; w++)
+      for (int k = max(0, issued[w] - SW); k < issued[w]; k++)
+        mbar_wait_bounded(&full[w * SW + k % SW], (unsigned)((k / SW) & 1), WAIT_LIMIT_NS);
     return;
   }
 
   // ------------------------------------------------------------ consumers
+  // q is stored pre-scaled by 1/sqrt(dh) * log2(e): scores are base-2 logits
+  const float qscale = scale * 1.4426950408889634f;
   const int sub = lane % LPK, grp = lane / LPK;
-  TileCursor<T, KT> cc{};
-  cc.start(g, blockIdx.x, stride);
   float qr[VEC];
   SoftAcc<VEC> st;
-  int gidx = 0;
-  bool aborted = false;
-  while (!cc.done()) {
-    if (cc.j == 0) {  // new unit: its query slice, fresh softmax state
-      const float *qp = q + (size_t)cc.cur.ih * DH + sub * VEC;
+  st.init();
+  for (int k = 0;; k++) {
+    const int s = warp * SW + k % SW;
+    uint8_t *stg = smem + (size_t)s * S::STAGE;
+    if (!mbar_wait_bounded(&full[s], (unsigned)((k / SW) & 1), WAIT_LIMIT_NS)) {
+      if (lane == 0) {  // the stream failed: nothing more will come
+        atomicExch(s_abort, 1);
+        set_error(err, DEV_ERR_TIMEOUT);
+      }
+      break;
+    }
+    const AttnHdr hd = *reinterpret_cast<const AttnHdr *>(stg);
+    if (hd.flags & 4) break;  // this warp's units are all done
+    const T *kt = reinterpret_cast<const T *>(stg + S::HDR + S::QB);
+    const T *vt = kt + KT * DH;
+    if (hd.flags & 1) {
+      const float *qs = reinterpret_cast<const float *>(stg + S::HDR);
 #pragma unroll
-      for (int v = 0; v < VEC; v++) qr[v] = __ldg(qp + v) * scale;
+      for (int v = 0; v < VEC; v++) qr[v] = qs[sub * VEC + v] * qscale;
       st.init();
     }
-    if (cc.j % NC == warp && !aborted) {
-      const int s = gidx % STAGES;
-      if (!mbar_wait_bounded(&full[s], (unsigned)((gidx / STAGES) & 1), WAIT_LIMIT_NS) ||
-          *(volatile int *)s_abort) {
-        aborted = true;
-        if (lane == 0) {
-          atomicExch(s_abort, 1);
-          set_error(err, DEV_ERR_TIMEOUT);
+#pragma unroll
+    for (int p0 = 0; p0 < P; p0 += PG) {
+      float sc[PG], vf[PG][VEC];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int p = 0; p < PG; p++) {
+        const int row = (p0 + p) * KPP + grp;
+        float kf[VEC];
+        if (row < hd.rows) {
+          lds16_fast(kt + row * DH + sub * VEC, kf);
+          lds16_fast(vt + row * DH + sub * VEC, vf[p]);
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; v++) kf[v] = vf[p][v] = 0.f;
         }
-      } else {
-        const int rows = min(KT, cc.cur.r1 - (cc.cur.r0 + cc.j * KT));
-        const T *kt = tiles + (size_t)s * 2 * KT * DH;
-        const T *vt = kt + KT * DH;
+        float d0 = 0.f;
 #pragma unroll
-        for (int p0 = 0; p0 < P; p0 += PG) {
-          float sc[PG], vf[PG][VEC];
-          float mt = -INFINITY;
+        for (int v = 0; v < VEC; v++) d0 = fmaf(qr[v], kf[v], d0);
 #pragma unroll
-          for (int p = 0; p < PG; p++) {
-            const int row = (p0 + p) * KPP + grp;
-            float kf[VEC];
-            if (row < rows) {
-              lds16(kt + row * DH + sub * VEC, kf);
-              lds16(vt + row * DH + sub * VEC, vf[p]);
-            } else {
+        for (int o = 1; o < LPK; o <<= 1) d0 += __shfl_xor_sync(FULL_MASK, d0, o);
+        sc[p] = row < hd.rows ? d0 : -INFINITY;
+        mt = fmaxf(mt, sc[p]);
+      }
+      if (mt != -INFINITY) {
+        const float mn = fmaxf(st.m, mt);
+        const float cr = exp2f(st.m - mn);  // st.m = -inf gives 0
+        st.l *= cr;
 #pragma unroll
-              for (int v = 0; v < VEC; v++) kf[v] = vf[p][v] = 0.f;
-            }
-            float d0 = 0.f;
+        for (int v = 0; v < VEC; v++) st.acc[v] *= cr;
 #pragma unroll
-            for (int v = 0; v < VEC; v++) d0 = fmaf(qr[v], kf[v], d0);
+        for (int p = 0; p < PG; p++) {
+          const float e = exp2f(sc[p] - mn);  // masked keys give 0
+          st.l += e;
 #pragma unroll
-            for (int o = 1; o < LPK; o <<= 1) d0 += __shfl_xor_sync(FULL_MASK, d0, o);
-            sc[p] = row < rows ? d0 : -INFINITY;
-            mt = fmaxf(mt, sc[p]);
-          }
-          if (mt != -INFINITY) {
-            const float mn = fmaxf(st.m, mt);
-            const float cr = expf(st.m - mn);  // st.m = -inf gives 0
-            st.l *= cr;
-#pragma unroll
-            for (int v = 0; v < VEC; v++) st.acc[v] *= cr;
-#pragma unroll
-            for (int p = 0; p < PG; p++) {
-              const float e = expf(sc[p] - mn);  // masked keys give 0
-              st.l += e;
-#pragma unroll
-              for (int v = 0; v < VEC; v++) st.acc[v] = fmaf(e, vf[p][v], st.acc[v]);
-            }
-            st.m = mn;
-          }
+          for (int v = 0; v < VEC; v++) st.acc[v] = fmaf(e, vf[p][v], st.acc[v]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // stage back to the producer
+        st.m = mn;
       }
     }
-    gidx++;
-    const bool last = (cc.j + 1 == cc.ntiles);
-    const AttnUnit unit = cc.cur;
-    cc.next(g, stride);
-    if (!last) continue;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);  // stage back to the producer
+    if (!(hd.flags & 2)) continue;
 
-    // ---- unit done: merge key groups, then the consumer warps in order
+    // ---- unit done: merge this warp's key groups (fixed xor order)
 #pragma unroll
-    for (int o = LPK; o < 32; o <<= 1) st.merge_xor(o);
-    float *rw = red + warp * (DH + 2);
+    for (int o = LPK; o < 32; o <<= 1) st.merge_xor2(o);
+    if (*(volatile int *)s_abort) break;
+    T *o_row = out + (size_t)hd.ih * DH;
+    if (hd.nch == 1) {
+      if (lane < LPK) {
+        const float inv = 1.f / st.l;
+#pragma unroll
+        for (int v = 0; v < VEC; v++) o_row[sub * VEC + v] = from_f<T>(st.acc[v] * inv);
+      }
+      continue;
+    }
+    float *pp = part + ((size_t)hd.ih * max_chunks + hd.c) * (DH + 2);
     if (lane < LPK) {
 #pragma unroll
-      for (int v = 0; v < VEC; v++) rw[sub * VEC + v] = st.acc[v];
+      for (int v = 0; v < VEC; v++) pp[sub * VEC + v] = st.acc[v];
     }
     if (lane == 0) {
-      rw[DH] = st.m;
-      rw[DH + 1] = st.l;
+      pp[DH] = st.m;
+      pp[DH + 1] = st.l;
     }
-    consumers_sync();
-    if (warp == 0 && !*(volatile int *)s_abort) {
-      const int t = __ldg(pos + unit.ih / H);
-      const int L = window > 0 ? min(t + 1, window) : t + 1;
-      const int nch = (L + CH - 1) / CH;
-      T *o_row = out + (size_t)unit.ih * DH;
-      float *pp = part + ((size_t)unit.ih * max_chunks + unit.c) * (DH + 2);
-      float mx = -INFINITY;
-      for (int w = 0; w < NC; w++) mx = fmaxf(mx, red[w * (DH + 2) + DH]);
-      float lsum = 0.f;
-      for (int w = 0; w < NC; w++) {
-        const float mw = red[w * (DH + 2) + DH];
-        lsum += (mw == -INFINITY ? 0.f : expf(mw - mx)) * red[w * (DH + 2) + DH + 1];
-      }
-      for (int dd = lane; dd < DH; dd += 32) {
-        float a = 0.f;
-        for (int w = 0; w < NC; w++) {
-          const float mw = red[w * (DH + 2) + DH];
-          a += (mw == -INFINITY ? 0.f : expf(mw - mx)) * red[w * (DH + 2) + dd];
-        }
-        if (nch == 1)
-          o_row[dd] = from_f<T>(a / lsum);
-        else
-          pp[dd] = a;
-      }
-      if (nch > 1) {
-        if (lane == 0) {
-          pp[DH] = mx;
-          pp[DH + 1] = lsum;
-        }
-        // the last chunk of this row to finish merges all chunks in order
-        __threadfence();
-        __syncwarp();
-        int last_in = 0;
-        if (lane == 0) last_in = (atomicAdd(&counters[unit.ih], 1) == nch - 1);
-        last_in = __shfl_sync(FULL_MASK, last_in, 0);
-        if (last_in) {
-          __threadfence();
-          const float *p0 = part + (size_t)unit.ih * max_chunks * (DH + 2);
-          float mx2 = -INFINITY;
-          for (int k = 0; k < nch; k++) mx2 = fmaxf(mx2, __ldcg(p0 + k * (DH + 2) + DH));
-          float l2 = 0.f;
-          for (int k = 0; k < nch; k++)
-            l2 += expf(__ldcg(p0 + k * (DH + 2) + DH) - mx2) * __ldcg(p0 + k * (DH + 2) + DH + 1);
-          for (int dd = lane; dd < DH; dd += 32) {
-            float a = 0.f;
-            for (int k = 0; k < nch; k++)
-              a += expf(__ldcg(p0 + k * (DH + 2) + DH) - mx2) * __ldcg(p0 + k * (DH + 2) + dd);
-            o_row[dd] = from_f<T>(a / l2);
-          }
-          if (lane == 0) counters[unit.ih] = 0;
-        }
-      }
+    // the last chunk of this row to finish merges all chunks in chunk order
+    __threadfence();
+    __syncwarp();
+    int last_in = 0;
+    if (lane == 0) last_in = (atomicAdd(&counters[hd.ih], 1) == hd.nch - 1);
+    last_in = __shfl_sync(FULL_MASK, last_in, 0);
+    if (!last_in) continue;
+    __threadfence();
+    const float *p0 = part + (size_t)hd.ih * max_chunks * (DH + 2);
+    float mx = -INFINITY;
+    for (int c = 0; c < hd.nch; c++) mx = fmaxf(mx, __ldcg(p0 + c * (DH + 2) + DH));
+    float lsum = 0.f;
+    for (int c = 0; c < hd.nch; c++)
+      lsum += exp2f(__ldcg(p0 + c * (DH + 2) + DH) - mx) * __ldcg(p0 + c * (DH + 2) + DH + 1);
+    const float inv = 1.f / lsum;
+    for (int dd = lane; dd < DH; dd += 32) {
+      float a = 0.f;
+      for (int c = 0; c < hd.nch; c++)
+        a += exp2f(__ldcg(p0 + c * (DH + 2) + DH) - mx) * __ldcg(p0 + c * (DH + 2) + dd);
+      o_row[dd] = from_f<T>(a * inv);
     }
-    consumers_sync();  // red is rewritten by the next unit
+    if (lane == 0) counters[hd.ih] = 0;
   }
 }
 

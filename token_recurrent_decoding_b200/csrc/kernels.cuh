@@ -144,6 +144,21 @@ template <int VEC> struct SoftAcc {
     }
     m = mn;
   }
+  // Same merge for states kept in base-2 logits (exp2 instead of exp).
+  __device__ void merge_xor2(int off) {
+    float m2 = __shfl_xor_sync(FULL_MASK, m, off);
+    float l2 = __shfl_xor_sync(FULL_MASK, l, off);
+    float mn = fmaxf(m, m2);
+    float c1 = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+    float c2 = (m2 == -INFINITY) ? 0.f : exp2f(m2 - mn);
+    l = l * c1 + l2 * c2;
+#pragma unroll
+    for (int v = 0; v < VEC; v++) {
+      float a2 = __shfl_xor_sync(FULL_MASK, acc[v], off);
+      acc[v] = acc[v] * c1 + a2 * c2;
+    }
+    m = mn;
+  }
 };
 
 // One warp attends one query over keys p in [p_lo, p_hi] whose rows sit at

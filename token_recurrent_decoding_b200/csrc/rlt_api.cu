@@ -28,7 +28,7 @@ using namespace rlt;
 
 namespace {
 
-constexpr int XCH = 512;  // memory positions per cross-attention split
+constexpr int XCH = 256;  // memory positions per cross-attention split
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
