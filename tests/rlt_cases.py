@@ -16,6 +16,9 @@ SMALL = {
                                       ffn_dim=512, vocab=512, window=16),
     "ragged_like": configs.RAGGED_MODEL.replace(d=128, n_heads=2, n_enc=1, n_dec=2,
                                                 ffn_dim=256, vocab=512, window=16),
+    # FFN width 1536: the down projection (K = 1536) runs split-K
+    "splitk_like": configs.M50.replace(d=128, n_heads=2, n_enc=1, n_dec=2, ffn_dim=1536,
+                                       vocab=512, window=8),
 }
 
 # Tolerances (north-star): step-wise max|err| / RMS(s), trajectory rel-L2 of s.

@@ -176,7 +176,7 @@ __global__ void __launch_bounds__((ATTN_NC + 1) * 32)
       for (int w = 0; w < NC; w++) {
         if (ended[w]) continue;
         const int k = issued[w], s = w * SW + k % SW;
-        if (k >= SW && !mbar_try_wait(&empty[s], (unsigned)((k / SW - 1) & 1))) continue;
+        if (k >= SW && !mbar_test_wait(&empty[s], (unsigned)((k / SW - 1) & 1))) continue;
         UnitWalk<T, KT> &x = wk[w];
         uint8_t *st = smem + (size_t)s * S::STAGE;
         progress = true;

@@ -133,6 +133,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of phase `parity` of `bar` (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for phase `parity` of `bar`, giving up after limit_ns of device time.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity,
                                                   uint64_t limit_ns) {

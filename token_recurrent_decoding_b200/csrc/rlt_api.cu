@@ -112,10 +112,10 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->counters = take(S * H * 4);
   {
     // split-K scratch: largest splits * N over the decoder GEMMs, per row
-    auto sn = [](size_t n, size_t k) { return (size_t)gemm_splits((int)k) * n; };
+    auto sn = [](size_t n, size_t k) { return (size_t)tc_splits((int)k) * n; };
     const size_t per_row = std::max({sn(d, 2 * d), sn(3 * d, d), sn(d, d), sn(F, d), sn(d, F)});
-    const size_t rows = (S + 63) / 64 * 64;
-    const size_t tiles = rows / 64 * ((std::max({3 * d, F, d}) + 63) / 64);
+    const size_t rows = (S + 127) / 128 * 128;  // row tiles of 128
+    const size_t tiles = rows / 128 * ((std::max({3 * d, F, d}) + 31) / 32);
     for (int ch = 0; ch < 2; ch++) {
       L->gpart[ch] = take(c->dtype == RLT_BF16 ? per_row * rows * 4 : 0);
       L->gcnt[ch] = take(tiles * 4);
@@ -261,14 +261,15 @@ const CUtensorMap *tmap_bf16(rlt_model *M, const void *ptr, uint64_t rows, uint6
   return &M->tmaps.emplace(key, m).first->second;
 }
 
-// tcgen05 GEMM of the encoder: A [a_rows][k] activations (only the first m
-// rows are used), B [n][k] weights.
-template <class Epi>
-cudaError_t gemm_tc(rlt_model *M, int m, int a_rows, int n, int k, const bf16 *A, const bf16 *B,
-                    Epi epi, cudaStream_t st) {
-  constexpr int BN = 128, STAGES = 3;
+// tcgen05 GEMM: rows [a_row0 + m, ...) of A [a_rows][k] (activations) times
+// B [n][k] (weights). m_grid bounds the rows (grid); Mdev, if set, gives the
+// rows at run time. The encoder's large row counts use 128-wide N tiles; the
+// decoder's small batches use 32/64-wide tiles (more CTAs stream the weights)
+// and split-K over large K into `ws`.
+template <int BN, int STAGES, class Epi>
+cudaError_t launch_tc(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
+                      int k, const bf16 *A, const bf16 *B, Epi epi, SplitK sk, cudaStream_t st) {
   constexpr int smem = TcSmem<BN, STAGES>::BYTES;
-  if (m <= 0) return cudaSuccess;
   const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
   const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
   if (!ma || !mb) return cudaErrorInvalidValue;
@@ -278,9 +279,24 @@ cudaError_t gemm_tc(rlt_model *M, int m, int a_rows, int n, int k, const bf16 *A
     RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     attr = true;
   }
-  dim3 grid((n + BN - 1) / BN, (m + TC_BM - 1) / TC_BM);
-  kern<<<grid, 128, smem, st>>>(*ma, *mb, m, n, k, epi, M->at<int>(M->L.err));
+  dim3 grid((n + BN - 1) / BN, (m_grid + TC_BM - 1) / TC_BM, sk.splits);
+  kern<<<grid, 128, smem, st>>>(*ma, *mb, m_grid, Mdev, a_row0, n, k, epi, sk,
+                                M->at<int>(M->L.err));
   return cudaGetLastError();
+}
+
+template <class Epi>
+cudaError_t gemm_tc(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
+                    int k, const bf16 *A, const bf16 *B, Epi epi, const SplitK *ws,
+                    cudaStream_t st) {
+  if (m_grid <= 0) return cudaSuccess;
+  SplitK one{1, nullptr, nullptr};
+  if (m_grid >= 1024)
+    return launch_tc<128, 3>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, one, st);
+  SplitK sk = one;
+  if (ws && ws->part && tc_splits(k) > 1) sk = {tc_splits(k), ws->part, ws->counters};
+  if (n >= 2048) return launch_tc<64, 4>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, sk, st);
+  return launch_tc<32, 4>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, sk, st);
 }
 
 cudaEvent_t take_event(rlt_model *M) {
@@ -338,7 +354,7 @@ cudaError_t gemm_enc(rlt_model *M, int m, int n, int k, const T *A, const T *B, 
   Span sp(M, st, RLT_K_ENC, (double)n * k * es + (double)m * k * es + (double)m * n * 4.0,
           2.0 * m * n * k);
   if constexpr (std::is_same<T, bf16>::value)
-    return gemm_tc(M, m, M->L.ptok, n, k, A, B, epi, st);
+    return gemm_tc(M, m, nullptr, M->L.ptok, 0, n, k, A, B, epi, nullptr, st);
   else
     return gemm(m, nullptr, n, k, A, k, B, k, epi, st);
 }
@@ -411,8 +427,10 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   float *s32 = M->at<float>(L.s32) + r0 * d, *qkv = M->at<float>(L.qkv) + r0 * 3 * d;
   float *q = M->at<float>(L.q) + r0 * d, *fa = M->at<float>(L.fa) + r0 * F;
   float *s = M->at<float>(L.s);
-  T *xin = M->at<T>(L.xin) + r0 * 2 * d, *a = M->at<T>(L.a) + r0 * d, *u = M->at<T>(L.u) + r0 * d;
-  T *f = M->at<T>(L.f) + r0 * F;
+  // activation buffers: whole-buffer bases (GEMM operands, addressed by row
+  // offset r0) and this chain's rows (written by the other kernels)
+  T *xin_b = M->at<T>(L.xin), *a_b = M->at<T>(L.a), *u_b = M->at<T>(L.u), *f_b = M->at<T>(L.f);
+  T *xin = xin_b + r0 * 2 * d, *a = a_b + r0 * d, *u = u_b + r0 * d, *f = f_b + r0 * F;
   T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem);
   const float2 *rope = M->at<float2>(L.rope);
   const bool a0 = c.alpha == 0.0f;
@@ -421,11 +439,14 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   const int rows_blocks = blocks_for((long)n * 32, 256);
   const double nr = si.n;  // real rows, for the algorithmic byte counts
   const double row_bytes = nr * d * (4 + es);
-  auto G = [&](int kind, int m, int nn, int k, const T *A, int lda, const T *B, int ldb,
-               auto epi) {
+  // y = A_rows(r0..) W^T with A one of the whole activation buffers above
+  auto G = [&](int kind, int nn, int k, const T *A_base, const T *B, auto epi) {
     Span sp(M, st, kind, (double)nn * k * es + nr * k * es + nr * nn * 4.0, 2.0 * nr * nn * k);
     const SplitK sk{0, M->at<float>(L.gpart[si.chain]), M->at<int>(L.gcnt[si.chain])};
-    return gemm(m, nd, nn, k, A, lda, B, ldb, epi, st, &sk);
+    if constexpr (std::is_same<T, bf16>::value)
+      return gemm_tc(M, n, nd, c.max_seqs, (int)r0, nn, k, A_base, B, epi, &sk, st);
+    else
+      return gemm(n, nd, nn, k, A_base + r0 * k, k, B, k, epi, st);
   };
 
   {
@@ -435,7 +456,7 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   }
   RLT_TRY(cudaGetLastError());
   if (!a0)
-    RLT_TRY(G(RLT_K_GEMM, n, d, 2 * d, xin, 2 * d, (const T *)M->w.gate_w, 2 * d,
+    RLT_TRY(G(RLT_K_GEMM, d, 2 * d, xin_b, (const T *)M->w.gate_w,
               EpiGate{e32, s32, (const float *)M->w.gate_b, c.alpha, h, d}));
   for (int l = 0; l < c.n_dec_layers; l++) {
     T *ring_l = ring + (size_t)l * ring_layer;
@@ -446,7 +467,7 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
       k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln1[l], eps,
                                                 u);
     }
-    RLT_TRY(G(RLT_K_GEMM, n, 3 * d, d, u, d, W_<T>::qkv(M, l), d, EpiStoreF32{qkv, 3 * d}));
+    RLT_TRY(G(RLT_K_GEMM, 3 * d, d, u_b, W_<T>::qkv(M, l), EpiStoreF32{qkv, 3 * d}));
     {
       Span sp(M, st, RLT_K_OTHER, nr * 3 * d * 4 + nr * d * (4 + 2 * es));
       k_dec_qkv_post<T><<<blocks_for((long)n * H * (DH / 2), 256), 256, 0, st>>>(
@@ -458,20 +479,20 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
       RLT_TRY((launch_attn<T, DH>(M, si, W, 1, ring_l, (long)H * 2 * W * DH, 2L * W * DH,
                                   (long)W * DH, a, st)));
     }
-    RLT_TRY(G(RLT_K_GEMM, n, d, d, a, d, W_<T>::o(M, l), d, EpiResid{h, d}));
+    RLT_TRY(G(RLT_K_GEMM, d, d, a_b, W_<T>::o(M, l), EpiResid{h, d}));
     // cross-attention sublayer over M<=t
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
       k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln2[l], eps,
                                                 u);
     }
-    RLT_TRY(G(RLT_K_GEMM, n, d, d, u, d, (const T *)M->w.dec_wqx[l], d, EpiStoreF32{q, d}));
+    RLT_TRY(G(RLT_K_GEMM, d, d, u_b, (const T *)M->w.dec_wqx[l], EpiStoreF32{q, d}));
     {
       Span sp(M, st, RLT_K_XATTN, si.sum_keys * 2.0 * d * es, 4.0 * d * si.sum_keys);
       RLT_TRY((launch_attn<T, DH>(M, si, 0, si.xchunks, mem_g, (long)H * 2 * c.max_len * DH,
                                   2L * c.max_len * DH, (long)c.max_len * DH, a, st)));
     }
-    RLT_TRY(G(RLT_K_GEMM, n, d, d, a, d, (const T *)M->w.dec_wox[l], d, EpiResid{h, d}));
+    RLT_TRY(G(RLT_K_GEMM, d, d, a_b, (const T *)M->w.dec_wox[l], EpiResid{h, d}));
     // FFN sublayer
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
@@ -479,12 +500,12 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
                                                 u);
     }
     if (c.ffn_kind == RLT_GELU) {
-      RLT_TRY(G(RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiGelu<T>{f, F}));
+      RLT_TRY(G(RLT_K_GEMM, F, d, u_b, W_<T>::w1(M, l), EpiGelu<T>{f, F}));
     } else {
-      RLT_TRY(G(RLT_K_GEMM, n, F, d, u, d, W_<T>::w1(M, l), d, EpiStoreF32{fa, F}));
-      RLT_TRY(G(RLT_K_GEMM, n, F, d, u, d, W_<T>::wb(M, l), d, EpiSwiglu<T>{fa, f, F}));
+      RLT_TRY(G(RLT_K_GEMM, F, d, u_b, W_<T>::w1(M, l), EpiStoreF32{fa, F}));
+      RLT_TRY(G(RLT_K_GEMM, F, d, u_b, W_<T>::wb(M, l), EpiSwiglu<T>{fa, f, F}));
     }
-    RLT_TRY(G(RLT_K_GEMM, n, d, F, f, F, W_<T>::w2(M, l), F, EpiResid{h, d}));
+    RLT_TRY(G(RLT_K_GEMM, d, F, f_b, W_<T>::w2(M, l), EpiResid{h, d}));
   }
   {
     Span sp(M, st, RLT_K_OTHER, nr * d * 8);
