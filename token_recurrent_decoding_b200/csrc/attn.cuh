@@ -37,11 +37,18 @@ namespace rlt {
 // Bounded device waits give up after this long and report RLT_ERR_TIMEOUT.
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
-constexpr int ATTN_NC = 4;  // consumer warps per CTA
-constexpr int ATTN_SW = 3;  // stages per consumer warp
+// Batches up to this many rows keep their positions and slot ids in shared
+// memory for the unit walk.
+constexpr int ATTN_SMEM_ROWS = 1024;
 
-template <typename T, int DH> struct AttnShape {
-  static constexpr int KT = 4096 / (DH * (int)sizeof(T));  // rows per 4 KB tile
+// Launch shape of the decode attention: consumer warps per CTA, stages per
+// consumer warp, bytes of one K (or V) tile.
+struct AttnCfg {
+  static constexpr int NC = 4, SW = 3, TILE_BYTES = 4096;
+};
+
+template <typename T, int DH, int TILE_BYTES = AttnCfg::TILE_BYTES> struct AttnShape {
+  static constexpr int KT = TILE_BYTES / (DH * (int)sizeof(T));  // rows per tile
   static constexpr int VEC = V16<T>::N;
   static constexpr int LPK = DH / VEC;       // lanes per key
   static constexpr int KPP = 32 / LPK;       // keys per warp pass
@@ -55,8 +62,10 @@ template <typename T, int DH> struct AttnShape {
   static constexpr int STAGE = HDR + QB + 2 * TILE;  // multiple of 16
 };
 
-template <typename T, int DH> constexpr int attn_smem_bytes() {
-  return ATTN_NC * ATTN_SW * AttnShape<T, DH>::STAGE + 2 * ATTN_NC * ATTN_SW * 8 + 16;
+template <typename T, int DH, int NC = AttnCfg::NC, int SW = AttnCfg::SW,
+          int TB = AttnCfg::TILE_BYTES>
+constexpr int attn_smem_bytes() {
+  return NC * SW * AttnShape<T, DH, TB>::STAGE + 2 * NC * SW * 8 + 16 + 2 * ATTN_SMEM_ROWS * 4;
 }
 
 // Header the producer writes into a stage for its consumer.
@@ -68,7 +77,9 @@ struct AttnHdr {
   int nch;    // chunks of this row
 };
 
-// Geometry shared by every thread of the grid.
+// Geometry shared by every thread of the grid. pos / ready point at the
+// CTA's shared-memory copies when the batch fits (ATTN_SMEM_ROWS), else at
+// global memory.
 struct AttnGeom {
   int n, H, window, CH, xchunks, units;
   const int *ready, *pos;
@@ -86,7 +97,7 @@ template <typename T, int KT> struct UnitWalk {
     ih = u % pairs;
     const int i = ih / g.H, h = ih % g.H;
     if (i >= g.n) return false;
-    const int t = __ldg(g.pos + i);
+    const int t = g.pos[i];
     const int L = g.window > 0 ? min(t + 1, g.window) : t + 1;
     nch = (L + g.CH - 1) / g.CH;
     if (c >= nch) return false;
@@ -94,7 +105,7 @@ template <typename T, int KT> struct UnitWalk {
     r1 = min(L, r0 + g.CH);
     ntiles = (r1 - r0 + KT - 1) / KT;
     j = 0;
-    const int seq = __ldg(g.ready + i);
+    const int seq = g.ready[i];
     K = static_cast<const T *>(g.base) + (size_t)seq * g.seq_stride + (size_t)h * g.head_stride;
     return true;
   }
@@ -126,24 +137,35 @@ __device__ __forceinline__ void lds16_fast(const bf16 *p, float *f) {
 }
 __device__ __forceinline__ void lds16_fast(const float *p, float *f) { lds16(p, f); }
 
-template <typename T, int DH>
-__global__ void __launch_bounds__((ATTN_NC + 1) * 32)
+template <typename T, int DH, int NC = AttnCfg::NC, int SW = AttnCfg::SW,
+          int TB = AttnCfg::TILE_BYTES>
+__global__ void __launch_bounds__((NC + 1) * 32)
     k_attn_decode(const int *__restrict__ n_dev, int H, int window, int CH, int xchunks,
                   int max_chunks, int n_grid, const int *__restrict__ ready,
                   const int *__restrict__ pos, const float *__restrict__ q,
                   const T *__restrict__ base, long seq_stride, long head_stride, long v_offset,
                   float *__restrict__ part, int *__restrict__ counters, T *__restrict__ out,
                   float scale, int *err) {
-  using S = AttnShape<T, DH>;
+  using S = AttnShape<T, DH, TB>;
   constexpr int KT = S::KT, VEC = S::VEC, LPK = S::LPK, KPP = S::KPP, P = S::P, PG = S::PG;
-  constexpr int NC = ATTN_NC, SW = ATTN_SW;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + NC * SW * S::STAGE);
   uint64_t *empty = full + NC * SW;
   int *s_abort = reinterpret_cast<int *>(empty + NC * SW);
+  int *s_pos = s_abort + 4, *s_ready = s_pos + ATTN_SMEM_ROWS;
 
-  const AttnGeom g{*n_dev, H, window, CH, xchunks, n_grid * H * xchunks, ready, pos, base,
-                   seq_stride, head_stride};
+  pdl_trigger();
+  pdl_wait();  // q, the ring slot of t and the positions come from earlier kernels
+  const int n = *n_dev;
+  const bool cached = n <= ATTN_SMEM_ROWS;
+  if (cached) {  // the unit walk reads positions and slots from shared memory
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      s_pos[i] = pos[i];
+      s_ready[i] = ready[i];
+    }
+  }
+  const AttnGeom g{n, H, window, CH, xchunks, n_grid * H * xchunks, cached ? s_ready : ready,
+                   cached ? s_pos : pos, base, seq_stride, head_stride};
   const int stride = gridDim.x * NC;  // consumer warps in the grid
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -339,16 +361,18 @@ __global__ void __launch_bounds__((ATTN_NC + 1) * 32)
 }
 
 // Resident CTAs of a persistent attention launch (SMs x occupancy), cached.
-template <typename T, int DH> int attn_grid_ctas() {
+template <typename T, int DH, int NC = AttnCfg::NC, int SW = AttnCfg::SW,
+          int TB = AttnCfg::TILE_BYTES>
+int attn_grid_ctas() {
   static int ctas = 0;
   if (!ctas) {
     int dev = 0, sms = 0, occ = 0;
-    constexpr int smem = attn_smem_bytes<T, DH>();
+    constexpr int smem = attn_smem_bytes<T, DH, NC, SW, TB>();
+    auto kern = k_attn_decode<T, DH, NC, SW, TB>;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaFuncSetAttribute(k_attn_decode<T, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_attn_decode<T, DH>,
-                                                  (ATTN_NC + 1) * 32, smem);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, (NC + 1) * 32, smem);
     ctas = (sms > 0 ? sms : 148) * (occ > 0 ? occ : 1);
   }
   return ctas;

@@ -88,6 +88,16 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Under programmatic stream serialisation a kernel may start while its
+// predecessor finishes: pdl_wait() blocks until every prerequisite grid has
+// completed and its writes are visible; pdl_trigger() lets the successor
+// launch. Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // ------------------------------------------------- bulk async copies + mbarrier
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

@@ -169,11 +169,22 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  pdl_trigger();
   if (warp == 0 && lane == 0) {
-    // producer: TMA into the ring
-    for (int kb = 0; kb < KB; kb++) {
+    // producer: TMA into the ring. The weight tiles of the first stages do
+    // not depend on the previous kernel, so they stream before the wait.
+    const int pre = KB < STAGES ? KB : STAGES;
+    for (int kb = 0; kb < pre; kb++) {
+      uint8_t *b = tsm + kb * SM::STAGE + SM::A_BYTES;
+      mbar_expect_tx(&full[kb], SM::STAGE);
+      tma_load_2d(b, &tmB, (kb0 + kb) * TC_BK, n0, &full[kb]);
+    }
+    pdl_wait();
+    for (int kb = 0; kb < pre; kb++)
+      tma_load_2d(tsm + kb * SM::STAGE, &tmA, (kb0 + kb) * TC_BK, a_row0 + m0, &full[kb]);
+    for (int kb = pre; kb < KB; kb++) {
       const int s = kb % STAGES, u = kb / STAGES;
-      if (u > 0 && !mbar_wait_bounded(&empty[s], (u - 1) & 1, WAIT_LIMIT_NS_TC)) {
+      if (!mbar_wait_bounded(&empty[s], (u - 1) & 1, WAIT_LIMIT_NS_TC)) {
         atomicExch(&s_fail, 1);
         break;
       }
@@ -207,6 +218,7 @@ __global__ void __launch_bounds__(128, 1)
     umma_commit(accum);
   }
   __syncwarp();
+  pdl_wait();  // the epilogue reads and writes buffers of earlier kernels
   // epilogue: wait for the accumulator, read this warp's 32 rows
   const bool acc_ok = mbar_wait_bounded(accum, 0, WAIT_LIMIT_NS_TC);
   tc_fence_after();

@@ -30,6 +30,8 @@ template <typename T>
 __global__ void k_rmsnorm(int rows, const int *__restrict__ rows_dev, int d,
                           const float *__restrict__ x, const float *__restrict__ gamma, float eps,
                           T *__restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (rows_dev) rows = *rows_dev;
   if (r >= rows) return;
@@ -62,6 +64,8 @@ __global__ void k_step_gather(const int *__restrict__ n_dev, int d, int max_len,
                               const T *__restrict__ e, const float *__restrict__ s,
                               T *__restrict__ xin, float *__restrict__ e32,
                               float *__restrict__ s32, float *__restrict__ h, int alpha_zero) {
+  pdl_wait();
+  pdl_trigger();
   int i = blockIdx.x;
   if (i >= *n_dev) return;
   int seq = ready[i];
@@ -89,6 +93,8 @@ __global__ void k_dec_qkv_post(const int *__restrict__ n_dev, int H, int dh, int
                                const int *__restrict__ ready, const int *__restrict__ pos,
                                const float *__restrict__ qkv, const float2 *__restrict__ rope,
                                float *__restrict__ q_out, T *__restrict__ ring_l) {
+  pdl_wait();
+  pdl_trigger();
   int half = dh / 2, d = H * dh;
   long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long)(*n_dev) * H * half) return;
@@ -203,6 +209,8 @@ __device__ __forceinline__ void warp_attend(const float *qr, const T *__restrict
 __global__ void k_step_final(const int *__restrict__ n_dev, int d, const int *__restrict__ ready,
                              int *__restrict__ t_dec, const float *__restrict__ h,
                              const float *__restrict__ gamma, float eps, float *__restrict__ s) {
+  pdl_wait();
+  pdl_trigger();
   int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (i >= *n_dev) return;
   int seq = ready[i];

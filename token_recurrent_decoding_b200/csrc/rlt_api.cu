@@ -218,6 +218,29 @@ namespace {
 
 inline int blocks_for(long threads, int bs) { return (int)((threads + bs - 1) / bs); }
 
+// Launch a step kernel; on a non-legacy stream with programmatic stream
+// serialisation, so it starts while its predecessor drains (the kernel calls
+// pdl_wait() before reading what the predecessor wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args... args) {
+  if (st == nullptr) {
+    kern<<<grid, block, smem, st>>>(args...);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -280,9 +303,8 @@ cudaError_t launch_tc(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int
     attr = true;
   }
   dim3 grid((n + BN - 1) / BN, (m_grid + TC_BM - 1) / TC_BM, sk.splits);
-  kern<<<grid, 128, smem, st>>>(*ma, *mb, m_grid, Mdev, a_row0, n, k, epi, sk,
-                                M->at<int>(M->L.err));
-  return cudaGetLastError();
+  return launch_k(kern, grid, dim3(128), smem, st, *ma, *mb, m_grid, Mdev, a_row0, n, k, epi, sk,
+                  M->at<int>(M->L.err));
 }
 
 template <class Epi>
@@ -403,12 +425,13 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
   const size_t r0 = si.row0, H = c.n_heads;
   const int units = si.n_grid * c.n_heads * xchunks;
   const int grid = std::min(units, attn_grid_ctas<T, DH>());  // also sets the smem limit
-  k_attn_decode<T, DH><<<grid, (ATTN_NC + 1) * 32, smem, st>>>(
-      M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks, si.n_grid,
-      M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0, M->at<float>(L.q) + r0 * c.d, base,
-      seq_stride, head_stride, v_offset, M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
-      M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH), M->at<int>(L.err));
-  return cudaGetLastError();
+  return launch_k(k_attn_decode<T, DH>, dim3(grid), dim3((AttnCfg::NC + 1) * 32), smem, st,
+                  M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks,
+                  si.n_grid, M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0,
+                  M->at<float>(L.q) + r0 * c.d, base, seq_stride, head_stride, v_offset,
+                  M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
+                  M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH),
+                  M->at<int>(L.err));
 }
 
 template <typename T, int DH>
@@ -451,10 +474,9 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
 
   {
     Span sp(M, st, RLT_K_OTHER, nr * d * (es + 4) + row_bytes);
-    k_step_gather<T><<<n, 256, 0, st>>>(nd, d, c.max_len, ready, t_dec, pos, M->at<T>(L.e), s,
-                                        xin, e32, s32, h, a0);
+    RLT_TRY(launch_k(k_step_gather<T>, dim3(n), dim3(256), 0, st, nd, d, c.max_len, ready, t_dec,
+                     pos, M->at<T>(L.e), s, xin, e32, s32, h, (int)a0));
   }
-  RLT_TRY(cudaGetLastError());
   if (!a0)
     RLT_TRY(G(RLT_K_GEMM, d, 2 * d, xin_b, (const T *)M->w.gate_w,
               EpiGate{e32, s32, (const float *)M->w.gate_b, c.alpha, h, d}));
@@ -464,14 +486,14 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
     // sliding-window self-attention sublayer
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln1[l], eps,
-                                                u);
+      RLT_TRY(launch_k(k_rmsnorm<T>, dim3(rows_blocks), dim3(256), 0, st, n, nd, d, h,
+                       (const float *)M->w.dec_ln1[l], eps, u));
     }
     RLT_TRY(G(RLT_K_GEMM, 3 * d, d, u_b, W_<T>::qkv(M, l), EpiStoreF32{qkv, 3 * d}));
     {
       Span sp(M, st, RLT_K_OTHER, nr * 3 * d * 4 + nr * d * (4 + 2 * es));
-      k_dec_qkv_post<T><<<blocks_for((long)n * H * (DH / 2), 256), 256, 0, st>>>(
-          nd, H, DH, W, ready, pos, qkv, rope, q, ring_l);
+      RLT_TRY(launch_k(k_dec_qkv_post<T>, dim3(blocks_for((long)n * H * (DH / 2), 256)),
+                       dim3(256), 0, st, nd, H, DH, W, ready, pos, qkv, rope, q, ring_l));
     }
     {
       Span sp(M, st, RLT_K_SWA, si.sum_win * 2.0 * d * es + nr * d * (4 + es),
@@ -483,8 +505,8 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
     // cross-attention sublayer over M<=t
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln2[l], eps,
-                                                u);
+      RLT_TRY(launch_k(k_rmsnorm<T>, dim3(rows_blocks), dim3(256), 0, st, n, nd, d, h,
+                       (const float *)M->w.dec_ln2[l], eps, u));
     }
     RLT_TRY(G(RLT_K_GEMM, d, d, u_b, (const T *)M->w.dec_wqx[l], EpiStoreF32{q, d}));
     {
@@ -496,8 +518,8 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
     // FFN sublayer
     {
       Span sp(M, st, RLT_K_OTHER, row_bytes);
-      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(n, nd, d, h, (const float *)M->w.dec_ln3[l], eps,
-                                                u);
+      RLT_TRY(launch_k(k_rmsnorm<T>, dim3(rows_blocks), dim3(256), 0, st, n, nd, d, h,
+                       (const float *)M->w.dec_ln3[l], eps, u));
     }
     if (c.ffn_kind == RLT_GELU) {
       RLT_TRY(G(RLT_K_GEMM, F, d, u_b, W_<T>::w1(M, l), EpiGelu<T>{f, F}));
@@ -509,8 +531,8 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   }
   {
     Span sp(M, st, RLT_K_OTHER, nr * d * 8);
-    k_step_final<<<rows_blocks, 256, 0, st>>>(nd, d, ready, t_dec, h,
-                                              (const float *)M->w.dec_lnf, eps, s);
+    RLT_TRY(launch_k(k_step_final, dim3(rows_blocks), dim3(256), 0, st, nd, d, ready, t_dec, h,
+                     (const float *)M->w.dec_lnf, eps, s));
   }
   return cudaGetLastError();
 }
@@ -901,7 +923,7 @@ cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengt
   RLT_TRY(cudaGetLastError());
   const int xchunks = (lmax + XCH - 1) / XCH, max_chunks = (cap + XCH - 1) / XCH;
   const int grid = std::min(n * H * xchunks, ctas);
-  k_attn_decode<T, DH><<<grid, (ATTN_NC + 1) * 32, smem, st>>>(
+  k_attn_decode<T, DH><<<grid, (AttnCfg::NC + 1) * 32, smem, st>>>(
       reinterpret_cast<int *>(ws + w.err) + 1, H, 0, XCH, xchunks, max_chunks, n,
       reinterpret_cast<int *>(ws + w.ready), reinterpret_cast<int *>(ws + w.pos), q,
       static_cast<const T *>(kv), (long)H * 2 * cap * DH, 2L * cap * DH, (long)cap * DH,
