@@ -68,6 +68,13 @@ constexpr int attn_smem_bytes() {
   return NC * SW * AttnShape<T, DH, TB>::STAGE + 2 * NC * SW * 8 + 16 + 2 * ATTN_SMEM_ROWS * 4;
 }
 
+// Up to six byte ranges (e.g. the weights of the GEMMs that follow) that the
+// idle lanes of the producer warps pull into L2 while the attention streams.
+struct L2Prefetch {
+  const char *p[6];
+  unsigned long long n[6];
+};
+
 // Header the producer writes into a stage for its consumer.
 struct AttnHdr {
   int ih;     // slot * H + head
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
                   const int *__restrict__ pos, const float *__restrict__ q,
                   const T *__restrict__ base, long seq_stride, long head_stride, long v_offset,
                   float *__restrict__ part, int *__restrict__ counters, T *__restrict__ out,
-                  float scale, int *err) {
+                  float scale, int *err, L2Prefetch pf) {
   using S = AttnShape<T, DH, TB>;
   constexpr int KT = S::KT, VEC = S::VEC, LPK = S::LPK, KPP = S::KPP, P = S::P, PG = S::PG;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -181,7 +188,25 @@ __global__ void __launch_bounds__((NC + 1) * 32)
 
   if (warp == NC) {
     // ---------------------------------------------------------- producer
-    if (lane != 0) return;
+    if (lane != 0) {
+      // lanes 1..31 of every producer warp share the L2 prefetch, 64 KB pieces
+      constexpr unsigned PIECE = 64u << 10;
+      const long worker = (long)blockIdx.x * 31 + (lane - 1), workers = (long)gridDim.x * 31;
+      long base_piece = 0;
+      for (int r = 0; r < 6; r++) {
+        if (!pf.p[r] || !pf.n[r]) continue;
+        const long pieces = (long)((pf.n[r] + PIECE - 1) / PIECE);
+        for (long c = ((worker - base_piece) % workers + workers) % workers; c < pieces;
+             c += workers) {
+          const unsigned long long off = (unsigned long long)c * PIECE;
+          const unsigned long long len = pf.n[r] - off < PIECE ? pf.n[r] - off : PIECE;
+          bulk_prefetch_l2(pf.p[r] + off, (unsigned)len);
+        }
+        base_piece += pieces;
+      }
+      return;
+    }
+    const uint64_t kv_policy = l2_evict_first_policy();
     UnitWalk<T, KT> wk[NC];
     int issued[NC];
     bool ended[NC];
@@ -223,9 +248,9 @@ __global__ void __launch_bounds__((NC + 1) * 32)
         // the arrive below releases the header writes to the consumer
         mbar_expect_tx(&full[s], 2 * bytes + (first ? S::QB : 0));
         if (first) bulk_g2s(st + S::HDR, q + (size_t)x.ih * DH, S::QB, &full[s]);
-        bulk_g2s(st + S::HDR + S::QB, x.K + (size_t)row0 * DH, bytes, &full[s]);
-        bulk_g2s(st + S::HDR + S::QB + S::TILE, x.K + v_offset + (size_t)row0 * DH, bytes,
-                 &full[s]);
+        bulk_g2s_hint(st + S::HDR + S::QB, x.K + (size_t)row0 * DH, bytes, &full[s], kv_policy);
+        bulk_g2s_hint(st + S::HDR + S::QB + S::TILE, x.K + v_offset + (size_t)row0 * DH, bytes,
+                      &full[s], kv_policy);
         x.next(g, stride);
       }
       if (progress) {
@@ -376,6 +401,18 @@ int attn_grid_ctas() {
     ctas = (sms > 0 ? sms : 148) * (occ > 0 ? occ : 1);
   }
   return ctas;
+}
+
+// CTAs for `units` units: as few consumer warps as give every warp the same
+// number of units (k = ceil(units / resident warps)), so no warp runs a tail
+// of one extra unit while the others idle.
+template <typename T, int DH, int NC = AttnCfg::NC, int SW = AttnCfg::SW,
+          int TB = AttnCfg::TILE_BYTES>
+int attn_balanced_ctas(int units) {
+  const int max_warps = attn_grid_ctas<T, DH, NC, SW, TB>() * NC;
+  const int k = (units + max_warps - 1) / max_warps;
+  const int warps = (units + k - 1) / k;
+  return (warps + NC - 1) / NC;
 }
 
 }  // namespace rlt
