@@ -44,7 +44,7 @@ constexpr int ATTN_SMEM_ROWS = 1024;
 // Launch shape of the decode attention: consumer warps per CTA, stages per
 // consumer warp, bytes of one K (or V) tile.
 struct AttnCfg {
-  static constexpr int NC = 4, SW = 3, TILE_BYTES = 4096;
+  static constexpr int NC = 4, SW = 2, TILE_BYTES = 4096;
 };
 
 template <typename T, int DH, int TILE_BYTES = AttnCfg::TILE_BYTES> struct AttnShape {
