@@ -78,14 +78,6 @@ template <typename T> struct EpiMem {
   }
 };
 
-// Split-K scratch of one GEMM call: `splits` partial tiles [split][M][N] in
-// fp32 and one arrival counter per output tile (zero between calls).
-struct SplitK {
-  int splits;
-  float *part;
-  int *counters;
-};
-
 // --------------------------------------------------------------- fp32 SIMT GEMM
 // 64x64 output tile, 256 threads, 4x4 outputs per thread, K in steps of 16.
 template <class Epi>
@@ -136,7 +128,7 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------ launcher
 template <class Epi>
 cudaError_t gemm(int M, const int *Mdev, int N, int K, const float *A, int lda, const float *B,
-                 int ldb, Epi epi, cudaStream_t st, const SplitK * = nullptr) {
+                 int ldb, Epi epi, cudaStream_t st) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + 63) / 64, (M + 63) / 64);
   k_gemm_f32<Epi><<<grid, 256, 0, st>>>(M, Mdev, N, K, A, lda, B, ldb, epi);

@@ -1,0 +1,441 @@
+// Decoder-step projections on the tcgen05 tensor cores, for the small row
+// counts of one decode step (at most a few hundred rows):
+//   C[m][n] = sum_k A[m][k] * B[n][k],  A = activations [rows][K] (bf16),
+//   B = weights [N][K] (bf16), fp32 accumulation in tensor memory.
+//
+// A decode-step GEMM is latency-bound: the weights are read once and the
+// FLOPs are few, so the design goal is to touch every SM with little data
+// each. Grid (N/BN, row tiles of 128, S) with a thread-block cluster of S
+// CTAs along z: CTA z of a cluster runs K blocks [z*KB/S, (z+1)*KB/S) of one
+// 128 x BN output tile into its own TMEM accumulator (warp 0 streams the A
+// and B tiles with TMA, warp 1 issues tcgen05.mma), then all four warps copy
+// the fp32 partial tile from TMEM to shared memory. After a cluster barrier
+// CTA z owns a contiguous share of the tile's valid rows: it sums the S
+// partials of those rows over distributed shared memory in rank order (so a
+// result never depends on the batch size or on timing) and applies the
+// epilogue with threads laid along the columns (coalesced stores). A second
+// cluster barrier keeps every CTA's shared memory alive until its peers have
+// read it. S is a function of N and K only.
+//
+// The epilogues fuse the decoder's elementwise work:
+//  * RMSNorm. A residual-stream update (h += C) also writes the next
+//    sublayer's input as bf16(h * gamma) and, per row, the sum of squares of
+//    h over its BN columns. A GEMM that consumes that input recovers the row
+//    scale r = 1/sqrt(mean(h^2) + eps) from the partial sums (added in column
+//    tile order) and scales its result rows by r, since
+//    RMSNorm(h) W^T = r * ((h * gamma) W^T).
+//  * Rotary embedding, the ring write of k and v, and the fp32 copy of q
+//    after the q/k/v projection (one head per BN columns).
+// Every mbarrier wait is bounded in device time; a CTA that gives up records
+// the error and still takes part in both cluster barriers.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+namespace rlt {
+
+// ---------------------------------------------------------------- PTX pieces
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+
+// All threads of every CTA of the cluster; release/acquire orders the shared
+// memory writes before the barrier with the peers' reads after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n"
+      "barrier.cluster.wait.acquire.aligned;\n" ::
+          : "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float2 ld_dsmem_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];\n"
+               : "=f"(v.x), "=f"(v.y)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// ------------------------------------------------------------- epilogue kinds
+// kPair:  v(row, col), v(row, col + 1)             -> epi.pair(row, col, v0, v1, r)
+// kRope:  v(row, col..col+1) and the same columns
+//         half a head further on (rotate-half)      -> epi.rotary(row, col, a0, a1, b0, b1, r)
+// kNorm:  like kPair; epi.pair returns its share of the row's sum of squares,
+//         the kernel adds the shares of a row's BN/2 threads (shuffle tree)
+//         and hands the total to epi.row_sum(row, column tile, ss)
+enum DecEpiKind { kPair = 0, kRope = 1, kNorm = 2 };
+
+// Row scale input of the consumers of a fused RMSNorm: nsq[row][np] partial
+// sums of squares of h over column tiles, d and eps of the norm.
+struct RowScaleIn {
+  const float *nsq;
+  int np;
+  float inv_d, eps;
+};
+
+// y = r * C  in fp32 (the cross-attention query; SwiGLU's gate half)
+struct EpiRsF32 {
+  static constexpr int kKind = kPair;
+  static constexpr bool kRowScale = true;
+  RowScaleIn rsi;
+  float *out;
+  int ld;
+  __device__ void pair(int m, int n, float a, float b, float r) const {
+    *reinterpret_cast<float2 *>(out + (size_t)m * ld + n) = make_float2(a * r, b * r);
+  }
+};
+
+// f = bf16(GELU(r * C))
+template <typename T> struct EpiRsGelu {
+  static constexpr int kKind = kPair;
+  static constexpr bool kRowScale = true;
+  RowScaleIn rsi;
+  T *out;
+  int ld;
+  __device__ void pair(int m, int n, float a, float b, float r) const {
+    out[(size_t)m * ld + n] = from_f<T>(gelu_erf(a * r));
+    out[(size_t)m * ld + n + 1] = from_f<T>(gelu_erf(b * r));
+  }
+};
+
+// f = bf16(SiLU(a_in) * (r * C)), a_in = the gate half already scaled
+template <typename T> struct EpiRsSwiglu {
+  static constexpr int kKind = kPair;
+  static constexpr bool kRowScale = true;
+  RowScaleIn rsi;
+  const float *a_in;
+  T *out;
+  int ld;
+  __device__ void pair(int m, int n, float a, float b, float r) const {
+    const size_t i = (size_t)m * ld + n;
+    out[i] = from_f<T>(silu(a_in[i]) * (a * r));
+    out[i + 1] = from_f<T>(silu(a_in[i + 1]) * (b * r));
+  }
+};
+
+// Residual update h += C; with gamma set, also the next sublayer's input
+// u = bf16(h * gamma) and the sum of squares of h over this column tile.
+template <typename T> struct EpiResidNorm {
+  static constexpr int kKind = kNorm;
+  static constexpr bool kRowScale = false;
+  RowScaleIn rsi;  // unused
+  float *h;
+  int ld;
+  const float *gamma;  // null: the next consumer normalises by itself
+  T *u;
+  float *nsq;
+  int np;
+  __device__ float pair(int m, int n, float a, float b, float) const {
+    float2 *p = reinterpret_cast<float2 *>(h + (size_t)m * ld + n);
+    float2 v = *p;
+    v.x += a;
+    v.y += b;
+    *p = v;
+    if (gamma) {
+      u[(size_t)m * ld + n] = from_f<T>(v.x * gamma[n]);
+      u[(size_t)m * ld + n + 1] = from_f<T>(v.y * gamma[n + 1]);
+    }
+    return v.x * v.x + v.y * v.y;
+  }
+  __device__ void row_sum(int m, int tile, float ss) const {
+    if (gamma) nsq[(size_t)m * np + tile] = ss;
+  }
+};
+
+// Gated merge h = e + alpha * sigmoid(C + b_g) * s, plus the first decoder
+// block's normalised input as in EpiResidNorm.
+template <typename T> struct EpiGateNorm {
+  static constexpr int kKind = kNorm;
+  static constexpr bool kRowScale = false;
+  RowScaleIn rsi;  // unused
+  const float *e, *s, *bias;
+  float alpha;
+  float *h;
+  int ld;
+  const float *gamma;
+  T *u;
+  float *nsq;
+  int np;
+  __device__ float pair(int m, int n, float a, float b, float) const {
+    const size_t i = (size_t)m * ld + n;
+    const float g0 = sigmoidf_(a + bias[n]), g1 = sigmoidf_(b + bias[n + 1]);
+    const float h0 = e[i] + alpha * g0 * s[i], h1 = e[i + 1] + alpha * g1 * s[i + 1];
+    h[i] = h0;
+    h[i + 1] = h1;
+    u[i] = from_f<T>(h0 * gamma[n]);
+    u[i + 1] = from_f<T>(h1 * gamma[n + 1]);
+    return h0 * h0 + h1 * h1;
+  }
+  __device__ void row_sum(int m, int tile, float ss) const { nsq[(size_t)m * np + tile] = ss; }
+};
+
+// q/k/v projection of the decoder's sliding-window sublayer: r * C, then
+// rotary q and k at the row's position t (pairs j, j + dh/2 of a head), q in
+// fp32 for the attention, k and v in the layer's ring at slot t mod W.
+// Ring layout per layer: [max_seqs][H][2][W][dh].
+template <typename T> struct EpiQkvRope {
+  static constexpr int kKind = kRope;
+  static constexpr bool kRowScale = true;
+  RowScaleIn rsi;
+  float *q;
+  T *ring_l;
+  const int *ready, *pos;
+  const float2 *rope;
+  int H, DH, W, d;
+  __device__ void rotary(int m, int col, float a0, float a1, float b0, float b1, float r) const {
+    a0 *= r;
+    a1 *= r;
+    b0 *= r;
+    b1 *= r;
+    const int which = col / d, c = col - which * d;
+    const int hh = c / DH, j = c - hh * DH, half = DH / 2;
+    const int t = pos[m];
+    if (which == 0 || which == 1) {
+      const float2 c0 = rope[(size_t)t * half + j], c1 = rope[(size_t)t * half + j + 1];
+      const float x0 = a0 * c0.x - b0 * c0.y, y0 = b0 * c0.x + a0 * c0.y;
+      const float x1 = a1 * c1.x - b1 * c1.y, y1 = b1 * c1.x + a1 * c1.y;
+      if (which == 0) {
+        float *qr = q + (size_t)m * d + hh * DH + j;
+        *reinterpret_cast<float2 *>(qr) = make_float2(x0, x1);
+        *reinterpret_cast<float2 *>(qr + half) = make_float2(y0, y1);
+        return;
+      }
+      a0 = x0;
+      a1 = x1;
+      b0 = y0;
+      b1 = y1;
+    }
+    T *kb = ring_l + (((size_t)ready[m] * H + hh) * 2 + (which == 2 ? 1 : 0)) * W * DH +
+            (size_t)(t % W) * DH + j;
+    kb[0] = from_f<T>(a0);
+    kb[1] = from_f<T>(a1);
+    kb[half] = from_f<T>(b0);
+    kb[half + 1] = from_f<T>(b1);
+  }
+};
+
+// ------------------------------------------------------------- shared memory
+constexpr int DEC_BAR_BYTES = 1024;  // barriers + TMEM slot, keeps tiles 1024-aligned
+
+template <int BN> struct DecSmem {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int P_LD = BN + 2;  // fp32 partial tile row stride (8-byte aligned pairs)
+  static constexpr int P_BYTES = TC_BM * P_LD * 4;
+  // dynamic bytes for `ns` ring stages: alignment slack + barriers + the
+  // larger of the ring and the partial tile (which reuses the ring)
+  static constexpr int bytes(int ns) {
+    return 1024 + DEC_BAR_BYTES + (ns * STAGE > P_BYTES ? ns * STAGE : P_BYTES);
+  }
+};
+
+// Cluster split count of a decode GEMM: about one CTA per SM over the N
+// tiles, at most 8 (the portable cluster size) and at most one per K block.
+inline int dec_splits(int n_tiles, int kb, int num_sms) {
+  int s = num_sms / (n_tiles > 0 ? n_tiles : 1);
+  if (s > 8) s = 8;
+  if (s > kb) s = kb;
+  return s < 1 ? 1 : s;
+}
+
+template <int BN, int STAGES, class Epi>
+__global__ void __launch_bounds__(128, 2)
+    k_gemm_dec(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const int *__restrict__ Mdev, int a_row0, int N, int K, int ns, Epi epi,
+               int *err) {
+  static_assert(BN == 32 || BN == 64 || BN == 128, "TMEM columns are a power of two >= 32");
+  using SM = DecSmem<BN>;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(base);
+  uint64_t *empty = full + STAGES;
+  uint64_t *accum = empty + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+  uint8_t *tiles = base + DEC_BAR_BYTES;
+  float *P = reinterpret_cast<float *>(tiles);  // partial tile, after the main loop
+  __shared__ float s_rs[TC_BM];
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * TC_BM, n0 = blockIdx.x * BN;
+  // the step's row count is staged before its first kernel starts
+  const int M = *Mdev;
+  if (m0 >= M) return;  // the whole cluster (same blockIdx.y), before any barrier
+  const int S = gridDim.z;
+  const int z = (int)cluster_ctarank();
+  const int kb_all = K / TC_BK;
+  const int kb0 = z * kb_all / S, KB = (z + 1) * kb_all / S - kb0;
+  const int rv = M - m0 < TC_BM ? M - m0 : TC_BM;       // valid rows of the tile
+  const int share = (rv + S - 1) / S;                   // rows reduced per CTA
+  const int r_lo = z * share < rv ? z * share : rv;
+  const int r_hi = r_lo + share < rv ? r_lo + share : rv;
+
+  if (threadIdx.x == 0) {
+    s_fail = 0;
+    for (int s = 0; s < ns; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  pdl_trigger();
+  if (warp == 0 && lane == 0) {
+    // producer: the weight tiles of the first stages do not depend on the
+    // previous kernel and stream before the dependency wait
+    const int pre = KB < ns ? KB : ns;
+    for (int kb = 0; kb < pre; kb++) {
+      mbar_expect_tx(&full[kb], SM::STAGE);
+      tma_load_2d(tiles + kb * SM::STAGE + SM::A_BYTES, &tmB, (kb0 + kb) * TC_BK, n0, &full[kb]);
+    }
+    pdl_wait();
+    for (int kb = 0; kb < pre; kb++)
+      tma_load_2d(tiles + kb * SM::STAGE, &tmA, (kb0 + kb) * TC_BK, a_row0 + m0, &full[kb]);
+    for (int kb = pre; kb < KB; kb++) {
+      const int s = kb % ns, u = kb / ns;
+      if (!mbar_wait_bounded(&empty[s], (u - 1) & 1, WAIT_LIMIT_NS_TC)) {
+        atomicExch(&s_fail, 1);
+        break;
+      }
+      uint8_t *a = tiles + s * SM::STAGE;
+      mbar_expect_tx(&full[s], SM::STAGE);
+      tma_load_2d(a, &tmA, (kb0 + kb) * TC_BK, a_row0 + m0, &full[s]);
+      tma_load_2d(a + SM::A_BYTES, &tmB, (kb0 + kb) * TC_BK, n0, &full[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
+    for (int kb = 0; kb < KB; kb++) {
+      const int s = kb % ns, u = kb / ns;
+      if (!mbar_wait_bounded(&full[s], u & 1, WAIT_LIMIT_NS_TC)) {
+        atomicExch(&s_fail, 1);
+        break;
+      }
+      tc_fence_after();
+      const uint8_t *a = tiles + s * SM::STAGE;
+      const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + SM::A_BYTES);
+#pragma unroll
+      for (int k = 0; k < TC_BK / 16; k++)
+        umma_bf16(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc,
+                  (kb > 0 || k > 0) ? 1u : 0u);
+      umma_commit(&empty[s]);
+    }
+    umma_commit(accum);
+  } else if (Epi::kRowScale && warp >= 2) {
+    // warps 2-3: row scales of this CTA's share of rows, from the partial
+    // sums of squares the producer of the input wrote (column tile order)
+    pdl_wait();
+    for (int i = threadIdx.x - 64; i < r_hi - r_lo; i += 64) {
+      const float *p = epi.rsi.nsq + (size_t)(m0 + r_lo + i) * epi.rsi.np;
+      float ss = 0.f;
+      for (int t = 0; t < epi.rsi.np; t++) ss += p[t];
+      s_rs[i] = rsqrtf(ss * epi.rsi.inv_d + epi.rsi.eps);
+    }
+  }
+  __syncwarp();
+  pdl_wait();  // the epilogue reads and writes buffers of earlier kernels
+
+  // partial tile: TMEM -> shared memory (warp w holds rows 32w..32w+31)
+  const bool acc_ok = mbar_wait_bounded(accum, 0, WAIT_LIMIT_NS_TC);
+  tc_fence_after();
+  if (!acc_ok) atomicExch(&s_fail, 1);
+  __syncthreads();
+  const bool ok = !s_fail;
+  if (ok && warp * 32 < rv) {
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      float v[16];
+      tmem_ld16(lane_base + c0, v);
+      float2 *pr = reinterpret_cast<float2 *>(P + (size_t)row * SM::P_LD + c0);
+#pragma unroll
+      for (int j = 0; j < 8; j++) pr[j] = make_float2(v[2 * j], v[2 * j + 1]);
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();  // every partial tile of the cluster is in shared memory
+
+  if (!ok) {
+    if (threadIdx.x == 0) set_error(err, DEV_ERR_TIMEOUT);
+  } else {
+    const uint32_t p_local = smem_u32(P);
+    uint32_t p_rank[8];
+#pragma unroll
+    for (int q = 0; q < 8; q++) p_rank[q] = q < S ? mapa_shared(p_local, q) : 0u;
+    const int rows = r_hi - r_lo;
+    auto sum_at = [&](int r, int c) {
+      float2 acc = make_float2(0.f, 0.f);
+      const uint32_t off = (uint32_t)((r * SM::P_LD + c) * 4);
+#pragma unroll
+      for (int q = 0; q < 8; q++)
+        if (q < S) {
+          const float2 p = ld_dsmem_f2(p_rank[q] + off);
+          acc.x += p.x;
+          acc.y += p.y;
+        }
+      return acc;
+    };
+    if constexpr (Epi::kKind == kRope) {
+      const int DH = epi.DH, half = DH / 2;
+      constexpr int PPR = BN / 4;  // first-half column pairs per row
+      for (int idx = threadIdx.x; idx < rows * PPR; idx += blockDim.x) {
+        const int rl = idx / PPR, p = idx - rl * PPR;
+        const int hh = (2 * p) / half, j = 2 * p - hh * half;
+        const int c = hh * DH + j, r = r_lo + rl;
+        const float2 a = sum_at(r, c), b = sum_at(r, c + half);
+        epi.rotary(m0 + r, n0 + c, a.x, a.y, b.x, b.y, Epi::kRowScale ? s_rs[rl] : 1.f);
+      }
+    } else {
+      constexpr int PPR = BN / 2;  // column pairs per row
+      const int total = rows * PPR;
+      // uniform trip count: the row sums shuffle over a row's PPR lanes
+      for (int b0 = 0; b0 < total; b0 += blockDim.x) {
+        const int idx = b0 + threadIdx.x;
+        const bool act = idx < total;
+        const int rl = act ? idx / PPR : 0, p = idx - (idx / PPR) * PPR;
+        float ss = 0.f;
+        if (act) {
+          const float2 v = sum_at(r_lo + rl, 2 * p);
+          const float r = Epi::kRowScale ? s_rs[rl] : 1.f;
+          if constexpr (Epi::kKind == kNorm)
+            ss = epi.pair(m0 + r_lo + rl, n0 + 2 * p, v.x, v.y, r);
+          else
+            epi.pair(m0 + r_lo + rl, n0 + 2 * p, v.x, v.y, r);
+        }
+        if constexpr (Epi::kKind == kNorm) {
+          static_assert(PPR == 16 || PPR == 32, "row groups of a half or a whole warp");
+#pragma unroll
+          for (int o = PPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          if (act && p == 0) epi.row_sum(m0 + r_lo + rl, blockIdx.x, ss);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();  // peers are done reading this CTA's partial tile
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, BN);
+}
+
+}  // namespace rlt

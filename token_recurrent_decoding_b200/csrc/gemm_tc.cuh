@@ -1,4 +1,5 @@
-// tcgen05 / TMEM GEMM for the large projections of the encoder prefill:
+// tcgen05 / TMEM GEMM for the large projections of the encoder prefill
+// (the decode step's small-row GEMMs are in gemm_dec.cuh):
 //   C[m][n] = sum_k A[m][k] * B[n][k],  A = activations [M][K], B = weights
 //   [N][K], both bf16 K-major, fp32 accumulation in tensor memory.
 //
@@ -114,26 +115,12 @@ template <int BN, int STAGES> struct TcSmem {
   static constexpr int BYTES = STAGES * STAGE + (2 * STAGES + 1) * 8 + 16 + 1024;
 };
 
-// Split-K for the tensor-core GEMM: K blocks of 64 divided into `splits`
-// contiguous ranges (a function of K only, so a row's result never depends on
-// the batch size). Large K only: below that one CTA walks all of K.
-inline int tc_splits(int K) {
-  const int kt = K / TC_BK;
-  int s = 1;
-  for (int c = 1; c <= K / 768; c++)
-    if (kt % c == 0) s = c;
-  return s;
-}
-
 // Row block m0.. of A (plus a_row0 inside A's tensor map) times all of B's
-// rows n0..n0+BN. Mdev (optional) gives the rows at run time; a split-K
-// launch (gridDim.z > 1) writes fp32 partial tiles to sk.part and the last
-// split of a tile to arrive sums them in split order and runs the epilogue.
+// rows n0..n0+BN.
 template <int BN, int STAGES, class Epi>
 __global__ void __launch_bounds__(128, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              int M, const int *__restrict__ Mdev, int a_row0, int N, int K, Epi epi,
-              SplitK sk, int *err) {
+              int M, int a_row0, int N, int K, Epi epi, int *err) {
   static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256,
                 "TMEM columns are a power of two >= 32");
   using SM = TcSmem<BN, STAGES>;
@@ -144,15 +131,12 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t *empty = full + STAGES;
   uint64_t *accum = empty + STAGES;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
-  __shared__ int s_fail, s_last;
+  __shared__ int s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * TC_BM, n0 = blockIdx.x * BN;
-  if (Mdev) M = *Mdev;
   if (m0 >= M) return;  // whole CTA, before any barrier or TMEM
-  const int splits = gridDim.z, z = blockIdx.z;
-  const int kb_all = K / TC_BK;
-  const int kb0 = z * kb_all / splits, KB = (z + 1) * kb_all / splits - kb0;
+  const int kb0 = 0, KB = K / TC_BK;
 
   if (threadIdx.x == 0) {
     s_fail = 0;
@@ -227,7 +211,7 @@ __global__ void __launch_bounds__(128, 1)
   const bool ok = acc_ok && !s_fail;
   if (!ok) {
     if (threadIdx.x == 0) set_error(err, DEV_ERR_TIMEOUT);
-  } else if (splits == 1) {
+  } else {
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 16) {
       float v[16];
@@ -240,53 +224,10 @@ __global__ void __launch_bounds__(128, 1)
         }
       }
     }
-  } else {
-    const int M_grid = gridDim.y * TC_BM;
-    float *pz = sk.part + (size_t)z * M_grid * N;
-#pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 16) {
-      float v[16];
-      tmem_ld16(lane_base + c0, v);
-      if (row < M) {
-#pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          if (n0 + c0 + j < N)
-            *reinterpret_cast<float4 *>(pz + (size_t)row * N + n0 + c0 + j) =
-                make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-      }
-    }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, BN);
-  if (!ok || splits == 1) return;
-  // split-K: the last split of this tile sums the partials in split order
-  __threadfence();
-  __syncthreads();
-  const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-  if (threadIdx.x == 0) s_last = (atomicAdd(&sk.counters[tile], 1) == splits - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  if (row < M) {
-    const int M_grid = gridDim.y * TC_BM;
-    for (int c = 0; c < BN; c += 4) {
-      const int col = n0 + c;
-      if (col >= N) break;
-      float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int zz = 0; zz < splits; zz++) {
-        const float4 p = __ldcg(reinterpret_cast<const float4 *>(
-            sk.part + ((size_t)zz * M_grid + row) * N + col));
-        acc4.x += p.x;
-        acc4.y += p.y;
-        acc4.z += p.z;
-        acc4.w += p.w;
-      }
-      epi(row, col, acc4.x, acc4.y);
-      epi(row, col + 2, acc4.z, acc4.w);
-    }
-  }
-  if (threadIdx.x == 0) sk.counters[tile] = 0;
 }
 
 }  // namespace rlt

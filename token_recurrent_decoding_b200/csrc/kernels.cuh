@@ -56,16 +56,22 @@ __global__ void k_rmsnorm(int rows, const int *__restrict__ rows_dev, int d,
 
 // ----------------------------------------------------------- decoder step
 // Step start: position of each ready slot, GEMM input [e_t ; s_{t-1}] and fp32
-// copies for the gated merge. With feedback off the residual is e_t itself.
+// copies for the gated merge. With feedback off the residual is e_t itself;
+// then, given gamma1 (the first block's RMSNorm gain), the block also writes
+// that block's input bf16(e_t * gamma1) and the row's sum of squares (in
+// partial slot 0 of np, the rest zero) for a GEMM that applies the norm.
 template <typename T>
 __global__ void k_step_gather(const int *__restrict__ n_dev, int d, int max_len,
                               const int *__restrict__ ready,
                               const int *__restrict__ t_dec, int *__restrict__ pos,
                               const T *__restrict__ e, const float *__restrict__ s,
                               T *__restrict__ xin, float *__restrict__ e32,
-                              float *__restrict__ s32, float *__restrict__ h, int alpha_zero) {
+                              float *__restrict__ s32, float *__restrict__ h, int alpha_zero,
+                              const float *__restrict__ gamma1, T *__restrict__ u,
+                              float *__restrict__ nsq, int np) {
   pdl_wait();
   pdl_trigger();
+  __shared__ float red[32];
   int i = blockIdx.x;
   if (i >= *n_dev) return;
   int seq = ready[i];
@@ -73,6 +79,8 @@ __global__ void k_step_gather(const int *__restrict__ n_dev, int d, int max_len,
   if (threadIdx.x == 0) pos[i] = t;
   const T *er = e + ((size_t)seq * max_len + t) * d;
   const float *sr = s + (size_t)seq * d;
+  const bool norm = alpha_zero && gamma1;
+  float ss = 0.f;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     T ev = er[c];
     float sv = sr[c];
@@ -82,7 +90,22 @@ __global__ void k_step_gather(const int *__restrict__ n_dev, int d, int max_len,
     e32[(size_t)i * d + c] = ef;
     s32[(size_t)i * d + c] = sv;
     if (alpha_zero) h[(size_t)i * d + c] = ef;
+    if (norm) {
+      u[(size_t)i * d + c] = from_f<T>(ef * gamma1[c]);
+      ss += ef * ef;
+    }
   }
+  if (!norm) return;
+  ss = warp_sum(ss);
+  const int w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int k = 0; k < nw; k++) tot += red[k];
+    nsq[(size_t)i * np] = tot;
+  }
+  for (int k = 1 + threadIdx.x; k < np; k += blockDim.x) nsq[(size_t)i * np + k] = 0.f;
 }
 
 // After the q/k/v projection: rotary q (fp32, kept for the SWA), rotary k and

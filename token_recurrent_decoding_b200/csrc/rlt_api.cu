@@ -23,6 +23,7 @@
 #include "attn.cuh"
 #include "enc_attn.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_dec.cuh"
 
 using namespace rlt;
 
@@ -37,7 +38,7 @@ struct Layout {
   size_t s, t_dec, t_enc, e, mem, ring, rope, err;
   // decoder step work buffers (max_seqs rows)
   size_t nready, ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part, counters;
-  size_t gpart[2], gcnt[2];  // split-K scratch of each step chain
+  size_t nsq;  // per-row partial sums of squares of h over 32-column tiles (bf16 models)
   // encoder work buffers (ptok rows)
   size_t tok, tok_slot, tok_pos, tok_start, blk, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
   size_t staging, staging_bytes;
@@ -110,17 +111,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->f = take(S * F * es);
   L->part = take(S * H * L->max_chunks * (dh + 2) * 4);
   L->counters = take(S * H * 4);
-  {
-    // split-K scratch: largest splits * N over the decoder GEMMs, per row
-    auto sn = [](size_t n, size_t k) { return (size_t)tc_splits((int)k) * n; };
-    const size_t per_row = std::max({sn(d, 2 * d), sn(3 * d, d), sn(d, d), sn(F, d), sn(d, F)});
-    const size_t rows = (S + 127) / 128 * 128;  // row tiles of 128
-    const size_t tiles = rows / 128 * ((std::max({3 * d, F, d}) + 31) / 32);
-    for (int ch = 0; ch < 2; ch++) {
-      L->gpart[ch] = take(c->dtype == RLT_BF16 ? per_row * rows * 4 : 0);
-      L->gcnt[ch] = take(tiles * 4);
-    }
-  }
+  L->nsq = take(c->dtype == RLT_BF16 ? S * (d / 32) * 4 : 0);
   size_t P = (size_t)ptok;
   L->tok = take(P * 4);
   L->tok_slot = take(P * 4);
@@ -173,6 +164,7 @@ struct rlt_model {
   Layout L;
   uint8_t *arena = nullptr;
   int device = 0;
+  int num_sms = 148;  // SMs of the device (decode GEMM split counts)
   std::vector<int> t_dec, t_enc;
   cudaStream_t last_stream = nullptr;
   template <typename X> X *at(size_t off) const { return reinterpret_cast<X *>(arena + off); }
@@ -284,14 +276,12 @@ const CUtensorMap *tmap_bf16(rlt_model *M, const void *ptr, uint64_t rows, uint6
   return &M->tmaps.emplace(key, m).first->second;
 }
 
-// tcgen05 GEMM: rows [a_row0 + m, ...) of A [a_rows][k] (activations) times
-// B [n][k] (weights). m_grid bounds the rows (grid); Mdev, if set, gives the
-// rows at run time. The encoder's large row counts use 128-wide N tiles; the
-// decoder's small batches use 32/64-wide tiles (more CTAs stream the weights)
-// and split-K over large K into `ws`.
+// tcgen05 GEMM of the encoder: rows [a_row0 + m, ...) of A [a_rows][k]
+// (activations) times B [n][k] (weights), 128 x BN tiles; m_grid bounds the
+// rows (grid). Large row counts use 128-wide N tiles.
 template <int BN, int STAGES, class Epi>
-cudaError_t launch_tc(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
-                      int k, const bf16 *A, const bf16 *B, Epi epi, SplitK sk, cudaStream_t st) {
+cudaError_t launch_tc(rlt_model *M, int m_grid, int a_rows, int a_row0, int n, int k,
+                      const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
   constexpr int smem = TcSmem<BN, STAGES>::BYTES;
   const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
   const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
@@ -302,23 +292,63 @@ cudaError_t launch_tc(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int
     RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     attr = true;
   }
-  dim3 grid((n + BN - 1) / BN, (m_grid + TC_BM - 1) / TC_BM, sk.splits);
-  return launch_k(kern, grid, dim3(128), smem, st, *ma, *mb, m_grid, Mdev, a_row0, n, k, epi, sk,
+  dim3 grid((n + BN - 1) / BN, (m_grid + TC_BM - 1) / TC_BM);
+  return launch_k(kern, grid, dim3(128), smem, st, *ma, *mb, m_grid, a_row0, n, k, epi,
                   M->at<int>(M->L.err));
 }
 
 template <class Epi>
-cudaError_t gemm_tc(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
-                    int k, const bf16 *A, const bf16 *B, Epi epi, const SplitK *ws,
-                    cudaStream_t st) {
+cudaError_t gemm_tc(rlt_model *M, int m_grid, int a_rows, int a_row0, int n, int k,
+                    const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
   if (m_grid <= 0) return cudaSuccess;
-  SplitK one{1, nullptr, nullptr};
-  if (m_grid >= 1024)
-    return launch_tc<128, 3>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, one, st);
-  SplitK sk = one;
-  if (ws && ws->part && tc_splits(k) > 1) sk = {tc_splits(k), ws->part, ws->counters};
-  if (n >= 2048) return launch_tc<64, 4>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, sk, st);
-  return launch_tc<32, 4>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, sk, st);
+  if (m_grid >= 1024) return launch_tc<128, 3>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
+  if (n >= 2048) return launch_tc<64, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
+  return launch_tc<32, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
+}
+
+// Decode-step GEMM (gemm_dec.cuh): rows [a_row0 + m, ...) of A [a_rows][k]
+// times B [n][k] with BN-wide output tiles and a cluster of S split-K CTAs
+// per tile; m_grid bounds the rows, Mdev holds the row count at run time.
+template <int BN, class Epi>
+cudaError_t launch_dec(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
+                       int k, const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
+  constexpr int STAGES = 4;
+  if (m_grid <= 0) return cudaSuccess;
+  if (n % BN || k % TC_BK) return cudaErrorInvalidValue;
+  const int kb = k / TC_BK, tiles = n / BN;
+  const int S = dec_splits(tiles, kb, M->num_sms);
+  const int kb_max = (kb + S - 1) / S;
+  const int ns = kb_max < STAGES ? kb_max : STAGES;
+  const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
+  const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
+  if (!ma || !mb) return cudaErrorInvalidValue;
+  auto kern = k_gemm_dec<BN, STAGES, Epi>;
+  static bool attr = false;
+  if (!attr) {
+    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DecSmem<BN>::bytes(STAGES)));
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(tiles, (m_grid + TC_BM - 1) / TC_BM, S);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = DecSmem<BN>::bytes(ns);
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = S;
+  int na = 1;
+  if (st != nullptr) {
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    na = 2;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, *ma, *mb, Mdev, a_row0, n, k, ns, epi,
+                            M->at<int>(M->L.err));
 }
 
 cudaEvent_t take_event(rlt_model *M) {
@@ -376,7 +406,7 @@ cudaError_t gemm_enc(rlt_model *M, int m, int n, int k, const T *A, const T *B, 
   Span sp(M, st, RLT_K_ENC, (double)n * k * es + (double)m * k * es + (double)m * n * 4.0,
           2.0 * m * n * k);
   if constexpr (std::is_same<T, bf16>::value)
-    return gemm_tc(M, m, nullptr, M->L.ptok, 0, n, k, A, B, epi, nullptr, st);
+    return gemm_tc(M, m, M->L.ptok, 0, n, k, A, B, epi, st);
   else
     return gemm(m, nullptr, n, k, A, k, B, k, epi, st);
 }
@@ -434,6 +464,7 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
                   M->at<int>(L.err), pf);
 }
 
+// fp32 models: exact SIMT GEMMs with separate RMSNorm and rotary kernels.
 template <typename T, int DH>
 cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   const rlt_config &c = M->cfg;
@@ -465,17 +496,14 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   // y = A_rows(r0..) W^T with A one of the whole activation buffers above
   auto G = [&](int kind, int nn, int k, const T *A_base, const T *B, auto epi) {
     Span sp(M, st, kind, (double)nn * k * es + nr * k * es + nr * nn * 4.0, 2.0 * nr * nn * k);
-    const SplitK sk{0, M->at<float>(L.gpart[si.chain]), M->at<int>(L.gcnt[si.chain])};
-    if constexpr (std::is_same<T, bf16>::value)
-      return gemm_tc(M, n, nd, c.max_seqs, (int)r0, nn, k, A_base, B, epi, &sk, st);
-    else
-      return gemm(n, nd, nn, k, A_base + r0 * k, k, B, k, epi, st);
+    return gemm(n, nd, nn, k, A_base + r0 * k, k, B, k, epi, st);
   };
 
   {
     Span sp(M, st, RLT_K_OTHER, nr * d * (es + 4) + row_bytes);
     RLT_TRY(launch_k(k_step_gather<T>, dim3(n), dim3(256), 0, st, nd, d, c.max_len, ready, t_dec,
-                     pos, M->at<T>(L.e), s, xin, e32, s32, h, (int)a0));
+                     pos, M->at<T>(L.e), s, xin, e32, s32, h, (int)a0, (const float *)nullptr,
+                     (T *)nullptr, (float *)nullptr, 0));
   }
   if (!a0)
     RLT_TRY(G(RLT_K_GEMM, d, 2 * d, xin_b, (const T *)M->w.gate_w,
@@ -544,6 +572,107 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
       RLT_TRY(G(RLT_K_GEMM, F, d, u_b, W_<T>::wb(M, l), EpiSwiglu<T>{fa, f, F}));
     }
     RLT_TRY(G(RLT_K_GEMM, d, F, f_b, W_<T>::w2(M, l), EpiResid{h, d}));
+  }
+  {
+    Span sp(M, st, RLT_K_OTHER, nr * d * 8);
+    RLT_TRY(launch_k(k_step_final, dim3(rows_blocks), dim3(256), 0, st, nd, d, ready, t_dec, h,
+                     (const float *)M->w.dec_lnf, eps, s));
+  }
+  return cudaGetLastError();
+}
+
+// bf16 models: the same transition on the tensor cores with the RMSNorms,
+// the rotary embedding and the ring write fused into the decode GEMMs
+// (gemm_dec.cuh). Per block: q/k/v GEMM (norm scale, rotary, ring, q) ->
+// SWA -> W_o GEMM (h +=, next input, norm partials) -> W_qx GEMM (norm scale)
+// -> cross-attention -> W_ox GEMM (h +=, ...) -> FFN up (norm scale,
+// activation) -> FFN down (h +=, next block's input).
+template <int DH>
+cudaError_t step_impl_tc(rlt_model *M, const StepInfo &si, cudaStream_t st) {
+  using T = bf16;
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const int n = si.n_grid;  // grid bound; the kernels read the real n on the device
+  const int *nd = M->at<int>(L.nready) + si.chain;
+  const int d = c.d, H = c.n_heads, F = c.ffn_dim, W = c.window;
+  const float eps = c.rms_eps;
+  const double es = sizeof(T);
+  const size_t r0 = si.row0;  // this chain's rows of every per-row buffer
+  const int np = d / 32;      // column tiles of the N = d GEMMs (norm partials per row)
+  int *ready = M->at<int>(L.ready) + r0, *pos = M->at<int>(L.pos) + r0;
+  int *t_dec = M->at<int>(L.t_dec);
+  float *h = M->at<float>(L.h) + r0 * d, *e32 = M->at<float>(L.e32) + r0 * d;
+  float *s32 = M->at<float>(L.s32) + r0 * d;
+  float *q = M->at<float>(L.q) + r0 * d, *fa = M->at<float>(L.fa) + r0 * F;
+  float *nsq = M->at<float>(L.nsq) + r0 * np;
+  float *s = M->at<float>(L.s);
+  T *xin_b = M->at<T>(L.xin), *a_b = M->at<T>(L.a), *u_b = M->at<T>(L.u), *f_b = M->at<T>(L.f);
+  T *xin = xin_b + r0 * 2 * d, *u = u_b + r0 * d, *f = f_b + r0 * F;
+  T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem);
+  const float2 *rope = M->at<float2>(L.rope);
+  const bool a0 = c.alpha == 0.0f;
+  const size_t ring_layer = (size_t)c.max_seqs * H * 2 * W * DH;
+  const size_t mem_group = (size_t)c.max_seqs * H * 2 * c.max_len * DH;
+  const int rows_blocks = blocks_for((long)n * 32, 256);
+  const double nr = si.n;  // real rows, for the algorithmic byte counts
+  const RowScaleIn rsi{nsq, np, 1.0f / (float)d, eps};
+  const L2Prefetch no_pf{};
+  const float *const *ln1 = (const float *const *)M->w.dec_ln1;
+  // y = A_rows(r0..) W^T with A one of the whole activation buffers above
+  auto G = [&](auto bn, int nn, int k, const T *A_base, const T *B, auto epi) {
+    Span sp(M, st, RLT_K_GEMM, (double)nn * k * es + nr * k * es + nr * nn * 4.0,
+            2.0 * nr * nn * k);
+    return launch_dec<decltype(bn)::value>(M, n, nd, c.max_seqs, (int)r0, nn, k, A_base, B, epi,
+                                          st);
+  };
+  using BN32 = std::integral_constant<int, 32>;
+  using BNQ = std::integral_constant<int, (DH >= 32 ? DH : 32)>;
+  using BN64 = std::integral_constant<int, 64>;
+
+  {
+    Span sp(M, st, RLT_K_OTHER, nr * d * (es + 4) + nr * d * (4 + es));
+    RLT_TRY(launch_k(k_step_gather<T>, dim3(n), dim3(256), 0, st, nd, d, c.max_len, ready, t_dec,
+                     pos, M->at<T>(L.e), s, xin, e32, s32, h, (int)a0, a0 ? ln1[0] : nullptr,
+                     u, nsq, np));
+  }
+  if (!a0)
+    RLT_TRY(G(BN32{}, d, 2 * d, xin_b, (const T *)M->w.gate_w,
+              EpiGateNorm<T>{{}, e32, s32, (const float *)M->w.gate_b, c.alpha, h, d, ln1[0], u,
+                             nsq, np}));
+  for (int l = 0; l < c.n_dec_layers; l++) {
+    T *ring_l = ring + (size_t)l * ring_layer;
+    const T *mem_g = mem + (size_t)(c.mem_groups == 1 ? 0 : l) * mem_group;
+    const bool last = l + 1 == c.n_dec_layers;
+    // sliding-window self-attention sublayer
+    RLT_TRY(G(BNQ{}, 3 * d, d, u_b, W_<T>::qkv(M, l),
+              EpiQkvRope<T>{rsi, q, ring_l, ready, pos, rope, H, DH, W, d}));
+    {
+      Span sp(M, st, RLT_K_SWA, si.sum_win * 2.0 * d * es + nr * d * (4 + es),
+              4.0 * d * si.sum_win);
+      RLT_TRY((launch_attn<T, DH>(M, si, W, 1, ring_l, (long)H * 2 * W * DH, 2L * W * DH,
+                                  (long)W * DH, M->at<T>(L.a) + r0 * d, no_pf, st)));
+    }
+    RLT_TRY(G(BN32{}, d, d, a_b, W_<T>::o(M, l),
+              EpiResidNorm<T>{{}, h, d, (const float *)M->w.dec_ln2[l], u, nsq, np}));
+    // cross-attention sublayer over M<=t
+    RLT_TRY(G(BN32{}, d, d, u_b, (const T *)M->w.dec_wqx[l], EpiRsF32{rsi, q, d}));
+    {
+      Span sp(M, st, RLT_K_XATTN, si.sum_keys * 2.0 * d * es, 4.0 * d * si.sum_keys);
+      RLT_TRY((launch_attn<T, DH>(M, si, 0, si.xchunks, mem_g, (long)H * 2 * c.max_len * DH,
+                                  2L * c.max_len * DH, (long)c.max_len * DH,
+                                  M->at<T>(L.a) + r0 * d, no_pf, st)));
+    }
+    RLT_TRY(G(BN32{}, d, d, a_b, (const T *)M->w.dec_wox[l],
+              EpiResidNorm<T>{{}, h, d, (const float *)M->w.dec_ln3[l], u, nsq, np}));
+    // FFN sublayer
+    if (c.ffn_kind == RLT_GELU) {
+      RLT_TRY(G(BN64{}, F, d, u_b, W_<T>::w1(M, l), EpiRsGelu<T>{rsi, f, F}));
+    } else {
+      RLT_TRY(G(BN64{}, F, d, u_b, W_<T>::w1(M, l), EpiRsF32{rsi, fa, F}));
+      RLT_TRY(G(BN64{}, F, d, u_b, W_<T>::wb(M, l), EpiRsSwiglu<T>{rsi, fa, f, F}));
+    }
+    RLT_TRY(G(BN32{}, d, F, f_b, W_<T>::w2(M, l),
+              EpiResidNorm<T>{{}, h, d, last ? nullptr : ln1[l + 1], u, nsq, np}));
   }
   {
     Span sp(M, st, RLT_K_OTHER, nr * d * 8);
@@ -683,7 +812,10 @@ cudaError_t get_memory_impl(rlt_model *M, int seq, int t_enc, cudaStream_t st) {
 }
 
 template <typename T, int DH> void bind(rlt_model *M) {
-  M->step = step_impl<T, DH>;
+  if constexpr (std::is_same<T, bf16>::value)
+    M->step = step_impl_tc<DH>;
+  else
+    M->step = step_impl<T, DH>;
   M->prefill = prefill_impl<T, DH>;
   M->get_window = get_window_impl<T>;
   M->set_window = set_window_impl<T>;
@@ -1078,6 +1210,8 @@ RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *w, void *d_aren
   M->t_enc.assign(cfg->max_seqs, 0);
   if (cfg->dtype == RLT_BF16) bind_dh<bf16>(M); else bind_dh<float>(M);
   cudaError_t e = cudaSetDevice(M->device);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&M->num_sms, cudaDevAttrMultiProcessorCount, M->device);
   int half = cfg->head_dim / 2;
   if (e == cudaSuccess) e = cudaMemsetAsync(M->arena, 0, L.total, 0);
   if (e == cudaSuccess) {

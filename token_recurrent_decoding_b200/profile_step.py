@@ -7,8 +7,11 @@ Decoder steps at a chosen position:
 prefills the encoder for the batch, places every sequence at position t with a
 random state imported through rlt_set_state (s and the window of every layer),
 and runs `steps` decoder steps with direct launches on the legacy stream, so a
-profiler sees each kernel once per layer per step. Prints the CUDA-event time
-of each step and its algorithmic bytes.
+profiler sees each kernel once per layer per step. With --graph the steps run
+on a side stream instead, i.e. through the captured step graphs (two chains
+for large batches, programmatic dependent launch between kernels), as a
+serving loop would; the first step captures. Prints the CUDA-event time of
+each step and its algorithmic bytes.
 
 The decode attention kernel alone, through rlt_attend:
 
@@ -48,18 +51,24 @@ def run_steps(args):
         m.set_state(i, s, cache, args.t)
     torch.cuda.synchronize()
     ids = list(range(B))
+    st = torch.cuda.Stream() if args.graph else None
     times = []
     for k in range(args.steps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        m.decoder_step(ids)
-        b.record()
+        if st is not None:
+            a.record(st)
+            m.decoder_step(ids, stream=st)
+            b.record(st)
+        else:
+            a.record()
+            m.decoder_step(ids)
+            b.record()
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
     assert m.poll_device_error() == 0
     ts = [np.full(B, args.t + k) for k in range(args.steps)]
     byts = [roofline.decoder_step_bytes(cfg, x) for x in ts]
-    print(json.dumps({"workload": args.workload, "batch": B, "t": args.t,
+    print(json.dumps({"workload": args.workload, "batch": B, "t": args.t, "graph": args.graph,
                       "step_ms": times, "step_GB": [x / 1e9 for x in byts],
                       "GB_s": [x / (ms / 1e3) / 1e9 for x, ms in zip(byts, times)]}))
 
@@ -96,6 +105,7 @@ def main():
     ap.add_argument("--t", type=int, default=512)
     ap.add_argument("--steps", type=int, default=2)
     ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--graph", action="store_true")
     ap.add_argument("--attend", action="store_true")
     ap.add_argument("--n", type=int, default=256)
     ap.add_argument("--heads", type=int, default=12)
