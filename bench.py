@@ -42,6 +42,31 @@ WORKLOAD_TEXT = {
 }
 
 
+# DRAM traffic of the dominant kernel from its committed Nsight Compute
+# summary: bytes read + written per algorithmic byte, valid only while the
+# kernel source hashes to the value recorded with the capture.
+ATTN_PROFILE = os.path.join(ROOT, "profiles", "k_attn_decode_bf16_dh64_n256_len512.md")
+ATTN_SOURCE = os.path.join(ROOT, "token_recurrent_decoding_b200", "csrc", "attn.cuh")
+
+
+def attn_traffic_ratio():
+    import hashlib
+    if not os.path.exists(ATTN_PROFILE):
+        return None, "no profile"
+    ratio = sha = None
+    with open(ATTN_PROFILE) as f:
+        for line in f:
+            if line.startswith("source sha256"):
+                sha = line.split(":", 1)[1].strip().strip("`")
+            elif line.startswith("dram bytes per algorithmic byte"):
+                ratio = float(line.split(":", 1)[1].strip().strip("`"))
+    with open(ATTN_SOURCE, "rb") as f:
+        cur = hashlib.sha256(f.read()).hexdigest()
+    if ratio is None or sha != cur:
+        return None, "kernel changed since the capture" if ratio is not None else "no ratio"
+    return ratio, os.path.relpath(ATTN_PROFILE, ROOT)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -242,6 +267,8 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
     roof = roofline.run_roofline(cfg, wl.lengths, hbm, tc)
     x = stats["xattn"]
     achieved = (x["bytes"] / x["launches"]) / (x["ms"] / x["launches"] / 1e3) / 1e9 if x["launches"] else None
+    ratio, traffic_src = attn_traffic_ratio()
+    traffic = ratio * x["bytes"] / x["launches"] if (ratio and x["launches"]) else None
     dec_s = dec_ms / 1e3 / args.steps
     enc_s = enc_ms / 1e3 / args.steps
     out = {
@@ -276,13 +303,16 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
             "peaks": f"{peaks_src}: HBM {hbm} GB/s, bf16 {tc} TFLOP/s (sustained)",
         },
         "roofline": {
-            "kernel": "k_xattn_partial (decoder cross-attention over M<=t)",
+            "kernel": "k_attn_decode (decoder cross-attention over M<=t)",
             "bound": "hbm",
             "achieved": achieved,
             "peak": hbm,
             "unit": "GB/s",
             "frac": achieved / hbm if achieved else None,
-            "traffic": None,
+            "traffic": traffic,
+            "traffic_source": traffic_src,
+            "algorithmic_bytes_per_launch": (x["bytes"] / x["launches"]) if x["launches"] else None,
+            "launches_timed": x["launches"],
             "peak_source": peaks_src,
         },
         "kernel_classes": {k: {"ms_per_step": v["ms"] / args.steps,
@@ -370,7 +400,7 @@ def main():
                     help="one JSON line per workload (not the default contract line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-positions", type=int, default=24)
-    ap.add_argument("--profile-stride", type=int, default=16,
+    ap.add_argument("--profile-stride", type=int, default=64,
                     help="event-time every k-th decoder step for the per-kernel roofline")
     args = ap.parse_args()
 

@@ -4,7 +4,8 @@ Decoder steps at a chosen position:
 
     python -m token_recurrent_decoding_b200.profile_step --workload m140_bf16 --t 512 --steps 2
 
-prefills the encoder for the batch, places every sequence at position t with a
+prefills the encoder for the batch (--max-len shrinks the sequence length and
+so the arena), places every sequence at position t with a
 random state imported through rlt_set_state (s and the window of every layer),
 and runs `steps` decoder steps with direct launches on the legacy stream, so a
 profiler sees each kernel once per layer per step. With --graph the steps run
@@ -34,7 +35,9 @@ def run_steps(args):
     wl = configs.workloads()[args.workload]
     cfg = wl.model
     B = args.batch or wl.batch
-    T = wl.max_len
+    T = args.max_len or wl.max_len
+    if args.t + args.steps > T:
+        raise SystemExit(f"--t {args.t} + --steps {args.steps} exceeds the sequence length {T}")
     lengths = [T] * B
     w = inputs.make_weights(cfg)
     tok = inputs.make_tokens(cfg.vocab, lengths)
@@ -105,6 +108,9 @@ def main():
     ap.add_argument("--t", type=int, default=512)
     ap.add_argument("--steps", type=int, default=2)
     ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--max-len", type=int, default=0,
+                    help="sequence length of the arena (default: the workload's); small "
+                         "values keep a profiler's device memory small")
     ap.add_argument("--graph", action="store_true")
     ap.add_argument("--attend", action="store_true")
     ap.add_argument("--n", type=int, default=256)
