@@ -34,6 +34,12 @@
  *   window    SWA at t attends positions max(0, t-W+1) .. t
  * Matrices are row-major [out][in] (y_j = sum_i W[j][i] x_i). The q/k/v
  * projection stacks rows q | k | v; head h owns entries h*dh .. h*dh+dh-1.
+ *
+ * Pins: every piece, the ring window, the gate at alpha = 0, causality, the
+ * carried-state split, the G and tying plumbing are checked against closed
+ * forms, brute force and textbook routines by the CPU tests. The whole
+ * model's outputs are parity unpinned against the pages: they print no
+ * values for any configuration.
  */
 #include <math.h>
 #include <stdlib.h>
