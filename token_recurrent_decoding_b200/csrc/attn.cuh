@@ -25,6 +25,13 @@
 // own t, so results never depend on the batch around the row or on which
 // warp ran which unit. Every wait is bounded in device time.
 //
+// Inside a decoder step (t_seq given: positions by sequence id, which no
+// kernel of the step writes) the producer starts before its programmatic
+// dependency wait: it fills the first stages of every warp with K/V tiles
+// that the previous kernels do not write (all memory tiles; every ring tile
+// but the one holding slot t mod W), while the preceding GEMM still runs,
+// and adds the queries of those stages after the wait.
+//
 // Page key: [RLT-96] "RLT Runs 96 Blocks Per Token With Recurrent State, No
 // Resets" (aimastery.page).
 #pragma once
@@ -68,13 +75,6 @@ constexpr int attn_smem_bytes() {
   return NC * SW * AttnShape<T, DH, TB>::STAGE + 2 * NC * SW * 8 + 16 + 2 * ATTN_SMEM_ROWS * 4;
 }
 
-// Up to six byte ranges (e.g. the weights of the GEMMs that follow) that the
-// idle lanes of the producer warps pull into L2 while the attention streams.
-struct L2Prefetch {
-  const char *p[6];
-  unsigned long long n[6];
-};
-
 // Header the producer writes into a stage for its consumer.
 struct AttnHdr {
   int ih;     // slot * H + head
@@ -97,6 +97,7 @@ struct AttnGeom {
 // Producer-side walk over one consumer warp's units and their tiles.
 template <typename T, int KT> struct UnitWalk {
   int u, j, ntiles, nch, ih, c, r0, r1;
+  int dep_row;  // SWA: ring row written by this step (slot t mod W), else -1
   const T *K;
   __device__ bool load(const AttnGeom &g) {
     const int pairs = g.units / g.xchunks;  // n_grid * H
@@ -110,6 +111,7 @@ template <typename T, int KT> struct UnitWalk {
     if (c >= nch) return false;
     r0 = c * g.CH;
     r1 = min(L, r0 + g.CH);
+    dep_row = g.window > 0 ? t % g.window : -1;
     ntiles = (r1 - r0 + KT - 1) / KT;
     j = 0;
     const int seq = g.ready[i];
@@ -149,10 +151,11 @@ template <typename T, int DH, int NC = AttnCfg::NC, int SW = AttnCfg::SW,
 __global__ void __launch_bounds__((NC + 1) * 32)
     k_attn_decode(const int *__restrict__ n_dev, int H, int window, int CH, int xchunks,
                   int max_chunks, int n_grid, const int *__restrict__ ready,
-                  const int *__restrict__ pos, const float *__restrict__ q,
+                  const int *__restrict__ pos, const int *__restrict__ t_seq,
+                  const float *__restrict__ q,
                   const T *__restrict__ base, long seq_stride, long head_stride, long v_offset,
                   float *__restrict__ part, int *__restrict__ counters, T *__restrict__ out,
-                  float scale, int *err, L2Prefetch pf) {
+                  float scale, int *err) {
   using S = AttnShape<T, DH, TB>;
   constexpr int KT = S::KT, VEC = S::VEC, LPK = S::LPK, KPP = S::KPP, P = S::P, PG = S::PG;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -162,15 +165,23 @@ __global__ void __launch_bounds__((NC + 1) * 32)
   int *s_pos = s_abort + 4, *s_ready = s_pos + ATTN_SMEM_ROWS;
 
   pdl_trigger();
-  pdl_wait();  // q, the ring slot of t and the positions come from earlier kernels
+  // Positions: by row from `pos` (written by an earlier kernel: wait first),
+  // or t_seq[ready[i]] (steady through a decoder step: no wait needed yet).
+  const bool early = t_seq != nullptr;
+  if (!early) pdl_wait();
   const int n = *n_dev;
   const bool cached = n <= ATTN_SMEM_ROWS;
   if (cached) {  // the unit walk reads positions and slots from shared memory
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      s_pos[i] = pos[i];
-      s_ready[i] = ready[i];
+      const int sq = ready[i];
+      s_pos[i] = early ? t_seq[sq] : pos[i];
+      s_ready[i] = sq;
     }
+  } else if (early) {
+    // no room for the positions: they come from `pos`, after the wait
+    pdl_wait();
   }
+  const bool pre = early && cached;  // K/V copies may start before the wait
   const AttnGeom g{n, H, window, CH, xchunks, n_grid * H * xchunks, cached ? s_ready : ready,
                    cached ? s_pos : pos, base, seq_stride, head_stride};
   const int stride = gridDim.x * NC;  // consumer warps in the grid
@@ -188,24 +199,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
 
   if (warp == NC) {
     // ---------------------------------------------------------- producer
-    if (lane != 0) {
-      // lanes 1..31 of every producer warp share the L2 prefetch, 64 KB pieces
-      constexpr unsigned PIECE = 64u << 10;
-      const long worker = (long)blockIdx.x * 31 + (lane - 1), workers = (long)gridDim.x * 31;
-      long base_piece = 0;
-      for (int r = 0; r < 6; r++) {
-        if (!pf.p[r] || !pf.n[r]) continue;
-        const long pieces = (long)((pf.n[r] + PIECE - 1) / PIECE);
-        for (long c = ((worker - base_piece) % workers + workers) % workers; c < pieces;
-             c += workers) {
-          const unsigned long long off = (unsigned long long)c * PIECE;
-          const unsigned long long len = pf.n[r] - off < PIECE ? pf.n[r] - off : PIECE;
-          bulk_prefetch_l2(pf.p[r] + off, (unsigned)len);
-        }
-        base_piece += pieces;
-      }
-      return;
-    }
+    if (lane != 0) return;
     const uint64_t kv_policy = l2_evict_first_policy();
     UnitWalk<T, KT> wk[NC];
     int issued[NC];
@@ -216,6 +210,46 @@ __global__ void __launch_bounds__((NC + 1) * 32)
       wk[w].seek(g, stride);
       issued[w] = 0;
       ended[w] = false;
+    }
+    if (pre) {
+      // before the dependency wait: K/V of the first stages of every warp,
+      // up to the first tile that holds a row this step writes; the queries
+      // of the unit-first stages follow after the wait
+      static_assert(NC * SW <= 32, "pending queries fit one mask");
+      unsigned qpend = 0;  // stages whose query follows after the wait
+      for (int w = 0; w < NC; w++) {
+        UnitWalk<T, KT> &x = wk[w];
+        while (issued[w] < SW && !x.done()) {
+          const int row0 = x.r0 + x.j * KT;
+          const int rows = min(KT, x.r1 - row0);
+          if (x.dep_row >= row0 && x.dep_row < row0 + rows) break;
+          const int s = w * SW + issued[w];
+          uint8_t *st = smem + (size_t)s * S::STAGE;
+          const bool first = x.j == 0;
+          AttnHdr *hd = reinterpret_cast<AttnHdr *>(st);
+          hd->ih = x.ih;
+          hd->c = x.c;
+          hd->rows = rows;
+          hd->flags = (first ? 1 : 0) | (x.j + 1 == x.ntiles ? 2 : 0);
+          hd->nch = x.nch;
+          const unsigned bytes = (unsigned)(rows * DH * (int)sizeof(T));
+          mbar_expect_tx(&full[s], 2 * bytes + (first ? S::QB : 0));
+          if (first) qpend |= 1u << s;
+          bulk_g2s_hint(st + S::HDR + S::QB, x.K + (size_t)row0 * DH, bytes, &full[s],
+                        kv_policy);
+          bulk_g2s_hint(st + S::HDR + S::QB + S::TILE, x.K + v_offset + (size_t)row0 * DH,
+                        bytes, &full[s], kv_policy);
+          issued[w]++;
+          x.next(g, stride);
+        }
+      }
+      pdl_wait();  // q and the ring slot of t are now written
+      for (int s = 0; s < NC * SW; s++)
+        if (qpend >> s & 1) {
+          uint8_t *st = smem + (size_t)s * S::STAGE;
+          bulk_g2s(st + S::HDR, q + (size_t)reinterpret_cast<const AttnHdr *>(st)->ih * DH,
+                   S::QB, &full[s]);
+        }
     }
     uint64_t t0 = globaltimer_ns();
     while (live > 0) {
@@ -310,9 +344,12 @@ __global__ void __launch_bounds__((NC + 1) * 32)
 #pragma unroll
           for (int v = 0; v < VEC; v++) kf[v] = vf[p][v] = 0.f;
         }
-        float d0 = 0.f;
+        // dot product on the packed fp32 pipe (two partial sums)
+        float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int v = 0; v < VEC; v++) d0 = fmaf(qr[v], kf[v], d0);
+        for (int v = 0; v < VEC; v += 2)
+          d2 = __ffma2_rn(make_float2(qr[v], qr[v + 1]), make_float2(kf[v], kf[v + 1]), d2);
+        float d0 = d2.x + d2.y;
 #pragma unroll
         for (int o = 1; o < LPK; o <<= 1) d0 += __shfl_xor_sync(FULL_MASK, d0, o);
         sc[p] = row < hd.rows ? d0 : -INFINITY;
@@ -322,14 +359,23 @@ __global__ void __launch_bounds__((NC + 1) * 32)
         const float mn = fmaxf(st.m, mt);
         const float cr = exp2f(st.m - mn);  // st.m = -inf gives 0
         st.l *= cr;
+        float2 acc2[VEC / 2];
 #pragma unroll
-        for (int v = 0; v < VEC; v++) st.acc[v] *= cr;
+        for (int v = 0; v < VEC; v += 2)
+          acc2[v / 2] = __fmul2_rn(make_float2(st.acc[v], st.acc[v + 1]), make_float2(cr, cr));
 #pragma unroll
         for (int p = 0; p < PG; p++) {
           const float e = exp2f(sc[p] - mn);  // masked keys give 0
           st.l += e;
 #pragma unroll
-          for (int v = 0; v < VEC; v++) st.acc[v] = fmaf(e, vf[p][v], st.acc[v]);
+          for (int v = 0; v < VEC; v += 2)
+            acc2[v / 2] = __ffma2_rn(make_float2(e, e), make_float2(vf[p][v], vf[p][v + 1]),
+                                     acc2[v / 2]);
+        }
+#pragma unroll
+        for (int v = 0; v < VEC; v += 2) {
+          st.acc[v] = acc2[v / 2].x;
+          st.acc[v + 1] = acc2[v / 2].y;
         }
         st.m = mn;
       }

@@ -448,7 +448,7 @@ template <typename T> struct W_ {
 template <typename T, int DH>
 cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunks,
                         const T *base, long seq_stride, long head_stride, long v_offset,
-                        T *out, const L2Prefetch &pf, cudaStream_t st) {
+                        T *out, cudaStream_t st) {
   constexpr int smem = attn_smem_bytes<T, DH>();
   const Layout &L = M->L;
   const rlt_config &c = M->cfg;
@@ -458,10 +458,11 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
   return launch_k(k_attn_decode<T, DH>, dim3(grid), dim3((AttnCfg::NC + 1) * 32), smem, st,
                   M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks,
                   si.n_grid, M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0,
-                  M->at<float>(L.q) + r0 * c.d, base, seq_stride, head_stride, v_offset,
+                  (const int *)M->at<int>(L.t_dec), M->at<float>(L.q) + r0 * c.d, base,
+                  seq_stride, head_stride, v_offset,
                   M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
                   M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH),
-                  M->at<int>(L.err), pf);
+                  M->at<int>(L.err));
 }
 
 // fp32 models: exact SIMT GEMMs with separate RMSNorm and rotary kernels.
@@ -526,11 +527,8 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
     {
       Span sp(M, st, RLT_K_SWA, si.sum_win * 2.0 * d * es + nr * d * (4 + es),
               4.0 * d * si.sum_win);
-      // while the SWA streams the ring, pull the next two GEMMs' weights into L2
-      const L2Prefetch pf{{(const char *)W_<T>::o(M, l), (const char *)M->w.dec_wqx[l]},
-                          {(unsigned long long)(d * d * es), (unsigned long long)(d * d * es)}};
       RLT_TRY((launch_attn<T, DH>(M, si, W, 1, ring_l, (long)H * 2 * W * DH, 2L * W * DH,
-                                  (long)W * DH, a, pf, st)));
+                                  (long)W * DH, a, st)));
     }
     RLT_TRY(G(RLT_K_GEMM, d, d, a_b, W_<T>::o(M, l), EpiResid{h, d}));
     // cross-attention sublayer over M<=t
@@ -542,21 +540,8 @@ cudaError_t step_impl(rlt_model *M, const StepInfo &si, cudaStream_t st) {
     RLT_TRY(G(RLT_K_GEMM, d, d, u_b, (const T *)M->w.dec_wqx[l], EpiStoreF32{q, d}));
     {
       Span sp(M, st, RLT_K_XATTN, si.sum_keys * 2.0 * d * es, 4.0 * d * si.sum_keys);
-      // while the memory streams, pull the rest of this layer's and the next
-      // layer's first weights into L2 (the gate and q/k/v of the next step
-      // after the last layer)
-      const bool last_l = l + 1 == c.n_dec_layers;
-      const unsigned long long dd = (unsigned long long)(d * d * es),
-                               fd = (unsigned long long)(F * d * es);
-      const L2Prefetch pf{
-          {(const char *)M->w.dec_wox[l], (const char *)W_<T>::w1(M, l),
-           c.ffn_kind == RLT_SWIGLU ? (const char *)W_<T>::wb(M, l) : nullptr,
-           (const char *)W_<T>::w2(M, l),
-           (const char *)(last_l ? W_<T>::qkv(M, 0) : W_<T>::qkv(M, l + 1)),
-           a0 || !last_l ? nullptr : (const char *)M->w.gate_w},
-          {dd, fd, fd, fd, 3 * dd, 2 * dd}};
       RLT_TRY((launch_attn<T, DH>(M, si, 0, si.xchunks, mem_g, (long)H * 2 * c.max_len * DH,
-                                  2L * c.max_len * DH, (long)c.max_len * DH, a, pf, st)));
+                                  2L * c.max_len * DH, (long)c.max_len * DH, a, st)));
     }
     RLT_TRY(G(RLT_K_GEMM, d, d, a_b, (const T *)M->w.dec_wox[l], EpiResid{h, d}));
     // FFN sublayer
@@ -616,7 +601,6 @@ cudaError_t step_impl_tc(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   const int rows_blocks = blocks_for((long)n * 32, 256);
   const double nr = si.n;  // real rows, for the algorithmic byte counts
   const RowScaleIn rsi{nsq, np, 1.0f / (float)d, eps};
-  const L2Prefetch no_pf{};
   const float *const *ln1 = (const float *const *)M->w.dec_ln1;
   // y = A_rows(r0..) W^T with A one of the whole activation buffers above
   auto G = [&](auto bn, int nn, int k, const T *A_base, const T *B, auto epi) {
@@ -650,7 +634,7 @@ cudaError_t step_impl_tc(rlt_model *M, const StepInfo &si, cudaStream_t st) {
       Span sp(M, st, RLT_K_SWA, si.sum_win * 2.0 * d * es + nr * d * (4 + es),
               4.0 * d * si.sum_win);
       RLT_TRY((launch_attn<T, DH>(M, si, W, 1, ring_l, (long)H * 2 * W * DH, 2L * W * DH,
-                                  (long)W * DH, M->at<T>(L.a) + r0 * d, no_pf, st)));
+                                  (long)W * DH, M->at<T>(L.a) + r0 * d, st)));
     }
     RLT_TRY(G(BN32{}, d, d, a_b, W_<T>::o(M, l),
               EpiResidNorm<T>{{}, h, d, (const float *)M->w.dec_ln2[l], u, nsq, np}));
@@ -660,7 +644,7 @@ cudaError_t step_impl_tc(rlt_model *M, const StepInfo &si, cudaStream_t st) {
       Span sp(M, st, RLT_K_XATTN, si.sum_keys * 2.0 * d * es, 4.0 * d * si.sum_keys);
       RLT_TRY((launch_attn<T, DH>(M, si, 0, si.xchunks, mem_g, (long)H * 2 * c.max_len * DH,
                                   2L * c.max_len * DH, (long)c.max_len * DH,
-                                  M->at<T>(L.a) + r0 * d, no_pf, st)));
+                                  M->at<T>(L.a) + r0 * d, st)));
     }
     RLT_TRY(G(BN32{}, d, d, a_b, (const T *)M->w.dec_wox[l],
               EpiResidNorm<T>{{}, h, d, (const float *)M->w.dec_ln3[l], u, nsq, np}));
@@ -1074,11 +1058,11 @@ cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengt
   (void)ctas;
   k_attn_decode<T, DH><<<grid, (AttnCfg::NC + 1) * 32, smem, st>>>(
       reinterpret_cast<int *>(ws + w.err) + 1, H, 0, XCH, xchunks, max_chunks, n,
-      reinterpret_cast<int *>(ws + w.ready), reinterpret_cast<int *>(ws + w.pos), q,
-      static_cast<const T *>(kv), (long)H * 2 * cap * DH, 2L * cap * DH, (long)cap * DH,
-      reinterpret_cast<float *>(ws + w.part), reinterpret_cast<int *>(ws + w.counters),
-      static_cast<T *>(out), 1.0f / sqrtf((float)DH), reinterpret_cast<int *>(ws + w.err),
-      L2Prefetch{});
+      reinterpret_cast<int *>(ws + w.ready), reinterpret_cast<int *>(ws + w.pos),
+      (const int *)nullptr, q, static_cast<const T *>(kv), (long)H * 2 * cap * DH,
+      2L * cap * DH, (long)cap * DH, reinterpret_cast<float *>(ws + w.part),
+      reinterpret_cast<int *>(ws + w.counters), static_cast<T *>(out),
+      1.0f / sqrtf((float)DH), reinterpret_cast<int *>(ws + w.err));
   return cudaGetLastError();
 }
 
