@@ -95,9 +95,13 @@ struct AttnGeom {
 };
 
 // Producer-side walk over one consumer warp's units and their tiles.
+// The tile holding the ring row this step writes (SWA: slot t mod W) is
+// walked last, so the tiles before it can be copied before the dependency
+// wait; the order depends on t only.
 template <typename T, int KT> struct UnitWalk {
   int u, j, ntiles, nch, ih, c, r0, r1;
-  int dep_row;  // SWA: ring row written by this step (slot t mod W), else -1
+  int dep_row;   // SWA: ring row written by this step (slot t mod W), else -1
+  int dep_tile;  // tile of this chunk holding dep_row, or ntiles (none)
   const T *K;
   __device__ bool load(const AttnGeom &g) {
     const int pairs = g.units / g.xchunks;  // n_grid * H
@@ -113,6 +117,7 @@ template <typename T, int KT> struct UnitWalk {
     r1 = min(L, r0 + g.CH);
     dep_row = g.window > 0 ? t % g.window : -1;
     ntiles = (r1 - r0 + KT - 1) / KT;
+    dep_tile = dep_row >= r0 && dep_row < r1 ? (dep_row - r0) / KT : ntiles;
     j = 0;
     const int seq = g.ready[i];
     K = static_cast<const T *>(g.base) + (size_t)seq * g.seq_stride + (size_t)h * g.head_stride;
@@ -128,6 +133,13 @@ template <typename T, int KT> struct UnitWalk {
     seek(g, stride);
   }
   __device__ bool done() const { return ntiles == 0; }
+  // first row of the j-th tile walked
+  __device__ int row0() const {
+    const int k = j < dep_tile ? j : (j + 1 < ntiles ? j + 1 : dep_tile);
+    return r0 + k * KT;
+  }
+  // the j-th tile walked is the one this step writes into
+  __device__ bool dependent() const { return dep_tile < ntiles && j + 1 == ntiles; }
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -220,9 +232,9 @@ __global__ void __launch_bounds__((NC + 1) * 32)
       for (int w = 0; w < NC; w++) {
         UnitWalk<T, KT> &x = wk[w];
         while (issued[w] < SW && !x.done()) {
-          const int row0 = x.r0 + x.j * KT;
+          if (x.dependent()) break;
+          const int row0 = x.row0();
           const int rows = min(KT, x.r1 - row0);
-          if (x.dep_row >= row0 && x.dep_row < row0 + rows) break;
           const int s = w * SW + issued[w];
           uint8_t *st = smem + (size_t)s * S::STAGE;
           const bool first = x.j == 0;
@@ -269,7 +281,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
           live--;
           continue;
         }
-        const int row0 = x.r0 + x.j * KT;
+        const int row0 = x.row0();
         const int rows = min(KT, x.r1 - row0);
         const bool first = x.j == 0;
         AttnHdr *hd = reinterpret_cast<AttnHdr *>(st);

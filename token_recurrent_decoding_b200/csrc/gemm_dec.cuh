@@ -8,12 +8,15 @@
 // each. Grid (N/BN, row tiles of 128, S) with a thread-block cluster of S
 // CTAs along z: CTA z of a cluster runs K blocks [z*KB/S, (z+1)*KB/S) of one
 // 128 x BN output tile into its own TMEM accumulator (warp 0 streams the A
-// and B tiles with TMA, warp 1 issues tcgen05.mma), then all four warps copy
-// the fp32 partial tile from TMEM to shared memory. After a cluster barrier
+// and B tiles with TMA, warp 1 issues tcgen05.mma), then all eight warps copy
+// the fp32 partial tile from TMEM to shared memory (warp w: TMEM lanes of
+// warp w mod 4, column half w / 4). After a cluster barrier
 // CTA z owns a contiguous share of the tile's valid rows: it sums the S
 // partials of those rows over distributed shared memory in rank order (so a
 // result never depends on the batch size or on timing) and applies the
-// epilogue with threads laid along the columns (coalesced stores). A second
+// epilogue with threads laid along the columns (coalesced stores; four
+// columns per thread and slot, S a template parameter so the rank loops
+// unroll: the reduction is instruction-bound, not memory-bound). A second
 // cluster barrier keeps every CTA's shared memory alive until its peers have
 // read it. S is a function of N and K only.
 //
@@ -53,6 +56,16 @@ __device__ __forceinline__ void cluster_sync_all() {
           : "memory");
 }
 
+// Cluster barrier without release semantics: it only marks that this
+// thread's reads of its peers' shared memory are done (their values have
+// been used), and does not wait for its own global stores to be performed.
+__device__ __forceinline__ void cluster_sync_relaxed() {
+  asm volatile(
+      "barrier.cluster.arrive.relaxed.aligned;\n"
+      "barrier.cluster.wait.aligned;\n" ::
+          : "memory");
+}
+
 // Address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
@@ -60,10 +73,10 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ float2 ld_dsmem_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];\n"
-               : "=f"(v.x), "=f"(v.y)
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr)
                : "memory");
   return v;
@@ -74,7 +87,7 @@ __device__ __forceinline__ float2 ld_dsmem_f2(uint32_t addr) {
 // kRope:  v(row, col..col+1) and the same columns
 //         half a head further on (rotate-half)      -> epi.rotary(row, col, a0, a1, b0, b1, r)
 // kNorm:  like kPair; epi.pair returns its share of the row's sum of squares,
-//         the kernel adds the shares of a row's BN/2 threads (shuffle tree)
+//         the kernel adds the shares of a row's BN/4 threads (shuffle tree)
 //         and hands the total to epi.row_sum(row, column tile, ss)
 enum DecEpiKind { kPair = 0, kRope = 1, kNorm = 2 };
 
@@ -234,7 +247,9 @@ template <int BN> struct DecSmem {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int P_LD = BN + 2;  // fp32 partial tile row stride (8-byte aligned pairs)
+  // fp32 partial tile row stride: 16-byte aligned rows, and the float4
+  // stores of 8 consecutive rows hit distinct banks
+  static constexpr int P_LD = BN + 4;
   static constexpr int P_BYTES = TC_BM * P_LD * 4;
   // dynamic bytes for `ns` ring stages: alignment slack + barriers + the
   // larger of the ring and the partial tile (which reuses the ring)
@@ -244,20 +259,26 @@ template <int BN> struct DecSmem {
 };
 
 // Cluster split count of a decode GEMM: about one CTA per SM over the N
-// tiles, at most 8 (the portable cluster size) and at most one per K block.
+// tiles, at most 8 (the portable cluster size) and at most one per K block,
+// rounded down to one of the compiled counts 1, 2, 3, 4, 6, 8.
 inline int dec_splits(int n_tiles, int kb, int num_sms) {
   int s = num_sms / (n_tiles > 0 ? n_tiles : 1);
   if (s > 8) s = 8;
   if (s > kb) s = kb;
+  if (s == 5) s = 4;
+  if (s == 7) s = 6;
   return s < 1 ? 1 : s;
 }
 
-template <int BN, int STAGES, class Epi>
-__global__ void __launch_bounds__(128, 2)
+constexpr int DEC_THREADS = 256;
+
+template <int BN, int STAGES, int S, class Epi>
+__global__ void __launch_bounds__(DEC_THREADS, 2)
     k_gemm_dec(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const int *__restrict__ Mdev, int a_row0, int N, int K, int ns, Epi epi,
                int *err) {
   static_assert(BN == 32 || BN == 64 || BN == 128, "TMEM columns are a power of two >= 32");
+  static_assert(S >= 1 && S <= 8, "portable cluster size");
   using SM = DecSmem<BN>;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -276,7 +297,6 @@ __global__ void __launch_bounds__(128, 2)
   // the step's row count is staged before its first kernel starts
   const int M = *Mdev;
   if (m0 >= M) return;  // the whole cluster (same blockIdx.y), before any barrier
-  const int S = gridDim.z;
   const int z = (int)cluster_ctarank();
   const int kb_all = K / TC_BK;
   const int kb0 = z * kb_all / S, KB = (z + 1) * kb_all / S - kb0;
@@ -342,10 +362,10 @@ __global__ void __launch_bounds__(128, 2)
     }
     umma_commit(accum);
   } else if (Epi::kRowScale && warp >= 2) {
-    // warps 2-3: row scales of this CTA's share of rows, from the partial
+    // warps 2-7: row scales of this CTA's share of rows, from the partial
     // sums of squares the producer of the input wrote (column tile order)
     pdl_wait();
-    for (int i = threadIdx.x - 64; i < r_hi - r_lo; i += 64) {
+    for (int i = threadIdx.x - 64; i < r_hi - r_lo; i += DEC_THREADS - 64) {
       const float *p = epi.rsi.nsq + (size_t)(m0 + r_lo + i) * epi.rsi.np;
       float ss = 0.f;
       for (int t = 0; t < epi.rsi.np; t++) ss += p[t];
@@ -361,16 +381,18 @@ __global__ void __launch_bounds__(128, 2)
   if (!acc_ok) atomicExch(&s_fail, 1);
   __syncthreads();
   const bool ok = !s_fail;
-  if (ok && warp * 32 < rv) {
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 16) {
+  const int lg = warp & 3, ch = warp >> 2;  // TMEM lane group, column half
+  if (ok && lg * 32 < rv) {
+    const int row = lg * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(lg * 32) << 16);
+#pragma unroll
+    for (int c0 = ch * (BN / 2); c0 < (ch + 1) * (BN / 2); c0 += 16) {
       float v[16];
       tmem_ld16(lane_base + c0, v);
-      float2 *pr = reinterpret_cast<float2 *>(P + (size_t)row * SM::P_LD + c0);
+      float4 *pr = reinterpret_cast<float4 *>(P + (size_t)row * SM::P_LD + c0);
 #pragma unroll
-      for (int j = 0; j < 8; j++) pr[j] = make_float2(v[2 * j], v[2 * j + 1]);
+      for (int j = 0; j < 4; j++)
+        pr[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     }
   }
   tc_fence_before();
@@ -380,51 +402,61 @@ __global__ void __launch_bounds__(128, 2)
     if (threadIdx.x == 0) set_error(err, DEV_ERR_TIMEOUT);
   } else {
     const uint32_t p_local = smem_u32(P);
-    uint32_t p_rank[8];
+    uint32_t p_rank[S];
 #pragma unroll
-    for (int q = 0; q < 8; q++) p_rank[q] = q < S ? mapa_shared(p_local, q) : 0u;
-    const int rows = r_hi - r_lo;
-    auto sum_at = [&](int r, int c) {
-      float2 acc = make_float2(0.f, 0.f);
+    for (int q = 0; q < S; q++) p_rank[q] = mapa_shared(p_local, q);
+    // sum of the S partials of four columns, rank order; all S loads are
+    // issued before the first add
+    auto sum4 = [&](int r, int c) {
       const uint32_t off = (uint32_t)((r * SM::P_LD + c) * 4);
+      float4 v[S];
 #pragma unroll
-      for (int q = 0; q < 8; q++)
-        if (q < S) {
-          const float2 p = ld_dsmem_f2(p_rank[q] + off);
-          acc.x += p.x;
-          acc.y += p.y;
-        }
+      for (int q = 0; q < S; q++) v[q] = ld_dsmem_f4(p_rank[q] + off);
+      float4 acc = v[0];
+#pragma unroll
+      for (int q = 1; q < S; q++) {
+        acc.x += v[q].x;
+        acc.y += v[q].y;
+        acc.z += v[q].z;
+        acc.w += v[q].w;
+      }
       return acc;
     };
+    const int rows = r_hi - r_lo;
     if constexpr (Epi::kKind == kRope) {
       const int DH = epi.DH, half = DH / 2;
-      constexpr int PPR = BN / 4;  // first-half column pairs per row
-      for (int idx = threadIdx.x; idx < rows * PPR; idx += blockDim.x) {
+      constexpr int PPR = BN / 8;  // four-column slots of the first halves, per row
+      for (int idx = threadIdx.x; idx < rows * PPR; idx += DEC_THREADS) {
         const int rl = idx / PPR, p = idx - rl * PPR;
-        const int hh = (2 * p) / half, j = 2 * p - hh * half;
+        const int hh = (4 * p) / half, j = 4 * p - hh * half;
         const int c = hh * DH + j, r = r_lo + rl;
-        const float2 a = sum_at(r, c), b = sum_at(r, c + half);
-        epi.rotary(m0 + r, n0 + c, a.x, a.y, b.x, b.y, Epi::kRowScale ? s_rs[rl] : 1.f);
+        const float4 a = sum4(r, c), b = sum4(r, c + half);
+        const float sc = Epi::kRowScale ? s_rs[rl] : 1.f;
+        epi.rotary(m0 + r, n0 + c, a.x, a.y, b.x, b.y, sc);
+        epi.rotary(m0 + r, n0 + c + 2, a.z, a.w, b.z, b.w, sc);
       }
     } else {
-      constexpr int PPR = BN / 2;  // column pairs per row
+      constexpr int PPR = BN / 4;  // four-column slots per row
       const int total = rows * PPR;
       // uniform trip count: the row sums shuffle over a row's PPR lanes
-      for (int b0 = 0; b0 < total; b0 += blockDim.x) {
+      for (int b0 = 0; b0 < total; b0 += DEC_THREADS) {
         const int idx = b0 + threadIdx.x;
         const bool act = idx < total;
         const int rl = act ? idx / PPR : 0, p = idx - (idx / PPR) * PPR;
         float ss = 0.f;
         if (act) {
-          const float2 v = sum_at(r_lo + rl, 2 * p);
-          const float r = Epi::kRowScale ? s_rs[rl] : 1.f;
-          if constexpr (Epi::kKind == kNorm)
-            ss = epi.pair(m0 + r_lo + rl, n0 + 2 * p, v.x, v.y, r);
-          else
-            epi.pair(m0 + r_lo + rl, n0 + 2 * p, v.x, v.y, r);
+          const float4 v = sum4(r_lo + rl, 4 * p);
+          const float sc = Epi::kRowScale ? s_rs[rl] : 1.f;
+          const int m = m0 + r_lo + rl, n = n0 + 4 * p;
+          if constexpr (Epi::kKind == kNorm) {
+            ss = epi.pair(m, n, v.x, v.y, sc) + epi.pair(m, n + 2, v.z, v.w, sc);
+          } else {
+            epi.pair(m, n, v.x, v.y, sc);
+            epi.pair(m, n + 2, v.z, v.w, sc);
+          }
         }
         if constexpr (Epi::kKind == kNorm) {
-          static_assert(PPR == 16 || PPR == 32, "row groups of a half or a whole warp");
+          static_assert(PPR == 8 || PPR == 16 || PPR == 32, "row groups inside a warp");
 #pragma unroll
           for (int o = PPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
           if (act && p == 0) epi.row_sum(m0 + r_lo + rl, blockIdx.x, ss);
@@ -433,7 +465,7 @@ __global__ void __launch_bounds__(128, 2)
     }
   }
   tc_fence_before();
-  cluster_sync_all();  // peers are done reading this CTA's partial tile
+  cluster_sync_relaxed();  // peers are done reading this CTA's partial tile
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, BN);
 }

@@ -306,23 +306,16 @@ cudaError_t gemm_tc(rlt_model *M, int m_grid, int a_rows, int a_row0, int n, int
   return launch_tc<32, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
 }
 
-// Decode-step GEMM (gemm_dec.cuh): rows [a_row0 + m, ...) of A [a_rows][k]
-// times B [n][k] with BN-wide output tiles and a cluster of S split-K CTAs
-// per tile; m_grid bounds the rows, Mdev holds the row count at run time.
-template <int BN, class Epi>
-cudaError_t launch_dec(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
-                       int k, const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
+// One decode GEMM launch with a compile-time cluster split count S.
+template <int BN, int S, class Epi>
+cudaError_t launch_dec_s(rlt_model *M, int m_grid, const int *Mdev, int a_row0, int n, int k,
+                         const CUtensorMap &ma, const CUtensorMap &mb, Epi epi,
+                         cudaStream_t st) {
   constexpr int STAGES = 4;
-  if (m_grid <= 0) return cudaSuccess;
-  if (n % BN || k % TC_BK) return cudaErrorInvalidValue;
   const int kb = k / TC_BK, tiles = n / BN;
-  const int S = dec_splits(tiles, kb, M->num_sms);
   const int kb_max = (kb + S - 1) / S;
   const int ns = kb_max < STAGES ? kb_max : STAGES;
-  const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
-  const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
-  if (!ma || !mb) return cudaErrorInvalidValue;
-  auto kern = k_gemm_dec<BN, STAGES, Epi>;
+  auto kern = k_gemm_dec<BN, STAGES, S, Epi>;
   static bool attr = false;
   if (!attr) {
     RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -331,7 +324,7 @@ cudaError_t launch_dec(rlt_model *M, int m_grid, const int *Mdev, int a_rows, in
   }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(tiles, (m_grid + TC_BM - 1) / TC_BM, S);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(DEC_THREADS);
   cfg.dynamicSmemBytes = DecSmem<BN>::bytes(ns);
   cfg.stream = st;
   cudaLaunchAttribute at[2];
@@ -347,8 +340,29 @@ cudaError_t launch_dec(rlt_model *M, int m_grid, const int *Mdev, int a_rows, in
   }
   cfg.attrs = at;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, *ma, *mb, Mdev, a_row0, n, k, ns, epi,
+  return cudaLaunchKernelEx(&cfg, kern, ma, mb, Mdev, a_row0, n, k, ns, epi,
                             M->at<int>(M->L.err));
+}
+
+// Decode-step GEMM (gemm_dec.cuh): rows [a_row0 + m, ...) of A [a_rows][k]
+// times B [n][k] with BN-wide output tiles and a cluster of S split-K CTAs
+// per tile; m_grid bounds the rows, Mdev holds the row count at run time.
+template <int BN, class Epi>
+cudaError_t launch_dec(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
+                       int k, const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
+  if (m_grid <= 0) return cudaSuccess;
+  if (n % BN || k % TC_BK) return cudaErrorInvalidValue;
+  const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
+  const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
+  if (!ma || !mb) return cudaErrorInvalidValue;
+  switch (dec_splits(n / BN, k / TC_BK, M->num_sms)) {
+    case 1: return launch_dec_s<BN, 1>(M, m_grid, Mdev, a_row0, n, k, *ma, *mb, epi, st);
+    case 2: return launch_dec_s<BN, 2>(M, m_grid, Mdev, a_row0, n, k, *ma, *mb, epi, st);
+    case 3: return launch_dec_s<BN, 3>(M, m_grid, Mdev, a_row0, n, k, *ma, *mb, epi, st);
+    case 4: return launch_dec_s<BN, 4>(M, m_grid, Mdev, a_row0, n, k, *ma, *mb, epi, st);
+    case 6: return launch_dec_s<BN, 6>(M, m_grid, Mdev, a_row0, n, k, *ma, *mb, epi, st);
+    default: return launch_dec_s<BN, 8>(M, m_grid, Mdev, a_row0, n, k, *ma, *mb, epi, st);
+  }
 }
 
 cudaEvent_t take_event(rlt_model *M) {
