@@ -167,7 +167,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
                   const float *__restrict__ q,
                   const T *__restrict__ base, long seq_stride, long head_stride, long v_offset,
                   float *__restrict__ part, int *__restrict__ counters, T *__restrict__ out,
-                  float scale, int *err) {
+                  float scale, int kv_reuse, int *err) {
   using S = AttnShape<T, DH, TB>;
   constexpr int KT = S::KT, VEC = S::VEC, LPK = S::LPK, KPP = S::KPP, P = S::P, PG = S::PG;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -212,7 +212,9 @@ __global__ void __launch_bounds__((NC + 1) * 32)
   if (warp == NC) {
     // ---------------------------------------------------------- producer
     if (lane != 0) return;
-    const uint64_t kv_policy = l2_evict_first_policy();
+    // K/V read once per step leave L2 first; a block every decoder layer
+    // reads again (one memory group for all layers) keeps the normal policy
+    const uint64_t kv_policy = kv_reuse ? l2_evict_normal_policy() : l2_evict_first_policy();
     UnitWalk<T, KT> wk[NC];
     int issued[NC];
     bool ended[NC];

@@ -139,6 +139,12 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+__device__ __forceinline__ uint64_t l2_evict_normal_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
+}
+
 // bulk_g2s with an L2 cache-eviction policy.
 __device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, unsigned bytes,
                                               uint64_t *bar, uint64_t policy) {

@@ -476,6 +476,7 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
                   seq_stride, head_stride, v_offset,
                   M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
                   M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH),
+                  (window == 0 && c.mem_groups == 1 && c.n_dec_layers > 1) ? 1 : 0,
                   M->at<int>(L.err));
 }
 
@@ -1076,7 +1077,7 @@ cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengt
       (const int *)nullptr, q, static_cast<const T *>(kv), (long)H * 2 * cap * DH,
       2L * cap * DH, (long)cap * DH, reinterpret_cast<float *>(ws + w.part),
       reinterpret_cast<int *>(ws + w.counters), static_cast<T *>(out),
-      1.0f / sqrtf((float)DH), reinterpret_cast<int *>(ws + w.err));
+      1.0f / sqrtf((float)DH), 0, reinterpret_cast<int *>(ws + w.err));
   return cudaGetLastError();
 }
 
