@@ -11,11 +11,27 @@
 namespace rlt {
 
 // ---------------------------------------------------------------- epilogues
+// operator()(m, n, a, b): columns n, n + 1 of row m (SIMT GEMM).
+// vec16(m, n, v): columns n .. n + 15 of row m, n a multiple of 16 (the
+// tensor-core GEMM, one TMEM row per thread): whole 16-byte vector stores,
+// so every 32-byte sector a thread touches is written in full.
+
+// 16 values of type T stored at p (16-byte aligned) with vector stores.
+template <typename T> __device__ __forceinline__ void store16(T *p, const float *v) {
+  alignas(16) T t[16];
+#pragma unroll
+  for (int i = 0; i < 16; i++) t[i] = from_f<T>(v[i]);
+#pragma unroll
+  for (int i = 0; i < (int)(16 * sizeof(T) / 16); i++)
+    reinterpret_cast<uint4 *>(p)[i] = reinterpret_cast<const uint4 *>(t)[i];
+}
+
 struct EpiStoreF32 {
   float *out; int ld;
   __device__ void operator()(int m, int n, float a, float b) const {
     *reinterpret_cast<float2 *>(out + (size_t)m * ld + n) = make_float2(a, b);
   }
+  __device__ void vec16(int m, int n, const float *v) const { store16(out + (size_t)m * ld + n, v); }
 };
 
 template <typename T> struct EpiStore {
@@ -35,6 +51,16 @@ struct EpiResid {
     v.x += a; v.y += b;
     *p = v;
   }
+  __device__ void vec16(int m, int n, const float *v) const {
+    float4 *p = reinterpret_cast<float4 *>(h + (size_t)m * ld + n);
+    float4 x[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) x[i] = p[i];
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+      p[i] = make_float4(x[i].x + v[4 * i], x[i].y + v[4 * i + 1], x[i].z + v[4 * i + 2],
+                         x[i].w + v[4 * i + 3]);
+  }
 };
 
 template <typename T> struct EpiGelu {
@@ -42,6 +68,12 @@ template <typename T> struct EpiGelu {
   __device__ void operator()(int m, int n, float a, float b) const {
     out[(size_t)m * ld + n] = from_f<T>(gelu_erf(a));
     out[(size_t)m * ld + n + 1] = from_f<T>(gelu_erf(b));
+  }
+  __device__ void vec16(int m, int n, const float *v) const {
+    float g[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) g[i] = gelu_erf(v[i]);
+    store16(out + (size_t)m * ld + n, g);
   }
 };
 
@@ -52,6 +84,19 @@ template <typename T> struct EpiSwiglu {
     size_t i = (size_t)m * ld + n;
     out[i] = from_f<T>(silu(a_in[i]) * a);
     out[i + 1] = from_f<T>(silu(a_in[i + 1]) * b);
+  }
+  __device__ void vec16(int m, int n, const float *v) const {
+    const float4 *pa = reinterpret_cast<const float4 *>(a_in + (size_t)m * ld + n);
+    float g[16];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const float4 x = pa[i];
+      g[4 * i] = silu(x.x) * v[4 * i];
+      g[4 * i + 1] = silu(x.y) * v[4 * i + 1];
+      g[4 * i + 2] = silu(x.z) * v[4 * i + 2];
+      g[4 * i + 3] = silu(x.w) * v[4 * i + 3];
+    }
+    store16(out + (size_t)m * ld + n, g);
   }
 };
 
@@ -75,6 +120,12 @@ template <typename T> struct EpiMem {
     size_t idx = ((((size_t)slot * H + h) * 2 + kv) * max_len + p) * DH + j;
     mem_g[idx] = from_f<T>(a);
     mem_g[idx + 1] = from_f<T>(b);
+  }
+  // 16 columns of one head (DH >= 16): contiguous in the head-major layout
+  __device__ void vec16(int m, int n, const float *v) const {
+    const int slot = tok_slot[m], p = tok_pos[m];
+    const int h = n / DH, j = n % DH;
+    store16(mem_g + ((((size_t)slot * H + h) * 2 + kv) * max_len + p) * DH + j, v);
   }
 };
 

@@ -10,8 +10,8 @@
 // instruction), releasing each stage with tcgen05.commit on its "empty"
 // barrier. After the last K block a commit on the accumulator barrier hands
 // the tile to all four warps, which read it back with tcgen05.ld (warp w owns
-// TMEM lanes 32w..32w+31 = tile rows) and apply the epilogue functor two
-// columns at a time. Every mbarrier wait is bounded in device time.
+// TMEM lanes 32w..32w+31 = tile rows) and apply the epilogue functor to 16
+// consecutive columns at a time (vector stores). Every mbarrier wait is bounded in device time.
 #pragma once
 
 #include <cuda.h>
@@ -212,17 +212,12 @@ __global__ void __launch_bounds__(128, 1)
   if (!ok) {
     if (threadIdx.x == 0) set_error(err, DEV_ERR_TIMEOUT);
   } else {
+    // N is a multiple of 16: whole 16-column groups
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 16) {
       float v[16];
       tmem_ld16(lane_base + c0, v);
-      if (row < M) {
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          const int col = n0 + c0 + j;
-          if (col < N) epi(row, col, v[j], v[j + 1]);
-        }
-      }
+      if (row < M && n0 + c0 < N) epi.vec16(row, n0 + c0, v);
     }
   }
   tc_fence_before();
