@@ -258,12 +258,16 @@ template <int BN> struct DecSmem {
   }
 };
 
-// Cluster split count of a decode GEMM: about one CTA per SM over the N
-// tiles, at most 8 (the portable cluster size) and at most one per K block,
-// rounded down to one of the compiled counts 1, 2, 3, 4, 6, 8.
+// Cluster split count of a decode GEMM, a function of N, K and the SM count
+// only: about one CTA per SM over the N tiles, at most 8 (the portable
+// cluster size), at least three K blocks per CTA once K allows four splits
+// (each further split adds partial-tile traffic over distributed shared
+// memory), rounded down to one of the compiled counts 1, 2, 3, 4, 6, 8.
 inline int dec_splits(int n_tiles, int kb, int num_sms) {
   int s = num_sms / (n_tiles > 0 ? n_tiles : 1);
   if (s > 8) s = 8;
+  const int by_k = kb / 3 > 4 ? kb / 3 : 4;
+  if (s > by_k) s = by_k;
   if (s > kb) s = kb;
   if (s == 5) s = 4;
   if (s == 7) s = 6;
