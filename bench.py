@@ -195,6 +195,25 @@ class Runner:
         if host:
             self._read_states()
 
+    def time_parallel(self, steps, warmup):
+        """Token-parallel decoder pass (feedback-off models, equal lengths):
+        encoder prefill, then all positions of every sequence at once; the
+        device time of the passes alone."""
+        torch = self.torch
+        T = int(self.lengths[0])
+        ms = []
+        for k in range(warmup + steps):
+            self.m.prefill_encoder(self.tok_dev, self.ids, self.offsets, self.lengths)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+            self.m.decoder_parallel(self.ids, T)
+            b.record(self.stream)
+            torch.cuda.synchronize()
+            if k >= warmup:
+                ms.append(a.elapsed_time(b))
+        return sum(ms) / len(ms)
+
     def _read_states(self):
         # one d2h copy per sequence of its final s into pinned host memory
         import ctypes as C
@@ -326,6 +345,18 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
     }
+    if cfg.alpha == 0.0 and not r.ragged:
+        # the feedback-off model also runs its decoder token-parallel
+        par_ms = max_over_ranks(r.time_parallel(args.steps, 1), dist)
+        pr = roofline.decoder_parallel_roofline(cfg, wl.lengths, hbm, tc)
+        out["decoder_parallel"] = {
+            "seq_steps_per_s": world * seq_steps / (par_ms / 1e3),
+            "ms_per_step": par_ms,
+            "roofline_s": pr["seconds"],
+            "frac": pr["seconds"] / (par_ms / 1e3),
+            "TFLOP_s": pr["flops"] / (par_ms / 1e3) / 1e12,
+            "bound": "tensor" if pr["flops"] / (tc * 1e12) >= pr["bytes"] / (hbm * 1e9) else "hbm",
+        }
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_positions)
     return out

@@ -171,6 +171,25 @@ RLT_API int rlt_decoder_step(rlt_model *model, const int32_t *h_ready_ids,
 RLT_API int rlt_run_sequence(rlt_model *model, const int32_t *h_seq_ids, int n,
                              int n_steps, rlt_stream stream);
 
+/* Token-parallel decoder pass for feedback off (alpha = 0). With alpha = 0
+ * the transition at t never reads s_{t-1} (x_t = e_t), so every decoder
+ * quantity at t depends only on e_0..e_t: the n_steps transitions of a fresh
+ * sequence can run for all positions at once, block by block, as a
+ * window-masked causal prefill (the feedback-off ablation of [RLT-PV]
+ * "Per-token recurrence, no quality gain" and the parallel-training argument
+ * of [RLT-FT] "How slow is per-token recurrence to train?"). The result is
+ * the recurrent state after n_steps transitions: s = s_{n_steps-1}, each
+ * layer's window of rotary k and v, t_dec = n_steps, so rlt_decoder_step
+ * continues from there. s_all (optional, device memory, fp32
+ * [n][n_steps][d], row i of sequence h_seq_ids[i]) receives every s_t.
+ * Sequences are processed in chunks of whole sequences that fit the prefill
+ * buffers (max_prefill_tokens).
+ * Errors: INVALID_ARG (bad ids, n_steps < 0, or a sequence that has already
+ * taken a decoder step), DUPLICATE_ID, NOT_READY (t_enc < n_steps),
+ * CAPACITY (n_steps > max_len), UNSUPPORTED (alpha != 0). */
+RLT_API int rlt_decoder_parallel(rlt_model *model, const int32_t *h_seq_ids, int n,
+                                 int n_steps, float *s_all, rlt_stream stream);
+
 /* Ready-set scheduler: sequence h_seq_ids[i] still needs h_steps[i]
  * transitions. Each tick batches every sequence with a pending step into one
  * decoder step, until none is left (ragged batches: sequences drop out as

@@ -9,6 +9,11 @@
 //
 // Work list: blk[4*b .. 4*b+3] = (first chunk row of the sequence, sequence
 // length, query block, unused) for CTA b of a head; blockIdx.y = head.
+// window > 0 restricts every query at position q to keys q - window + 1 .. q
+// (the decoder's sliding window in the token-parallel pass). SPLIT carries
+// the query and the softmax probabilities as bf16 high + low parts (Qlo the
+// low part of Q; two MMAs each for S and for O), about 16 mantissa bits
+// instead of 8, for the decoder whose recurrent form keeps them in fp32.
 #pragma once
 
 #include "common.cuh"
@@ -57,11 +62,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int DH>
+template <int DH, bool SPLIT = false>
 __global__ void __launch_bounds__(128)
     k_enc_flash(int ntok, const int *__restrict__ blk, const bf16 *__restrict__ Qh,
                 const bf16 *__restrict__ Kh, const bf16 *__restrict__ Vh, bf16 *__restrict__ out,
-                int H, float scale_log2) {
+                int H, float scale_log2, int window, const bf16 *__restrict__ Qlo) {
   constexpr int NCH = DH / 8;      // 16-byte chunks per row
   constexpr int KS = DH / 16;      // k-steps of QK^T
   constexpr int NT = FA_BK / 8;    // n-tiles of S per warp
@@ -93,18 +98,25 @@ __global__ void __launch_bounds__(128)
   // this warp's 16 query rows as A fragments, straight from global memory
   const int g = lane >> 2, tq = lane & 3;
   const int qr0 = q0 + warp * 16 + g, qr1 = qr0 + 8;
-  uint32_t qa[KS][4];
+  uint32_t qa[KS][4], ql[SPLIT ? KS : 1][4];
 #pragma unroll
   for (int ks = 0; ks < KS; ks++) {
     int k0 = ks * 16 + tq * 2;
-    auto ld2 = [&](int row, int col) -> uint32_t {
+    auto ld2 = [&](const bf16 *Q, int row, int col) -> uint32_t {
       if (row >= len) return 0u;
-      return *reinterpret_cast<const uint32_t *>(Qs + (size_t)row * DH + col);
+      return *reinterpret_cast<const uint32_t *>(Q + (size_t)row * DH + col);
     };
-    qa[ks][0] = ld2(qr0, k0);
-    qa[ks][1] = ld2(qr1, k0);
-    qa[ks][2] = ld2(qr0, k0 + 8);
-    qa[ks][3] = ld2(qr1, k0 + 8);
+    qa[ks][0] = ld2(Qs, qr0, k0);
+    qa[ks][1] = ld2(Qs, qr1, k0);
+    qa[ks][2] = ld2(Qs, qr0, k0 + 8);
+    qa[ks][3] = ld2(Qs, qr1, k0 + 8);
+    if constexpr (SPLIT) {
+      const bf16 *Ql = Qlo + (hb + start) * DH;
+      ql[ks][0] = ld2(Ql, qr0, k0);
+      ql[ks][1] = ld2(Ql, qr1, k0);
+      ql[ks][2] = ld2(Ql, qr0, k0 + 8);
+      ql[ks][3] = ld2(Ql, qr1, k0 + 8);
+    }
   }
 
   float o[ONT][4];
@@ -114,9 +126,12 @@ __global__ void __launch_bounds__(128)
 
   const int last_row = min(len, q0 + FA_BQ) - 1;
   const int nkb = last_row / FA_BK + 1;  // causal: key blocks up to the diagonal
-  load_kv(0, 0);
+  // window: keys q - window + 1 .. q only, so blocks before the first
+  // query's band are skipped
+  const int kb0 = window > 0 ? max(0, q0 - window + 1) / FA_BK : 0;
+  load_kv(kb0 & 1, kb0);
   cp_async_commit();
-  for (int kb = 0; kb < nkb; kb++) {
+  for (int kb = kb0; kb < nkb; kb++) {
     if (kb + 1 < nkb) load_kv((kb + 1) & 1, kb + 1);
     cp_async_commit();
     cp_async_wait<1>();
@@ -138,6 +153,10 @@ __global__ void __launch_bounds__(128)
         uint32_t b0[2] = {b4[0], b4[1]}, b1[2] = {b4[2], b4[3]};
         mma_bf16_16816(s[2 * jp], qa[ks], b0);
         mma_bf16_16816(s[2 * jp + 1], qa[ks], b1);
+        if constexpr (SPLIT) {
+          mma_bf16_16816(s[2 * jp], ql[ks], b0);
+          mma_bf16_16816(s[2 * jp + 1], ql[ks], b1);
+        }
       }
     }
     // causal / length mask and online softmax (base-2 exponent, pre-scaled)
@@ -147,8 +166,8 @@ __global__ void __launch_bounds__(128)
       int kc = kb * FA_BK + j * 8 + tq * 2;
 #pragma unroll
       for (int e = 0; e < 2; e++) {
-        bool ok0 = (kc + e) <= qr0 && (kc + e) < len;
-        bool ok1 = (kc + e) <= qr1 && (kc + e) < len;
+        bool ok0 = (kc + e) <= qr0 && (kc + e) < len && (window <= 0 || kc + e > qr0 - window);
+        bool ok1 = (kc + e) <= qr1 && (kc + e) < len && (window <= 0 || kc + e > qr1 - window);
         s[j][e] = ok0 ? s[j][e] * scale_log2 : -INFINITY;
         s[j][2 + e] = ok1 ? s[j][2 + e] * scale_log2 : -INFINITY;
         mx0 = fmaxf(mx0, s[j][e]);
@@ -165,7 +184,7 @@ __global__ void __launch_bounds__(128)
     const float base0 = (mx0 == -INFINITY) ? 0.f : mx0;
     const float base1 = (mx1 == -INFINITY) ? 0.f : mx1;
     float rs0 = 0.f, rs1 = 0.f;
-    uint32_t pa[NT / 2][4];
+    uint32_t pa[NT / 2][4], pl[SPLIT ? NT / 2 : 1][4];
 #pragma unroll
     for (int j = 0; j < NT; j++) {
       float p0 = exp2f(s[j][0] - base0), p1 = exp2f(s[j][1] - base0);
@@ -174,6 +193,11 @@ __global__ void __launch_bounds__(128)
       rs1 += p2 + p3;
       pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p0, p1);
       pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16(p2, p3);
+      if constexpr (SPLIT) {  // low parts: p minus its bf16 rounding
+        auto lo = [](float p) { return p - __bfloat162float(__float2bfloat16_rn(p)); };
+        pl[j >> 1][(j & 1) * 2 + 0] = pack_bf16(lo(p0), lo(p1));
+        pl[j >> 1][(j & 1) * 2 + 1] = pack_bf16(lo(p2), lo(p3));
+      }
     }
     rs0 += __shfl_xor_sync(FULL_MASK, rs0, 1);
     rs0 += __shfl_xor_sync(FULL_MASK, rs0, 2);
@@ -202,6 +226,11 @@ __global__ void __launch_bounds__(128)
         uint32_t b0[2] = {b4[0], b4[1]}, b1[2] = {b4[2], b4[3]};
         mma_bf16_16816(o[2 * jp], a, b0);
         mma_bf16_16816(o[2 * jp + 1], a, b1);
+        if constexpr (SPLIT) {
+          uint32_t al[4] = {pl[kk][0], pl[kk][1], pl[kk][2], pl[kk][3]};
+          mma_bf16_16816(o[2 * jp], al, b0);
+          mma_bf16_16816(o[2 * jp + 1], al, b1);
+        }
       }
     }
     __syncthreads();

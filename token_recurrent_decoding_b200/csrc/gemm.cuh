@@ -111,6 +111,33 @@ struct EpiGate {
   }
 };
 
+// Head-major store of a projection: out[h][m][j] for column n = h * DH + j
+// (the query of the token-parallel cross-attention); lo (optional) receives
+// the low part v - out of each stored value, same layout.
+template <typename T> struct EpiHeadMajor {
+  T *out; int ntok, DH; T *lo;
+  __device__ void operator()(int m, int n, float a, float b) const {
+    const size_t i = ((size_t)(n / DH) * ntok + m) * DH + n % DH;
+    out[i] = from_f<T>(a);
+    out[i + 1] = from_f<T>(b);
+    if (lo) {
+      lo[i] = from_f<T>(a - to_f(from_f<T>(a)));
+      lo[i + 1] = from_f<T>(b - to_f(from_f<T>(b)));
+    }
+  }
+  // 16 columns of one head (DH >= 16)
+  __device__ void vec16(int m, int n, const float *v) const {
+    const size_t i = ((size_t)(n / DH) * ntok + m) * DH + n % DH;
+    store16(out + i, v);
+    if (lo) {
+      float r[16];
+#pragma unroll
+      for (int k = 0; k < 16; k++) r[k] = v[k] - to_f(from_f<T>(v[k]));
+      store16(lo + i, r);
+    }
+  }
+};
+
 // Memory projection: token row m (slot, position) -> head-major M.
 template <typename T> struct EpiMem {
   T *mem_g; const int *tok_slot; const int *tok_pos; int H, DH, max_len, kv;

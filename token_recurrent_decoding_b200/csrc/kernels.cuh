@@ -246,6 +246,79 @@ __global__ void k_step_final(const int *__restrict__ n_dev, int d, const int *__
   if (lane == 0) t_dec[seq] += 1;
 }
 
+// ------------------------------------------- token-parallel decoder pass
+// (feedback off: the transition at t reads e_t, the memory prefix and the
+// layer's own window, never s_{t-1}). Tokens are staged as for the encoder:
+// row m = (slot, position), each sequence's positions contiguous from 0.
+
+// h[m] = e_t of the token's sequence and position.
+template <typename T>
+__global__ void k_dpar_gather(int ntok, int d, int max_len, const int *__restrict__ tok_slot,
+                              const int *__restrict__ tok_pos, const T *__restrict__ e,
+                              float *__restrict__ h) {
+  const int m = blockIdx.x;
+  if (m >= ntok) return;
+  const T *er = e + ((size_t)tok_slot[m] * max_len + tok_pos[m]) * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) h[(size_t)m * d + c] = to_f(er[c]);
+}
+
+// Memory rows of each token's own position into head-major K/V [H][ntok][dh]:
+// a causal prefix over the staged positions needs no other memory rows.
+template <typename T>
+__global__ void k_mem_to_hm(int ntok, int H, int DH, int max_len, const int *__restrict__ tok_slot,
+                            const int *__restrict__ tok_pos, const T *__restrict__ mem_g,
+                            T *__restrict__ Kh, T *__restrict__ Vh) {
+  const int per = DH * (int)sizeof(T) / 16;  // 16-byte pieces of one row
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)ntok * H * per) return;
+  const int c = (int)(i % per), h = (int)((i / per) % H), m = (int)(i / ((long)per * H));
+  const T *k = mem_g + ((((size_t)tok_slot[m] * H + h) * 2 + 0) * max_len + tok_pos[m]) * DH;
+  const size_t o = ((size_t)h * ntok + m) * DH;
+  reinterpret_cast<uint4 *>(Kh + o)[c] = reinterpret_cast<const uint4 *>(k)[c];
+  reinterpret_cast<uint4 *>(Vh + o)[c] = reinterpret_cast<const uint4 *>(k + (size_t)max_len * DH)[c];
+}
+
+// The recurrent window after the pass: rotary k and v of positions
+// n_steps - W .. n_steps - 1 into ring slot p mod W of this layer.
+template <typename T>
+__global__ void k_ring_from_hm(int ntok, int H, int DH, int W, int n_steps,
+                               const int *__restrict__ tok_slot, const int *__restrict__ tok_pos,
+                               const T *__restrict__ Kh, const T *__restrict__ Vh,
+                               T *__restrict__ ring_l) {
+  const int per = DH * (int)sizeof(T) / 16;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)ntok * H * per) return;
+  const int c = (int)(i % per), h = (int)((i / per) % H), m = (int)(i / ((long)per * H));
+  const int p = tok_pos[m];
+  if (p < n_steps - W) return;
+  T *kb = ring_l + (((size_t)tok_slot[m] * H + h) * 2) * W * DH + (size_t)(p % W) * DH;
+  const size_t o = ((size_t)h * ntok + m) * DH;
+  reinterpret_cast<uint4 *>(kb)[c] = reinterpret_cast<const uint4 *>(Kh + o)[c];
+  reinterpret_cast<uint4 *>(kb + (size_t)W * DH)[c] = reinterpret_cast<const uint4 *>(Vh + o)[c];
+}
+
+// s_t = RMSNorm_f(h) of every staged token: into s_rows[m] when given, and
+// into the state s of the sequence at its last position n_steps - 1.
+__global__ void k_dpar_final(int ntok, int d, int n_steps, const int *__restrict__ tok_slot,
+                             const int *__restrict__ tok_pos, const float *__restrict__ h,
+                             const float *__restrict__ gamma, float eps, float *__restrict__ s,
+                             float *__restrict__ s_rows) {
+  const int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (m >= ntok) return;
+  const float *hr = h + (size_t)m * d;
+  float ss = 0.f;
+  for (int c = lane; c < d; c += 32) ss += hr[c] * hr[c];
+  ss = warp_sum(ss);
+  const float rs = rsqrtf(ss / d + eps);
+  const bool last = tok_pos[m] == n_steps - 1;
+  float *so = s + (size_t)tok_slot[m] * d;
+  for (int c = lane; c < d; c += 32) {
+    const float v = hr[c] * rs * gamma[c];
+    if (s_rows) s_rows[(size_t)m * d + c] = v;
+    if (last) so[c] = v;
+  }
+}
+
 // ----------------------------------------------------------------- prefill
 // Token embedding rows into the fp32 residual stream; out-of-range token ids
 // record an error and embed zeros.
@@ -262,10 +335,12 @@ __global__ void k_embed(int ntok, int d, int vocab, const int *__restrict__ tok,
 }
 
 // Encoder q/k/v: rotary q, k at each token's position; head-major [H][ntok][dh].
+// Qlo (optional): the low part q - Qh of the stored query, same layout.
 template <typename T>
 __global__ void k_enc_qkv_post(int ntok, int H, int dh, const int *__restrict__ tok_pos,
                                const float *__restrict__ qkv, const float2 *__restrict__ rope,
-                               T *__restrict__ Qh, T *__restrict__ Kh, T *__restrict__ Vh) {
+                               T *__restrict__ Qh, T *__restrict__ Kh, T *__restrict__ Vh,
+                               T *__restrict__ Qlo) {
   int half = dh / 2, d = H * dh;
   long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long)ntok * H * half) return;
@@ -278,8 +353,13 @@ __global__ void k_enc_qkv_post(int ntok, int H, int dh, const int *__restrict__ 
   int c1 = h * dh + j, c2 = c1 + half;
   size_t o = ((size_t)h * ntok + m) * dh;
   float q1 = row[c1], q2 = row[c2], k1 = row[d + c1], k2 = row[d + c2];
-  Qh[o + j] = from_f<T>(q1 * cs.x - q2 * cs.y);
-  Qh[o + j + half] = from_f<T>(q2 * cs.x + q1 * cs.y);
+  const float qa = q1 * cs.x - q2 * cs.y, qb = q2 * cs.x + q1 * cs.y;
+  Qh[o + j] = from_f<T>(qa);
+  Qh[o + j + half] = from_f<T>(qb);
+  if (Qlo) {
+    Qlo[o + j] = from_f<T>(qa - to_f(from_f<T>(qa)));
+    Qlo[o + j + half] = from_f<T>(qb - to_f(from_f<T>(qb)));
+  }
   Kh[o + j] = from_f<T>(k1 * cs.x - k2 * cs.y);
   Kh[o + j + half] = from_f<T>(k2 * cs.x + k1 * cs.y);
   Vh[o + j] = from_f<T>(row[2 * d + c1]);
@@ -294,7 +374,7 @@ template <typename T, int DH>
 __global__ void k_enc_attn_simt(int ntok, int H, const int *__restrict__ tok_pos,
                                 const int *__restrict__ tok_start, const T *__restrict__ Qh,
                                 const T *__restrict__ Kh, const T *__restrict__ Vh,
-                                T *__restrict__ out, float scale) {
+                                T *__restrict__ out, float scale, int window) {
   constexpr int VEC = V16<T>::N, LPK = DH / VEC;
   int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (gw >= ntok * H) return;
@@ -308,7 +388,8 @@ __global__ void k_enc_attn_simt(int ntok, int H, const int *__restrict__ tok_pos
   const T *K = Kh + ((size_t)h * ntok + st0) * DH;
   const T *V = Vh + ((size_t)h * ntok + st0) * DH;
   SoftAcc<VEC> st;
-  warp_attend<T, DH, false>(qr, K, V, 0, p, 0, lane, st);
+  // causal; with a window, positions p - window + 1 .. p only
+  warp_attend<T, DH, false>(qr, K, V, window > 0 ? max(0, p - window + 1) : 0, p, 0, lane, st);
   if (lane < LPK) {
     float inv = 1.f / st.l;
 #pragma unroll

@@ -195,6 +195,7 @@ struct rlt_model {
   std::map<std::tuple<const void *, uint64_t, uint64_t, uint32_t>, CUtensorMap> tmaps;
   cudaError_t (*step)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
   cudaError_t (*prefill)(rlt_model *, int, int, cudaStream_t) = nullptr;
+  cudaError_t (*dpar)(rlt_model *, int, int, int, float *, cudaStream_t) = nullptr;
   cudaError_t (*get_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
   cudaError_t (*set_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
   cudaError_t (*get_memory)(rlt_model *, int, int, cudaStream_t) = nullptr;
@@ -688,24 +689,125 @@ cudaError_t step_impl_tc(rlt_model *M, const StepInfo &si, cudaStream_t st) {
 // models, the per-query SIMT kernel for fp32 models.
 template <typename T, int DH>
 cudaError_t enc_attention(rlt_model *M, int ntok, int nblk, const T *Qh, const T *Kh, const T *Vh,
-                          T *ea, cudaStream_t st) {
+                          T *ea, cudaStream_t st, int window = 0, const T *Qlo = nullptr) {
   const Layout &L = M->L;
   const int H = M->cfg.n_heads;
   if constexpr (std::is_same<T, bf16>::value && DH >= 32) {
     constexpr int smem = FaSmem<DH>::BYTES;
     static bool attr = false;
     if (!attr) {
-      RLT_TRY(cudaFuncSetAttribute(k_enc_flash<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   smem));
+      RLT_TRY(cudaFuncSetAttribute(k_enc_flash<DH, false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+      RLT_TRY(cudaFuncSetAttribute(k_enc_flash<DH, true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
       attr = true;
     }
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
-    k_enc_flash<DH><<<dim3(nblk, H), 128, smem, st>>>(ntok, M->at<int>(L.blk), Qh, Kh, Vh, ea, H,
-                                                       scale_log2);
+    if (Qlo)
+      k_enc_flash<DH, true><<<dim3(nblk, H), 128, smem, st>>>(
+          ntok, M->at<int>(L.blk), Qh, Kh, Vh, ea, H, scale_log2, window, Qlo);
+    else
+      k_enc_flash<DH, false><<<dim3(nblk, H), 128, smem, st>>>(
+          ntok, M->at<int>(L.blk), Qh, Kh, Vh, ea, H, scale_log2, window, nullptr);
   } else {
     k_enc_attn_simt<T, DH><<<blocks_for((long)ntok * H * 32, 256), 256, 0, st>>>(
         ntok, H, M->at<int>(L.tok_pos), M->at<int>(L.tok_start), Qh, Kh, Vh, ea,
-        1.0f / sqrtf((float)DH));
+        1.0f / sqrtf((float)DH), window);
+  }
+  return cudaGetLastError();
+}
+
+// Token-parallel decoder pass over positions 0..n_steps-1 of the staged
+// sequences, for feedback off (alpha = 0: x_t = e_t, the transition never
+// reads s_{t-1}), layer by layer on the encoder's machinery: per block the
+// window-masked causal self-attention (the SWA), the causal cross-attention
+// over the memory rows of the same positions (M<=t), and the FFN, each with
+// its pre-RMSNorm ([RLT-96] "Architecture"); then s_t = RMSNorm_f(h). The
+// rotary k and v of the last W positions go into each layer's ring, so the
+// recurrent step continues from t = n_steps. s_rows (optional) receives every
+// s_t of the chunk, row m of the staging.
+template <typename T, int DH>
+cudaError_t dpar_impl(rlt_model *M, int ntok, int nblk, int n_steps, float *s_rows,
+                      cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const rlt_weights &w = M->w;
+  const int d = c.d, H = c.n_heads, F = c.ffn_dim, W = c.window;
+  const float eps = c.rms_eps;
+  const int K = RLT_K_ENC;
+  int *tslot = M->at<int>(L.tok_slot), *tpos = M->at<int>(L.tok_pos);
+  float *eh = M->at<float>(L.eh), *eqkv = M->at<float>(L.eqkv), *efa = M->at<float>(L.efa);
+  T *eu = M->at<T>(L.eu), *Qh = M->at<T>(L.Qh), *Kh = M->at<T>(L.Kh), *Vh = M->at<T>(L.Vh);
+  T *ea = M->at<T>(L.ea), *ef = M->at<T>(L.ef);
+  const float2 *rope = M->at<float2>(L.rope);
+  const int rows_blocks = blocks_for((long)ntok * 32, 256);
+  const int hm_blocks = blocks_for((long)ntok * H * (DH * (int)sizeof(T) / 16), 256);
+  const size_t ring_layer = (size_t)c.max_seqs * H * 2 * W * DH;
+  const size_t mem_group = (size_t)c.max_seqs * H * 2 * c.max_len * DH;
+  // bf16 models: the low part of each stored query (head-major, in the FFN
+  // activation buffer, free during the attention sublayers) for the split
+  // tensor-core attention; fp32 models keep the query exact
+  T *qlo = std::is_same<T, bf16>::value && F >= d ? ef : nullptr;
+  {
+    Span sp(M, st, K);
+    k_dpar_gather<T><<<ntok, 256, 0, st>>>(ntok, d, c.max_len, tslot, tpos, M->at<T>(L.e), eh);
+  }
+  RLT_TRY(cudaGetLastError());
+  for (int l = 0; l < c.n_dec_layers; l++) {
+    const T *mem_g = M->at<T>(L.mem) + (size_t)(c.mem_groups == 1 ? 0 : l) * mem_group;
+    // sliding-window self-attention sublayer
+    {
+      Span sp(M, st, K);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh,
+                                                (const float *)w.dec_ln1[l], eps, eu);
+    }
+    RLT_TRY(gemm_enc(M, ntok, 3 * d, d, eu, W_<T>::qkv(M, l), EpiStoreF32{eqkv, 3 * d}, st));
+    {
+      Span sp(M, st, K);
+      k_enc_qkv_post<T><<<blocks_for((long)ntok * H * (DH / 2), 256), 256, 0, st>>>(
+          ntok, H, DH, tpos, eqkv, rope, Qh, Kh, Vh, qlo);
+      k_ring_from_hm<T><<<hm_blocks, 256, 0, st>>>(ntok, H, DH, W, n_steps, tslot, tpos, Kh, Vh,
+                                                    M->at<T>(L.ring) + (size_t)l * ring_layer);
+    }
+    {
+      Span sp(M, st, K);
+      RLT_TRY((enc_attention<T, DH>(M, ntok, nblk, Qh, Kh, Vh, ea, st, W, qlo)));
+    }
+    RLT_TRY(gemm_enc(M, ntok, d, d, ea, W_<T>::o(M, l), EpiResid{eh, d}, st));
+    // cross-attention sublayer over M<=t
+    {
+      Span sp(M, st, K);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh,
+                                                (const float *)w.dec_ln2[l], eps, eu);
+      k_mem_to_hm<T><<<hm_blocks, 256, 0, st>>>(ntok, H, DH, c.max_len, tslot, tpos, mem_g, Kh,
+                                                 Vh);
+    }
+    RLT_TRY(gemm_enc(M, ntok, d, d, eu, (const T *)w.dec_wqx[l],
+                     EpiHeadMajor<T>{Qh, ntok, DH, qlo}, st));
+    {
+      Span sp(M, st, K);
+      RLT_TRY((enc_attention<T, DH>(M, ntok, nblk, Qh, Kh, Vh, ea, st, 0, qlo)));
+    }
+    RLT_TRY(gemm_enc(M, ntok, d, d, ea, (const T *)w.dec_wox[l], EpiResid{eh, d}, st));
+    // FFN sublayer
+    {
+      Span sp(M, st, K);
+      k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh,
+                                                (const float *)w.dec_ln3[l], eps, eu);
+    }
+    if (c.ffn_kind == RLT_GELU) {
+      RLT_TRY(gemm_enc(M, ntok, F, d, eu, W_<T>::w1(M, l), EpiGelu<T>{ef, F}, st));
+    } else {
+      RLT_TRY(gemm_enc(M, ntok, F, d, eu, W_<T>::w1(M, l), EpiStoreF32{efa, F}, st));
+      RLT_TRY(gemm_enc(M, ntok, F, d, eu, W_<T>::wb(M, l), EpiSwiglu<T>{efa, ef, F}, st));
+    }
+    RLT_TRY(gemm_enc(M, ntok, d, F, ef, W_<T>::w2(M, l), EpiResid{eh, d}, st));
+  }
+  {
+    Span sp(M, st, K);
+    k_dpar_final<<<rows_blocks, 256, 0, st>>>(ntok, d, n_steps, tslot, tpos, eh,
+                                              (const float *)w.dec_lnf, eps, M->at<float>(L.s),
+                                              s_rows);
   }
   return cudaGetLastError();
 }
@@ -743,7 +845,7 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, int nblk, cudaStream_t st) {
     {
       Span sp(M, st, K);
       k_enc_qkv_post<T><<<blocks_for((long)ntok * H * (DH / 2), 256), 256, 0, st>>>(
-          ntok, H, DH, tpos, eqkv, rope, Qh, Kh, Vh);
+          ntok, H, DH, tpos, eqkv, rope, Qh, Kh, Vh, (T *)nullptr);
     }
     {
       Span sp(M, st, K);
@@ -816,6 +918,7 @@ template <typename T, int DH> void bind(rlt_model *M) {
   else
     M->step = step_impl<T, DH>;
   M->prefill = prefill_impl<T, DH>;
+  M->dpar = dpar_impl<T, DH>;
   M->get_window = get_window_impl<T>;
   M->set_window = set_window_impl<T>;
   M->get_memory = get_memory_impl<T>;
@@ -1392,6 +1495,61 @@ RLT_API int rlt_run_sequence(rlt_model *M, const int32_t *ids, int n, int n_step
     advance(M, idv.data(), n);
   }
   return cuda_status(e);
+}
+
+RLT_API int rlt_decoder_parallel(rlt_model *M, const int32_t *ids, int n, int n_steps,
+                                 float *s_all, rlt_stream stream) {
+  if (n_steps < 0) return RLT_ERR_INVALID_ARG;
+  int rc = check_batch(M, ids, n, n_steps);
+  if (rc != RLT_OK) return rc;
+  if (M->cfg.alpha != 0.0f) return RLT_ERR_UNSUPPORTED;  // s_{t-1} feeds step t
+  for (int i = 0; i < n; i++)
+    if (M->t_dec[ids[i]] != 0) return RLT_ERR_INVALID_ARG;  // fresh sequences only
+  if (n == 0 || n_steps == 0) return RLT_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  const Layout &L = M->L;
+  const int per_chunk = std::max(1, L.ptok / n_steps);  // whole sequences per chunk
+  std::vector<int> slot, pos, start, blk;
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < n && e == cudaSuccess; i += per_chunk) {
+    const int j = std::min(n, i + per_chunk);
+    const int ntok = (j - i) * n_steps;
+    slot.resize(ntok);
+    pos.resize(ntok);
+    start.resize(ntok);
+    blk.clear();
+    for (int k = i, m = 0; k < j; k++) {
+      for (int qb = 0; qb * 64 < n_steps; qb++) {
+        blk.push_back(m);
+        blk.push_back(n_steps);
+        blk.push_back(qb);
+        blk.push_back(0);
+      }
+      for (int p = 0; p < n_steps; p++, m++) {
+        slot[m] = ids[k];
+        pos[m] = p;
+        start[m] = m - p;
+      }
+    }
+    e = cudaMemcpyAsync(M->at<int>(L.tok_slot), slot.data(), 4 * (size_t)ntok,
+                        cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(M->at<int>(L.tok_pos), pos.data(), 4 * (size_t)ntok,
+                          cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(M->at<int>(L.tok_start), start.data(), 4 * (size_t)ntok,
+                          cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(M->at<int>(L.blk), blk.data(), 4 * blk.size(), cudaMemcpyHostToDevice,
+                          st);
+    if (e == cudaSuccess)
+      e = M->dpar(M, ntok, (int)(blk.size() / 4), n_steps,
+                  s_all ? s_all + (size_t)i * n_steps * M->cfg.d : nullptr, st);
+  }
+  if (e != cudaSuccess) return cuda_status(e);
+  for (int i = 0; i < n; i++) M->t_dec[ids[i]] = n_steps;
+  return cuda_status(push_positions(M, st));
 }
 
 RLT_API int rlt_plan_ragged(const int32_t *steps, int n, int32_t *order, int32_t *tick_sizes,

@@ -81,6 +81,7 @@ def _declare(lib):
     lib.rlt_prefill_encoder.argtypes = [P, P, P, P, P, I, P]
     lib.rlt_decoder_step.argtypes = [P, P, I, P]
     lib.rlt_run_sequence.argtypes = [P, P, I, I, P]
+    lib.rlt_decoder_parallel.argtypes = [P, P, I, I, P, P]
     lib.rlt_run_ragged.argtypes = [P, P, P, I, P]
     lib.rlt_plan_ragged.argtypes = [P, I, P, P, I, C.POINTER(I)]
     lib.rlt_get_state.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
@@ -296,6 +297,18 @@ class Model:
         ids = _i32(seq_ids)
         _check(_lib().rlt_run_sequence(self._h, _p(ids), ids.shape[0], int(n_steps),
                                        self._st(stream)), "rlt_run_sequence")
+
+    def decoder_parallel(self, seq_ids, n_steps: int, s_all=None, stream=None):
+        """Token-parallel decoder pass of fresh sequences (alpha = 0 models);
+        s_all: optional fp32 device tensor [n][n_steps][d] for every s_t."""
+        ids = _i32(seq_ids)
+        ptr = None
+        if s_all is not None:
+            assert s_all.is_cuda and s_all.dtype == self.torch.float32 and s_all.is_contiguous()
+            assert tuple(s_all.shape) == (ids.shape[0], int(n_steps), self.cfg.d)
+            ptr = C.c_void_p(s_all.data_ptr())
+        _check(_lib().rlt_decoder_parallel(self._h, _p(ids), ids.shape[0], int(n_steps), ptr,
+                                           self._st(stream)), "rlt_decoder_parallel")
 
     def run_ragged(self, seq_ids, steps, stream=None):
         ids, st = _i32(seq_ids), _i32(steps)

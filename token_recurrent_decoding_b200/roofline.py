@@ -87,3 +87,22 @@ def run_roofline(cfg: RLTConfig, lengths, hbm_gbs: float, tensor_tflops: float,
     return {"decoder_s": dec_t, "decoder_bytes": dec_bytes, "decoder_flops": dec_flops,
             "encoder_s": enc_f / (tensor_tflops * 1e12), "encoder_flops": enc_f,
             "seq_steps": int(lengths.sum())}
+
+
+def decoder_parallel_roofline(cfg: RLTConfig, lengths, hbm_gbs: float, tensor_tflops: float):
+    """Roofline of the token-parallel decoder pass (feedback off) over full
+    sequences: FLOPs = 2 x decoder matmul parameters per token plus the
+    window-masked and prefix attention, bytes = weights once, e_t and the
+    memory rows read once per group, s_t written; the larger time bounds."""
+    lengths = np.asarray(lengths)
+    es = elem_bytes(cfg)
+    d, W = cfg.d, cfg.window
+    flops = 0.0
+    for T in lengths:
+        t = np.arange(T, dtype=np.float64)
+        flops += 2 * dec_matmul_params(cfg) * T
+        flops += np.sum(cfg.n_dec * 4 * d * (np.minimum(t + 1, W) + t + 1))
+    tok = float(lengths.sum())
+    byts = dec_matmul_params(cfg) * es + tok * d * (es + 4) + cfg.mem_groups * tok * 2 * d * es
+    return {"seconds": max(flops / (tensor_tflops * 1e12), byts / (hbm_gbs * 1e9)),
+            "flops": float(flops), "bytes": float(byts), "seq_steps": int(tok)}
