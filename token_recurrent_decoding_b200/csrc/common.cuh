@@ -155,11 +155,6 @@ __device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, unsign
       : "memory");
 }
 
-// Pull [src, src + bytes) into L2 (16-byte aligned, size a multiple of 16).
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, unsigned bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
   uint32_t ok;
   asm volatile(

@@ -34,14 +34,6 @@ struct EpiStoreF32 {
   __device__ void vec16(int m, int n, const float *v) const { store16(out + (size_t)m * ld + n, v); }
 };
 
-template <typename T> struct EpiStore {
-  T *out; int ld;
-  __device__ void operator()(int m, int n, float a, float b) const {
-    out[(size_t)m * ld + n] = from_f<T>(a);
-    out[(size_t)m * ld + n + 1] = from_f<T>(b);
-  }
-};
-
 // Residual stream update h += C.
 struct EpiResid {
   float *h; int ld;

@@ -426,15 +426,6 @@ cudaError_t gemm_enc(rlt_model *M, int m, int n, int k, const T *A, const T *B, 
     return gemm(m, nullptr, n, k, A, k, B, k, epi, st);
 }
 
-template <typename T, class Epi>
-cudaError_t gemm_k(rlt_model *M, int kind, int m, int n, int k, const T *A, int lda, const T *B,
-                   int ldb, Epi epi, cudaStream_t st) {
-  double es = sizeof(T);
-  Span sp(M, st, kind, (double)n * k * es + (double)m * k * es + (double)m * n * 4.0,
-          2.0 * m * n * k);
-  return gemm(m, nullptr, n, k, A, lda, B, ldb, epi, st);
-}
-
 template <typename T> struct W_ {
   // Decoder matrices of layer l, honouring weight tying.
   static const T *qkv(const rlt_model *M, int l) {
