@@ -16,6 +16,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -103,6 +105,62 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
 }
+
+// q/k/v projection of the encoder (and of the token-parallel decoder pass)
+// straight into head-major Q, K, V [H][ntok][DH] with the rotary embedding
+// at each token's position (pairs j, j + DH/2 of a head), instead of an fp32
+// row-major intermediate and a separate rotary pass. One TMEM row = one
+// token; the tile holds whole heads (BN a multiple of DH, DH >= 32), and the
+// epilogue reads the two 16-column groups of a rotary pair together. Qlo
+// (optional) receives the low part q - Qh of each stored query.
+template <typename T> struct EpiEncQkvRope {
+  static constexpr bool kTileEpilogue = true;
+  T *Qh, *Kh, *Vh, *Qlo;
+  const int *tok_pos;
+  const float2 *rope;
+  int ntok, DH, d, N;
+  // every lane of the warp runs the TMEM loads; `valid` gates the stores
+  template <int BN>
+  __device__ void tile(int m, bool valid, int n0, uint32_t lane_base) const {
+    const int half = DH / 2;
+    const int t = valid ? tok_pos[m] : 0;
+    for (int hb = 0; hb < BN; hb += DH)
+      for (int j0 = 0; j0 < half; j0 += 16) {
+        float a[16], b[16];
+        tmem_ld16(lane_base + hb + j0, a);
+        tmem_ld16(lane_base + hb + j0 + half, b);
+        const int col = n0 + hb;  // first column of this head
+        if (!valid || col >= N) continue;
+        const int which = col / d, h = (col - which * d) / DH;
+        if (which < 2) {
+#pragma unroll
+          for (int i = 0; i < 16; i++) {
+            const float2 cs = rope[(size_t)t * half + j0 + i];
+            const float x = a[i] * cs.x - b[i] * cs.y, y = b[i] * cs.x + a[i] * cs.y;
+            a[i] = x;
+            b[i] = y;
+          }
+        }
+        T *dst = (which == 0 ? Qh : which == 1 ? Kh : Vh) + ((size_t)h * ntok + m) * DH + j0;
+        store16(dst, a);
+        store16(dst + half, b);
+        if (which == 0 && Qlo) {
+#pragma unroll
+          for (int i = 0; i < 16; i++) {
+            a[i] -= to_f(from_f<T>(a[i]));
+            b[i] -= to_f(from_f<T>(b[i]));
+          }
+          T *lo = Qlo + ((size_t)h * ntok + m) * DH + j0;
+          store16(lo, a);
+          store16(lo + half, b);
+        }
+      }
+  }
+};
+
+template <class E, class = void> struct epi_has_tile : std::false_type {};
+template <class E>
+struct epi_has_tile<E, std::void_t<decltype(E::kTileEpilogue)>> : std::true_type {};
 
 constexpr int TC_BM = 128, TC_BK = 64;
 constexpr uint64_t WAIT_LIMIT_NS_TC = 2000000000ull;  // bounded waits: 2 s of device time
@@ -211,6 +269,8 @@ __global__ void __launch_bounds__(128, 1)
   const bool ok = acc_ok && !s_fail;
   if (!ok) {
     if (threadIdx.x == 0) set_error(err, DEV_ERR_TIMEOUT);
+  } else if constexpr (epi_has_tile<Epi>::value) {
+    epi.template tile<BN>(row, row < M, n0, lane_base);
   } else {
     // N is a multiple of 16: whole 16-column groups
 #pragma unroll 1

@@ -414,6 +414,18 @@ struct Span {
 // algorithmic traffic of one pass over the weights and activations.
 // Encoder GEMM: tcgen05 for bf16 models, exact fp32 SIMT for fp32 models.
 // A is an encoder work buffer of ptok rows and k columns (lda = k).
+// Encoder-side q/k/v GEMM with the rotary head-major epilogue (bf16 models,
+// DH >= 32): a tile holds whole heads, BN = 128 or 64.
+template <int DH>
+cudaError_t gemm_enc_qkv(rlt_model *M, int m, const bf16 *A, const bf16 *Wqkv,
+                         EpiEncQkvRope<bf16> epi, cudaStream_t st) {
+  const double d = M->cfg.d;
+  Span sp(M, st, RLT_K_ENC, 3 * d * d * 2 + m * d * 2 + m * 3 * d * 2, 2.0 * m * 3 * d * d);
+  if (DH >= 128 || m >= 1024)
+    return launch_tc<128, 3>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
+  return launch_tc<64, 4>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
+}
+
 template <typename T, class Epi>
 cudaError_t gemm_enc(rlt_model *M, int m, int n, int k, const T *A, const T *B, Epi epi,
                      cudaStream_t st) {
@@ -752,11 +764,19 @@ cudaError_t dpar_impl(rlt_model *M, int ntok, int nblk, int n_steps, float *s_ro
       k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh,
                                                 (const float *)w.dec_ln1[l], eps, eu);
     }
-    RLT_TRY(gemm_enc(M, ntok, 3 * d, d, eu, W_<T>::qkv(M, l), EpiStoreF32{eqkv, 3 * d}, st));
-    {
+    if constexpr (std::is_same<T, bf16>::value && DH >= 32) {
+      RLT_TRY(gemm_enc_qkv<DH>(M, ntok, eu, W_<T>::qkv(M, l),
+                               EpiEncQkvRope<bf16>{Qh, Kh, Vh, qlo, tpos, rope, ntok, DH, d,
+                                                   3 * d},
+                               st));
+    } else {
+      RLT_TRY(gemm_enc(M, ntok, 3 * d, d, eu, W_<T>::qkv(M, l), EpiStoreF32{eqkv, 3 * d}, st));
       Span sp(M, st, K);
       k_enc_qkv_post<T><<<blocks_for((long)ntok * H * (DH / 2), 256), 256, 0, st>>>(
           ntok, H, DH, tpos, eqkv, rope, Qh, Kh, Vh, qlo);
+    }
+    {
+      Span sp(M, st, K);
       k_ring_from_hm<T><<<hm_blocks, 256, 0, st>>>(ntok, H, DH, W, n_steps, tslot, tpos, Kh, Vh,
                                                     M->at<T>(L.ring) + (size_t)l * ring_layer);
     }
@@ -831,9 +851,14 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, int nblk, cudaStream_t st) {
       k_rmsnorm<T><<<rows_blocks, 256, 0, st>>>(ntok, nullptr, d, eh, (const float *)w.enc_ln1[l],
                                                 eps, eu);
     }
-    RLT_TRY(gemm_enc(M, ntok, 3 * d, d, eu, (const T *)w.enc_wqkv[l], EpiStoreF32{eqkv, 3 * d},
-                     st));
-    {
+    if constexpr (std::is_same<T, bf16>::value && DH >= 32) {
+      RLT_TRY(gemm_enc_qkv<DH>(M, ntok, eu, (const bf16 *)w.enc_wqkv[l],
+                               EpiEncQkvRope<bf16>{Qh, Kh, Vh, nullptr, tpos, rope, ntok, DH,
+                                                   d, 3 * d},
+                               st));
+    } else {
+      RLT_TRY(gemm_enc(M, ntok, 3 * d, d, eu, (const T *)w.enc_wqkv[l],
+                       EpiStoreF32{eqkv, 3 * d}, st));
       Span sp(M, st, K);
       k_enc_qkv_post<T><<<blocks_for((long)ntok * H * (DH / 2), 256), 256, 0, st>>>(
           ntok, H, DH, tpos, eqkv, rope, Qh, Kh, Vh, (T *)nullptr);
