@@ -225,6 +225,11 @@ RLT_API int rlt_get_encoder_output(rlt_model *model, int seq, void *e_out,
                                    void *mem_out, int64_t *t_enc_out,
                                    rlt_stream stream);
 
+/* Memory positions per split of the decode attention (rlt_attend and the
+ * decoder's cross-attention): rows longer than this are split into chunks of
+ * this many positions and merged in chunk order. */
+#define RLT_ATTEND_CHUNK 1024
+
 /* Bytes of device workspace rlt_attend needs (0 if the shape is invalid). */
 RLT_API size_t rlt_attend_workspace_bytes(int n, int n_heads, int head_dim, int cap);
 
@@ -243,9 +248,13 @@ RLT_API size_t rlt_attend_workspace_bytes(int n, int n_heads, int head_dim, int 
  *           cap) bytes, 256-byte aligned, owned by the caller; its first
  *           int32 is a device error word (0 = ok, RLT_ERR_TIMEOUT if a
  *           bounded wait gave up). Calls sharing a workspace must not overlap.
- * Rows are split into chunks of 256 positions merged in chunk order, so a
- * row's result does not depend on the other rows. Errors: INVALID_ARG,
- * UNSUPPORTED (head_dim not 16/32/64/128), CAPACITY (workspace too small). */
+ * Rows are split into chunks of RLT_ATTEND_CHUNK (1024) positions, each
+ * chunk attended by one warp; the chunks of a row are merged in chunk order,
+ * so a row's result does not depend on the other rows or on timing.
+ * The call copies the per-row positions from pageable host memory on
+ * `stream`, so it must not be made while `stream` is being captured into a
+ * CUDA graph. Errors: INVALID_ARG, UNSUPPORTED (head_dim not
+ * 16/32/64/128), CAPACITY (workspace too small). */
 RLT_API int rlt_attend(const float *q, const void *kv, const int32_t *h_lengths, int n,
                        int n_heads, int head_dim, int cap, int dtype, void *out,
                        void *workspace, size_t workspace_bytes, rlt_stream stream);
@@ -266,7 +275,11 @@ RLT_API int rlt_attend(const float *q, const void *kv, const int32_t *h_lengths,
  *   - All calls on a device share its one array; each call clears what must
  *     start at zero, but calls that overlap on the GPU (for example on two
  *     streams) race on the array: serialise them.
- *   - The device error word of rlt_attend is not reported. */
+ *   - Like rlt_attend, it must not be called while `stream` is being
+ *     captured into a CUDA graph.
+ *   - The device error word of rlt_attend is not reported. If a bounded
+ *     device wait gives up (RLT_ERR_TIMEOUT in rlt_attend's error word), the
+ *     call still returns RLT_OK and the contents of `out` are unspecified. */
 RLT_API int rlt_attend_noalloc(const float *q, const void *kv, const int32_t *h_lengths, int n,
                                int n_heads, int head_dim, int cap, int dtype, void *out,
                                rlt_stream stream);
@@ -301,6 +314,24 @@ RLT_API int rlt_profile(rlt_model *model, int enable);
 /* Synchronises the model's last stream, folds every completed event pair
  * into the per-class sums and copies the counters into *out. */
 RLT_API int rlt_get_stats(rlt_model *model, rlt_stats *out);
+
+/* Faults rlt_set_fault can plant (failure detection, tested without
+ * faulting the GPU). */
+enum {
+  RLT_FAULT_NONE = 0,
+  /* the decoder attention's producer fills no stage: every consumer's
+   * bounded wait runs out, records RLT_ERR_TIMEOUT and the kernel returns */
+  RLT_FAULT_SKIP_ATTN_PRODUCER = 1
+};
+
+/* Failure-detection hook (no counterpart in the method). Synchronises the
+ * model's last stream, then makes every later decoder-attention launch of
+ * this model run with `fault` planted and its bounded device waits limited
+ * to wait_limit_ns of device time (0 = the default bound, 2 s). The
+ * attention output of a faulted step is unspecified; rlt_poll_device_error
+ * reports RLT_ERR_TIMEOUT. Captured step graphs read the controls at run
+ * time. Errors: INVALID_ARG (unknown fault, negative limit), CUDA. */
+RLT_API int rlt_set_fault(rlt_model *model, int fault, int64_t wait_limit_ns);
 
 /* Synchronises the model's last stream and returns the first device-side
  * error recorded since the previous poll (RLT_OK if none), then clears it. */

@@ -1,7 +1,8 @@
 """The decoder's cross-attention kernel through the standalone C-ABI call
 rlt_attend, against the oracle's attention (fp64) row by row: ragged lengths
-that span several 256-position chunks and a ragged tail, one-row prefixes,
-both storage types, and a full-size sample (256 rows x 12 heads x 1024)."""
+within one 1024-position chunk, lengths that split into several chunks merged
+in chunk order (1025 .. 4096, with ragged tail chunks), one-row prefixes, both
+storage types, and a full-size sample (256 rows x 12 heads x 1024)."""
 import numpy as np
 import pytest
 import torch
@@ -42,6 +43,20 @@ def test_attend_matches_oracle_ragged(dtype, dh):
     q, kv, out = _case(n, H, dh, cap, lengths, dtype)
     # bf16 output: one storage rounding (2^-9 relative); fp32: accumulation only
     _check(q, kv, out, lengths, range(n), 1e-2 if dtype == torch.bfloat16 else 1e-5)
+
+
+@pytest.mark.parametrize("dtype,dh", [(torch.bfloat16, 64), (torch.bfloat16, 128),
+                                      (torch.float32, 32)])
+def test_attend_split_kv_chunks_match_oracle(dtype, dh):
+    """Rows longer than one 1024-position chunk: partials of every chunk,
+    merged by the row's last finishing unit in chunk order."""
+    lengths = [1025, 2047, 2048, 3000, 4096, 1, 1024, 2049, 4095, 1500]
+    n, H, cap = len(lengths), 2, 4096
+    q, kv, out = _case(n, H, dh, cap, lengths, dtype, seed=5)
+    _check(q, kv, out, lengths, range(n), 1e-2 if dtype == torch.bfloat16 else 1e-5)
+    # a second call agrees bitwise: a row's result depends on its own length only
+    q2, kv2, out2 = _case(n, H, dh, cap, lengths, dtype, seed=5)
+    np.testing.assert_array_equal(out, out2)
 
 
 def test_attend_full_size_sampled():

@@ -7,8 +7,8 @@ import pytest
 import torch
 
 import oracle
-from rlt_cases import (SMALL, STEP_TOL, TRAJ_TOL, make_model, prefill_all, rel_l2, rms,
-                       to_np)
+from rlt_cases import (CACHE_TOL, SMALL, STEP_TOL, TRAJ_TOL, make_model, prefill_all, rel_l2,
+                       rms, to_np)
 from token_recurrent_decoding_b200 import configs, inputs
 from token_recurrent_decoding_b200.rlt import Model, RLTError
 
@@ -18,8 +18,6 @@ pytestmark = pytest.mark.gpu
 # adds one storage rounding (2^-9 relative) on top of the residual-stream
 # error; bound max|err| / RMS and rel-L2.
 ENC_TOL = {configs.F32: (1e-5, 1e-6), configs.BF16: (6e-2, 1.5e-2)}
-# newest K/V entries written by one step (bf16: one storage rounding on top)
-CACHE_TOL = {configs.F32: 1e-5, configs.BF16: 5e-2}
 
 
 @pytest.mark.parametrize("name,lengths", [(n, [37, 70, 5, 1]) for n in SMALL]
@@ -266,3 +264,56 @@ def test_encoder_is_causal_at_full_size_bitwise():
         assert torch.equal(e0[: k + 1], e1[: k + 1])
         assert torch.equal(m0[:, : k + 1], m1[:, : k + 1])
         assert not torch.equal(e0[k + 1:], e1[k + 1:])
+
+
+@pytest.mark.parametrize("name", ["ragged_like", "tied_like", "m140_like"])
+def test_stepwise_parity_past_one_memory_chunk(name):
+    """Positions past 1024: the cross-attention over M<=t splits into several
+    1024-row chunks (partials merged in chunk order, a ragged tail chunk);
+    step-wise against the oracle fed the GPU's own state."""
+    cfg = SMALL[name]
+    T = 2100
+    m, w, tok = make_model(cfg, [T] * 2)
+    o = oracle.Oracle(cfg, w)
+    e_g, mem_g = (to_np(x) for x in m.get_encoder_output(1))
+    tol = STEP_TOL[cfg.dtype]
+    done = 0
+    for t in (1023, 1024, 1025, 2047, 2048, T - 1):
+        m.run_sequence([0, 1], t - done)
+        s_prev, c_prev, tt = m.get_state(1)
+        assert tt == t
+        m.run_sequence([0, 1], 1)
+        done = t + 1
+        s_ref, win_ref = o.step(e_g[t], mem_g, t, to_np(s_prev), to_np(c_prev))
+        s_new, c_new, _ = m.get_state(1)
+        err = np.abs(to_np(s_new) - s_ref).max() / rms(s_ref)
+        assert err <= tol, (name, t, err)
+        newest = to_np(c_new)[:, :, -1]
+        assert np.abs(newest - win_ref[:, :, -1]).max() <= CACHE_TOL[cfg.dtype] * rms(
+            win_ref[:, :, -1])
+
+
+def test_bounded_wait_timeout_is_reported_and_model_recovers():
+    """Failure detection without faulting the GPU: a planted fault makes the
+    decoder attention's producer fill nothing, so its consumers' bounded waits
+    (limited to 2 ms for the test) run out; the step returns, the device error
+    word reads RLT_ERR_TIMEOUT, and after the fault is cleared and the slots
+    are prefilled again the model computes the same states as a fresh one."""
+    from token_recurrent_decoding_b200 import rlt as R
+    cfg = SMALL["m50_like"]
+    lengths = [24, 24]
+    m, w, tok = make_model(cfg, lengths)
+    m.set_fault(R.FAULT_SKIP_ATTN_PRODUCER, 2_000_000)
+    m.decoder_step([0, 1])
+    assert m.poll_device_error() == 7  # RLT_ERR_TIMEOUT
+    assert m.poll_device_error() == 0  # the poll cleared it
+    m.set_fault(R.FAULT_NONE, 0)
+    prefill_all(m, tok, lengths)
+    m.run_sequence([0, 1], 24)
+    assert m.poll_device_error() == 0
+    ref, _, _ = make_model(cfg, lengths)
+    ref.run_sequence([0, 1], 24)
+    for i in range(2):
+        assert torch.equal(m.get_state(i)[0], ref.get_state(i)[0])
+    with pytest.raises(RLTError):
+        m.set_fault(99, 0)

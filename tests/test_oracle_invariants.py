@@ -361,3 +361,84 @@ def test_decoder_swa_is_band_masked_rotary_attention(W):
     h = e + _mha(cfg, u, w["dec.0.wqkv"], band) @ w["dec.0.wo"].T
     ref = np.stack([_rms(r, w["dec.lnf"], cfg.rms_eps) for r in h])
     np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11)
+
+
+# ---------------------------------------------- encoder FFN and layer stacking
+def _enc_rows(cfg, w, x, l):
+    """One encoder block with its attention output zeroed, through torch:
+    x + W2 act(W1 RMSNorm_2(x)) per position (GELU or SwiGLU)."""
+    u = torch.tensor(np.stack([_rms(r, w[f"enc.{l}.ln2"], cfg.rms_eps) for r in x]))
+    if cfg.ffn_kind == configs.GELU:
+        f = F.gelu(u @ torch.tensor(w[f"enc.{l}.w1"]).T)
+    else:
+        f = F.silu(u @ torch.tensor(w[f"enc.{l}.wa"]).T) * (u @ torch.tensor(w[f"enc.{l}.wb"]).T)
+    return x + (f @ torch.tensor(w[f"enc.{l}.w2"]).T).numpy()
+
+
+@pytest.mark.parametrize("kind", [configs.GELU, configs.SWIGLU])
+def test_encoder_ffn_sublayer_closed_form(kind):
+    """One encoder block whose attention writes nothing (W_o = 0): e_t =
+    RMSNorm_E(x + W2 act(W1 RMSNorm_2(x))), x = E[tok_t]; memory rows are
+    W_mk e, W_mv e."""
+    cfg = BASE.replace(n_enc=1, ffn_kind=kind)
+    w = _weights(cfg)
+    _zero(w, ["enc.0.wo"])
+    tok = _tokens(cfg)[0]
+    e, mem = oracle.Oracle(cfg, w).encode(tok)
+    h = _enc_rows(cfg, w, w["embed"][tok], 0)
+    ref = np.stack([_rms(r, w["enc.lnf"], cfg.rms_eps) for r in h])
+    np.testing.assert_allclose(e, ref, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(mem[0, :T, 1], ref @ w["mem.0.wv"].T, rtol=1e-11, atol=1e-12)
+
+
+def _one_block_copy(w, src_layer, n_enc_names=True, prefix="enc"):
+    """Weights of a one-block model whose block 0 is block `src_layer`."""
+    out = {k: v for k, v in w.items() if not k.startswith(prefix + ".")
+           or k == prefix + ".lnf"}
+    for k, v in w.items():
+        parts = k.split(".")
+        if parts[0] == prefix and parts[1].isdigit() and int(parts[1]) == src_layer:
+            out[f"{prefix}.0.{'.'.join(parts[2:])}"] = v
+    return out
+
+
+@pytest.mark.parametrize("zeroed,kept", [(1, 0), (0, 1)])
+def test_encoder_blocks_stack_in_order(zeroed, kept):
+    """A two-block encoder with one block's output matrices zeroed (the block
+    is the identity) equals the one-block encoder made of the other block:
+    every block uses its own matrices and norms, in layer order."""
+    cfg2 = BASE.replace(n_enc=2)
+    w = _weights(cfg2)
+    _zero(w, [f"enc.{zeroed}.wo", f"enc.{zeroed}.w2"])
+    tok = _tokens(cfg2)[0]
+    e2, m2 = oracle.Oracle(cfg2, w).encode(tok)
+    cfg1 = BASE.replace(n_enc=1)
+    e1, m1 = oracle.Oracle(cfg1, _one_block_copy(w, kept)).encode(tok)
+    np.testing.assert_array_equal(e2, e1)
+    np.testing.assert_array_equal(m2, m1)
+    # and the kept block is not the identity
+    e0, _ = oracle.Oracle(BASE.replace(n_enc=0), w).encode(tok)
+    assert np.abs(e2 - e0).max() > 1e-3
+
+
+@pytest.mark.parametrize("G", ["shared", "per_layer"])
+@pytest.mark.parametrize("zeroed,kept", [(0, 1), (1, 0)])
+def test_decoder_layers_stack_in_order(zeroed, kept, G):
+    """A two-layer decoder whose layer `zeroed` writes nothing (W_o, W_ox, W_2
+    zero: the layer is the identity on the residual stream) equals the
+    one-layer decoder made of layer `kept` -- its q/k/v, W_o, W_qx, W_ox, FFN,
+    its three norms and (G = L_D) its own memory group. Pins the layer index
+    of every decoder sublayer, which the brute-force twin shares."""
+    groups = 2 if G == "per_layer" else 1
+    cfg2 = BASE.replace(n_dec=2, mem_groups=groups)
+    w = _weights(cfg2)
+    _zero(w, [f"dec.{zeroed}.wo", f"dec.{zeroed}.wox", f"dec.{zeroed}.w2"])
+    tok = _tokens(cfg2)[0]
+    got2, _, _ = oracle.Oracle(cfg2, w).run(tok)
+    cfg1 = BASE.replace(n_dec=1, mem_groups=1)
+    w1 = _one_block_copy(w, kept, prefix="dec")
+    w1 = {k: v for k, v in w1.items() if not k.startswith("mem.")}
+    g = kept if groups > 1 else 0
+    w1["mem.0.wk"], w1["mem.0.wv"] = w[f"mem.{g}.wk"], w[f"mem.{g}.wv"]
+    got1, _, _ = oracle.Oracle(cfg1, w1).run(tok)
+    np.testing.assert_array_equal(got2, got1)

@@ -50,6 +50,32 @@ MUTANTS = {
     "swiglu factors swapped": ("tmp_a[i] = orc_silu(tmp_a[i]) * tmp_b[i];",
                                "tmp_a[i] = tmp_a[i] * orc_silu(tmp_b[i]);"),
     "start state zero": ("memcpy(s, w->sstar, sizeof(real) * c->d);", "memset(s, 0, sizeof(real) * c->d);"),
+    "encoder ffn reads the attention norm": (
+        "orc_rmsnorm(h + (size_t)t * d, w->enc_ln2[l], d, c->rms_eps, u);",
+        "orc_rmsnorm(h + (size_t)t * d, w->enc_ln1[l], d, c->rms_eps, u);"),
+    "encoder ffn residual dropped": (
+        "ffn(c, w->enc_w1[l], w->enc_wb[l], w->enc_w2[l], u, o, ta, tb);\n"
+        "      for (int i = 0; i < d; i++) h[(size_t)t * d + i] += o[i];",
+        "ffn(c, w->enc_w1[l], w->enc_wb[l], w->enc_w2[l], u, o, ta, tb);\n"
+        "      for (int i = 0; i < d; i++) h[(size_t)t * d + i] = o[i];"),
+    "encoder blocks reuse block 0's ffn": ("ffn(c, w->enc_w1[l], w->enc_wb[l], w->enc_w2[l],",
+                                           "ffn(c, w->enc_w1[0], w->enc_wb[0], w->enc_w2[0],"),
+    "encoder blocks reuse block 0's q/k/v": (
+        "orc_linear(w->enc_wqkv[l], u, 3 * d, d, qkv + (size_t)t * 3 * d);",
+        "orc_linear(w->enc_wqkv[0], u, 3 * d, d, qkv + (size_t)t * 3 * d);"),
+    "decoder q/k/v of layer 0": ("orc_linear(w->dec_wqkv[l], s->u, 3 * d, d, s->q);",
+                                 "orc_linear(w->dec_wqkv[0], s->u, 3 * d, d, s->q);"),
+    "decoder output projection of layer 0": ("orc_linear(w->dec_wo[l], sc->a, d, d, sc->o);",
+                                             "orc_linear(w->dec_wo[0], sc->a, d, d, sc->o);"),
+    "decoder cross-attention query of layer 0": ("orc_linear(w->dec_wqx[l], s->u, d, d, s->q);",
+                                                 "orc_linear(w->dec_wqx[0], s->u, d, d, s->q);"),
+    "decoder cross-attention output of layer 0": ("orc_linear(w->dec_wox[l], s->a, d, d, s->o);",
+                                                  "orc_linear(w->dec_wox[0], s->a, d, d, s->o);"),
+    "decoder ffn of layer 0": ("ffn(c, w->dec_w1[l], w->dec_wb[l], w->dec_w2[l],",
+                               "ffn(c, w->dec_w1[0], w->dec_wb[0], w->dec_w2[0],"),
+    "decoder cross-attention norms in reverse layer order": (
+        "orc_rmsnorm(h, w->dec_ln2[l], d, c->rms_eps, s->u);",
+        "orc_rmsnorm(h, w->dec_ln2[c->n_dec - 1 - l], d, c->rms_eps, s->u);"),
 }
 
 PIN_FILES = ["tests/test_oracle_pieces.py", "tests/test_oracle_invariants.py"]

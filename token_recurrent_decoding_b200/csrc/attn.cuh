@@ -167,7 +167,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
                   const float *__restrict__ q,
                   const T *__restrict__ base, long seq_stride, long head_stride, long v_offset,
                   float *__restrict__ part, int *__restrict__ counters, T *__restrict__ out,
-                  float scale, int kv_reuse, int *err) {
+                  float scale, int kv_reuse, int *err, const DevCtl *ctl) {
   using S = AttnShape<T, DH, TB>;
   constexpr int KT = S::KT, VEC = S::VEC, LPK = S::LPK, KPP = S::KPP, P = S::P, PG = S::PG;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -175,6 +175,10 @@ __global__ void __launch_bounds__((NC + 1) * 32)
   uint64_t *empty = full + NC * SW;
   int *s_abort = reinterpret_cast<int *>(empty + NC * SW);
   int *s_pos = s_abort + 4, *s_ready = s_pos + ATTN_SMEM_ROWS;
+
+  // failure-detection controls (null: defaults, no planted fault)
+  const uint64_t wait_limit = ctl && ctl->wait_limit_ns ? ctl->wait_limit_ns : WAIT_LIMIT_NS;
+  const bool skip_producer = ctl && ctl->fault == DEV_FAULT_SKIP_ATTN_PRODUCER;
 
   pdl_trigger();
   // Positions: by row from `pos` (written by an earlier kernel: wait first),
@@ -212,6 +216,12 @@ __global__ void __launch_bounds__((NC + 1) * 32)
   if (warp == NC) {
     // ---------------------------------------------------------- producer
     if (lane != 0) return;
+    if (skip_producer) {
+      // planted fault: no stage is ever filled, so every consumer's bounded
+      // wait runs out and reports RLT_ERR_TIMEOUT (no copy is in flight)
+      pdl_wait();
+      return;
+    }
     // K/V read once per step leave L2 first; a block every decoder layer
     // reads again (one memory group for all layers) keeps the normal policy
     const uint64_t kv_policy = kv_reuse ? l2_evict_normal_policy() : l2_evict_first_policy();
@@ -303,7 +313,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
       }
       if (progress) {
         t0 = globaltimer_ns();
-      } else if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      } else if (globaltimer_ns() - t0 > wait_limit) {
         atomicExch(s_abort, 1);
         set_error(err, DEV_ERR_TIMEOUT);
         break;
@@ -312,7 +322,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
     // let every copy this CTA issued land before the CTA may exit
     for (int w = 0; w < NC; w++)
       for (int k = max(0, issued[w] - SW); k < issued[w]; k++)
-        mbar_wait_bounded(&full[w * SW + k % SW], (unsigned)((k / SW) & 1), WAIT_LIMIT_NS);
+        mbar_wait_bounded(&full[w * SW + k % SW], (unsigned)((k / SW) & 1), wait_limit);
     return;
   }
 
@@ -326,7 +336,7 @@ __global__ void __launch_bounds__((NC + 1) * 32)
   for (int k = 0;; k++) {
     const int s = warp * SW + k % SW;
     uint8_t *stg = smem + (size_t)s * S::STAGE;
-    if (!mbar_wait_bounded(&full[s], (unsigned)((k / SW) & 1), WAIT_LIMIT_NS)) {
+    if (!mbar_wait_bounded(&full[s], (unsigned)((k / SW) & 1), wait_limit)) {
       if (lane == 0) {  // the stream failed: nothing more will come
         atomicExch(s_abort, 1);
         set_error(err, DEV_ERR_TIMEOUT);
@@ -445,22 +455,28 @@ __global__ void __launch_bounds__((NC + 1) * 32)
   }
 }
 
-// Resident CTAs of a persistent attention launch (SMs x occupancy), cached.
+// Resident CTAs of a persistent attention launch (SMs x occupancy) on the
+// current device, cached per device; also raises the kernel's shared-memory
+// limit on that device. 0 if the device cannot be queried.
 template <typename T, int DH, int NC = AttnCfg::NC, int SW = AttnCfg::SW,
           int TB = AttnCfg::TILE_BYTES>
 int attn_grid_ctas() {
-  static int ctas = 0;
-  if (!ctas) {
-    int dev = 0, sms = 0, occ = 0;
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static int ctas[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 0;
+  std::lock_guard<std::mutex> g(mu);
+  if (!ctas[dev]) {
+    int sms = 0, occ = 0;
     constexpr int smem = attn_smem_bytes<T, DH, NC, SW, TB>();
     auto kern = k_attn_decode<T, DH, NC, SW, TB>;
-    cudaGetDevice(&dev);
+    if (ensure_smem_limit(kern, smem) != cudaSuccess) return 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, (NC + 1) * 32, smem);
-    ctas = (sms > 0 ? sms : 148) * (occ > 0 ? occ : 1);
+    ctas[dev] = (sms > 0 ? sms : 148) * (occ > 0 ? occ : 1);
   }
-  return ctas;
+  return ctas[dev];
 }
 
 // CTAs for `units` units: as few consumer warps as give every warp the same
@@ -469,7 +485,9 @@ int attn_grid_ctas() {
 template <typename T, int DH, int NC = AttnCfg::NC, int SW = AttnCfg::SW,
           int TB = AttnCfg::TILE_BYTES>
 int attn_balanced_ctas(int units) {
-  const int max_warps = attn_grid_ctas<T, DH, NC, SW, TB>() * NC;
+  const int ctas = attn_grid_ctas<T, DH, NC, SW, TB>();
+  if (ctas <= 0) return 0;  // the launch then fails and reports the CUDA error
+  const int max_warps = ctas * NC;
   const int k = (units + max_warps - 1) / max_warps;
   const int warps = (units + k - 1) / k;
   return (warps + NC - 1) / NC;

@@ -5,6 +5,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 namespace rlt {
 
 using bf16 = __nv_bfloat16;
@@ -16,6 +20,34 @@ enum : int { DEV_OK = 0, DEV_ERR_TOKEN = 8, DEV_ERR_TIMEOUT = 7 };
 
 __device__ __forceinline__ void set_error(int *err, int code) {
   atomicCAS(err, 0, code);
+}
+
+// Failure-detection controls in device memory, set from the host between
+// steps (rlt_set_fault): a planted fault and the bound of the device waits
+// that read them (0 = the kernel's default bound).
+enum : int { DEV_FAULT_NONE = 0, DEV_FAULT_SKIP_ATTN_PRODUCER = 1 };
+struct DevCtl {
+  int fault;
+  int pad;
+  unsigned long long wait_limit_ns;
+};
+
+// cudaFuncSetAttribute applies to the device that is current when it is
+// called, so a kernel's dynamic shared-memory limit is raised once per
+// (kernel, device) pair, under a lock (a process may drive several devices).
+template <typename Kern>
+cudaError_t ensure_smem_limit(Kern *kern, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void *>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const std::pair<int, const void *> key{dev, reinterpret_cast<const void *>(kern)};
+  std::lock_guard<std::mutex> g(mu);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
 }
 
 __device__ __forceinline__ float to_f(float x) { return x; }

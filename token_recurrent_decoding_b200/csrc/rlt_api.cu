@@ -29,13 +29,13 @@ using namespace rlt;
 
 namespace {
 
-constexpr int XCH = 1024;  // memory positions per cross-attention split
+constexpr int XCH = RLT_ATTEND_CHUNK;  // memory positions per cross-attention split
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
   // persistent state
-  size_t s, t_dec, t_enc, e, mem, ring, rope, err;
+  size_t s, t_dec, t_enc, e, mem, ring, rope, err, ctl;
   // decoder step work buffers (max_seqs rows)
   size_t nready, ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part, counters;
   size_t nsq;  // per-row partial sums of squares of h over 32-column tiles (bf16 models)
@@ -96,6 +96,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->ring = take(LD * S * H * 2 * W * dh * es);
   L->rope = take(T * (dh / 2) * 8);
   L->err = take(16);
+  L->ctl = take(sizeof(DevCtl));
   L->nready = take(2 * 4);
   L->ready = take(S * 4);
   L->pos = take(S * 4);
@@ -288,11 +289,7 @@ cudaError_t launch_tc(rlt_model *M, int m_grid, int a_rows, int a_row0, int n, i
   const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
   if (!ma || !mb) return cudaErrorInvalidValue;
   auto kern = k_gemm_tc<BN, STAGES, Epi>;
-  static bool attr = false;
-  if (!attr) {
-    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    attr = true;
-  }
+  RLT_TRY(ensure_smem_limit(kern, smem));
   dim3 grid((n + BN - 1) / BN, (m_grid + TC_BM - 1) / TC_BM);
   return launch_k(kern, grid, dim3(128), smem, st, *ma, *mb, m_grid, a_row0, n, k, epi,
                   M->at<int>(M->L.err));
@@ -317,12 +314,7 @@ cudaError_t launch_dec_s(rlt_model *M, int m_grid, const int *Mdev, int a_row0, 
   const int kb_max = (kb + S - 1) / S;
   const int ns = kb_max < STAGES ? kb_max : STAGES;
   auto kern = k_gemm_dec<BN, STAGES, S, Epi>;
-  static bool attr = false;
-  if (!attr) {
-    RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DecSmem<BN>::bytes(STAGES)));
-    attr = true;
-  }
+  RLT_TRY(ensure_smem_limit(kern, DecSmem<BN>::bytes(STAGES)));
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(tiles, (m_grid + TC_BM - 1) / TC_BM, S);
   cfg.blockDim = dim3(DEC_THREADS);
@@ -481,7 +473,7 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
                   M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
                   M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH),
                   (window == 0 && c.mem_groups == 1 && c.n_dec_layers > 1) ? 1 : 0,
-                  M->at<int>(L.err));
+                  M->at<int>(L.err), (const DevCtl *)M->at<DevCtl>(L.ctl));
 }
 
 // fp32 models: exact SIMT GEMMs with separate RMSNorm and rotary kernels.
@@ -697,14 +689,8 @@ cudaError_t enc_attention(rlt_model *M, int ntok, int nblk, const T *Qh, const T
   const int H = M->cfg.n_heads;
   if constexpr (std::is_same<T, bf16>::value && DH >= 32) {
     constexpr int smem = FaSmem<DH>::BYTES;
-    static bool attr = false;
-    if (!attr) {
-      RLT_TRY(cudaFuncSetAttribute(k_enc_flash<DH, false>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-      RLT_TRY(cudaFuncSetAttribute(k_enc_flash<DH, true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-      attr = true;
-    }
+    RLT_TRY(ensure_smem_limit(k_enc_flash<DH, false>, smem));
+    RLT_TRY(ensure_smem_limit(k_enc_flash<DH, true>, smem));
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
     if (Qlo)
       k_enc_flash<DH, true><<<dim3(nblk, H), 128, smem, st>>>(
@@ -1196,7 +1182,7 @@ cudaError_t attend_launch(const float *q, const void *kv, const int32_t *h_lengt
       (const int *)nullptr, q, static_cast<const T *>(kv), (long)H * 2 * cap * DH,
       2L * cap * DH, (long)cap * DH, reinterpret_cast<float *>(ws + w.part),
       reinterpret_cast<int *>(ws + w.counters), static_cast<T *>(out),
-      1.0f / sqrtf((float)DH), 0, reinterpret_cast<int *>(ws + w.err));
+      1.0f / sqrtf((float)DH), 0, reinterpret_cast<int *>(ws + w.err), (const DevCtl *)nullptr);
   return cudaGetLastError();
 }
 
@@ -1729,6 +1715,16 @@ RLT_API int rlt_get_stats(rlt_model *M, rlt_stats *out) {
   }
   M->pending.clear();
   *out = M->stats;
+  return RLT_OK;
+}
+
+RLT_API int rlt_set_fault(rlt_model *M, int fault, int64_t wait_limit_ns) {
+  if (!M || wait_limit_ns < 0) return RLT_ERR_INVALID_ARG;
+  if (fault != RLT_FAULT_NONE && fault != RLT_FAULT_SKIP_ATTN_PRODUCER) return RLT_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(M->last_stream) != cudaSuccess) return RLT_ERR_CUDA;
+  DevCtl c{fault, 0, (unsigned long long)wait_limit_ns};
+  if (cudaMemcpy(M->at<DevCtl>(M->L.ctl), &c, sizeof(c), cudaMemcpyHostToDevice) != cudaSuccess)
+    return RLT_ERR_CUDA;
   return RLT_OK;
 }
 

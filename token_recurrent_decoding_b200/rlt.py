@@ -57,6 +57,7 @@ class rlt_weights(C.Structure):
 
 
 K_XATTN, K_SWA, K_GEMM, K_OTHER, K_ENC = range(5)
+FAULT_NONE, FAULT_SKIP_ATTN_PRODUCER = 0, 1
 K_NAMES = ("xattn", "swa", "gemm", "other", "encoder")
 
 
@@ -88,6 +89,7 @@ def _declare(lib):
     lib.rlt_set_state.argtypes = [P, I, P, P, C.c_int64, P]
     lib.rlt_get_encoder_output.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
     lib.rlt_poll_device_error.argtypes = [P]
+    lib.rlt_set_fault.argtypes = [P, I, C.c_int64]
     lib.rlt_attend_workspace_bytes.argtypes = [I, I, I, I]
     lib.rlt_attend_workspace_bytes.restype = C.c_size_t
     lib.rlt_attend.argtypes = [P, P, P, I, I, I, I, I, P, P, C.c_size_t, P]
@@ -363,6 +365,11 @@ class Model:
             out[name] = {"launches": int(st.kernel_launches[k]), "ms": float(st.kernel_ms[k]),
                          "bytes": float(st.kernel_bytes[k]), "flops": float(st.kernel_flops[k])}
         return out
+
+    def set_fault(self, fault: int, wait_limit_ns: int = 0):
+        """Plant a fault (FAULT_*) in later decoder-attention launches and
+        bound their device waits (0 = default); FAULT_NONE clears it."""
+        _check(_lib().rlt_set_fault(self._h, int(fault), int(wait_limit_ns)), "rlt_set_fault")
 
     def poll_device_error(self) -> int:
         return int(_lib().rlt_poll_device_error(self._h))
