@@ -27,12 +27,23 @@ def _case(n, H, dh, cap, lengths, dtype, seed=0):
 
 
 def _check(q, kv, out, lengths, rows, tol):
+    """bf16 outputs (tol 1e-2): each element is one round-to-nearest-even of
+    the fp32 result, so its error is bounded element by element, 2^-8 |ref|
+    (twice the half-ulp bound), plus 1e-3 RMS for the fp32 accumulation; a
+    bound relative to the row RMS alone fails long rows, whose average of
+    many values has an RMS well below its largest element. fp32 outputs:
+    accumulation only, tol x RMS."""
     for i in rows:
         L = lengths[i]
         for h in range(q.shape[1]):
             ref = oracle.attend(q[i, h], kv[i, h, 0, :L], kv[i, h, 1, :L])
-            err = np.abs(out[i, h] - ref).max()
-            assert err <= tol * max(np.sqrt(np.mean(ref ** 2)), 1e-3), (i, h, L, err)
+            scale = max(np.sqrt(np.mean(ref ** 2)), 1e-3)
+            if tol >= 1e-2:
+                bound = 2.0 ** -8 * np.abs(ref) + 1e-3 * scale
+            else:
+                bound = tol * scale
+            err = np.abs(out[i, h] - ref)
+            assert (err <= bound).all(), (i, h, L, float(err.max()))
 
 
 @pytest.mark.parametrize("dtype,dh", [(torch.bfloat16, 64), (torch.bfloat16, 128),
