@@ -78,7 +78,7 @@ typedef struct rlt_config {
   int ffn_dim;      /* F */
   int ffn_kind;     /* RLT_GELU: W2 GELU(W1 u); RLT_SWIGLU: W2 (SiLU(Wa u) * Wb u) */
   int vocab;        /* V */
-  int window;       /* W >= 1 */
+  int window;       /* W >= 1, at most RLT_ATTEND_CHUNK (1024) */
   int mem_groups;   /* G: 1 or n_dec_layers */
   int tied;         /* 1: decoder layer l uses encoder layer l's q/k/v, o and
                        FFN matrices ([RLT-96] "Architecture", tied config) */
@@ -190,6 +190,29 @@ RLT_API int rlt_run_sequence(rlt_model *model, const int32_t *h_seq_ids, int n,
 RLT_API int rlt_decoder_parallel(rlt_model *model, const int32_t *h_seq_ids, int n,
                                  int n_steps, float *s_all, rlt_stream stream);
 
+/* How a bf16 model's decoder step runs.
+ *   RLT_STEP_FUSED: one launch of a persistent kernel per step. Thread-block
+ *     clusters, as many as can be resident, walk the step's work -- GEMM
+ *     tiles of every projection on the tensor cores, attention units, the
+ *     gather and the final norm -- in one global order (layer, sublayer
+ *     phase, 128-row tile), each waiting on dependency counters in the arena
+ *     instead of on kernel boundaries ([RLT-96] "Three design principles and
+ *     their caveats": kernel fusion and batched ready updates). The default
+ *     for bf16 models it covers (up to 8192 slots, 64 decoder layers).
+ *   RLT_STEP_CHAIN: a captured chain of about eight kernels per decoder
+ *     block (the only form for fp32 models).
+ * Both compute the same transition; results agree within the bf16
+ * tolerance, not bit for bit (different split-K partitions). */
+enum { RLT_STEP_CHAIN = 0, RLT_STEP_FUSED = 1 };
+
+/* Select the step kernel for later steps. Errors: INVALID_ARG (unknown
+ * kind), UNSUPPORTED (RLT_STEP_FUSED for a model it does not cover). */
+RLT_API int rlt_set_step_kernel(rlt_model *model, int kind);
+
+/* The step kernel later steps use (RLT_STEP_CHAIN or RLT_STEP_FUSED); -1 for
+ * a NULL model. */
+RLT_API int rlt_get_step_kernel(rlt_model *model);
+
 /* Ready-set scheduler: sequence h_seq_ids[i] still needs h_steps[i]
  * transitions. Each tick batches every sequence with a pending step into one
  * decoder step, until none is left (ragged batches: sequences drop out as
@@ -291,7 +314,8 @@ enum {
   RLT_K_GEMM = 2,  /* decoder projections / FFN / gate GEMMs */
   RLT_K_OTHER = 3, /* decoder norms, rotary/ring writes, gather, final norm */
   RLT_K_ENC = 4,   /* every encoder prefill kernel */
-  RLT_K_COUNT = 5
+  RLT_K_STEP = 5,  /* the persistent decoder-step kernel (a whole step, one launch) */
+  RLT_K_COUNT = 6
 };
 
 typedef struct rlt_stats {

@@ -40,11 +40,25 @@ def test_encoder_and_memory_parity(name, lengths):
         assert rel_l2(mem_g, mr) <= trel
 
 
-@pytest.mark.parametrize("name", list(SMALL))
-def test_stepwise_parity_on_gpu_state(name):
+KERNELS = [(n, k) for n in SMALL for k in ("fused", "chain")
+           if k == "chain" or SMALL[n].dtype == configs.BF16]
+
+
+def _use(m, kernel):
+    from token_recurrent_decoding_b200 import rlt as R
+    if m.cfg.dtype == configs.BF16:
+        assert m.get_step_kernel() == R.STEP_FUSED  # the default for bf16 models
+    m.set_step_kernel(R.STEP_FUSED if kernel == "fused" else R.STEP_CHAIN)
+
+
+@pytest.mark.parametrize("name,kernel", KERNELS)
+def test_stepwise_parity_on_gpu_state(name, kernel):
+    """Both step kernels of a bf16 model (the persistent one-launch step and
+    the chain of kernels), and the fp32 chain."""
     cfg = SMALL[name]
     T = 40
     m, w, tok = make_model(cfg, [T] * 3)
+    _use(m, kernel)
     o = oracle.Oracle(cfg, w)
     e_g, mem_g = (to_np(x) for x in m.get_encoder_output(1))
     checks = sorted({0, 1, cfg.window - 1, cfg.window, cfg.window + 1, 23, T - 1})
@@ -69,11 +83,12 @@ def test_stepwise_parity_on_gpu_state(name):
                 np.testing.assert_array_equal(to_np(c_new)[:, :, :-1], c_prev[:, :, 1:])
 
 
-@pytest.mark.parametrize("name", list(SMALL))
-def test_trajectory_parity_from_tokens(name):
+@pytest.mark.parametrize("name,kernel", KERNELS)
+def test_trajectory_parity_from_tokens(name, kernel):
     cfg = SMALL[name]
     B, T = 2, 64
     m, w, tok = make_model(cfg, [T] * B)
+    _use(m, kernel)
     o = oracle.Oracle(cfg, w)
     tol = TRAJ_TOL[cfg.dtype]
     ref0, _, _ = o.run(tok[0])
@@ -266,14 +281,16 @@ def test_encoder_is_causal_at_full_size_bitwise():
         assert not torch.equal(e0[k + 1:], e1[k + 1:])
 
 
-@pytest.mark.parametrize("name", ["ragged_like", "tied_like", "m140_like"])
-def test_stepwise_parity_past_one_memory_chunk(name):
+@pytest.mark.parametrize("name,kernel", [("ragged_like", "fused"), ("tied_like", "fused"),
+                                         ("m140_like", "fused"), ("m140_like", "chain")])
+def test_stepwise_parity_past_one_memory_chunk(name, kernel):
     """Positions past 1024: the cross-attention over M<=t splits into several
     1024-row chunks (partials merged in chunk order, a ragged tail chunk);
     step-wise against the oracle fed the GPU's own state."""
     cfg = SMALL[name]
     T = 2100
     m, w, tok = make_model(cfg, [T] * 2)
+    _use(m, kernel)
     o = oracle.Oracle(cfg, w)
     e_g, mem_g = (to_np(x) for x in m.get_encoder_output(1))
     tol = STEP_TOL[cfg.dtype]
@@ -293,7 +310,8 @@ def test_stepwise_parity_past_one_memory_chunk(name):
             win_ref[:, :, -1])
 
 
-def test_bounded_wait_timeout_is_reported_and_model_recovers():
+@pytest.mark.parametrize("kernel", ["fused", "chain"])
+def test_bounded_wait_timeout_is_reported_and_model_recovers(kernel):
     """Failure detection without faulting the GPU: a planted fault makes the
     decoder attention's producer fill nothing, so its consumers' bounded waits
     (limited to 2 ms for the test) run out; the step returns, the device error
@@ -303,6 +321,7 @@ def test_bounded_wait_timeout_is_reported_and_model_recovers():
     cfg = SMALL["m50_like"]
     lengths = [24, 24]
     m, w, tok = make_model(cfg, lengths)
+    _use(m, kernel)
     m.set_fault(R.FAULT_SKIP_ATTN_PRODUCER, 2_000_000)
     m.decoder_step([0, 1])
     assert m.poll_device_error() == 7  # RLT_ERR_TIMEOUT
@@ -312,8 +331,30 @@ def test_bounded_wait_timeout_is_reported_and_model_recovers():
     m.run_sequence([0, 1], 24)
     assert m.poll_device_error() == 0
     ref, _, _ = make_model(cfg, lengths)
+    _use(ref, kernel)
     ref.run_sequence([0, 1], 24)
     for i in range(2):
         assert torch.equal(m.get_state(i)[0], ref.get_state(i)[0])
     with pytest.raises(RLTError):
         m.set_fault(99, 0)
+
+
+def test_fused_and_chain_kernels_agree():
+    """The persistent one-launch step and the chain of kernels compute the
+    same transition (bf16 tolerance: different split-K partitions), on a
+    batch of more than one 128-row tile, for a whole trajectory."""
+    cfg = SMALL["m140_like"]
+    lengths = [70] * 200
+    a, w, tok = make_model(cfg, lengths)
+    b, _, _ = make_model(cfg, lengths)
+    _use(a, "fused")
+    _use(b, "chain")
+    ids = list(range(len(lengths)))
+    a.run_sequence(ids, 70)
+    b.run_sequence(ids, 70)
+    for i in (0, 99, 127, 128, 199):
+        assert rel_l2(to_np(a.get_state(i)[0]), to_np(b.get_state(i)[0])) <= TRAJ_TOL[cfg.dtype]
+    o = oracle.Oracle(cfg, w)
+    for i in (0, 150):
+        assert rel_l2(to_np(a.get_state(i)[0]), o.run(tok[i])[1]) <= TRAJ_TOL[cfg.dtype]
+    assert a.poll_device_error() == 0

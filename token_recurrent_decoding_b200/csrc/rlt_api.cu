@@ -24,6 +24,7 @@
 #include "enc_attn.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_dec.cuh"
+#include "step_fused.cuh"
 
 using namespace rlt;
 
@@ -42,8 +43,10 @@ struct Layout {
   // encoder work buffers (ptok rows)
   size_t tok, tok_slot, tok_pos, tok_start, blk, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
   size_t staging, staging_bytes;
+  // persistent step kernel: dependency counters + abort word, tensor-map table
+  size_t fs_cnt, fs_cnt_bytes, fs_maps;
   size_t total;
-  int max_chunks, ptok;
+  int max_chunks, ptok, fs_rt;
 };
 
 int elem_size(const rlt_config *c) { return c->dtype == RLT_BF16 ? 2 : 4; }
@@ -57,6 +60,8 @@ int check_config(const rlt_config *c) {
     return RLT_ERR_INVALID_ARG;
   if (c->ffn_dim <= 0 || c->vocab <= 0 || c->window < 1 || c->max_seqs < 1 || c->max_len < 1)
     return RLT_ERR_INVALID_ARG;
+  // the sliding window is attended as one chunk of the decode attention
+  if (c->window > RLT_ATTEND_CHUNK) return RLT_ERR_UNSUPPORTED;
   if (c->ffn_kind != RLT_GELU && c->ffn_kind != RLT_SWIGLU) return RLT_ERR_INVALID_ARG;
   if (c->dtype != RLT_F32 && c->dtype != RLT_BF16) return RLT_ERR_INVALID_ARG;
   if (c->mem_groups != 1 && c->mem_groups != c->n_dec_layers) return RLT_ERR_UNSUPPORTED;
@@ -132,6 +137,10 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   size_t st = std::max(LD * 2 * (W > 1 ? W - 1 : 1) * d * es, G * T * 2 * d * es);
   L->staging_bytes = st;
   L->staging = take(st);
+  L->fs_rt = (int)((S + FS_RT - 1) / FS_RT);
+  L->fs_cnt_bytes = ((LD + 1) * FS_NPH * (size_t)L->fs_rt + 1) * 4;
+  L->fs_cnt = take(L->fs_cnt_bytes);
+  L->fs_maps = take(c->dtype == RLT_BF16 ? fs_map_count((int)LD) * sizeof(CUtensorMap) : 0);
   L->total = off;
   return off;
 }
@@ -195,6 +204,13 @@ struct rlt_model {
   // TMA descriptors of bf16 [rows][cols] matrices, keyed by (pointer, rows, cols, box rows)
   std::map<std::tuple<const void *, uint64_t, uint64_t, uint32_t>, CUtensorMap> tmaps;
   cudaError_t (*step)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
+  // persistent step kernel (bf16 models): one launch per decoder step
+  bool fused_ok = false;   // set up and covering this model
+  bool use_fused = false;  // decoder steps run it (rlt_set_step_kernel)
+  int fs_ctas = 0;         // CTAs of a launch: resident clusters x FS_S
+  FsParams fs{};           // everything but the per-step fields
+  cudaError_t (*step_fused)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
+  cudaError_t (*fused_setup)(rlt_model *) = nullptr;
   cudaError_t (*prefill)(rlt_model *, int, int, cudaStream_t) = nullptr;
   cudaError_t (*dpar)(rlt_model *, int, int, int, float *, cudaStream_t) = nullptr;
   cudaError_t (*get_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
@@ -677,6 +693,175 @@ cudaError_t step_impl_tc(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Algorithmic bytes and FLOPs of one decoder step over the rows of `si`
+// (counted once: weights once per launch; per row e_t and s_{t-1} in, s_t
+// out; per layer the retained window read and the new k/v written; the memory
+// rows 0..t once per group, a shared group once per step).
+void step_traffic(const rlt_model *M, const StepInfo &si, double *bytes, double *flops) {
+  const rlt_config &c = M->cfg;
+  const double d = c.d, F = c.ffn_dim, L = c.n_dec_layers, n = si.n;
+  const double es = c.dtype == RLT_BF16 ? 2.0 : 4.0;
+  const double ffn = (c.ffn_kind == RLT_SWIGLU ? 3.0 : 2.0) * d * F;
+  const double params = (c.alpha != 0.0f ? 2.0 * d * d : 0.0) + L * (6.0 * d * d + ffn);
+  const double g_eff = c.mem_groups == 1 ? 1.0 : L;
+  *bytes = params * es + n * (d * es + 8.0 * d) + L * (si.sum_win - n) * 2.0 * d * es +
+           L * n * 2.0 * d * es + g_eff * si.sum_keys * 2.0 * d * es;
+  *flops = 2.0 * params * n + L * 4.0 * d * (si.sum_win + si.sum_keys);
+}
+
+// One decoder step as ONE launch of the persistent step kernel
+// (step_fused.cuh): the dependency counters are cleared, then every cluster
+// that can be resident runs. No programmatic overlap with the previous
+// kernel: the kernel relies on all its clusters being resident at once.
+template <int DH>
+cudaError_t step_impl_fused(rlt_model *M, const StepInfo &si, cudaStream_t st) {
+  const Layout &L = M->L;
+  FsParams P = M->fs;
+  P.xch = si.xchunks;
+  P.n_dev = M->at<int>(L.nready) + si.chain;
+  double bytes = 0, flops = 0;
+  step_traffic(M, si, &bytes, &flops);
+  Span sp(M, st, RLT_K_STEP, bytes, flops);
+  RLT_TRY(cudaMemsetAsync(M->at<uint8_t>(L.fs_cnt), 0, L.fs_cnt_bytes, st));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(M->fs_ctas);
+  cfg.blockDim = dim3(FS_THREADS);
+  cfg.dynamicSmemBytes = FsSmem<DH>::BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = FS_S;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_step_fused<DH>, P);
+}
+
+// Set-up of the persistent step kernel at rlt_create: the tensor-map table
+// (activation buffers and every decoder weight) in the arena, the number of
+// clusters that can be resident, and the launch-invariant parameters.
+// Returns an error (and the model keeps the chain of kernels) when the
+// kernel does not cover the model.
+template <int DH> cudaError_t fused_setup_impl(rlt_model *M) {
+  using T = bf16;
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const int d = c.d, F = c.ffn_dim, LD = c.n_dec_layers, S = c.max_seqs;
+  constexpr int BNQ = FsSmem<DH>::BNQ;
+  if (L.fs_rt > FS_MAX_RT || LD > FS_MAX_LAYERS) return cudaErrorNotSupported;
+  if ((3 * d) % BNQ || d % 64 || F % 64) return cudaErrorNotSupported;
+  std::vector<CUtensorMap> maps(fs_map_count(LD));
+  bool ok = true;
+  auto put = [&](int idx, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box) {
+    const CUtensorMap *m = ok ? tmap_bf16(M, ptr, rows, cols, box) : nullptr;
+    if (!m) {
+      ok = false;
+      return;
+    }
+    maps[idx] = *m;
+  };
+  put(MAP_A_XIN, M->at<T>(L.xin), S, 2 * d, TC_BM);
+  put(MAP_A_U, M->at<T>(L.u), S, d, TC_BM);
+  put(MAP_A_A, M->at<T>(L.a), S, d, TC_BM);
+  put(MAP_A_F, M->at<T>(L.f), S, F, TC_BM);
+  if (c.alpha != 0.0f)
+    put(MAP_GATE, M->w.gate_w, d, 2 * d, 32);
+  else if (ok)
+    maps[MAP_GATE] = maps[MAP_A_XIN];  // never read
+  for (int l = 0; l < LD && ok; l++) {
+    put(fs_map_index(l, MAPL_QKV), W_<T>::qkv(M, l), 3 * d, d, BNQ);
+    put(fs_map_index(l, MAPL_O), W_<T>::o(M, l), d, d, 32);
+    put(fs_map_index(l, MAPL_QX), M->w.dec_wqx[l], d, d, 32);
+    put(fs_map_index(l, MAPL_OX), M->w.dec_wox[l], d, d, 32);
+    put(fs_map_index(l, MAPL_W1), W_<T>::w1(M, l), F, d, 64);
+    if (c.ffn_kind == RLT_SWIGLU)
+      put(fs_map_index(l, MAPL_WB), W_<T>::wb(M, l), F, d, 64);
+    else if (ok)
+      maps[fs_map_index(l, MAPL_WB)] = maps[fs_map_index(l, MAPL_W1)];  // never read
+    put(fs_map_index(l, MAPL_W2), W_<T>::w2(M, l), d, F, 32);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  RLT_TRY(cudaMemcpy(M->at<uint8_t>(L.fs_maps), maps.data(), maps.size() * sizeof(CUtensorMap),
+                     cudaMemcpyHostToDevice));
+  auto kern = k_step_fused<DH>;
+  constexpr int smem = FsSmem<DH>::BYTES;
+  RLT_TRY(ensure_smem_limit(kern, smem));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(FS_S * M->num_sms);
+  cfg.blockDim = dim3(FS_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = FS_S;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  RLT_TRY(cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg));
+  if (clusters < 1) return cudaErrorNotSupported;
+  M->fs_ctas = clusters * FS_S;
+
+  FsParams &P = M->fs;
+  P = FsParams{};
+  P.n_dev = M->at<int>(L.nready);
+  P.ready = M->at<int>(L.ready);
+  P.t_dec = M->at<int>(L.t_dec);
+  P.pos = M->at<int>(L.pos);
+  P.e = M->at<T>(L.e);
+  P.s = M->at<float>(L.s);
+  P.xin = M->at<T>(L.xin);
+  P.a = M->at<T>(L.a);
+  P.u = M->at<T>(L.u);
+  P.f = M->at<T>(L.f);
+  P.e32 = M->at<float>(L.e32);
+  P.s32 = M->at<float>(L.s32);
+  P.h = M->at<float>(L.h);
+  P.q = M->at<float>(L.q);
+  P.fa = M->at<float>(L.fa);
+  P.nsq = M->at<float>(L.nsq);
+  P.ring = M->at<T>(L.ring);
+  P.mem = M->at<T>(L.mem);
+  P.rope = M->at<float2>(L.rope);
+  P.part = M->at<float>(L.part);
+  P.counters = M->at<int>(L.counters);
+  P.cnt = M->at<int>(L.fs_cnt);
+  P.abort = P.cnt + (size_t)(LD + 1) * FS_NPH * L.fs_rt;
+  P.err = M->at<int>(L.err);
+  P.ctl = M->at<DevCtl>(L.ctl);
+  P.maps = M->at<CUtensorMap>(L.fs_maps);
+  P.gate_b = (const float *)M->w.gate_b;
+  P.lnf = (const float *)M->w.dec_lnf;
+  for (int l = 0; l < LD; l++) {
+    P.ln1[l] = (const float *)M->w.dec_ln1[l];
+    P.ln2[l] = (const float *)M->w.dec_ln2[l];
+    P.ln3[l] = (const float *)M->w.dec_ln3[l];
+  }
+  P.d = d;
+  P.H = c.n_heads;
+  P.F = F;
+  P.W = c.window;
+  P.L = LD;
+  P.G = c.mem_groups;
+  P.max_len = c.max_len;
+  P.max_seqs = S;
+  P.swiglu = c.ffn_kind == RLT_SWIGLU;
+  P.alpha0 = c.alpha == 0.0f;
+  P.xch = 1;
+  P.max_chunks = L.max_chunks;
+  P.CH = XCH;
+  P.rt_max = L.fs_rt;
+  P.kv_reuse = (c.mem_groups == 1 && LD > 1) ? 1 : 0;
+  P.alpha = c.alpha;
+  P.eps = c.rms_eps;
+  P.inv_d = 1.0f / (float)d;
+  P.scale = 1.0f / sqrtf((float)DH);
+  P.ring_layer = (long)S * c.n_heads * 2 * c.window * DH;
+  P.mem_group = (long)S * c.n_heads * 2 * c.max_len * DH;
+  return cudaSuccess;
+}
+
 // Encoder over one chunk of ntok tokens already staged in the arena (token
 // ids, slot, position, sequence start), then the memory projection
 // ([RLT-96] "Architecture"; [RLT-TC] "What is this technology").
@@ -915,10 +1100,13 @@ cudaError_t get_memory_impl(rlt_model *M, int seq, int t_enc, cudaStream_t st) {
 }
 
 template <typename T, int DH> void bind(rlt_model *M) {
-  if constexpr (std::is_same<T, bf16>::value)
+  if constexpr (std::is_same<T, bf16>::value) {
     M->step = step_impl_tc<DH>;
-  else
+    M->step_fused = step_impl_fused<DH>;
+    M->fused_setup = fused_setup_impl<DH>;
+  } else {
     M->step = step_impl<T, DH>;
+  }
   M->prefill = prefill_impl<T, DH>;
   M->dpar = dpar_impl<T, DH>;
   M->get_window = get_window_impl<T>;
@@ -998,6 +1186,7 @@ int make_chains(const rlt_model *M, const StepInfo &all, StepInfo ch[2]) {
 
 // Launch the chains of one step on `st` (and the side stream).
 cudaError_t launch_chains(rlt_model *M, const StepInfo *ch, int nch, cudaStream_t st) {
+  if (M->use_fused) return M->step_fused(M, ch[0], st);
   if (nch == 1) return M->step(M, ch[0], st);
   RLT_TRY(cudaEventRecord(M->ev_fork, st));
   RLT_TRY(cudaStreamWaitEvent(M->side, M->ev_fork, 0));
@@ -1025,6 +1214,8 @@ cudaError_t fold_profile(rlt_model *M, const rlt_model::ProfGraph &pg, const Ste
     } else if (p.kind == RLT_K_SWA) {
       bytes = si.sum_win * 2.0 * d * es + (double)si.n * d * (4 + es);
       flops = 4.0 * d * si.sum_win;
+    } else if (p.kind == RLT_K_STEP) {
+      step_traffic(M, si, &bytes, &flops);
     }
     M->stats.kernel_ms[p.kind] += ms;
     M->stats.kernel_launches[p.kind] += 1;
@@ -1067,14 +1258,15 @@ cudaError_t enqueue_step(rlt_model *M, const StepInfo &all, cudaStream_t st) {
   const bool prof = M->profiling && M->prof_stride > 0 && (M->step_counter % M->prof_stride == 0);
   M->step_counter++;
   int nch = 1;
-  if (st == nullptr || prof)
+  if (st == nullptr || prof || M->use_fused)
     ch[0] = all;
   else
     nch = make_chains(M, all, ch);
   int nval[2] = {ch[0].n, nch == 2 ? ch[1].n : 0};
   RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.nready), nval, sizeof(nval), cudaMemcpyHostToDevice,
                           st));  // pageable source: staged before return
-  auto key = std::make_tuple(ch[0].n_grid, nch == 2 ? ch[1].n_grid : 0, all.xchunks);
+  auto key = std::make_tuple(ch[0].n_grid, M->use_fused ? -1 : (nch == 2 ? ch[1].n_grid : 0),
+                             all.xchunks);
   const bool saved = M->profiling;
   if (st == nullptr) {  // legacy stream: cannot capture
     M->profiling = prof;
@@ -1341,6 +1533,14 @@ RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *w, void *d_aren
   if (e != cudaSuccess) {
     rlt_destroy(M);
     return RLT_ERR_CUDA;
+  }
+  // bf16 models step with the persistent kernel when it covers them
+  if (M->fused_setup) {
+    if (M->fused_setup(M) == cudaSuccess) {
+      M->fused_ok = M->use_fused = true;
+    } else {
+      cudaGetLastError();
+    }
   }
   *out = M;
   return RLT_OK;
@@ -1736,7 +1936,23 @@ RLT_API int rlt_poll_device_error(rlt_model *M) {
     return RLT_ERR_CUDA;
   if (v != 0 && cudaMemset(M->at<int>(M->L.err), 0, sizeof(int)) != cudaSuccess)
     return RLT_ERR_CUDA;
+  // a step that gave up may have left split-KV merge counters raised
+  if (v != 0 && cudaMemset(M->at<int>(M->L.counters), 0,
+                           sizeof(int) * (size_t)M->cfg.max_seqs * M->cfg.n_heads) != cudaSuccess)
+    return RLT_ERR_CUDA;
   return v;
+}
+
+RLT_API int rlt_set_step_kernel(rlt_model *M, int kind) {
+  if (!M || (kind != RLT_STEP_CHAIN && kind != RLT_STEP_FUSED)) return RLT_ERR_INVALID_ARG;
+  if (kind == RLT_STEP_FUSED && !M->fused_ok) return RLT_ERR_UNSUPPORTED;
+  M->use_fused = kind == RLT_STEP_FUSED;
+  return RLT_OK;
+}
+
+RLT_API int rlt_get_step_kernel(rlt_model *M) {
+  if (!M) return -1;
+  return M->use_fused ? RLT_STEP_FUSED : RLT_STEP_CHAIN;
 }
 
 }  // extern "C"

@@ -4,7 +4,8 @@ Decoder steps at a chosen position:
 
     python -m token_recurrent_decoding_b200.profile_step --workload m140_bf16 --t 512 --steps 2
 
-prefills the encoder for the batch (--max-len shrinks the sequence length and
+prefills the encoder for the batch (--kernel picks the persistent one-launch
+step or the chain of kernels; --max-len shrinks the sequence length and
 so the arena), places every sequence at position t with a
 random state imported through rlt_set_state (s and the window of every layer),
 and runs `steps` decoder steps with direct launches on the legacy stream, so a
@@ -43,6 +44,9 @@ def run_steps(args):
     tok = inputs.make_tokens(cfg.vocab, lengths)
     m = Model(cfg, w, B, T)
     del w
+    if args.kernel:
+        from . import rlt
+        m.set_step_kernel(rlt.STEP_FUSED if args.kernel == "fused" else rlt.STEP_CHAIN)
     flat = torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda()
     offsets = np.arange(B, dtype=np.int32) * T
     m.prefill_encoder(flat, list(range(B)), offsets, lengths)
@@ -72,6 +76,7 @@ def run_steps(args):
     ts = [np.full(B, args.t + k) for k in range(args.steps)]
     byts = [roofline.decoder_step_bytes(cfg, x) for x in ts]
     print(json.dumps({"workload": args.workload, "batch": B, "t": args.t, "graph": args.graph,
+                      "kernel": "fused" if m.get_step_kernel() == 1 else "chain",
                       "step_ms": times, "step_GB": [x / 1e9 for x in byts],
                       "GB_s": [x / (ms / 1e3) / 1e9 for x, ms in zip(byts, times)]}))
 
@@ -112,6 +117,8 @@ def main():
                     help="sequence length of the arena (default: the workload's); small "
                          "values keep a profiler's device memory small")
     ap.add_argument("--graph", action="store_true")
+    ap.add_argument("--kernel", choices=["fused", "chain"], default=None,
+                    help="decoder step kernel (default: the model's default)")
     ap.add_argument("--attend", action="store_true")
     ap.add_argument("--n", type=int, default=256)
     ap.add_argument("--heads", type=int, default=12)

@@ -56,15 +56,16 @@ class rlt_weights(C.Structure):
                 + [("dec_lnf", C.c_void_p)])
 
 
-K_XATTN, K_SWA, K_GEMM, K_OTHER, K_ENC = range(5)
+K_XATTN, K_SWA, K_GEMM, K_OTHER, K_ENC, K_STEP = range(6)
 FAULT_NONE, FAULT_SKIP_ATTN_PRODUCER = 0, 1
-K_NAMES = ("xattn", "swa", "gemm", "other", "encoder")
+STEP_CHAIN, STEP_FUSED = 0, 1
+K_NAMES = ("xattn", "swa", "gemm", "other", "encoder", "step")
 
 
 class rlt_stats(C.Structure):
-    _fields_ = [("launches", C.c_int64), ("kernel_launches", C.c_int64 * 5),
-                ("kernel_ms", C.c_double * 5), ("kernel_bytes", C.c_double * 5),
-                ("kernel_flops", C.c_double * 5)]
+    _fields_ = [("launches", C.c_int64), ("kernel_launches", C.c_int64 * 6),
+                ("kernel_ms", C.c_double * 6), ("kernel_bytes", C.c_double * 6),
+                ("kernel_flops", C.c_double * 6)]
 
 
 _LIB = None
@@ -90,6 +91,8 @@ def _declare(lib):
     lib.rlt_get_encoder_output.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
     lib.rlt_poll_device_error.argtypes = [P]
     lib.rlt_set_fault.argtypes = [P, I, C.c_int64]
+    lib.rlt_set_step_kernel.argtypes = [P, I]
+    lib.rlt_get_step_kernel.argtypes = [P]
     lib.rlt_attend_workspace_bytes.argtypes = [I, I, I, I]
     lib.rlt_attend_workspace_bytes.restype = C.c_size_t
     lib.rlt_attend.argtypes = [P, P, P, I, I, I, I, I, P, P, C.c_size_t, P]
@@ -365,6 +368,13 @@ class Model:
             out[name] = {"launches": int(st.kernel_launches[k]), "ms": float(st.kernel_ms[k]),
                          "bytes": float(st.kernel_bytes[k]), "flops": float(st.kernel_flops[k])}
         return out
+
+    def set_step_kernel(self, kind: int):
+        """STEP_FUSED (one persistent launch per step) or STEP_CHAIN."""
+        _check(_lib().rlt_set_step_kernel(self._h, int(kind)), "rlt_set_step_kernel")
+
+    def get_step_kernel(self) -> int:
+        return int(_lib().rlt_get_step_kernel(self._h))
 
     def set_fault(self, fault: int, wait_limit_ns: int = 0):
         """Plant a fault (FAULT_*) in later decoder-attention launches and
