@@ -511,7 +511,12 @@ __device__ void fs_gemm_task(const FsParams &P, const FsShared &sh, FsRun &run,
 #pragma unroll
     for (int c0 = chh * (BN / 2); c0 < (chh + 1) * (BN / 2); c0 += 16) {
       float v[16];
-      tmem_ld16(lane_base + c0, v);
+      if (KB > 0) {
+        tmem_ld16(lane_base + c0, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; j++) v[j] = 0.f;  // short K: this CTA holds no K block
+      }
       float4 *pr = reinterpret_cast<float4 *>(Pt + (size_t)row * P_LD + c0);
 #pragma unroll
       for (int j = 0; j < 4; j++)
