@@ -213,6 +213,24 @@ RLT_API int rlt_set_step_kernel(rlt_model *model, int kind);
  * a NULL model. */
 RLT_API int rlt_get_step_kernel(rlt_model *model);
 
+/* CTAs of one persistent-step launch (0 if the model does not have it). */
+RLT_API int rlt_step_kernel_ctas(rlt_model *model);
+
+/* Measurement hook of the persistent step (no counterpart in the method).
+ * d_buf (device, 8-byte aligned, NULL = off) receives, for every CTA c and
+ * work item k it runs in a step, 4 uint64 words at
+ * ((c * cap + k) * 4): item id, start, dependency met, end, in device
+ * globaltimer nanoseconds; cap = bytes / (32 * rlt_step_kernel_ctas()).
+ * Item id = (layer + 1) << 16 | phase << 8 | row tile, where phase bit 7
+ * marks an attention sublayer (phases: 0 q/k/v GEMM, 1 SWA, 2 W_o, 3 W_qx,
+ * 4 cross-attention, 5 W_ox, 6 FFN up, 7 SwiGLU value half, 8 FFN down;
+ * layer slot L_D: 1 gate GEMM, 0x20 gather, 0x21 final norm). Slots a step
+ * does not use keep their contents: clear the buffer between steps.
+ * Synchronises the model's last stream and drops its captured step graphs.
+ * Errors: INVALID_ARG (misaligned or smaller than one record per CTA),
+ * UNSUPPORTED (no persistent step for this model). */
+RLT_API int rlt_set_step_trace(rlt_model *model, void *d_buf, size_t bytes);
+
 /* Ready-set scheduler: sequence h_seq_ids[i] still needs h_steps[i]
  * transitions. Each tick batches every sequence with a pending step into one
  * decoder step, until none is left (ragged batches: sequences drop out as

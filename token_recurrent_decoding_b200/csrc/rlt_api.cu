@@ -209,6 +209,8 @@ struct rlt_model {
   bool use_fused = false;  // decoder steps run it (rlt_set_step_kernel)
   int fs_ctas = 0;         // CTAs of a launch: resident clusters x FS_S
   FsParams fs{};           // everything but the per-step fields
+  unsigned long long *trace = nullptr;  // measurement hook of the fused step (rlt_set_step_trace)
+  int trace_cap = 0;
   cudaError_t (*step_fused)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
   cudaError_t (*fused_setup)(rlt_model *) = nullptr;
   cudaError_t (*prefill)(rlt_model *, int, int, cudaStream_t) = nullptr;
@@ -718,6 +720,8 @@ cudaError_t step_impl_fused(rlt_model *M, const StepInfo &si, cudaStream_t st) {
   const Layout &L = M->L;
   FsParams P = M->fs;
   P.xch = si.xchunks;
+  P.trace = M->trace;
+  P.trace_cap = M->trace_cap;
   P.n_dev = M->at<int>(L.nready) + si.chain;
   double bytes = 0, flops = 0;
   step_traffic(M, si, &bytes, &flops);
@@ -1947,6 +1951,33 @@ RLT_API int rlt_set_step_kernel(rlt_model *M, int kind) {
   if (!M || (kind != RLT_STEP_CHAIN && kind != RLT_STEP_FUSED)) return RLT_ERR_INVALID_ARG;
   if (kind == RLT_STEP_FUSED && !M->fused_ok) return RLT_ERR_UNSUPPORTED;
   M->use_fused = kind == RLT_STEP_FUSED;
+  return RLT_OK;
+}
+
+RLT_API int rlt_step_kernel_ctas(rlt_model *M) {
+  if (!M) return -1;
+  return M->fused_ok ? M->fs_ctas : 0;
+}
+
+RLT_API int rlt_set_step_trace(rlt_model *M, void *d_buf, size_t bytes) {
+  if (!M) return RLT_ERR_INVALID_ARG;
+  if (d_buf && !M->fused_ok) return RLT_ERR_UNSUPPORTED;
+  const size_t per = (size_t)(M->fs_ctas > 0 ? M->fs_ctas : 1) * 4 * sizeof(unsigned long long);
+  if (d_buf && (((uintptr_t)d_buf & 7) || bytes < per)) return RLT_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(M->last_stream) != cudaSuccess) return RLT_ERR_CUDA;
+  // captured step graphs hold the old parameters: drop them
+  for (auto &g : M->graphs) cudaGraphExecDestroy(g.second.exec);
+  M->graphs.clear();
+  for (auto &g : M->prof_graphs) {
+    cudaGraphExecDestroy(g.second.exec);
+    for (auto &p : g.second.spans) {
+      cudaEventDestroy(p.a);
+      cudaEventDestroy(p.b);
+    }
+  }
+  M->prof_graphs.clear();
+  M->trace = static_cast<unsigned long long *>(d_buf);
+  M->trace_cap = d_buf ? (int)std::min<size_t>(bytes / per, 1 << 20) : 0;
   return RLT_OK;
 }
 

@@ -114,7 +114,29 @@ struct FsParams {
   int kv_reuse;             // one memory group read by every layer (G = 1, L_D > 1)
   float alpha, eps, inv_d, scale;
   long ring_layer, mem_group;
+  // measurement hook (null: off): per CTA, trace_cap records of 4 words
+  // {item id, start, dependency met, end} in globaltimer nanoseconds
+  unsigned long long *trace;
+  int trace_cap;
 };
+
+// Trace item id: (layer slot + 1) << 16 | phase << 8 | row tile; attention
+// phases carry bit 7 of the phase byte, the gather and final norm use layer
+// slot L_D with phases 0x20 / 0x21.
+__host__ __device__ constexpr int fs_trace_id(int l, int ph, int r, bool attn) {
+  return ((l + 1) << 16) | ((ph | (attn ? 0x80 : 0)) << 8) | r;
+}
+
+__device__ __forceinline__ void fs_trace(const FsParams &P, int &slot, int id, uint64_t t0,
+                                         uint64_t t1, uint64_t t2) {
+  if (!P.trace || slot >= P.trace_cap) return;
+  unsigned long long *e = P.trace + ((size_t)blockIdx.x * P.trace_cap + slot) * 4;
+  e[0] = (unsigned long long)id;
+  e[1] = t0;
+  e[2] = t1;
+  e[3] = t2;
+  slot++;
+}
 
 __device__ __forceinline__ int fs_cnt_index(const FsParams &P, int l, int p, int r) {
   return (l * FS_NPH + p) * P.rt_max + r;
@@ -233,18 +255,20 @@ struct FsCtlSmem {
   int consumed[FS_NC];         // attention stages consumed per consumer warp
   int outputs[8];              // attention outputs written per warp in this phase
   int rows_done[FS_MAX_RT];    // gathered rows per row tile
+  unsigned long long tdep;     // when the attention producer's dependency was met (trace)
 };
 
 template <int DH> struct FsSmem {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int BNQ = DH >= 32 ? DH : 32;  // q/k/v tiles hold whole heads
-  static constexpr int NSQ = BNQ >= 128 ? 3 : 4;  // ring stages of the q/k/v GEMM
-  static constexpr int NS = 4;                    // ring stages of the other GEMMs
+  // ring stages of every GEMM task: one count for the whole launch, so a
+  // stage's barrier phase follows from the k blocks that went through the ring
+  static constexpr int NS = BNQ >= 128 ? 3 : 4;
   static constexpr int stage(int bn) { return A_BYTES + bn * TC_BK * 2; }
   static constexpr int part(int bn) { return TC_BM * (bn + 4) * 4; }
   static constexpr int mx(int a, int b) { return a > b ? a : b; }
   static constexpr int GEMM_BYTES =
-      mx(mx(NSQ * stage(BNQ), part(BNQ)), mx(mx(NS * stage(64), part(64)), NS * stage(32)));
+      mx(mx(NS * stage(BNQ), part(BNQ)), mx(mx(NS * stage(64), part(64)), NS * stage(32)));
   using AS = AttnShape<bf16, DH>;
   static constexpr int ATTN_BYTES = FS_NC * FS_SW * AS::STAGE;
   static constexpr int TILES = mx(GEMM_BYTES, ATTN_BYTES);
@@ -365,7 +389,9 @@ template <int BN, int NS, class Epi>
 __device__ void fs_gemm_task(const FsParams &P, const FsShared &sh, FsRun &run,
                              const CUtensorMap *mA, const CUtensorMap *mB, int m0, int rv,
                              int tile, int K, const int *dep, int dep_target, int *signal,
-                             const Epi &epi, float *s_rs) {
+                             const Epi &epi, float *s_rs, int trace_id, int &tslot) {
+  const uint64_t t_begin = P.trace ? globaltimer_ns() : 0;
+  uint64_t t_dep = 0;
   constexpr int S = FS_S;
   constexpr int A_BYTES = TC_BM * TC_BK * 2, STAGE = A_BYTES + BN * TC_BK * 2;
   constexpr int P_LD = BN + 4;
@@ -406,6 +432,7 @@ __device__ void fs_gemm_task(const FsParams &P, const FsShared &sh, FsRun &run,
         armed++;
       }
       if (ok && dep) ok = fs_wait_count(P, dep, dep_target);
+      if (P.trace) t_dep = globaltimer_ns();
       if (ok) {
         fence_proxy_async_global();  // other CTAs' generic stores -> this TMA
         for (int kb = 0; kb < armed; kb++) {
@@ -535,6 +562,7 @@ __device__ void fs_gemm_task(const FsParams &P, const FsShared &sh, FsRun &run,
   run.task += 1;
   __syncthreads();
   if (threadIdx.x == 0 && ok && signal) fs_signal(signal, 1);
+  if (threadIdx.x == 0) fs_trace(P, tslot, trace_id, t_begin, t_dep, globaltimer_ns());
 }
 
 // ------------------------------------------------------------ attention phase
@@ -594,7 +622,8 @@ template <int KT> struct FsWalk {
 template <int DH>
 __device__ void fs_attn_phase(const FsParams &P, const FsShared &sh, const FsAttnGeom &g,
                               int gcta, int ncta, const int *dep, int dep_target, int *signal,
-                              int *s_skip) {
+                              int *s_skip, int trace_id, int &tslot) {
+  const uint64_t t_begin = P.trace ? globaltimer_ns() : 0;
   using AS = AttnShape<bf16, DH>;
   constexpr int KT = AS::KT, VEC = AS::VEC, LPK = AS::LPK, KPP = AS::KPP, PP = AS::P,
                 PG = AS::PG;
@@ -668,6 +697,7 @@ __device__ void fs_attn_phase(const FsParams &P, const FsShared &sh, const FsAtt
       }
     }
     if (ok && dep) ok = fs_wait_count(P, dep, dep_target);
+    if (P.trace) ctl->tdep = globaltimer_ns();
     if (ok) fence_proxy_async_global();  // the query / ring row writes of other CTAs
     for (int s = 0; s < FS_NC * FS_SW; s++)
       if (qpend >> s & 1) {
@@ -851,6 +881,10 @@ __device__ void fs_attn_phase(const FsParams &P, const FsShared &sh, const FsAtt
     for (int w = 0; w < FS_NC; w++) tot += ctl->outputs[w];
     if (tot > 0 && !fs_aborted(P)) fs_signal(signal, tot);
   }
+  if (threadIdx.x == 0 && P.trace) {
+    fs_trace(P, tslot, trace_id, t_begin, skip ? t_begin : ctl->tdep, globaltimer_ns());
+    ctl->tdep = t_begin;
+  }
   fence_proxy_async_shared();  // header / stage reads before later copies into the region
 }
 
@@ -862,13 +896,13 @@ template <int BN, int NS, class Epi>
 __device__ void fs_gemm_phase(const FsParams &P, const FsShared &sh, FsRun &run, int cl, int C,
                               int &rot, int m0, int rv, int N, int K, int map_a, int map_b,
                               const int *dep, int dep_target, int *signal, const Epi &epi,
-                              float *s_rs) {
+                              float *s_rs, int trace_id, int &tslot) {
   const int T = N / BN;
   int j = (cl - rot) % C;
   if (j < 0) j += C;
   for (; j < T; j += C)
     fs_gemm_task<BN, NS, Epi>(P, sh, run, &P.maps[map_a], &P.maps[map_b], m0, rv, j, K, dep,
-                              dep_target, signal, epi, s_rs);
+                              dep_target, signal, epi, s_rs, trace_id, tslot);
   rot = (rot + T) % C;
 }
 
@@ -920,7 +954,7 @@ __device__ void fs_final_row(const FsParams &P, int i, int lane) {
 template <int DH>
 __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_constant__ FsParams P) {
   using SM = FsSmem<DH>;
-  constexpr int BNQ = SM::BNQ, NSQ = SM::NSQ, NS = SM::NS;
+  constexpr int BNQ = SM::BNQ, NS = SM::NS;
   extern __shared__ uint8_t fs_raw[];
   __shared__ float s_rs[FS_RT];
   __shared__ int s_pos[FS_RT], s_ready[FS_RT];
@@ -956,6 +990,8 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
 
   FsRun run{0, 0};
   int rot = 0;
+  int tslot = 0;  // trace records of this CTA (thread 0)
+  const uint64_t t_start = P.trace ? globaltimer_ns() : 0;
   auto cnt = [&](int l, int ph, int r) { return P.cnt + fs_cnt_index(P, l, ph, r); };
   auto rows_of = [&](int r) { return min(FS_RT, n - r * FS_RT); };
   const RowScaleIn rsi{P.nsq, np, P.inv_d, P.eps};
@@ -969,6 +1005,8 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
   __syncthreads();
   if (threadIdx.x < RT && ctl->rows_done[threadIdx.x] > 0)
     fs_signal(cnt(L, PH_GATHER, threadIdx.x), ctl->rows_done[threadIdx.x]);
+  if (threadIdx.x == 0)
+    fs_trace(P, tslot, fs_trace_id(L, 0x20, 0, false), t_start, t_start, globaltimer_ns());
 
   // ---- gated merge h = e + alpha sigmoid(W_g [e; s] + b) s, first norm input
   if (!P.alpha0)
@@ -977,7 +1015,7 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
                             MAP_GATE, cnt(L, PH_GATHER, r), rows_of(r), cnt(L, PH_GATE, r),
                             EpiGateNorm<bf16>{{}, P.e32, P.s32, P.gate_b, P.alpha, P.h, d,
                                               P.ln1[0], P.u, P.nsq, np},
-                            s_rs);
+                            s_rs, fs_trace_id(L, PH_GATE, r, false), tslot);
 
   for (int l = 0; l < L; l++) {
     bf16 *ring_l = P.ring + (size_t)l * P.ring_layer;
@@ -988,11 +1026,11 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
       const int *dep = l == 0 ? (P.alpha0 ? cnt(L, PH_GATHER, r) : cnt(L, PH_GATE, r))
                               : cnt(l - 1, PH_FFN2, r);
       const int tgt = l == 0 ? (P.alpha0 ? rows_of(r) : T_d * FS_S) : T_d * FS_S;
-      fs_gemm_phase<BNQ, NSQ>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), 3 * d, d, MAP_A_U,
+      fs_gemm_phase<BNQ, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), 3 * d, d, MAP_A_U,
                               fs_map_index(l, MAPL_QKV), dep, tgt, cnt(l, PH_QKV, r),
                               EpiQkvRope<bf16>{rsi, P.q, ring_l, P.ready, P.pos, P.rope, H, DH,
                                                P.W, d},
-                              s_rs);
+                              s_rs, fs_trace_id(l, PH_QKV, r, false), tslot);
     }
     // sliding-window attention over the ring
     for (int r = 0; r < RT; r++) {
@@ -1004,19 +1042,19 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
       const FsAttnGeom g{m0, rv, H, P.W, P.CH, 1, rv * H, rv * H, ring_l,
                          (long)H * 2 * P.W * DH, 2L * P.W * DH, (long)P.W * DH, s_ready, s_pos};
       fs_attn_phase<DH>(P, sh, g, gcta, ncta, cnt(l, PH_QKV, r), T_q * FS_S, cnt(l, PH_SWA, r),
-                        &s_skip);
+                        &s_skip, fs_trace_id(l, PH_SWA, r, true), tslot);
     }
     // W_o, residual, cross-attention norm input
     for (int r = 0; r < RT; r++)
       fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, d, MAP_A_A,
                             fs_map_index(l, MAPL_O), cnt(l, PH_SWA, r), rows_of(r) * H,
                             cnt(l, PH_WO, r),
-                            EpiResidNorm<bf16>{{}, P.h, d, P.ln2[l], P.u, P.nsq, np}, s_rs);
+                            EpiResidNorm<bf16>{{}, P.h, d, P.ln2[l], P.u, P.nsq, np}, s_rs, fs_trace_id(l, PH_WO, r, false), tslot);
     // cross-attention query
     for (int r = 0; r < RT; r++)
       fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, d, MAP_A_U,
                             fs_map_index(l, MAPL_QX), cnt(l, PH_WO, r), T_d * FS_S,
-                            cnt(l, PH_WQX, r), EpiRsF32{rsi, P.q, d}, s_rs);
+                            cnt(l, PH_WQX, r), EpiRsF32{rsi, P.q, d}, s_rs, fs_trace_id(l, PH_WQX, r, false), tslot);
     // cross-attention over M<=t
     for (int r = 0; r < RT; r++) {
       const int m0 = r * FS_RT, rv = rows_of(r);
@@ -1028,30 +1066,30 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
                          (long)H * 2 * P.max_len * DH, 2L * P.max_len * DH,
                          (long)P.max_len * DH, s_ready, s_pos};
       fs_attn_phase<DH>(P, sh, g, gcta, ncta, cnt(l, PH_WQX, r), T_d * FS_S,
-                        cnt(l, PH_XATTN, r), &s_skip);
+                        cnt(l, PH_XATTN, r), &s_skip, fs_trace_id(l, PH_XATTN, r, true), tslot);
     }
     // W_ox, residual, FFN norm input
     for (int r = 0; r < RT; r++)
       fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, d, MAP_A_A,
                             fs_map_index(l, MAPL_OX), cnt(l, PH_XATTN, r), rows_of(r) * H,
                             cnt(l, PH_WOX, r),
-                            EpiResidNorm<bf16>{{}, P.h, d, P.ln3[l], P.u, P.nsq, np}, s_rs);
+                            EpiResidNorm<bf16>{{}, P.h, d, P.ln3[l], P.u, P.nsq, np}, s_rs, fs_trace_id(l, PH_WOX, r, false), tslot);
     // FFN up
     for (int r = 0; r < RT; r++) {
       if (!P.swiglu)
         fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), F, d, MAP_A_U,
                               fs_map_index(l, MAPL_W1), cnt(l, PH_WOX, r), T_d * FS_S,
-                              cnt(l, PH_FFN1, r), EpiRsGelu<bf16>{rsi, P.f, F}, s_rs);
+                              cnt(l, PH_FFN1, r), EpiRsGelu<bf16>{rsi, P.f, F}, s_rs, fs_trace_id(l, PH_FFN1, r, false), tslot);
       else
         fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), F, d, MAP_A_U,
                               fs_map_index(l, MAPL_W1), cnt(l, PH_WOX, r), T_d * FS_S,
-                              cnt(l, PH_FFN1, r), EpiRsF32{rsi, P.fa, F}, s_rs);
+                              cnt(l, PH_FFN1, r), EpiRsF32{rsi, P.fa, F}, s_rs, fs_trace_id(l, PH_FFN1, r, false), tslot);
     }
     if (P.swiglu)
       for (int r = 0; r < RT; r++)
         fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), F, d, MAP_A_U,
                               fs_map_index(l, MAPL_WB), cnt(l, PH_FFN1, r), T_f * FS_S,
-                              cnt(l, PH_FFN1B, r), EpiRsSwiglu<bf16>{rsi, P.fa, P.f, F}, s_rs);
+                              cnt(l, PH_FFN1B, r), EpiRsSwiglu<bf16>{rsi, P.fa, P.f, F}, s_rs, fs_trace_id(l, PH_FFN1B, r, false), tslot);
     // FFN down, residual, next block's input
     for (int r = 0; r < RT; r++)
       fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, F, MAP_A_F,
@@ -1060,20 +1098,24 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
                             cnt(l, PH_FFN2, r),
                             EpiResidNorm<bf16>{{}, P.h, d, last ? nullptr : P.ln1[l + 1], P.u,
                                                P.nsq, np},
-                            s_rs);
+                            s_rs, fs_trace_id(l, PH_FFN2, r, false), tslot);
   }
 
   // ---- s_t = RMSNorm_f(h), t_dec += 1 (one warp per row, after the row
   // tile's last FFN)
   for (int r = 0; r < RT; r++) {
     const int m0 = r * FS_RT, hi = m0 + rows_of(r);
+    const uint64_t t0 = P.trace ? globaltimer_ns() : 0;
     if (threadIdx.x == 0) s_skip = fs_wait_count(P, cnt(L - 1, PH_FFN2, r), T_d * FS_S) ? 0 : 1;
+    const uint64_t t1 = P.trace ? globaltimer_ns() : 0;
     __syncthreads();
     const bool ok = s_skip == 0;
     __syncthreads();
     if (ok)
       for (int i = gcta * 8 + warp; i < hi; i += ncta * 8)
         if (i >= m0) fs_final_row(P, i, lane);
+    if (threadIdx.x == 0)
+      fs_trace(P, tslot, fs_trace_id(L, 0x21, r, false), t0, t1, globaltimer_ns());
   }
 
   // ---- teardown: every cluster peer is past its last shared-memory read

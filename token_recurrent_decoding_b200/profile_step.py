@@ -59,8 +59,15 @@ def run_steps(args):
     torch.cuda.synchronize()
     ids = list(range(B))
     st = torch.cuda.Stream() if args.graph else None
+    trace = None
+    if args.trace:
+        ctas = m.step_kernel_ctas()
+        trace = torch.zeros((ctas, args.trace_cap, 4), dtype=torch.int64, device="cuda")
+        m.set_step_trace(trace)
     times = []
     for k in range(args.steps):
+        if trace is not None:
+            trace.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if st is not None:
             a.record(st)
@@ -73,12 +80,55 @@ def run_steps(args):
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
     assert m.poll_device_error() == 0
+    if trace is not None:
+        rec = trace.cpu().numpy()
+        np.save(args.trace, rec)
+        print(json.dumps(trace_summary(rec, cfg.n_dec)))
     ts = [np.full(B, args.t + k) for k in range(args.steps)]
     byts = [roofline.decoder_step_bytes(cfg, x) for x in ts]
     print(json.dumps({"workload": args.workload, "batch": B, "t": args.t, "graph": args.graph,
                       "kernel": "fused" if m.get_step_kernel() == 1 else "chain",
                       "step_ms": times, "step_GB": [x / 1e9 for x in byts],
                       "GB_s": [x / (ms / 1e3) / 1e9 for x, ms in zip(byts, times)]}))
+
+
+PHASES = {0: "qkv", 0x81: "swa", 2: "wo", 3: "wqx", 0x84: "xattn", 5: "wox", 6: "ffn1",
+          7: "ffn1b", 8: "ffn2"}
+
+
+def trace_summary(rec, n_dec):
+    """Where a persistent step's time goes, from its trace records
+    [ctas][cap][4] = (item id, start, dependency met, end): per item kind,
+    the mean over layers and row tiles of the span from the first CTA's
+    start to the last CTA's end, of the part after the last dependency was
+    met, and of the CTA-busy time per item."""
+    r = rec.reshape(-1, 4)
+    r = r[r[:, 0] != 0]
+    if not len(r):
+        return {"trace": "empty"}
+    t0 = r[:, 1].min()
+    groups = {}
+    for idv, a, dp, e in r:
+        groups.setdefault(int(idv), []).append((a - t0, dp - t0, e - t0))
+    kinds = {}
+    for idv, items in groups.items():
+        layer, ph, row = (idv >> 16) - 1, (idv >> 8) & 0xFF, idv & 0xFF
+        name = PHASES.get(ph, "pre" if layer == n_dec else str(ph))
+        if layer == n_dec:
+            name = {1: "gate", 0x20: "gather", 0x21: "final"}.get(ph, name)
+        x = np.asarray(items, dtype=np.float64)
+        k = kinds.setdefault(name, {"span": [], "after_dep": [], "busy": [], "items": 0})
+        k["span"].append(x[:, 2].max() - x[:, 0].min())
+        k["after_dep"].append(x[:, 2].max() - x[:, 1].max())
+        k["busy"].append(float(np.mean(x[:, 2] - x[:, 1])))
+        k["items"] += len(items)
+    out = {name: {"groups": len(v["span"]), "items": v["items"],
+                  "span_us": round(float(np.mean(v["span"])) / 1e3, 2),
+                  "after_last_dep_us": round(float(np.mean(v["after_dep"])) / 1e3, 2),
+                  "busy_per_item_us": round(float(np.mean(v["busy"])) / 1e3, 2)}
+           for name, v in kinds.items()}
+    out["kernel_us"] = round(float(r[:, 3].max() - t0) / 1e3, 1)
+    return out
 
 
 def run_attend(args):
@@ -117,6 +167,10 @@ def main():
                     help="sequence length of the arena (default: the workload's); small "
                          "values keep a profiler's device memory small")
     ap.add_argument("--graph", action="store_true")
+    ap.add_argument("--trace", default="",
+                    help="record the persistent step's work items into this .npy file and "
+                         "print where the time goes (last step)")
+    ap.add_argument("--trace-cap", type=int, default=1024)
     ap.add_argument("--kernel", choices=["fused", "chain"], default=None,
                     help="decoder step kernel (default: the model's default)")
     ap.add_argument("--attend", action="store_true")

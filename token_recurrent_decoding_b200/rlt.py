@@ -93,6 +93,8 @@ def _declare(lib):
     lib.rlt_set_fault.argtypes = [P, I, C.c_int64]
     lib.rlt_set_step_kernel.argtypes = [P, I]
     lib.rlt_get_step_kernel.argtypes = [P]
+    lib.rlt_step_kernel_ctas.argtypes = [P]
+    lib.rlt_set_step_trace.argtypes = [P, P, C.c_size_t]
     lib.rlt_attend_workspace_bytes.argtypes = [I, I, I, I]
     lib.rlt_attend_workspace_bytes.restype = C.c_size_t
     lib.rlt_attend.argtypes = [P, P, P, I, I, I, I, I, P, P, C.c_size_t, P]
@@ -375,6 +377,16 @@ class Model:
 
     def get_step_kernel(self) -> int:
         return int(_lib().rlt_get_step_kernel(self._h))
+
+    def step_kernel_ctas(self) -> int:
+        return int(_lib().rlt_step_kernel_ctas(self._h))
+
+    def set_step_trace(self, buf):
+        """buf: int64 device tensor [ctas][cap][4] (None: off); see rlt_set_step_trace."""
+        self._trace_keep = buf
+        ptr = C.c_void_p(buf.data_ptr()) if buf is not None else None
+        nbytes = buf.numel() * buf.element_size() if buf is not None else 0
+        _check(_lib().rlt_set_step_trace(self._h, ptr, nbytes), "rlt_set_step_trace")
 
     def set_fault(self, fault: int, wait_limit_ns: int = 0):
         """Plant a fault (FAULT_*) in later decoder-attention launches and
