@@ -170,6 +170,11 @@ __device__ __forceinline__ bool fs_aborted(const FsParams &P) {
   return *reinterpret_cast<volatile const int *>(P.abort) != 0;
 }
 
+// Polling loops read the abort word (a global load) only every 16 us of
+// their own waiting, so a busy loop reacts to its barrier or counter at
+// once.
+constexpr uint64_t FS_ABORT_POLL_NS = 16000;
+
 __device__ __forceinline__ uint64_t fs_wait_limit(const FsParams &P) {
   return P.ctl && P.ctl->wait_limit_ns ? P.ctl->wait_limit_ns : WAIT_LIMIT_NS;
 }
@@ -186,11 +191,15 @@ __device__ __forceinline__ void fs_fail(const FsParams &P) {
 __device__ bool fs_wait_count(const FsParams &P, const int *c, int target) {
   if (ld_acquire_gpu(c) >= target) return true;
   const uint64_t limit = fs_wait_limit(P), t0 = globaltimer_ns();
-  for (int spin = 0;; spin++) {
+  uint64_t next_check = t0 + FS_ABORT_POLL_NS;
+  for (;;) {
     if (ld_acquire_gpu(c) >= target) return true;
-    if (fs_aborted(P)) return false;
-    if (spin > 64) __nanosleep(64);  // long waits poll L2 less often
-    if (globaltimer_ns() - t0 > limit) {
+    const uint64_t now = globaltimer_ns();
+    if (now > next_check) {
+      if (fs_aborted(P)) return false;
+      next_check = now + FS_ABORT_POLL_NS;
+    }
+    if (now - t0 > limit) {
       fs_fail(P);
       return false;
     }
@@ -201,10 +210,15 @@ __device__ bool fs_wait_count(const FsParams &P, const int *c, int target) {
 __device__ bool fs_mbar_wait(const FsParams &P, uint64_t *bar, unsigned parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t limit = fs_wait_limit(P), t0 = globaltimer_ns();
+  uint64_t next_check = t0 + FS_ABORT_POLL_NS;
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (fs_aborted(P)) return false;
-    if (globaltimer_ns() - t0 > limit) {
+    const uint64_t now = globaltimer_ns();
+    if (now > next_check) {
+      if (fs_aborted(P)) return false;
+      next_check = now + FS_ABORT_POLL_NS;
+    }
+    if (now - t0 > limit) {
       fs_fail(P);
       return false;
     }
@@ -216,17 +230,22 @@ __device__ bool fs_mbar_wait(const FsParams &P, uint64_t *bar, unsigned parity) 
 // is taken by lane 0 and shared, so the warp never splits.
 __device__ bool fs_mbar_wait_warp(const FsParams &P, uint64_t *bar, unsigned parity) {
   const uint64_t limit = fs_wait_limit(P);
-  uint64_t t0 = 0;
+  uint64_t t0 = 0, next_check = 0;
   for (bool first = true;; first = false) {
     const bool got = mbar_try_wait(bar, parity);
     if (__all_sync(FULL_MASK, got)) return true;
     int stop = 0;
     if ((threadIdx.x & 31) == 0) {
       const uint64_t now = globaltimer_ns();
-      if (first) t0 = now;
-      if (fs_aborted(P)) {
-        stop = 1;
-      } else if (now - t0 > limit) {
+      if (first) {
+        t0 = now;
+        next_check = now + FS_ABORT_POLL_NS;
+      }
+      if (now > next_check) {
+        if (fs_aborted(P)) stop = 1;
+        next_check = now + FS_ABORT_POLL_NS;
+      }
+      if (!stop && now - t0 > limit) {
         fs_fail(P);
         stop = 1;
       }
@@ -386,7 +405,7 @@ __device__ void fs_gemm_epilogue(const FsParams &P, float *Pt, int m0, int n0, i
 // CTA takes part in both cluster barriers whatever happened, so a failed or
 // skipped task never strands its peers.
 template <int BN, int NS, class Epi>
-__device__ void fs_gemm_task(const FsParams &P, const FsShared &sh, FsRun &run,
+__device__ __noinline__ void fs_gemm_task(const FsParams &P, const FsShared &sh, FsRun &run,
                              const CUtensorMap *mA, const CUtensorMap *mB, int m0, int rv,
                              int tile, int K, const int *dep, int dep_target, int *signal,
                              const Epi &epi, float *s_rs, int trace_id, int &tslot) {
@@ -468,10 +487,17 @@ __device__ void fs_gemm_task(const FsParams &P, const FsShared &sh, FsRun &run,
         const unsigned par = (unsigned)((g / NS) & 1);
         bool got = mbar_try_wait(&sh.gfull[s], par);
         const uint64_t t0 = globaltimer_ns();
+        uint64_t next_check = t0 + FS_ABORT_POLL_NS;
         while (!got) {
           const int nf = *vnfill;
           if (nf >= 0 && kb >= nf) break;  // the producer stopped before this stage
-          if (globaltimer_ns() - t0 > limit || fs_aborted(P)) {
+          const uint64_t now = globaltimer_ns();
+          bool stop = now - t0 > limit;
+          if (!stop && now > next_check) {
+            stop = fs_aborted(P);
+            next_check = now + FS_ABORT_POLL_NS;
+          }
+          if (stop) {
             fs_fail(P);
             *vfail = 1;
             break;
@@ -620,7 +646,7 @@ template <int KT> struct FsWalk {
 };
 
 template <int DH>
-__device__ void fs_attn_phase(const FsParams &P, const FsShared &sh, const FsAttnGeom &g,
+__device__ __noinline__ void fs_attn_phase(const FsParams &P, const FsShared &sh, const FsAttnGeom &g,
                               int gcta, int ncta, const int *dep, int dep_target, int *signal,
                               int *s_skip, int trace_id, int &tslot) {
   const uint64_t t_begin = P.trace ? globaltimer_ns() : 0;
@@ -730,11 +756,14 @@ __device__ void fs_attn_phase(const FsParams &P, const FsShared &sh, const FsAtt
       }
       if (progress) {
         t0 = globaltimer_ns();
-      } else if (fs_aborted(P)) {
-        ok = false;
-      } else if (globaltimer_ns() - t0 > limit) {
-        fs_fail(P);
-        ok = false;
+      } else {
+        const uint64_t now = globaltimer_ns();
+        if (now - t0 > limit) {
+          fs_fail(P);
+          ok = false;
+        } else if (now - t0 > FS_ABORT_POLL_NS && fs_aborted(P)) {
+          ok = false;
+        }
       }
     }
     // let every copy this CTA issued land before shared memory is reused

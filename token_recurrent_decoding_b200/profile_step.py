@@ -88,6 +88,7 @@ def run_steps(args):
     byts = [roofline.decoder_step_bytes(cfg, x) for x in ts]
     print(json.dumps({"workload": args.workload, "batch": B, "t": args.t, "graph": args.graph,
                       "kernel": "fused" if m.get_step_kernel() == 1 else "chain",
+                      "step_kernel_ctas": m.step_kernel_ctas(),
                       "step_ms": times, "step_GB": [x / 1e9 for x in byts],
                       "GB_s": [x / (ms / 1e3) / 1e9 for x, ms in zip(byts, times)]}))
 
