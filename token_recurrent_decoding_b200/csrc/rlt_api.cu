@@ -791,7 +791,7 @@ template <int DH> cudaError_t fused_setup_impl(rlt_model *M) {
   auto kern = k_step_fused<DH>;
   constexpr int smem = FsSmem<DH>::BYTES;
   RLT_TRY(ensure_smem_limit(kern, smem));
-  // two CTAs per SM need the whole unified L1 as shared memory
+  // the CTA's stages need (nearly) the whole unified L1 as shared memory
   RLT_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(FS_S * M->num_sms);

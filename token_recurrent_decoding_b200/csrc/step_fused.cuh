@@ -14,7 +14,7 @@
 // boundaries, and the residual stream and activations move through L2.
 //
 // Grid: thread-block clusters of FS_S CTAs, as many as can be resident at
-// once (two CTAs per SM), 8 warps per CTA. Rows of the ready list are cut
+// once (one CTA per SM), 16 warps per CTA. Rows of the ready list are cut
 // into row tiles of 128 (the tcgen05 M). Work items:
 //  * GEMM tile task (one cluster): a 128 x BN output tile of one projection
 //    for one row tile, K split across the FS_S CTAs of the cluster (TMA ring,
@@ -24,7 +24,8 @@
 //    the ring or the cross-attention over M<=t, fed by a producer warp with
 //    bulk copies (the design of attn.cuh);
 //  * per-row gather (ready rows, [e_t ; s_{t-1}]) and final norm.
-// Every CTA walks the same global task order, (layer, phase, row tile), and
+// Every CTA walks the same global task order (layer and phase, row tiles
+// staggered by FS_STAGGER phases), and
 // does the items the static assignment gives it; an item waits (one thread,
 // acquire load, bounded in device time) until the counter of the phase it
 // depends on reaches its target, and signals its own phase's counter
@@ -52,13 +53,15 @@
 
 namespace rlt {
 
-constexpr int FS_THREADS = 256;  // 8 warps
-constexpr int FS_S = 4;          // cluster size = split-K factor of every GEMM tile
+constexpr int FS_THREADS = 512;  // 16 warps, one CTA per SM
+constexpr int FS_WARPS = FS_THREADS / 32;
+constexpr int FS_S = 2;          // cluster size = split-K factor of every GEMM tile
 constexpr int FS_RT = 128;       // rows per row tile (tcgen05 M)
-constexpr int FS_NC = 6;         // attention consumer warps 0..5; warp 7 produces
+constexpr int FS_NC = 12;        // attention consumer warps 0..11; warp 15 produces
 constexpr int FS_SW = 2;         // attention stages per consumer warp
-constexpr int FS_PROD_WARP = 7;
+constexpr int FS_PROD_WARP = 15;
 constexpr int FS_MAX_LAYERS = 64;
+constexpr int FS_STAGGER = 1;    // items row tile r runs behind row tile r - 1
 
 // Phases of one decoder block, in dependency order. The pre-block phases
 // (gather, gate) use the counters of layer slot L_D.
@@ -272,7 +275,7 @@ struct FsCtlSmem {
   int nfill;                   // ring stages this GEMM task fills (-1: not known yet)
   int issued[FS_NC];           // attention stages filled per consumer warp (producer)
   int consumed[FS_NC];         // attention stages consumed per consumer warp
-  int outputs[8];              // attention outputs written per warp in this phase
+  int outputs[FS_WARPS];       // attention outputs written per warp in this phase
   int rows_done[FS_MAX_RT];    // gathered rows per row tile
   unsigned long long tdep;     // when the attention producer's dependency was met (trace)
 };
@@ -521,7 +524,7 @@ __device__ __noinline__ void fs_gemm_task(const FsParams &P, const FsShared &sh,
       // ---- row scales of this CTA's rows, from the partial sums of squares
       // the producer of the input wrote (column-tile order)
       if (warp == 2 && lane == 0 && dep && !fs_wait_count(P, dep, dep_target)) *vfail = 1;
-      asm volatile("bar.sync 1, 192;\n" ::: "memory");
+      asm volatile("bar.sync 1, %0;\n" ::"n"(FS_THREADS - 64) : "memory");
       if (!*vfail)
         for (int i = threadIdx.x - 64; i < r_hi - r_lo; i += FS_THREADS - 64) {
           const float *p = epi.rsi.nsq + (size_t)(m0 + r_lo + i) * epi.rsi.np;
@@ -557,8 +560,9 @@ __device__ __noinline__ void fs_gemm_task(const FsParams &P, const FsShared &sh,
     }
     __syncthreads();
   }
+  // warps 0-7 move the accumulator: TMEM lanes of warp w mod 4, column half w / 4
   const int lg = warp & 3, chh = warp >> 2;
-  if (ok && lg * 32 < rv) {
+  if (ok && warp < 8 && lg * 32 < rv) {
     const int row = lg * 32 + lane;
     const uint32_t lane_base = ctl->tmem + ((uint32_t)(lg * 32) << 16);
 #pragma unroll
@@ -657,7 +661,7 @@ __device__ __noinline__ void fs_attn_phase(const FsParams &P, const FsShared &sh
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int stride = ncta * FS_NC;
   if (threadIdx.x == 0) *s_skip = fs_aborted(P) ? 1 : 0;
-  if (threadIdx.x < 8) ctl->outputs[threadIdx.x] = 0;
+  if (threadIdx.x < FS_WARPS) ctl->outputs[threadIdx.x] = 0;
   __syncthreads();
   const bool skip = *s_skip != 0;
   const uint64_t limit = fs_wait_limit(P);
@@ -981,7 +985,7 @@ __device__ void fs_final_row(const FsParams &P, int i, int lane) {
 
 // ------------------------------------------------------------ the kernel
 template <int DH>
-__global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_constant__ FsParams P) {
+__global__ void __launch_bounds__(FS_THREADS, 1) k_step_fused(const __grid_constant__ FsParams P) {
   using SM = FsSmem<DH>;
   constexpr int BNQ = SM::BNQ, NS = SM::NS;
   extern __shared__ uint8_t fs_raw[];
@@ -1027,7 +1031,7 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
   const int T_q = 3 * d / BNQ, T_d = d / 32, T_f = F / 64;
 
   // ---- gather: one warp per ready row
-  for (int i = gcta * 8 + warp; i < n; i += ncta * 8) {
+  for (int i = gcta * FS_WARPS + warp; i < n; i += ncta * FS_WARPS) {
     fs_gather_row(P, i, lane);
     if (lane == 0) atomicAdd(&ctl->rows_done[i / FS_RT], 1);
   }
@@ -1037,98 +1041,119 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
   if (threadIdx.x == 0)
     fs_trace(P, tslot, fs_trace_id(L, 0x20, 0, false), t_start, t_start, globaltimer_ns());
 
-  // ---- gated merge h = e + alpha sigmoid(W_g [e; s] + b) s, first norm input
-  if (!P.alpha0)
-    for (int r = 0; r < RT; r++)
-      fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, 2 * d, MAP_A_XIN,
-                            MAP_GATE, cnt(L, PH_GATHER, r), rows_of(r), cnt(L, PH_GATE, r),
-                            EpiGateNorm<bf16>{{}, P.e32, P.s32, P.gate_b, P.alpha, P.h, d,
-                                              P.ln1[0], P.u, P.nsq, np},
-                            s_rs, fs_trace_id(L, PH_GATE, r, false), tslot);
-
-  for (int l = 0; l < L; l++) {
+  // ---- the work items of every row tile, one decoder sublayer phase at a
+  // time: item j = 0 is the gated merge, item j >= 1 phase (j-1) mod FS_NPH of
+  // layer (j-1) / FS_NPH. Row tile r runs FS_STAGGER items behind row tile
+  // r-1 (while one tile streams its attention, the next one's GEMMs run);
+  // every CTA walks the same order, and each item depends only on items
+  // earlier in it.
+  const int n_items = 1 + L * FS_NPH;
+  auto run_item = [&](int j, int r) {
+    const int m0 = r * FS_RT, rv = rows_of(r);
+    if (j == 0) {
+      // gated merge h = e + alpha sigmoid(W_g [e; s] + b) s, first norm input
+      if (!P.alpha0)
+        fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, m0, rv, d, 2 * d, MAP_A_XIN, MAP_GATE,
+                              cnt(L, PH_GATHER, r), rv, cnt(L, PH_GATE, r),
+                              EpiGateNorm<bf16>{{}, P.e32, P.s32, P.gate_b, P.alpha, P.h, d,
+                                                P.ln1[0], P.u, P.nsq, np},
+                              s_rs, fs_trace_id(L, PH_GATE, r, false), tslot);
+      return;
+    }
+    const int l = (j - 1) / FS_NPH, ph = (j - 1) % FS_NPH;
     bf16 *ring_l = P.ring + (size_t)l * P.ring_layer;
-    const bf16 *mem_g = P.mem + (size_t)(P.G == 1 ? 0 : l) * P.mem_group;
-    const bool last = l + 1 == L;
-    // q/k/v with rotary, ring write of k and v
-    for (int r = 0; r < RT; r++) {
-      const int *dep = l == 0 ? (P.alpha0 ? cnt(L, PH_GATHER, r) : cnt(L, PH_GATE, r))
-                              : cnt(l - 1, PH_FFN2, r);
-      const int tgt = l == 0 ? (P.alpha0 ? rows_of(r) : T_d * FS_S) : T_d * FS_S;
-      fs_gemm_phase<BNQ, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), 3 * d, d, MAP_A_U,
-                              fs_map_index(l, MAPL_QKV), dep, tgt, cnt(l, PH_QKV, r),
-                              EpiQkvRope<bf16>{rsi, P.q, ring_l, P.ready, P.pos, P.rope, H, DH,
-                                               P.W, d},
-                              s_rs, fs_trace_id(l, PH_QKV, r, false), tslot);
-    }
-    // sliding-window attention over the ring
-    for (int r = 0; r < RT; r++) {
-      const int m0 = r * FS_RT, rv = rows_of(r);
-      for (int i = threadIdx.x; i < rv; i += FS_THREADS) {
-        s_ready[i] = P.ready[m0 + i];
-        s_pos[i] = P.t_dec[s_ready[i]];
+    switch (ph) {
+      case PH_QKV: {  // q/k/v with rotary, ring write of k and v
+        const int *dep = l == 0 ? (P.alpha0 ? cnt(L, PH_GATHER, r) : cnt(L, PH_GATE, r))
+                                : cnt(l - 1, PH_FFN2, r);
+        const int tgt = (l == 0 && P.alpha0) ? rv : T_d * FS_S;
+        fs_gemm_phase<BNQ, NS>(P, sh, run, cl, C, rot, m0, rv, 3 * d, d, MAP_A_U,
+                               fs_map_index(l, MAPL_QKV), dep, tgt, cnt(l, PH_QKV, r),
+                               EpiQkvRope<bf16>{rsi, P.q, ring_l, P.ready, P.pos, P.rope, H, DH,
+                                                P.W, d},
+                               s_rs, fs_trace_id(l, PH_QKV, r, false), tslot);
+        break;
       }
-      const FsAttnGeom g{m0, rv, H, P.W, P.CH, 1, rv * H, rv * H, ring_l,
-                         (long)H * 2 * P.W * DH, 2L * P.W * DH, (long)P.W * DH, s_ready, s_pos};
-      fs_attn_phase<DH>(P, sh, g, gcta, ncta, cnt(l, PH_QKV, r), T_q * FS_S, cnt(l, PH_SWA, r),
-                        &s_skip, fs_trace_id(l, PH_SWA, r, true), tslot);
-    }
-    // W_o, residual, cross-attention norm input
-    for (int r = 0; r < RT; r++)
-      fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, d, MAP_A_A,
-                            fs_map_index(l, MAPL_O), cnt(l, PH_SWA, r), rows_of(r) * H,
-                            cnt(l, PH_WO, r),
-                            EpiResidNorm<bf16>{{}, P.h, d, P.ln2[l], P.u, P.nsq, np}, s_rs, fs_trace_id(l, PH_WO, r, false), tslot);
-    // cross-attention query
-    for (int r = 0; r < RT; r++)
-      fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, d, MAP_A_U,
-                            fs_map_index(l, MAPL_QX), cnt(l, PH_WO, r), T_d * FS_S,
-                            cnt(l, PH_WQX, r), EpiRsF32{rsi, P.q, d}, s_rs, fs_trace_id(l, PH_WQX, r, false), tslot);
-    // cross-attention over M<=t
-    for (int r = 0; r < RT; r++) {
-      const int m0 = r * FS_RT, rv = rows_of(r);
-      for (int i = threadIdx.x; i < rv; i += FS_THREADS) {
-        s_ready[i] = P.ready[m0 + i];
-        s_pos[i] = P.t_dec[s_ready[i]];
+      case PH_SWA: {  // sliding-window attention over the ring
+        for (int i = threadIdx.x; i < rv; i += FS_THREADS) {
+          s_ready[i] = P.ready[m0 + i];
+          s_pos[i] = P.t_dec[s_ready[i]];
+        }
+        const FsAttnGeom g{m0, rv, H, P.W, P.CH, 1, rv * H, rv * H, ring_l,
+                           (long)H * 2 * P.W * DH, 2L * P.W * DH, (long)P.W * DH, s_ready,
+                           s_pos};
+        fs_attn_phase<DH>(P, sh, g, gcta, ncta, cnt(l, PH_QKV, r), T_q * FS_S,
+                          cnt(l, PH_SWA, r), &s_skip, fs_trace_id(l, PH_SWA, r, true), tslot);
+        break;
       }
-      const FsAttnGeom g{m0, rv, H, 0, P.CH, P.xch, rv * H, rv * H * P.xch, mem_g,
-                         (long)H * 2 * P.max_len * DH, 2L * P.max_len * DH,
-                         (long)P.max_len * DH, s_ready, s_pos};
-      fs_attn_phase<DH>(P, sh, g, gcta, ncta, cnt(l, PH_WQX, r), T_d * FS_S,
-                        cnt(l, PH_XATTN, r), &s_skip, fs_trace_id(l, PH_XATTN, r, true), tslot);
+      case PH_WO:  // W_o, residual, cross-attention norm input
+        fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, m0, rv, d, d, MAP_A_A,
+                              fs_map_index(l, MAPL_O), cnt(l, PH_SWA, r), rv * H, cnt(l, PH_WO, r),
+                              EpiResidNorm<bf16>{{}, P.h, d, P.ln2[l], P.u, P.nsq, np}, s_rs,
+                              fs_trace_id(l, PH_WO, r, false), tslot);
+        break;
+      case PH_WQX:  // cross-attention query
+        fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, m0, rv, d, d, MAP_A_U,
+                              fs_map_index(l, MAPL_QX), cnt(l, PH_WO, r), T_d * FS_S,
+                              cnt(l, PH_WQX, r), EpiRsF32{rsi, P.q, d}, s_rs,
+                              fs_trace_id(l, PH_WQX, r, false), tslot);
+        break;
+      case PH_XATTN: {  // cross-attention over M<=t
+        const bf16 *mem_g = P.mem + (size_t)(P.G == 1 ? 0 : l) * P.mem_group;
+        for (int i = threadIdx.x; i < rv; i += FS_THREADS) {
+          s_ready[i] = P.ready[m0 + i];
+          s_pos[i] = P.t_dec[s_ready[i]];
+        }
+        const FsAttnGeom g{m0, rv, H, 0, P.CH, P.xch, rv * H, rv * H * P.xch, mem_g,
+                           (long)H * 2 * P.max_len * DH, 2L * P.max_len * DH,
+                           (long)P.max_len * DH, s_ready, s_pos};
+        fs_attn_phase<DH>(P, sh, g, gcta, ncta, cnt(l, PH_WQX, r), T_d * FS_S,
+                          cnt(l, PH_XATTN, r), &s_skip, fs_trace_id(l, PH_XATTN, r, true),
+                          tslot);
+        break;
+      }
+      case PH_WOX:  // W_ox, residual, FFN norm input
+        fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, m0, rv, d, d, MAP_A_A,
+                              fs_map_index(l, MAPL_OX), cnt(l, PH_XATTN, r), rv * H,
+                              cnt(l, PH_WOX, r),
+                              EpiResidNorm<bf16>{{}, P.h, d, P.ln3[l], P.u, P.nsq, np}, s_rs,
+                              fs_trace_id(l, PH_WOX, r, false), tslot);
+        break;
+      case PH_FFN1:  // FFN up: GELU, or the SwiGLU gate half
+        if (!P.swiglu)
+          fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, m0, rv, F, d, MAP_A_U,
+                                fs_map_index(l, MAPL_W1), cnt(l, PH_WOX, r), T_d * FS_S,
+                                cnt(l, PH_FFN1, r), EpiRsGelu<bf16>{rsi, P.f, F}, s_rs,
+                                fs_trace_id(l, PH_FFN1, r, false), tslot);
+        else
+          fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, m0, rv, F, d, MAP_A_U,
+                                fs_map_index(l, MAPL_W1), cnt(l, PH_WOX, r), T_d * FS_S,
+                                cnt(l, PH_FFN1, r), EpiRsF32{rsi, P.fa, F}, s_rs,
+                                fs_trace_id(l, PH_FFN1, r, false), tslot);
+        break;
+      case PH_FFN1B:  // SwiGLU value half
+        if (P.swiglu)
+          fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, m0, rv, F, d, MAP_A_U,
+                                fs_map_index(l, MAPL_WB), cnt(l, PH_FFN1, r), T_f * FS_S,
+                                cnt(l, PH_FFN1B, r), EpiRsSwiglu<bf16>{rsi, P.fa, P.f, F}, s_rs,
+                                fs_trace_id(l, PH_FFN1B, r, false), tslot);
+        break;
+      default:  // PH_FFN2: FFN down, residual, next block's input
+        fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, m0, rv, d, F, MAP_A_F,
+                              fs_map_index(l, MAPL_W2),
+                              P.swiglu ? cnt(l, PH_FFN1B, r) : cnt(l, PH_FFN1, r), T_f * FS_S,
+                              cnt(l, PH_FFN2, r),
+                              EpiResidNorm<bf16>{{}, P.h, d, l + 1 == L ? nullptr : P.ln1[l + 1],
+                                                 P.u, P.nsq, np},
+                              s_rs, fs_trace_id(l, PH_FFN2, r, false), tslot);
+        break;
     }
-    // W_ox, residual, FFN norm input
-    for (int r = 0; r < RT; r++)
-      fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, d, MAP_A_A,
-                            fs_map_index(l, MAPL_OX), cnt(l, PH_XATTN, r), rows_of(r) * H,
-                            cnt(l, PH_WOX, r),
-                            EpiResidNorm<bf16>{{}, P.h, d, P.ln3[l], P.u, P.nsq, np}, s_rs, fs_trace_id(l, PH_WOX, r, false), tslot);
-    // FFN up
+  };
+  for (int k = 0; k < n_items + (RT - 1) * FS_STAGGER; k++)
     for (int r = 0; r < RT; r++) {
-      if (!P.swiglu)
-        fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), F, d, MAP_A_U,
-                              fs_map_index(l, MAPL_W1), cnt(l, PH_WOX, r), T_d * FS_S,
-                              cnt(l, PH_FFN1, r), EpiRsGelu<bf16>{rsi, P.f, F}, s_rs, fs_trace_id(l, PH_FFN1, r, false), tslot);
-      else
-        fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), F, d, MAP_A_U,
-                              fs_map_index(l, MAPL_W1), cnt(l, PH_WOX, r), T_d * FS_S,
-                              cnt(l, PH_FFN1, r), EpiRsF32{rsi, P.fa, F}, s_rs, fs_trace_id(l, PH_FFN1, r, false), tslot);
+      const int j = k - r * FS_STAGGER;
+      if (j >= 0 && j < n_items) run_item(j, r);
     }
-    if (P.swiglu)
-      for (int r = 0; r < RT; r++)
-        fs_gemm_phase<64, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), F, d, MAP_A_U,
-                              fs_map_index(l, MAPL_WB), cnt(l, PH_FFN1, r), T_f * FS_S,
-                              cnt(l, PH_FFN1B, r), EpiRsSwiglu<bf16>{rsi, P.fa, P.f, F}, s_rs, fs_trace_id(l, PH_FFN1B, r, false), tslot);
-    // FFN down, residual, next block's input
-    for (int r = 0; r < RT; r++)
-      fs_gemm_phase<32, NS>(P, sh, run, cl, C, rot, r * FS_RT, rows_of(r), d, F, MAP_A_F,
-                            fs_map_index(l, MAPL_W2),
-                            P.swiglu ? cnt(l, PH_FFN1B, r) : cnt(l, PH_FFN1, r), T_f * FS_S,
-                            cnt(l, PH_FFN2, r),
-                            EpiResidNorm<bf16>{{}, P.h, d, last ? nullptr : P.ln1[l + 1], P.u,
-                                               P.nsq, np},
-                            s_rs, fs_trace_id(l, PH_FFN2, r, false), tslot);
-  }
 
   // ---- s_t = RMSNorm_f(h), t_dec += 1 (one warp per row, after the row
   // tile's last FFN)
@@ -1141,7 +1166,7 @@ __global__ void __launch_bounds__(FS_THREADS, 2) k_step_fused(const __grid_const
     const bool ok = s_skip == 0;
     __syncthreads();
     if (ok)
-      for (int i = gcta * 8 + warp; i < hi; i += ncta * 8)
+      for (int i = gcta * FS_WARPS + warp; i < hi; i += ncta * FS_WARPS)
         if (i >= m0) fs_final_row(P, i, lane);
     if (threadIdx.x == 0)
       fs_trace(P, tslot, fs_trace_id(L, 0x21, r, false), t0, t1, globaltimer_ns());
