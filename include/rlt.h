@@ -197,10 +197,11 @@ RLT_API int rlt_decoder_parallel(rlt_model *model, const int32_t *h_seq_ids, int
  *     gather and the final norm -- in one global order (layer, sublayer
  *     phase, 128-row tile), each waiting on dependency counters in the arena
  *     instead of on kernel boundaries ([RLT-96] "Three design principles and
- *     their caveats": kernel fusion and batched ready updates). The default
- *     for bf16 models it covers (up to 8192 slots, 64 decoder layers).
+ *     their caveats": kernel fusion and batched ready updates). Available
+ *     for the bf16 models it covers (up to 8192 slots, 64 decoder layers).
  *   RLT_STEP_CHAIN: a captured chain of about eight kernels per decoder
- *     block (the only form for fp32 models).
+ *     block; the default (measured faster), and the only form for fp32
+ *     models.
  * Both compute the same transition; results agree within the bf16
  * tolerance, not bit for bit (different split-K partitions). */
 enum { RLT_STEP_CHAIN = 0, RLT_STEP_FUSED = 1 };

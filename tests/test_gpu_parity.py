@@ -46,9 +46,11 @@ KERNELS = [(n, k) for n in SMALL for k in ("fused", "chain")
 
 def _use(m, kernel):
     from token_recurrent_decoding_b200 import rlt as R
+    assert m.get_step_kernel() == R.STEP_CHAIN  # the default
     if m.cfg.dtype == configs.BF16:
-        assert m.get_step_kernel() == R.STEP_FUSED  # the default for bf16 models
+        assert m.step_kernel_ctas() > 0  # the persistent step covers the model
     m.set_step_kernel(R.STEP_FUSED if kernel == "fused" else R.STEP_CHAIN)
+    assert m.get_step_kernel() == (R.STEP_FUSED if kernel == "fused" else R.STEP_CHAIN)
 
 
 @pytest.mark.parametrize("name,kernel", KERNELS)

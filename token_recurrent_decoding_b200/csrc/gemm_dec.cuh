@@ -263,8 +263,11 @@ template <int BN> struct DecSmem {
 // cluster size), at least three K blocks per CTA once K allows four splits
 // (each further split adds partial-tile traffic over distributed shared
 // memory), rounded down to one of the compiled counts 1, 2, 3, 4, 6, 8.
+#ifndef RLT_DEC_CTAS_PER_SM
+#define RLT_DEC_CTAS_PER_SM 1  // CTAs per SM the split count aims for
+#endif
 inline int dec_splits(int n_tiles, int kb, int num_sms) {
-  int s = num_sms / (n_tiles > 0 ? n_tiles : 1);
+  int s = RLT_DEC_CTAS_PER_SM * num_sms / (n_tiles > 0 ? n_tiles : 1);
   if (s > 8) s = 8;
   const int by_k = kb / 3 > 4 ? kb / 3 : 4;
   if (s > by_k) s = by_k;

@@ -1540,10 +1540,12 @@ RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *w, void *d_aren
     rlt_destroy(M);
     return RLT_ERR_CUDA;
   }
-  // bf16 models step with the persistent kernel when it covers them
+  // bf16 models may step with the persistent kernel when it covers them
+  // (rlt_set_step_kernel); the chain of kernels stays the default: it
+  // measured faster on every workload
   if (M->fused_setup) {
     if (M->fused_setup(M) == cudaSuccess) {
-      M->fused_ok = M->use_fused = true;
+      M->fused_ok = true;
     } else {
       cudaGetLastError();
     }
