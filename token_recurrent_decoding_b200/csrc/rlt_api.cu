@@ -30,7 +30,17 @@ using namespace rlt;
 
 namespace {
 
-constexpr int XCH = RLT_ATTEND_CHUNK;  // memory positions per cross-attention split
+constexpr int XCH = RLT_ATTEND_CHUNK;  // memory positions per split of rlt_attend
+
+// Memory positions per split of the decoder's cross-attention: rows are cut
+// into chunks of this many positions, one warp per chunk, merged in chunk
+// order. Models with few (slot, head) pairs use shorter chunks so a step has
+// enough units to keep every SM's warps streaming (a warp is latency-bound
+// on its own rows). A function of the configuration only, so a row's result
+// depends on its own t and never on the batch around it.
+int xattn_chunk(const rlt_config *c) {
+  return (long)c->max_seqs * c->n_heads < 2048 ? 256 : XCH;
+}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -47,6 +57,7 @@ struct Layout {
   size_t fs_cnt, fs_cnt_bytes, fs_maps;
   size_t total;
   int max_chunks, ptok, fs_rt;
+  int xch;  // memory positions per cross-attention split (xattn_chunk)
 };
 
 int elem_size(const rlt_config *c) { return c->dtype == RLT_BF16 ? 2 : 4; }
@@ -61,7 +72,7 @@ int check_config(const rlt_config *c) {
   if (c->ffn_dim <= 0 || c->vocab <= 0 || c->window < 1 || c->max_seqs < 1 || c->max_len < 1)
     return RLT_ERR_INVALID_ARG;
   // the sliding window is attended as one chunk of the decode attention
-  if (c->window > RLT_ATTEND_CHUNK) return RLT_ERR_UNSUPPORTED;
+  if (c->window > xattn_chunk(c)) return RLT_ERR_UNSUPPORTED;
   if (c->ffn_kind != RLT_GELU && c->ffn_kind != RLT_SWIGLU) return RLT_ERR_INVALID_ARG;
   if (c->dtype != RLT_F32 && c->dtype != RLT_BF16) return RLT_ERR_INVALID_ARG;
   if (c->mem_groups != 1 && c->mem_groups != c->n_dec_layers) return RLT_ERR_UNSUPPORTED;
@@ -92,7 +103,8 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
                                         : std::min<long>((long)S * T, 131072L);
   ptok = std::max<long>(ptok, c->max_len);
   L->ptok = (int)ptok;
-  L->max_chunks = (int)((T + XCH - 1) / XCH);
+  L->xch = xattn_chunk(c);
+  L->max_chunks = (int)((T + L->xch - 1) / L->xch);
   L->s = take(S * d * 4);
   L->t_dec = take(S * 4);
   L->t_enc = take(S * 4);
@@ -484,7 +496,7 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
   const int units = si.n_grid * c.n_heads * xchunks;
   const int grid = attn_balanced_ctas<T, DH>(units);  // also sets the smem limit
   return launch_k(k_attn_decode<T, DH>, dim3(grid), dim3((AttnCfg::NC + 1) * 32), smem, st,
-                  M->at<int>(L.nready) + si.chain, c.n_heads, window, XCH, xchunks, L.max_chunks,
+                  M->at<int>(L.nready) + si.chain, c.n_heads, window, L.xch, xchunks, L.max_chunks,
                   si.n_grid, M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0,
                   (const int *)M->at<int>(L.t_dec), M->at<float>(L.q) + r0 * c.d, base,
                   seq_stride, head_stride, v_offset,
@@ -856,7 +868,7 @@ template <int DH> cudaError_t fused_setup_impl(rlt_model *M) {
   P.alpha0 = c.alpha == 0.0f;
   P.xch = 1;
   P.max_chunks = L.max_chunks;
-  P.CH = XCH;
+  P.CH = L.xch;
   P.rt_max = L.fs_rt;
   P.kv_reuse = (c.mem_groups == 1 && LD > 1) ? 1 : 0;
   P.alpha = c.alpha;
@@ -1167,7 +1179,7 @@ StepInfo step_info(const rlt_model *M, const int32_t *ids, int n) {
     si.sum_keys += t + 1;
     si.sum_win += std::min(t + 1, M->cfg.window);
   }
-  si.xchunks = std::min(M->L.max_chunks, tmax / XCH + 1);
+  si.xchunks = std::min(M->L.max_chunks, tmax / M->L.xch + 1);
   si.n_grid = std::min(si.n_grid, M->cfg.max_seqs);
   return si;
 }
