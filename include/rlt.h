@@ -61,7 +61,8 @@ typedef enum rlt_status {
   RLT_ERR_DUPLICATE_ID = 5, /* a sequence listed twice in one batch */
   RLT_ERR_CUDA = 6,         /* a CUDA runtime call failed */
   RLT_ERR_TIMEOUT = 7,      /* a bounded device wait gave up */
-  RLT_ERR_DEVICE = 8        /* a kernel's own bounds check fired */
+  RLT_ERR_DEVICE = 8,       /* a kernel's own bounds check fired */
+  RLT_ERR_STALE = 9         /* snapshot of another configuration or other weights */
 } rlt_status;
 
 enum { RLT_GELU = 0, RLT_SWIGLU = 1 }; /* FFN form */
@@ -87,6 +88,10 @@ typedef struct rlt_config {
   int max_seqs;     /* sequence slots in the arena */
   int max_len;      /* positions per sequence (encoder memory capacity) */
   int max_prefill_tokens; /* encoder work buffer, tokens; 0 = automatic */
+  int enc_cache;    /* 1: keep every encoder layer's rotary keys and values of
+                       every position, so tokens can be appended one at a time
+                       (rlt_append_encoder, rlt_serve_step) and snapshots carry
+                       the encoder cache; 0: whole-sequence prefill only */
   float alpha;      /* feedback scale of the gated merge; 0 turns feedback off */
   float rms_eps;    /* RMSNorm epsilon (1e-6) */
   float rope_theta; /* rotary base (1e4) */
@@ -260,6 +265,105 @@ RLT_API int rlt_get_state(rlt_model *model, int seq, float *s_out,
  * <= max_len. Inputs may be device or pinned host memory. */
 RLT_API int rlt_set_state(rlt_model *model, int seq, const float *s_in,
                           const void *cache_in, int64_t t, rlt_stream stream);
+
+/* ------------------------------------------------------------ serving loop
+ * Once tokens are no longer given, each generated token goes back into the
+ * encoder, so the encoder cache and memory are part of the serving state
+ * ([RLT-96] "Training and serving implications"). These calls need a model
+ * created with enc_cache = 1. */
+
+/* Append one token to the encoder of each listed sequence (tokens[i] for
+ * h_seq_ids[i]; device or pinned host int32): the causal encoder runs at
+ * position t = t_enc over the encoder cache of positions 0..t-1 (the
+ * encoder is causal, [RLT-TC] "What is this technology", so this equals a
+ * whole-sequence prefill of the longer prompt at that position), writes e_t
+ * and the memory rows M_t of every group, and t_enc += 1.
+ * Errors: INVALID_ARG, DUPLICATE_ID, UNSUPPORTED (enc_cache = 0), CAPACITY
+ * (t_enc = max_len); out-of-range tokens set RLT_ERR_DEVICE. */
+RLT_API int rlt_append_encoder(rlt_model *model, const int32_t *tokens,
+                               const int32_t *h_seq_ids, int n, rlt_stream stream);
+
+/* Next-token logits from each listed sequence's current s_t ([RLT-96]
+ * "Architecture": the next-token distribution is read from s_t), with the
+ * embedding matrix as the output head: logits[i][v] = embed[v] . s (device
+ * float32 [n][vocab]). bf16 models round s to bf16 for the tensor cores.
+ * Errors: INVALID_ARG, DUPLICATE_ID, UNSUPPORTED (bf16 with vocab % 64). */
+RLT_API int rlt_lm_head(rlt_model *model, const int32_t *h_seq_ids, int n, float *logits,
+                        rlt_stream stream);
+
+/* One token per row from logits (device float32 [n][vocab]) into tokens_out
+ * (device int32 [n]). temperature 0: the argmax (lowest index among equal
+ * maxima). temperature > 0: the inverse CDF of softmax(logits /
+ * temperature) at uniforms[i] (device float32 [n] in [0, 1), drawn by the
+ * caller): the smallest v whose cumulative weight exceeds uniforms[i] times
+ * the total, summed in a fixed order in fp32 (reproducible).
+ * Errors: INVALID_ARG (negative or non-finite temperature, null pointers). */
+RLT_API int rlt_sample(rlt_model *model, const float *logits, int n, float temperature,
+                       const float *uniforms, int32_t *tokens_out, rlt_stream stream);
+
+/* One autoregressive step for each listed sequence, whose decoder stands at
+ * its last known token (t_dec = t_enc - 1): the transition at t = t_dec,
+ * logits from the new s_t (rlt_lm_head; `logits` is caller workspace,
+ * device float32 [n][vocab], left holding them), a token drawn as
+ * rlt_sample does into tokens_out (device int32 [n]), and that token
+ * appended to the encoder (rlt_append_encoder), so the next call continues.
+ * Errors: as the calls it runs; NOT_READY when t_dec != t_enc - 1. */
+RLT_API int rlt_serve_step(rlt_model *model, const int32_t *h_seq_ids, int n,
+                           float temperature, const float *uniforms, float *logits,
+                           int32_t *tokens_out, rlt_stream stream);
+
+/* ------------------------------------------------------------ snapshots
+ * An exact prefix snapshot of one slot: everything a later transition of
+ * that sequence reads, so restoring it into any slot of a model with the
+ * same configuration and the same weight values continues bit for bit as
+ * if nothing had happened ([RLT-96] "Training and serving implications":
+ * encoder cache and memory, the full decoder state, position metadata, the
+ * window convention and a model version; "RLT carries decoder state between
+ * tokens..." (lub-systems.com), "How to prepare systems for state storage
+ * and transfer": a weight update invalidates stored states).
+ * Layout: this header, then the sections at the header's byte offsets
+ * (256-byte aligned), in the model dtype unless noted:
+ *   s        [d] float32                      decoder output s_{t_dec - 1}
+ *   window   [L_D][2][W-1][d]                 as rlt_get_state
+ *   e        [t_enc][d]                       encoder outputs
+ *   mem      [G][t_enc][2][d]                 memory rows (K row, V row)
+ *   enc_kv   [L_E][t_enc][2][d]               encoder cache (enc_cache only)
+ * The fingerprint is a 64-bit hash of the configuration and of every weight
+ * value the model reads, computed on the device when the snapshot is taken
+ * and again when it is restored. */
+#define RLT_SNAPSHOT_MAGIC 0x3150414E53544C52ull /* "RLTSNAP1", little-endian */
+typedef struct rlt_snapshot_header {
+  uint64_t magic;       /* RLT_SNAPSHOT_MAGIC */
+  uint64_t fingerprint; /* configuration and weight values */
+  uint64_t bytes;       /* the whole snapshot, header included */
+  uint64_t off_s, off_window, off_e, off_mem, off_enc_kv; /* section offsets */
+  int64_t t_dec, t_enc; /* transitions taken, encoder positions known */
+  int32_t version;      /* 1 */
+  int32_t d, n_heads, head_dim, n_enc_layers, n_dec_layers, ffn_dim, ffn_kind, vocab;
+  int32_t window, mem_groups, tied, dtype, enc_cache;
+  float alpha, rms_eps, rope_theta;
+} rlt_snapshot_header;
+
+/* Host only. Bytes of slot `seq`'s snapshot as it stands (0 if invalid). */
+RLT_API size_t rlt_snapshot_bytes(rlt_model *model, int seq);
+
+/* Write slot `seq`'s snapshot to buf (device or pinned host memory, >=
+ * rlt_snapshot_bytes); complete when `stream` reaches this point.
+ * Errors: INVALID_ARG, CAPACITY (bytes too small). */
+RLT_API int rlt_get_snapshot(rlt_model *model, int seq, void *buf, size_t bytes,
+                             rlt_stream stream);
+
+/* Restore a snapshot (device or pinned host memory) into slot `seq`. Reads
+ * and checks the header and recomputes the weight fingerprint before
+ * returning (synchronising `stream`), then enqueues the copies. Errors:
+ * INVALID_ARG (not a snapshot, sizes), STALE (another configuration or other
+ * weight values), CAPACITY (positions beyond max_len). */
+RLT_API int rlt_set_snapshot(rlt_model *model, int seq, const void *buf, size_t bytes,
+                             rlt_stream stream);
+
+/* Host only (synchronous): the fingerprint snapshots carry for this model's
+ * configuration and current weight values. */
+RLT_API int rlt_model_fingerprint(rlt_model *model, uint64_t *out);
 
 /* Export the encoder output of slot `seq`: e_out [t_enc][d] and mem_out
  * [G][t_enc][2][d] (K row then V row per position) in the model dtype.

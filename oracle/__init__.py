@@ -88,6 +88,9 @@ def _declare(lib):
     lib.orc_decode_parallel_nofeedback.argtypes = [P, P, P, P, C.c_int, C.c_int, P]
     lib.orc_run_batch.argtypes = [P, P, P, C.c_int, P, C.c_int, C.c_int, P]
     lib.orc_run_batch.restype = C.c_int
+    lib.orc_lm_head.argtypes = [P, P, P, P]
+    lib.orc_sample.argtypes = [P, C.c_int, C.c_double, C.c_double]
+    lib.orc_sample.restype = C.c_int
 
 
 def _ptr(a: np.ndarray):
@@ -242,6 +245,13 @@ class Oracle:
                                                 mem.shape[1], T, _ptr(out))
         return out[:T]
 
+    def lm_head(self, s):
+        """Next-token logits [V] read from s_t."""
+        s = self._a(s, (self.cfg.d,))
+        out = np.zeros(self.cfg.vocab, self.dt)
+        self.lib.orc_lm_head(*self._args(), _ptr(s), _ptr(out))
+        return out
+
     def run_batch(self, tokens, lengths, n_threads=0):
         """Full runs of B sequences in parallel; returns (s_final [B][d], threads)."""
         tok = np.ascontiguousarray(tokens, dtype=np.int32)
@@ -291,6 +301,14 @@ def attend(q, K, V, precision="f64"):
     out = np.zeros(q.shape[0], dt)
     lib.orc_attend_dense(_ptr(q), _ptr(K), _ptr(V), K.shape[0], q.shape[0], _ptr(out))
     return out
+
+
+def sample(logits, temperature, u, precision="f64"):
+    """One token from logits (argmax at temperature 0, else inverse CDF at u)."""
+    lib = _lib(precision)
+    dt = np.float64 if precision == "f64" else np.float32
+    lg = np.ascontiguousarray(logits, dt)
+    return int(lib.orc_sample(_ptr(lg), lg.shape[0], float(temperature), float(u)))
 
 
 def scalar(fn: str, x: float) -> float:

@@ -524,6 +524,40 @@ void orc_decode_parallel_nofeedback(const orc_cfg *c, const orc_weights *w,
   scratch_free(&sc);
 }
 
+/* -------------------------------------------------------- serving loop */
+
+/* Next-token logits read from the decoder output s_t ([RLT-96]
+ * "Architecture": the next-token distribution is read from s_t), with the
+ * embedding matrix as the output head (reading: tied input and output
+ * embeddings; the pages name no separate head). logits [V]. */
+void orc_lm_head(const orc_cfg *c, const orc_weights *w, const real *s,
+                 real *logits) {
+  orc_linear(w->embed, s, c->vocab, c->d, logits);
+}
+
+/* One token from logits (reading: the pages leave decoding open).
+ * tau = 0: the first index of the largest logit. tau > 0: inverse-CDF
+ * sampling of softmax(logits / tau) at u in [0, 1): the smallest v whose
+ * cumulative weight exceeds u times the total, with weights
+ * exp((logit_v - max) / tau). */
+int orc_sample(const real *logits, int V, double tau, double u) {
+  int arg = 0;
+  for (int v = 1; v < V; v++)
+    if (logits[v] > logits[arg]) arg = v;
+  if (!(tau > 0)) return arg;
+  double Z = 0;
+  for (int v = 0; v < V; v++) Z += exp(((double)logits[v] - (double)logits[arg]) / tau);
+  double target = u * Z, cum = 0;
+  int last = arg;
+  for (int v = 0; v < V; v++) {
+    double p = exp(((double)logits[v] - (double)logits[arg]) / tau);
+    cum += p;
+    if (p > 0) last = v;
+    if (cum > target) return v;
+  }
+  return last;
+}
+
 /* Independent sequences in parallel (OpenMP over sequences only): full
  * encoder + decoder run of each; s_final [B][d] gets each sequence's last s.
  * tok [B][tok_stride]. Returns the number of threads used. */

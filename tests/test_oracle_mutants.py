@@ -73,6 +73,13 @@ MUTANTS = {
                                                   "orc_linear(w->dec_wox[0], s->a, d, d, s->o);"),
     "decoder ffn of layer 0": ("ffn(c, w->dec_w1[l], w->dec_wb[l], w->dec_w2[l],",
                                "ffn(c, w->dec_w1[0], w->dec_wb[0], w->dec_w2[0],"),
+    "sampler keeps the last maximum": ("if (logits[v] > logits[arg]) arg = v;",
+                                       "if (logits[v] >= logits[arg]) arg = v;"),
+    "sampler total weight at the inverse temperature": (
+        "for (int v = 0; v < V; v++) Z += exp(((double)logits[v] - (double)logits[arg]) / tau);",
+        "for (int v = 0; v < V; v++) Z += exp(((double)logits[v] - (double)logits[arg]) * tau);"),
+    "lm head reads s at an offset": ("orc_linear(w->embed, s, c->vocab, c->d, logits);",
+                                     "orc_linear(w->embed + 1, s, c->vocab - 1, c->d, logits);"),
     "decoder cross-attention norms in reverse layer order": (
         "orc_rmsnorm(h, w->dec_ln2[l], d, c->rms_eps, s->u);",
         "orc_rmsnorm(h, w->dec_ln2[c->n_dec - 1 - l], d, c->rms_eps, s->u);"),

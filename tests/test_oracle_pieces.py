@@ -101,3 +101,49 @@ def test_attend_special_cases():
     q = np.full(dh, 100.0)
     K = np.zeros((5, dh)); K[3] = 10.0
     np.testing.assert_allclose(oracle.attend(q, K, V), V[3], rtol=1e-13)
+
+
+# ---------------------------------------------------------- serving loop
+def test_lm_head_is_embedding_matmul():
+    """Next-token logits = E s_t (the embedding matrix as the output head)."""
+    from token_recurrent_decoding_b200 import configs, inputs
+    cfg = configs.TINY
+    w = {k: v.astype(np.float64) for k, v in inputs.make_weights(cfg, 0, True).items()}
+    o = oracle.Oracle(cfg, w)
+    s = rng.standard_normal(cfg.d)
+    ref = (torch.tensor(w["embed"]) @ torch.tensor(s)).numpy()
+    np.testing.assert_allclose(o.lm_head(s), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_sample_temperature_zero_is_first_argmax():
+    lg = np.array([0.5, 2.0, -1.0, 2.0, 1.9])
+    assert oracle.sample(lg, 0.0, 0.7) == 1  # the first of the two maxima
+    for k in range(20):
+        x = rng.standard_normal(33)
+        assert oracle.sample(x, 0.0, 0.3) == int(np.argmax(x))
+
+
+def test_sample_frequencies_on_a_uniform_grid_match_softmax():
+    """At u_k = (k + 1/2) / N the draws split into counts N p_v (within one
+    per boundary) -- the defining property of inverse-CDF sampling -- with p
+    from torch.softmax of logits / temperature."""
+    lg = np.array([1.0, -0.5, 0.25, 2.0, -3.0, 0.0, 0.7])
+    N = 20000
+    for tau in (0.5, 1.0, 2.5):
+        counts = np.zeros(lg.size, int)
+        for k in range(N):
+            counts[oracle.sample(lg, tau, (k + 0.5) / N)] += 1
+        p = torch.softmax(torch.tensor(lg) / tau, 0).numpy()
+        assert np.all(np.abs(counts - N * p) <= 1.0 + 1e-9), (tau, counts, N * p)
+
+
+def test_sample_temperature_scales_logits():
+    """Temperature tau on logits l draws what temperature 1 draws on l / tau
+    (away from CDF boundaries), and the ends of u give the first and the
+    last token with weight."""
+    lg = rng.standard_normal(50)
+    for tau in (0.3, 3.0):
+        for u in (0.013, 0.25, 0.5, 0.77, 0.991):
+            assert oracle.sample(lg, tau, u) == oracle.sample(lg / tau, 1.0, u)
+    assert oracle.sample(lg, 1.0, 0.0) == 0
+    assert oracle.sample(lg, 1.0, 1.0 - 1e-15) == lg.size - 1

@@ -240,6 +240,35 @@ template <typename T> struct EpiQkvRope {
   }
 };
 
+// y = C in fp32, no row scale (next-token logits from s_t)
+struct EpiF32Dec {
+  static constexpr int kKind = kPair;
+  static constexpr bool kRowScale = false;
+  RowScaleIn rsi;  // unused
+  float *out;
+  int ld;
+  __device__ void pair(int m, int n, float a, float b, float) const {
+    *reinterpret_cast<float2 *>(out + (size_t)m * ld + n) = make_float2(a, b);
+  }
+};
+
+// Memory rows of appended positions: K (kv = 0) or V (kv = 1) of row m into
+// the head-major memory group at (ready[m], pos[m]).
+template <typename T> struct EpiMemRow {
+  static constexpr int kKind = kPair;
+  static constexpr bool kRowScale = false;
+  RowScaleIn rsi;  // unused
+  T *mem_g;
+  const int *ready, *pos;
+  int H, DH, max_len, kv;
+  __device__ void pair(int m, int n, float a, float b, float) const {
+    const int h = n / DH, j = n - h * DH;
+    const size_t i = ((((size_t)ready[m] * H + h) * 2 + kv) * max_len + pos[m]) * DH + j;
+    mem_g[i] = from_f<T>(a);
+    mem_g[i + 1] = from_f<T>(b);
+  }
+};
+
 // ------------------------------------------------------------- shared memory
 constexpr int DEC_BAR_BYTES = 1024;  // barriers + TMEM slot, keeps tiles 1024-aligned
 

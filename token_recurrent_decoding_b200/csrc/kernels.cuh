@@ -479,6 +479,210 @@ __global__ void k_get_memory(int G, int H, int dh, int max_seqs, int max_len, in
   }
 }
 
+// [G][T_enc][2][d] -> memory of one slot (all groups); the inverse of
+// k_get_memory (also used for the encoder cache, G = L_E).
+template <typename T>
+__global__ void k_set_memory(int G, int H, int dh, int max_seqs, int max_len, int seq, int T_enc,
+                             const T *__restrict__ in, T *__restrict__ mem) {
+  int d = H * dh;
+  long total = (long)G * T_enc * 2 * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    int c = (int)(idx % d);
+    int kv = (int)((idx / d) % 2);
+    int p = (int)((idx / (2L * d)) % T_enc);
+    int g = (int)(idx / (2L * d * T_enc));
+    int h = c / dh, j = c % dh;
+    mem[(((((size_t)g * max_seqs + seq) * H + h) * 2 + kv) * max_len + p) * dh + j] = in[idx];
+  }
+}
+
+// 64-bit finalizer of the SplitMix64 generator (Steele, Lea and Flood,
+// "Fast splittable pseudorandom number generators", with Vigna's published
+// constants): a bijection of 64-bit words that spreads every input bit.
+__host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Weight fingerprint: *acc += sum over the 32-bit words w[i] of one tensor of
+// mix64(word, salt + i). A sum modulo 2^64, so the result does not depend on
+// the order the threads add in; any changed word changes it with
+// overwhelming probability.
+__global__ void k_fingerprint(const uint32_t *__restrict__ w, size_t n, uint64_t salt,
+                              unsigned long long *acc) {
+  uint64_t h = 0;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    h += mix64(((uint64_t)w[i] << 32) ^ (salt + i * 0x9E3779B97F4A7C15ull));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) h += __shfl_xor_sync(FULL_MASK, h, o);
+  if ((threadIdx.x & 31) == 0) atomicAdd(acc, (unsigned long long)h);
+}
+
+// ------------------------------------------------------------ serving loop
+// One appended token per row i < n: h = E[tok_i] (fp32); with gamma1 also the
+// first encoder block's input bf16(h * gamma1) and the row's sum of squares
+// (partial 0; partials 1..np-1 zero), the form the decode GEMMs' fused
+// RMSNorm reads. An out-of-range token records RLT_ERR_DEVICE and embeds 0.
+template <typename T>
+__global__ void k_append_embed(int n, int d, int vocab, const int *__restrict__ tok,
+                               const T *__restrict__ E, float *__restrict__ h,
+                               const float *__restrict__ gamma1, T *__restrict__ u,
+                               float *__restrict__ nsq, int np, int *err) {
+  __shared__ float red[32];
+  const int i = blockIdx.x;
+  if (i >= n) return;
+  const int id = tok[i];
+  const bool ok = id >= 0 && id < vocab;
+  if (!ok && threadIdx.x == 0) set_error(err, DEV_ERR_TOKEN);
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float v = ok ? to_f(E[(size_t)id * d + c]) : 0.f;
+    h[(size_t)i * d + c] = v;
+    if (gamma1) {
+      u[(size_t)i * d + c] = from_f<T>(v * gamma1[c]);
+      ss += v * v;
+    }
+  }
+  if (!gamma1) return;
+  ss = warp_sum(ss);
+  const int w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int k = 0; k < nw; k++) tot += red[k];
+    nsq[(size_t)i * np] = tot;
+  }
+  for (int k = 1 + threadIdx.x; k < np; k += blockDim.x) nsq[(size_t)i * np + k] = 0.f;
+}
+
+// out[i] = s[ready[i]] in the GEMM input type (row i of the next-token head).
+template <typename T>
+__global__ void k_stage_s(int n, int d, const int *__restrict__ ready, const float *__restrict__ s,
+                          T *__restrict__ out) {
+  const int i = blockIdx.x;
+  if (i >= n) return;
+  const float *sr = s + (size_t)ready[i] * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) out[(size_t)i * d + c] = from_f<T>(sr[c]);
+}
+
+// Next token of row i (one 1024-thread block per row) from its logits:
+// temperature 0 takes the argmax (the lowest index among equal maxima);
+// otherwise the inverse CDF of softmax(logits / temperature) at the row's
+// uniform u in [0, 1): the smallest v whose cumulative weight exceeds u Z,
+// Z the total weight, weights exp((l_v - max) / temperature) in fp32. Every
+// sum runs in a fixed order (each thread a contiguous segment, then a scan of
+// the segment sums in thread order), so the draw is reproducible.
+constexpr int SAMPLE_THREADS = 1024;
+
+__global__ void __launch_bounds__(SAMPLE_THREADS)
+    k_sample(int V, const float *__restrict__ logits, float tau,
+             const float *__restrict__ uniforms, int *__restrict__ tokens) {
+  __shared__ float s_f[SAMPLE_THREADS / 32];
+  __shared__ int s_i[SAMPLE_THREADS / 32];
+  __shared__ float s_excl[SAMPLE_THREADS];
+  __shared__ float s_bcast;
+  __shared__ int s_tok, s_arg;
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float *lr = logits + (size_t)row * V;
+  const int seg = (V + SAMPLE_THREADS - 1) / SAMPLE_THREADS;
+  const int lo = min(V, tid * seg), hi = min(V, lo + seg);
+  // maximum and its lowest index
+  float mx = -INFINITY;
+  int arg = V;
+  for (int v = lo; v < hi; v++)
+    if (lr[v] > mx) {
+      mx = lr[v];
+      arg = v;
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(FULL_MASK, mx, o);
+    const int a2 = __shfl_xor_sync(FULL_MASK, arg, o);
+    if (m2 > mx || (m2 == mx && a2 < arg)) {
+      mx = m2;
+      arg = a2;
+    }
+  }
+  if (lane == 0) {
+    s_f[warp] = mx;
+    s_i[warp] = arg;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    mx = s_f[lane];
+    arg = s_i[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(FULL_MASK, mx, o);
+      const int a2 = __shfl_xor_sync(FULL_MASK, arg, o);
+      if (m2 > mx || (m2 == mx && a2 < arg)) {
+        mx = m2;
+        arg = a2;
+      }
+    }
+    if (lane == 0) {
+      s_bcast = mx;
+      s_arg = arg;
+    }
+  }
+  __syncthreads();
+  if (!(tau > 0.f)) {
+    if (tid == 0) tokens[row] = s_arg;
+    return;
+  }
+  mx = s_bcast;
+  const float inv_tau = 1.f / tau;
+  // segment weight, then the exclusive scan of segment weights in thread order
+  float w = 0.f;
+  for (int v = lo; v < hi; v++) w += expf((lr[v] - mx) * inv_tau);
+  float incl = w;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(FULL_MASK, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_f[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    float t = s_f[lane], ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(FULL_MASK, ti, o);
+      if (lane >= o) ti += y;
+    }
+    s_f[lane] = ti - t;  // exclusive prefix of the warp totals
+    if (lane == 31) s_bcast = ti;  // Z
+  }
+  __syncthreads();
+  const float excl = s_f[warp] + incl - w;
+  s_excl[tid] = excl;
+  if (tid == 0) s_tok = -1;
+  __syncthreads();
+  const float Z = s_bcast;
+  const float target = uniforms[row] * Z;
+  // the segment holding the target: excl <= target < the next non-empty
+  // segment's excl (the last non-empty segment takes everything above)
+  const int last = (V - 1) / seg;
+  const float next = tid < last ? s_excl[tid + 1] : INFINITY;
+  if (hi > lo && excl <= target && target < next) {
+    float cum = excl;
+    int tok = lo;
+    for (int v = lo; v < hi; v++) {
+      const float p = expf((lr[v] - mx) * inv_tau);
+      cum += p;
+      if (p > 0.f) tok = v;  // rounding that never passes the target: last weighted token
+      if (cum > target) break;
+    }
+    atomicMax(&s_tok, tok);
+  }
+  __syncthreads();
+  if (tid == 0) tokens[row] = s_tok >= 0 ? s_tok : s_arg;
+}
+
 // s <- s* for the listed slots.
 __global__ void k_reset_s(int n, int d, const int *__restrict__ ids, const float *__restrict__ sstar,
                           float *__restrict__ s) {

@@ -47,6 +47,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Layout {
   // persistent state
   size_t s, t_dec, t_enc, e, mem, ring, rope, err, ctl;
+  size_t enc_kv;  // encoder cache [L_E][max_seqs][H][2][max_len][dh] (enc_cache)
+  size_t fp;      // weight fingerprint accumulator (one uint64)
   // decoder step work buffers (max_seqs rows)
   size_t nready, ready, pos, h, xin, e32, s32, qkv, q, a, u, fa, f, part, counters;
   size_t nsq;  // per-row partial sums of squares of h over 32-column tiles (bf16 models)
@@ -80,6 +82,7 @@ int check_config(const rlt_config *c) {
   if (!std::isfinite(c->alpha) || !(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f))
     return RLT_ERR_INVALID_ARG;
   if (c->max_prefill_tokens < 0) return RLT_ERR_INVALID_ARG;
+  if (c->enc_cache != 0 && c->enc_cache != 1) return RLT_ERR_INVALID_ARG;
   if (c->max_prefill_tokens > 0 && c->max_prefill_tokens < c->max_len) return RLT_ERR_INVALID_ARG;
   int dh = c->head_dim;
   if (dh != 16 && dh != 32 && dh != 64 && dh != 128) return RLT_ERR_UNSUPPORTED;
@@ -111,6 +114,8 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->e = take(S * T * d * es);
   L->mem = take(G * S * H * 2 * T * dh * es);
   L->ring = take(LD * S * H * 2 * W * dh * es);
+  L->enc_kv = take(c->enc_cache ? (size_t)c->n_enc_layers * S * H * 2 * T * dh * es : 0);
+  L->fp = take(8);
   L->rope = take(T * (dh / 2) * 8);
   L->err = take(16);
   L->ctl = take(sizeof(DevCtl));
@@ -147,6 +152,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->ef = take(P * F * es);
   L->etok = take(P * d * es);
   size_t st = std::max(LD * 2 * (W > 1 ? W - 1 : 1) * d * es, G * T * 2 * d * es);
+  if (c->enc_cache) st = std::max(st, (size_t)c->n_enc_layers * T * 2 * d * es);
   L->staging_bytes = st;
   L->staging = take(st);
   L->fs_rt = (int)((S + FS_RT - 1) / FS_RT);
@@ -230,6 +236,9 @@ struct rlt_model {
   cudaError_t (*get_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
   cudaError_t (*set_window)(rlt_model *, int, long, cudaStream_t) = nullptr;
   cudaError_t (*get_memory)(rlt_model *, int, int, cudaStream_t) = nullptr;
+  cudaError_t (*hm_copy)(rlt_model *, size_t, int, int, int, bool, cudaStream_t) = nullptr;
+  cudaError_t (*append)(rlt_model *, int, int, cudaStream_t) = nullptr;
+  cudaError_t (*lm_head)(rlt_model *, int, float *, cudaStream_t) = nullptr;
 };
 
 namespace {
@@ -488,7 +497,7 @@ template <typename T> struct W_ {
 template <typename T, int DH>
 cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunks,
                         const T *base, long seq_stride, long head_stride, long v_offset,
-                        T *out, cudaStream_t st) {
+                        T *out, cudaStream_t st, const int *t_seq = nullptr) {
   constexpr int smem = attn_smem_bytes<T, DH>();
   const Layout &L = M->L;
   const rlt_config &c = M->cfg;
@@ -498,7 +507,7 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
   return launch_k(k_attn_decode<T, DH>, dim3(grid), dim3((AttnCfg::NC + 1) * 32), smem, st,
                   M->at<int>(L.nready) + si.chain, c.n_heads, window, L.xch, xchunks, L.max_chunks,
                   si.n_grid, M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0,
-                  (const int *)M->at<int>(L.t_dec), M->at<float>(L.q) + r0 * c.d, base,
+                  t_seq ? t_seq : (const int *)M->at<int>(L.t_dec), M->at<float>(L.q) + r0 * c.d, base,
                   seq_stride, head_stride, v_offset,
                   M->at<float>(L.part) + r0 * H * L.max_chunks * (DH + 2),
                   M->at<int>(L.counters) + r0 * H, out, 1.0f / sqrtf((float)DH),
@@ -1052,6 +1061,15 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, int nblk, cudaStream_t st) {
       k_enc_qkv_post<T><<<blocks_for((long)ntok * H * (DH / 2), 256), 256, 0, st>>>(
           ntok, H, DH, tpos, eqkv, rope, Qh, Kh, Vh, (T *)nullptr);
     }
+    if (c.enc_cache) {
+      // every position's rotary key and value, for later one-token appends
+      Span sp(M, st, K);
+      k_ring_from_hm<T><<<blocks_for((long)ntok * H * (DH * (int)sizeof(T) / 16), 256), 256, 0,
+                          st>>>(ntok, H, DH, c.max_len, 0, tslot, tpos, Kh, Vh,
+                                M->at<T>(L.enc_kv) + (size_t)l * c.max_seqs * H * 2 *
+                                                         c.max_len * DH);
+      RLT_TRY(cudaGetLastError());
+    }
     {
       Span sp(M, st, K);
       RLT_TRY((enc_attention<T, DH>(M, ntok, nblk, Qh, Kh, Vh, ea, st)));
@@ -1087,6 +1105,150 @@ cudaError_t prefill_impl(rlt_model *M, int ntok, int nblk, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------ serving loop
+// One token appended to the encoder of each ready-list row i < n (slot
+// ready[i], token tok[i], position pos[i] = its t_enc): the causal encoder
+// step of that position against the encoder cache of positions 0..t-1
+// ([RLT-96] "Training and serving implications": the encoder cache is part
+// of serving state), then e_t and the memory rows M_t of every group. The
+// same sublayers as the prefill, in the decode step's form: decode GEMMs with
+// the fused norms (bf16) or SIMT GEMMs (fp32), and the decode attention over
+// the cache rows 0..t with the row written by this call walked last.
+template <typename T, int DH>
+cudaError_t append_impl(rlt_model *M, int n, int tmax, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const rlt_weights &w = M->w;
+  const int d = c.d, H = c.n_heads, F = c.ffn_dim, np = d / 32;
+  const float eps = c.rms_eps;
+  const int ng = std::min((n + 63) / 64 * 64, c.max_seqs);
+  const int *nd = M->at<int>(L.nready);
+  int *ready = M->at<int>(L.ready), *pos = M->at<int>(L.pos);
+  float *h = M->at<float>(L.h), *q = M->at<float>(L.q), *fa = M->at<float>(L.fa);
+  float *nsq = M->at<float>(L.nsq), *qkv = M->at<float>(L.qkv);
+  T *u = M->at<T>(L.u), *a = M->at<T>(L.a), *f = M->at<T>(L.f);
+  const float2 *rope = M->at<float2>(L.rope);
+  const size_t cache_layer = (size_t)c.max_seqs * H * 2 * c.max_len * DH;
+  const size_t mem_group = cache_layer;
+  const int xch = std::min(L.max_chunks, tmax / L.xch + 1);
+  const StepInfo si{0, n, ng, 0, xch, 0.0, 0.0};
+  const int K = RLT_K_ENC;
+  constexpr bool tc = std::is_same<T, bf16>::value;
+  const RowScaleIn rsi{nsq, np, 1.0f / (float)d, eps};
+  {
+    Span sp(M, st, K);
+    k_append_embed<T><<<n, 256, 0, st>>>(
+        n, d, c.vocab, M->at<int>(L.tok), (const T *)w.embed, h,
+        tc && c.n_enc_layers > 0 ? (const float *)w.enc_ln1[0] : nullptr, u, nsq, np,
+        M->at<int>(L.err));
+    RLT_TRY(cudaGetLastError());
+  }
+  for (int l = 0; l < c.n_enc_layers; l++) {
+    T *cache_l = M->at<T>(L.enc_kv) + (size_t)l * cache_layer;
+    if constexpr (tc) {
+      using BNQ = std::integral_constant<int, (DH >= 32 ? DH : 32)>;
+      Span sp(M, st, K);
+      RLT_TRY(launch_dec<BNQ::value>(M, ng, nd, c.max_seqs, 0, 3 * d, d, u,
+                                     (const bf16 *)w.enc_wqkv[l],
+                                     EpiQkvRope<bf16>{rsi, q, cache_l, ready, pos, rope, H, DH,
+                                                      c.max_len, d},
+                                     st));
+    } else {
+      Span sp(M, st, K);
+      k_rmsnorm<T><<<blocks_for((long)n * 32, 256), 256, 0, st>>>(
+          n, nullptr, d, h, (const float *)w.enc_ln1[l], eps, u);
+      RLT_TRY(gemm(n, nullptr, 3 * d, d, u, d, (const T *)w.enc_wqkv[l], d,
+                   EpiStoreF32{qkv, 3 * d}, st));
+      k_dec_qkv_post<T><<<blocks_for((long)n * H * (DH / 2), 256), 256, 0, st>>>(
+          nd, H, DH, c.max_len, ready, pos, qkv, rope, q, cache_l);
+      RLT_TRY(cudaGetLastError());
+    }
+    {
+      Span sp(M, st, K);
+      RLT_TRY((launch_attn<T, DH>(M, si, c.max_len, xch, cache_l, (long)H * 2 * c.max_len * DH,
+                                  2L * c.max_len * DH, (long)c.max_len * DH, a, st,
+                                  M->at<int>(L.t_enc))));
+    }
+    if constexpr (tc) {
+      Span sp(M, st, K);
+      const bf16 *W1 = (const bf16 *)w.enc_w1[l], *W2 = (const bf16 *)w.enc_w2[l];
+      RLT_TRY(launch_dec<32>(M, ng, nd, c.max_seqs, 0, d, d, a, (const bf16 *)w.enc_wo[l],
+                             EpiResidNorm<bf16>{{}, h, d, (const float *)w.enc_ln2[l], u, nsq, np},
+                             st));
+      if (c.ffn_kind == RLT_GELU) {
+        RLT_TRY(launch_dec<64>(M, ng, nd, c.max_seqs, 0, F, d, u, W1,
+                               EpiRsGelu<bf16>{rsi, f, F}, st));
+      } else {
+        RLT_TRY(launch_dec<64>(M, ng, nd, c.max_seqs, 0, F, d, u, W1, EpiRsF32{rsi, fa, F}, st));
+        RLT_TRY(launch_dec<64>(M, ng, nd, c.max_seqs, 0, F, d, u, (const bf16 *)w.enc_wb[l],
+                               EpiRsSwiglu<bf16>{rsi, fa, f, F}, st));
+      }
+      const bool last = l + 1 == c.n_enc_layers;
+      RLT_TRY(launch_dec<32>(M, ng, nd, c.max_seqs, 0, d, F, f, W2,
+                             EpiResidNorm<bf16>{{}, h, d,
+                                                last ? nullptr : (const float *)w.enc_ln1[l + 1],
+                                                u, nsq, np},
+                             st));
+    } else {
+      Span sp(M, st, K);
+      RLT_TRY(gemm(n, nullptr, d, d, a, d, (const T *)w.enc_wo[l], d, EpiResid{h, d}, st));
+      k_rmsnorm<T><<<blocks_for((long)n * 32, 256), 256, 0, st>>>(
+          n, nullptr, d, h, (const float *)w.enc_ln2[l], eps, u);
+      if (c.ffn_kind == RLT_GELU) {
+        RLT_TRY(gemm(n, nullptr, F, d, u, d, (const T *)w.enc_w1[l], d, EpiGelu<T>{f, F}, st));
+      } else {
+        RLT_TRY(gemm(n, nullptr, F, d, u, d, (const T *)w.enc_w1[l], d, EpiStoreF32{fa, F}, st));
+        RLT_TRY(gemm(n, nullptr, F, d, u, d, (const T *)w.enc_wb[l], d,
+                     EpiSwiglu<T>{fa, f, F}, st));
+      }
+      RLT_TRY(gemm(n, nullptr, d, F, f, F, (const T *)w.enc_w2[l], F, EpiResid{h, d}, st));
+    }
+  }
+  {
+    // e_t = RMSNorm_E(h) into e and into the rows the memory GEMMs read
+    Span sp(M, st, K);
+    k_enc_final<T><<<blocks_for((long)n * 32, 256), 256, 0, st>>>(
+        n, d, c.max_len, h, (const float *)w.enc_lnf, eps, ready, pos, a, M->at<T>(L.e));
+    RLT_TRY(cudaGetLastError());
+  }
+  for (int g = 0; g < c.mem_groups; g++) {
+    T *mg = M->at<T>(L.mem) + (size_t)g * mem_group;
+    Span sp(M, st, K);
+    for (int kv = 0; kv < 2; kv++) {
+      const T *Wm = (const T *)(kv ? w.mem_wv[g] : w.mem_wk[g]);
+      if constexpr (tc)
+        RLT_TRY(launch_dec<32>(M, ng, nd, c.max_seqs, 0, d, d, a, Wm,
+                               EpiMemRow<bf16>{{}, mg, ready, pos, H, DH, c.max_len, kv}, st));
+      else
+        RLT_TRY(gemm(n, nullptr, d, d, a, d, Wm, d,
+                     EpiMem<T>{mg, ready, pos, H, DH, c.max_len, kv}, st));
+    }
+  }
+  return cudaGetLastError();
+}
+
+// Next-token logits of each ready-list row i < n from its s_t: logits[i][v] =
+// E[v] . s_t (the embedding matrix read as the output head). bf16 models
+// round s_t to bf16 for the tensor-core GEMM, like every other GEMM input.
+template <typename T>
+cudaError_t lm_head_impl(rlt_model *M, int n, float *logits, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const int d = c.d, V = c.vocab;
+  T *u = M->at<T>(L.u);
+  Span sp(M, st, RLT_K_GEMM, (double)V * d * sizeof(T) + (double)n * d * 4 + (double)n * V * 4,
+          2.0 * n * V * d);
+  k_stage_s<T><<<n, 256, 0, st>>>(n, d, M->at<int>(L.ready), M->at<float>(L.s), u);
+  RLT_TRY(cudaGetLastError());
+  if constexpr (std::is_same<T, bf16>::value) {
+    const int ng = std::min((n + 63) / 64 * 64, c.max_seqs);
+    return launch_dec<64>(M, ng, M->at<int>(L.nready), c.max_seqs, 0, V, d, u,
+                          (const bf16 *)M->w.embed, EpiF32Dec{{}, logits, V}, st);
+  } else {
+    return gemm(n, nullptr, V, d, u, d, (const T *)M->w.embed, d, EpiStoreF32{logits, V}, st);
+  }
+}
+
 template <typename T>
 cudaError_t get_window_impl(rlt_model *M, int seq, long t, cudaStream_t st) {
   const rlt_config &c = M->cfg;
@@ -1117,6 +1279,22 @@ cudaError_t get_memory_impl(rlt_model *M, int seq, int t_enc, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// One slot's rows 0..t_enc-1 of a head-major block [G][max_seqs][H][2][max_len][dh]
+// at arena offset `base` to the staging buffer ([G][t_enc][2][d]), or back.
+template <typename T>
+cudaError_t hm_copy_impl(rlt_model *M, size_t base, int G, int seq, int t_enc, bool out,
+                         cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  if (t_enc == 0 || G == 0) return cudaSuccess;
+  if (out)
+    k_get_memory<T><<<512, 256, 0, st>>>(G, c.n_heads, c.head_dim, c.max_seqs, c.max_len, seq,
+                                         t_enc, M->at<T>(base), M->at<T>(M->L.staging));
+  else
+    k_set_memory<T><<<512, 256, 0, st>>>(G, c.n_heads, c.head_dim, c.max_seqs, c.max_len, seq,
+                                         t_enc, M->at<T>(M->L.staging), M->at<T>(base));
+  return cudaGetLastError();
+}
+
 template <typename T, int DH> void bind(rlt_model *M) {
   if constexpr (std::is_same<T, bf16>::value) {
     M->step = step_impl_tc<DH>;
@@ -1130,6 +1308,9 @@ template <typename T, int DH> void bind(rlt_model *M) {
   M->get_window = get_window_impl<T>;
   M->set_window = set_window_impl<T>;
   M->get_memory = get_memory_impl<T>;
+  M->hm_copy = hm_copy_impl<T>;
+  M->append = append_impl<T, DH>;
+  M->lm_head = lm_head_impl<T>;
 }
 
 template <typename T> void bind_dh(rlt_model *M) {
@@ -1445,6 +1626,135 @@ size_t attend_workspace_internal(int n, int H, int dh, int cap) {
 
 }  // namespace rlt
 
+// ------------------------------------------------------------ snapshots
+namespace {
+
+// Every weight tensor the model reads, in a fixed order: (pointer, bytes).
+std::vector<std::pair<const void *, size_t>> weight_tensors(const rlt_model *M) {
+  const rlt_config &c = M->cfg;
+  const rlt_weights &w = M->w;
+  const size_t es = elem_size(&c), d = c.d, F = c.ffn_dim, V = c.vocab;
+  std::vector<std::pair<const void *, size_t>> t;
+  auto add = [&](const void *p, size_t b) {
+    if (p) t.emplace_back(p, b);
+  };
+  add(w.embed, V * d * es);
+  for (int l = 0; l < c.n_enc_layers; l++) {
+    add(w.enc_ln1[l], d * 4);
+    add(w.enc_wqkv[l], 3 * d * d * es);
+    add(w.enc_wo[l], d * d * es);
+    add(w.enc_ln2[l], d * 4);
+    add(w.enc_w1[l], F * d * es);
+    if (c.ffn_kind == RLT_SWIGLU) add(w.enc_wb[l], F * d * es);
+    add(w.enc_w2[l], d * F * es);
+  }
+  add(w.enc_lnf, d * 4);
+  for (int g = 0; g < c.mem_groups; g++) {
+    add(w.mem_wk[g], d * d * es);
+    add(w.mem_wv[g], d * d * es);
+  }
+  if (c.alpha != 0.0f) add(w.gate_w, 2 * d * d * es);
+  add(w.gate_b, d * 4);
+  add(w.sstar, d * 4);
+  for (int l = 0; l < c.n_dec_layers; l++) {
+    add(w.dec_ln1[l], d * 4);
+    add(w.dec_ln2[l], d * 4);
+    add(w.dec_ln3[l], d * 4);
+    add(w.dec_wqx[l], d * d * es);
+    add(w.dec_wox[l], d * d * es);
+    if (!c.tied) {
+      add(w.dec_wqkv[l], 3 * d * d * es);
+      add(w.dec_wo[l], d * d * es);
+      add(w.dec_w1[l], F * d * es);
+      if (c.ffn_kind == RLT_SWIGLU) add(w.dec_wb[l], F * d * es);
+      add(w.dec_w2[l], d * F * es);
+    }
+  }
+  add(w.dec_lnf, d * 4);
+  return t;
+}
+
+// Hash of the configuration fields a snapshot depends on.
+uint64_t config_hash(const rlt_config &c) {
+  const int32_t f[] = {c.d, c.n_heads, c.head_dim, c.n_enc_layers, c.n_dec_layers, c.ffn_dim,
+                       c.ffn_kind, c.vocab, c.window, c.mem_groups, c.tied, c.dtype,
+                       c.enc_cache};
+  uint64_t h = 0x5EEDull;
+  for (size_t i = 0; i < sizeof(f) / sizeof(f[0]); i++) h = mix64(h ^ (uint32_t)f[i]);
+  uint32_t fl[3];
+  std::memcpy(&fl[0], &c.alpha, 4);
+  std::memcpy(&fl[1], &c.rms_eps, 4);
+  std::memcpy(&fl[2], &c.rope_theta, 4);
+  for (uint32_t x : fl) h = mix64(h ^ x);
+  return h;
+}
+
+// Enqueue the fingerprint (configuration hash + weight sum) into the arena
+// word L.fp (on `st`).
+cudaError_t enqueue_fingerprint(rlt_model *M, cudaStream_t st) {
+  unsigned long long *acc = M->at<unsigned long long>(M->L.fp);
+  const unsigned long long start = config_hash(M->cfg);  // pageable: staged before return
+  RLT_TRY(cudaMemcpyAsync(acc, &start, 8, cudaMemcpyHostToDevice, st));
+  const auto tensors = weight_tensors(M);
+  for (size_t i = 0; i < tensors.size(); i++) {
+    const size_t words = tensors[i].second / 4;
+    const int blocks = (int)std::min<size_t>((words + 255) / 256, 4096);
+    k_fingerprint<<<blocks, 256, 0, st>>>(static_cast<const uint32_t *>(tensors[i].first), words,
+                                          mix64(i + 1), acc);
+    RLT_TRY(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Header of a snapshot at positions (t_dec, t_enc) (fingerprint left zero).
+rlt_snapshot_header snapshot_header(const rlt_model *M, int64_t t_dec, int64_t t_enc) {
+  const rlt_config &c = M->cfg;
+  const size_t es = elem_size(&c), d = c.d;
+  const size_t te = (size_t)t_enc;
+  rlt_snapshot_header h{};
+  h.magic = RLT_SNAPSHOT_MAGIC;
+  h.version = 1;
+  h.d = c.d;
+  h.n_heads = c.n_heads;
+  h.head_dim = c.head_dim;
+  h.n_enc_layers = c.n_enc_layers;
+  h.n_dec_layers = c.n_dec_layers;
+  h.ffn_dim = c.ffn_dim;
+  h.ffn_kind = c.ffn_kind;
+  h.vocab = c.vocab;
+  h.window = c.window;
+  h.mem_groups = c.mem_groups;
+  h.tied = c.tied;
+  h.dtype = c.dtype;
+  h.enc_cache = c.enc_cache;
+  h.alpha = c.alpha;
+  h.rms_eps = c.rms_eps;
+  h.rope_theta = c.rope_theta;
+  h.t_dec = t_dec;
+  h.t_enc = t_enc;
+  h.off_s = a256(sizeof(rlt_snapshot_header));
+  h.off_window = h.off_s + a256(d * 4);
+  h.off_e = h.off_window + a256((size_t)c.n_dec_layers * 2 * (c.window > 1 ? c.window - 1 : 0) *
+                                d * es);
+  h.off_mem = h.off_e + a256(te * d * es);
+  h.off_enc_kv = h.off_mem + a256((size_t)c.mem_groups * te * 2 * d * es);
+  h.bytes = h.off_enc_kv + a256(c.enc_cache ? (size_t)c.n_enc_layers * te * 2 * d * es : 0);
+  return h;
+}
+
+bool same_model(const rlt_snapshot_header &a, const rlt_snapshot_header &b) {
+  return a.d == b.d && a.n_heads == b.n_heads && a.head_dim == b.head_dim &&
+         a.n_enc_layers == b.n_enc_layers && a.n_dec_layers == b.n_dec_layers &&
+         a.ffn_dim == b.ffn_dim && a.ffn_kind == b.ffn_kind && a.vocab == b.vocab &&
+         a.window == b.window && a.mem_groups == b.mem_groups && a.tied == b.tied &&
+         a.dtype == b.dtype && a.enc_cache == b.enc_cache && a.alpha == b.alpha &&
+         a.rms_eps == b.rms_eps && a.rope_theta == b.rope_theta;
+}
+
+}  // namespace
+
 // ===================================================================== C ABI
 extern "C" {
 
@@ -1459,6 +1769,7 @@ RLT_API const char *rlt_status_string(int s) {
     case RLT_ERR_CUDA: return "CUDA runtime error";
     case RLT_ERR_TIMEOUT: return "bounded device wait timed out";
     case RLT_ERR_DEVICE: return "device-side check failed (bad token id)";
+    case RLT_ERR_STALE: return "snapshot of another configuration or other weight values";
     default: return "unknown status";
   }
 }
@@ -1774,6 +2085,135 @@ RLT_API int rlt_decoder_parallel(rlt_model *M, const int32_t *ids, int n, int n_
   return cuda_status(push_positions(M, st));
 }
 
+// ------------------------------------------------------------ serving loop
+namespace {
+
+// Ids valid and unique; n within the work buffers.
+int check_ids(const rlt_model *M, const int32_t *ids, int n) {
+  if (!M || n < 0 || (n > 0 && !ids)) return RLT_ERR_INVALID_ARG;
+  if (n > M->cfg.max_seqs || n > M->L.ptok) return RLT_ERR_CAPACITY;
+  std::vector<char> seen(M->cfg.max_seqs, 0);
+  for (int i = 0; i < n; i++) {
+    const int s = ids[i];
+    if (s < 0 || s >= M->cfg.max_seqs) return RLT_ERR_INVALID_ARG;
+    if (seen[s]) return RLT_ERR_DUPLICATE_ID;
+    seen[s] = 1;
+  }
+  return RLT_OK;
+}
+
+// Rows of the next launches: the ready list and its device row count.
+cudaError_t stage_rows(rlt_model *M, const int32_t *ids, int n, cudaStream_t st) {
+  const int nval[2] = {n, 0};
+  std::vector<int32_t> idv(ids, ids + n);  // pageable: staged before return
+  RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.ready), idv.data(), 4 * (size_t)n,
+                          cudaMemcpyHostToDevice, st));
+  return cudaMemcpyAsync(M->at<int>(M->L.nready), nval, sizeof(nval), cudaMemcpyHostToDevice, st);
+}
+
+// Append the tokens already in the arena's token buffer to the listed rows.
+cudaError_t enqueue_append(rlt_model *M, const int32_t *ids, int n, cudaStream_t st) {
+  std::vector<int32_t> pos(n);
+  int tmax = 0;
+  for (int i = 0; i < n; i++) {
+    pos[i] = M->t_enc[ids[i]];
+    tmax = std::max(tmax, pos[i]);
+  }
+  RLT_TRY(stage_rows(M, ids, n, st));
+  RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.pos), pos.data(), 4 * (size_t)n,
+                          cudaMemcpyHostToDevice, st));
+  RLT_TRY(M->append(M, n, tmax, st));
+  for (int i = 0; i < n; i++) M->t_enc[ids[i]] += 1;
+  return push_positions(M, st);
+}
+
+}  // namespace
+
+RLT_API int rlt_append_encoder(rlt_model *M, const int32_t *tokens, const int32_t *ids, int n,
+                               rlt_stream stream) {
+  int rc = check_ids(M, ids, n);
+  if (rc != RLT_OK) return rc;
+  if (!M->cfg.enc_cache) return RLT_ERR_UNSUPPORTED;
+  for (int i = 0; i < n; i++)
+    if (M->t_enc[ids[i]] >= M->cfg.max_len) return RLT_ERR_CAPACITY;
+  if (n == 0) return RLT_OK;
+  if (!tokens) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  cudaError_t e = cudaMemcpyAsync(M->at<int>(M->L.tok), tokens, 4 * (size_t)n, cudaMemcpyDefault,
+                                  st);
+  if (e == cudaSuccess) e = enqueue_append(M, ids, n, st);
+  return cuda_status(e);
+}
+
+RLT_API int rlt_lm_head(rlt_model *M, const int32_t *ids, int n, float *logits,
+                        rlt_stream stream) {
+  int rc = check_ids(M, ids, n);
+  if (rc != RLT_OK) return rc;
+  if (n == 0) return RLT_OK;
+  if (!logits) return RLT_ERR_INVALID_ARG;
+  if (M->cfg.dtype == RLT_BF16 && M->cfg.vocab % 64) return RLT_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  cudaError_t e = stage_rows(M, ids, n, st);
+  if (e == cudaSuccess) e = M->lm_head(M, n, logits, st);
+  return cuda_status(e);
+}
+
+RLT_API int rlt_sample(rlt_model *M, const float *logits, int n, float temperature,
+                       const float *uniforms, int32_t *tokens_out, rlt_stream stream) {
+  if (!M || n < 0 || !(temperature >= 0.0f) || !std::isfinite(temperature))
+    return RLT_ERR_INVALID_ARG;
+  if (n == 0) return RLT_OK;
+  if (!logits || !tokens_out || (temperature > 0.0f && !uniforms)) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  M->stats.launches++;
+  k_sample<<<n, SAMPLE_THREADS, 0, st>>>(M->cfg.vocab, logits, temperature, uniforms, tokens_out);
+  return cuda_status(cudaGetLastError());
+}
+
+RLT_API int rlt_serve_step(rlt_model *M, const int32_t *ids, int n, float temperature,
+                           const float *uniforms, float *logits, int32_t *tokens_out,
+                           rlt_stream stream) {
+  int rc = check_ids(M, ids, n);
+  if (rc != RLT_OK) return rc;
+  if (!M->cfg.enc_cache) return RLT_ERR_UNSUPPORTED;
+  if (!(temperature >= 0.0f) || !std::isfinite(temperature)) return RLT_ERR_INVALID_ARG;
+  if (M->cfg.dtype == RLT_BF16 && M->cfg.vocab % 64) return RLT_ERR_UNSUPPORTED;
+  for (int i = 0; i < n; i++) {
+    const int s = ids[i];
+    if (M->t_enc[s] >= M->cfg.max_len) return RLT_ERR_CAPACITY;
+    // the decoder must stand at the last known token: its s_t reads the next
+    if (M->t_dec[s] + 1 != M->t_enc[s]) return RLT_ERR_NOT_READY;
+  }
+  if (n == 0) return RLT_OK;
+  if (!logits || !tokens_out || (temperature > 0.0f && !uniforms)) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  // 1. the transition at t = t_enc - 1
+  std::vector<int32_t> idv(ids, ids + n);
+  cudaError_t e = cudaMemcpyAsync(M->at<int>(M->L.ready), idv.data(), 4 * (size_t)n,
+                                  cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = enqueue_step(M, step_info(M, ids, n), st);
+  if (e != cudaSuccess) return RLT_ERR_CUDA;
+  advance(M, ids, n);
+  // 2. logits from s_t, 3. the next token, 4. that token into the encoder
+  e = stage_rows(M, ids, n, st);
+  if (e == cudaSuccess) e = M->lm_head(M, n, logits, st);
+  if (e == cudaSuccess) {
+    M->stats.launches++;
+    k_sample<<<n, SAMPLE_THREADS, 0, st>>>(M->cfg.vocab, logits, temperature, uniforms,
+                                           tokens_out);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(M->at<int>(M->L.tok), tokens_out, 4 * (size_t)n, cudaMemcpyDeviceToDevice,
+                        st);
+  if (e == cudaSuccess) e = enqueue_append(M, ids, n, st);
+  return cuda_status(e);
+}
+
 RLT_API int rlt_plan_ragged(const int32_t *steps, int n, int32_t *order, int32_t *tick_sizes,
                             int max_ticks, int *n_ticks) {
   if (n < 0 || (n > 0 && (!steps || !order)) || !n_ticks) return RLT_ERR_INVALID_ARG;
@@ -1875,6 +2315,119 @@ RLT_API int rlt_set_state(rlt_model *M, int seq, const float *s_in, const void *
   }
   if (e != cudaSuccess) return RLT_ERR_CUDA;
   M->t_dec[seq] = (int)t;
+  return cuda_status(push_positions(M, st));
+}
+
+RLT_API size_t rlt_snapshot_bytes(rlt_model *M, int seq) {
+  if (!M || seq < 0 || seq >= M->cfg.max_seqs) return 0;
+  return snapshot_header(M, M->t_dec[seq], M->t_enc[seq]).bytes;
+}
+
+RLT_API int rlt_model_fingerprint(rlt_model *M, uint64_t *out) {
+  if (!M || !out) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = M->last_stream;
+  unsigned long long v = 0;
+  cudaError_t e = enqueue_fingerprint(M, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(&v, M->at<unsigned long long>(M->L.fp), 8, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return RLT_ERR_CUDA;
+  *out = v;
+  return RLT_OK;
+}
+
+RLT_API int rlt_get_snapshot(rlt_model *M, int seq, void *buf, size_t bytes, rlt_stream stream) {
+  if (!M || seq < 0 || seq >= M->cfg.max_seqs || !buf) return RLT_ERR_INVALID_ARG;
+  const rlt_config &c = M->cfg;
+  const rlt_snapshot_header h = snapshot_header(M, M->t_dec[seq], M->t_enc[seq]);
+  if (bytes < h.bytes) return RLT_ERR_CAPACITY;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  uint8_t *b = static_cast<uint8_t *>(buf);
+  const size_t es = elem_size(&c), d = c.d, te = (size_t)h.t_enc;
+  const Layout &L = M->L;
+  // every host source below is pageable: staged before its call returns
+  cudaError_t e = cudaMemcpyAsync(b, &h, sizeof(h), cudaMemcpyDefault, st);
+  if (e == cudaSuccess) e = enqueue_fingerprint(M, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(b + offsetof(rlt_snapshot_header, fingerprint), M->at<uint8_t>(L.fp), 8,
+                        cudaMemcpyDefault, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(b + h.off_s, M->at<float>(L.s) + (size_t)seq * d, d * 4,
+                        cudaMemcpyDefault, st);
+  if (e == cudaSuccess && c.window > 1) {
+    e = M->get_window(M, seq, (long)h.t_dec, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(b + h.off_window, M->at<uint8_t>(L.staging),
+                          (size_t)c.n_dec_layers * 2 * (c.window - 1) * d * es, cudaMemcpyDefault,
+                          st);
+  }
+  if (e == cudaSuccess && te > 0) {
+    e = cudaMemcpyAsync(b + h.off_e, M->at<uint8_t>(L.e) + (size_t)seq * c.max_len * d * es,
+                        te * d * es, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = M->hm_copy(M, L.mem, c.mem_groups, seq, (int)te, true, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(b + h.off_mem, M->at<uint8_t>(L.staging),
+                          (size_t)c.mem_groups * te * 2 * d * es, cudaMemcpyDefault, st);
+    if (e == cudaSuccess && c.enc_cache) {
+      e = M->hm_copy(M, L.enc_kv, c.n_enc_layers, seq, (int)te, true, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(b + h.off_enc_kv, M->at<uint8_t>(L.staging),
+                            (size_t)c.n_enc_layers * te * 2 * d * es, cudaMemcpyDefault, st);
+    }
+  }
+  return cuda_status(e);
+}
+
+RLT_API int rlt_set_snapshot(rlt_model *M, int seq, const void *buf, size_t bytes,
+                             rlt_stream stream) {
+  if (!M || seq < 0 || seq >= M->cfg.max_seqs || !buf) return RLT_ERR_INVALID_ARG;
+  if (bytes < sizeof(rlt_snapshot_header)) return RLT_ERR_INVALID_ARG;
+  const rlt_config &c = M->cfg;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  const uint8_t *b = static_cast<const uint8_t *>(buf);
+  rlt_snapshot_header h{};
+  if (cudaMemcpyAsync(&h, b, sizeof(h), cudaMemcpyDefault, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return RLT_ERR_CUDA;
+  if (h.magic != RLT_SNAPSHOT_MAGIC || h.version != 1) return RLT_ERR_INVALID_ARG;
+  if (!same_model(h, snapshot_header(M, 0, 0))) return RLT_ERR_STALE;
+  if (h.t_enc < 0 || h.t_dec < 0 || h.t_dec > h.t_enc) return RLT_ERR_INVALID_ARG;
+  if (h.t_enc > c.max_len) return RLT_ERR_CAPACITY;
+  const rlt_snapshot_header want = snapshot_header(M, h.t_dec, h.t_enc);
+  if (h.bytes != want.bytes || h.off_s != want.off_s || h.off_window != want.off_window ||
+      h.off_e != want.off_e || h.off_mem != want.off_mem || h.off_enc_kv != want.off_enc_kv ||
+      bytes < h.bytes)
+    return RLT_ERR_INVALID_ARG;
+  uint64_t fp = 0;
+  if (rlt_model_fingerprint(M, &fp) != RLT_OK) return RLT_ERR_CUDA;
+  if (fp != h.fingerprint) return RLT_ERR_STALE;
+  const Layout &L = M->L;
+  const size_t es = elem_size(&c), d = c.d, te = (size_t)h.t_enc;
+  cudaError_t e = cudaMemcpyAsync(M->at<float>(L.s) + (size_t)seq * d, b + h.off_s, d * 4,
+                                  cudaMemcpyDefault, st);
+  if (e == cudaSuccess && c.window > 1) {
+    e = cudaMemcpyAsync(M->at<uint8_t>(L.staging), b + h.off_window,
+                        (size_t)c.n_dec_layers * 2 * (c.window - 1) * d * es, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = M->set_window(M, seq, (long)h.t_dec, st);
+  }
+  if (e == cudaSuccess && te > 0) {
+    e = cudaMemcpyAsync(M->at<uint8_t>(L.e) + (size_t)seq * c.max_len * d * es, b + h.off_e,
+                        te * d * es, cudaMemcpyDefault, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(M->at<uint8_t>(L.staging), b + h.off_mem,
+                          (size_t)c.mem_groups * te * 2 * d * es, cudaMemcpyDefault, st);
+    if (e == cudaSuccess) e = M->hm_copy(M, L.mem, c.mem_groups, seq, (int)te, false, st);
+    if (e == cudaSuccess && c.enc_cache) {
+      e = cudaMemcpyAsync(M->at<uint8_t>(L.staging), b + h.off_enc_kv,
+                          (size_t)c.n_enc_layers * te * 2 * d * es, cudaMemcpyDefault, st);
+      if (e == cudaSuccess) e = M->hm_copy(M, L.enc_kv, c.n_enc_layers, seq, (int)te, false, st);
+    }
+  }
+  if (e != cudaSuccess) return RLT_ERR_CUDA;
+  M->t_dec[seq] = (int)h.t_dec;
+  M->t_enc[seq] = (int)h.t_enc;
   return cuda_status(push_positions(M, st));
 }
 

@@ -23,7 +23,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "rlt.h")
 RLT_OK = 0
 STATUS = {0: "RLT_OK", 1: "RLT_ERR_INVALID_ARG", 2: "RLT_ERR_UNSUPPORTED",
           3: "RLT_ERR_NOT_READY", 4: "RLT_ERR_CAPACITY", 5: "RLT_ERR_DUPLICATE_ID",
-          6: "RLT_ERR_CUDA", 7: "RLT_ERR_TIMEOUT", 8: "RLT_ERR_DEVICE"}
+          6: "RLT_ERR_CUDA", 7: "RLT_ERR_TIMEOUT", 8: "RLT_ERR_DEVICE", 9: "RLT_ERR_STALE"}
 
 
 class RLTError(RuntimeError):
@@ -37,7 +37,7 @@ class rlt_config(C.Structure):
     _fields_ = [(n, C.c_int) for n in (
         "d", "n_heads", "head_dim", "n_enc_layers", "n_dec_layers", "ffn_dim",
         "ffn_kind", "vocab", "window", "mem_groups", "tied", "dtype", "max_seqs",
-        "max_len", "max_prefill_tokens")] + [
+        "max_len", "max_prefill_tokens", "enc_cache")] + [
         ("alpha", C.c_float), ("rms_eps", C.c_float), ("rope_theta", C.c_float)]
 
 
@@ -91,6 +91,15 @@ def _declare(lib):
     lib.rlt_get_encoder_output.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
     lib.rlt_poll_device_error.argtypes = [P]
     lib.rlt_set_fault.argtypes = [P, I, C.c_int64]
+    lib.rlt_append_encoder.argtypes = [P, P, P, I, P]
+    lib.rlt_lm_head.argtypes = [P, P, I, P, P]
+    lib.rlt_sample.argtypes = [P, P, I, C.c_float, P, P, P]
+    lib.rlt_serve_step.argtypes = [P, P, I, C.c_float, P, P, P, P]
+    lib.rlt_snapshot_bytes.argtypes = [P, I]
+    lib.rlt_snapshot_bytes.restype = C.c_size_t
+    lib.rlt_get_snapshot.argtypes = [P, I, P, C.c_size_t, P]
+    lib.rlt_set_snapshot.argtypes = [P, I, P, C.c_size_t, P]
+    lib.rlt_model_fingerprint.argtypes = [P, C.POINTER(C.c_uint64)]
     lib.rlt_set_step_kernel.argtypes = [P, I]
     lib.rlt_get_step_kernel.argtypes = [P]
     lib.rlt_step_kernel_ctas.argtypes = [P]
@@ -135,11 +144,12 @@ def _p(a: np.ndarray):
     return a.ctypes.data_as(C.c_void_p)
 
 
-def make_config(cfg: RLTConfig, max_seqs: int, max_len: int, max_prefill_tokens: int = 0):
+def make_config(cfg: RLTConfig, max_seqs: int, max_len: int, max_prefill_tokens: int = 0,
+                enc_cache: bool = False):
     return rlt_config(cfg.d, cfg.n_heads, cfg.head_dim, cfg.n_enc, cfg.n_dec, cfg.ffn_dim,
                       cfg.ffn_kind, cfg.vocab, cfg.window, cfg.mem_groups, int(cfg.tied),
-                      cfg.dtype, max_seqs, max_len, max_prefill_tokens, float(cfg.alpha),
-                      float(cfg.rms_eps), float(cfg.rope_theta))
+                      cfg.dtype, max_seqs, max_len, max_prefill_tokens, int(enc_cache),
+                      float(cfg.alpha), float(cfg.rms_eps), float(cfg.rope_theta))
 
 
 def check_config(cfg: RLTConfig, max_seqs: int, max_len: int) -> int:
@@ -147,8 +157,9 @@ def check_config(cfg: RLTConfig, max_seqs: int, max_len: int) -> int:
     return _lib().rlt_check_config(C.byref(c))
 
 
-def arena_bytes(cfg: RLTConfig, max_seqs: int, max_len: int, max_prefill_tokens: int = 0) -> int:
-    c = make_config(cfg, max_seqs, max_len, max_prefill_tokens)
+def arena_bytes(cfg: RLTConfig, max_seqs: int, max_len: int, max_prefill_tokens: int = 0,
+                enc_cache: bool = False) -> int:
+    c = make_config(cfg, max_seqs, max_len, max_prefill_tokens, enc_cache)
     return int(_lib().rlt_arena_bytes(C.byref(c)))
 
 
@@ -198,7 +209,7 @@ class Model:
 
     def __init__(self, cfg: RLTConfig, weights: Dict[str, np.ndarray], max_seqs: int,
                  max_len: int, device: str = "cuda", max_prefill_tokens: int = 0,
-                 stream=None):
+                 stream=None, enc_cache: bool = False):
         import torch
         self.torch = torch
         self.cfg = cfg
@@ -207,7 +218,8 @@ class Model:
         self.wdtype = torch.bfloat16 if cfg.dtype == BF16 else torch.float32
         self.stream = stream
         lib = _lib()
-        self._c = make_config(cfg, max_seqs, max_len, max_prefill_tokens)
+        self._c = make_config(cfg, max_seqs, max_len, max_prefill_tokens, enc_cache)
+        self.enc_cache = bool(enc_cache)
         rc = lib.rlt_check_config(C.byref(self._c))
         _check(rc, "rlt_check_config")
         self.arena_bytes = int(lib.rlt_arena_bytes(C.byref(self._c)))
@@ -357,6 +369,74 @@ class Model:
                                                  C.c_void_p(mem.data_ptr()), C.byref(t),
                                                  self._st(stream)), "rlt_get_encoder_output")
         return e, mem
+
+    # -- serving loop ---------------------------------------------------
+    def append_encoder(self, tokens, seq_ids, stream=None):
+        """tokens: int32 tensor [n] (device or pinned host), one per id."""
+        ids = _i32(seq_ids)
+        self._tok_keep = tokens
+        _check(_lib().rlt_append_encoder(self._h, C.c_void_p(tokens.data_ptr()), _p(ids),
+                                         ids.shape[0], self._st(stream)), "rlt_append_encoder")
+
+    def lm_head(self, seq_ids, logits=None, stream=None):
+        """Logits [n][V] (fp32 device tensor) from each sequence's s_t."""
+        ids = _i32(seq_ids)
+        if logits is None:
+            logits = self.torch.empty((ids.shape[0], self.cfg.vocab), dtype=self.torch.float32,
+                                      device=self.device)
+        _check(_lib().rlt_lm_head(self._h, _p(ids), ids.shape[0],
+                                  C.c_void_p(logits.data_ptr()), self._st(stream)), "rlt_lm_head")
+        return logits
+
+    def sample(self, logits, temperature: float, uniforms=None, out=None, stream=None):
+        n = logits.shape[0]
+        if out is None:
+            out = self.torch.empty(n, dtype=self.torch.int32, device=self.device)
+        up = C.c_void_p(uniforms.data_ptr()) if uniforms is not None else None
+        _check(_lib().rlt_sample(self._h, C.c_void_p(logits.data_ptr()), n, float(temperature),
+                                 up, C.c_void_p(out.data_ptr()), self._st(stream)), "rlt_sample")
+        return out
+
+    def serve_step(self, seq_ids, temperature: float, uniforms=None, logits=None, out=None,
+                   stream=None):
+        """One autoregressive step; returns (tokens int32 [n], logits [n][V])."""
+        ids = _i32(seq_ids)
+        n = ids.shape[0]
+        torch = self.torch
+        if logits is None:
+            logits = torch.empty((n, self.cfg.vocab), dtype=torch.float32, device=self.device)
+        if out is None:
+            out = torch.empty(n, dtype=torch.int32, device=self.device)
+        self._serve_keep = (uniforms, logits, out)
+        up = C.c_void_p(uniforms.data_ptr()) if uniforms is not None else None
+        _check(_lib().rlt_serve_step(self._h, _p(ids), n, float(temperature), up,
+                                     C.c_void_p(logits.data_ptr()), C.c_void_p(out.data_ptr()),
+                                     self._st(stream)), "rlt_serve_step")
+        return out, logits
+
+    # -- exact prefix snapshots ------------------------------------------
+    def snapshot_bytes(self, seq: int) -> int:
+        return int(_lib().rlt_snapshot_bytes(self._h, seq))
+
+    def get_snapshot(self, seq: int, out=None, stream=None):
+        """Slot `seq`'s snapshot into `out` (uint8 tensor on the device or in
+        pinned host memory; allocated on the device if None); returns it."""
+        n = self.snapshot_bytes(seq)
+        if out is None:
+            out = self.torch.empty(n, dtype=self.torch.uint8, device=self.device)
+        _check(_lib().rlt_get_snapshot(self._h, seq, C.c_void_p(out.data_ptr()), out.numel(),
+                                       self._st(stream)), "rlt_get_snapshot")
+        return out
+
+    def set_snapshot(self, seq: int, buf, stream=None):
+        self._snap_keep = buf
+        _check(_lib().rlt_set_snapshot(self._h, seq, C.c_void_p(buf.data_ptr()), buf.numel(),
+                                       self._st(stream)), "rlt_set_snapshot")
+
+    def fingerprint(self) -> int:
+        v = C.c_uint64(0)
+        _check(_lib().rlt_model_fingerprint(self._h, C.byref(v)), "rlt_model_fingerprint")
+        return int(v.value)
 
     def profile(self, stride: int):
         """stride k > 0: profile every k-th decoder step (and every prefill); 0: off."""
