@@ -506,4 +506,224 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
   if (warp == 1) tmem_dealloc(tmem, BN);
 }
 
+// ------------------------------------------------------------- swapped operands
+// The same decode GEMM for small batches (at most 64 rows): the weights are
+// the 128-row MMA operand and the batch rows the N side (BR = 32 or 64), so
+// a ring stage carries a 128-feature weight slab and only BR activation
+// rows instead of 128 rows of which most are padding. CTA (x, y, z) of a
+// cluster of S computes features [128 x, 128 x + 128) for rows [BR y, BR y +
+// BR) over its K share; the accumulator (TMEM lanes = features, columns =
+// rows) is written to shared memory transposed, [row][feature], and from
+// there the split-K reduction in rank order and the epilogue functors run
+// exactly as in k_gemm_dec with 128-column tiles. A 128-column tile covers
+// four of the 32-column slots of the norm partial sums: the epilogue writes
+// the row's sum over the tile into the first and zero into the other three.
+template <int BR> struct DecSwSmem {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;  // weights, 128 features x 64 K
+  static constexpr int B_BYTES = BR * TC_BK * 2;     // activations, BR rows x 64 K
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int P_LD = TC_BM + 4;             // [row][feature] partial tile
+  static constexpr int P_BYTES = BR * P_LD * 4;
+  static constexpr int bytes(int ns) {
+    return 1024 + DEC_BAR_BYTES + (ns * STAGE > P_BYTES ? ns * STAGE : P_BYTES);
+  }
+};
+
+template <int BR, int STAGES, int S, class Epi>
+__global__ void __launch_bounds__(DEC_THREADS, 2)
+    k_gemm_dec_sw(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                  const int *__restrict__ Mdev, int a_row0, int N, int K, int ns, Epi epi,
+                  int *err) {
+  static_assert(BR == 32 || BR == 64, "TMEM columns are a power of two >= 32");
+  static_assert(S >= 1 && S <= 8, "portable cluster size");
+  using SM = DecSwSmem<BR>;
+  constexpr int BNE = TC_BM;  // output columns of a tile
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(base);
+  uint64_t *empty = full + STAGES;
+  uint64_t *accum = empty + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+  uint8_t *tiles = base + DEC_BAR_BYTES;
+  float *P = reinterpret_cast<float *>(tiles);
+  __shared__ float s_rs[BR];
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BR, n0 = blockIdx.x * BNE;
+  const int M = *Mdev;
+  if (m0 >= M) return;  // the whole cluster (same blockIdx.y), before any barrier
+  const int z = (int)cluster_ctarank();
+  const int kb_all = K / TC_BK;
+  const int kb0 = z * kb_all / S, KB = (z + 1) * kb_all / S - kb0;
+  const int rv = M - m0 < BR ? M - m0 : BR;
+  const int share = (rv + S - 1) / S;
+  const int r_lo = z * share < rv ? z * share : rv;
+  const int r_hi = r_lo + share < rv ? r_lo + share : rv;
+
+  if (threadIdx.x == 0) {
+    s_fail = 0;
+    for (int s = 0; s < ns; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, BR);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  pdl_trigger();
+  if (warp == 0 && lane == 0) {
+    // weight slabs of the first stages stream before the dependency wait
+    const int pre = KB < ns ? KB : ns;
+    for (int kb = 0; kb < pre; kb++) {
+      mbar_expect_tx(&full[kb], SM::STAGE);
+      tma_load_2d(tiles + kb * SM::STAGE, &tmW, (kb0 + kb) * TC_BK, n0, &full[kb]);
+    }
+    pdl_wait();
+    for (int kb = 0; kb < pre; kb++)
+      tma_load_2d(tiles + kb * SM::STAGE + SM::A_BYTES, &tmX, (kb0 + kb) * TC_BK, a_row0 + m0,
+                  &full[kb]);
+    for (int kb = pre; kb < KB; kb++) {
+      const int s = kb % ns, u = kb / ns;
+      if (!mbar_wait_bounded(&empty[s], (u - 1) & 1, WAIT_LIMIT_NS_TC)) {
+        atomicExch(&s_fail, 1);
+        break;
+      }
+      uint8_t *a = tiles + s * SM::STAGE;
+      mbar_expect_tx(&full[s], SM::STAGE);
+      tma_load_2d(a, &tmW, (kb0 + kb) * TC_BK, n0, &full[s]);
+      tma_load_2d(a + SM::A_BYTES, &tmX, (kb0 + kb) * TC_BK, a_row0 + m0, &full[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BR);
+    for (int kb = 0; kb < KB; kb++) {
+      const int s = kb % ns, u = kb / ns;
+      if (!mbar_wait_bounded(&full[s], u & 1, WAIT_LIMIT_NS_TC)) {
+        atomicExch(&s_fail, 1);
+        break;
+      }
+      tc_fence_after();
+      const uint8_t *a = tiles + s * SM::STAGE;
+      const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + SM::A_BYTES);
+#pragma unroll
+      for (int k = 0; k < TC_BK / 16; k++)
+        umma_bf16(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc,
+                  (kb > 0 || k > 0) ? 1u : 0u);
+      umma_commit(&empty[s]);
+    }
+    umma_commit(accum);
+  } else if (Epi::kRowScale && warp >= 2) {
+    pdl_wait();
+    for (int i = threadIdx.x - 64; i < r_hi - r_lo; i += DEC_THREADS - 64) {
+      const float *p = epi.rsi.nsq + (size_t)(m0 + r_lo + i) * epi.rsi.np;
+      float ss = 0.f;
+      for (int t = 0; t < epi.rsi.np; t++) ss += p[t];
+      s_rs[i] = rsqrtf(ss * epi.rsi.inv_d + epi.rsi.eps);
+    }
+  }
+  __syncwarp();
+  pdl_wait();
+
+  // accumulator -> shared memory, transposed: warp w reads TMEM lanes
+  // (features) 32 (w mod 4) .. + 31 and the rows of column half w / 4
+  const bool acc_ok = mbar_wait_bounded(accum, 0, WAIT_LIMIT_NS_TC);
+  tc_fence_after();
+  if (!acc_ok) atomicExch(&s_fail, 1);
+  __syncthreads();
+  const bool ok = !s_fail;
+  const int lg = warp & 3, chh = warp >> 2;
+  if (ok) {
+    const int f = lg * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(lg * 32) << 16);
+#pragma unroll
+    for (int c0 = chh * (BR / 2); c0 < (chh + 1) * (BR / 2); c0 += 16) {
+      float v[16];
+      if (KB > 0) {
+        tmem_ld16(lane_base + c0, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; j++) v[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; j++) P[(size_t)(c0 + j) * SM::P_LD + f] = v[j];
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();
+
+  if (!ok) {
+    if (threadIdx.x == 0) set_error(err, DEV_ERR_TIMEOUT);
+  } else {
+    const uint32_t p_local = smem_u32(P);
+    uint32_t p_rank[S];
+#pragma unroll
+    for (int q = 0; q < S; q++) p_rank[q] = mapa_shared(p_local, q);
+    auto sum4 = [&](int r, int c) {
+      const uint32_t off = (uint32_t)((r * SM::P_LD + c) * 4);
+      float4 v[S];
+#pragma unroll
+      for (int q = 0; q < S; q++) v[q] = ld_dsmem_f4(p_rank[q] + off);
+      float4 acc = v[0];
+#pragma unroll
+      for (int q = 1; q < S; q++) {
+        acc.x += v[q].x;
+        acc.y += v[q].y;
+        acc.z += v[q].z;
+        acc.w += v[q].w;
+      }
+      return acc;
+    };
+    const int rows = r_hi - r_lo;
+    if constexpr (Epi::kKind == kRope) {
+      const int DH = epi.DH, half = DH / 2;
+      constexpr int PPR = BNE / 8;
+      for (int idx = threadIdx.x; idx < rows * PPR; idx += DEC_THREADS) {
+        const int rl = idx / PPR, p = idx - rl * PPR;
+        const int hh = (4 * p) / half, j = 4 * p - hh * half;
+        const int c = hh * DH + j, r = r_lo + rl;
+        const float4 a = sum4(r, c), b = sum4(r, c + half);
+        const float sc = Epi::kRowScale ? s_rs[rl] : 1.f;
+        epi.rotary(m0 + r, n0 + c, a.x, a.y, b.x, b.y, sc);
+        epi.rotary(m0 + r, n0 + c + 2, a.z, a.w, b.z, b.w, sc);
+      }
+    } else {
+      constexpr int PPR = BNE / 4;  // 32: one warp per row
+      const int total = rows * PPR;
+      for (int b0 = 0; b0 < total; b0 += DEC_THREADS) {
+        const int idx = b0 + threadIdx.x;
+        const bool act = idx < total;
+        const int rl = act ? idx / PPR : 0, p = idx - (idx / PPR) * PPR;
+        float ss = 0.f;
+        if (act) {
+          const float4 v = sum4(r_lo + rl, 4 * p);
+          const float sc = Epi::kRowScale ? s_rs[rl] : 1.f;
+          const int m = m0 + r_lo + rl, n = n0 + 4 * p;
+          if constexpr (Epi::kKind == kNorm) {
+            ss = epi.pair(m, n, v.x, v.y, sc) + epi.pair(m, n + 2, v.z, v.w, sc);
+          } else {
+            epi.pair(m, n, v.x, v.y, sc);
+            epi.pair(m, n + 2, v.z, v.w, sc);
+          }
+        }
+        if constexpr (Epi::kKind == kNorm) {
+#pragma unroll
+          for (int o = PPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          // the tile covers four 32-column slots of the row's norm partials
+          if (act && p < 4) epi.row_sum(m0 + r_lo + rl, 4 * blockIdx.x + p, p == 0 ? ss : 0.f);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync_relaxed();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, BR);
+}
+
 }  // namespace rlt

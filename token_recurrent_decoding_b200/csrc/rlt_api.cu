@@ -193,6 +193,7 @@ struct rlt_model {
   uint8_t *arena = nullptr;
   int device = 0;
   int num_sms = 148;  // SMs of the device (decode GEMM split counts)
+  int swap_br = 0;    // decode GEMMs with swapped operands: batch rows per tile (0 = off)
   std::vector<int> t_dec, t_enc;
   cudaStream_t last_stream = nullptr;
   template <typename X> X *at(size_t off) const { return reinterpret_cast<X *>(arena + off); }
@@ -376,13 +377,72 @@ cudaError_t launch_dec_s(rlt_model *M, int m_grid, const int *Mdev, int a_row0, 
                             M->at<int>(M->L.err));
 }
 
+// One swapped-operand decode GEMM launch (k_gemm_dec_sw) with cluster size S.
+template <int BR, int S, class Epi>
+cudaError_t launch_dec_sw_s(rlt_model *M, int m_grid, const int *Mdev, int a_row0, int n, int k,
+                            const CUtensorMap &mw, const CUtensorMap &mx, Epi epi,
+                            cudaStream_t st) {
+  constexpr int STAGES = 4;
+  const int kb = k / TC_BK;
+  const int kb_max = (kb + S - 1) / S;
+  const int ns = kb_max < STAGES ? kb_max : STAGES;
+  auto kern = k_gemm_dec_sw<BR, STAGES, S, Epi>;
+  RLT_TRY(ensure_smem_limit(kern, DecSwSmem<BR>::bytes(STAGES)));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(n / TC_BM, (m_grid + BR - 1) / BR, S);
+  cfg.blockDim = dim3(DEC_THREADS);
+  cfg.dynamicSmemBytes = DecSwSmem<BR>::bytes(ns);
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = S;
+  int na = 1;
+  if (st != nullptr) {
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    na = 2;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, mw, mx, Mdev, a_row0, n, k, ns, epi,
+                            M->at<int>(M->L.err));
+}
+
+// Decode GEMM with the weights as the 128-row MMA operand and BR batch rows
+// as N (models of at most 64 slots); N a multiple of 128.
+template <int BR, class Epi>
+cudaError_t launch_dec_sw(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0,
+                          int n, int k, const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
+  const CUtensorMap *mw = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, TC_BM);
+  const CUtensorMap *mx = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, BR);
+  if (!mw || !mx) return cudaErrorInvalidValue;
+  switch (dec_splits(n / TC_BM, k / TC_BK, M->num_sms)) {
+    case 1: return launch_dec_sw_s<BR, 1>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
+    case 2: return launch_dec_sw_s<BR, 2>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
+    case 3: return launch_dec_sw_s<BR, 3>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
+    case 4: return launch_dec_sw_s<BR, 4>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
+    case 6: return launch_dec_sw_s<BR, 6>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
+    default: return launch_dec_sw_s<BR, 8>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
+  }
+}
+
 // Decode-step GEMM (gemm_dec.cuh): rows [a_row0 + m, ...) of A [a_rows][k]
 // times B [n][k] with BN-wide output tiles and a cluster of S split-K CTAs
 // per tile; m_grid bounds the rows, Mdev holds the row count at run time.
+// Models of at most 64 slots take the swapped-operand form (weights on the
+// 128-row side) for every GEMM whose N is a multiple of 128: a choice fixed
+// per model, so a row's result never depends on the batch around it.
 template <int BN, class Epi>
 cudaError_t launch_dec(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
                        int k, const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
   if (m_grid <= 0) return cudaSuccess;
+  if (M->swap_br && n % TC_BM == 0 && k % TC_BK == 0) {
+    if (M->swap_br == 32)
+      return launch_dec_sw<32>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, st);
+    return launch_dec_sw<64>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, st);
+  }
   if (n % BN || k % TC_BK) return cudaErrorInvalidValue;
   const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
   const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
@@ -1833,6 +1893,7 @@ RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *w, void *d_aren
   M->device = pa.device;
   M->t_dec.assign(cfg->max_seqs, 0);
   M->t_enc.assign(cfg->max_seqs, 0);
+  if (cfg->dtype == RLT_BF16 && cfg->max_seqs <= 64) M->swap_br = cfg->max_seqs <= 32 ? 32 : 64;
   if (cfg->dtype == RLT_BF16) bind_dh<bf16>(M); else bind_dh<float>(M);
   cudaError_t e = cudaSetDevice(M->device);
   if (e == cudaSuccess)
