@@ -432,13 +432,15 @@ cudaError_t launch_dec_sw(rlt_model *M, int m_grid, const int *Mdev, int a_rows,
 // times B [n][k] with BN-wide output tiles and a cluster of S split-K CTAs
 // per tile; m_grid bounds the rows, Mdev holds the row count at run time.
 // Models of at most 64 slots take the swapped-operand form (weights on the
-// 128-row side) for every GEMM whose N is a multiple of 128: a choice fixed
-// per model, so a row's result never depends on the batch around it.
+// 128-row side) for every GEMM whose N is a multiple of 128 with at least
+// 12 feature tiles (narrower GEMMs would occupy too few SMs even at eight
+// splits): a choice fixed by the model and the GEMM shape, so a row's result
+// never depends on the batch around it.
 template <int BN, class Epi>
 cudaError_t launch_dec(rlt_model *M, int m_grid, const int *Mdev, int a_rows, int a_row0, int n,
                        int k, const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
   if (m_grid <= 0) return cudaSuccess;
-  if (M->swap_br && n % TC_BM == 0 && k % TC_BK == 0) {
+  if (M->swap_br && n % TC_BM == 0 && n / TC_BM >= 12 && k % TC_BK == 0) {
     if (M->swap_br == 32)
       return launch_dec_sw<32>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, st);
     return launch_dec_sw<64>(M, m_grid, Mdev, a_rows, a_row0, n, k, A, B, epi, st);
