@@ -79,8 +79,7 @@ typedef struct rlt_config {
   int ffn_dim;      /* F */
   int ffn_kind;     /* RLT_GELU: W2 GELU(W1 u); RLT_SWIGLU: W2 (SiLU(Wa u) * Wb u) */
   int vocab;        /* V */
-  int window;       /* W >= 1; at most one split of the decoder attention:
-                       256 positions when max_seqs * n_heads < 2048, else 1024 */
+  int window;       /* W >= 1, at most RLT_ATTEND_CHUNK (1024) */
   int mem_groups;   /* G: 1 or n_dec_layers */
   int tied;         /* 1: decoder layer l uses encoder layer l's q/k/v, o and
                        FFN matrices ([RLT-96] "Architecture", tied config) */
@@ -373,9 +372,9 @@ RLT_API int rlt_get_encoder_output(rlt_model *model, int seq, void *e_out,
                                    rlt_stream stream);
 
 /* Memory positions per split of rlt_attend (and of the decoder's
- * cross-attention for models with max_seqs * n_heads >= 2048; 256 below):
- * rows longer than this are split into chunks of this many positions and
- * merged in chunk order. */
+ * cross-attention for models with max_seqs * n_heads >= 2048; 256 below
+ * that, 128 below 1024): rows longer than this are split into chunks of
+ * this many positions and merged in chunk order. */
 #define RLT_ATTEND_CHUNK 1024
 
 /* Bytes of device workspace rlt_attend needs (0 if the shape is invalid). */
@@ -397,8 +396,8 @@ RLT_API size_t rlt_attend_workspace_bytes(int n, int n_heads, int head_dim, int 
  *           int32 is a device error word (0 = ok, RLT_ERR_TIMEOUT if a
  *           bounded wait gave up). Calls sharing a workspace must not overlap.
  * Rows are split into chunks of RLT_ATTEND_CHUNK (1024) positions (the
- * decoder's own cross-attention uses 256-position chunks for models with
- * max_seqs * n_heads < 2048, so that few long rows still occupy every SM), each
+ * decoder's own cross-attention uses shorter chunks for models with few
+ * (slot, head) pairs, so that few long rows still occupy every SM), each
  * chunk attended by one warp; the chunks of a row are merged in chunk order,
  * so a row's result does not depend on the other rows or on timing.
  * The call copies the per-row positions from pageable host memory on

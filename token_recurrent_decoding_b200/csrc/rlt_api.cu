@@ -39,7 +39,8 @@ constexpr int XCH = RLT_ATTEND_CHUNK;  // memory positions per split of rlt_atte
 // on its own rows). A function of the configuration only, so a row's result
 // depends on its own t and never on the batch around it.
 int xattn_chunk(const rlt_config *c) {
-  return (long)c->max_seqs * c->n_heads < 2048 ? 256 : XCH;
+  const long pairs = (long)c->max_seqs * c->n_heads;
+  return pairs < 1024 ? 128 : pairs < 2048 ? 256 : XCH;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -74,7 +75,7 @@ int check_config(const rlt_config *c) {
   if (c->ffn_dim <= 0 || c->vocab <= 0 || c->window < 1 || c->max_seqs < 1 || c->max_len < 1)
     return RLT_ERR_INVALID_ARG;
   // the sliding window is attended as one chunk of the decode attention
-  if (c->window > xattn_chunk(c)) return RLT_ERR_UNSUPPORTED;
+  if (c->window > XCH) return RLT_ERR_UNSUPPORTED;
   if (c->ffn_kind != RLT_GELU && c->ffn_kind != RLT_SWIGLU) return RLT_ERR_INVALID_ARG;
   if (c->dtype != RLT_F32 && c->dtype != RLT_BF16) return RLT_ERR_INVALID_ARG;
   if (c->mem_groups != 1 && c->mem_groups != c->n_dec_layers) return RLT_ERR_UNSUPPORTED;
@@ -418,7 +419,10 @@ cudaError_t launch_dec_sw(rlt_model *M, int m_grid, const int *Mdev, int a_rows,
   const CUtensorMap *mw = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, TC_BM);
   const CUtensorMap *mx = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, BR);
   if (!mw || !mx) return cudaErrorInvalidValue;
-  switch (dec_splits(n / TC_BM, k / TC_BK, M->num_sms)) {
+#ifndef RLT_DEC_SW_CTAS_PER_SM
+#define RLT_DEC_SW_CTAS_PER_SM 1  // CTAs per SM the swapped split count aims for
+#endif
+  switch (dec_splits(n / TC_BM, k / TC_BK, RLT_DEC_SW_CTAS_PER_SM * M->num_sms)) {
     case 1: return launch_dec_sw_s<BR, 1>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
     case 2: return launch_dec_sw_s<BR, 2>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
     case 3: return launch_dec_sw_s<BR, 3>(M, m_grid, Mdev, a_row0, n, k, *mw, *mx, epi, st);
@@ -567,7 +571,9 @@ cudaError_t launch_attn(rlt_model *M, const StepInfo &si, int window, int xchunk
   const int units = si.n_grid * c.n_heads * xchunks;
   const int grid = attn_balanced_ctas<T, DH>(units);  // also sets the smem limit
   return launch_k(k_attn_decode<T, DH>, dim3(grid), dim3((AttnCfg::NC + 1) * 32), smem, st,
-                  M->at<int>(L.nready) + si.chain, c.n_heads, window, L.xch, xchunks, L.max_chunks,
+                  M->at<int>(L.nready) + si.chain, c.n_heads, window,
+                  // the window (W <= XCH) is one chunk; the memory is split by L.xch
+                  window > 0 && window <= XCH ? XCH : L.xch, xchunks, L.max_chunks,
                   si.n_grid, M->at<int>(L.ready) + r0, M->at<int>(L.pos) + r0,
                   t_seq ? t_seq : (const int *)M->at<int>(L.t_dec), M->at<float>(L.q) + r0 * c.d, base,
                   seq_stride, head_stride, v_offset,
@@ -940,6 +946,7 @@ template <int DH> cudaError_t fused_setup_impl(rlt_model *M) {
   P.xch = 1;
   P.max_chunks = L.max_chunks;
   P.CH = L.xch;
+  P.CH_swa = XCH;
   P.rt_max = L.fs_rt;
   P.kv_reuse = (c.mem_groups == 1 && LD > 1) ? 1 : 0;
   P.alpha = c.alpha;

@@ -113,6 +113,7 @@ struct FsParams {
   int d, H, F, W, L, G, max_len, max_seqs;
   int swiglu, alpha0;
   int xch, max_chunks, CH;  // cross-attention chunks launched, chunk capacity, rows per chunk
+  int CH_swa;               // rows per chunk of the SWA (>= W: one chunk)
   int rt_max;               // row tiles of the launch bound
   int kv_reuse;             // one memory group read by every layer (G = 1, L_D > 1)
   float alpha, eps, inv_d, scale;
@@ -1079,7 +1080,7 @@ __global__ void __launch_bounds__(FS_THREADS, 1) k_step_fused(const __grid_const
           s_ready[i] = P.ready[m0 + i];
           s_pos[i] = P.t_dec[s_ready[i]];
         }
-        const FsAttnGeom g{m0, rv, H, P.W, P.CH, 1, rv * H, rv * H, ring_l,
+        const FsAttnGeom g{m0, rv, H, P.W, P.CH_swa, 1, rv * H, rv * H, ring_l,
                            (long)H * 2 * P.W * DH, 2L * P.W * DH, (long)P.W * DH, s_ready,
                            s_pos};
         fs_attn_phase<DH>(P, sh, g, gcta, ncta, cnt(l, PH_QKV, r), T_q * FS_S,
