@@ -373,7 +373,7 @@ RLT_API int rlt_get_encoder_output(rlt_model *model, int seq, void *e_out,
 
 /* Memory positions per split of rlt_attend (and of the decoder's
  * cross-attention for models with max_seqs * n_heads >= 2048; 256 below
- * that, 128 below 1024): rows longer than this are split into chunks of
+ * that): rows longer than this are split into chunks of
  * this many positions and merged in chunk order. */
 #define RLT_ATTEND_CHUNK 1024
 

@@ -39,8 +39,7 @@ constexpr int XCH = RLT_ATTEND_CHUNK;  // memory positions per split of rlt_atte
 // on its own rows). A function of the configuration only, so a row's result
 // depends on its own t and never on the batch around it.
 int xattn_chunk(const rlt_config *c) {
-  const long pairs = (long)c->max_seqs * c->n_heads;
-  return pairs < 1024 ? 128 : pairs < 2048 ? 256 : XCH;
+  return (long)c->max_seqs * c->n_heads < 2048 ? 256 : XCH;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
