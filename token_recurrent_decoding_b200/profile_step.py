@@ -35,6 +35,9 @@ def run_steps(args):
     from .rlt import Model
     wl = configs.workloads()[args.workload]
     cfg = wl.model
+    if args.layers:  # same shapes, fewer blocks (a profiler's device memory stays small)
+        cfg = cfg.replace(n_enc=args.layers, n_dec=args.layers,
+                          mem_groups=1 if cfg.mem_groups == 1 else args.layers)
     B = args.batch or wl.batch
     T = args.max_len or wl.max_len
     if args.t + args.steps > T:
@@ -168,6 +171,8 @@ def main():
                     help="sequence length of the arena (default: the workload's); small "
                          "values keep a profiler's device memory small")
     ap.add_argument("--graph", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="encoder and decoder blocks (default: the workload's)")
     ap.add_argument("--trace", default="",
                     help="record the persistent step's work items into this .npy file and "
                          "print where the time goes (last step)")
