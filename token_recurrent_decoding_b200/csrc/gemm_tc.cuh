@@ -285,4 +285,190 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 1) tmem_dealloc(tmem, BN);
 }
 
+// ------------------------------------------------------------ persistent form
+// The same GEMM for large row counts as a persistent kernel: each CTA walks
+// output tiles blockIdx.x, + gridDim.x, ... (N tiles fastest, so the CTAs
+// running at one time share their A row blocks in L2). Warp roles: warp 0
+// (one lane) streams A and B tiles through the ring with TMA, continuously
+// across tiles; warp 1 (one lane) issues tcgen05.mma into one of two TMEM
+// accumulators (2 x BN columns) and commits it to that accumulator's "full"
+// barrier; warps 2-5 drain an accumulator (TMEM lanes 32 (w mod 4)..+31 =
+// tile rows) through the epilogue and hand it back on its "empty" barrier.
+// So the MMAs of tile i + 1 run while tile i's epilogue stores. Every wait is
+// bounded; a CTA that gives up records RLT_ERR_TIMEOUT, stops issuing, and
+// lets its copies land before it exits.
+constexpr int TCP_THREADS = 192;
+
+__device__ __forceinline__ void tc_mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int BN, int STAGES> struct TcpSmem {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int BYTES = STAGES * STAGE + (2 * STAGES + 4) * 8 + 16 + 1024;
+};
+
+template <int BN, int STAGES, class Epi>
+__global__ void __launch_bounds__(TCP_THREADS, 1)
+    k_gemm_tcp(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               int M, int a_row0, int N, int K, Epi epi, int *err) {
+  static_assert(BN == 32 || BN == 64 || BN == 128, "two accumulators of BN columns");
+  using SM = TcpSmem<BN, STAGES>;
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t *tsm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(tsm + STAGES * SM::STAGE);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;  // [2] accumulator ready for the epilogue
+  uint64_t *tempty = tfull + 2;      // [2] accumulator drained
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_n = (N + BN - 1) / BN, tiles_m = (M + TC_BM - 1) / TC_BM;
+  const int total = tiles_m * tiles_n;
+  const int KB = K / TC_BK;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int *vabort = &s_abort;
+
+  pdl_trigger();
+  if (warp == 0 && lane == 0) {
+    // ---- producer
+    int it = 0;
+    bool first = true;
+    for (int tile = blockIdx.x; tile < total && !*vabort; tile += gridDim.x) {
+      const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
+      int kb = 0;
+      if (first) {
+        // the first stages' weight tiles stream before the dependency wait
+        const int pre = KB < STAGES ? KB : STAGES;
+        for (int j = 0; j < pre; j++) {
+          mbar_expect_tx(&full[j], SM::STAGE);
+          tma_load_2d(tsm + j * SM::STAGE + SM::A_BYTES, &tmB, j * TC_BK, n0, &full[j]);
+        }
+        pdl_wait();
+        for (int j = 0; j < pre; j++)
+          tma_load_2d(tsm + j * SM::STAGE, &tmA, j * TC_BK, a_row0 + m0, &full[j]);
+        kb = pre;
+        it = pre;
+        first = false;
+      }
+      for (; kb < KB; kb++, it++) {
+        const int s = it % STAGES, u = it / STAGES;
+        if (u > 0 && !mbar_wait_bounded(&empty[s], (u - 1) & 1, WAIT_LIMIT_NS_TC)) {
+          atomicExch(&s_abort, 1);
+          break;
+        }
+        uint8_t *a = tsm + s * SM::STAGE;
+        mbar_expect_tx(&full[s], SM::STAGE);
+        tma_load_2d(a, &tmA, kb * TC_BK, a_row0 + m0, &full[s]);
+        tma_load_2d(a + SM::A_BYTES, &tmB, kb * TC_BK, n0, &full[s]);
+      }
+    }
+    if (*vabort) {
+      // let the copies of the last use of every stage land
+      for (int j = it > STAGES ? it - STAGES : 0; j < it; j++)
+        mbar_wait_bounded(&full[j % STAGES], (unsigned)((j / STAGES) & 1), WAIT_LIMIT_NS_TC);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN);
+    int it = 0, i = 0, last = -1;  // last: tile index of the latest accumulator commit
+    for (int tile = blockIdx.x; tile < total && !*vabort; tile += gridDim.x, i++) {
+      const int buf = i & 1;
+      if (i >= 2 && !mbar_wait_bounded(&tempty[buf], (unsigned)(((i >> 1) - 1) & 1),
+                                        WAIT_LIMIT_NS_TC)) {
+        atomicExch(&s_abort, 1);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(buf * BN);
+      bool ok = true;
+      for (int kb = 0; kb < KB; kb++, it++) {
+        const int s = it % STAGES, u = it / STAGES;
+        if (!mbar_wait_bounded(&full[s], u & 1, WAIT_LIMIT_NS_TC)) {
+          atomicExch(&s_abort, 1);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint8_t *a = tsm + s * SM::STAGE;
+        const uint64_t ad = smem_desc_sw128(a), bd = smem_desc_sw128(a + SM::A_BYTES);
+#pragma unroll
+        for (int k = 0; k < TC_BK / 16; k++)
+          umma_bf16(acc, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc,
+                    (kb > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(&tfull[buf]);  // also after a failure: every issued MMA completes
+      last = i;
+      if (!ok) break;
+    }
+    // after a failure the epilogue may not drain the last accumulator: wait
+    // for its MMAs here, so no MMA is in flight when TMEM is released
+    if (*vabort && last >= 0)
+      mbar_wait_bounded(&tfull[last & 1], (unsigned)((last >> 1) & 1), WAIT_LIMIT_NS_TC);
+  } else if (warp >= 2) {
+    // ---- epilogue warps 2..5
+    pdl_wait();  // the epilogue reads and writes buffers of earlier kernels
+    const int g = warp & 3;  // TMEM lane group of this warp
+    int i = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, i++) {
+      const int buf = i & 1;
+      // lane 0 waits and decides for the whole warp (the TMEM loads below
+      // are warp-collective)
+      int go = 0;
+      if (lane == 0) {
+        go = !*vabort && mbar_wait_bounded(&tfull[buf], (unsigned)((i >> 1) & 1),
+                                           WAIT_LIMIT_NS_TC);
+        if (!go) atomicExch(&s_abort, 1);
+      }
+      go = __shfl_sync(0xffffffffu, go, 0);
+      __syncwarp();
+      if (!go) break;
+      tc_fence_after();
+      const int m0 = (tile / tiles_n) * TC_BM, n0 = (tile % tiles_n) * BN;
+      const int row = m0 + g * 32 + lane;
+      const uint32_t lane_base = tmem + (uint32_t)(buf * BN) + ((uint32_t)(g * 32) << 16);
+      if constexpr (epi_has_tile<Epi>::value) {
+        epi.template tile<BN>(row, row < M, n0, lane_base);
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(lane_base + c0, v);
+          if (row < M && n0 + c0 < N) epi.vec16(row, n0 + c0, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc_mbar_arrive(&tempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *vabort) set_error(err, DEV_ERR_TIMEOUT);
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 2 * BN);
+}
+
 }  // namespace rlt

@@ -194,6 +194,7 @@ struct rlt_model {
   int device = 0;
   int num_sms = 148;  // SMs of the device (decode GEMM split counts)
   int swap_br = 0;    // decode GEMMs with swapped operands: batch rows per tile (0 = off)
+  bool tc_persistent = true;  // encoder GEMMs of >= 1024 rows: persistent form
   std::vector<int> t_dec, t_enc;
   cudaStream_t last_stream = nullptr;
   template <typename X> X *at(size_t off) const { return reinterpret_cast<X *>(arena + off); }
@@ -335,10 +336,30 @@ cudaError_t launch_tc(rlt_model *M, int m_grid, int a_rows, int a_row0, int n, i
                   M->at<int>(M->L.err));
 }
 
+// Persistent encoder GEMM (k_gemm_tcp): one CTA per SM walks the 128 x BN
+// tiles with two TMEM accumulators, the epilogue of one tile overlapping the
+// MMAs of the next.
+template <int BN, int STAGES, class Epi>
+cudaError_t launch_tcp(rlt_model *M, int m, int a_rows, int a_row0, int n, int k, const bf16 *A,
+                       const bf16 *B, Epi epi, cudaStream_t st) {
+  constexpr int smem = TcpSmem<BN, STAGES>::BYTES;
+  const CUtensorMap *ma = tmap_bf16(M, A, (uint64_t)a_rows, (uint64_t)k, TC_BM);
+  const CUtensorMap *mb = tmap_bf16(M, B, (uint64_t)n, (uint64_t)k, BN);
+  if (!ma || !mb) return cudaErrorInvalidValue;
+  auto kern = k_gemm_tcp<BN, STAGES, Epi>;
+  RLT_TRY(ensure_smem_limit(kern, smem));
+  const int tiles = ((m + TC_BM - 1) / TC_BM) * ((n + BN - 1) / BN);
+  const int grid = std::min(tiles, M->num_sms);
+  return launch_k(kern, dim3(grid), dim3(TCP_THREADS), smem, st, *ma, *mb, m, a_row0, n, k, epi,
+                  M->at<int>(M->L.err));
+}
+
 template <class Epi>
 cudaError_t gemm_tc(rlt_model *M, int m_grid, int a_rows, int a_row0, int n, int k,
                     const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
   if (m_grid <= 0) return cudaSuccess;
+  if (m_grid >= 1024 && M->tc_persistent)
+    return launch_tcp<128, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
   if (m_grid >= 1024) return launch_tc<128, 3>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
   if (n >= 2048) return launch_tc<64, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
   return launch_tc<32, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
@@ -517,6 +538,8 @@ cudaError_t gemm_enc_qkv(rlt_model *M, int m, const bf16 *A, const bf16 *Wqkv,
                          EpiEncQkvRope<bf16> epi, cudaStream_t st) {
   const double d = M->cfg.d;
   Span sp(M, st, RLT_K_ENC, 3 * d * d * 2 + m * d * 2 + m * 3 * d * 2, 2.0 * m * 3 * d * d);
+  if (m >= 1024 && M->tc_persistent)
+    return launch_tcp<128, 4>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
   if (DH >= 128 || m >= 1024)
     return launch_tc<128, 3>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
   return launch_tc<64, 4>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
