@@ -314,7 +314,8 @@ template <int BN, int STAGES, class Epi>
 __global__ void __launch_bounds__(TCP_THREADS, 1)
     k_gemm_tcp(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                int M, int a_row0, int N, int K, Epi epi, int *err) {
-  static_assert(BN == 32 || BN == 64 || BN == 128, "two accumulators of BN columns");
+  static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256,
+                "two accumulators of BN columns fit the 512 TMEM columns");
   using SM = TcpSmem<BN, STAGES>;
   extern __shared__ uint8_t tsm_raw[];
   uint8_t *tsm = reinterpret_cast<uint8_t *>(
