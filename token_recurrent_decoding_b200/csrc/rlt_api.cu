@@ -358,8 +358,11 @@ template <class Epi>
 cudaError_t gemm_tc(rlt_model *M, int m_grid, int a_rows, int a_row0, int n, int k,
                     const bf16 *A, const bf16 *B, Epi epi, cudaStream_t st) {
   if (m_grid <= 0) return cudaSuccess;
-  if (m_grid >= 1024 && M->tc_persistent)
+  if (m_grid >= 1024 && M->tc_persistent) {
+    // 256-column tiles read a quarter fewer operand bytes per FLOP
+    if (n % 256 == 0) return launch_tcp<256, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
     return launch_tcp<128, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
+  }
   if (m_grid >= 1024) return launch_tc<128, 3>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
   if (n >= 2048) return launch_tc<64, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
   return launch_tc<32, 4>(M, m_grid, a_rows, a_row0, n, k, A, B, epi, st);
@@ -538,8 +541,11 @@ cudaError_t gemm_enc_qkv(rlt_model *M, int m, const bf16 *A, const bf16 *Wqkv,
                          EpiEncQkvRope<bf16> epi, cudaStream_t st) {
   const double d = M->cfg.d;
   Span sp(M, st, RLT_K_ENC, 3 * d * d * 2 + m * d * 2 + m * 3 * d * 2, 2.0 * m * 3 * d * d);
-  if (m >= 1024 && M->tc_persistent)
+  if (m >= 1024 && M->tc_persistent) {
+    if ((3 * M->cfg.d) % 256 == 0)
+      return launch_tcp<256, 4>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
     return launch_tcp<128, 4>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
+  }
   if (DH >= 128 || m >= 1024)
     return launch_tc<128, 3>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
   return launch_tc<64, 4>(M, m, M->L.ptok, 0, 3 * M->cfg.d, M->cfg.d, A, Wqkv, epi, st);
