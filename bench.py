@@ -371,9 +371,56 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
             "TFLOP_s": pr["flops"] / (par_ms / 1e3) / 1e12,
             "bound": "tensor" if pr["flops"] / (tc * 1e12) >= pr["bytes"] / (hbm * 1e9) else "hbm",
         }
+    if args.serve and wl.prompt_lengths and not r.ragged and cfg.dtype == configs.BF16:
+        out["serve"] = time_serve(wl, r, dist)
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_positions)
     return out
+
+
+def time_serve(wl, r, dist):
+    """The autoregressive form of the workload (outside the contract timing):
+    prefill the prompts only, run the decoder over them, then generate the
+    response tokens with rlt_serve_step (transition, next-token head,
+    temperature-1 draw from seeded uniforms, encoder append) on a model that
+    keeps the encoder cache. Reports generated tokens per second."""
+    import torch
+    from token_recurrent_decoding_b200.rlt import Model
+    cfg = wl.model
+    P = int(wl.prompt_lengths[0])
+    G = wl.max_len - P
+    w = inputs.make_weights(cfg)
+    m = Model(cfg, w, wl.batch, wl.max_len, stream=r.stream, enc_cache=True)
+    del w
+    r.m.close()  # the contract model and its arena are no longer needed
+    r.m.arena = None
+    torch.cuda.empty_cache()
+    tok = r.tok[:, :P]
+    flat = torch.from_numpy(np.ascontiguousarray(tok).reshape(-1).astype(np.int32)).cuda()
+    ids = np.arange(wl.batch, dtype=np.int32)
+    m.prefill_encoder(flat, ids, ids * P, [P] * wl.batch)
+    m.run_sequence(ids, P - 1)
+    g = torch.Generator(device="cuda").manual_seed(1)
+    uni = torch.rand((G, wl.batch), generator=g, device="cuda")
+    logits = torch.empty((wl.batch, cfg.vocab), dtype=torch.float32, device="cuda")
+    out = torch.empty(wl.batch, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    barrier(dist)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(r.stream)
+    for k in range(G):
+        m.serve_step(ids, 1.0, uni[k], logits, out)
+    b.record(r.stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), dist)
+    assert m.poll_device_error() == 0
+    m.close()
+    world = dist.get_world_size() if dist is not None else 1
+    return {"generated_tokens_per_s": world * wl.batch * G / (ms / 1e3), "ms_per_token_step": ms / G,
+            "sequences": wl.batch, "prompt": P, "generated": G,
+            "note": "prompt prefill + decoder over the prompt, then rlt_serve_step per token "
+                    "(transition, head E s_t, temperature-1 draw, encoder append)"}
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -444,6 +491,8 @@ def main():
     ap.add_argument("--all-workloads", action="store_true",
                     help="one JSON line per workload (not the default contract line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serve", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time the autoregressive form (generated tokens/s)")
     ap.add_argument("--cpu-positions", type=int, default=24)
     ap.add_argument("--profile-stride", type=int, default=64,
                     help="event-time every k-th decoder step for the per-kernel roofline")

@@ -256,3 +256,28 @@ def test_serving_errors_change_no_state():
     assert e.value.status == 4
     assert m2.get_state(0)[2] == 11
     assert m2.get_encoder_output(0)[0].shape[0] == 12
+
+
+def test_serve_step_on_a_two_chain_batch():
+    """Batches of 128 rows and more step as two half-batch chains; the serve
+    step's head, draw and append follow the same rows: greedy draws equal the
+    argmax of the logits the oracle reads from the GPU's s_t."""
+    cfg = SMALL["m140_like"]
+    B, P = 160, 6
+    w = inputs.make_weights(cfg, 0, True)
+    tok = inputs.make_tokens(cfg.vocab, [P + 3] * B)
+    m = Model(cfg, w, B, P + 3, enc_cache=True)
+    prefill_all(m, tok, [P] * B)
+    ids = list(range(B))
+    m.run_sequence(ids, P - 1)
+    o = oracle.Oracle(cfg, w)
+    for step in range(3):
+        out, logits = m.serve_step(ids, 0.0)
+        toks = out.cpu().numpy()
+        lg = to_np(logits)
+        for i in (0, 79, 80, 159):
+            ref = o.lm_head(to_np(m.get_state(i)[0]))
+            assert np.abs(lg[i] - ref).max() <= STEP_TOL[cfg.dtype] * rms(ref)
+            assert lg[i][toks[i]] == lg[i].max()
+    assert m.get_state(0)[2] == P + 2
+    assert m.poll_device_error() == 0
