@@ -119,7 +119,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->rope = take(T * (dh / 2) * 8);
   L->err = take(16);
   L->ctl = take(sizeof(DevCtl));
-  L->nready = take(2 * 4);
+  L->nready = take(4 * 4);
   L->ready = take(S * 4);
   L->pos = take(S * 4);
   L->h = take(S * d * 4);
@@ -219,8 +219,8 @@ struct rlt_model {
     int64_t launches;
   };
   std::map<std::tuple<int, int, int>, ProfGraph> prof_graphs;
-  cudaStream_t side = nullptr;  // second chain of a split step
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaStream_t side[3] = {};  // chains 1.. of a split step
+  cudaEvent_t ev_fork = nullptr, ev_join[3] = {};
   // TMA descriptors of bf16 [rows][cols] matrices, keyed by (pointer, rows, cols, box rows)
   std::map<std::tuple<const void *, uint64_t, uint64_t, uint32_t>, CUtensorMap> tmaps;
   cudaError_t (*step)(rlt_model *, const StepInfo &, cudaStream_t) = nullptr;
@@ -1462,34 +1462,44 @@ StepInfo step_info(const rlt_model *M, const int32_t *ids, int n) {
   return si;
 }
 
-// Batches of at least this many rows run as two half-batch chains.
+// Batches of at least this many rows run as parallel chains over equal
+// shares of the rows (sequences are independent, so one chain's GEMMs run
+// while another's attention streams K/V); at most MAX_CHAINS of them, each
+// of at least CHAIN_MIN_ROWS rows.
 constexpr int SPLIT_MIN_ROWS = 128;
+constexpr int MAX_CHAINS = 2;
+constexpr int CHAIN_MIN_ROWS = 64;
 
 // Split a whole-batch step into its chains (byte sums shared in proportion).
-int make_chains(const rlt_model *M, const StepInfo &all, StepInfo ch[2]) {
-  if (all.n < SPLIT_MIN_ROWS || !M->side) {
+int make_chains(const rlt_model *M, const StepInfo &all, StepInfo ch[4]) {
+  if (all.n < SPLIT_MIN_ROWS || !M->side[0]) {
     ch[0] = all;
     return 1;
   }
-  const int na = (all.n + 1) / 2, nb = all.n - na;
-  const double fa = (double)na / all.n;
-  ch[0] = {0, na, std::min((na + 63) / 64 * 64, M->cfg.max_seqs), 0, all.xchunks,
-           all.sum_keys * fa, all.sum_win * fa};
-  ch[1] = {na, nb, std::min((nb + 63) / 64 * 64, M->cfg.max_seqs - na), 1, all.xchunks,
-           all.sum_keys * (1 - fa), all.sum_win * (1 - fa)};
-  return 2;
+  const int nch = std::max(2, std::min(MAX_CHAINS, all.n / CHAIN_MIN_ROWS));
+  for (int c = 0; c < nch; c++) {
+    const int lo = (int)((long)all.n * c / nch), hi = (int)((long)all.n * (c + 1) / nch);
+    const double f = (double)(hi - lo) / all.n;
+    ch[c] = {lo, hi - lo, std::min((hi - lo + 63) / 64 * 64, M->cfg.max_seqs - lo), c,
+             all.xchunks, all.sum_keys * f, all.sum_win * f};
+  }
+  return nch;
 }
 
-// Launch the chains of one step on `st` (and the side stream).
+// Launch the chains of one step: chain 0 on `st`, the others on the side
+// streams, forked from and joined back into `st`.
 cudaError_t launch_chains(rlt_model *M, const StepInfo *ch, int nch, cudaStream_t st) {
   if (M->use_fused) return M->step_fused(M, ch[0], st);
   if (nch == 1) return M->step(M, ch[0], st);
   RLT_TRY(cudaEventRecord(M->ev_fork, st));
-  RLT_TRY(cudaStreamWaitEvent(M->side, M->ev_fork, 0));
+  for (int c = 1; c < nch; c++) RLT_TRY(cudaStreamWaitEvent(M->side[c - 1], M->ev_fork, 0));
   RLT_TRY(M->step(M, ch[0], st));
-  RLT_TRY(M->step(M, ch[1], M->side));
-  RLT_TRY(cudaEventRecord(M->ev_join, M->side));
-  return cudaStreamWaitEvent(st, M->ev_join, 0);
+  for (int c = 1; c < nch; c++) RLT_TRY(M->step(M, ch[c], M->side[c - 1]));
+  for (int c = 1; c < nch; c++) {
+    RLT_TRY(cudaEventRecord(M->ev_join[c - 1], M->side[c - 1]));
+    RLT_TRY(cudaStreamWaitEvent(st, M->ev_join[c - 1], 0));
+  }
+  return cudaSuccess;
 }
 
 // One decoder step of the slots already listed in the arena's ready list:
@@ -1550,7 +1560,7 @@ cudaError_t capture(rlt_model *M, cudaStream_t st, Fn fn, cudaGraphExec_t *out, 
 // whose event-record nodes bracket each kernel, so every kernel is timed
 // alone and without host gaps; that step is synchronised and folded.
 cudaError_t enqueue_step(rlt_model *M, const StepInfo &all, cudaStream_t st) {
-  StepInfo ch[2];
+  StepInfo ch[4];
   const bool prof = M->profiling && M->prof_stride > 0 && (M->step_counter % M->prof_stride == 0);
   M->step_counter++;
   int nch = 1;
@@ -1558,10 +1568,13 @@ cudaError_t enqueue_step(rlt_model *M, const StepInfo &all, cudaStream_t st) {
     ch[0] = all;
   else
     nch = make_chains(M, all, ch);
-  int nval[2] = {ch[0].n, nch == 2 ? ch[1].n : 0};
+  int nval[4] = {ch[0].n, 0, 0, 0};
+  for (int c = 1; c < nch; c++) nval[c] = ch[c].n;
   RLT_TRY(cudaMemcpyAsync(M->at<int>(M->L.nready), nval, sizeof(nval), cudaMemcpyHostToDevice,
                           st));  // pageable source: staged before return
-  auto key = std::make_tuple(ch[0].n_grid, M->use_fused ? -1 : (nch == 2 ? ch[1].n_grid : 0),
+  // the chain shapes follow from the row count: the first and last chains'
+  // row bounds and the chain count identify the graph
+  auto key = std::make_tuple(ch[0].n_grid, M->use_fused ? -1 : nch * 100000 + ch[nch - 1].n_grid,
                              all.xchunks);
   const bool saved = M->profiling;
   if (st == nullptr) {  // legacy stream: cannot capture
@@ -1953,9 +1966,11 @@ RLT_API int rlt_create(const rlt_config *cfg, const rlt_weights *w, void *d_aren
       e = cudaGetLastError();
     }
   }
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&M->side, cudaStreamNonBlocking);
+  for (int c = 0; c < 3 && e == cudaSuccess; c++) {
+    e = cudaStreamCreateWithFlags(&M->side[c], cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&M->ev_join[c], cudaEventDisableTiming);
+  }
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&M->ev_fork, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&M->ev_join, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     rlt_destroy(M);
@@ -1991,12 +2006,14 @@ RLT_API void rlt_destroy(rlt_model *M) {
       cudaEventDestroy(p.b);
     }
   }
-  if (M->side) {
-    cudaStreamSynchronize(M->side);
-    cudaStreamDestroy(M->side);
+  for (int c = 0; c < 3; c++) {
+    if (M->side[c]) {
+      cudaStreamSynchronize(M->side[c]);
+      cudaStreamDestroy(M->side[c]);
+    }
+    if (M->ev_join[c]) cudaEventDestroy(M->ev_join[c]);
   }
   if (M->ev_fork) cudaEventDestroy(M->ev_fork);
-  if (M->ev_join) cudaEventDestroy(M->ev_join);
   delete M;
 }
 
