@@ -161,6 +161,38 @@ def run_attend(args):
                       "GB_s": [byts / (t / 1e3) / 1e9 for t in times]}))
 
 
+def run_parallel(args):
+    """Encoder prefill, then the token-parallel decoder pass (feedback-off
+    workloads), `--steps` times; prints each pass's CUDA-event time."""
+    import torch
+
+    from . import configs, inputs
+    from .rlt import Model
+    wl = configs.workloads()[args.workload]
+    cfg = wl.model
+    B = args.batch or wl.batch
+    T = args.max_len or wl.max_len
+    lengths = [T] * B
+    w = inputs.make_weights(cfg)
+    tok = inputs.make_tokens(cfg.vocab, lengths)
+    m = Model(cfg, w, B, T)
+    del w
+    flat = torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda()
+    offsets = np.arange(B, dtype=np.int32) * T
+    ids = list(range(B))
+    times = []
+    for _ in range(args.steps):
+        m.prefill_encoder(flat, ids, offsets, lengths)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        m.decoder_parallel(ids, T)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    assert m.poll_device_error() == 0
+    print(json.dumps({"workload": args.workload, "batch": B, "T": T, "parallel_ms": times}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="m140_bf16")
@@ -180,6 +212,8 @@ def main():
     ap.add_argument("--kernel", choices=["fused", "chain"], default=None,
                     help="decoder step kernel (default: the model's default)")
     ap.add_argument("--attend", action="store_true")
+    ap.add_argument("--parallel", action="store_true",
+                    help="time the token-parallel decoder pass (feedback-off workloads)")
     ap.add_argument("--n", type=int, default=256)
     ap.add_argument("--heads", type=int, default=12)
     ap.add_argument("--dh", type=int, default=64)
@@ -189,6 +223,8 @@ def main():
     args = ap.parse_args()
     if args.attend:
         run_attend(args)
+    elif args.parallel:
+        run_parallel(args)
     else:
         run_steps(args)
 
