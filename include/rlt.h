@@ -364,6 +364,78 @@ RLT_API int rlt_set_snapshot(rlt_model *model, int seq, const void *buf, size_t 
  * configuration and current weight values. */
 RLT_API int rlt_model_fingerprint(rlt_model *model, uint64_t *out);
 
+/* ---------------------------------------------------------------- training
+ * Backpropagation through time of the decoder recurrence. The decoder is
+ * trained by full backpropagation through time ([RLT-PV] "Per-token
+ * recurrence, no quality gain", body: a custom reverse-traversal backward
+ * pass), and both parts of the carried state H_t = (s_t, C_t^D) carry
+ * gradient: the state-to-state Jacobian has cross-terms through the decoder
+ * cache, so a truncation that detaches s alone leaves paths open through it
+ * ([RLT-96] "Training and serving implications").
+ *
+ * Gradients of the decoder's parameters and of the memory projection:
+ * float32 device buffers the caller owns, each shaped like its weight
+ * (rlt_weights), ADDED into (zero them before the first call; successive
+ * calls accumulate, as chunks and batches of one optimizer step should). For
+ * a tied model dec_wqkv, dec_wo, dec_w1, dec_wb, dec_w2 receive the decoder's
+ * use of the shared encoder matrices. dec_wb only for SwiGLU; mem_wk/mem_wv
+ * for g < G. */
+typedef struct rlt_grads {
+  float *gate_w, *gate_b, *sstar, *dec_lnf;
+  float *dec_ln1[RLT_MAX_LAYERS], *dec_wqkv[RLT_MAX_LAYERS], *dec_wo[RLT_MAX_LAYERS],
+      *dec_ln2[RLT_MAX_LAYERS], *dec_wqx[RLT_MAX_LAYERS], *dec_wox[RLT_MAX_LAYERS],
+      *dec_ln3[RLT_MAX_LAYERS], *dec_w1[RLT_MAX_LAYERS], *dec_wb[RLT_MAX_LAYERS],
+      *dec_w2[RLT_MAX_LAYERS];
+  float *mem_wk[RLT_MAX_LAYERS], *mem_wv[RLT_MAX_LAYERS];
+} rlt_grads;
+
+/* Floats per row of a carried state gradient: [s: d] then the cache
+ * [L_D][2][W-1][d] in the rlt_get_state layout (positions tb-(W-1) .. tb-1,
+ * oldest first; entries of negative positions are zero). */
+#define RLT_CARRY_FLOATS(d, n_dec_layers, window) \
+  ((size_t)(d) * (1 + 2 * (size_t)(n_dec_layers) * ((window) - 1)))
+
+/* Host only. Device workspace bytes of rlt_backward for n rows and n_steps
+ * positions (0 if the configuration is invalid). It holds the recorded s_t
+ * and keys/values of the chunk, one step's activations, the saved
+ * cross-attention terms and the memory-row gradients: about
+ * n * n_steps * L_D * d * 8 + G * n * max_len * d * 8 bytes. */
+RLT_API size_t rlt_backward_workspace_bytes(const rlt_config *cfg, int n, int n_steps);
+
+/* One chunk of backpropagation through time for the listed sequences, all
+ * at the same position t0 = t_dec (e.g. 0 after rlt_reset_seq).
+ *   1. The forward of positions t0 .. t1-1 (t1 = t0 + n_steps) runs on the
+ *      model's own step kernels, exactly as rlt_run_sequence, recording s_t
+ *      and every layer's (k_t, v_t) in the workspace; the sequences end at
+ *      t_dec = t1 as after rlt_run_sequence.
+ *   2. Reverse traversal t = t1-1 .. t0: the step's forward is recomputed
+ *      from the recorded state and differentiated layer by layer; a key or
+ *      value entry's gradient accumulates over the steps that read it.
+ *   3. The gradient of the memory rows M<=t1-1 is pushed through the memory
+ *      projection into e and the mem_wk / mem_wv gradients.
+ * The loss is L = sum_t <d_sgrad[i][t-t0], s_t> (+ <d_carry_in, H_{t1-1}>):
+ *   d_sgrad     device float32 [n][n_steps][d]: dL/ds_t (e.g. from an LM head)
+ *   d_carry_in  device float32 [n][RLT_CARRY_FLOATS] or NULL: the gradient of
+ *               the state leaving the chunk (from the chunk after it)
+ *   d_carry_out device float32 [n][RLT_CARRY_FLOATS] or NULL: written with the
+ *               gradient of the state entering the chunk, H_{t0-1}
+ *   d_egrad     device float32 [n][max_len][d], ADDED into: dL/de_j for rows
+ *               j < t1 (the encoder's gradient, for the encoder's backward)
+ *   grads       accumulated parameter gradients; when t0 = 0 the gradient of
+ *               s_{-1} = s* is also added into grads->sstar.
+ * Exact chunked backpropagation: run the forward over all chunks keeping the
+ * state at each chunk start (rlt_get_state), then for the chunks in reverse
+ * restore that state (rlt_set_state) and call this with the previous call's
+ * d_carry_out as d_carry_in. Arithmetic is fp32 with the weights in the model
+ * dtype; the recorded keys and values are the forward's own.
+ * Errors: INVALID_ARG (null pointers, n < 1, n_steps < 1, sequences at
+ * different t_dec, workspace too small or not 256-byte aligned, a needed
+ * gradient buffer missing), DUPLICATE_ID, CAPACITY, NOT_READY (t1 > t_enc). */
+RLT_API int rlt_backward(rlt_model *model, const int32_t *h_seq_ids, int n, int n_steps,
+                         const float *d_sgrad, const float *d_carry_in, float *d_carry_out,
+                         float *d_egrad, const rlt_grads *grads, void *d_work,
+                         size_t work_bytes, rlt_stream stream);
+
 /* Export the encoder output of slot `seq`: e_out [t_enc][d] and mem_out
  * [G][t_enc][2][d] (K row then V row per position) in the model dtype.
  * Either may be NULL. */

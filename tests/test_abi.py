@@ -74,3 +74,17 @@ def test_attend_workspace_sizing():
     a = rlt.attend_workspace_bytes(256, 12, 64, 1024)
     assert a > 256 * 12 * 66 * 4  # partials of more than one chunk per (row, head)
     assert rlt.attend_workspace_bytes(256, 12, 64, 2048) > a
+
+
+def test_backward_workspace_bytes_host_only():
+    """rlt_backward_workspace_bytes is host arithmetic: 0 for an invalid
+    configuration or empty chunk, growing with rows and positions."""
+    from token_recurrent_decoding_b200 import configs, rlt
+    lib = rlt._lib()
+    c = rlt.make_config(configs.TINY, 4, 64)
+    import ctypes as C
+    f = lambda n, s: lib.rlt_backward_workspace_bytes(C.byref(c), n, s)
+    assert f(0, 8) == 0 and f(2, 0) == 0
+    assert 0 < f(1, 8) < f(2, 8) and f(2, 8) < f(2, 16)
+    bad = rlt.make_config(configs.TINY.replace(window=2000), 4, 64)
+    assert lib.rlt_backward_workspace_bytes(C.byref(bad), 2, 8) == 0

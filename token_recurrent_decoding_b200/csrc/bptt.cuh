@@ -1,0 +1,658 @@
+// Backpropagation through time of the RLT decoder recurrence.
+//
+// The decoder is trained with full backpropagation through time ([RLT-PV]
+// "Per-token recurrence, no quality gain" (news.promtvault.app), body: a
+// custom reverse-traversal backward pass), and the carried state has two
+// parts that both carry gradient: s_t and the decoder's retained keys and
+// values ([RLT-96] "RLT Runs 96 Blocks Per Token With Recurrent State, No
+// Resets" (aimastery.page), "Training and serving implications": the
+// state-to-state Jacobian has cross-terms through the decoder cache, so
+// detaching s alone leaves paths open through it).
+//
+// Reverse traversal over a chunk of positions t0 .. t1-1: the forward of the
+// chunk runs first on the product step kernels while s_t and every layer's
+// (k_t, v_t) are recorded; then for t = t1-1 down to t0 one step's forward is
+// recomputed from (s_{t-1}, the recorded keys and values, e_t, M<=t) keeping
+// its activations, and the step is differentiated layer by layer in reverse.
+// The gradient of a key/value entry accumulates in a ring of W slots per
+// (layer, row, head) and is complete once step t has run (steps t .. t+W-1
+// read it); the cross-attention's gradient into the memory rows does not
+// feed back into the recurrence, so it is formed after the traversal from
+// the saved queries, output gradients and softmax statistics, as the
+// key/value half of a causal attention backward, then pushed through the
+// memory projection into e.
+//
+// Everything here computes in fp32 (weights read in the model dtype).
+#pragma once
+
+#include "common.cuh"
+
+namespace rlt {
+
+// ------------------------------------------------------------------ GEMM
+// C[m][n] (= or +=) sum_k A(m, k) B(n, k); A(m, k) = A[m * lda + k] when AK
+// (k contiguous) else A[k * lda + m]; B likewise with BK. 64 x 64 tiles,
+// 256 threads, 4 x 4 outputs per thread, k in steps of 16. The loader walks
+// the contiguous index fastest for either layout.
+template <typename TA, typename TB, bool AK, bool BK>
+__global__ void __launch_bounds__(256)
+    k_bw_gemm(int M, int N, int K, const TA *__restrict__ A, long lda, const TB *__restrict__ B,
+              long ldb, float *__restrict__ C, long ldc, int acc) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float c[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = tid; i < 64 * 16; i += 256) {
+      int r, k;
+      if (AK) { r = i / 16; k = i % 16; } else { k = i / 64; r = i % 64; }
+      int gm = m0 + r, gk = k0 + k;
+      As[k][r] = (gm < M && gk < K) ? to_f(AK ? A[(size_t)gm * lda + gk] : A[(size_t)gk * lda + gm])
+                                    : 0.f;
+      if (BK) { r = i / 16; k = i % 16; } else { k = i / 64; r = i % 64; }
+      int gn = n0 + r;
+      gk = k0 + k;
+      Bs[k][r] = (gn < N && gk < K) ? to_f(BK ? B[(size_t)gn * ldb + gk] : B[(size_t)gk * ldb + gn])
+                                    : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; i++) a[i] = As[k][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; j++) b[j] = Bs[k][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) c[i][j] = fmaf(a[i], b[j], c[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    int r = m0 + ty * 4 + i;
+    if (r >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      int col = n0 + tx * 4 + j;
+      if (col >= N) continue;
+      float *p = C + (size_t)r * ldc + col;
+      *p = acc ? *p + c[i][j] : c[i][j];
+    }
+  }
+}
+
+// --------------------------------------------------------------- helpers
+// Sum over the block (blockDim.x a multiple of 32, at most 1024).
+__device__ __forceinline__ float bw_block_sum(float v, float *red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int i = 0; i < nw; i++) s += red[i];
+  return s;
+}
+
+__device__ __forceinline__ float gelu_grad(float x) {
+  const float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
+  const float pdf = 0.39894228040143268f * expf(-0.5f * x * x);
+  return cdf + x * pdf;
+}
+
+// ------------------------------------------------------ forward recording
+// Window entering the chunk: hist position p (0 .. W-2) holds position
+// t0 - (W-1) + p from the ring (zero for negative positions); s_{t0-1}.
+// kv_hist [L][n][H][2][P][dh], P = n_steps + W - 1.
+template <typename T>
+__global__ void k_bw_hist_init(int n, const int *__restrict__ ready, const T *__restrict__ ring,
+                               const float *__restrict__ s, int L, int H, int dh, int W,
+                               int max_seqs, long t0, int P, T *__restrict__ kv_hist,
+                               float *__restrict__ s_hist0) {
+  const int d = H * dh, Wm1 = W - 1;
+  const long total = (long)L * n * H * 2 * Wm1 * dh;
+  const long stride = (long)gridDim.x * blockDim.x;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += stride) {
+    const int e = (int)(idx % dh);
+    long r = idx / dh;
+    const int p = (int)(r % Wm1);
+    r /= Wm1;
+    const int kv = (int)(r % 2);
+    r /= 2;
+    const int h = (int)(r % H);
+    r /= H;
+    const int i = (int)(r % n);
+    const int l = (int)(r / n);
+    const long pos = t0 - Wm1 + p;
+    T v = from_f<T>(0.f);
+    if (pos >= 0)
+      v = ring[((((size_t)l * max_seqs + ready[i]) * H + h) * 2 + kv) * W * dh +
+               (size_t)(pos % W) * dh + e];
+    kv_hist[((((size_t)l * n + i) * H + h) * 2 + kv) * P * dh + (size_t)p * dh + e] = v;
+  }
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < (long)n * d; idx += stride)
+    s_hist0[idx] = s[(size_t)ready[idx / d] * d + idx % d];
+}
+
+// After the product step at position t: its (k_t, v_t) of every layer into
+// hist position p, and s_t.
+template <typename T>
+__global__ void k_bw_hist_step(int n, const int *__restrict__ ready, const T *__restrict__ ring,
+                               const float *__restrict__ s, int L, int H, int dh, int W,
+                               int max_seqs, long t, int p, int P, T *__restrict__ kv_hist,
+                               float *__restrict__ s_hist_k) {
+  const int d = H * dh;
+  const long total = (long)L * n * H * 2 * dh;
+  const long stride = (long)gridDim.x * blockDim.x;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += stride) {
+    const int e = (int)(idx % dh);
+    long r = idx / dh;
+    const int kv = (int)(r % 2);
+    r /= 2;
+    const int h = (int)(r % H);
+    r /= H;
+    const int i = (int)(r % n);
+    const int l = (int)(r / n);
+    kv_hist[((((size_t)l * n + i) * H + h) * 2 + kv) * P * dh + (size_t)p * dh + e] =
+        ring[((((size_t)l * max_seqs + ready[i]) * H + h) * 2 + kv) * W * dh +
+             (size_t)(t % W) * dh + e];
+  }
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < (long)n * d; idx += stride)
+    s_hist_k[idx] = s[(size_t)ready[idx / d] * d + idx % d];
+}
+
+// ---------------------------------------------------- forward recompute
+// cat = [e_t ; s_{t-1}] per row.
+template <typename T>
+__global__ void k_bw_gate_cat(int n, int d, const int *__restrict__ ready, const T *__restrict__ e,
+                              int max_len, long t, const float *__restrict__ s_prev,
+                              float *__restrict__ cat) {
+  const long total = (long)n * 2 * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / (2 * d)), c = (int)(idx % (2 * d));
+    cat[idx] = c < d ? to_f(e[((size_t)ready[i] * max_len + t) * d + c])
+                     : s_prev[(size_t)i * d + c - d];
+  }
+}
+
+// g = sigmoid(gpre + b_g), x = e_t + alpha g s_{t-1}.
+__global__ void k_bw_gate_fwd(int n, int d, const float *__restrict__ gpre,
+                              const float *__restrict__ gate_b, const float *__restrict__ cat,
+                              float alpha, float *__restrict__ g, float *__restrict__ x) {
+  const long total = (long)n * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / d), c = (int)(idx % d);
+    const float gg = sigmoidf_(gpre[idx] + gate_b[c]);
+    g[idx] = gg;
+    x[idx] = cat[(size_t)i * 2 * d + c] + alpha * gg * cat[(size_t)i * 2 * d + d + c];
+  }
+}
+
+// u = h r gamma, r = 1 / sqrt(mean(h^2) + eps); one block per row.
+__global__ void k_bw_rms_fwd(int d, float eps, const float *__restrict__ h,
+                             const float *__restrict__ gamma, float *__restrict__ u,
+                             float *__restrict__ r) {
+  __shared__ float red[32];
+  const float *x = h + (size_t)blockIdx.x * d;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) ss += x[c] * x[c];
+  ss = bw_block_sum(ss, red);
+  const float rr = rsqrtf(ss / d + eps);
+  if (threadIdx.x == 0) r[blockIdx.x] = rr;
+  for (int c = threadIdx.x; c < d; c += blockDim.x)
+    u[(size_t)blockIdx.x * d + c] = x[c] * rr * gamma[c];
+}
+
+// Rotary encoding of the q part of a [n][3d] q/k/v row at position t.
+__global__ void k_bw_rope_q(int n, int H, int dh, long t, const float2 *__restrict__ rope,
+                            const float *__restrict__ qkv, float *__restrict__ q) {
+  const int d = H * dh, half = dh / 2;
+  const long total = (long)n * H * half;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int j = (int)(idx % half), h = (int)((idx / half) % H), i = (int)(idx / half / H);
+    const float2 cs = rope[(size_t)t * half + j];
+    const float a = qkv[(size_t)i * 3 * d + h * dh + j], b = qkv[(size_t)i * 3 * d + h * dh + j + half];
+    q[(size_t)i * d + h * dh + j] = a * cs.x - b * cs.y;
+    q[(size_t)i * d + h * dh + j + half] = b * cs.x + a * cs.y;
+  }
+}
+
+// GELU or SwiGLU activation of the FFN: act = GELU(z) or SiLU(z) zb.
+__global__ void k_bw_act_fwd(long total, int swiglu, const float *__restrict__ z,
+                             const float *__restrict__ zb, float *__restrict__ act) {
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x)
+    act[idx] = swiglu ? silu(z[idx]) * zb[idx] : gelu_erf(z[idx]);
+}
+
+// Where the keys of one (row, head) live. SWA: the recorded window in
+// kv_hist; cross-attention: the memory group in the arena.
+template <typename T> struct BwKeys {
+  const T *base;    // kv_hist or memory
+  const int *ready;
+  long l_or_g;      // layer (SWA) or group (cross)
+  int n, H, dh, P;  // SWA: rows, heads, head size, hist positions
+  int max_seqs, max_len;
+  bool swa;
+  __device__ const T *k(int i, int h) const {
+    if (swa) return base + ((((size_t)l_or_g * n + i) * H + h) * 2 + 0) * P * dh;
+    return base + ((((size_t)l_or_g * max_seqs + ready[i]) * H + h) * 2 + 0) * max_len * dh;
+  }
+  __device__ const T *v(int i, int h) const {
+    if (swa) return base + ((((size_t)l_or_g * n + i) * H + h) * 2 + 1) * P * dh;
+    return base + ((((size_t)l_or_g * max_seqs + ready[i]) * H + h) * 2 + 1) * max_len * dh;
+  }
+};
+
+// Attention of one query per (row, head) over key rows j_lo .. j_hi of the
+// key table (one warp each; lanes split the head dimension): a and the
+// log-sum-exp of the scaled scores.
+template <typename T, int DH>
+__global__ void k_bw_attn_fwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
+                              const float *__restrict__ q, float *__restrict__ a,
+                              float *__restrict__ lse) {
+  constexpr int EPL = (DH + 31) / 32;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= n * H) return;
+  const int i = warp / H, h = warp % H, d = H * DH;
+  const T *K = keys.k(i, h), *V = keys.v(i, h);
+  float qv[EPL], acc[EPL];
+#pragma unroll
+  for (int x = 0; x < EPL; x++) {
+    const int e = lane + 32 * x;
+    qv[x] = e < DH ? q[(size_t)i * d + h * DH + e] : 0.f;
+    acc[x] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int j = j_lo; j <= j_hi; j++) {
+    float dot = 0.f;
+#pragma unroll
+    for (int x = 0; x < EPL; x++) {
+      const int e = lane + 32 * x;
+      if (e < DH) dot += qv[x] * to_f(K[(size_t)j * DH + e]);
+    }
+    const float s = warp_sum(dot) * scale;
+    const float mn = fmaxf(m, s);
+    const float corr = expf(m - mn), p = expf(s - mn);
+    l = l * corr + p;
+#pragma unroll
+    for (int x = 0; x < EPL; x++) {
+      const int e = lane + 32 * x;
+      acc[x] = acc[x] * corr + (e < DH ? p * to_f(V[(size_t)j * DH + e]) : 0.f);
+    }
+    m = mn;
+  }
+#pragma unroll
+  for (int x = 0; x < EPL; x++) {
+    const int e = lane + 32 * x;
+    if (e < DH) a[(size_t)i * d + h * DH + e] = acc[x] / l;
+  }
+  if (lane == 0) lse[(size_t)i * H + h] = m + logf(l);
+}
+
+// ------------------------------------------------------------ backward
+// Attention backward of one query per (row, head) over key rows
+// j_lo .. j_hi: P_j = exp(scale q.k_j - lse), dS_j = P_j (da.v_j - da.a),
+// dq = scale sum_j dS_j k_j. SWA (dring != null): also dk_j += scale dS_j q
+// and dv_j += P_j da into the gradient ring slot of position pos0 + j.
+// Cross-attention (xq != null): q, da, lse and D = da.a are saved for the
+// memory-gradient pass.
+template <typename T, int DH>
+__global__ void k_bw_attn_bwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
+                              const float *__restrict__ q, const float *__restrict__ a,
+                              const float *__restrict__ lse, const float *__restrict__ da,
+                              float *__restrict__ dq, float *__restrict__ dring, int W, long pos0,
+                              float *__restrict__ xq, float *__restrict__ xda,
+                              float *__restrict__ xlse, float *__restrict__ xD) {
+  constexpr int EPL = (DH + 31) / 32;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= n * H) return;
+  const int i = warp / H, h = warp % H, d = H * DH;
+  const T *K = keys.k(i, h), *V = keys.v(i, h);
+  const size_t off = (size_t)i * d + h * DH;
+  float qv[EPL], dav[EPL], dqv[EPL];
+  float Dp = 0.f;
+#pragma unroll
+  for (int x = 0; x < EPL; x++) {
+    const int e = lane + 32 * x;
+    qv[x] = e < DH ? q[off + e] : 0.f;
+    dav[x] = e < DH ? da[off + e] : 0.f;
+    Dp += e < DH ? dav[x] * a[off + e] : 0.f;
+    dqv[x] = 0.f;
+  }
+  const float D = warp_sum(Dp);
+  const float L = lse[(size_t)i * H + h];
+  float *dk_ring = dring ? dring + ((((size_t)keys.l_or_g * n + i) * H + h) * 2 + 0) * W * DH
+                         : nullptr;
+  float *dv_ring = dring ? dk_ring + (size_t)W * DH : nullptr;
+  for (int j = j_lo; j <= j_hi; j++) {
+    float dot = 0.f, dp = 0.f;
+    float kv[EPL];
+#pragma unroll
+    for (int x = 0; x < EPL; x++) {
+      const int e = lane + 32 * x;
+      kv[x] = e < DH ? to_f(K[(size_t)j * DH + e]) : 0.f;
+      dot += qv[x] * kv[x];
+      dp += e < DH ? dav[x] * to_f(V[(size_t)j * DH + e]) : 0.f;
+    }
+    const float s = warp_sum(dot) * scale;
+    dp = warp_sum(dp);
+    const float p = expf(s - L);
+    const float ds = p * (dp - D);
+#pragma unroll
+    for (int x = 0; x < EPL; x++) dqv[x] += scale * ds * kv[x];
+    if (dk_ring) {
+      const size_t slot = (size_t)((pos0 + j) % W) * DH;
+#pragma unroll
+      for (int x = 0; x < EPL; x++) {
+        const int e = lane + 32 * x;
+        if (e < DH) {
+          dk_ring[slot + e] += scale * ds * qv[x];
+          dv_ring[slot + e] += p * dav[x];
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < EPL; x++) {
+    const int e = lane + 32 * x;
+    if (e < DH) {
+      dq[off + e] = dqv[x];
+      if (xq) {
+        xq[off + e] = qv[x];
+        xda[off + e] = dav[x];
+      }
+    }
+  }
+  if (xq && lane == 0) {
+    xlse[(size_t)i * H + h] = L;
+    xD[(size_t)i * H + h] = D;
+  }
+}
+
+// d(q|k|v) of the SWA projection at position t: the rotary encoding undone
+// on dq (post-rotary gradient) and on the now complete dk_t of the ring slot
+// t mod W; dv_t as is. The slot is cleared for position t - W.
+__global__ void k_bw_qkv_grad(int n, int H, int dh, int W, long t, const float2 *__restrict__ rope,
+                              const float *__restrict__ dq, float *__restrict__ dring_l,
+                              float *__restrict__ dqkv) {
+  const int d = H * dh, half = dh / 2;
+  const long total = (long)n * H * half;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int j = (int)(idx % half), h = (int)((idx / half) % H), i = (int)(idx / half / H);
+    const float2 cs = rope[(size_t)t * half + j];
+    float *dk = dring_l + ((((size_t)i * H + h) * 2 + 0) * W + t % W) * dh;
+    float *dv = dring_l + ((((size_t)i * H + h) * 2 + 1) * W + t % W) * dh;
+    float *o = dqkv + (size_t)i * 3 * d + h * dh;
+    const float qa = dq[(size_t)i * d + h * dh + j], qb = dq[(size_t)i * d + h * dh + j + half];
+    o[j] = qa * cs.x + qb * cs.y;
+    o[j + half] = -qa * cs.y + qb * cs.x;
+    const float ka = dk[j], kb = dk[j + half];
+    o[d + j] = ka * cs.x + kb * cs.y;
+    o[d + j + half] = -ka * cs.y + kb * cs.x;
+    o[2 * d + j] = dv[j];
+    o[2 * d + j + half] = dv[j + half];
+    dk[j] = dk[j + half] = 0.f;
+    dv[j] = dv[j + half] = 0.f;
+  }
+}
+
+// RMSNorm backward of one row (one block per row): with u = h r gamma,
+// dh += r gamma du - h r^3 / d sum_c du_c gamma_c h_c (or dh = ... when
+// `assign`).
+__global__ void k_bw_rms_bwd(int d, const float *__restrict__ h, const float *__restrict__ r,
+                             const float *__restrict__ gamma, const float *__restrict__ du,
+                             float *__restrict__ dh, int assign) {
+  __shared__ float red[32];
+  const size_t o = (size_t)blockIdx.x * d;
+  float sp = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) sp += du[o + c] * gamma[c] * h[o + c];
+  const float S = bw_block_sum(sp, red);
+  const float rr = r[blockIdx.x], k3 = rr * rr * rr * S / d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float g = rr * gamma[c] * du[o + c] - h[o + c] * k3;
+    dh[o + c] = assign ? g : dh[o + c] + g;
+  }
+}
+
+// Column sums over rows: out[c] += sum_i X[i][c] (Y[i][c] r[i] when Y).
+__global__ void k_bw_colsum(int n, int d, const float *__restrict__ X, const float *__restrict__ Y,
+                            const float *__restrict__ r, float *__restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= d) return;
+  float s = 0.f;
+  for (int i = 0; i < n; i++) {
+    float v = X[(size_t)i * d + c];
+    if (Y) v *= Y[(size_t)i * d + c] * r[i];
+    s += v;
+  }
+  out[c] += s;
+}
+
+// FFN activation backward: GELU dz = dact GELU'(z); SwiGLU act = SiLU(z) zb:
+// dz = dact zb SiLU'(z), dzb = dact SiLU(z).
+__global__ void k_bw_act_bwd(long total, int swiglu, const float *__restrict__ z,
+                             const float *__restrict__ zb, const float *__restrict__ dact,
+                             float *__restrict__ dz, float *__restrict__ dzb) {
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const float x = z[idx], g = dact[idx];
+    if (swiglu) {
+      const float sg = sigmoidf_(x);
+      dz[idx] = g * zb[idx] * sg * (1.f + x * (1.f - sg));
+      dzb[idx] = g * x * sg;
+    } else {
+      dz[idx] = g * gelu_grad(x);
+    }
+  }
+}
+
+// Gated merge backward, first half: dgpre = alpha dx s g (1 - g);
+// ds_{t-1} = alpha dx g; de_t += dx.
+__global__ void k_bw_gate_bwd(int n, int d, float alpha, const float *__restrict__ dx,
+                              const float *__restrict__ cat, const float *__restrict__ g,
+                              float *__restrict__ dgpre, float *__restrict__ ds_prev,
+                              float *__restrict__ egrad, int max_len, long t) {
+  const long total = (long)n * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / d), c = (int)(idx % d);
+    const float gg = g[idx], x = dx[idx], sp = cat[(size_t)i * 2 * d + d + c];
+    dgpre[idx] = alpha * x * sp * gg * (1.f - gg);
+    ds_prev[idx] = alpha * x * gg;
+    egrad[((size_t)i * max_len + t) * d + c] += x;
+  }
+}
+
+// Second half: the gate input's gradient dcat = dgpre W_g split into e_t and
+// s_{t-1}.
+__global__ void k_bw_gate_bwd2(int n, int d, const float *__restrict__ dcat,
+                               float *__restrict__ ds_prev, float *__restrict__ egrad, int max_len,
+                               long t) {
+  const long total = (long)n * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / d), c = (int)(idx % d);
+    egrad[((size_t)i * max_len + t) * d + c] += dcat[(size_t)i * 2 * d + c];
+    ds_prev[idx] += dcat[(size_t)i * 2 * d + d + c];
+  }
+}
+
+// ds_t = G_t + the gradient s_t received from step t+1.
+__global__ void k_bw_ds_total(int n, int d, int n_steps, int k, const float *__restrict__ sgrad,
+                              const float *__restrict__ carry, float *__restrict__ ds) {
+  const long total = (long)n * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / d), c = (int)(idx % d);
+    ds[idx] = sgrad[((size_t)i * n_steps + k) * d + c] + carry[idx];
+  }
+}
+
+// Carried gradient of the state between a chunk and its caller: per row
+// [s: d][cache: L][2][W-1][d] (the rlt_get_state cache layout, fp32); cache
+// entry p is position tb - (W-1) + p. in: into the gradient ring and ds;
+// out: from them.
+__global__ void k_bw_carry(int n, int L, int H, int dh, int W, long tb, float *__restrict__ carry,
+                           float *__restrict__ ds, float *__restrict__ dring, int out) {
+  const int d = H * dh, Wm1 = W - 1;
+  const long per = (long)d * (1 + 2L * L * Wm1);
+  const long total = (long)n * per;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx / per);
+    long r = idx % per;
+    if (r < d) {
+      if (out) carry[idx] = ds[(size_t)i * d + r];
+      else ds[(size_t)i * d + r] = carry[idx];
+      continue;
+    }
+    r -= d;
+    const int c = (int)(r % d);
+    const int p = (int)((r / d) % Wm1);
+    const int kv = (int)((r / d / Wm1) % 2);
+    const int l = (int)(r / d / Wm1 / 2);
+    const long pos = tb - Wm1 + p;
+    const int h = c / dh, e = c % dh;
+    float *slot = pos >= 0 ? dring + ((((size_t)l * n + i) * H + h) * 2 + kv) * W * dh +
+                                 (size_t)(pos % W) * dh + e
+                           : nullptr;
+    if (out) carry[idx] = slot ? *slot : 0.f;
+    else if (slot) *slot = carry[idx];
+  }
+}
+
+// ------------------------------------------------- memory gradient pass
+// dK_j = scale sum_t dS_{t,j} q_t and dV_j = sum_t P_{t,j} da_t over the
+// chunk's steps t >= j and the layers reading the group, for memory rows
+// j of one (group, row, head), 64 rows per CTA against 64 steps at a time
+// (the key/value half of a causal attention backward). Saved per (layer,
+// step, row): q, da [d], lse, D [H]. dmem [G][n][t1][2][d] (written).
+template <typename T, int DH> struct BwDmemSmem {
+  static constexpr int BYTES = (4 * 64 * DH + 2 * 64 * 65 + 2 * 64) * 4;
+};
+
+template <typename T, int DH>
+__global__ void __launch_bounds__(256)
+    k_bw_dmem(int n, int H, int G, int L, int n_steps, long t0, int max_seqs, int max_len,
+              const int *__restrict__ ready, const T *__restrict__ mem,
+              const float *__restrict__ xq, const float *__restrict__ xda,
+              const float *__restrict__ xlse, const float *__restrict__ xD, float scale,
+              float *__restrict__ dmem) {
+  extern __shared__ __align__(16) float sm[];
+  float *Kj = sm, *Vj = Kj + 64 * DH, *Qt = Vj + 64 * DH, *At = Qt + 64 * DH;
+  float *Ps = At + 64 * DH, *Ss = Ps + 64 * 65, *ls = Ss + 64 * 65, *Ds = ls + 64;
+  constexpr int EPT = DH / 4;  // head entries per thread in the accumulators
+  const int tid = threadIdx.x;
+  const int j0 = blockIdx.x * 64, h = blockIdx.y, i = blockIdx.z % n, g = blockIdx.z / n;
+  const int d = H * DH;
+  const long t1 = t0 + n_steps;
+  const int seq = ready[i];
+  for (int x = tid; x < 64 * DH; x += 256) {
+    const int jj = x / DH, e = x % DH, j = j0 + jj;
+    const size_t base = ((((size_t)g * max_seqs + seq) * H + h) * 2) * max_len * DH;
+    Kj[x] = j < t1 ? to_f(mem[base + (size_t)j * DH + e]) : 0.f;
+    Vj[x] = j < t1 ? to_f(mem[base + (size_t)max_len * DH + (size_t)j * DH + e]) : 0.f;
+  }
+  const int ojj = tid / 4, oe0 = (tid % 4) * EPT;
+  float dK[EPT], dV[EPT];
+#pragma unroll
+  for (int x = 0; x < EPT; x++) dK[x] = dV[x] = 0.f;
+  const int l_lo = G == 1 ? 0 : g, l_hi = G == 1 ? L : g + 1;
+  const int k_first = (int)(j0 > t0 ? (j0 - t0) / 64 * 64 : 0);
+  for (int l = l_lo; l < l_hi; l++) {
+    for (int k0 = k_first; k0 < n_steps; k0 += 64) {
+      __syncthreads();
+      for (int x = tid; x < 64 * DH; x += 256) {
+        const int kk = x / DH, e = x % DH, k = k0 + kk;
+        const size_t o = (((size_t)l * n_steps + k) * n + i) * d + h * DH + e;
+        Qt[x] = k < n_steps ? xq[o] : 0.f;
+        At[x] = k < n_steps ? xda[o] : 0.f;
+      }
+      if (tid < 64) {
+        const int k = k0 + tid;
+        const size_t o = (((size_t)l * n_steps + k) * n + i) * H + h;
+        ls[tid] = k < n_steps ? xlse[o] : 0.f;
+        Ds[tid] = k < n_steps ? xD[o] : 0.f;
+      }
+      __syncthreads();
+      // P and dS for the 64 x 64 (row j, step k) tile: thread owns row
+      // tid / 4 and steps tid % 4 + 4 m
+      {
+        const int jj = tid / 4, j = j0 + jj;
+        for (int m = 0; m < 16; m++) {
+          const int kk = tid % 4 + 4 * m, k = k0 + kk;
+          const long t = t0 + k;
+          float p = 0.f, ds = 0.f;
+          if (k < n_steps && j <= t && j < t1) {
+            float s = 0.f, dp = 0.f;
+#pragma unroll 8
+            for (int e = 0; e < DH; e++) {
+              s += Kj[jj * DH + e] * Qt[kk * DH + e];
+              dp += Vj[jj * DH + e] * At[kk * DH + e];
+            }
+            p = expf(s * scale - ls[kk]);
+            ds = p * (dp - Ds[kk]);
+          }
+          Ps[jj * 65 + kk] = p;
+          Ss[jj * 65 + kk] = ds;
+        }
+      }
+      __syncthreads();
+      for (int kk = 0; kk < 64; kk++) {
+        const float p = Ps[ojj * 65 + kk], ds = Ss[ojj * 65 + kk] * scale;
+#pragma unroll
+        for (int x = 0; x < EPT; x++) {
+          dK[x] += ds * Qt[kk * DH + oe0 + x];
+          dV[x] += p * At[kk * DH + oe0 + x];
+        }
+      }
+    }
+  }
+  const int j = j0 + ojj;
+  if (j < t1) {
+    float *o = dmem + ((((size_t)g * n + i) * t1 + j) * 2) * d + h * DH + oe0;
+#pragma unroll
+    for (int x = 0; x < EPT; x++) {
+      o[x] = dK[x];
+      o[d + x] = dV[x];
+    }
+  }
+}
+
+// e rows 0..t1-1 of the listed sequences, fp32 [n][t1][d].
+template <typename T>
+__global__ void k_bw_gather_e(int n, int d, long t1, int max_len, const int *__restrict__ ready,
+                              const T *__restrict__ e, float *__restrict__ out) {
+  const long total = (long)n * t1 * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int c = (int)(idx % d);
+    const long j = (idx / d) % t1;
+    const int i = (int)(idx / d / t1);
+    out[idx] = to_f(e[((size_t)ready[i] * max_len + j) * d + c]);
+  }
+}
+
+// egrad[i][j] += de[i][j] for j < t1 (egrad [n][max_len][d], de [n][t1][d]).
+__global__ void k_bw_add_e(int n, int d, long t1, int max_len, const float *__restrict__ de,
+                           float *__restrict__ egrad) {
+  const long total = (long)n * t1 * d;
+  for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long)gridDim.x * blockDim.x) {
+    const int c = (int)(idx % d);
+    const long j = (idx / d) % t1;
+    const int i = (int)(idx / d / t1);
+    egrad[((size_t)i * max_len + j) * d + c] += de[idx];
+  }
+}
+
+}  // namespace rlt

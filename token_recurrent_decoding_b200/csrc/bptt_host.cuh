@@ -1,0 +1,338 @@
+// Host side of the decoder's backpropagation through time (kernels in
+// bptt.cuh). Part of the rlt_api.cu translation unit: it drives the model's
+// own step (enqueue_step) for the recorded forward and reads the arena's
+// encoder outputs, memory and rotary table.
+#pragma once
+
+// Workspace of one rlt_backward call: n rows, NS steps. Offsets in bytes.
+struct BwLayout {
+  size_t s_hist, kv_hist, step, dring, xq, xda, xlse, xD, dmem, e32, de, total;
+  size_t step_floats;
+  int P;  // recorded positions t0 - (W-1) .. t1 - 1
+};
+
+size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes ? bytes : 1);
+    return o;
+  };
+  const size_t d = c.d, F = c.ffn_dim, H = c.n_heads, L = c.n_dec_layers, W = c.window;
+  const size_t N = n, S = NS, es = elem_size(&c);
+  B->P = (int)(S + W - 1);
+  B->s_hist = take((S + 1) * N * d * 4);
+  B->kv_hist = take(L * N * H * 2 * B->P * (d / H) * es);
+  // one step's activations and gradient scratch (see BwStep)
+  B->step_floats = N * (2 * d + 2 * d + (3 * L + 1) * d + 3 * L * d + 4 * L * d + 3 * L * F +
+                        3 * d + d) +
+                   N * ((3 * L + 1) + 2 * L * H) +
+                   N * (d + std::max(std::max(3 * d, F), 2 * d) + 2 * F + d + 3 * d + d + d +
+                        d + d + d);
+  B->step = take(B->step_floats * 4);
+  B->dring = take(L * N * H * 2 * W * (d / H) * 4);
+  B->xq = take(L * S * N * d * 4);
+  B->xda = take(L * S * N * d * 4);
+  B->xlse = take(L * S * N * H * 4);
+  B->xD = take(L * S * N * H * 4);
+  B->dmem = take((size_t)c.mem_groups * N * c.max_len * 2 * d * 4);
+  B->e32 = take(N * c.max_len * d * 4);
+  B->de = take(N * c.max_len * d * 4);
+  B->total = off;
+  return off;
+}
+
+// Pointers into one step's region.
+struct BwStep {
+  float *cat, *gpre, *gs, *h, *u, *q1, *a1, *qx, *a2, *z, *zb, *act, *qkv, *ulast;
+  float *r, *lse1, *lse2;
+  float *dh, *dtmp, *dz, *dzb, *dq, *dqkv, *du, *dgpre, *ds, *dcarry;
+  BwStep(float *base, const rlt_config &c, int n) {
+    const size_t d = c.d, F = c.ffn_dim, H = c.n_heads, L = c.n_dec_layers, N = n;
+    float *p = base;
+    auto take = [&](size_t cnt) {
+      float *o = p;
+      p += cnt;
+      return o;
+    };
+    cat = take(N * 2 * d);
+    gpre = take(N * d);
+    gs = take(N * d);
+    h = take((3 * L + 1) * N * d);  // per layer: h1, h2, h3; then the final residual
+    u = take(3 * L * N * d);
+    q1 = take(L * N * d);
+    a1 = take(L * N * d);
+    qx = take(L * N * d);
+    a2 = take(L * N * d);
+    z = take(L * N * F);
+    zb = take(L * N * F);
+    act = take(L * N * F);
+    qkv = take(N * 3 * d);
+    ulast = take(N * d);
+    r = take((3 * L + 1) * N);
+    lse1 = take(L * N * H);
+    lse2 = take(L * N * H);
+    dh = take(N * d);
+    dtmp = take(N * std::max(std::max(3 * d, F), 2 * d));
+    dz = take(N * F);
+    dzb = take(N * F);
+    dq = take(N * d);
+    dqkv = take(N * 3 * d);
+    du = take(N * d);
+    dgpre = take(N * d);
+    ds = take(N * d);
+    dcarry = take(N * d);
+  }
+};
+
+template <bool AK, bool BK, typename TA, typename TB>
+cudaError_t bw_gemm(int m, int n, int k, const TA *A, long lda, const TB *B, long ldb, float *C,
+                    long ldc, bool acc, cudaStream_t st) {
+  if (m <= 0 || n <= 0) return cudaSuccess;
+  dim3 grid((n + 63) / 64, (m + 63) / 64);
+  k_bw_gemm<TA, TB, AK, BK><<<grid, 256, 0, st>>>(m, n, k, A, lda, B, ldb, C, ldc, acc ? 1 : 0);
+  return cudaGetLastError();
+}
+
+inline int bw_blocks(long total) { return (int)std::min<long>((total + 255) / 256, 148L * 16); }
+
+bool bw_grads_complete(const rlt_config &c, const rlt_grads *g) {
+  bool ok = g && g->gate_w && g->gate_b && g->sstar && g->dec_lnf;
+  for (int l = 0; ok && l < c.n_dec_layers; l++) {
+    ok = g->dec_ln1[l] && g->dec_wqkv[l] && g->dec_wo[l] && g->dec_ln2[l] && g->dec_wqx[l] &&
+         g->dec_wox[l] && g->dec_ln3[l] && g->dec_w1[l] && g->dec_w2[l];
+    if (c.ffn_kind == RLT_SWIGLU) ok = ok && g->dec_wb[l];
+  }
+  for (int q = 0; ok && q < c.mem_groups; q++) ok = g->mem_wk[q] && g->mem_wv[q];
+  return ok;
+}
+
+// Forward of the chunk on the model's own step kernels, recording s_t and
+// every layer's (k_t, v_t); then the reverse traversal; then the memory
+// gradient and its projection into e.
+template <typename T, int DH>
+cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float *sgrad,
+                    const float *carry_in, float *carry_out, float *egrad, const rlt_grads *gr,
+                    void *ws, cudaStream_t st) {
+  const rlt_config &c = M->cfg;
+  const Layout &L = M->L;
+  const int d = c.d, H = c.n_heads, F = c.ffn_dim, LD = c.n_dec_layers, W = c.window,
+            Wm1 = W - 1, G = c.mem_groups;
+  const bool swiglu = c.ffn_kind == RLT_SWIGLU;
+  const long t0 = M->t_dec[ids[0]], t1 = t0 + NS;
+  const float scale = 1.0f / sqrtf((float)DH);
+  BwLayout B;
+  bw_layout(c, n, NS, &B);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  float *s_hist = reinterpret_cast<float *>(base + B.s_hist);
+  T *kv_hist = reinterpret_cast<T *>(base + B.kv_hist);
+  float *dring = reinterpret_cast<float *>(base + B.dring);
+  float *xq = reinterpret_cast<float *>(base + B.xq), *xda = reinterpret_cast<float *>(base + B.xda);
+  float *xlse = reinterpret_cast<float *>(base + B.xlse), *xD = reinterpret_cast<float *>(base + B.xD);
+  float *dmem = reinterpret_cast<float *>(base + B.dmem);
+  float *e32 = reinterpret_cast<float *>(base + B.e32), *de = reinterpret_cast<float *>(base + B.de);
+  BwStep S(reinterpret_cast<float *>(base + B.step), c, n);
+  const int *ready = M->at<int>(L.ready);
+  const T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem), *e = M->at<T>(L.e);
+  const float *s_arena = M->at<float>(L.s);
+  const float2 *rope = M->at<float2>(L.rope);
+  const size_t nd = (size_t)n * d;
+
+  // ---- forward of the chunk, recorded
+  std::vector<int32_t> idv(ids, ids + n);
+  RLT_TRY(cudaMemcpyAsync(M->at<int>(L.ready), idv.data(), 4 * n, cudaMemcpyHostToDevice, st));
+  k_bw_hist_init<T><<<bw_blocks((long)LD * n * 2 * d * std::max(Wm1, 1) + (long)nd), 256, 0, st>>>(
+      n, ready, ring, s_arena, LD, H, DH, W, c.max_seqs, t0, B.P, kv_hist, s_hist);
+  RLT_TRY(cudaGetLastError());
+  for (int k = 0; k < NS; k++) {
+    RLT_TRY(enqueue_step(M, step_info(M, idv.data(), n), st));
+    advance(M, idv.data(), n);
+    k_bw_hist_step<T><<<bw_blocks((long)LD * n * 2 * d), 256, 0, st>>>(
+        n, ready, ring, s_arena, LD, H, DH, W, c.max_seqs, t0 + k, Wm1 + k, B.P, kv_hist,
+        s_hist + (size_t)(k + 1) * nd);
+    RLT_TRY(cudaGetLastError());
+  }
+
+  // ---- reverse traversal
+  RLT_TRY(cudaMemsetAsync(dring, 0, (size_t)LD * n * 2 * d * W * 4, st));
+  RLT_TRY(cudaMemsetAsync(S.dcarry, 0, nd * 4, st));
+  if (carry_in) {
+    k_bw_carry<<<bw_blocks((long)n * d * (1 + 2L * LD * Wm1)), 256, 0, st>>>(
+        n, LD, H, DH, W, t1, const_cast<float *>(carry_in), S.dcarry, dring, 0);
+    RLT_TRY(cudaGetLastError());
+  }
+  const int attn_blocks = (n * H * 32 + 127) / 128;
+  auto hbuf = [&](int l, int which) { return S.h + ((size_t)3 * l + which) * nd; };
+  auto ubuf = [&](int l, int which) { return S.u + ((size_t)3 * l + which) * nd; };
+  auto rbuf = [&](int l, int which) { return S.r + ((size_t)3 * l + which) * n; };
+  for (int k = NS - 1; k >= 0; k--) {
+    const long t = t0 + k;
+    const float *s_prev = s_hist + (size_t)k * nd;
+    // recompute the forward of step t
+    k_bw_gate_cat<T><<<bw_blocks(2 * (long)nd), 256, 0, st>>>(n, d, ready, e, c.max_len, t, s_prev,
+                                                              S.cat);
+    if (c.alpha != 0.0f)
+      RLT_TRY((bw_gemm<true, true>(n, d, 2 * d, S.cat, 2 * d, (const T *)M->w.gate_w, 2 * d, S.gpre,
+                                   d, false, st)));
+    else
+      RLT_TRY(cudaMemsetAsync(S.gpre, 0, nd * 4, st));
+    k_bw_gate_fwd<<<bw_blocks(nd), 256, 0, st>>>(n, d, S.gpre, (const float *)M->w.gate_b, S.cat,
+                                                 c.alpha, S.gs, hbuf(0, 0));
+    for (int l = 0; l < LD; l++) {
+      const int g = G == 1 ? 0 : l;
+      float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2), *hn = hbuf(l + 1, 0);
+      float *u1 = ubuf(l, 0), *u2 = ubuf(l, 1), *u3 = ubuf(l, 2);
+      float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
+      float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
+            *act = S.act + (size_t)l * n * F;
+      k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h1, (const float *)M->w.dec_ln1[l], u1,
+                                      rbuf(l, 0));
+      RLT_TRY((bw_gemm<true, true>(n, 3 * d, d, u1, d, W_<T>::qkv(M, l), d, S.qkv, 3 * d, false,
+                                   st)));
+      k_bw_rope_q<<<bw_blocks((long)n * d / 2), 256, 0, st>>>(n, H, DH, t, rope, S.qkv, q1);
+      BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
+      const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
+      k_bw_attn_fwd<T, DH><<<attn_blocks, 128, 0, st>>>(n, H, swa, p_lo, p_hi, scale, q1, a1,
+                                                        S.lse1 + (size_t)l * n * H);
+      RLT_TRY(cudaMemcpyAsync(h2, h1, nd * 4, cudaMemcpyDeviceToDevice, st));
+      RLT_TRY((bw_gemm<true, true>(n, d, d, a1, d, W_<T>::o(M, l), d, h2, d, true, st)));
+      k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h2, (const float *)M->w.dec_ln2[l], u2,
+                                      rbuf(l, 1));
+      RLT_TRY((bw_gemm<true, true>(n, d, d, u2, d, (const T *)M->w.dec_wqx[l], d, qx, d, false,
+                                   st)));
+      BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
+      k_bw_attn_fwd<T, DH><<<attn_blocks, 128, 0, st>>>(n, H, xk, 0, (int)t, scale, qx, a2,
+                                                        S.lse2 + (size_t)l * n * H);
+      RLT_TRY(cudaMemcpyAsync(h3, h2, nd * 4, cudaMemcpyDeviceToDevice, st));
+      RLT_TRY((bw_gemm<true, true>(n, d, d, a2, d, (const T *)M->w.dec_wox[l], d, h3, d, true,
+                                   st)));
+      k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h3, (const float *)M->w.dec_ln3[l], u3,
+                                      rbuf(l, 2));
+      RLT_TRY((bw_gemm<true, true>(n, F, d, u3, d, W_<T>::w1(M, l), d, z, F, false, st)));
+      if (swiglu)
+        RLT_TRY((bw_gemm<true, true>(n, F, d, u3, d, W_<T>::wb(M, l), d, zb, F, false, st)));
+      k_bw_act_fwd<<<bw_blocks((long)n * F), 256, 0, st>>>((long)n * F, swiglu, z, zb, act);
+      RLT_TRY(cudaMemcpyAsync(hn, h3, nd * 4, cudaMemcpyDeviceToDevice, st));
+      RLT_TRY((bw_gemm<true, true>(n, d, F, act, F, W_<T>::w2(M, l), F, hn, d, true, st)));
+    }
+    float *rf = S.r + (size_t)3 * LD * n;
+    k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, hbuf(LD, 0), (const float *)M->w.dec_lnf,
+                                    S.ulast, rf);
+    RLT_TRY(cudaGetLastError());
+
+    // differentiate step t: s_t = RMSNorm_f(h_L)
+    k_bw_ds_total<<<bw_blocks(nd), 256, 0, st>>>(n, d, NS, k, sgrad, S.dcarry, S.ds);
+    k_bw_rms_bwd<<<n, 256, 0, st>>>(d, hbuf(LD, 0), rf, (const float *)M->w.dec_lnf, S.ds, S.dh,
+                                    1);
+    k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.ds, hbuf(LD, 0), rf, gr->dec_lnf);
+    for (int l = LD - 1; l >= 0; l--) {
+      float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2);
+      float *u1 = ubuf(l, 0), *u2 = ubuf(l, 1), *u3 = ubuf(l, 2);
+      float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
+      float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
+            *act = S.act + (size_t)l * n * F;
+      // FFN: h_out = h3 + W2 act(W1 u3)
+      RLT_TRY((bw_gemm<true, false>(n, F, d, S.dh, d, W_<T>::w2(M, l), F, S.dtmp, F, false, st)));
+      RLT_TRY((bw_gemm<false, false>(d, F, n, S.dh, d, act, F, gr->dec_w2[l], F, true, st)));
+      k_bw_act_bwd<<<bw_blocks((long)n * F), 256, 0, st>>>((long)n * F, swiglu, z, zb, S.dtmp,
+                                                           S.dz, S.dzb);
+      RLT_TRY((bw_gemm<false, false>(F, d, n, S.dz, F, u3, d, gr->dec_w1[l], d, true, st)));
+      RLT_TRY((bw_gemm<true, false>(n, d, F, S.dz, F, W_<T>::w1(M, l), d, S.du, d, false, st)));
+      if (swiglu) {
+        RLT_TRY((bw_gemm<false, false>(F, d, n, S.dzb, F, u3, d, gr->dec_wb[l], d, true, st)));
+        RLT_TRY((bw_gemm<true, false>(n, d, F, S.dzb, F, W_<T>::wb(M, l), d, S.du, d, true, st)));
+      }
+      k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h3, rbuf(l, 2), (const float *)M->w.dec_ln3[l], S.du,
+                                      S.dh, 0);
+      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.du, h3, rbuf(l, 2), gr->dec_ln3[l]);
+      // cross-attention: h3 = h2 + W_ox attn(W_qx u2, M<=t)
+      const int g = G == 1 ? 0 : l;
+      RLT_TRY((bw_gemm<true, false>(n, d, d, S.dh, d, (const T *)M->w.dec_wox[l], d, S.dtmp, d,
+                                    false, st)));
+      RLT_TRY((bw_gemm<false, false>(d, d, n, S.dh, d, a2, d, gr->dec_wox[l], d, true, st)));
+      BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
+      const size_t xo = ((size_t)l * NS + k) * nd, xs = ((size_t)l * NS + k) * n * H;
+      k_bw_attn_bwd<T, DH><<<attn_blocks, 128, 0, st>>>(
+          n, H, xk, 0, (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, S.dtmp, S.dq, nullptr,
+          W, 0, xq + xo, xda + xo, xlse + xs, xD + xs);
+      RLT_TRY((bw_gemm<false, false>(d, d, n, S.dq, d, u2, d, gr->dec_wqx[l], d, true, st)));
+      RLT_TRY((bw_gemm<true, false>(n, d, d, S.dq, d, (const T *)M->w.dec_wqx[l], d, S.du, d,
+                                    false, st)));
+      k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h2, rbuf(l, 1), (const float *)M->w.dec_ln2[l], S.du,
+                                      S.dh, 0);
+      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.du, h2, rbuf(l, 1), gr->dec_ln2[l]);
+      // SWA: h2 = h1 + W_o attn(q_t over the window); k_t, v_t enter the cache
+      RLT_TRY((bw_gemm<true, false>(n, d, d, S.dh, d, W_<T>::o(M, l), d, S.dtmp, d, false, st)));
+      RLT_TRY((bw_gemm<false, false>(d, d, n, S.dh, d, a1, d, gr->dec_wo[l], d, true, st)));
+      BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
+      const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
+      k_bw_attn_bwd<T, DH><<<attn_blocks, 128, 0, st>>>(
+          n, H, swa, p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H, S.dtmp, S.dq, dring,
+          W, t0 - Wm1, nullptr, nullptr, nullptr, nullptr);
+      k_bw_qkv_grad<<<bw_blocks((long)n * d / 2), 256, 0, st>>>(
+          n, H, DH, W, t, rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv);
+      RLT_TRY((bw_gemm<false, false>(3 * d, d, n, S.dqkv, 3 * d, u1, d, gr->dec_wqkv[l], d, true,
+                                     st)));
+      RLT_TRY((bw_gemm<true, false>(n, d, 3 * d, S.dqkv, 3 * d, W_<T>::qkv(M, l), d, S.du, d,
+                                    false, st)));
+      k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h1, rbuf(l, 0), (const float *)M->w.dec_ln1[l], S.du,
+                                      S.dh, 0);
+      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.du, h1, rbuf(l, 0), gr->dec_ln1[l]);
+    }
+    // gated merge: x = e_t + alpha sigmoid(W_g [e_t; s_{t-1}] + b_g) s_{t-1}
+    k_bw_gate_bwd<<<bw_blocks(nd), 256, 0, st>>>(n, d, c.alpha, S.dh, S.cat, S.gs, S.dgpre,
+                                                 S.dcarry, egrad, c.max_len, t);
+    if (c.alpha != 0.0f) {
+      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.dgpre, nullptr, nullptr, gr->gate_b);
+      RLT_TRY((bw_gemm<false, false>(d, 2 * d, n, S.dgpre, d, S.cat, 2 * d, gr->gate_w, 2 * d,
+                                     true, st)));
+      RLT_TRY((bw_gemm<true, false>(n, 2 * d, d, S.dgpre, d, (const T *)M->w.gate_w, 2 * d,
+                                    S.dtmp, 2 * d, false, st)));
+      k_bw_gate_bwd2<<<bw_blocks(nd), 256, 0, st>>>(n, d, S.dtmp, S.dcarry, egrad, c.max_len, t);
+    }
+    RLT_TRY(cudaGetLastError());
+  }
+  // the state entering the chunk
+  if (carry_out) {
+    k_bw_carry<<<bw_blocks((long)n * d * (1 + 2L * LD * Wm1)), 256, 0, st>>>(
+        n, LD, H, DH, W, t0, carry_out, S.dcarry, dring, 1);
+    RLT_TRY(cudaGetLastError());
+  }
+  if (t0 == 0)  // s_{-1} is the learned start state s*
+    k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.dcarry, nullptr, nullptr, gr->sstar);
+
+  // ---- memory rows: dK, dV from the saved cross-attention terms, then
+  // K^g = W_mk^g e, V^g = W_mv^g e differentiated into e and the projections
+  constexpr int dm_smem = BwDmemSmem<T, DH>::BYTES;
+  RLT_TRY(ensure_smem_limit(k_bw_dmem<T, DH>, dm_smem));
+  k_bw_dmem<T, DH><<<dim3((unsigned)((t1 + 63) / 64), H, n * G), 256, dm_smem, st>>>(
+      n, H, G, LD, NS, t0, c.max_seqs, c.max_len, ready, mem, xq, xda, xlse, xD, scale, dmem);
+  k_bw_gather_e<T><<<bw_blocks((long)n * t1 * d), 256, 0, st>>>(n, d, t1, c.max_len, ready, e, e32);
+  RLT_TRY(cudaGetLastError());
+  const int rows = (int)(n * t1);
+  for (int g = 0; g < G; g++) {
+    const float *dk = dmem + (size_t)g * rows * 2 * d, *dv = dk + d;
+    RLT_TRY((bw_gemm<true, false>(rows, d, d, dk, 2 * d, (const T *)M->w.mem_wk[g], d, de, d,
+                                  g > 0, st)));
+    RLT_TRY((bw_gemm<true, false>(rows, d, d, dv, 2 * d, (const T *)M->w.mem_wv[g], d, de, d,
+                                  true, st)));
+    RLT_TRY((bw_gemm<false, false>(d, d, rows, dk, 2 * d, e32, d, gr->mem_wk[g], d, true, st)));
+    RLT_TRY((bw_gemm<false, false>(d, d, rows, dv, 2 * d, e32, d, gr->mem_wv[g], d, true, st)));
+  }
+  k_bw_add_e<<<bw_blocks((long)rows * d), 256, 0, st>>>(n, d, t1, c.max_len, de, egrad);
+  return cudaGetLastError();
+}
+
+cudaError_t bw_dispatch(rlt_model *M, const int32_t *ids, int n, int NS, const float *sgrad,
+                        const float *carry_in, float *carry_out, float *egrad,
+                        const rlt_grads *gr, void *ws, cudaStream_t st) {
+#define RLT_BW(T, DH) bw_impl<T, DH>(M, ids, n, NS, sgrad, carry_in, carry_out, egrad, gr, ws, st)
+  const bool b = M->cfg.dtype == RLT_BF16;
+  switch (M->cfg.head_dim) {
+    case 16: return b ? RLT_BW(bf16, 16) : RLT_BW(float, 16);
+    case 32: return b ? RLT_BW(bf16, 32) : RLT_BW(float, 32);
+    case 64: return b ? RLT_BW(bf16, 64) : RLT_BW(float, 64);
+    default: return b ? RLT_BW(bf16, 128) : RLT_BW(float, 128);
+  }
+#undef RLT_BW
+}

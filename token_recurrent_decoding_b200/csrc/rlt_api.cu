@@ -25,6 +25,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_dec.cuh"
 #include "step_fused.cuh"
+#include "bptt.cuh"
 
 using namespace rlt;
 
@@ -1863,6 +1864,8 @@ bool same_model(const rlt_snapshot_header &a, const rlt_snapshot_header &b) {
          a.rms_eps == b.rms_eps && a.rope_theta == b.rope_theta;
 }
 
+#include "bptt_host.cuh"
+
 }  // namespace
 
 // ===================================================================== C ABI
@@ -2143,6 +2146,31 @@ RLT_API int rlt_run_sequence(rlt_model *M, const int32_t *ids, int n, int n_step
     advance(M, idv.data(), n);
   }
   return cuda_status(e);
+}
+
+RLT_API size_t rlt_backward_workspace_bytes(const rlt_config *cfg, int n, int n_steps) {
+  if (check_config(cfg) != RLT_OK || n < 1 || n_steps < 1) return 0;
+  BwLayout B;
+  return bw_layout(*cfg, n, n_steps, &B);
+}
+
+RLT_API int rlt_backward(rlt_model *M, const int32_t *ids, int n, int n_steps,
+                         const float *sgrad, const float *carry_in, float *carry_out,
+                         float *egrad, const rlt_grads *grads, void *ws, size_t ws_bytes,
+                         rlt_stream stream) {
+  if (!M || n < 1 || n_steps < 1 || !sgrad || !egrad || !ws || ((uintptr_t)ws & 255))
+    return RLT_ERR_INVALID_ARG;
+  int rc = check_batch(M, ids, n, n_steps);
+  if (rc != RLT_OK) return rc;
+  for (int i = 1; i < n; i++)
+    if (M->t_dec[ids[i]] != M->t_dec[ids[0]]) return RLT_ERR_INVALID_ARG;
+  if (!bw_grads_complete(M->cfg, grads)) return RLT_ERR_INVALID_ARG;
+  BwLayout B;
+  if (ws_bytes < bw_layout(M->cfg, n, n_steps, &B)) return RLT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  M->last_stream = st;
+  return cuda_status(bw_dispatch(M, ids, n, n_steps, sgrad, carry_in, carry_out, egrad, grads,
+                                 ws, st));
 }
 
 RLT_API int rlt_decoder_parallel(rlt_model *M, const int32_t *ids, int n, int n_steps,

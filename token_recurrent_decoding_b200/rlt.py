@@ -56,6 +56,12 @@ class rlt_weights(C.Structure):
                 + [("dec_lnf", C.c_void_p)])
 
 
+class rlt_grads(C.Structure):
+    _fields_ = ([(n, C.c_void_p) for n in ("gate_w", "gate_b", "sstar", "dec_lnf")]
+                + [(n, C.c_void_p * MAX_LAYERS) for n in _DEC]
+                + [("mem_wk", C.c_void_p * MAX_LAYERS), ("mem_wv", C.c_void_p * MAX_LAYERS)])
+
+
 K_XATTN, K_SWA, K_GEMM, K_OTHER, K_ENC, K_STEP = range(6)
 FAULT_NONE, FAULT_SKIP_ATTN_PRODUCER = 0, 1
 STEP_CHAIN, STEP_FUSED = 0, 1
@@ -84,6 +90,9 @@ def _declare(lib):
     lib.rlt_decoder_step.argtypes = [P, P, I, P]
     lib.rlt_run_sequence.argtypes = [P, P, I, I, P]
     lib.rlt_decoder_parallel.argtypes = [P, P, I, I, P, P]
+    lib.rlt_backward_workspace_bytes.argtypes = [P, I, I]
+    lib.rlt_backward_workspace_bytes.restype = C.c_size_t
+    lib.rlt_backward.argtypes = [P, P, I, I, P, P, P, P, P, P, C.c_size_t, P]
     lib.rlt_run_ragged.argtypes = [P, P, P, I, P]
     lib.rlt_plan_ragged.argtypes = [P, I, P, P, I, C.POINTER(I)]
     lib.rlt_get_state.argtypes = [P, I, P, P, C.POINTER(C.c_int64), P]
@@ -328,6 +337,92 @@ class Model:
             ptr = C.c_void_p(s_all.data_ptr())
         _check(_lib().rlt_decoder_parallel(self._h, _p(ids), ids.shape[0], int(n_steps), ptr,
                                            self._st(stream)), "rlt_decoder_parallel")
+
+    def grad_shapes(self) -> Dict[str, tuple]:
+        """Name (the weight generator's) -> shape of every gradient rlt_backward
+        accumulates."""
+        c = self.cfg
+        d, F = c.d, c.ffn_dim
+        sw = c.ffn_kind == SWIGLU
+        out = {"gate.w": (d, 2 * d), "gate.b": (d,), "sstar": (d,), "dec.lnf": (d,)}
+        for l in range(c.n_dec):
+            out[f"dec.{l}.ln1"] = (d,)
+            out[f"dec.{l}.wqkv"] = (3 * d, d)
+            out[f"dec.{l}.wo"] = (d, d)
+            out[f"dec.{l}.ln2"] = (d,)
+            out[f"dec.{l}.wqx"] = (d, d)
+            out[f"dec.{l}.wox"] = (d, d)
+            out[f"dec.{l}.ln3"] = (d,)
+            out[f"dec.{l}.wa" if sw else f"dec.{l}.w1"] = (F, d)
+            if sw:
+                out[f"dec.{l}.wb"] = (F, d)
+            out[f"dec.{l}.w2"] = (d, F)
+        for g in range(c.mem_groups):
+            out[f"mem.{g}.wk"] = (d, d)
+            out[f"mem.{g}.wv"] = (d, d)
+        return out
+
+    def carry_floats(self) -> int:
+        c = self.cfg
+        return c.d * (1 + 2 * c.n_dec * (c.window - 1))
+
+    def backward_workspace_bytes(self, n: int, n_steps: int) -> int:
+        return int(_lib().rlt_backward_workspace_bytes(C.byref(self._c), int(n), int(n_steps)))
+
+    def backward(self, seq_ids, sgrad, grads=None, egrad=None, carry_in=None, carry_out=True,
+                 workspace=None, stream=None):
+        """Backpropagation through time over the next sgrad.shape[1] positions of
+        the listed sequences (rlt_backward): runs their forward, then the
+        reverse traversal. sgrad: fp32 device [n][n_steps][d] = dL/ds_t.
+        grads (name -> fp32 device tensor, accumulated) and egrad ([n][max_len][d],
+        accumulated) are allocated zeroed when None. Returns (grads, egrad,
+        carry_out or None)."""
+        torch = self.torch
+        ids = _i32(seq_ids)
+        n, n_steps = ids.shape[0], int(sgrad.shape[1])
+        c = self.cfg
+        assert sgrad.is_cuda and sgrad.dtype == torch.float32 and sgrad.is_contiguous()
+        assert tuple(sgrad.shape) == (n, n_steps, c.d)
+        dev = self.device
+        if grads is None:
+            grads = {k: torch.zeros(v, dtype=torch.float32, device=dev)
+                     for k, v in self.grad_shapes().items()}
+        if egrad is None:
+            egrad = torch.zeros((n, self.max_len, c.d), dtype=torch.float32, device=dev)
+        g = rlt_grads()
+        sw = c.ffn_kind == SWIGLU
+        for k, fld in (("gate.w", "gate_w"), ("gate.b", "gate_b"), ("sstar", "sstar"),
+                       ("dec.lnf", "dec_lnf")):
+            setattr(g, fld, grads[k].data_ptr())
+        for l in range(c.n_dec):
+            for k, fld in (("ln1", "dec_ln1"), ("wqkv", "dec_wqkv"), ("wo", "dec_wo"),
+                           ("ln2", "dec_ln2"), ("wqx", "dec_wqx"), ("wox", "dec_wox"),
+                           ("ln3", "dec_ln3"), ("wa" if sw else "w1", "dec_w1"),
+                           ("w2", "dec_w2")):
+                getattr(g, fld)[l] = grads[f"dec.{l}.{k}"].data_ptr()
+            if sw:
+                g.dec_wb[l] = grads[f"dec.{l}.wb"].data_ptr()
+        for q in range(c.mem_groups):
+            g.mem_wk[q] = grads[f"mem.{q}.wk"].data_ptr()
+            g.mem_wv[q] = grads[f"mem.{q}.wv"].data_ptr()
+        cin = None
+        if carry_in is not None:
+            assert tuple(carry_in.shape) == (n, self.carry_floats())
+            assert carry_in.dtype == torch.float32 and carry_in.is_contiguous()
+            cin = C.c_void_p(carry_in.data_ptr())
+        cout = None
+        if carry_out:
+            cout_t = torch.empty((n, self.carry_floats()), dtype=torch.float32, device=dev)
+            cout = C.c_void_p(cout_t.data_ptr())
+        if workspace is None:
+            workspace = torch.empty(self.backward_workspace_bytes(n, n_steps),
+                                    dtype=torch.uint8, device=dev)
+        _check(_lib().rlt_backward(self._h, _p(ids), n, n_steps, C.c_void_p(sgrad.data_ptr()),
+                                   cin, cout, C.c_void_p(egrad.data_ptr()), C.byref(g),
+                                   C.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                   self._st(stream)), "rlt_backward")
+        self._bw_keep = (workspace, grads, egrad, carry_in)
+        return grads, egrad, (cout_t if carry_out else None)
 
     def run_ragged(self, seq_ids, steps, stream=None):
         ids, st = _i32(seq_ids), _i32(steps)
