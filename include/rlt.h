@@ -562,6 +562,12 @@ RLT_API int rlt_poll_device_error(rlt_model *model);
 /* Static description of a status code (never NULL). */
 RLT_API const char *rlt_status_string(int status);
 
+/* Host only. The first CUDA error the calling thread met inside the library
+ * since the previous call (after an RLT_ERR_CUDA): returns its cudaError_t
+ * value (0 if none) and writes its name and the library source line that saw
+ * it into buf (len bytes, may be NULL). Reading it clears it. */
+RLT_API int rlt_last_cuda_error(char *buf, size_t len);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,7 +22,12 @@
 // key/value half of a causal attention backward, then pushed through the
 // memory projection into e.
 //
-// Everything here computes in fp32 (weights read in the model dtype).
+// Arithmetic: the projections of bf16 models run on the tcgen05 tensor cores
+// (decode GEMMs for the recomputed forward and the activation gradients, with
+// the weights transposed once per call; tile GEMMs for the weight gradients,
+// reduced over the batch rows), their operands rounded to bf16 and fp32
+// accumulation, as the forward does; fp32 models use the SIMT GEMM below.
+// Attention, norms, activations and every accumulation are fp32.
 #pragma once
 
 #include "common.cuh"
@@ -82,6 +87,94 @@ __global__ void __launch_bounds__(256)
       float *p = C + (size_t)r * ldc + col;
       *p = acc ? *p + c[i][j] : c[i][j];
     }
+  }
+}
+
+// ------------------------------------------ tensor-core forms (bf16 models)
+// Decode-GEMM epilogues (k_gemm_dec / k_gemm_dec_sw): out = base + C, and
+// out += C. Every output element has one owner after the split-K reduction.
+struct EpiAddF32Dec {
+  static constexpr int kKind = kPair;
+  static constexpr bool kRowScale = false;
+  RowScaleIn rsi;  // unused
+  const float *base;
+  float *out;
+  int ld;
+  __device__ void pair(int m, int n, float a, float b, float) const {
+    const float2 x = *reinterpret_cast<const float2 *>(base + (size_t)m * ld + n);
+    *reinterpret_cast<float2 *>(out + (size_t)m * ld + n) = make_float2(x.x + a, x.y + b);
+  }
+};
+
+struct EpiAccF32Dec {
+  static constexpr int kKind = kPair;
+  static constexpr bool kRowScale = false;
+  RowScaleIn rsi;  // unused
+  float *out;
+  int ld;
+  __device__ void pair(int m, int n, float a, float b, float) const {
+    float2 *p = reinterpret_cast<float2 *>(out + (size_t)m * ld + n);
+    const float2 x = *p;
+    *p = make_float2(x.x + a, x.y + b);
+  }
+};
+
+// Weight-gradient accumulation of the tile GEMM (k_gemm_tc / k_gemm_tcp):
+// out[m][n .. n+15] += C.
+struct EpiAccF32 {
+  float *out;
+  int ld;
+  __device__ void operator()(int m, int n, float a, float b) const {
+    float2 *p = reinterpret_cast<float2 *>(out + (size_t)m * ld + n);
+    const float2 x = *p;
+    *p = make_float2(x.x + a, x.y + b);
+  }
+  __device__ void vec16(int m, int n, const float *v) const {
+    float *p = out + (size_t)m * ld + n;
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float2 x = *reinterpret_cast<const float2 *>(p + i);
+      *reinterpret_cast<float2 *>(p + i) = make_float2(x.x + v[i], x.y + v[i + 1]);
+    }
+  }
+};
+
+// bf16 operands of the tensor-core GEMMs from an fp32 [n][ld] matrix (its
+// first K columns): row-major Xb [n_pad][K] and/or transposed XT [K][n_pad],
+// rows n .. n_pad-1 zero. 32 x 32 tiles through shared memory, so both
+// layouts are written with contiguous runs.
+__global__ void k_bw_pack(int n, int n_pad, int K, const float *__restrict__ X, long ld,
+                          bf16 *__restrict__ Xb, bf16 *__restrict__ XT) {
+  __shared__ float tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int y = ty; y < 32; y += 8) {
+    const int r = r0 + y, c = c0 + tx;
+    float v = (r < n && c < K) ? X[(size_t)r * ld + c] : 0.f;
+    tile[y][tx] = v;
+    if (Xb && r < n_pad && c < K) Xb[(size_t)r * K + c] = __float2bfloat16_rn(v);
+  }
+  if (!XT) return;
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int c = c0 + y, r = r0 + tx;
+    if (c < K && r < n_pad) XT[(size_t)c * n_pad + r] = __float2bfloat16_rn(tile[tx][y]);
+  }
+}
+
+// WT [K][N] = W^T of a bf16 [N][K] weight (32 x 32 tiles).
+__global__ void k_bw_transpose(int N, int K, const bf16 *__restrict__ W, bf16 *__restrict__ WT) {
+  __shared__ bf16 tile[32][34];
+  const int k0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int y = ty; y < 32; y += 8) {
+    const int r = n0 + y, c = k0 + tx;
+    tile[y][tx] = (r < N && c < K) ? W[(size_t)r * K + c] : __float2bfloat16_rn(0.f);
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int c = k0 + y, r = n0 + tx;
+    if (c < K && r < N) WT[(size_t)c * N + r] = tile[tx][y];
   }
 }
 
@@ -424,17 +517,26 @@ __global__ void k_bw_rms_bwd(int d, const float *__restrict__ h, const float *__
 }
 
 // Column sums over rows: out[c] += sum_i X[i][c] (Y[i][c] r[i] when Y).
+// Block of 32 columns x 8 row groups; the groups' partial sums are added in
+// a fixed order, so the result does not depend on scheduling.
 __global__ void k_bw_colsum(int n, int d, const float *__restrict__ X, const float *__restrict__ Y,
                             const float *__restrict__ r, float *__restrict__ out) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= d) return;
+  __shared__ float part[8][33];
+  const int c = blockIdx.x * 32 + threadIdx.x, g = threadIdx.y;
   float s = 0.f;
-  for (int i = 0; i < n; i++) {
-    float v = X[(size_t)i * d + c];
-    if (Y) v *= Y[(size_t)i * d + c] * r[i];
-    s += v;
+  if (c < d)
+    for (int i = g; i < n; i += 8) {
+      float v = X[(size_t)i * d + c];
+      if (Y) v *= Y[(size_t)i * d + c] * r[i];
+      s += v;
+    }
+  part[g][threadIdx.x] = s;
+  __syncthreads();
+  if (g == 0 && c < d) {
+    float t = 0.f;
+    for (int k = 0; k < 8; k++) t += part[k][threadIdx.x];
+    out[c] += t;
   }
-  out[c] += s;
 }
 
 // FFN activation backward: GELU dz = dact GELU'(z); SwiGLU act = SiLU(z) zb:

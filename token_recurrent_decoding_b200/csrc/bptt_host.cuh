@@ -7,52 +7,25 @@
 // Workspace of one rlt_backward call: n rows, NS steps. Offsets in bytes.
 struct BwLayout {
   size_t s_hist, kv_hist, step, dring, xq, xda, xlse, xD, dmem, e32, de, total;
+  size_t wt, xb, xt, yt, n_dev;  // tensor-core operands (bf16 models)
   size_t step_floats;
-  int P;  // recorded positions t0 - (W-1) .. t1 - 1
+  int P;      // recorded positions t0 - (W-1) .. t1 - 1
+  int n_pad;  // rows of the bf16 operands (a multiple of 64)
 };
 
-size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    size_t o = off;
-    off += align256(bytes ? bytes : 1);
-    return o;
-  };
-  const size_t d = c.d, F = c.ffn_dim, H = c.n_heads, L = c.n_dec_layers, W = c.window;
-  const size_t N = n, S = NS, es = elem_size(&c);
-  B->P = (int)(S + W - 1);
-  B->s_hist = take((S + 1) * N * d * 4);
-  B->kv_hist = take(L * N * H * 2 * B->P * (d / H) * es);
-  // one step's activations and gradient scratch (see BwStep)
-  B->step_floats = N * (2 * d + 2 * d + (3 * L + 1) * d + 3 * L * d + 4 * L * d + 3 * L * F +
-                        3 * d + d) +
-                   N * ((3 * L + 1) + 2 * L * H) +
-                   N * (d + std::max(std::max(3 * d, F), 2 * d) + 2 * F + d + 3 * d + d + d +
-                        d + d + d);
-  B->step = take(B->step_floats * 4);
-  B->dring = take(L * N * H * 2 * W * (d / H) * 4);
-  B->xq = take(L * S * N * d * 4);
-  B->xda = take(L * S * N * d * 4);
-  B->xlse = take(L * S * N * H * 4);
-  B->xD = take(L * S * N * H * 4);
-  B->dmem = take((size_t)c.mem_groups * N * c.max_len * 2 * d * 4);
-  B->e32 = take(N * c.max_len * d * 4);
-  B->de = take(N * c.max_len * d * 4);
-  B->total = off;
-  return off;
-}
-
-// Pointers into one step's region.
+// Pointers into one step's region; every buffer starts on a 256-byte
+// boundary (the tensor-core epilogues store float2 / float4 vectors).
 struct BwStep {
   float *cat, *gpre, *gs, *h, *u, *q1, *a1, *qx, *a2, *z, *zb, *act, *qkv, *ulast;
   float *r, *lse1, *lse2;
   float *dh, *dtmp, *dz, *dzb, *dq, *dqkv, *du, *dgpre, *ds, *dcarry;
+  size_t used = 0;  // floats taken
+  static size_t floats(const rlt_config &c, int n) { return BwStep(nullptr, c, n).used; }
   BwStep(float *base, const rlt_config &c, int n) {
     const size_t d = c.d, F = c.ffn_dim, H = c.n_heads, L = c.n_dec_layers, N = n;
-    float *p = base;
     auto take = [&](size_t cnt) {
-      float *o = p;
-      p += cnt;
+      float *o = base ? base + used : nullptr;
+      used += (cnt + 63) / 64 * 64;
       return o;
     };
     cat = take(N * 2 * d);
@@ -84,6 +57,43 @@ struct BwStep {
     dcarry = take(N * d);
   }
 };
+
+size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes ? bytes : 1);
+    return o;
+  };
+  const size_t d = c.d, F = c.ffn_dim, H = c.n_heads, L = c.n_dec_layers, W = c.window;
+  const size_t N = n, S = NS, es = elem_size(&c);
+  B->P = (int)(S + W - 1);
+  B->s_hist = take((S + 1) * N * d * 4);
+  B->kv_hist = take(L * N * H * 2 * B->P * (d / H) * es);
+  // one step's activations and gradient scratch (see BwStep)
+  B->step_floats = BwStep::floats(c, n);
+  B->step = take(B->step_floats * 4);
+  B->dring = take(L * N * H * 2 * W * (d / H) * 4);
+  B->xq = take(L * S * N * d * 4);
+  B->xda = take(L * S * N * d * 4);
+  B->xlse = take(L * S * N * H * 4);
+  B->xD = take(L * S * N * H * 4);
+  // bf16 models: transposed weights and the bf16 GEMM operands
+  const bool tc = c.dtype == RLT_BF16;
+  const size_t NP = (N + 63) / 64 * 64, WMAX = std::max(std::max(3 * d, F), 2 * d);
+  const size_t ffn_mats = c.ffn_kind == RLT_SWIGLU ? 3 : 2;
+  B->n_pad = (int)NP;
+  B->wt = take(tc ? (L * (6 * d * d + ffn_mats * d * F) + 2 * d * d) * 2 : 0);
+  B->xb = take(tc ? NP * WMAX * 2 : 0);
+  B->xt = take(tc ? NP * WMAX * 2 : 0);
+  B->yt = take(tc ? NP * WMAX * 2 : 0);
+  B->n_dev = take(4);
+  B->dmem = take((size_t)c.mem_groups * N * c.max_len * 2 * d * 4);
+  B->e32 = take(N * c.max_len * d * 4);
+  B->de = take(N * c.max_len * d * 4);
+  B->total = off;
+  return off;
+}
 
 template <bool AK, bool BK, typename TA, typename TB>
 cudaError_t bw_gemm(int m, int n, int k, const TA *A, long lda, const TB *B, long ldb, float *C,
@@ -137,6 +147,83 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   const float *s_arena = M->at<float>(L.s);
   const float2 *rope = M->at<float2>(L.rope);
   const size_t nd = (size_t)n * d;
+  const int n_pad = B.n_pad;
+  bf16 *xb = reinterpret_cast<bf16 *>(base + B.xb), *xt = reinterpret_cast<bf16 *>(base + B.xt),
+       *yt = reinterpret_cast<bf16 *>(base + B.yt);
+  int *n_dev = reinterpret_cast<int *>(base + B.n_dev);
+  RLT_TRY(cudaMemcpyAsync(n_dev, &n, 4, cudaMemcpyHostToDevice, st));  // pageable: staged
+
+  // Transposed weights of the tensor-core forms (dX = dY W as a GEMM whose
+  // B operand is W^T, K-major like every tcgen05 operand here).
+  struct WT {
+    const bf16 *qkv, *o, *qx, *ox, *w1, *wb, *w2;
+  };
+  std::vector<WT> wt(LD);
+  const bf16 *wt_gate = nullptr;
+  auto pack = [&](const float *X, long ld, int K, bf16 *row_major, bf16 *transposed) {
+    k_bw_pack<<<dim3((K + 31) / 32, n_pad / 32), dim3(32, 8), 0, st>>>(n, n_pad, K, X, ld,
+                                                                        row_major, transposed);
+    return cudaGetLastError();
+  };
+  if constexpr (std::is_same<T, bf16>::value) {
+    bf16 *p = reinterpret_cast<bf16 *>(base + B.wt);
+    auto tr = [&](const bf16 *Wm, int N, int K) {
+      bf16 *o = p;
+      p += (size_t)N * K;
+      k_bw_transpose<<<dim3((K + 31) / 32, (N + 31) / 32), dim3(32, 8), 0, st>>>(N, K, Wm, o);
+      return (const bf16 *)o;
+    };
+    for (int l = 0; l < LD; l++) {
+      wt[l].qkv = tr(W_<T>::qkv(M, l), 3 * d, d);
+      wt[l].o = tr(W_<T>::o(M, l), d, d);
+      wt[l].qx = tr((const T *)M->w.dec_wqx[l], d, d);
+      wt[l].ox = tr((const T *)M->w.dec_wox[l], d, d);
+      wt[l].w1 = tr(W_<T>::w1(M, l), F, d);
+      wt[l].wb = swiglu ? tr(W_<T>::wb(M, l), F, d) : nullptr;
+      wt[l].w2 = tr(W_<T>::w2(M, l), d, F);
+    }
+    if (c.alpha != 0.0f) wt_gate = tr((const T *)M->w.gate_w, d, 2 * d);
+    RLT_TRY(cudaGetLastError());
+  }
+  // out [n][N] = X [n][K] Wm^T (+ base)
+  auto fwd = [&](const float *X, int K, const T *Wm, int N, float *out,
+                 const float *base_) -> cudaError_t {
+    if constexpr (std::is_same<T, bf16>::value) {
+      RLT_TRY(pack(X, K, K, xb, nullptr));
+      if (base_)
+        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, xb, Wm,
+                              EpiAddF32Dec{{}, base_, out, N}, st);
+      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, xb, Wm, EpiF32Dec{{}, out, N}, st);
+    } else {
+      if (base_) RLT_TRY(cudaMemcpyAsync(out, base_, (size_t)n * N * 4, cudaMemcpyDeviceToDevice, st));
+      return bw_gemm<true, true>(n, N, K, X, K, Wm, K, out, N, base_ != nullptr, st);
+    }
+  };
+  // out [n][K] (=|+=) dY [n][N] Wm, Wm [N][K] (WTm its transpose)
+  auto dx = [&](const float *dY, int N, const T *Wm, const bf16 *WTm, int K, float *out,
+                bool acc) -> cudaError_t {
+    if constexpr (std::is_same<T, bf16>::value) {
+      RLT_TRY(pack(dY, N, N, xb, nullptr));
+      if (acc)
+        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, xb, WTm, EpiAccF32Dec{{}, out, K},
+                              st);
+      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, xb, WTm, EpiF32Dec{{}, out, K}, st);
+    } else {
+      (void)WTm;
+      return bw_gemm<true, false>(n, K, N, dY, N, Wm, K, out, K, acc, st);
+    }
+  };
+  // dW [N][K] += dY [n][N]^T X [n][K] (X with row pitch ldx)
+  auto dw = [&](const float *dY, int N, const float *X, long ldx, int K,
+                float *dW) -> cudaError_t {
+    if constexpr (std::is_same<T, bf16>::value) {
+      RLT_TRY(pack(dY, N, N, nullptr, yt));
+      RLT_TRY(pack(X, ldx, K, nullptr, xt));
+      return gemm_tc(M, N, N, 0, K, n_pad, yt, xt, EpiAccF32{dW, K}, st);
+    } else {
+      return bw_gemm<false, false>(N, K, n, dY, N, X, ldx, dW, K, true, st);
+    }
+  };
 
   // ---- forward of the chunk, recorded
   std::vector<int32_t> idv(ids, ids + n);
@@ -172,8 +259,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     k_bw_gate_cat<T><<<bw_blocks(2 * (long)nd), 256, 0, st>>>(n, d, ready, e, c.max_len, t, s_prev,
                                                               S.cat);
     if (c.alpha != 0.0f)
-      RLT_TRY((bw_gemm<true, true>(n, d, 2 * d, S.cat, 2 * d, (const T *)M->w.gate_w, 2 * d, S.gpre,
-                                   d, false, st)));
+      RLT_TRY(fwd(S.cat, 2 * d, (const T *)M->w.gate_w, d, S.gpre, nullptr));
     else
       RLT_TRY(cudaMemsetAsync(S.gpre, 0, nd * 4, st));
     k_bw_gate_fwd<<<bw_blocks(nd), 256, 0, st>>>(n, d, S.gpre, (const float *)M->w.gate_b, S.cat,
@@ -187,33 +273,26 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
             *act = S.act + (size_t)l * n * F;
       k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h1, (const float *)M->w.dec_ln1[l], u1,
                                       rbuf(l, 0));
-      RLT_TRY((bw_gemm<true, true>(n, 3 * d, d, u1, d, W_<T>::qkv(M, l), d, S.qkv, 3 * d, false,
-                                   st)));
+      RLT_TRY(fwd(u1, d, W_<T>::qkv(M, l), 3 * d, S.qkv, nullptr));
       k_bw_rope_q<<<bw_blocks((long)n * d / 2), 256, 0, st>>>(n, H, DH, t, rope, S.qkv, q1);
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
       const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
       k_bw_attn_fwd<T, DH><<<attn_blocks, 128, 0, st>>>(n, H, swa, p_lo, p_hi, scale, q1, a1,
                                                         S.lse1 + (size_t)l * n * H);
-      RLT_TRY(cudaMemcpyAsync(h2, h1, nd * 4, cudaMemcpyDeviceToDevice, st));
-      RLT_TRY((bw_gemm<true, true>(n, d, d, a1, d, W_<T>::o(M, l), d, h2, d, true, st)));
+      RLT_TRY(fwd(a1, d, W_<T>::o(M, l), d, h2, h1));
       k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h2, (const float *)M->w.dec_ln2[l], u2,
                                       rbuf(l, 1));
-      RLT_TRY((bw_gemm<true, true>(n, d, d, u2, d, (const T *)M->w.dec_wqx[l], d, qx, d, false,
-                                   st)));
+      RLT_TRY(fwd(u2, d, (const T *)M->w.dec_wqx[l], d, qx, nullptr));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
       k_bw_attn_fwd<T, DH><<<attn_blocks, 128, 0, st>>>(n, H, xk, 0, (int)t, scale, qx, a2,
                                                         S.lse2 + (size_t)l * n * H);
-      RLT_TRY(cudaMemcpyAsync(h3, h2, nd * 4, cudaMemcpyDeviceToDevice, st));
-      RLT_TRY((bw_gemm<true, true>(n, d, d, a2, d, (const T *)M->w.dec_wox[l], d, h3, d, true,
-                                   st)));
+      RLT_TRY(fwd(a2, d, (const T *)M->w.dec_wox[l], d, h3, h2));
       k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h3, (const float *)M->w.dec_ln3[l], u3,
                                       rbuf(l, 2));
-      RLT_TRY((bw_gemm<true, true>(n, F, d, u3, d, W_<T>::w1(M, l), d, z, F, false, st)));
-      if (swiglu)
-        RLT_TRY((bw_gemm<true, true>(n, F, d, u3, d, W_<T>::wb(M, l), d, zb, F, false, st)));
+      RLT_TRY(fwd(u3, d, W_<T>::w1(M, l), F, z, nullptr));
+      if (swiglu) RLT_TRY(fwd(u3, d, W_<T>::wb(M, l), F, zb, nullptr));
       k_bw_act_fwd<<<bw_blocks((long)n * F), 256, 0, st>>>((long)n * F, swiglu, z, zb, act);
-      RLT_TRY(cudaMemcpyAsync(hn, h3, nd * 4, cudaMemcpyDeviceToDevice, st));
-      RLT_TRY((bw_gemm<true, true>(n, d, F, act, F, W_<T>::w2(M, l), F, hn, d, true, st)));
+      RLT_TRY(fwd(act, F, W_<T>::w2(M, l), d, hn, h3));
     }
     float *rf = S.r + (size_t)3 * LD * n;
     k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, hbuf(LD, 0), (const float *)M->w.dec_lnf,
@@ -224,7 +303,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     k_bw_ds_total<<<bw_blocks(nd), 256, 0, st>>>(n, d, NS, k, sgrad, S.dcarry, S.ds);
     k_bw_rms_bwd<<<n, 256, 0, st>>>(d, hbuf(LD, 0), rf, (const float *)M->w.dec_lnf, S.ds, S.dh,
                                     1);
-    k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.ds, hbuf(LD, 0), rf, gr->dec_lnf);
+    k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.ds, hbuf(LD, 0), rf, gr->dec_lnf);
     for (int l = LD - 1; l >= 0; l--) {
       float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2);
       float *u1 = ubuf(l, 0), *u2 = ubuf(l, 1), *u3 = ubuf(l, 2);
@@ -232,38 +311,36 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
       float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
             *act = S.act + (size_t)l * n * F;
       // FFN: h_out = h3 + W2 act(W1 u3)
-      RLT_TRY((bw_gemm<true, false>(n, F, d, S.dh, d, W_<T>::w2(M, l), F, S.dtmp, F, false, st)));
-      RLT_TRY((bw_gemm<false, false>(d, F, n, S.dh, d, act, F, gr->dec_w2[l], F, true, st)));
+      RLT_TRY(dx(S.dh, d, W_<T>::w2(M, l), wt[l].w2, F, S.dtmp, false));
+      RLT_TRY(dw(S.dh, d, act, F, F, gr->dec_w2[l]));
       k_bw_act_bwd<<<bw_blocks((long)n * F), 256, 0, st>>>((long)n * F, swiglu, z, zb, S.dtmp,
                                                            S.dz, S.dzb);
-      RLT_TRY((bw_gemm<false, false>(F, d, n, S.dz, F, u3, d, gr->dec_w1[l], d, true, st)));
-      RLT_TRY((bw_gemm<true, false>(n, d, F, S.dz, F, W_<T>::w1(M, l), d, S.du, d, false, st)));
+      RLT_TRY(dw(S.dz, F, u3, d, d, gr->dec_w1[l]));
+      RLT_TRY(dx(S.dz, F, W_<T>::w1(M, l), wt[l].w1, d, S.du, false));
       if (swiglu) {
-        RLT_TRY((bw_gemm<false, false>(F, d, n, S.dzb, F, u3, d, gr->dec_wb[l], d, true, st)));
-        RLT_TRY((bw_gemm<true, false>(n, d, F, S.dzb, F, W_<T>::wb(M, l), d, S.du, d, true, st)));
+        RLT_TRY(dw(S.dzb, F, u3, d, d, gr->dec_wb[l]));
+        RLT_TRY(dx(S.dzb, F, W_<T>::wb(M, l), wt[l].wb, d, S.du, true));
       }
       k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h3, rbuf(l, 2), (const float *)M->w.dec_ln3[l], S.du,
                                       S.dh, 0);
-      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.du, h3, rbuf(l, 2), gr->dec_ln3[l]);
+      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.du, h3, rbuf(l, 2), gr->dec_ln3[l]);
       // cross-attention: h3 = h2 + W_ox attn(W_qx u2, M<=t)
       const int g = G == 1 ? 0 : l;
-      RLT_TRY((bw_gemm<true, false>(n, d, d, S.dh, d, (const T *)M->w.dec_wox[l], d, S.dtmp, d,
-                                    false, st)));
-      RLT_TRY((bw_gemm<false, false>(d, d, n, S.dh, d, a2, d, gr->dec_wox[l], d, true, st)));
+      RLT_TRY(dx(S.dh, d, (const T *)M->w.dec_wox[l], wt[l].ox, d, S.dtmp, false));
+      RLT_TRY(dw(S.dh, d, a2, d, d, gr->dec_wox[l]));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
       const size_t xo = ((size_t)l * NS + k) * nd, xs = ((size_t)l * NS + k) * n * H;
       k_bw_attn_bwd<T, DH><<<attn_blocks, 128, 0, st>>>(
           n, H, xk, 0, (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, S.dtmp, S.dq, nullptr,
           W, 0, xq + xo, xda + xo, xlse + xs, xD + xs);
-      RLT_TRY((bw_gemm<false, false>(d, d, n, S.dq, d, u2, d, gr->dec_wqx[l], d, true, st)));
-      RLT_TRY((bw_gemm<true, false>(n, d, d, S.dq, d, (const T *)M->w.dec_wqx[l], d, S.du, d,
-                                    false, st)));
+      RLT_TRY(dw(S.dq, d, u2, d, d, gr->dec_wqx[l]));
+      RLT_TRY(dx(S.dq, d, (const T *)M->w.dec_wqx[l], wt[l].qx, d, S.du, false));
       k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h2, rbuf(l, 1), (const float *)M->w.dec_ln2[l], S.du,
                                       S.dh, 0);
-      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.du, h2, rbuf(l, 1), gr->dec_ln2[l]);
+      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.du, h2, rbuf(l, 1), gr->dec_ln2[l]);
       // SWA: h2 = h1 + W_o attn(q_t over the window); k_t, v_t enter the cache
-      RLT_TRY((bw_gemm<true, false>(n, d, d, S.dh, d, W_<T>::o(M, l), d, S.dtmp, d, false, st)));
-      RLT_TRY((bw_gemm<false, false>(d, d, n, S.dh, d, a1, d, gr->dec_wo[l], d, true, st)));
+      RLT_TRY(dx(S.dh, d, W_<T>::o(M, l), wt[l].o, d, S.dtmp, false));
+      RLT_TRY(dw(S.dh, d, a1, d, d, gr->dec_wo[l]));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
       const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
       k_bw_attn_bwd<T, DH><<<attn_blocks, 128, 0, st>>>(
@@ -271,23 +348,19 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
           W, t0 - Wm1, nullptr, nullptr, nullptr, nullptr);
       k_bw_qkv_grad<<<bw_blocks((long)n * d / 2), 256, 0, st>>>(
           n, H, DH, W, t, rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv);
-      RLT_TRY((bw_gemm<false, false>(3 * d, d, n, S.dqkv, 3 * d, u1, d, gr->dec_wqkv[l], d, true,
-                                     st)));
-      RLT_TRY((bw_gemm<true, false>(n, d, 3 * d, S.dqkv, 3 * d, W_<T>::qkv(M, l), d, S.du, d,
-                                    false, st)));
+      RLT_TRY(dw(S.dqkv, 3 * d, u1, d, d, gr->dec_wqkv[l]));
+      RLT_TRY(dx(S.dqkv, 3 * d, W_<T>::qkv(M, l), wt[l].qkv, d, S.du, false));
       k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h1, rbuf(l, 0), (const float *)M->w.dec_ln1[l], S.du,
                                       S.dh, 0);
-      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.du, h1, rbuf(l, 0), gr->dec_ln1[l]);
+      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.du, h1, rbuf(l, 0), gr->dec_ln1[l]);
     }
     // gated merge: x = e_t + alpha sigmoid(W_g [e_t; s_{t-1}] + b_g) s_{t-1}
     k_bw_gate_bwd<<<bw_blocks(nd), 256, 0, st>>>(n, d, c.alpha, S.dh, S.cat, S.gs, S.dgpre,
                                                  S.dcarry, egrad, c.max_len, t);
     if (c.alpha != 0.0f) {
-      k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.dgpre, nullptr, nullptr, gr->gate_b);
-      RLT_TRY((bw_gemm<false, false>(d, 2 * d, n, S.dgpre, d, S.cat, 2 * d, gr->gate_w, 2 * d,
-                                     true, st)));
-      RLT_TRY((bw_gemm<true, false>(n, 2 * d, d, S.dgpre, d, (const T *)M->w.gate_w, 2 * d,
-                                    S.dtmp, 2 * d, false, st)));
+      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.dgpre, nullptr, nullptr, gr->gate_b);
+      RLT_TRY(dw(S.dgpre, d, S.cat, 2 * d, 2 * d, gr->gate_w));
+      RLT_TRY(dx(S.dgpre, d, (const T *)M->w.gate_w, wt_gate, 2 * d, S.dtmp, false));
       k_bw_gate_bwd2<<<bw_blocks(nd), 256, 0, st>>>(n, d, S.dtmp, S.dcarry, egrad, c.max_len, t);
     }
     RLT_TRY(cudaGetLastError());
@@ -299,7 +372,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     RLT_TRY(cudaGetLastError());
   }
   if (t0 == 0)  // s_{-1} is the learned start state s*
-    k_bw_colsum<<<(d + 255) / 256, 256, 0, st>>>(n, d, S.dcarry, nullptr, nullptr, gr->sstar);
+    k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.dcarry, nullptr, nullptr, gr->sstar);
 
   // ---- memory rows: dK, dV from the saved cross-attention terms, then
   // K^g = W_mk^g e, V^g = W_mv^g e differentiated into e and the projections

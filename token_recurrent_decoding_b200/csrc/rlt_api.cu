@@ -17,6 +17,8 @@
 
 #include "../../include/rlt.h"
 #include "internal.h"
+#include <cstdio>
+
 #include "common.cuh"
 #include "gemm.cuh"
 #include "kernels.cuh"
@@ -246,10 +248,22 @@ struct rlt_model {
 
 namespace {
 
-#define RLT_TRY(x)                           \
-  do {                                       \
-    cudaError_t e_ = (x);                    \
-    if (e_ != cudaSuccess) return e_;        \
+// The first CUDA error of the calling thread since rlt_last_cuda_error last
+// read it: its name and the source line that saw it.
+thread_local cudaError_t g_err = cudaSuccess;
+thread_local int g_err_line = 0;
+inline cudaError_t note_error(cudaError_t e, int line) {
+  if (e != cudaSuccess && g_err == cudaSuccess) {
+    g_err = e;
+    g_err_line = line;
+  }
+  return e;
+}
+
+#define RLT_TRY(x)                                         \
+  do {                                                     \
+    cudaError_t e_ = (x);                                  \
+    if (e_ != cudaSuccess) return note_error(e_, __LINE__); \
   } while (0)
 
 inline int blocks_for(long threads, int bs) { return (int)((threads + bs - 1) / bs); }
@@ -1420,7 +1434,10 @@ template <typename T> void bind_dh(rlt_model *M) {
   }
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? RLT_OK : RLT_ERR_CUDA; }
+int cuda_status(cudaError_t e) {
+  note_error(e, 0);
+  return e == cudaSuccess ? RLT_OK : RLT_ERR_CUDA;
+}
 
 // Host mirrors of t_dec / t_enc -> device (stream ordered).
 cudaError_t push_positions(rlt_model *M, cudaStream_t st) {
@@ -1888,6 +1905,17 @@ RLT_API const char *rlt_status_string(int s) {
 }
 
 RLT_API int rlt_check_config(const rlt_config *cfg) { return check_config(cfg); }
+
+RLT_API int rlt_last_cuda_error(char *buf, size_t len) {
+  const int e = (int)g_err;
+  if (buf && len) {
+    snprintf(buf, len, "%s (line %d of the library source)",
+             e ? cudaGetErrorName(g_err) : "cudaSuccess", g_err_line);
+  }
+  g_err = cudaSuccess;
+  g_err_line = 0;
+  return e;
+}
 
 RLT_API size_t rlt_attend_workspace_bytes(int n, int n_heads, int head_dim, int cap) {
   return rlt::attend_workspace_internal(n, n_heads, head_dim, cap);

@@ -193,6 +193,54 @@ def run_parallel(args):
     print(json.dumps({"workload": args.workload, "batch": B, "T": T, "parallel_ms": times}))
 
 
+def run_backward(args):
+    """Backpropagation through time over the first `--max-len` positions of
+    the batch (rlt_backward: recorded forward, reverse traversal, memory
+    gradient), `--steps` times from the same start state; prints each call's
+    CUDA-event time and seq-steps/s."""
+    import torch
+
+    from . import configs, inputs, roofline
+    from .rlt import Model
+    wl = configs.workloads()[args.workload]
+    cfg = wl.model
+    if args.layers:
+        cfg = cfg.replace(n_enc=args.layers, n_dec=args.layers,
+                          mem_groups=1 if cfg.mem_groups == 1 else args.layers)
+    B = args.batch or wl.batch
+    T = args.max_len or wl.max_len
+    lengths = [T] * B
+    w = inputs.make_weights(cfg)
+    tok = inputs.make_tokens(cfg.vocab, lengths)
+    m = Model(cfg, w, B, T)
+    del w
+    flat = torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda()
+    ids = list(range(B))
+    m.prefill_encoder(flat, ids, np.arange(B, dtype=np.int32) * T, lengths)
+    start = [m.get_state(i) for i in ids]
+    sgrad = torch.randn((B, T, cfg.d), device="cuda", generator=torch.Generator("cuda").manual_seed(3))
+    ws = torch.empty(m.backward_workspace_bytes(B, T), dtype=torch.uint8, device="cuda")
+    grads = {k: torch.zeros(v, device="cuda") for k, v in m.grad_shapes().items()}
+    egrad = torch.zeros((B, T, cfg.d), device="cuda")
+    times = []
+    for _ in range(args.steps):
+        for i, (s, c, t) in zip(ids, start):
+            m.set_state(i, s, c, t)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        m.backward(ids, sgrad, grads=grads, egrad=egrad, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    assert m.poll_device_error() == 0
+    flops = roofline.backward_flops(cfg, lengths)
+    best = min(times)
+    print(json.dumps({"workload": args.workload, "batch": B, "T": T, "backward_ms": times,
+                      "seq_steps_per_s": B * T / (best / 1e3),
+                      "tflops": flops / (best / 1e3) / 1e12,
+                      "workspace_gb": ws.numel() / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="m140_bf16")
@@ -212,6 +260,8 @@ def main():
     ap.add_argument("--kernel", choices=["fused", "chain"], default=None,
                     help="decoder step kernel (default: the model's default)")
     ap.add_argument("--attend", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time rlt_backward over --max-len positions of --batch sequences")
     ap.add_argument("--parallel", action="store_true",
                     help="time the token-parallel decoder pass (feedback-off workloads)")
     ap.add_argument("--n", type=int, default=256)
@@ -225,6 +275,8 @@ def main():
         run_attend(args)
     elif args.parallel:
         run_parallel(args)
+    elif args.backward:
+        run_backward(args)
     else:
         run_steps(args)
 

@@ -119,6 +119,7 @@ def _declare(lib):
     lib.rlt_profile.argtypes = [P, I]
     lib.rlt_get_stats.argtypes = [P, P]
     lib.rlt_status_string.argtypes = [I]
+    lib.rlt_last_cuda_error.argtypes = [C.c_char_p, C.c_size_t]
     lib.rlt_status_string.restype = C.c_char_p
 
 
@@ -142,6 +143,10 @@ def header_symbols():
 
 def _check(rc: int, what: str):
     if rc != RLT_OK:
+        if rc == 6:  # RLT_ERR_CUDA
+            buf = C.create_string_buffer(160)
+            _lib().rlt_last_cuda_error(buf, 160)
+            what = f"{what}: {buf.value.decode()}"
         raise RLTError(rc, what)
 
 

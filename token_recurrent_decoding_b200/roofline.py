@@ -106,3 +106,17 @@ def decoder_parallel_roofline(cfg: RLTConfig, lengths, hbm_gbs: float, tensor_tf
     byts = dec_matmul_params(cfg) * es + tok * d * (es + 4) + cfg.mem_groups * tok * 2 * d * es
     return {"seconds": max(flops / (tensor_tflops * 1e12), byts / (hbm_gbs * 1e9)),
             "flops": float(flops), "bytes": float(byts), "seq_steps": int(tok)}
+
+
+def backward_flops(cfg: RLTConfig, lengths) -> float:
+    """FLOPs of one backpropagation through time over full sequences: the
+    recomputed forward (the step's FLOPs) plus twice that for the gradients
+    of every matmul (activations and weights) and of the attentions, plus the
+    recorded forward itself: 4 x the decoder run's FLOPs. The memory
+    projection's backward adds 2 x 2 x 2 d^2 G per position."""
+    lengths = np.asarray(lengths)
+    tot = 0.0
+    for T in lengths:
+        t = np.arange(T, dtype=np.float64)
+        tot += 4 * decoder_step_flops(cfg, t) + 8.0 * cfg.d * cfg.d * cfg.mem_groups * T
+    return float(tot)
