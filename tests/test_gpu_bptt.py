@@ -120,9 +120,13 @@ def test_chunked_backward_composes(name):
         m.set_state(i, s, c, t)
     m.backward(ids, Gd[:, :k].contiguous(), grads=late, egrad=e_acc, carry_in=carry)
     torch.cuda.synchronize()
+    # fp32: the same arithmetic regrouped; bf16: each chunk rounds its own
+    # partial memory-row gradients to bf16 for the projection's tensor-core
+    # GEMMs (2^-9 relative per element, on either side)
+    bound = 1e-5 if cfg.dtype == configs.F32 else 1e-2
     for key in full:
-        assert _rel(to_np(late[key]), to_np(full[key])) <= 1e-5, key
-    assert _rel(to_np(e_acc), to_np(e_full)) <= 1e-5
+        assert _rel(to_np(late[key]), to_np(full[key])) <= bound, key
+    assert _rel(to_np(e_acc), to_np(e_full)) <= bound
     for a, b in zip(end_full, end_late):
         assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and a[2] == b[2] == T
     # against the oracle as two chunks too: the late chunk from the GPU's state at k

@@ -34,6 +34,15 @@
 
 namespace rlt {
 
+// Kernels of the traversal are launched with programmatic stream
+// serialisation: each waits for its predecessor's results, then lets its
+// successor launch (and stream its weights) while it runs.
+#define BW_PDL()   \
+  do {             \
+    pdl_wait();    \
+    pdl_trigger(); \
+  } while (0)
+
 // ------------------------------------------------------------------ GEMM
 // C[m][n] (= or +=) sum_k A(m, k) B(n, k); A(m, k) = A[m * lda + k] when AK
 // (k contiguous) else A[k * lda + m]; B likewise with BK. 64 x 64 tiles,
@@ -43,6 +52,7 @@ template <typename TA, typename TB, bool AK, bool BK>
 __global__ void __launch_bounds__(256)
     k_bw_gemm(int M, int N, int K, const TA *__restrict__ A, long lda, const TB *__restrict__ B,
               long ldb, float *__restrict__ C, long ldc, int acc) {
+  BW_PDL();
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
@@ -140,11 +150,12 @@ struct EpiAccF32 {
 };
 
 // bf16 operands of the tensor-core GEMMs from an fp32 [n][ld] matrix (its
-// first K columns): row-major Xb [n_pad][K] and/or transposed XT [K][n_pad],
-// rows n .. n_pad-1 zero. 32 x 32 tiles through shared memory, so both
-// layouts are written with contiguous runs.
+// first K columns): row-major Xb [n_pad][K] and/or the transposed block
+// XT[c][col0 + r] (row pitch `pitch`), rows n .. n_pad-1 zero. 32 x 32 tiles
+// through shared memory, so both layouts are written with contiguous runs.
 __global__ void k_bw_pack(int n, int n_pad, int K, const float *__restrict__ X, long ld,
-                          bf16 *__restrict__ Xb, bf16 *__restrict__ XT) {
+                          bf16 *__restrict__ Xb, bf16 *__restrict__ XT, long pitch, long col0) {
+  BW_PDL();
   __shared__ float tile[32][33];
   const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
@@ -158,7 +169,7 @@ __global__ void k_bw_pack(int n, int n_pad, int K, const float *__restrict__ X, 
   __syncthreads();
   for (int y = ty; y < 32; y += 8) {
     const int c = c0 + y, r = r0 + tx;
-    if (c < K && r < n_pad) XT[(size_t)c * n_pad + r] = __float2bfloat16_rn(tile[tx][y]);
+    if (c < K && r < n_pad) XT[(size_t)c * pitch + col0 + r] = __float2bfloat16_rn(tile[tx][y]);
   }
 }
 
@@ -238,6 +249,7 @@ __global__ void k_bw_hist_step(int n, const int *__restrict__ ready, const T *__
                                const float *__restrict__ s, int L, int H, int dh, int W,
                                int max_seqs, long t, int p, int P, T *__restrict__ kv_hist,
                                float *__restrict__ s_hist_k) {
+  BW_PDL();
   const int d = H * dh;
   const long total = (long)L * n * H * 2 * dh;
   const long stride = (long)gridDim.x * blockDim.x;
@@ -264,6 +276,7 @@ template <typename T>
 __global__ void k_bw_gate_cat(int n, int d, const int *__restrict__ ready, const T *__restrict__ e,
                               int max_len, long t, const float *__restrict__ s_prev,
                               float *__restrict__ cat) {
+  BW_PDL();
   const long total = (long)n * 2 * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
@@ -277,6 +290,7 @@ __global__ void k_bw_gate_cat(int n, int d, const int *__restrict__ ready, const
 __global__ void k_bw_gate_fwd(int n, int d, const float *__restrict__ gpre,
                               const float *__restrict__ gate_b, const float *__restrict__ cat,
                               float alpha, float *__restrict__ g, float *__restrict__ x) {
+  BW_PDL();
   const long total = (long)n * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
@@ -291,6 +305,7 @@ __global__ void k_bw_gate_fwd(int n, int d, const float *__restrict__ gpre,
 __global__ void k_bw_rms_fwd(int d, float eps, const float *__restrict__ h,
                              const float *__restrict__ gamma, float *__restrict__ u,
                              float *__restrict__ r) {
+  BW_PDL();
   __shared__ float red[32];
   const float *x = h + (size_t)blockIdx.x * d;
   float ss = 0.f;
@@ -305,6 +320,7 @@ __global__ void k_bw_rms_fwd(int d, float eps, const float *__restrict__ h,
 // Rotary encoding of the q part of a [n][3d] q/k/v row at position t.
 __global__ void k_bw_rope_q(int n, int H, int dh, long t, const float2 *__restrict__ rope,
                             const float *__restrict__ qkv, float *__restrict__ q) {
+  BW_PDL();
   const int d = H * dh, half = dh / 2;
   const long total = (long)n * H * half;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
@@ -320,6 +336,7 @@ __global__ void k_bw_rope_q(int n, int H, int dh, long t, const float2 *__restri
 // GELU or SwiGLU activation of the FFN: act = GELU(z) or SiLU(z) zb.
 __global__ void k_bw_act_fwd(long total, int swiglu, const float *__restrict__ z,
                              const float *__restrict__ zb, float *__restrict__ act) {
+  BW_PDL();
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x)
     act[idx] = swiglu ? silu(z[idx]) * zb[idx] : gelu_erf(z[idx]);
@@ -344,129 +361,215 @@ template <typename T> struct BwKeys {
   }
 };
 
+// Eight consecutive head entries of a key or value row as floats.
+__device__ __forceinline__ void bw_ld8(const bf16 *p, float *f) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const bf16 *b = reinterpret_cast<const bf16 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; i++) f[i] = __bfloat162float(b[i]);
+}
+__device__ __forceinline__ void bw_ld8(const float *p, float *f) {
+  const float4 x = reinterpret_cast<const float4 *>(p)[0], y = reinterpret_cast<const float4 *>(p)[1];
+  f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+  f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
+}
+
+// Sum over the DH / 8 lanes that hold one key's head slices.
+template <int LPK> __device__ __forceinline__ float bw_group_sum(float v) {
+#pragma unroll
+  for (int o = LPK / 2; o > 0; o >>= 1) v += __shfl_xor_sync(FULL_MASK, v, o);
+  return v;
+}
+
+// Online-softmax state (max, denominator, 8 output entries) of two key sets
+// merged into the first.
+__device__ __forceinline__ void bw_merge(float &m, float &l, float *acc, float m2, float l2,
+                                         const float *acc2) {
+  const float M = fmaxf(m, m2);
+  if (M == -INFINITY) return;
+  const float c1 = m == -INFINITY ? 0.f : expf(m - M), c2 = m2 == -INFINITY ? 0.f : expf(m2 - M);
+  l = l * c1 + l2 * c2;
+#pragma unroll
+  for (int e = 0; e < 8; e++) acc[e] = acc[e] * c1 + acc2[e] * c2;
+  m = M;
+}
+
+constexpr int BW_ATT_WARPS = 4;
+
 // Attention of one query per (row, head) over key rows j_lo .. j_hi of the
-// key table (one warp each; lanes split the head dimension): a and the
-// log-sum-exp of the scaled scores.
+// key table: one CTA of four warps per (row, head); a key is read by DH / 8
+// lanes (eight head entries each, one 16-byte load for bf16), so a warp
+// takes 256 / DH keys at a time and the CTA 4x that. Each lane group keeps
+// its own online-softmax state; the states are merged in a fixed tree (lane
+// groups by shuffles, then the warps in order), so the result does not
+// depend on timing. Writes a and the log-sum-exp of the scaled scores.
 template <typename T, int DH>
-__global__ void k_bw_attn_fwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
-                              const float *__restrict__ q, float *__restrict__ a,
-                              float *__restrict__ lse) {
-  constexpr int EPL = (DH + 31) / 32;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= n * H) return;
-  const int i = warp / H, h = warp % H, d = H * DH;
+__global__ void __launch_bounds__(32 * BW_ATT_WARPS)
+    k_bw_attn_fwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
+                  const float *__restrict__ q, float *__restrict__ a, float *__restrict__ lse) {
+  BW_PDL();
+  constexpr int LPK = DH / 8, KPW = 32 / LPK;
+  __shared__ float red[BW_ATT_WARPS][2 + DH];
+  const int i = blockIdx.x / H, h = blockIdx.x % H, d = H * DH;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane / LPK, sl = lane % LPK;
   const T *K = keys.k(i, h), *V = keys.v(i, h);
-  float qv[EPL], acc[EPL];
+  float qv[8], acc[8];
+  bw_ld8(q + (size_t)i * d + h * DH + sl * 8, qv);
 #pragma unroll
-  for (int x = 0; x < EPL; x++) {
-    const int e = lane + 32 * x;
-    qv[x] = e < DH ? q[(size_t)i * d + h * DH + e] : 0.f;
-    acc[x] = 0.f;
-  }
+  for (int e = 0; e < 8; e++) acc[e] = 0.f;
   float m = -INFINITY, l = 0.f;
-  for (int j = j_lo; j <= j_hi; j++) {
+  for (int base = j_lo + warp * KPW; base <= j_hi; base += BW_ATT_WARPS * KPW) {
+    const int j = base + grp;
+    const bool ok = j <= j_hi;
+    float kv[8], vv[8];
     float dot = 0.f;
+    if (ok) {
+      bw_ld8(K + (size_t)j * DH + sl * 8, kv);
+      bw_ld8(V + (size_t)j * DH + sl * 8, vv);
 #pragma unroll
-    for (int x = 0; x < EPL; x++) {
-      const int e = lane + 32 * x;
-      if (e < DH) dot += qv[x] * to_f(K[(size_t)j * DH + e]);
+      for (int e = 0; e < 8; e++) dot += qv[e] * kv[e];
     }
-    const float s = warp_sum(dot) * scale;
-    const float mn = fmaxf(m, s);
-    const float corr = expf(m - mn), p = expf(s - mn);
-    l = l * corr + p;
+    dot = bw_group_sum<LPK>(dot);
+    if (ok) {
+      const float s = dot * scale, mn = fmaxf(m, s);
+      const float corr = m == -INFINITY ? 0.f : expf(m - mn), p = expf(s - mn);
+      l = l * corr + p;
 #pragma unroll
-    for (int x = 0; x < EPL; x++) {
-      const int e = lane + 32 * x;
-      acc[x] = acc[x] * corr + (e < DH ? p * to_f(V[(size_t)j * DH + e]) : 0.f);
+      for (int e = 0; e < 8; e++) acc[e] = acc[e] * corr + p * vv[e];
+      m = mn;
     }
-    m = mn;
   }
+  // lane groups of the warp (same slice), then the warps in order
 #pragma unroll
-  for (int x = 0; x < EPL; x++) {
-    const int e = lane + 32 * x;
-    if (e < DH) a[(size_t)i * d + h * DH + e] = acc[x] / l;
+  for (int o = LPK; o < 32; o <<= 1) {
+    float acc2[8];
+    const float m2 = __shfl_xor_sync(FULL_MASK, m, o), l2 = __shfl_xor_sync(FULL_MASK, l, o);
+#pragma unroll
+    for (int e = 0; e < 8; e++) acc2[e] = __shfl_xor_sync(FULL_MASK, acc[e], o);
+    bw_merge(m, l, acc, m2, l2, acc2);
   }
-  if (lane == 0) lse[(size_t)i * H + h] = m + logf(l);
+  if (grp == 0) {
+    if (sl == 0) {
+      red[warp][0] = m;
+      red[warp][1] = l;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; e++) red[warp][2 + sl * 8 + e] = acc[e];
+  }
+  __syncthreads();
+  if (warp == 0 && grp == 0) {
+    for (int w = 1; w < BW_ATT_WARPS; w++) bw_merge(m, l, acc, red[w][0], red[w][1], &red[w][2 + sl * 8]);
+#pragma unroll
+    for (int e = 0; e < 8; e++) a[(size_t)i * d + h * DH + sl * 8 + e] = acc[e] / l;
+    if (sl == 0) lse[(size_t)i * H + h] = m + logf(l);
+  }
 }
 
 // ------------------------------------------------------------ backward
 // Attention backward of one query per (row, head) over key rows
-// j_lo .. j_hi: P_j = exp(scale q.k_j - lse), dS_j = P_j (da.v_j - da.a),
-// dq = scale sum_j dS_j k_j. SWA (dring != null): also dk_j += scale dS_j q
-// and dv_j += P_j da into the gradient ring slot of position pos0 + j.
-// Cross-attention (xq != null): q, da, lse and D = da.a are saved for the
-// memory-gradient pass.
+// j_lo .. j_hi, with the lane layout of k_bw_attn_fwd: P_j = exp(scale q.k_j
+// - lse), dS_j = P_j (da.v_j - da.a), dq = scale sum_j dS_j k_j (lane-group
+// partial sums merged in a fixed order). SWA (dring != null): also
+// dk_j += scale dS_j q and dv_j += P_j da into the gradient ring slot of
+// position pos0 + j (each key is owned by one lane group). Cross-attention
+// (xq != null): q, da, lse and D = da.a are saved for the memory-gradient
+// pass.
 template <typename T, int DH>
-__global__ void k_bw_attn_bwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
-                              const float *__restrict__ q, const float *__restrict__ a,
-                              const float *__restrict__ lse, const float *__restrict__ da,
-                              float *__restrict__ dq, float *__restrict__ dring, int W, long pos0,
-                              float *__restrict__ xq, float *__restrict__ xda,
-                              float *__restrict__ xlse, float *__restrict__ xD) {
-  constexpr int EPL = (DH + 31) / 32;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= n * H) return;
-  const int i = warp / H, h = warp % H, d = H * DH;
+__global__ void __launch_bounds__(32 * BW_ATT_WARPS)
+    k_bw_attn_bwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
+                  const float *__restrict__ q, const float *__restrict__ a,
+                  const float *__restrict__ lse, const float *__restrict__ da,
+                  float *__restrict__ dq, float *__restrict__ dring, int W, long pos0,
+                  float *__restrict__ xq, float *__restrict__ xda, float *__restrict__ xlse,
+                  float *__restrict__ xD) {
+  BW_PDL();
+  constexpr int LPK = DH / 8, KPW = 32 / LPK;
+  __shared__ float red[BW_ATT_WARPS][DH];
+  const int i = blockIdx.x / H, h = blockIdx.x % H, d = H * DH;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane / LPK, sl = lane % LPK;
   const T *K = keys.k(i, h), *V = keys.v(i, h);
-  const size_t off = (size_t)i * d + h * DH;
-  float qv[EPL], dav[EPL], dqv[EPL];
+  const size_t off = (size_t)i * d + h * DH + sl * 8;
+  float qv[8], dav[8], av[8], dqv[8];
+  bw_ld8(q + off, qv);
+  bw_ld8(da + off, dav);
+  bw_ld8(a + off, av);
   float Dp = 0.f;
 #pragma unroll
-  for (int x = 0; x < EPL; x++) {
-    const int e = lane + 32 * x;
-    qv[x] = e < DH ? q[off + e] : 0.f;
-    dav[x] = e < DH ? da[off + e] : 0.f;
-    Dp += e < DH ? dav[x] * a[off + e] : 0.f;
-    dqv[x] = 0.f;
+  for (int e = 0; e < 8; e++) {
+    Dp += dav[e] * av[e];
+    dqv[e] = 0.f;
   }
-  const float D = warp_sum(Dp);
+  const float D = bw_group_sum<LPK>(Dp);
   const float L = lse[(size_t)i * H + h];
   float *dk_ring = dring ? dring + ((((size_t)keys.l_or_g * n + i) * H + h) * 2 + 0) * W * DH
                          : nullptr;
   float *dv_ring = dring ? dk_ring + (size_t)W * DH : nullptr;
-  for (int j = j_lo; j <= j_hi; j++) {
+  for (int base = j_lo + warp * KPW; base <= j_hi; base += BW_ATT_WARPS * KPW) {
+    const int j = base + grp;
+    const bool ok = j <= j_hi;
+    float kv[8], vv[8];
     float dot = 0.f, dp = 0.f;
-    float kv[EPL];
+    if (ok) {
+      bw_ld8(K + (size_t)j * DH + sl * 8, kv);
+      bw_ld8(V + (size_t)j * DH + sl * 8, vv);
 #pragma unroll
-    for (int x = 0; x < EPL; x++) {
-      const int e = lane + 32 * x;
-      kv[x] = e < DH ? to_f(K[(size_t)j * DH + e]) : 0.f;
-      dot += qv[x] * kv[x];
-      dp += e < DH ? dav[x] * to_f(V[(size_t)j * DH + e]) : 0.f;
+      for (int e = 0; e < 8; e++) {
+        dot += qv[e] * kv[e];
+        dp += dav[e] * vv[e];
+      }
     }
-    const float s = warp_sum(dot) * scale;
-    dp = warp_sum(dp);
-    const float p = expf(s - L);
-    const float ds = p * (dp - D);
+    dot = bw_group_sum<LPK>(dot);
+    dp = bw_group_sum<LPK>(dp);
+    if (ok) {
+      const float p = expf(dot * scale - L);
+      const float ds = p * (dp - D);
 #pragma unroll
-    for (int x = 0; x < EPL; x++) dqv[x] += scale * ds * kv[x];
-    if (dk_ring) {
-      const size_t slot = (size_t)((pos0 + j) % W) * DH;
+      for (int e = 0; e < 8; e++) dqv[e] += scale * ds * kv[e];
+      if (dk_ring) {
+        const size_t slot = (size_t)((pos0 + j) % W) * DH + sl * 8;
+        float4 *pk = reinterpret_cast<float4 *>(dk_ring + slot);
+        float4 *pv = reinterpret_cast<float4 *>(dv_ring + slot);
 #pragma unroll
-      for (int x = 0; x < EPL; x++) {
-        const int e = lane + 32 * x;
-        if (e < DH) {
-          dk_ring[slot + e] += scale * ds * qv[x];
-          dv_ring[slot + e] += p * dav[x];
+        for (int x = 0; x < 2; x++) {
+          float4 k4 = pk[x], v4 = pv[x];
+          k4.x += scale * ds * qv[4 * x];
+          k4.y += scale * ds * qv[4 * x + 1];
+          k4.z += scale * ds * qv[4 * x + 2];
+          k4.w += scale * ds * qv[4 * x + 3];
+          v4.x += p * dav[4 * x];
+          v4.y += p * dav[4 * x + 1];
+          v4.z += p * dav[4 * x + 2];
+          v4.w += p * dav[4 * x + 3];
+          pk[x] = k4;
+          pv[x] = v4;
         }
       }
     }
   }
 #pragma unroll
-  for (int x = 0; x < EPL; x++) {
-    const int e = lane + 32 * x;
-    if (e < DH) {
-      dq[off + e] = dqv[x];
+  for (int o = LPK; o < 32; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; e++) dqv[e] += __shfl_xor_sync(FULL_MASK, dqv[e], o);
+  if (grp == 0)
+#pragma unroll
+    for (int e = 0; e < 8; e++) red[warp][sl * 8 + e] = dqv[e];
+  __syncthreads();
+  if (warp == 0 && grp == 0) {
+    for (int w = 1; w < BW_ATT_WARPS; w++)
+#pragma unroll
+      for (int e = 0; e < 8; e++) dqv[e] += red[w][sl * 8 + e];
+#pragma unroll
+    for (int e = 0; e < 8; e++) {
+      dq[off + e] = dqv[e];
       if (xq) {
-        xq[off + e] = qv[x];
-        xda[off + e] = dav[x];
+        xq[off + e] = qv[e];
+        xda[off + e] = dav[e];
       }
     }
-  }
-  if (xq && lane == 0) {
-    xlse[(size_t)i * H + h] = L;
-    xD[(size_t)i * H + h] = D;
+    if (xq && sl == 0) {
+      xlse[(size_t)i * H + h] = L;
+      xD[(size_t)i * H + h] = D;
+    }
   }
 }
 
@@ -476,6 +579,7 @@ __global__ void k_bw_attn_bwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, 
 __global__ void k_bw_qkv_grad(int n, int H, int dh, int W, long t, const float2 *__restrict__ rope,
                               const float *__restrict__ dq, float *__restrict__ dring_l,
                               float *__restrict__ dqkv) {
+  BW_PDL();
   const int d = H * dh, half = dh / 2;
   const long total = (long)n * H * half;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
@@ -501,9 +605,11 @@ __global__ void k_bw_qkv_grad(int n, int H, int dh, int W, long t, const float2 
 // RMSNorm backward of one row (one block per row): with u = h r gamma,
 // dh += r gamma du - h r^3 / d sum_c du_c gamma_c h_c (or dh = ... when
 // `assign`).
+// The gain's gradient per row, du h r, goes to gg (summed over rows later).
 __global__ void k_bw_rms_bwd(int d, const float *__restrict__ h, const float *__restrict__ r,
                              const float *__restrict__ gamma, const float *__restrict__ du,
-                             float *__restrict__ dh, int assign) {
+                             float *__restrict__ dh, int assign, float *__restrict__ gg) {
+  BW_PDL();
   __shared__ float red[32];
   const size_t o = (size_t)blockIdx.x * d;
   float sp = 0.f;
@@ -513,23 +619,20 @@ __global__ void k_bw_rms_bwd(int d, const float *__restrict__ h, const float *__
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     const float g = rr * gamma[c] * du[o + c] - h[o + c] * k3;
     dh[o + c] = assign ? g : dh[o + c] + g;
+    gg[o + c] = du[o + c] * h[o + c] * rr;
   }
 }
 
-// Column sums over rows: out[c] += sum_i X[i][c] (Y[i][c] r[i] when Y).
-// Block of 32 columns x 8 row groups; the groups' partial sums are added in
-// a fixed order, so the result does not depend on scheduling.
-__global__ void k_bw_colsum(int n, int d, const float *__restrict__ X, const float *__restrict__ Y,
-                            const float *__restrict__ r, float *__restrict__ out) {
+// Column sums over rows: out[c] += sum_i X[i][c]. Block of 32 columns x 8
+// row groups; the groups' partial sums are added in a fixed order, so the
+// result does not depend on scheduling.
+__global__ void k_bw_colsum(int n, int d, const float *__restrict__ X, float *__restrict__ out) {
+  BW_PDL();
   __shared__ float part[8][33];
   const int c = blockIdx.x * 32 + threadIdx.x, g = threadIdx.y;
   float s = 0.f;
   if (c < d)
-    for (int i = g; i < n; i += 8) {
-      float v = X[(size_t)i * d + c];
-      if (Y) v *= Y[(size_t)i * d + c] * r[i];
-      s += v;
-    }
+    for (int i = g; i < n; i += 8) s += X[(size_t)i * d + c];
   part[g][threadIdx.x] = s;
   __syncthreads();
   if (g == 0 && c < d) {
@@ -544,6 +647,7 @@ __global__ void k_bw_colsum(int n, int d, const float *__restrict__ X, const flo
 __global__ void k_bw_act_bwd(long total, int swiglu, const float *__restrict__ z,
                              const float *__restrict__ zb, const float *__restrict__ dact,
                              float *__restrict__ dz, float *__restrict__ dzb) {
+  BW_PDL();
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
     const float x = z[idx], g = dact[idx];
@@ -563,6 +667,7 @@ __global__ void k_bw_gate_bwd(int n, int d, float alpha, const float *__restrict
                               const float *__restrict__ cat, const float *__restrict__ g,
                               float *__restrict__ dgpre, float *__restrict__ ds_prev,
                               float *__restrict__ egrad, int max_len, long t) {
+  BW_PDL();
   const long total = (long)n * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
@@ -579,6 +684,7 @@ __global__ void k_bw_gate_bwd(int n, int d, float alpha, const float *__restrict
 __global__ void k_bw_gate_bwd2(int n, int d, const float *__restrict__ dcat,
                                float *__restrict__ ds_prev, float *__restrict__ egrad, int max_len,
                                long t) {
+  BW_PDL();
   const long total = (long)n * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
@@ -591,6 +697,7 @@ __global__ void k_bw_gate_bwd2(int n, int d, const float *__restrict__ dcat,
 // ds_t = G_t + the gradient s_t received from step t+1.
 __global__ void k_bw_ds_total(int n, int d, int n_steps, int k, const float *__restrict__ sgrad,
                               const float *__restrict__ carry, float *__restrict__ ds) {
+  BW_PDL();
   const long total = (long)n * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
@@ -648,7 +755,8 @@ __global__ void __launch_bounds__(256)
               const int *__restrict__ ready, const T *__restrict__ mem,
               const float *__restrict__ xq, const float *__restrict__ xda,
               const float *__restrict__ xlse, const float *__restrict__ xD, float scale,
-              float *__restrict__ dmem) {
+              float *__restrict__ dmem, bf16 *__restrict__ dkb, bf16 *__restrict__ dvb,
+              bf16 *__restrict__ dkT, bf16 *__restrict__ dvT, long rows_pad) {
   extern __shared__ __align__(16) float sm[];
   float *Kj = sm, *Vj = Kj + 64 * DH, *Qt = Vj + 64 * DH, *At = Qt + 64 * DH;
   float *Ps = At + 64 * DH, *Ss = Ps + 64 * 65, *ls = Ss + 64 * 65, *Ds = ls + 64;
@@ -721,12 +829,53 @@ __global__ void __launch_bounds__(256)
   }
   const int j = j0 + ojj;
   if (j < t1) {
-    float *o = dmem + ((((size_t)g * n + i) * t1 + j) * 2) * d + h * DH + oe0;
+    const size_t row = (size_t)i * t1 + j;  // row of the (sequence, position) matrices
+    if (dkb) {  // bf16 operands of the projection's tensor-core GEMMs
+      const size_t gr = (size_t)g * rows_pad;
 #pragma unroll
-    for (int x = 0; x < EPT; x++) {
-      o[x] = dK[x];
-      o[d + x] = dV[x];
+      for (int x = 0; x < EPT; x++) {
+        const int col = h * DH + oe0 + x;
+        dkb[(gr + row) * d + col] = __float2bfloat16_rn(dK[x]);
+        dvb[(gr + row) * d + col] = __float2bfloat16_rn(dV[x]);
+        dkT[((size_t)g * d + col) * rows_pad + row] = __float2bfloat16_rn(dK[x]);
+        dvT[((size_t)g * d + col) * rows_pad + row] = __float2bfloat16_rn(dV[x]);
+      }
+    } else {
+      float *o = dmem + ((size_t)g * n * t1 + row) * 2 * d + h * DH + oe0;
+#pragma unroll
+      for (int x = 0; x < EPT; x++) {
+        o[x] = dK[x];
+        o[d + x] = dV[x];
+      }
     }
+  }
+}
+
+// eT[c][i t1 + j] = e of position j of row i (bf16), columns up to rows_pad
+// zero: the transposed operand of the memory projection's weight gradient.
+template <typename T>
+__global__ void k_bw_e_transposed(int n, int d, long t1, int max_len, long rows_pad,
+                                  const int *__restrict__ ready, const T *__restrict__ e,
+                                  bf16 *__restrict__ eT) {
+  __shared__ float tile[32][33];
+  const long r0 = (long)blockIdx.y * 32;
+  const int c0 = blockIdx.x * 32, tx = threadIdx.x, ty = threadIdx.y;
+  for (int y = ty; y < 32; y += 8) {
+    const long r = r0 + y;
+    const int c = c0 + tx;
+    float v = 0.f;
+    if (r < (long)n * t1 && c < d) {
+      const int i = (int)(r / t1);
+      const long j = r % t1;
+      v = to_f(e[((size_t)ready[i] * max_len + j) * d + c]);
+    }
+    tile[y][tx] = v;
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int c = c0 + y;
+    const long r = r0 + tx;
+    if (c < d && r < rows_pad) eT[(size_t)c * rows_pad + r] = __float2bfloat16_rn(tile[tx][y]);
   }
 }
 

@@ -4,11 +4,18 @@
 // encoder outputs, memory and rotary table.
 #pragma once
 
+// Steps whose weight gradients one GEMM reduces (bf16 models): each step's
+// bf16 operands of the weight-gradient products (activations and output
+// gradients, transposed) land in column block `slot` of a group buffer, and
+// one tile GEMM per weight and group reduces over group x batch rows.
+constexpr int BW_GROUP = 8;
+
 // Workspace of one rlt_backward call: n rows, NS steps. Offsets in bytes.
 struct BwLayout {
   size_t s_hist, kv_hist, step, dring, xq, xda, xlse, xD, dmem, e32, de, total;
-  size_t wt, xb, xt, yt, n_dev;  // tensor-core operands (bf16 models)
-  size_t step_floats;
+  size_t wt, xb, grp, gg, n_dev;  // tensor-core operands; gain-gradient rows
+  size_t dmb, eT, wtm, rows_pad;   // memory-projection operands (bf16 models)
+  size_t step_floats, grp_layer_rows;
   int P;      // recorded positions t0 - (W-1) .. t1 - 1
   int n_pad;  // rows of the bf16 operands (a multiple of 64)
 };
@@ -18,7 +25,7 @@ struct BwLayout {
 struct BwStep {
   float *cat, *gpre, *gs, *h, *u, *q1, *a1, *qx, *a2, *z, *zb, *act, *qkv, *ulast;
   float *r, *lse1, *lse2;
-  float *dh, *dtmp, *dz, *dzb, *dq, *dqkv, *du, *dgpre, *ds, *dcarry;
+  float *dh, *dtmp, *dz, *dzb, *dq, *dqkv, *du, *ds, *dcarry;
   size_t used = 0;  // floats taken
   static size_t floats(const rlt_config &c, int n) { return BwStep(nullptr, c, n).used; }
   BwStep(float *base, const rlt_config &c, int n) {
@@ -52,11 +59,19 @@ struct BwStep {
     dq = take(N * d);
     dqkv = take(N * 3 * d);
     du = take(N * d);
-    dgpre = take(N * d);
     ds = take(N * d);
     dcarry = take(N * d);
   }
 };
+
+// Rows of one layer's group buffer: the transposed activations (u1, a1, u2,
+// a2, u3: d each; act: F) and output gradients (dqkv: 3d; dh at the SWA, the
+// cross-attention and the FFN outputs, dq of the cross-attention: d each;
+// dz, and dzb for SwiGLU: F).
+size_t bw_grp_layer_rows(const rlt_config &c) {
+  const size_t d = c.d, F = c.ffn_dim;
+  return 5 * d + F + 3 * d + 4 * d + F + (c.ffn_kind == RLT_SWIGLU ? F : 0);
+}
 
 size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
   size_t off = 0;
@@ -70,7 +85,6 @@ size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
   B->P = (int)(S + W - 1);
   B->s_hist = take((S + 1) * N * d * 4);
   B->kv_hist = take(L * N * H * 2 * B->P * (d / H) * es);
-  // one step's activations and gradient scratch (see BwStep)
   B->step_floats = BwStep::floats(c, n);
   B->step = take(B->step_floats * 4);
   B->dring = take(L * N * H * 2 * W * (d / H) * 4);
@@ -78,18 +92,27 @@ size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
   B->xda = take(L * S * N * d * 4);
   B->xlse = take(L * S * N * H * 4);
   B->xD = take(L * S * N * H * 4);
-  // bf16 models: transposed weights and the bf16 GEMM operands
+  // bf16 models: transposed weights, the row-major bf16 operand, the group
+  // buffers of the weight-gradient products
   const bool tc = c.dtype == RLT_BF16;
   const size_t NP = (N + 63) / 64 * 64, WMAX = std::max(std::max(3 * d, F), 2 * d);
   const size_t ffn_mats = c.ffn_kind == RLT_SWIGLU ? 3 : 2;
   B->n_pad = (int)NP;
+  B->grp_layer_rows = bw_grp_layer_rows(c);
   B->wt = take(tc ? (L * (6 * d * d + ffn_mats * d * F) + 2 * d * d) * 2 : 0);
   B->xb = take(tc ? NP * WMAX * 2 : 0);
-  B->xt = take(tc ? NP * WMAX * 2 : 0);
-  B->yt = take(tc ? NP * WMAX * 2 : 0);
+  B->grp = take(tc ? (L * B->grp_layer_rows + 3 * d) * BW_GROUP * NP * 2 : 0);
+  // per group: rows of the gain gradients (ln1..ln3 per layer, lnf) and of
+  // the gate bias (dgpre)
+  B->gg = take((3 * L + 2) * BW_GROUP * N * d * 4);
   B->n_dev = take(4);
-  B->dmem = take((size_t)c.mem_groups * N * c.max_len * 2 * d * 4);
-  B->e32 = take(N * c.max_len * d * 4);
+  const size_t G = c.mem_groups, RP = (N * c.max_len + 63) / 64 * 64;
+  B->rows_pad = RP;
+  B->dmem = take(tc ? 0 : G * N * c.max_len * 2 * d * 4);
+  B->dmb = take(tc ? 4 * G * RP * d * 2 : 0);  // dK, dV row-major; dK^T, dV^T
+  B->eT = take(tc ? d * RP * 2 : 0);
+  B->wtm = take(tc ? 2 * G * d * d * 2 : 0);   // W_mk^T, W_mv^T
+  B->e32 = take(tc ? 0 : N * c.max_len * d * 4);
   B->de = take(N * c.max_len * d * 4);
   B->total = off;
   return off;
@@ -100,8 +123,8 @@ cudaError_t bw_gemm(int m, int n, int k, const TA *A, long lda, const TB *B, lon
                     long ldc, bool acc, cudaStream_t st) {
   if (m <= 0 || n <= 0) return cudaSuccess;
   dim3 grid((n + 63) / 64, (m + 63) / 64);
-  k_bw_gemm<TA, TB, AK, BK><<<grid, 256, 0, st>>>(m, n, k, A, lda, B, ldb, C, ldc, acc ? 1 : 0);
-  return cudaGetLastError();
+  return launch_k(k_bw_gemm<TA, TB, AK, BK>, grid, dim3(256), 0, st, m, n, k, A, lda, B, ldb, C,
+                  ldc, acc ? 1 : 0);
 }
 
 inline int bw_blocks(long total) { return (int)std::min<long>((total + 255) / 256, 148L * 16); }
@@ -124,6 +147,7 @@ template <typename T, int DH>
 cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float *sgrad,
                     const float *carry_in, float *carry_out, float *egrad, const rlt_grads *gr,
                     void *ws, cudaStream_t st) {
+  constexpr bool TC = std::is_same<T, bf16>::value;
   const rlt_config &c = M->cfg;
   const Layout &L = M->L;
   const int d = c.d, H = c.n_heads, F = c.ffn_dim, LD = c.n_dec_layers, W = c.window,
@@ -141,6 +165,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   float *xlse = reinterpret_cast<float *>(base + B.xlse), *xD = reinterpret_cast<float *>(base + B.xD);
   float *dmem = reinterpret_cast<float *>(base + B.dmem);
   float *e32 = reinterpret_cast<float *>(base + B.e32), *de = reinterpret_cast<float *>(base + B.de);
+  float *gg = reinterpret_cast<float *>(base + B.gg);
   BwStep S(reinterpret_cast<float *>(base + B.step), c, n);
   const int *ready = M->at<int>(L.ready);
   const T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem), *e = M->at<T>(L.e);
@@ -148,24 +173,58 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   const float2 *rope = M->at<float2>(L.rope);
   const size_t nd = (size_t)n * d;
   const int n_pad = B.n_pad;
-  bf16 *xb = reinterpret_cast<bf16 *>(base + B.xb), *xt = reinterpret_cast<bf16 *>(base + B.xt),
-       *yt = reinterpret_cast<bf16 *>(base + B.yt);
+  bf16 *xb = reinterpret_cast<bf16 *>(base + B.xb);
   int *n_dev = reinterpret_cast<int *>(base + B.n_dev);
   RLT_TRY(cudaMemcpyAsync(n_dev, &n, 4, cudaMemcpyHostToDevice, st));  // pageable: staged
+
+  // ---- group buffers: per layer the transposed operands of its weight
+  // gradients; the gate's after the last layer
+  struct GrpL {
+    bf16 *u1, *a1, *u2, *a2, *u3, *act, *dqkv, *dhs, *dhx, *dqx, *dhf, *dz, *dzb;
+  };
+  std::vector<GrpL> grp(LD, GrpL{});
+  bf16 *grp_cat = nullptr, *grp_dgpre = nullptr;
+  if (TC) {
+    bf16 *p = reinterpret_cast<bf16 *>(base + B.grp);
+    const size_t blk = (size_t)BW_GROUP * n_pad;
+    auto take = [&](int rows) {
+      bf16 *o = p;
+      p += (size_t)rows * blk;
+      return o;
+    };
+    for (int l = 0; l < LD; l++) {
+      GrpL &q = grp[l];
+      q.u1 = take(d);
+      q.a1 = take(d);
+      q.u2 = take(d);
+      q.a2 = take(d);
+      q.u3 = take(d);
+      q.act = take(F);
+      q.dqkv = take(3 * d);
+      q.dhs = take(d);
+      q.dhx = take(d);
+      q.dqx = take(d);
+      q.dhf = take(d);
+      q.dz = take(F);
+      q.dzb = swiglu ? take(F) : nullptr;
+    }
+    grp_cat = take(2 * d);
+    grp_dgpre = take(d);
+  }
+  // gain-gradient rows of a group: ln1, ln2, ln3 of layer l at 3l .. 3l+2,
+  // lnf at 3L, the gate bias at 3L + 1; row block `slot` within each
+  auto ggbuf = [&](int which, int slot_) {
+    return gg + ((size_t)which * BW_GROUP + slot_) * nd;
+  };
 
   // Transposed weights of the tensor-core forms (dX = dY W as a GEMM whose
   // B operand is W^T, K-major like every tcgen05 operand here).
   struct WT {
     const bf16 *qkv, *o, *qx, *ox, *w1, *wb, *w2;
   };
-  std::vector<WT> wt(LD);
+  std::vector<WT> wt(LD, WT{});
   const bf16 *wt_gate = nullptr;
-  auto pack = [&](const float *X, long ld, int K, bf16 *row_major, bf16 *transposed) {
-    k_bw_pack<<<dim3((K + 31) / 32, n_pad / 32), dim3(32, 8), 0, st>>>(n, n_pad, K, X, ld,
-                                                                        row_major, transposed);
-    return cudaGetLastError();
-  };
-  if constexpr (std::is_same<T, bf16>::value) {
+  if constexpr (TC) {
     bf16 *p = reinterpret_cast<bf16 *>(base + B.wt);
     auto tr = [&](const bf16 *Wm, int N, int K) {
       bf16 *o = p;
@@ -185,44 +244,84 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     if (c.alpha != 0.0f) wt_gate = tr((const T *)M->w.gate_w, d, 2 * d);
     RLT_TRY(cudaGetLastError());
   }
-  // out [n][N] = X [n][K] Wm^T (+ base)
-  auto fwd = [&](const float *X, int K, const T *Wm, int N, float *out,
-                 const float *base_) -> cudaError_t {
-    if constexpr (std::is_same<T, bf16>::value) {
-      RLT_TRY(pack(X, K, K, xb, nullptr));
+
+  // The group being filled: `cnt` steps, this step's column block `slot`.
+  int cnt = 0, slot = 0;
+  auto pack = [&](const float *X, long ld, int K, bf16 *row_major, bf16 *gbuf) {
+    RLT_TRY(launch_k(k_bw_pack, dim3((K + 31) / 32, n_pad / 32), dim3(32, 8), 0, st, 
+        n, n_pad, K, X, ld, row_major, gbuf, (long)cnt * n_pad, (long)slot * n_pad));
+    return cudaGetLastError();
+  };
+  // out [n][N] = X [n][K] Wm^T (+ base_); for bf16 X^T also goes to its
+  // group buffer (the operand of Wm's weight gradient)
+  auto fwd = [&](const float *X, int K, const T *Wm, int N, float *out, const float *base_,
+                 bf16 *gbuf) -> cudaError_t {
+    if constexpr (TC) {
+      RLT_TRY(pack(X, K, K, xb, gbuf));
       if (base_)
         return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, xb, Wm,
                               EpiAddF32Dec{{}, base_, out, N}, st);
       return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, xb, Wm, EpiF32Dec{{}, out, N}, st);
     } else {
-      if (base_) RLT_TRY(cudaMemcpyAsync(out, base_, (size_t)n * N * 4, cudaMemcpyDeviceToDevice, st));
+      (void)gbuf;
+      if (base_)
+        RLT_TRY(cudaMemcpyAsync(out, base_, (size_t)n * N * 4, cudaMemcpyDeviceToDevice, st));
       return bw_gemm<true, true>(n, N, K, X, K, Wm, K, out, N, base_ != nullptr, st);
     }
   };
-  // out [n][K] (=|+=) dY [n][N] Wm, Wm [N][K] (WTm its transpose)
-  auto dx = [&](const float *dY, int N, const T *Wm, const bf16 *WTm, int K, float *out,
-                bool acc) -> cudaError_t {
-    if constexpr (std::is_same<T, bf16>::value) {
-      RLT_TRY(pack(dY, N, N, xb, nullptr));
+  // out [n][K] (=|+=) dY [n][N] Wm (Wm [N][K], WTm its transpose), and the
+  // weight gradient dW [N][K] += dY^T X: staged in the group buffer for bf16
+  // (reduced at the group's end), at once for fp32 (X [n][K], pitch ldx).
+  auto bwd = [&](const float *dY, int N, const T *Wm, const bf16 *WTm, int K, float *out,
+                 bool acc, bf16 *gbuf, const float *X, long ldx, float *dW) -> cudaError_t {
+    if constexpr (TC) {
+      (void)X;
+      (void)ldx;
+      (void)dW;
+      RLT_TRY(pack(dY, N, N, xb, gbuf));
       if (acc)
         return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, xb, WTm, EpiAccF32Dec{{}, out, K},
                               st);
       return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, xb, WTm, EpiF32Dec{{}, out, K}, st);
     } else {
       (void)WTm;
+      (void)gbuf;
+      RLT_TRY((bw_gemm<false, false>(N, K, n, dY, N, X, ldx, dW, K, true, st)));
       return bw_gemm<true, false>(n, K, N, dY, N, Wm, K, out, K, acc, st);
     }
   };
-  // dW [N][K] += dY [n][N]^T X [n][K] (X with row pitch ldx)
-  auto dw = [&](const float *dY, int N, const float *X, long ldx, int K,
-                float *dW) -> cudaError_t {
-    if constexpr (std::is_same<T, bf16>::value) {
-      RLT_TRY(pack(dY, N, N, nullptr, yt));
-      RLT_TRY(pack(X, ldx, K, nullptr, xt));
-      return gemm_tc(M, N, N, 0, K, n_pad, yt, xt, EpiAccF32{dW, K}, st);
-    } else {
-      return bw_gemm<false, false>(N, K, n, dY, N, X, ldx, dW, K, true, st);
+  // dW [N][K] += (dY^T block)(X^T block)^T over the group's cnt x n_pad rows
+  auto grp_gemm = [&](const bf16 *yT, int N, const bf16 *xT, int K, float *dW) {
+    return gemm_tc(M, N, N, 0, K, cnt * n_pad, yT, xT, EpiAccF32{dW, K}, st);
+  };
+  // end of a group: the weight gradients and gain / bias sums of its steps
+  auto flush = [&]() -> cudaError_t {
+    const int rows = cnt * n;
+    auto colsum = [&](int which, float *out) {
+      RLT_TRY(launch_k(k_bw_colsum, (d + 31) / 32, dim3(32, 8), 0, st, rows, d, ggbuf(which, 0), out));
+      return cudaGetLastError();
+    };
+    for (int l = 0; l < LD; l++) {
+      RLT_TRY(colsum(3 * l, gr->dec_ln1[l]));
+      RLT_TRY(colsum(3 * l + 1, gr->dec_ln2[l]));
+      RLT_TRY(colsum(3 * l + 2, gr->dec_ln3[l]));
     }
+    RLT_TRY(colsum(3 * LD, gr->dec_lnf));
+    if (c.alpha != 0.0f) RLT_TRY(colsum(3 * LD + 1, gr->gate_b));
+    if constexpr (TC) {
+      for (int l = 0; l < LD; l++) {
+        const GrpL &q = grp[l];
+        RLT_TRY(grp_gemm(q.dqkv, 3 * d, q.u1, d, gr->dec_wqkv[l]));
+        RLT_TRY(grp_gemm(q.dhs, d, q.a1, d, gr->dec_wo[l]));
+        RLT_TRY(grp_gemm(q.dqx, d, q.u2, d, gr->dec_wqx[l]));
+        RLT_TRY(grp_gemm(q.dhx, d, q.a2, d, gr->dec_wox[l]));
+        RLT_TRY(grp_gemm(q.dz, F, q.u3, d, gr->dec_w1[l]));
+        if (swiglu) RLT_TRY(grp_gemm(q.dzb, F, q.u3, d, gr->dec_wb[l]));
+        RLT_TRY(grp_gemm(q.dhf, d, q.act, F, gr->dec_w2[l]));
+      }
+      if (c.alpha != 0.0f) RLT_TRY(grp_gemm(grp_dgpre, d, grp_cat, 2 * d, gr->gate_w));
+    }
+    return cudaSuccess;
   };
 
   // ---- forward of the chunk, recorded
@@ -234,9 +333,9 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   for (int k = 0; k < NS; k++) {
     RLT_TRY(enqueue_step(M, step_info(M, idv.data(), n), st));
     advance(M, idv.data(), n);
-    k_bw_hist_step<T><<<bw_blocks((long)LD * n * 2 * d), 256, 0, st>>>(
+    RLT_TRY(launch_k(k_bw_hist_step<T>, bw_blocks((long)LD * n * 2 * d), 256, 0, st, 
         n, ready, ring, s_arena, LD, H, DH, W, c.max_seqs, t0 + k, Wm1 + k, B.P, kv_hist,
-        s_hist + (size_t)(k + 1) * nd);
+        s_hist + (size_t)(k + 1) * nd));
     RLT_TRY(cudaGetLastError());
   }
 
@@ -248,22 +347,29 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
         n, LD, H, DH, W, t1, const_cast<float *>(carry_in), S.dcarry, dring, 0);
     RLT_TRY(cudaGetLastError());
   }
-  const int attn_blocks = (n * H * 32 + 127) / 128;
+  const int attn_blocks = n * H;  // one CTA of BW_ATT_WARPS warps per (row, head)
   auto hbuf = [&](int l, int which) { return S.h + ((size_t)3 * l + which) * nd; };
   auto ubuf = [&](int l, int which) { return S.u + ((size_t)3 * l + which) * nd; };
   auto rbuf = [&](int l, int which) { return S.r + ((size_t)3 * l + which) * n; };
+  // groups in processing order (t descending), the partial one first, so a
+  // group's column pitch is known when it starts
   for (int k = NS - 1; k >= 0; k--) {
+    if (slot == cnt) {
+      const int done = NS - 1 - k;
+      cnt = done == 0 && NS % BW_GROUP ? NS % BW_GROUP : BW_GROUP;
+      slot = 0;
+    }
     const long t = t0 + k;
     const float *s_prev = s_hist + (size_t)k * nd;
     // recompute the forward of step t
-    k_bw_gate_cat<T><<<bw_blocks(2 * (long)nd), 256, 0, st>>>(n, d, ready, e, c.max_len, t, s_prev,
-                                                              S.cat);
+    RLT_TRY(launch_k(k_bw_gate_cat<T>, bw_blocks(2 * (long)nd), 256, 0, st, n, d, ready, e, c.max_len, t, s_prev,
+                                                              S.cat));
     if (c.alpha != 0.0f)
-      RLT_TRY(fwd(S.cat, 2 * d, (const T *)M->w.gate_w, d, S.gpre, nullptr));
+      RLT_TRY(fwd(S.cat, 2 * d, (const T *)M->w.gate_w, d, S.gpre, nullptr, grp_cat));
     else
       RLT_TRY(cudaMemsetAsync(S.gpre, 0, nd * 4, st));
-    k_bw_gate_fwd<<<bw_blocks(nd), 256, 0, st>>>(n, d, S.gpre, (const float *)M->w.gate_b, S.cat,
-                                                 c.alpha, S.gs, hbuf(0, 0));
+    RLT_TRY(launch_k(k_bw_gate_fwd, bw_blocks(nd), 256, 0, st, n, d, S.gpre, (const float *)M->w.gate_b, S.cat,
+                                                 c.alpha, S.gs, hbuf(0, 0)));
     for (int l = 0; l < LD; l++) {
       const int g = G == 1 ? 0 : l;
       float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2), *hn = hbuf(l + 1, 0);
@@ -271,99 +377,97 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
       float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
       float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
             *act = S.act + (size_t)l * n * F;
-      k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h1, (const float *)M->w.dec_ln1[l], u1,
-                                      rbuf(l, 0));
-      RLT_TRY(fwd(u1, d, W_<T>::qkv(M, l), 3 * d, S.qkv, nullptr));
-      k_bw_rope_q<<<bw_blocks((long)n * d / 2), 256, 0, st>>>(n, H, DH, t, rope, S.qkv, q1);
+      const GrpL &q = grp[l];
+      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h1, (const float *)M->w.dec_ln1[l], u1,
+                                      rbuf(l, 0)));
+      RLT_TRY(fwd(u1, d, W_<T>::qkv(M, l), 3 * d, S.qkv, nullptr, q.u1));
+      RLT_TRY(launch_k(k_bw_rope_q, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, t, rope, S.qkv, q1));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
       const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
-      k_bw_attn_fwd<T, DH><<<attn_blocks, 128, 0, st>>>(n, H, swa, p_lo, p_hi, scale, q1, a1,
-                                                        S.lse1 + (size_t)l * n * H);
-      RLT_TRY(fwd(a1, d, W_<T>::o(M, l), d, h2, h1));
-      k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h2, (const float *)M->w.dec_ln2[l], u2,
-                                      rbuf(l, 1));
-      RLT_TRY(fwd(u2, d, (const T *)M->w.dec_wqx[l], d, qx, nullptr));
+      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
+          n, H, swa, p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H));
+      RLT_TRY(fwd(a1, d, W_<T>::o(M, l), d, h2, h1, q.a1));
+      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h2, (const float *)M->w.dec_ln2[l], u2,
+                                      rbuf(l, 1)));
+      RLT_TRY(fwd(u2, d, (const T *)M->w.dec_wqx[l], d, qx, nullptr, q.u2));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
-      k_bw_attn_fwd<T, DH><<<attn_blocks, 128, 0, st>>>(n, H, xk, 0, (int)t, scale, qx, a2,
-                                                        S.lse2 + (size_t)l * n * H);
-      RLT_TRY(fwd(a2, d, (const T *)M->w.dec_wox[l], d, h3, h2));
-      k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, h3, (const float *)M->w.dec_ln3[l], u3,
-                                      rbuf(l, 2));
-      RLT_TRY(fwd(u3, d, W_<T>::w1(M, l), F, z, nullptr));
-      if (swiglu) RLT_TRY(fwd(u3, d, W_<T>::wb(M, l), F, zb, nullptr));
-      k_bw_act_fwd<<<bw_blocks((long)n * F), 256, 0, st>>>((long)n * F, swiglu, z, zb, act);
-      RLT_TRY(fwd(act, F, W_<T>::w2(M, l), d, hn, h3));
+      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
+          n, H, xk, 0, (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H));
+      RLT_TRY(fwd(a2, d, (const T *)M->w.dec_wox[l], d, h3, h2, q.a2));
+      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h3, (const float *)M->w.dec_ln3[l], u3,
+                                      rbuf(l, 2)));
+      RLT_TRY(fwd(u3, d, W_<T>::w1(M, l), F, z, nullptr, q.u3));
+      if (swiglu) RLT_TRY(fwd(u3, d, W_<T>::wb(M, l), F, zb, nullptr, nullptr));
+      RLT_TRY(launch_k(k_bw_act_fwd, bw_blocks((long)n * F), 256, 0, st, (long)n * F, swiglu, z, zb, act));
+      RLT_TRY(fwd(act, F, W_<T>::w2(M, l), d, hn, h3, q.act));
     }
     float *rf = S.r + (size_t)3 * LD * n;
-    k_bw_rms_fwd<<<n, 256, 0, st>>>(d, c.rms_eps, hbuf(LD, 0), (const float *)M->w.dec_lnf,
-                                    S.ulast, rf);
+    RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, hbuf(LD, 0), (const float *)M->w.dec_lnf,
+                                    S.ulast, rf));
     RLT_TRY(cudaGetLastError());
 
     // differentiate step t: s_t = RMSNorm_f(h_L)
-    k_bw_ds_total<<<bw_blocks(nd), 256, 0, st>>>(n, d, NS, k, sgrad, S.dcarry, S.ds);
-    k_bw_rms_bwd<<<n, 256, 0, st>>>(d, hbuf(LD, 0), rf, (const float *)M->w.dec_lnf, S.ds, S.dh,
-                                    1);
-    k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.ds, hbuf(LD, 0), rf, gr->dec_lnf);
+    RLT_TRY(launch_k(k_bw_ds_total, bw_blocks(nd), 256, 0, st, n, d, NS, k, sgrad, S.dcarry, S.ds));
+    RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, hbuf(LD, 0), rf, (const float *)M->w.dec_lnf, S.ds, S.dh,
+                                    1, ggbuf(3 * LD, slot)));
     for (int l = LD - 1; l >= 0; l--) {
       float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2);
       float *u1 = ubuf(l, 0), *u2 = ubuf(l, 1), *u3 = ubuf(l, 2);
       float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
       float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
             *act = S.act + (size_t)l * n * F;
+      const GrpL &q = grp[l];
       // FFN: h_out = h3 + W2 act(W1 u3)
-      RLT_TRY(dx(S.dh, d, W_<T>::w2(M, l), wt[l].w2, F, S.dtmp, false));
-      RLT_TRY(dw(S.dh, d, act, F, F, gr->dec_w2[l]));
-      k_bw_act_bwd<<<bw_blocks((long)n * F), 256, 0, st>>>((long)n * F, swiglu, z, zb, S.dtmp,
-                                                           S.dz, S.dzb);
-      RLT_TRY(dw(S.dz, F, u3, d, d, gr->dec_w1[l]));
-      RLT_TRY(dx(S.dz, F, W_<T>::w1(M, l), wt[l].w1, d, S.du, false));
-      if (swiglu) {
-        RLT_TRY(dw(S.dzb, F, u3, d, d, gr->dec_wb[l]));
-        RLT_TRY(dx(S.dzb, F, W_<T>::wb(M, l), wt[l].wb, d, S.du, true));
-      }
-      k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h3, rbuf(l, 2), (const float *)M->w.dec_ln3[l], S.du,
-                                      S.dh, 0);
-      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.du, h3, rbuf(l, 2), gr->dec_ln3[l]);
+      RLT_TRY(bwd(S.dh, d, W_<T>::w2(M, l), wt[l].w2, F, S.dtmp, false, q.dhf, act, F,
+                  gr->dec_w2[l]));
+      RLT_TRY(launch_k(k_bw_act_bwd, bw_blocks((long)n * F), 256, 0, st, (long)n * F, swiglu, z, zb, S.dtmp,
+                                                           S.dz, S.dzb));
+      RLT_TRY(bwd(S.dz, F, W_<T>::w1(M, l), wt[l].w1, d, S.du, false, q.dz, u3, d,
+                  gr->dec_w1[l]));
+      if (swiglu)
+        RLT_TRY(bwd(S.dzb, F, W_<T>::wb(M, l), wt[l].wb, d, S.du, true, q.dzb, u3, d,
+                    gr->dec_wb[l]));
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h3, rbuf(l, 2), (const float *)M->w.dec_ln3[l], S.du,
+                                      S.dh, 0, ggbuf(3 * l + 2, slot)));
       // cross-attention: h3 = h2 + W_ox attn(W_qx u2, M<=t)
       const int g = G == 1 ? 0 : l;
-      RLT_TRY(dx(S.dh, d, (const T *)M->w.dec_wox[l], wt[l].ox, d, S.dtmp, false));
-      RLT_TRY(dw(S.dh, d, a2, d, d, gr->dec_wox[l]));
+      RLT_TRY(bwd(S.dh, d, (const T *)M->w.dec_wox[l], wt[l].ox, d, S.dtmp, false, q.dhx, a2, d,
+                  gr->dec_wox[l]));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
       const size_t xo = ((size_t)l * NS + k) * nd, xs = ((size_t)l * NS + k) * n * H;
-      k_bw_attn_bwd<T, DH><<<attn_blocks, 128, 0, st>>>(
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
           n, H, xk, 0, (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, S.dtmp, S.dq, nullptr,
-          W, 0, xq + xo, xda + xo, xlse + xs, xD + xs);
-      RLT_TRY(dw(S.dq, d, u2, d, d, gr->dec_wqx[l]));
-      RLT_TRY(dx(S.dq, d, (const T *)M->w.dec_wqx[l], wt[l].qx, d, S.du, false));
-      k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h2, rbuf(l, 1), (const float *)M->w.dec_ln2[l], S.du,
-                                      S.dh, 0);
-      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.du, h2, rbuf(l, 1), gr->dec_ln2[l]);
+          W, 0, xq + xo, xda + xo, xlse + xs, xD + xs));
+      RLT_TRY(bwd(S.dq, d, (const T *)M->w.dec_wqx[l], wt[l].qx, d, S.du, false, q.dqx, u2, d,
+                  gr->dec_wqx[l]));
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h2, rbuf(l, 1), (const float *)M->w.dec_ln2[l], S.du,
+                                      S.dh, 0, ggbuf(3 * l + 1, slot)));
       // SWA: h2 = h1 + W_o attn(q_t over the window); k_t, v_t enter the cache
-      RLT_TRY(dx(S.dh, d, W_<T>::o(M, l), wt[l].o, d, S.dtmp, false));
-      RLT_TRY(dw(S.dh, d, a1, d, d, gr->dec_wo[l]));
+      RLT_TRY(bwd(S.dh, d, W_<T>::o(M, l), wt[l].o, d, S.dtmp, false, q.dhs, a1, d,
+                  gr->dec_wo[l]));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
       const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
-      k_bw_attn_bwd<T, DH><<<attn_blocks, 128, 0, st>>>(
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
           n, H, swa, p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H, S.dtmp, S.dq, dring,
-          W, t0 - Wm1, nullptr, nullptr, nullptr, nullptr);
-      k_bw_qkv_grad<<<bw_blocks((long)n * d / 2), 256, 0, st>>>(
-          n, H, DH, W, t, rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv);
-      RLT_TRY(dw(S.dqkv, 3 * d, u1, d, d, gr->dec_wqkv[l]));
-      RLT_TRY(dx(S.dqkv, 3 * d, W_<T>::qkv(M, l), wt[l].qkv, d, S.du, false));
-      k_bw_rms_bwd<<<n, 256, 0, st>>>(d, h1, rbuf(l, 0), (const float *)M->w.dec_ln1[l], S.du,
-                                      S.dh, 0);
-      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.du, h1, rbuf(l, 0), gr->dec_ln1[l]);
+          W, t0 - Wm1, nullptr, nullptr, nullptr, nullptr));
+      RLT_TRY(launch_k(k_bw_qkv_grad, bw_blocks((long)n * d / 2), 256, 0, st, 
+          n, H, DH, W, t, rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv));
+      RLT_TRY(bwd(S.dqkv, 3 * d, W_<T>::qkv(M, l), wt[l].qkv, d, S.du, false, q.dqkv, u1, d,
+                  gr->dec_wqkv[l]));
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h1, rbuf(l, 0), (const float *)M->w.dec_ln1[l], S.du,
+                                      S.dh, 0, ggbuf(3 * l, slot)));
     }
     // gated merge: x = e_t + alpha sigmoid(W_g [e_t; s_{t-1}] + b_g) s_{t-1}
-    k_bw_gate_bwd<<<bw_blocks(nd), 256, 0, st>>>(n, d, c.alpha, S.dh, S.cat, S.gs, S.dgpre,
-                                                 S.dcarry, egrad, c.max_len, t);
+    float *dgpre = ggbuf(3 * LD + 1, slot);
+    RLT_TRY(launch_k(k_bw_gate_bwd, bw_blocks(nd), 256, 0, st, n, d, c.alpha, S.dh, S.cat, S.gs, dgpre,
+                                                 S.dcarry, egrad, c.max_len, t));
     if (c.alpha != 0.0f) {
-      k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.dgpre, nullptr, nullptr, gr->gate_b);
-      RLT_TRY(dw(S.dgpre, d, S.cat, 2 * d, 2 * d, gr->gate_w));
-      RLT_TRY(dx(S.dgpre, d, (const T *)M->w.gate_w, wt_gate, 2 * d, S.dtmp, false));
-      k_bw_gate_bwd2<<<bw_blocks(nd), 256, 0, st>>>(n, d, S.dtmp, S.dcarry, egrad, c.max_len, t);
+      RLT_TRY(bwd(dgpre, d, (const T *)M->w.gate_w, wt_gate, 2 * d, S.dtmp, false, grp_dgpre,
+                  S.cat, 2 * d, gr->gate_w));
+      RLT_TRY(launch_k(k_bw_gate_bwd2, bw_blocks(nd), 256, 0, st, n, d, S.dtmp, S.dcarry, egrad, c.max_len, t));
     }
     RLT_TRY(cudaGetLastError());
+    if (++slot == cnt) RLT_TRY(flush());
   }
   // the state entering the chunk
   if (carry_out) {
@@ -372,25 +476,62 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     RLT_TRY(cudaGetLastError());
   }
   if (t0 == 0)  // s_{-1} is the learned start state s*
-    k_bw_colsum<<<(d + 31) / 32, dim3(32, 8), 0, st>>>(n, d, S.dcarry, nullptr, nullptr, gr->sstar);
+    RLT_TRY(launch_k(k_bw_colsum, (d + 31) / 32, dim3(32, 8), 0, st, n, d, S.dcarry, gr->sstar));
 
   // ---- memory rows: dK, dV from the saved cross-attention terms, then
   // K^g = W_mk^g e, V^g = W_mv^g e differentiated into e and the projections
   constexpr int dm_smem = BwDmemSmem<T, DH>::BYTES;
   RLT_TRY(ensure_smem_limit(k_bw_dmem<T, DH>, dm_smem));
-  k_bw_dmem<T, DH><<<dim3((unsigned)((t1 + 63) / 64), H, n * G), 256, dm_smem, st>>>(
-      n, H, G, LD, NS, t0, c.max_seqs, c.max_len, ready, mem, xq, xda, xlse, xD, scale, dmem);
-  k_bw_gather_e<T><<<bw_blocks((long)n * t1 * d), 256, 0, st>>>(n, d, t1, c.max_len, ready, e, e32);
-  RLT_TRY(cudaGetLastError());
   const int rows = (int)(n * t1);
-  for (int g = 0; g < G; g++) {
-    const float *dk = dmem + (size_t)g * rows * 2 * d, *dv = dk + d;
-    RLT_TRY((bw_gemm<true, false>(rows, d, d, dk, 2 * d, (const T *)M->w.mem_wk[g], d, de, d,
-                                  g > 0, st)));
-    RLT_TRY((bw_gemm<true, false>(rows, d, d, dv, 2 * d, (const T *)M->w.mem_wv[g], d, de, d,
-                                  true, st)));
-    RLT_TRY((bw_gemm<false, false>(d, d, rows, dk, 2 * d, e32, d, gr->mem_wk[g], d, true, st)));
-    RLT_TRY((bw_gemm<false, false>(d, d, rows, dv, 2 * d, e32, d, gr->mem_wv[g], d, true, st)));
+  const dim3 dm_grid((unsigned)((t1 + 63) / 64), H, n * G);
+  if constexpr (TC) {
+    const long RP = (long)B.rows_pad;
+    bf16 *dkb = reinterpret_cast<bf16 *>(base + B.dmb), *dvb = dkb + (size_t)G * RP * d;
+    bf16 *dkT = dvb + (size_t)G * RP * d, *dvT = dkT + (size_t)G * RP * d;
+    bf16 *eT = reinterpret_cast<bf16 *>(base + B.eT);
+    const long rp = (rows + 63) / 64 * 64;  // this chunk's reduction length
+    if (rp > rows) {  // padding columns of the transposed operands read as zero
+      RLT_TRY(cudaMemset2DAsync(dkT + rows, rp * 2, 0, (rp - rows) * 2, (size_t)G * d, st));
+      RLT_TRY(cudaMemset2DAsync(dvT + rows, rp * 2, 0, (rp - rows) * 2, (size_t)G * d, st));
+    }
+    k_bw_dmem<T, DH><<<dm_grid, 256, dm_smem, st>>>(n, H, G, LD, NS, t0, c.max_seqs, c.max_len,
+                                                    ready, mem, xq, xda, xlse, xD, scale,
+                                                    nullptr, dkb, dvb, dkT, dvT, rp);
+    k_bw_e_transposed<T><<<dim3((d + 31) / 32, (unsigned)(rp / 32)), dim3(32, 8), 0, st>>>(
+        n, d, t1, c.max_len, rp, ready, e, eT);
+    RLT_TRY(cudaGetLastError());
+    RLT_TRY(cudaMemsetAsync(de, 0, (size_t)rows * d * 4, st));
+    bf16 *wtm = reinterpret_cast<bf16 *>(base + B.wtm);
+    for (int g = 0; g < G; g++) {
+      bf16 *wk = wtm + (size_t)2 * g * d * d, *wv = wk + (size_t)d * d;
+      k_bw_transpose<<<dim3((d + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, st>>>(
+          d, d, (const bf16 *)M->w.mem_wk[g], wk);
+      k_bw_transpose<<<dim3((d + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, st>>>(
+          d, d, (const bf16 *)M->w.mem_wv[g], wv);
+      RLT_TRY(cudaGetLastError());
+      const bf16 *gk = dkb + (size_t)g * rp * d, *gv = dvb + (size_t)g * rp * d;
+      RLT_TRY(gemm_tc(M, rows, rows, 0, d, d, gk, wk, EpiAccF32{de, d}, st));
+      RLT_TRY(gemm_tc(M, rows, rows, 0, d, d, gv, wv, EpiAccF32{de, d}, st));
+      const bf16 *tk = dkT + (size_t)g * d * rp, *tv = dvT + (size_t)g * d * rp;
+      RLT_TRY(gemm_tc(M, d, d, 0, d, (int)rp, tk, eT, EpiAccF32{gr->mem_wk[g], d}, st));
+      RLT_TRY(gemm_tc(M, d, d, 0, d, (int)rp, tv, eT, EpiAccF32{gr->mem_wv[g], d}, st));
+    }
+  } else {
+    k_bw_dmem<T, DH><<<dm_grid, 256, dm_smem, st>>>(n, H, G, LD, NS, t0, c.max_seqs, c.max_len,
+                                                    ready, mem, xq, xda, xlse, xD, scale, dmem,
+                                                    nullptr, nullptr, nullptr, nullptr, 0);
+    k_bw_gather_e<T><<<bw_blocks((long)n * t1 * d), 256, 0, st>>>(n, d, t1, c.max_len, ready, e,
+                                                                  e32);
+    RLT_TRY(cudaGetLastError());
+    for (int g = 0; g < G; g++) {
+      const float *dk = dmem + (size_t)g * rows * 2 * d, *dv = dk + d;
+      RLT_TRY((bw_gemm<true, false>(rows, d, d, dk, 2 * d, (const T *)M->w.mem_wk[g], d, de, d,
+                                    g > 0, st)));
+      RLT_TRY((bw_gemm<true, false>(rows, d, d, dv, 2 * d, (const T *)M->w.mem_wv[g], d, de, d,
+                                    true, st)));
+      RLT_TRY((bw_gemm<false, false>(d, d, rows, dk, 2 * d, e32, d, gr->mem_wk[g], d, true, st)));
+      RLT_TRY((bw_gemm<false, false>(d, d, rows, dv, 2 * d, e32, d, gr->mem_wv[g], d, true, st)));
+    }
   }
   k_bw_add_e<<<bw_blocks((long)rows * d), 256, 0, st>>>(n, d, t1, c.max_len, de, egrad);
   return cudaGetLastError();
