@@ -371,11 +371,56 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
             "TFLOP_s": pr["flops"] / (par_ms / 1e3) / 1e12,
             "bound": "tensor" if pr["flops"] / (tc * 1e12) >= pr["bytes"] / (hbm * 1e9) else "hbm",
         }
+    if args.backward and not r.ragged and cfg.dtype == configs.BF16:
+        out["backward"] = time_backward(wl, r, dist, hbm, tc)
     if args.serve and wl.prompt_lengths and not r.ragged and cfg.dtype == configs.BF16:
         out["serve"] = time_serve(wl, r, dist)
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_positions)
     return out
+
+
+def time_backward(wl, r, dist, hbm, tc):
+    """Backpropagation through time over the whole workload (outside the
+    contract timing): encoder prefill, then one rlt_backward over every
+    position of every sequence (recorded forward, reverse traversal, memory
+    gradient), upstream gradients dL/ds_t seeded N(0, 1); one short call first
+    warms the graphs and tensor maps. Reports seq-steps/s of the timed call."""
+    import torch
+    cfg = wl.model
+    T = int(r.lengths[0])
+    m = r.m
+    g = torch.Generator(device="cuda").manual_seed(2)
+    sgrad = torch.randn((wl.batch, T, cfg.d), generator=g, device="cuda")
+    grads = {k: torch.zeros(v, device="cuda") for k, v in m.grad_shapes().items()}
+    egrad = torch.zeros((wl.batch, wl.max_len, cfg.d), device="cuda")
+    ws = torch.empty(m.backward_workspace_bytes(wl.batch, T), dtype=torch.uint8, device="cuda")
+    ids = r.ids
+    m.prefill_encoder(r.tok_dev, ids, r.offsets, r.lengths)
+    m.backward(ids, sgrad[:, :8].contiguous(), grads=grads, egrad=egrad, workspace=ws)
+    m.prefill_encoder(r.tok_dev, ids, r.offsets, r.lengths)
+    torch.cuda.synchronize()
+    barrier(dist)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(r.stream)
+    m.backward(ids, sgrad, grads=grads, egrad=egrad, workspace=ws)
+    b.record(r.stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), dist)
+    assert m.poll_device_error() == 0
+    finite = bool(torch.isfinite(grads["dec.0.wqkv"]).all().item())
+    gb = ws.numel() / 1e9
+    del ws, grads, egrad, sgrad
+    torch.cuda.empty_cache()
+    world = dist.get_world_size() if dist is not None else 1
+    br = roofline.backward_roofline(cfg, wl.lengths, hbm, tc)
+    return {"seq_steps_per_s": world * wl.batch * T / (ms / 1e3), "ms_per_pass": ms,
+            "roofline_s": br["seconds"], "frac": br["seconds"] / (ms / 1e3),
+            "TFLOP_s": br["flops"] / (ms / 1e3) / 1e12, "workspace_gb": gb,
+            "grads_finite": finite,
+            "note": "rlt_backward over all positions: recorded forward on the step kernels, "
+                    "reverse traversal, memory-row gradient and projection"}
 
 
 def time_serve(wl, r, dist):
@@ -493,6 +538,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--serve", action=argparse.BooleanOptionalAction, default=True,
                     help="also time the autoregressive form (generated tokens/s)")
+    ap.add_argument("--backward", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time backpropagation through time over the workload")
     ap.add_argument("--cpu-positions", type=int, default=24)
     ap.add_argument("--profile-stride", type=int, default=64,
                     help="event-time every k-th decoder step for the per-kernel roofline")

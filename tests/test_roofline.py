@@ -78,3 +78,17 @@ def test_parallel_pass_flops_match_an_enumeration():
     assert r["flops"] == pytest.approx(f, rel=1e-12)
     assert r["seq_steps"] == sum(lengths)
     assert r["seconds"] == pytest.approx(max(f / (TC * 1e12), r["bytes"] / (HBM * 1e9)))
+
+
+def test_backward_roofline_counts_three_forward_steps_of_bytes():
+    """The backward's bytes are three forward steps' per step (recorded,
+    recomputed, differentiated); its FLOPs four forward steps' plus the
+    memory projection's backward."""
+    cfg = configs.M140
+    lengths = [40, 40]
+    br = roofline.backward_roofline(cfg, lengths, 6650.0, 1400.0)
+    fw = roofline.run_roofline(cfg, lengths, 6650.0, 1400.0)
+    assert abs(br["bytes"] - 3 * fw["decoder_bytes"]) <= 1e-9 * br["bytes"]
+    extra = 8.0 * cfg.d * cfg.d * cfg.mem_groups * sum(lengths)
+    assert abs(br["flops"] - (4 * fw["decoder_flops"] + extra)) <= 1e-9 * br["flops"]
+    assert br["seconds"] >= 3 * fw["decoder_s"] * (1 - 1e-9)

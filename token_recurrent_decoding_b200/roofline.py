@@ -120,3 +120,24 @@ def backward_flops(cfg: RLTConfig, lengths) -> float:
         t = np.arange(T, dtype=np.float64)
         tot += 4 * decoder_step_flops(cfg, t) + 8.0 * cfg.d * cfg.d * cfg.mem_groups * T
     return float(tot)
+
+
+def backward_roofline(cfg: RLTConfig, lengths, hbm_gbs: float, tensor_tflops: float):
+    """Roofline of rlt_backward over full sequences (lock-step): per step the
+    recorded forward, the recomputed forward and the backward each move about
+    one forward step's bytes (weights, the window and memory rows; the
+    backward reads W^T and the same keys and values again), and the FLOPs are
+    backward_flops; the larger time bounds each step."""
+    lengths = np.asarray(lengths)
+    T = int(lengths.max())
+    sec = 0.0
+    tot_b = 0.0
+    for t in range(T):
+        n = int(np.sum(lengths > t))
+        ts = np.full(n, t)
+        b = 3.0 * decoder_step_bytes(cfg, ts)
+        f = 4.0 * decoder_step_flops(cfg, ts) + 8.0 * cfg.d * cfg.d * cfg.mem_groups * n
+        tot_b += b
+        sec += max(b / (hbm_gbs * 1e9), f / (tensor_tflops * 1e12))
+    return {"seconds": sec, "bytes": tot_b, "flops": backward_flops(cfg, lengths),
+            "seq_steps": int(lengths.sum())}
