@@ -31,6 +31,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "enc_attn.cuh"
 
 namespace rlt {
 
@@ -847,6 +848,177 @@ __global__ void __launch_bounds__(256)
         o[x] = dK[x];
         o[d + x] = dV[x];
       }
+    }
+  }
+}
+
+// The same memory-row gradient on the tensor cores (bf16 models, DH 32 or
+// 64), with the warp-level bf16 MMA of the flash attention kernel: a CTA of
+// four warps owns 64 memory rows j of one (group, row, head), 16 per warp,
+// their K_j and V_j rows held as A fragments; per tile of 64 steps the saved
+// queries and output gradients (rounded to bf16) sit in shared memory, and
+//   S = K_j Q^T,  dP = V_j dA^T  (16 x 64 per warp),
+//   P = exp(scale S - lse) on the causal set (j <= t), dS = P (dP - D),
+//   dV_j += P dA,  dK_j += scale dS Q
+// accumulate in registers (P and dS rounded to bf16 as MMA operands). The
+// results go out as the bf16 operands of the projection's GEMMs.
+template <int DH>
+__global__ void __launch_bounds__(128)
+    k_bw_dmem_mma(int n, int H, int G, int L, int n_steps, long t0, int max_seqs, int max_len,
+                  const int *__restrict__ ready, const bf16 *__restrict__ mem,
+                  const float *__restrict__ xq, const float *__restrict__ xda,
+                  const float *__restrict__ xlse, const float *__restrict__ xD, float scale,
+                  bf16 *__restrict__ dkb, bf16 *__restrict__ dvb, bf16 *__restrict__ dkT,
+                  bf16 *__restrict__ dvT, long rows_pad) {
+  static_assert(DH == 32 || DH == 64, "swizzled 64 x DH tiles of the flash kernel");
+  constexpr int KS = DH / 16;   // k-steps over the head dimension
+  constexpr int ONT = DH / 8;   // n-tiles of dK, dV
+  constexpr int NCH = DH / 8;   // 16-byte chunks per tile row
+  __shared__ __align__(128) bf16 Qs[64 * DH];
+  __shared__ __align__(128) bf16 As[64 * DH];
+  __shared__ float ls[64], Ds[64];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g_ = lane >> 2, tq = lane & 3;
+  const int j0 = blockIdx.x * 64, h = blockIdx.y, i = blockIdx.z % n, g = blockIdx.z / n;
+  const int d = H * DH;
+  const long t1 = t0 + n_steps;
+  const int seq = ready[i];
+  const bf16 *Kg = mem + ((((size_t)g * max_seqs + seq) * H + h) * 2) * max_len * DH;
+  const bf16 *Vg = Kg + (size_t)max_len * DH;
+  // this warp's 16 memory rows as A fragments (rows past t1 read as zero)
+  const int jr0 = j0 + warp * 16 + g_, jr1 = jr0 + 8;
+  uint32_t ka[KS][4], va[KS][4];
+#pragma unroll
+  for (int ks = 0; ks < KS; ks++) {
+    const int k0 = ks * 16 + tq * 2;
+    auto ld2 = [&](const bf16 *X, int row, int col) -> uint32_t {
+      if (row >= t1) return 0u;
+      return *reinterpret_cast<const uint32_t *>(X + (size_t)row * DH + col);
+    };
+    ka[ks][0] = ld2(Kg, jr0, k0);
+    ka[ks][1] = ld2(Kg, jr1, k0);
+    ka[ks][2] = ld2(Kg, jr0, k0 + 8);
+    ka[ks][3] = ld2(Kg, jr1, k0 + 8);
+    va[ks][0] = ld2(Vg, jr0, k0);
+    va[ks][1] = ld2(Vg, jr1, k0);
+    va[ks][2] = ld2(Vg, jr0, k0 + 8);
+    va[ks][3] = ld2(Vg, jr1, k0 + 8);
+  }
+  float dk[ONT][4], dv[ONT][4];
+#pragma unroll
+  for (int x = 0; x < ONT; x++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) dk[x][e] = dv[x][e] = 0.f;
+  const int l_lo = G == 1 ? 0 : g, l_hi = G == 1 ? L : g + 1;
+  const int k_first = (int)(j0 > t0 ? (j0 - t0) / 64 * 64 : 0);
+  for (int l = l_lo; l < l_hi; l++) {
+    for (int kt0 = k_first; kt0 < n_steps; kt0 += 64) {
+      __syncthreads();
+      // the tile's queries and output gradients, bf16 into swizzled rows
+      for (int c = tid; c < 64 * NCH; c += 128) {
+        const int r = c / NCH, ch = c % NCH, k = kt0 + r;
+        float qv[8], av[8];
+        if (k < n_steps) {
+          const size_t o = (((size_t)l * n_steps + k) * n + i) * d + h * DH + ch * 8;
+          bw_ld8(xq + o, qv);
+          bw_ld8(xda + o, av);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; e++) qv[e] = av[e] = 0.f;
+        }
+        uint4 qp, ap;
+        qp.x = pack_bf16(qv[0], qv[1]); qp.y = pack_bf16(qv[2], qv[3]);
+        qp.z = pack_bf16(qv[4], qv[5]); qp.w = pack_bf16(qv[6], qv[7]);
+        ap.x = pack_bf16(av[0], av[1]); ap.y = pack_bf16(av[2], av[3]);
+        ap.z = pack_bf16(av[4], av[5]); ap.w = pack_bf16(av[6], av[7]);
+        *reinterpret_cast<uint4 *>(Qs + fa_swz<DH>(r, ch)) = qp;
+        *reinterpret_cast<uint4 *>(As + fa_swz<DH>(r, ch)) = ap;
+      }
+      if (tid < 64) {
+        const int k = kt0 + tid;
+        const size_t o = (((size_t)l * n_steps + k) * n + i) * H + h;
+        ls[tid] = k < n_steps ? xlse[o] : 0.f;
+        Ds[tid] = k < n_steps ? xD[o] : 0.f;
+      }
+      __syncthreads();
+      // S = K_j Q^T and dP = V_j dA^T for 16 rows x 64 steps
+      float sc[8][4], dp[8][4];
+#pragma unroll
+      for (int x = 0; x < 8; x++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) sc[x][e] = dp[x][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ks++) {
+#pragma unroll
+        for (int jp = 0; jp < 4; jp++) {
+          const int r = jp * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int ch = ks * 2 + ((lane >> 3) & 1);
+          uint32_t b4[4];
+          ldmatrix_x4(b4, smem_u32(Qs + fa_swz<DH>(r, ch)));
+          uint32_t b0[2] = {b4[0], b4[1]}, b1[2] = {b4[2], b4[3]};
+          mma_bf16_16816(sc[2 * jp], ka[ks], b0);
+          mma_bf16_16816(sc[2 * jp + 1], ka[ks], b1);
+          ldmatrix_x4(b4, smem_u32(As + fa_swz<DH>(r, ch)));
+          uint32_t c0[2] = {b4[0], b4[1]}, c1[2] = {b4[2], b4[3]};
+          mma_bf16_16816(dp[2 * jp], va[ks], c0);
+          mma_bf16_16816(dp[2 * jp + 1], va[ks], c1);
+        }
+      }
+      // P and dS on the causal set, as bf16 A fragments (16 steps per k-step)
+      uint32_t pa[4][4], sa[4][4];
+#pragma unroll
+      for (int x = 0; x < 8; x++) {
+        float p[4], q[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const int kk = x * 8 + tq * 2 + (e & 1);
+          const int row = (e < 2) ? jr0 : jr1;
+          const long t = t0 + kt0 + kk;
+          const bool ok = kt0 + kk < n_steps && row <= t && row < t1;
+          const float pv = ok ? expf(sc[x][e] * scale - ls[kk]) : 0.f;
+          p[e] = pv;
+          q[e] = pv * (dp[x][e] - Ds[kk]);
+        }
+        pa[x >> 1][(x & 1) * 2 + 0] = pack_bf16(p[0], p[1]);
+        pa[x >> 1][(x & 1) * 2 + 1] = pack_bf16(p[2], p[3]);
+        sa[x >> 1][(x & 1) * 2 + 0] = pack_bf16(q[0], q[1]);
+        sa[x >> 1][(x & 1) * 2 + 1] = pack_bf16(q[2], q[3]);
+      }
+      // dV += P dA, dK += dS Q (B operands through ldmatrix.trans)
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) {
+#pragma unroll
+        for (int jp = 0; jp < ONT / 2; jp++) {
+          const int r = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+          const int ch = jp * 2 + (lane >> 4);
+          uint32_t b4[4];
+          ldmatrix_x4_trans(b4, smem_u32(As + fa_swz<DH>(r, ch)));
+          uint32_t b0[2] = {b4[0], b4[1]}, b1[2] = {b4[2], b4[3]};
+          mma_bf16_16816(dv[2 * jp], pa[kk], b0);
+          mma_bf16_16816(dv[2 * jp + 1], pa[kk], b1);
+          ldmatrix_x4_trans(b4, smem_u32(Qs + fa_swz<DH>(r, ch)));
+          uint32_t c0[2] = {b4[0], b4[1]}, c1[2] = {b4[2], b4[3]};
+          mma_bf16_16816(dk[2 * jp], sa[kk], c0);
+          mma_bf16_16816(dk[2 * jp + 1], sa[kk], c1);
+        }
+      }
+    }
+  }
+  // rows (i, j): bf16 row-major and transposed operands of the projection
+  const size_t gr = (size_t)g * rows_pad;
+#pragma unroll
+  for (int x = 0; x < ONT; x++) {
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int row = (e < 2) ? jr0 : jr1;
+      if (row >= t1) continue;
+      const int col = h * DH + x * 8 + tq * 2 + (e & 1);
+      const size_t rr = (size_t)i * t1 + row;
+      const bf16 kv = __float2bfloat16_rn(dk[x][e] * scale), vv = __float2bfloat16_rn(dv[x][e]);
+      dkb[(gr + rr) * d + col] = kv;
+      dvb[(gr + rr) * d + col] = vv;
+      dkT[((size_t)g * d + col) * rows_pad + rr] = kv;
+      dvT[((size_t)g * d + col) * rows_pad + rr] = vv;
     }
   }
 }

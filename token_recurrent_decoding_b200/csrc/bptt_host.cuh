@@ -494,9 +494,14 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
       RLT_TRY(cudaMemset2DAsync(dkT + rows, rp * 2, 0, (rp - rows) * 2, (size_t)G * d, st));
       RLT_TRY(cudaMemset2DAsync(dvT + rows, rp * 2, 0, (rp - rows) * 2, (size_t)G * d, st));
     }
-    k_bw_dmem<T, DH><<<dm_grid, 256, dm_smem, st>>>(n, H, G, LD, NS, t0, c.max_seqs, c.max_len,
-                                                    ready, mem, xq, xda, xlse, xD, scale,
-                                                    nullptr, dkb, dvb, dkT, dvT, rp);
+    if constexpr (DH == 32 || DH == 64)
+      k_bw_dmem_mma<DH><<<dm_grid, 128, 0, st>>>(n, H, G, LD, NS, t0, c.max_seqs, c.max_len,
+                                                 ready, (const bf16 *)mem, xq, xda, xlse, xD,
+                                                 scale, dkb, dvb, dkT, dvT, rp);
+    else
+      k_bw_dmem<T, DH><<<dm_grid, 256, dm_smem, st>>>(n, H, G, LD, NS, t0, c.max_seqs,
+                                                      c.max_len, ready, mem, xq, xda, xlse, xD,
+                                                      scale, nullptr, dkb, dvb, dkT, dvT, rp);
     k_bw_e_transposed<T><<<dim3((d + 31) / 32, (unsigned)(rp / 32)), dim3(32, 8), 0, st>>>(
         n, d, t1, c.max_len, rp, ready, e, eT);
     RLT_TRY(cudaGetLastError());

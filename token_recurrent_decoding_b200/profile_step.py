@@ -217,9 +217,13 @@ def run_backward(args):
     flat = torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda()
     ids = list(range(B))
     m.prefill_encoder(flat, ids, np.arange(B, dtype=np.int32) * T, lengths)
+    t0 = args.bw_start  # the chunk covers positions t0 .. T-1
+    if t0:
+        m.run_sequence(ids, t0)
     start = [m.get_state(i) for i in ids]
-    sgrad = torch.randn((B, T, cfg.d), device="cuda", generator=torch.Generator("cuda").manual_seed(3))
-    ws = torch.empty(m.backward_workspace_bytes(B, T), dtype=torch.uint8, device="cuda")
+    NS = T - t0
+    sgrad = torch.randn((B, NS, cfg.d), device="cuda", generator=torch.Generator("cuda").manual_seed(3))
+    ws = torch.empty(m.backward_workspace_bytes(B, NS), dtype=torch.uint8, device="cuda")
     grads = {k: torch.zeros(v, device="cuda") for k, v in m.grad_shapes().items()}
     egrad = torch.zeros((B, T, cfg.d), device="cuda")
     times = []
@@ -235,8 +239,8 @@ def run_backward(args):
     assert m.poll_device_error() == 0
     flops = roofline.backward_flops(cfg, lengths)
     best = min(times)
-    print(json.dumps({"workload": args.workload, "batch": B, "T": T, "backward_ms": times,
-                      "seq_steps_per_s": B * T / (best / 1e3),
+    print(json.dumps({"workload": args.workload, "batch": B, "T": T, "start": t0,
+                      "backward_ms": times, "seq_steps_per_s": B * NS / (best / 1e3),
                       "tflops": flops / (best / 1e3) / 1e12,
                       "workspace_gb": ws.numel() / 1e9}))
 
@@ -262,6 +266,8 @@ def main():
     ap.add_argument("--attend", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time rlt_backward over --max-len positions of --batch sequences")
+    ap.add_argument("--bw-start", type=int, default=0,
+                    help="backward chunk starts at this position (the forward runs there first)")
     ap.add_argument("--parallel", action="store_true",
                     help="time the token-parallel decoder pass (feedback-off workloads)")
     ap.add_argument("--n", type=int, default=256)
