@@ -190,6 +190,38 @@ __global__ void k_bw_transpose(int N, int K, const bf16 *__restrict__ W, bf16 *_
   }
 }
 
+// The transposed bf16 operands of one group's weight gradients: for each
+// listed matrix (row-major bf16 [n][K] as its producer wrote it), rows 0..n-1
+// into columns col0 .. col0+n-1 of dst [K][pitch], columns up to col0 + n_pad
+// zero. blockIdx.y picks the matrix; 32 x 32 tiles through shared memory.
+struct BwTr {
+  const bf16 *src;
+  bf16 *dst;
+  int K;
+};
+
+__global__ void k_bw_grp_transpose(const BwTr *__restrict__ list, int n, int n_pad, long pitch,
+                                   long col0) {
+  BW_PDL();
+  __shared__ bf16 tile[32][34];
+  const BwTr m = list[blockIdx.y];
+  const int tiles_c = (m.K + 31) / 32, tiles = tiles_c * (n_pad / 32);
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int b = blockIdx.x; b < tiles; b += gridDim.x) {
+    const int c0 = (b % tiles_c) * 32, r0 = (b / tiles_c) * 32;
+    __syncthreads();
+    for (int y = ty; y < 32; y += 8) {
+      const int r = r0 + y, c = c0 + tx;
+      tile[y][tx] = (r < n && c < m.K) ? m.src[(size_t)r * m.K + c] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    for (int y = ty; y < 32; y += 8) {
+      const int c = c0 + y, r = r0 + tx;
+      if (c < m.K && r < n_pad) m.dst[(size_t)c * pitch + col0 + r] = tile[tx][y];
+    }
+  }
+}
+
 // --------------------------------------------------------------- helpers
 // Sum over the block (blockDim.x a multiple of 32, at most 1024).
 __device__ __forceinline__ float bw_block_sum(float v, float *red) {
@@ -276,14 +308,16 @@ __global__ void k_bw_hist_step(int n, const int *__restrict__ ready, const T *__
 template <typename T>
 __global__ void k_bw_gate_cat(int n, int d, const int *__restrict__ ready, const T *__restrict__ e,
                               int max_len, long t, const float *__restrict__ s_prev,
-                              float *__restrict__ cat) {
+                              float *__restrict__ cat, bf16 *__restrict__ catb) {
   BW_PDL();
   const long total = (long)n * 2 * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
     const int i = (int)(idx / (2 * d)), c = (int)(idx % (2 * d));
-    cat[idx] = c < d ? to_f(e[((size_t)ready[i] * max_len + t) * d + c])
-                     : s_prev[(size_t)i * d + c - d];
+    const float v = c < d ? to_f(e[((size_t)ready[i] * max_len + t) * d + c])
+                          : s_prev[(size_t)i * d + c - d];
+    cat[idx] = v;
+    if (catb) catb[idx] = __float2bfloat16_rn(v);
   }
 }
 
@@ -305,7 +339,7 @@ __global__ void k_bw_gate_fwd(int n, int d, const float *__restrict__ gpre,
 // u = h r gamma, r = 1 / sqrt(mean(h^2) + eps); one block per row.
 __global__ void k_bw_rms_fwd(int d, float eps, const float *__restrict__ h,
                              const float *__restrict__ gamma, float *__restrict__ u,
-                             float *__restrict__ r) {
+                             float *__restrict__ r, bf16 *__restrict__ ub) {
   BW_PDL();
   __shared__ float red[32];
   const float *x = h + (size_t)blockIdx.x * d;
@@ -314,8 +348,11 @@ __global__ void k_bw_rms_fwd(int d, float eps, const float *__restrict__ h,
   ss = bw_block_sum(ss, red);
   const float rr = rsqrtf(ss / d + eps);
   if (threadIdx.x == 0) r[blockIdx.x] = rr;
-  for (int c = threadIdx.x; c < d; c += blockDim.x)
-    u[(size_t)blockIdx.x * d + c] = x[c] * rr * gamma[c];
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float v = x[c] * rr * gamma[c];
+    if (u) u[(size_t)blockIdx.x * d + c] = v;
+    if (ub) ub[(size_t)blockIdx.x * d + c] = __float2bfloat16_rn(v);
+  }
 }
 
 // Rotary encoding of the q part of a [n][3d] q/k/v row at position t.
@@ -336,11 +373,15 @@ __global__ void k_bw_rope_q(int n, int H, int dh, long t, const float2 *__restri
 
 // GELU or SwiGLU activation of the FFN: act = GELU(z) or SiLU(z) zb.
 __global__ void k_bw_act_fwd(long total, int swiglu, const float *__restrict__ z,
-                             const float *__restrict__ zb, float *__restrict__ act) {
+                             const float *__restrict__ zb, float *__restrict__ act,
+                             bf16 *__restrict__ actb) {
   BW_PDL();
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (long)gridDim.x * blockDim.x)
-    act[idx] = swiglu ? silu(z[idx]) * zb[idx] : gelu_erf(z[idx]);
+       idx += (long)gridDim.x * blockDim.x) {
+    const float v = swiglu ? silu(z[idx]) * zb[idx] : gelu_erf(z[idx]);
+    if (act) act[idx] = v;
+    if (actb) actb[idx] = __float2bfloat16_rn(v);
+  }
 }
 
 // Where the keys of one (row, head) live. SWA: the recorded window in
@@ -407,7 +448,8 @@ constexpr int BW_ATT_WARPS = 4;
 template <typename T, int DH>
 __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
     k_bw_attn_fwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
-                  const float *__restrict__ q, float *__restrict__ a, float *__restrict__ lse) {
+                  const float *__restrict__ q, float *__restrict__ a, float *__restrict__ lse,
+                  bf16 *__restrict__ ab) {
   BW_PDL();
   constexpr int LPK = DH / 8, KPW = 32 / LPK;
   __shared__ float red[BW_ATT_WARPS][2 + DH];
@@ -461,7 +503,11 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
   if (warp == 0 && grp == 0) {
     for (int w = 1; w < BW_ATT_WARPS; w++) bw_merge(m, l, acc, red[w][0], red[w][1], &red[w][2 + sl * 8]);
 #pragma unroll
-    for (int e = 0; e < 8; e++) a[(size_t)i * d + h * DH + sl * 8 + e] = acc[e] / l;
+    for (int e = 0; e < 8; e++) {
+      const float v = acc[e] / l;
+      a[(size_t)i * d + h * DH + sl * 8 + e] = v;
+      if (ab) ab[(size_t)i * d + h * DH + sl * 8 + e] = __float2bfloat16_rn(v);
+    }
     if (sl == 0) lse[(size_t)i * H + h] = m + logf(l);
   }
 }
@@ -482,7 +528,7 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
                   const float *__restrict__ lse, const float *__restrict__ da,
                   float *__restrict__ dq, float *__restrict__ dring, int W, long pos0,
                   float *__restrict__ xq, float *__restrict__ xda, float *__restrict__ xlse,
-                  float *__restrict__ xD) {
+                  float *__restrict__ xD, bf16 *__restrict__ dqb) {
   BW_PDL();
   constexpr int LPK = DH / 8, KPW = 32 / LPK;
   __shared__ float red[BW_ATT_WARPS][DH];
@@ -562,6 +608,7 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
 #pragma unroll
     for (int e = 0; e < 8; e++) {
       dq[off + e] = dqv[e];
+      if (dqb) dqb[off + e] = __float2bfloat16_rn(dqv[e]);
       if (xq) {
         xq[off + e] = qv[e];
         xda[off + e] = dav[e];
@@ -579,7 +626,7 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
 // t mod W; dv_t as is. The slot is cleared for position t - W.
 __global__ void k_bw_qkv_grad(int n, int H, int dh, int W, long t, const float2 *__restrict__ rope,
                               const float *__restrict__ dq, float *__restrict__ dring_l,
-                              float *__restrict__ dqkv) {
+                              float *__restrict__ dqkv, bf16 *__restrict__ dqkvb) {
   BW_PDL();
   const int d = H * dh, half = dh / 2;
   const long total = (long)n * H * half;
@@ -598,6 +645,15 @@ __global__ void k_bw_qkv_grad(int n, int H, int dh, int W, long t, const float2 
     o[d + j + half] = -ka * cs.y + kb * cs.x;
     o[2 * d + j] = dv[j];
     o[2 * d + j + half] = dv[j + half];
+    if (dqkvb) {
+      bf16 *b = dqkvb + (size_t)i * 3 * d + h * dh;
+      b[j] = __float2bfloat16_rn(o[j]);
+      b[j + half] = __float2bfloat16_rn(o[j + half]);
+      b[d + j] = __float2bfloat16_rn(o[d + j]);
+      b[d + j + half] = __float2bfloat16_rn(o[d + j + half]);
+      b[2 * d + j] = __float2bfloat16_rn(o[2 * d + j]);
+      b[2 * d + j + half] = __float2bfloat16_rn(o[2 * d + j + half]);
+    }
     dk[j] = dk[j + half] = 0.f;
     dv[j] = dv[j + half] = 0.f;
   }
@@ -609,7 +665,8 @@ __global__ void k_bw_qkv_grad(int n, int H, int dh, int W, long t, const float2 
 // The gain's gradient per row, du h r, goes to gg (summed over rows later).
 __global__ void k_bw_rms_bwd(int d, const float *__restrict__ h, const float *__restrict__ r,
                              const float *__restrict__ gamma, const float *__restrict__ du,
-                             float *__restrict__ dh, int assign, float *__restrict__ gg) {
+                             float *__restrict__ dh, int assign, float *__restrict__ gg,
+                             bf16 *__restrict__ dhb) {
   BW_PDL();
   __shared__ float red[32];
   const size_t o = (size_t)blockIdx.x * d;
@@ -619,7 +676,9 @@ __global__ void k_bw_rms_bwd(int d, const float *__restrict__ h, const float *__
   const float rr = r[blockIdx.x], k3 = rr * rr * rr * S / d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     const float g = rr * gamma[c] * du[o + c] - h[o + c] * k3;
-    dh[o + c] = assign ? g : dh[o + c] + g;
+    const float nv = assign ? g : dh[o + c] + g;
+    dh[o + c] = nv;
+    if (dhb) dhb[o + c] = __float2bfloat16_rn(nv);
     gg[o + c] = du[o + c] * h[o + c] * rr;
   }
 }
@@ -647,17 +706,25 @@ __global__ void k_bw_colsum(int n, int d, const float *__restrict__ X, float *__
 // dz = dact zb SiLU'(z), dzb = dact SiLU(z).
 __global__ void k_bw_act_bwd(long total, int swiglu, const float *__restrict__ z,
                              const float *__restrict__ zb, const float *__restrict__ dact,
-                             float *__restrict__ dz, float *__restrict__ dzb) {
+                             float *__restrict__ dz, float *__restrict__ dzb,
+                             bf16 *__restrict__ dz_b, bf16 *__restrict__ dzb_b) {
   BW_PDL();
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
     const float x = z[idx], g = dact[idx];
     if (swiglu) {
       const float sg = sigmoidf_(x);
-      dz[idx] = g * zb[idx] * sg * (1.f + x * (1.f - sg));
-      dzb[idx] = g * x * sg;
+      const float a = g * zb[idx] * sg * (1.f + x * (1.f - sg)), b = g * x * sg;
+      dz[idx] = a;
+      dzb[idx] = b;
+      if (dz_b) {
+        dz_b[idx] = __float2bfloat16_rn(a);
+        dzb_b[idx] = __float2bfloat16_rn(b);
+      }
     } else {
-      dz[idx] = g * gelu_grad(x);
+      const float a = g * gelu_grad(x);
+      dz[idx] = a;
+      if (dz_b) dz_b[idx] = __float2bfloat16_rn(a);
     }
   }
 }
@@ -667,7 +734,8 @@ __global__ void k_bw_act_bwd(long total, int swiglu, const float *__restrict__ z
 __global__ void k_bw_gate_bwd(int n, int d, float alpha, const float *__restrict__ dx,
                               const float *__restrict__ cat, const float *__restrict__ g,
                               float *__restrict__ dgpre, float *__restrict__ ds_prev,
-                              float *__restrict__ egrad, int max_len, long t) {
+                              float *__restrict__ egrad, int max_len, long t,
+                              bf16 *__restrict__ dgb) {
   BW_PDL();
   const long total = (long)n * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
@@ -675,6 +743,7 @@ __global__ void k_bw_gate_bwd(int n, int d, float alpha, const float *__restrict
     const int i = (int)(idx / d), c = (int)(idx % d);
     const float gg = g[idx], x = dx[idx], sp = cat[(size_t)i * 2 * d + d + c];
     dgpre[idx] = alpha * x * sp * gg * (1.f - gg);
+    if (dgb) dgb[idx] = __float2bfloat16_rn(dgpre[idx]);
     ds_prev[idx] = alpha * x * gg;
     egrad[((size_t)i * max_len + t) * d + c] += x;
   }

@@ -14,6 +14,7 @@ constexpr int BW_GROUP = 8;
 struct BwLayout {
   size_t s_hist, kv_hist, step, dring, xq, xda, xlse, xD, dmem, e32, de, total;
   size_t wt, xb, grp, gg, n_dev;  // tensor-core operands; gain-gradient rows
+  size_t trl;                      // the list of the per-step transposes
   size_t dmb, eT, wtm, rows_pad;   // memory-projection operands (bf16 models)
   size_t step_floats, grp_layer_rows;
   int P;      // recorded positions t0 - (W-1) .. t1 - 1
@@ -95,12 +96,13 @@ size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
   // bf16 models: transposed weights, the row-major bf16 operand, the group
   // buffers of the weight-gradient products
   const bool tc = c.dtype == RLT_BF16;
-  const size_t NP = (N + 63) / 64 * 64, WMAX = std::max(std::max(3 * d, F), 2 * d);
+  const size_t NP = (N + 63) / 64 * 64;
   const size_t ffn_mats = c.ffn_kind == RLT_SWIGLU ? 3 : 2;
   B->n_pad = (int)NP;
   B->grp_layer_rows = bw_grp_layer_rows(c);
   B->wt = take(tc ? (L * (6 * d * d + ffn_mats * d * F) + 2 * d * d) * 2 : 0);
-  B->xb = take(tc ? NP * WMAX * 2 : 0);
+  B->xb = take(tc ? (L * B->grp_layer_rows + 3 * d) * NP * 2 : 0);  // row-major operands
+  B->trl = take((13 * L + 2) * sizeof(BwTr));
   B->grp = take(tc ? (L * B->grp_layer_rows + 3 * d) * BW_GROUP * NP * 2 : 0);
   // per group: rows of the gain gradients (ln1..ln3 per layer, lnf) and of
   // the gate bias (dgpre)
@@ -173,44 +175,74 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   const float2 *rope = M->at<float2>(L.rope);
   const size_t nd = (size_t)n * d;
   const int n_pad = B.n_pad;
-  bf16 *xb = reinterpret_cast<bf16 *>(base + B.xb);
   int *n_dev = reinterpret_cast<int *>(base + B.n_dev);
   RLT_TRY(cudaMemcpyAsync(n_dev, &n, 4, cudaMemcpyHostToDevice, st));  // pageable: staged
 
-  // ---- group buffers: per layer the transposed operands of its weight
-  // gradients; the gate's after the last layer
-  struct GrpL {
+  // ---- the bf16 operands of the tensor-core GEMMs, per layer: row-major
+  // as their producers write them (the decode GEMMs' A), and transposed into
+  // the group buffers at the end of each step (the weight gradients' A and B)
+  struct Ops {
     bf16 *u1, *a1, *u2, *a2, *u3, *act, *dqkv, *dhs, *dhx, *dqx, *dhf, *dz, *dzb;
   };
-  std::vector<GrpL> grp(LD, GrpL{});
-  bf16 *grp_cat = nullptr, *grp_dgpre = nullptr;
+  std::vector<Ops> rb(LD, Ops{}), grp(LD, Ops{});
+  bf16 *rb_cat = nullptr, *rb_dg = nullptr, *grp_cat = nullptr, *grp_dgpre = nullptr;
+  std::vector<BwTr> trl;
   if (TC) {
-    bf16 *p = reinterpret_cast<bf16 *>(base + B.grp);
-    const size_t blk = (size_t)BW_GROUP * n_pad;
-    auto take = [&](int rows) {
-      bf16 *o = p;
-      p += (size_t)rows * blk;
-      return o;
+    auto carve = [&](bf16 *p, size_t blk, std::vector<Ops> &v, bf16 **cat, bf16 **dg) {
+      auto take = [&](int rows) {
+        bf16 *o = p;
+        p += (size_t)rows * blk;
+        return o;
+      };
+      for (int l = 0; l < LD; l++) {
+        Ops &q = v[l];
+        q.u1 = take(d);
+        q.a1 = take(d);
+        q.u2 = take(d);
+        q.a2 = take(d);
+        q.u3 = take(d);
+        q.act = take(F);
+        q.dqkv = take(3 * d);
+        q.dhs = take(d);
+        q.dhx = take(d);
+        q.dqx = take(d);
+        q.dhf = take(d);
+        q.dz = take(F);
+        q.dzb = swiglu ? take(F) : nullptr;
+      }
+      *cat = take(2 * d);
+      *dg = take(d);
     };
+    bf16 *rbase = reinterpret_cast<bf16 *>(base + B.xb);
+    carve(rbase, (size_t)n_pad, rb, &rb_cat, &rb_dg);
+    carve(reinterpret_cast<bf16 *>(base + B.grp), (size_t)BW_GROUP * n_pad, grp, &grp_cat,
+          &grp_dgpre);
+    // padding rows of the row-major operands stay zero
+    RLT_TRY(cudaMemsetAsync(rbase, 0, (LD * B.grp_layer_rows + 3 * d) * (size_t)n_pad * 2, st));
     for (int l = 0; l < LD; l++) {
-      GrpL &q = grp[l];
-      q.u1 = take(d);
-      q.a1 = take(d);
-      q.u2 = take(d);
-      q.a2 = take(d);
-      q.u3 = take(d);
-      q.act = take(F);
-      q.dqkv = take(3 * d);
-      q.dhs = take(d);
-      q.dhx = take(d);
-      q.dqx = take(d);
-      q.dhf = take(d);
-      q.dz = take(F);
-      q.dzb = swiglu ? take(F) : nullptr;
+      const Ops &a = rb[l], &b = grp[l];
+      trl.push_back({a.u1, b.u1, d});
+      trl.push_back({a.a1, b.a1, d});
+      trl.push_back({a.u2, b.u2, d});
+      trl.push_back({a.a2, b.a2, d});
+      trl.push_back({a.u3, b.u3, d});
+      trl.push_back({a.act, b.act, F});
+      trl.push_back({a.dqkv, b.dqkv, 3 * d});
+      trl.push_back({a.dhs, b.dhs, d});
+      trl.push_back({a.dhx, b.dhx, d});
+      trl.push_back({a.dqx, b.dqx, d});
+      trl.push_back({a.dhf, b.dhf, d});
+      trl.push_back({a.dz, b.dz, F});
+      if (swiglu) trl.push_back({a.dzb, b.dzb, F});
     }
-    grp_cat = take(2 * d);
-    grp_dgpre = take(d);
+    if (c.alpha != 0.0f) {
+      trl.push_back({rb_cat, grp_cat, 2 * d});
+      trl.push_back({rb_dg, grp_dgpre, d});
+    }
+    RLT_TRY(cudaMemcpyAsync(base + B.trl, trl.data(), trl.size() * sizeof(BwTr),
+                            cudaMemcpyHostToDevice, st));  // pageable: staged
   }
+  const BwTr *trl_dev = reinterpret_cast<const BwTr *>(base + B.trl);
   // gain-gradient rows of a group: ln1, ln2, ln3 of layer l at 3l .. 3l+2,
   // lnf at 3L, the gate bias at 3L + 1; row block `slot` within each
   auto ggbuf = [&](int which, int slot_) {
@@ -247,45 +279,41 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
 
   // The group being filled: `cnt` steps, this step's column block `slot`.
   int cnt = 0, slot = 0;
-  auto pack = [&](const float *X, long ld, int K, bf16 *row_major, bf16 *gbuf) {
-    RLT_TRY(launch_k(k_bw_pack, dim3((K + 31) / 32, n_pad / 32), dim3(32, 8), 0, st, 
-        n, n_pad, K, X, ld, row_major, gbuf, (long)cnt * n_pad, (long)slot * n_pad));
-    return cudaGetLastError();
-  };
-  // out [n][N] = X [n][K] Wm^T (+ base_); for bf16 X^T also goes to its
-  // group buffer (the operand of Wm's weight gradient)
-  auto fwd = [&](const float *X, int K, const T *Wm, int N, float *out, const float *base_,
-                 bf16 *gbuf) -> cudaError_t {
+  // out [n][N] = X [n][K] Wm^T (+ base_): bf16 models read the producer's
+  // bf16 copy Xb, fp32 models X
+  auto fwd = [&](const float *X, const bf16 *Xb, int K, const T *Wm, int N, float *out,
+                 const float *base_) -> cudaError_t {
     if constexpr (TC) {
-      RLT_TRY(pack(X, K, K, xb, gbuf));
+      (void)X;
       if (base_)
-        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, xb, Wm,
+        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, Xb, Wm,
                               EpiAddF32Dec{{}, base_, out, N}, st);
-      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, xb, Wm, EpiF32Dec{{}, out, N}, st);
+      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, Xb, Wm, EpiF32Dec{{}, out, N}, st);
     } else {
-      (void)gbuf;
+      (void)Xb;
       if (base_)
         RLT_TRY(cudaMemcpyAsync(out, base_, (size_t)n * N * 4, cudaMemcpyDeviceToDevice, st));
       return bw_gemm<true, true>(n, N, K, X, K, Wm, K, out, N, base_ != nullptr, st);
     }
   };
   // out [n][K] (=|+=) dY [n][N] Wm (Wm [N][K], WTm its transpose), and the
-  // weight gradient dW [N][K] += dY^T X: staged in the group buffer for bf16
-  // (reduced at the group's end), at once for fp32 (X [n][K], pitch ldx).
-  auto bwd = [&](const float *dY, int N, const T *Wm, const bf16 *WTm, int K, float *out,
-                 bool acc, bf16 *gbuf, const float *X, long ldx, float *dW) -> cudaError_t {
+  // weight gradient dW [N][K] += dY^T X: for bf16 the operands' transposes
+  // are reduced at the group's end, for fp32 at once (X [n][K], pitch ldx).
+  auto bwd = [&](const float *dY, const bf16 *dYb, int N, const T *Wm, const bf16 *WTm, int K,
+                 float *out, bool acc, const float *X, long ldx, float *dW) -> cudaError_t {
     if constexpr (TC) {
+      (void)dY;
       (void)X;
       (void)ldx;
       (void)dW;
-      RLT_TRY(pack(dY, N, N, xb, gbuf));
       if (acc)
-        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, xb, WTm, EpiAccF32Dec{{}, out, K},
-                              st);
-      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, xb, WTm, EpiF32Dec{{}, out, K}, st);
+        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, dYb, WTm,
+                              EpiAccF32Dec{{}, out, K}, st);
+      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, dYb, WTm, EpiF32Dec{{}, out, K},
+                            st);
     } else {
       (void)WTm;
-      (void)gbuf;
+      (void)dYb;
       RLT_TRY((bw_gemm<false, false>(N, K, n, dY, N, X, ldx, dW, K, true, st)));
       return bw_gemm<true, false>(n, K, N, dY, N, Wm, K, out, K, acc, st);
     }
@@ -310,7 +338,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     if (c.alpha != 0.0f) RLT_TRY(colsum(3 * LD + 1, gr->gate_b));
     if constexpr (TC) {
       for (int l = 0; l < LD; l++) {
-        const GrpL &q = grp[l];
+        const Ops &q = grp[l];
         RLT_TRY(grp_gemm(q.dqkv, 3 * d, q.u1, d, gr->dec_wqkv[l]));
         RLT_TRY(grp_gemm(q.dhs, d, q.a1, d, gr->dec_wo[l]));
         RLT_TRY(grp_gemm(q.dqx, d, q.u2, d, gr->dec_wqx[l]));
@@ -353,6 +381,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   auto rbuf = [&](int l, int which) { return S.r + ((size_t)3 * l + which) * n; };
   // groups in processing order (t descending), the partial one first, so a
   // group's column pitch is known when it starts
+  auto nb = [&](bf16 *p) { return TC ? p : nullptr; };  // bf16 outputs only for bf16 models
   for (int k = NS - 1; k >= 0; k--) {
     if (slot == cnt) {
       const int done = NS - 1 - k;
@@ -362,111 +391,126 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     const long t = t0 + k;
     const float *s_prev = s_hist + (size_t)k * nd;
     // recompute the forward of step t
-    RLT_TRY(launch_k(k_bw_gate_cat<T>, bw_blocks(2 * (long)nd), 256, 0, st, n, d, ready, e, c.max_len, t, s_prev,
-                                                              S.cat));
+    RLT_TRY(launch_k(k_bw_gate_cat<T>, bw_blocks(2 * (long)nd), 256, 0, st, n, d, ready, e,
+                     c.max_len, t, s_prev, S.cat, nb(rb_cat)));
     if (c.alpha != 0.0f)
-      RLT_TRY(fwd(S.cat, 2 * d, (const T *)M->w.gate_w, d, S.gpre, nullptr, grp_cat));
+      RLT_TRY(fwd(S.cat, rb_cat, 2 * d, (const T *)M->w.gate_w, d, S.gpre, nullptr));
     else
       RLT_TRY(cudaMemsetAsync(S.gpre, 0, nd * 4, st));
-    RLT_TRY(launch_k(k_bw_gate_fwd, bw_blocks(nd), 256, 0, st, n, d, S.gpre, (const float *)M->w.gate_b, S.cat,
-                                                 c.alpha, S.gs, hbuf(0, 0)));
+    RLT_TRY(launch_k(k_bw_gate_fwd, bw_blocks(nd), 256, 0, st, n, d, S.gpre,
+                     (const float *)M->w.gate_b, S.cat, c.alpha, S.gs, hbuf(0, 0)));
     for (int l = 0; l < LD; l++) {
       const int g = G == 1 ? 0 : l;
       float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2), *hn = hbuf(l + 1, 0);
-      float *u1 = ubuf(l, 0), *u2 = ubuf(l, 1), *u3 = ubuf(l, 2);
+      // fp32 copies of the GEMM inputs only for fp32 models
+      float *u1 = TC ? nullptr : ubuf(l, 0), *u2 = TC ? nullptr : ubuf(l, 1),
+            *u3 = TC ? nullptr : ubuf(l, 2);
       float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
       float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
-            *act = S.act + (size_t)l * n * F;
-      const GrpL &q = grp[l];
-      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h1, (const float *)M->w.dec_ln1[l], u1,
-                                      rbuf(l, 0)));
-      RLT_TRY(fwd(u1, d, W_<T>::qkv(M, l), 3 * d, S.qkv, nullptr, q.u1));
-      RLT_TRY(launch_k(k_bw_rope_q, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, t, rope, S.qkv, q1));
+            *act = TC ? nullptr : S.act + (size_t)l * n * F;
+      const Ops &o = rb[l];
+      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h1,
+                       (const float *)M->w.dec_ln1[l], u1, rbuf(l, 0), nb(o.u1)));
+      RLT_TRY(fwd(u1, o.u1, d, W_<T>::qkv(M, l), 3 * d, S.qkv, nullptr));
+      RLT_TRY(launch_k(k_bw_rope_q, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, t, rope,
+                       S.qkv, q1));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
       const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
-      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
-          n, H, swa, p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H));
-      RLT_TRY(fwd(a1, d, W_<T>::o(M, l), d, h2, h1, q.a1));
-      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h2, (const float *)M->w.dec_ln2[l], u2,
-                                      rbuf(l, 1)));
-      RLT_TRY(fwd(u2, d, (const T *)M->w.dec_wqx[l], d, qx, nullptr, q.u2));
+      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
+                       p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H, nb(o.a1)));
+      RLT_TRY(fwd(a1, o.a1, d, W_<T>::o(M, l), d, h2, h1));
+      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h2,
+                       (const float *)M->w.dec_ln2[l], u2, rbuf(l, 1), nb(o.u2)));
+      RLT_TRY(fwd(u2, o.u2, d, (const T *)M->w.dec_wqx[l], d, qx, nullptr));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
-      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
-          n, H, xk, 0, (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H));
-      RLT_TRY(fwd(a2, d, (const T *)M->w.dec_wox[l], d, h3, h2, q.a2));
-      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h3, (const float *)M->w.dec_ln3[l], u3,
-                                      rbuf(l, 2)));
-      RLT_TRY(fwd(u3, d, W_<T>::w1(M, l), F, z, nullptr, q.u3));
-      if (swiglu) RLT_TRY(fwd(u3, d, W_<T>::wb(M, l), F, zb, nullptr, nullptr));
-      RLT_TRY(launch_k(k_bw_act_fwd, bw_blocks((long)n * F), 256, 0, st, (long)n * F, swiglu, z, zb, act));
-      RLT_TRY(fwd(act, F, W_<T>::w2(M, l), d, hn, h3, q.act));
+      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, xk, 0,
+                       (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, nb(o.a2)));
+      RLT_TRY(fwd(a2, o.a2, d, (const T *)M->w.dec_wox[l], d, h3, h2));
+      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h3,
+                       (const float *)M->w.dec_ln3[l], u3, rbuf(l, 2), nb(o.u3)));
+      RLT_TRY(fwd(u3, o.u3, d, W_<T>::w1(M, l), F, z, nullptr));
+      if (swiglu) RLT_TRY(fwd(u3, o.u3, d, W_<T>::wb(M, l), F, zb, nullptr));
+      RLT_TRY(launch_k(k_bw_act_fwd, bw_blocks((long)n * F), 256, 0, st, (long)n * F, swiglu, z,
+                       zb, act, nb(o.act)));
+      RLT_TRY(fwd(act, o.act, F, W_<T>::w2(M, l), d, hn, h3));
     }
     float *rf = S.r + (size_t)3 * LD * n;
-    RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, hbuf(LD, 0), (const float *)M->w.dec_lnf,
-                                    S.ulast, rf));
-    RLT_TRY(cudaGetLastError());
+    RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, hbuf(LD, 0),
+                     (const float *)M->w.dec_lnf, S.ulast, rf, (bf16 *)nullptr));
 
     // differentiate step t: s_t = RMSNorm_f(h_L)
-    RLT_TRY(launch_k(k_bw_ds_total, bw_blocks(nd), 256, 0, st, n, d, NS, k, sgrad, S.dcarry, S.ds));
-    RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, hbuf(LD, 0), rf, (const float *)M->w.dec_lnf, S.ds, S.dh,
-                                    1, ggbuf(3 * LD, slot)));
+    RLT_TRY(launch_k(k_bw_ds_total, bw_blocks(nd), 256, 0, st, n, d, NS, k, sgrad, S.dcarry,
+                     S.ds));
+    RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, hbuf(LD, 0), rf,
+                     (const float *)M->w.dec_lnf, S.ds, S.dh, 1, ggbuf(3 * LD, slot),
+                     nb(rb[LD - 1].dhf)));
     for (int l = LD - 1; l >= 0; l--) {
       float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2);
       float *u1 = ubuf(l, 0), *u2 = ubuf(l, 1), *u3 = ubuf(l, 2);
       float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
       float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
             *act = S.act + (size_t)l * n * F;
-      const GrpL &q = grp[l];
+      const Ops &o = rb[l];
       // FFN: h_out = h3 + W2 act(W1 u3)
-      RLT_TRY(bwd(S.dh, d, W_<T>::w2(M, l), wt[l].w2, F, S.dtmp, false, q.dhf, act, F,
+      RLT_TRY(bwd(S.dh, o.dhf, d, W_<T>::w2(M, l), wt[l].w2, F, S.dtmp, false, act, F,
                   gr->dec_w2[l]));
-      RLT_TRY(launch_k(k_bw_act_bwd, bw_blocks((long)n * F), 256, 0, st, (long)n * F, swiglu, z, zb, S.dtmp,
-                                                           S.dz, S.dzb));
-      RLT_TRY(bwd(S.dz, F, W_<T>::w1(M, l), wt[l].w1, d, S.du, false, q.dz, u3, d,
+      RLT_TRY(launch_k(k_bw_act_bwd, bw_blocks((long)n * F), 256, 0, st, (long)n * F, swiglu, z,
+                       zb, S.dtmp, S.dz, S.dzb, nb(o.dz), nb(o.dzb)));
+      RLT_TRY(bwd(S.dz, o.dz, F, W_<T>::w1(M, l), wt[l].w1, d, S.du, false, u3, d,
                   gr->dec_w1[l]));
       if (swiglu)
-        RLT_TRY(bwd(S.dzb, F, W_<T>::wb(M, l), wt[l].wb, d, S.du, true, q.dzb, u3, d,
+        RLT_TRY(bwd(S.dzb, o.dzb, F, W_<T>::wb(M, l), wt[l].wb, d, S.du, true, u3, d,
                     gr->dec_wb[l]));
-      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h3, rbuf(l, 2), (const float *)M->w.dec_ln3[l], S.du,
-                                      S.dh, 0, ggbuf(3 * l + 2, slot)));
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h3, rbuf(l, 2),
+                       (const float *)M->w.dec_ln3[l], S.du, S.dh, 0, ggbuf(3 * l + 2, slot),
+                       nb(o.dhx)));
       // cross-attention: h3 = h2 + W_ox attn(W_qx u2, M<=t)
       const int g = G == 1 ? 0 : l;
-      RLT_TRY(bwd(S.dh, d, (const T *)M->w.dec_wox[l], wt[l].ox, d, S.dtmp, false, q.dhx, a2, d,
+      RLT_TRY(bwd(S.dh, o.dhx, d, (const T *)M->w.dec_wox[l], wt[l].ox, d, S.dtmp, false, a2, d,
                   gr->dec_wox[l]));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
       const size_t xo = ((size_t)l * NS + k) * nd, xs = ((size_t)l * NS + k) * n * H;
-      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
-          n, H, xk, 0, (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, S.dtmp, S.dq, nullptr,
-          W, 0, xq + xo, xda + xo, xlse + xs, xD + xs));
-      RLT_TRY(bwd(S.dq, d, (const T *)M->w.dec_wqx[l], wt[l].qx, d, S.du, false, q.dqx, u2, d,
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, xk, 0,
+                       (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, S.dtmp, S.dq,
+                       (float *)nullptr, W, 0L, xq + xo, xda + xo, xlse + xs, xD + xs,
+                       nb(o.dqx)));
+      RLT_TRY(bwd(S.dq, o.dqx, d, (const T *)M->w.dec_wqx[l], wt[l].qx, d, S.du, false, u2, d,
                   gr->dec_wqx[l]));
-      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h2, rbuf(l, 1), (const float *)M->w.dec_ln2[l], S.du,
-                                      S.dh, 0, ggbuf(3 * l + 1, slot)));
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h2, rbuf(l, 1),
+                       (const float *)M->w.dec_ln2[l], S.du, S.dh, 0, ggbuf(3 * l + 1, slot),
+                       nb(o.dhs)));
       // SWA: h2 = h1 + W_o attn(q_t over the window); k_t, v_t enter the cache
-      RLT_TRY(bwd(S.dh, d, W_<T>::o(M, l), wt[l].o, d, S.dtmp, false, q.dhs, a1, d,
+      RLT_TRY(bwd(S.dh, o.dhs, d, W_<T>::o(M, l), wt[l].o, d, S.dtmp, false, a1, d,
                   gr->dec_wo[l]));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
       const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
-      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, 
-          n, H, swa, p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H, S.dtmp, S.dq, dring,
-          W, t0 - Wm1, nullptr, nullptr, nullptr, nullptr));
-      RLT_TRY(launch_k(k_bw_qkv_grad, bw_blocks((long)n * d / 2), 256, 0, st, 
-          n, H, DH, W, t, rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv));
-      RLT_TRY(bwd(S.dqkv, 3 * d, W_<T>::qkv(M, l), wt[l].qkv, d, S.du, false, q.dqkv, u1, d,
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
+                       p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H, S.dtmp, S.dq,
+                       dring, W, (long)(t0 - Wm1), (float *)nullptr, (float *)nullptr,
+                       (float *)nullptr, (float *)nullptr, (bf16 *)nullptr));
+      RLT_TRY(launch_k(k_bw_qkv_grad, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, W, t,
+                       rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv, nb(o.dqkv)));
+      RLT_TRY(bwd(S.dqkv, o.dqkv, 3 * d, W_<T>::qkv(M, l), wt[l].qkv, d, S.du, false, u1, d,
                   gr->dec_wqkv[l]));
-      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h1, rbuf(l, 0), (const float *)M->w.dec_ln1[l], S.du,
-                                      S.dh, 0, ggbuf(3 * l, slot)));
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h1, rbuf(l, 0),
+                       (const float *)M->w.dec_ln1[l], S.du, S.dh, 0, ggbuf(3 * l, slot),
+                       l > 0 ? nb(rb[l - 1].dhf) : (bf16 *)nullptr));
     }
     // gated merge: x = e_t + alpha sigmoid(W_g [e_t; s_{t-1}] + b_g) s_{t-1}
     float *dgpre = ggbuf(3 * LD + 1, slot);
-    RLT_TRY(launch_k(k_bw_gate_bwd, bw_blocks(nd), 256, 0, st, n, d, c.alpha, S.dh, S.cat, S.gs, dgpre,
-                                                 S.dcarry, egrad, c.max_len, t));
+    RLT_TRY(launch_k(k_bw_gate_bwd, bw_blocks(nd), 256, 0, st, n, d, c.alpha, S.dh, S.cat, S.gs,
+                     dgpre, S.dcarry, egrad, c.max_len, t,
+                     c.alpha != 0.0f ? nb(rb_dg) : (bf16 *)nullptr));
     if (c.alpha != 0.0f) {
-      RLT_TRY(bwd(dgpre, d, (const T *)M->w.gate_w, wt_gate, 2 * d, S.dtmp, false, grp_dgpre,
-                  S.cat, 2 * d, gr->gate_w));
-      RLT_TRY(launch_k(k_bw_gate_bwd2, bw_blocks(nd), 256, 0, st, n, d, S.dtmp, S.dcarry, egrad, c.max_len, t));
+      RLT_TRY(bwd(dgpre, rb_dg, d, (const T *)M->w.gate_w, wt_gate, 2 * d, S.dtmp, false, S.cat,
+                  2 * d, gr->gate_w));
+      RLT_TRY(launch_k(k_bw_gate_bwd2, bw_blocks(nd), 256, 0, st, n, d, S.dtmp, S.dcarry, egrad,
+                       c.max_len, t));
     }
-    RLT_TRY(cudaGetLastError());
+    // this step's operands, transposed into the group's column block
+    if (TC)
+      RLT_TRY(launch_k(k_bw_grp_transpose, dim3(64, (unsigned)trl.size()), dim3(32, 8), 0, st,
+                       trl_dev, n, n_pad, (long)cnt * n_pad, (long)slot * n_pad));
     if (++slot == cnt) RLT_TRY(flush());
   }
   // the state entering the chunk
