@@ -416,6 +416,26 @@ __device__ __forceinline__ void bw_ld8(const float *p, float *f) {
   f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
 }
 
+// Eight head entries of a key or value row kept as loaded (bf16 pairs stay
+// packed, halving the registers a row in flight takes); at(e) widens one.
+template <typename T> struct BwRaw8;
+template <> struct BwRaw8<bf16> {
+  uint32_t w[4];
+  __device__ __forceinline__ void load(const bf16 *p) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+  }
+  __device__ __forceinline__ float at(int e) const {
+    const uint32_t x = w[e >> 1];
+    return __uint_as_float((e & 1) ? (x & 0xffff0000u) : (x << 16));
+  }
+};
+template <> struct BwRaw8<float> {
+  float f[8];
+  __device__ __forceinline__ void load(const float *p) { bw_ld8(p, f); }
+  __device__ __forceinline__ float at(int e) const { return f[e]; }
+};
+
 // Sum over the DH / 8 lanes that hold one key's head slices.
 template <int LPK> __device__ __forceinline__ float bw_group_sum(float v) {
 #pragma unroll
@@ -446,7 +466,7 @@ constexpr int BW_ATT_WARPS = 4;
 // groups by shuffles, then the warps in order), so the result does not
 // depend on timing. Writes a and the log-sum-exp of the scaled scores.
 template <typename T, int DH>
-__global__ void __launch_bounds__(32 * BW_ATT_WARPS)
+__global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
     k_bw_attn_fwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
                   const float *__restrict__ q, float *__restrict__ a, float *__restrict__ lse,
                   bf16 *__restrict__ ab) {
@@ -461,24 +481,37 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
 #pragma unroll
   for (int e = 0; e < 8; e++) acc[e] = 0.f;
   float m = -INFINITY, l = 0.f;
-  for (int base = j_lo + warp * KPW; base <= j_hi; base += BW_ATT_WARPS * KPW) {
-    const int j = base + grp;
-    const bool ok = j <= j_hi;
-    float kv[8], vv[8];
-    float dot = 0.f;
-    if (ok) {
-      bw_ld8(K + (size_t)j * DH + sl * 8, kv);
-      bw_ld8(V + (size_t)j * DH + sl * 8, vv);
+  // a lane group takes keys j, j + S, j + 2S, ... (S = keys per CTA pass),
+  // two per iteration so that both loads are in flight together
+  constexpr int S = BW_ATT_WARPS * KPW;
+  for (int base = j_lo + warp * KPW; base <= j_hi; base += 2 * S) {
+    BwRaw8<T> kv[2], vv[2];
+    float dot[2] = {0.f, 0.f};
+    bool ok[2];
 #pragma unroll
-      for (int e = 0; e < 8; e++) dot += qv[e] * kv[e];
+    for (int u = 0; u < 2; u++) {
+      const int j = base + grp + u * S;
+      ok[u] = j <= j_hi;
+      if (ok[u]) {
+        kv[u].load(K + (size_t)j * DH + sl * 8);
+        vv[u].load(V + (size_t)j * DH + sl * 8);
+      }
     }
-    dot = bw_group_sum<LPK>(dot);
-    if (ok) {
-      const float s = dot * scale, mn = fmaxf(m, s);
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      if (ok[u])
+#pragma unroll
+        for (int e = 0; e < 8; e++) dot[u] += qv[e] * kv[u].at(e);
+      dot[u] = bw_group_sum<LPK>(dot[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      if (!ok[u]) continue;
+      const float s = dot[u] * scale, mn = fmaxf(m, s);
       const float corr = m == -INFINITY ? 0.f : expf(m - mn), p = expf(s - mn);
       l = l * corr + p;
 #pragma unroll
-      for (int e = 0; e < 8; e++) acc[e] = acc[e] * corr + p * vv[e];
+      for (int e = 0; e < 8; e++) acc[e] = acc[e] * corr + p * vv[u].at(e);
       m = mn;
     }
   }
@@ -522,7 +555,7 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
 // (xq != null): q, da, lse and D = da.a are saved for the memory-gradient
 // pass.
 template <typename T, int DH>
-__global__ void __launch_bounds__(32 * BW_ATT_WARPS)
+__global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
     k_bw_attn_bwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
                   const float *__restrict__ q, const float *__restrict__ a,
                   const float *__restrict__ lse, const float *__restrict__ da,
@@ -551,27 +584,39 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS)
   float *dk_ring = dring ? dring + ((((size_t)keys.l_or_g * n + i) * H + h) * 2 + 0) * W * DH
                          : nullptr;
   float *dv_ring = dring ? dk_ring + (size_t)W * DH : nullptr;
-  for (int base = j_lo + warp * KPW; base <= j_hi; base += BW_ATT_WARPS * KPW) {
-    const int j = base + grp;
-    const bool ok = j <= j_hi;
-    float kv[8], vv[8];
-    float dot = 0.f, dp = 0.f;
-    if (ok) {
-      bw_ld8(K + (size_t)j * DH + sl * 8, kv);
-      bw_ld8(V + (size_t)j * DH + sl * 8, vv);
+  constexpr int S = BW_ATT_WARPS * KPW;  // keys per CTA pass; two passes per iteration
+  for (int base = j_lo + warp * KPW; base <= j_hi; base += 2 * S) {
+    BwRaw8<T> kv2[2], vv2[2];
+    float dot2[2] = {0.f, 0.f}, dp2[2] = {0.f, 0.f};
+    bool ok2[2];
 #pragma unroll
-      for (int e = 0; e < 8; e++) {
-        dot += qv[e] * kv[e];
-        dp += dav[e] * vv[e];
+    for (int u = 0; u < 2; u++) {
+      const int j = base + grp + u * S;
+      ok2[u] = j <= j_hi;
+      if (ok2[u]) {
+        kv2[u].load(K + (size_t)j * DH + sl * 8);
+        vv2[u].load(V + (size_t)j * DH + sl * 8);
       }
     }
-    dot = bw_group_sum<LPK>(dot);
-    dp = bw_group_sum<LPK>(dp);
-    if (ok) {
-      const float p = expf(dot * scale - L);
-      const float ds = p * (dp - D);
 #pragma unroll
-      for (int e = 0; e < 8; e++) dqv[e] += scale * ds * kv[e];
+    for (int u = 0; u < 2; u++) {
+      if (ok2[u])
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+          dot2[u] += qv[e] * kv2[u].at(e);
+          dp2[u] += dav[e] * vv2[u].at(e);
+        }
+      dot2[u] = bw_group_sum<LPK>(dot2[u]);
+      dp2[u] = bw_group_sum<LPK>(dp2[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      if (!ok2[u]) continue;
+      const int j = base + grp + u * S;
+      const float p = expf(dot2[u] * scale - L);
+      const float ds = p * (dp2[u] - D);
+#pragma unroll
+      for (int e = 0; e < 8; e++) dqv[e] += scale * ds * kv2[u].at(e);
       if (dk_ring) {
         const size_t slot = (size_t)((pos0 + j) % W) * DH + sl * 8;
         float4 *pk = reinterpret_cast<float4 *>(dk_ring + slot);
