@@ -7,8 +7,9 @@
 // Steps whose weight gradients one GEMM reduces (bf16 models): each step's
 // bf16 operands of the weight-gradient products (activations and output
 // gradients, transposed) land in column block `slot` of a group buffer, and
-// one tile GEMM per weight and group reduces over group x batch rows.
-constexpr int BW_GROUP = 8;
+// one tile GEMM per weight and group reduces over group x batch rows (32
+// steps: 8 left the GEMMs' fixed cost a visible share of the step).
+constexpr int BW_GROUP = 32;
 
 // Workspace of one rlt_backward call: n rows, NS steps. Offsets in bytes.
 struct BwLayout {
