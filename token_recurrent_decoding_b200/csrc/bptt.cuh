@@ -150,30 +150,6 @@ struct EpiAccF32 {
   }
 };
 
-// bf16 operands of the tensor-core GEMMs from an fp32 [n][ld] matrix (its
-// first K columns): row-major Xb [n_pad][K] and/or the transposed block
-// XT[c][col0 + r] (row pitch `pitch`), rows n .. n_pad-1 zero. 32 x 32 tiles
-// through shared memory, so both layouts are written with contiguous runs.
-__global__ void k_bw_pack(int n, int n_pad, int K, const float *__restrict__ X, long ld,
-                          bf16 *__restrict__ Xb, bf16 *__restrict__ XT, long pitch, long col0) {
-  BW_PDL();
-  __shared__ float tile[32][33];
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
-  for (int y = ty; y < 32; y += 8) {
-    const int r = r0 + y, c = c0 + tx;
-    float v = (r < n && c < K) ? X[(size_t)r * ld + c] : 0.f;
-    tile[y][tx] = v;
-    if (Xb && r < n_pad && c < K) Xb[(size_t)r * K + c] = __float2bfloat16_rn(v);
-  }
-  if (!XT) return;
-  __syncthreads();
-  for (int y = ty; y < 32; y += 8) {
-    const int c = c0 + y, r = r0 + tx;
-    if (c < K && r < n_pad) XT[(size_t)c * pitch + col0 + r] = __float2bfloat16_rn(tile[tx][y]);
-  }
-}
-
 // WT [K][N] = W^T of a bf16 [N][K] weight (32 x 32 tiles).
 __global__ void k_bw_transpose(int N, int K, const bf16 *__restrict__ W, bf16 *__restrict__ WT) {
   __shared__ bf16 tile[32][34];
