@@ -24,6 +24,7 @@
 #include "kernels.cuh"
 #include "attn.cuh"
 #include "enc_attn.cuh"
+#include "enc_attn_tc.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_dec.cuh"
 #include "step_fused.cuh"
@@ -57,6 +58,7 @@ struct Layout {
   size_t nsq;  // per-row partial sums of squares of h over 32-column tiles (bf16 models)
   // encoder work buffers (ptok rows)
   size_t tok, tok_slot, tok_pos, tok_start, blk, eh, eu, eqkv, Qh, Kh, Vh, ea, efa, ef, etok;
+  size_t blk2;  // work list of 128-row query blocks (tensor-core encoder attention)
   size_t staging, staging_bytes;
   // persistent step kernel: dependency counters + abort word, tensor-map table
   size_t fs_cnt, fs_cnt_bytes, fs_maps;
@@ -144,6 +146,7 @@ size_t compute_layout(const rlt_config *c, Layout *L) {
   L->tok_pos = take(P * 4);
   L->tok_start = take(P * 4);
   L->blk = take((P / 64 + S + 1) * 16);
+  L->blk2 = take((P / 128 + S + 1) * 16);
   L->eh = take(P * d * 4);
   L->eu = take(P * d * es);
   L->eqkv = take(P * 3 * d * 4);
@@ -198,6 +201,7 @@ struct rlt_model {
   int num_sms = 148;  // SMs of the device (decode GEMM split counts)
   int swap_br = 0;    // decode GEMMs with swapped operands: batch rows per tile (0 = off)
   bool tc_persistent = true;  // encoder GEMMs of >= 1024 rows: persistent form
+  int enc_blk2 = 0;           // 128-row query blocks of the staged encoder chunk (L.blk2)
   std::vector<int> t_dec, t_enc;
   cudaStream_t last_stream = nullptr;
   template <typename X> X *at(size_t off) const { return reinterpret_cast<X *>(arena + off); }
@@ -1011,6 +1015,20 @@ cudaError_t enc_attention(rlt_model *M, int ntok, int nblk, const T *Qh, const T
                           T *ea, cudaStream_t st, int window = 0, const T *Qlo = nullptr) {
   const Layout &L = M->L;
   const int H = M->cfg.n_heads;
+  if constexpr (std::is_same<T, bf16>::value && DH == EA_DH) {
+    // plain causal attention of the encoder: tcgen05 with S and O in TMEM
+    if (window == 0 && !Qlo && M->enc_blk2 > 0) {
+      const CUtensorMap *mq = tmap_bf16(M, Qh, (uint64_t)H * ntok, DH, EA_BQ);
+      const CUtensorMap *mk = tmap_bf16(M, Kh, (uint64_t)H * ntok, DH, EA_BK);
+      const CUtensorMap *mv = tmap_bf16(M, Vh, (uint64_t)H * ntok, DH, EA_BK);
+      if (!mq || !mk || !mv) return cudaErrorInvalidValue;
+      RLT_TRY(ensure_smem_limit(k_enc_attn_tc, EaSmem::BYTES));
+      const float scale_log2 = 1.4426950408889634f / sqrtf((float)DH);
+      k_enc_attn_tc<<<dim3(M->enc_blk2, H), EA_THREADS, EaSmem::BYTES, st>>>(
+          *mq, *mk, *mv, ntok, M->at<int>(L.blk2), ea, H, scale_log2, M->at<int>(L.err));
+      return cudaGetLastError();
+    }
+  }
   if constexpr (std::is_same<T, bf16>::value && DH >= 32) {
     constexpr int smem = FaSmem<DH>::BYTES;
     RLT_TRY(ensure_smem_limit(k_enc_flash<DH, false>, smem));
@@ -2079,7 +2097,7 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
   cudaStream_t st = (cudaStream_t)stream;
   M->last_stream = st;
   const Layout &L = M->L;
-  std::vector<int> slot, pos, start, blk;
+  std::vector<int> slot, pos, start, blk, blk2;
   int i = 0;
   while (i < n) {
     // pack whole sequences into one chunk of at most ptok tokens
@@ -2090,6 +2108,7 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
     pos.assign(ntok, 0);
     start.assign(ntok, 0);
     blk.clear();
+    blk2.clear();
     long m = 0;
     for (int k = i; k < j; k++) {
       if (lengths[k] == 0) continue;
@@ -2098,6 +2117,12 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
         blk.push_back(lengths[k]);
         blk.push_back(qb);
         blk.push_back(0);
+      }
+      for (int qb = 0; qb * 128 < lengths[k]; qb++) {
+        blk2.push_back((int)m);
+        blk2.push_back(lengths[k]);
+        blk2.push_back(qb);
+        blk2.push_back(0);
       }
       cudaError_t e = cudaMemcpyAsync(M->at<int>(L.tok) + m, tokens + offsets[k],
                                       sizeof(int32_t) * lengths[k], cudaMemcpyDefault, st);
@@ -2119,7 +2144,12 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
       if (e == cudaSuccess)
         e = cudaMemcpyAsync(M->at<int>(L.blk), blk.data(), 4 * blk.size(), cudaMemcpyHostToDevice,
                             st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(M->at<int>(L.blk2), blk2.data(), 4 * blk2.size(),
+                            cudaMemcpyHostToDevice, st);
+      M->enc_blk2 = (int)(blk2.size() / 4);
       if (e == cudaSuccess) e = M->prefill(M, (int)ntok, (int)(blk.size() / 4), st);
+      M->enc_blk2 = 0;
       if (e != cudaSuccess) return RLT_ERR_CUDA;
       // the host vectors are reused next chunk: pageable copies are staged
       // at enqueue time, so reuse is safe
