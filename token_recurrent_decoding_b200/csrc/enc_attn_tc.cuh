@@ -64,6 +64,14 @@ __device__ __forceinline__ bool ea_wait(uint64_t *bar, unsigned parity) {
   }
 }
 
+// 2^x with the special-function unit's instruction (ex2.approx; 2^-inf = 0):
+// its error is far below the bf16 rounding the probabilities get next.
+__device__ __forceinline__ float ea_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 32 consecutive columns of this warp's TMEM lanes (one row per thread):
 // two loads in flight, one wait.
 __device__ __forceinline__ void ea_tmem_ld32(uint32_t taddr, float v[32]) {
@@ -244,11 +252,20 @@ __global__ void __launch_bounds__(EA_THREADS, 3)
       ea_tmem_ld32(tS + lb, sc);
       ea_tmem_ld32(tS + lb + 32, sc + 32);
       float mx = -INFINITY;
+      if (kbase + EA_BK - 1 <= q0 && kbase + EA_BK <= len) {
+        // below the diagonal for every row of the CTA: nothing masked
 #pragma unroll
-      for (int e = 0; e < EA_BK; e++) {
-        const int key = kbase + e;
-        sc[e] = (key <= qpos && key < len) ? sc[e] * scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sc[e]);
+        for (int e = 0; e < EA_BK; e++) {
+          sc[e] *= scale_log2;
+          mx = fmaxf(mx, sc[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EA_BK; e++) {
+          const int key = kbase + e;
+          sc[e] = (key <= qpos && key < len) ? sc[e] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, sc[e]);
+        }
       }
       const float m_new = fmaxf(m, mx);
       const float base = m_new == -INFINITY ? 0.f : m_new;
@@ -279,7 +296,7 @@ __global__ void __launch_bounds__(EA_THREADS, 3)
       float sum = 0.f;
 #pragma unroll
       for (int e = 0; e < EA_BK; e++) {
-        sc[e] = exp2f(sc[e] - base);  // masked: exp2(-inf) = 0
+        sc[e] = ea_exp2(sc[e] - base);  // masked: 2^-inf = 0
         sum += sc[e];
       }
 #pragma unroll
