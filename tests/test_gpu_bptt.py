@@ -157,3 +157,35 @@ def test_backward_argument_checks():
         m.backward([0], Gd[:1].contiguous(), workspace=torch.empty(256, dtype=torch.uint8,
                                                                    device="cuda"))
     assert m.get_state(0)[2] == 0  # refused calls changed nothing
+
+
+def test_backward_full_size_m140_late_chunk():
+    """The ~140M model at its real shapes (d = 768, 12 + 12 layers, W = 128,
+    G = L_D, SwiGLU-free GELU FFN 3072) for two sequences: a chunk of
+    positions 1000 .. 1007 after 1000 recurrent steps (memory rows up to
+    1007, full windows), every parameter gradient, dL/de and the carried
+    state against the gradient oracle started from the GPU's own state."""
+    wl = configs.workloads()["m140_bf16"]
+    cfg = wl.model
+    T, t0, NS, B = 1024, 1000, 8, 2
+    m, w, tok = make_model(cfg, [T] * B)
+    ids = [0, 1]
+    m.run_sequence(ids, t0)
+    state = [m.get_state(i) for i in ids]
+    G, Gd = _sgrad(B, NS, cfg.d, seed=9)
+    grads, egrad, carry = m.backward(ids, Gd)
+    torch.cuda.synchronize()
+    assert m.poll_device_error() == 0
+    s0 = np.stack([to_np(x[0]) for x in state])
+    win0 = np.stack([to_np(x[1]) for x in state])
+    ref, per = _oracle(m, cfg, w, ids, NS, G, t0=t0, s0=s0, win0=win0)
+    tol = TRAJ_TOL[cfg.dtype]
+    worst = {k: _rel(to_np(grads[k]), v) for k, v in ref.items() if k != "sstar"}
+    print("m140 full size worst relative L2 error", max(worst.values()), max(worst, key=worst.get))
+    assert all(e <= tol for e in worst.values()), {k: e for k, e in worst.items() if e > tol}
+    eg = to_np(egrad)
+    c = to_np(carry)
+    for b in range(B):
+        assert _rel(eg[b, :t0 + NS], per[b]["e"]) <= tol
+        assert _rel(c[b, :cfg.d], per[b]["s0"]) <= tol
+        assert _rel(c[b, cfg.d:], per[b]["win0"].reshape(-1)) <= tol
