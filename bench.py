@@ -390,6 +390,12 @@ def time_backward(wl, r, dist, hbm, tc):
     cfg = wl.model
     T = int(r.lengths[0])
     m = r.m
+    need = m.backward_workspace_bytes(wl.batch, T)
+    free, _ = torch.cuda.mem_get_info()
+    if need + 3 * wl.batch * wl.max_len * cfg.d * 4 > 0.9 * free:
+        return {"skipped": "workspace %.1f GB for %d x %d positions exceeds free device memory "
+                           "%.1f GB (chunked backpropagation through rlt_backward's carried "
+                           "gradient covers such runs)" % (need / 1e9, wl.batch, T, free / 1e9)}
     g = torch.Generator(device="cuda").manual_seed(2)
     sgrad = torch.randn((wl.batch, T, cfg.d), generator=g, device="cuda")
     grads = {k: torch.zeros(v, device="cuda") for k, v in m.grad_shapes().items()}
