@@ -2118,7 +2118,9 @@ RLT_API int rlt_prefill_encoder(rlt_model *M, const int32_t *tokens, const int32
         blk.push_back(qb);
         blk.push_back(0);
       }
-      for (int qb = 0; qb * 128 < lengths[k]; qb++) {
+      // causal blocks carry 2 (qb + 1) key tiles: the heaviest go first, so
+      // the last wave of CTAs holds the short ones
+      for (int qb = (lengths[k] - 1) / 128; qb >= 0; qb--) {
         blk2.push_back((int)m);
         blk2.push_back(lengths[k]);
         blk2.push_back(qb);
