@@ -373,6 +373,8 @@ def run_ours(args, wl, rank, world, dist, peaks, peaks_src):
         }
     if args.backward and not r.ragged and cfg.dtype == configs.BF16:
         out["backward"] = time_backward(wl, r, dist, hbm, tc)
+        if rank == 0 and not args.no_cpu_baseline and "skipped" not in out["backward"]:
+            out["backward"]["cpu_baseline"] = cpu_backward_baseline(wl)
     if args.serve and wl.prompt_lengths and not r.ragged and cfg.dtype == configs.BF16:
         out["serve"] = time_serve(wl, r, dist)
     if rank == 0 and not args.no_cpu_baseline:
@@ -497,6 +499,30 @@ def cpu_baseline(wl, positions):
     return {"value": sum(lens) / dt, "unit": "seq-steps/s", "cores": used, "kind": "oracle",
             "sample": f"{nseq} sequences x first {lens[0]} positions (encoder + decoder, fp32 "
                       f"oracle, OpenMP over sequences), {dt:.1f} s"}
+
+
+def cpu_backward_baseline(wl, positions=8):
+    """The gradient oracle (float64 restatement differentiated by
+    torch.autograd) as it stands, on the host cores, over a bounded sample:
+    one sequence's first `positions` positions from s*, its encoder output
+    from the C oracle."""
+    import torch
+
+    import oracle
+    from oracle import bptt
+    cfg = wl.model
+    w = inputs.make_weights(cfg)
+    tok = inputs.make_tokens(cfg.vocab, wl.lengths)[0, :positions]
+    e, _ = oracle.Oracle(cfg, w).encode(tok)
+    G = np.random.default_rng(3).standard_normal((positions, cfg.d))
+    win0 = np.zeros((cfg.n_dec, 2, max(cfg.window - 1, 0), cfg.d))
+    t = time.perf_counter()
+    bptt.chunk_grads(cfg, w, e, w["sstar"], win0, 0, positions, G)
+    dt = time.perf_counter() - t
+    return {"value": positions / dt, "unit": "seq-steps/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"1 sequence x first {positions} positions (gradient oracle: float64 "
+                      f"torch autograd over the decoder), {dt:.1f} s"}
 
 
 def run_reference(args, wl, rank, world):
