@@ -150,6 +150,21 @@ struct EpiAccF32 {
   }
 };
 
+// Tile-GEMM epilogue (k_gemm_tc / k_gemm_tcp): out = base + C.
+struct EpiAddF32 {
+  const float *base;
+  float *out;
+  int ld;
+  __device__ void operator()(int m, int n, float a, float b) const {
+    const float2 x = *reinterpret_cast<const float2 *>(base + (size_t)m * ld + n);
+    *reinterpret_cast<float2 *>(out + (size_t)m * ld + n) = make_float2(x.x + a, x.y + b);
+  }
+  __device__ void vec16(int m, int n, const float *v) const {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) (*this)(m, n + i, v[i], v[i + 1]);
+  }
+};
+
 // WT [K][N] = W^T of a bf16 [N][K] weight (32 x 32 tiles).
 __global__ void k_bw_transpose(int N, int K, const bf16 *__restrict__ W, bf16 *__restrict__ WT) {
   __shared__ bf16 tile[32][34];
@@ -166,34 +181,38 @@ __global__ void k_bw_transpose(int N, int K, const bf16 *__restrict__ W, bf16 *_
   }
 }
 
-// The transposed bf16 operands of one group's weight gradients: for each
-// listed matrix (row-major bf16 [n][K] as its producer wrote it), rows 0..n-1
-// into columns col0 .. col0+n-1 of dst [K][pitch], columns up to col0 + n_pad
-// zero. blockIdx.y picks the matrix; 32 x 32 tiles through shared memory.
+// The transposed bf16 operands of one group's weight gradients: each listed
+// matrix holds the rows of `rb` steps as its producer wrote them (row-major
+// bf16 [rb n][K], row s n + i = step s, sequence i); step s lands in column
+// block (slot0 + rb - 1 - s) of dst [K][pitch] (steps run in descending
+// order through a group), rows n .. n_pad-1 of each block zero. blockIdx.y
+// picks the matrix; 32 x 32 tiles through shared memory.
 struct BwTr {
   const bf16 *src;
   bf16 *dst;
   int K;
 };
 
-__global__ void k_bw_grp_transpose(const BwTr *__restrict__ list, int n, int n_pad, long pitch,
-                                   long col0) {
+__global__ void k_bw_grp_transpose(const BwTr *__restrict__ list, int n, int n_pad, int rb,
+                                   long pitch, long slot0) {
   BW_PDL();
   __shared__ bf16 tile[32][34];
   const BwTr m = list[blockIdx.y];
-  const int tiles_c = (m.K + 31) / 32, tiles = tiles_c * (n_pad / 32);
+  const int tiles_c = (m.K + 31) / 32, tiles = tiles_c * (rb * n_pad / 32);
   const int tx = threadIdx.x, ty = threadIdx.y;
   for (int b = blockIdx.x; b < tiles; b += gridDim.x) {
-    const int c0 = (b % tiles_c) * 32, r0 = (b / tiles_c) * 32;
+    const int c0 = (b % tiles_c) * 32, v0 = (b / tiles_c) * 32;  // v: virtual row s n_pad + i
     __syncthreads();
     for (int y = ty; y < 32; y += 8) {
-      const int r = r0 + y, c = c0 + tx;
-      tile[y][tx] = (r < n && c < m.K) ? m.src[(size_t)r * m.K + c] : __float2bfloat16_rn(0.f);
+      const int v = v0 + y, c = c0 + tx, st = v / n_pad, i = v % n_pad;
+      tile[y][tx] = (i < n && c < m.K) ? m.src[((size_t)st * n + i) * m.K + c]
+                                       : __float2bfloat16_rn(0.f);
     }
     __syncthreads();
     for (int y = ty; y < 32; y += 8) {
-      const int c = c0 + y, r = r0 + tx;
-      if (c < m.K && r < n_pad) m.dst[(size_t)c * pitch + col0 + r] = tile[tx][y];
+      const int c = c0 + y, v = v0 + tx, st = v / n_pad, i = v % n_pad;
+      if (c < m.K)
+        m.dst[(size_t)c * pitch + (slot0 + rb - 1 - st) * n_pad + i] = tile[tx][y];
     }
   }
 }
@@ -280,18 +299,22 @@ __global__ void k_bw_hist_step(int n, const int *__restrict__ ready, const T *__
 }
 
 // ---------------------------------------------------- forward recompute
-// cat = [e_t ; s_{t-1}] per row.
+// cat = [e_t ; s_{t-1}] per row; rows of several steps, row = s n + i at
+// position tb + s (s_prev holds the rows in the same order).
 template <typename T>
-__global__ void k_bw_gate_cat(int n, int d, const int *__restrict__ ready, const T *__restrict__ e,
-                              int max_len, long t, const float *__restrict__ s_prev,
-                              float *__restrict__ cat, bf16 *__restrict__ catb) {
+__global__ void k_bw_gate_cat(int rows, int n, int d, const int *__restrict__ ready,
+                              const T *__restrict__ e, int max_len, long tb,
+                              const float *__restrict__ s_prev, float *__restrict__ cat,
+                              bf16 *__restrict__ catb) {
   BW_PDL();
-  const long total = (long)n * 2 * d;
+  const long total = (long)rows * 2 * d;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
-    const int i = (int)(idx / (2 * d)), c = (int)(idx % (2 * d));
+    const int row = (int)(idx / (2 * d)), c = (int)(idx % (2 * d));
+    const int i = row % n;
+    const long t = tb + row / n;
     const float v = c < d ? to_f(e[((size_t)ready[i] * max_len + t) * d + c])
-                          : s_prev[(size_t)i * d + c - d];
+                          : s_prev[(size_t)row * d + c - d];
     cat[idx] = v;
     if (catb) catb[idx] = __float2bfloat16_rn(v);
   }
@@ -331,15 +354,18 @@ __global__ void k_bw_rms_fwd(int d, float eps, const float *__restrict__ h,
   }
 }
 
-// Rotary encoding of the q part of a [n][3d] q/k/v row at position t.
-__global__ void k_bw_rope_q(int n, int H, int dh, long t, const float2 *__restrict__ rope,
-                            const float *__restrict__ qkv, float *__restrict__ q) {
+// Rotary encoding of the q part of [rows][3d] q/k/v rows, row = s n + i at
+// position tb + s.
+__global__ void k_bw_rope_q(int rows, int n, int H, int dh, long tb,
+                            const float2 *__restrict__ rope, const float *__restrict__ qkv,
+                            float *__restrict__ q) {
   BW_PDL();
   const int d = H * dh, half = dh / 2;
-  const long total = (long)n * H * half;
+  const long total = (long)rows * H * half;
   for (long idx = (long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long)gridDim.x * blockDim.x) {
     const int j = (int)(idx % half), h = (int)((idx / half) % H), i = (int)(idx / half / H);
+    const long t = tb + i / n;  // row i of step i / n
     const float2 cs = rope[(size_t)t * half + j];
     const float a = qkv[(size_t)i * 3 * d + h * dh + j], b = qkv[(size_t)i * 3 * d + h * dh + j + half];
     q[(size_t)i * d + h * dh + j] = a * cs.x - b * cs.y;
@@ -434,8 +460,9 @@ __device__ __forceinline__ void bw_merge(float &m, float &l, float *acc, float m
 
 constexpr int BW_ATT_WARPS = 4;
 
-// Attention of one query per (row, head) over key rows j_lo .. j_hi of the
-// key table: one CTA of four warps per (row, head); a key is read by DH / 8
+// Attention of one query per (row, head) over the keys of its position (the
+// SWA's window or the memory rows 0..t), rows of several steps (row = s n +
+// i at position tb + s): one CTA of four warps per (row, head); a key is read by DH / 8
 // lanes (eight head entries each, one 16-byte load for bf16), so a warp
 // takes 256 / DH keys at a time and the CTA 4x that. Each lane group keeps
 // its own online-softmax state; the states are merged in a fixed tree (lane
@@ -443,17 +470,23 @@ constexpr int BW_ATT_WARPS = 4;
 // depend on timing. Writes a and the log-sum-exp of the scaled scores.
 template <typename T, int DH>
 __global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
-    k_bw_attn_fwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
+    k_bw_attn_fwd(int n, int H, BwKeys<T> keys, long tb, long hist0, int Wm1, float scale,
                   const float *__restrict__ q, float *__restrict__ a, float *__restrict__ lse,
                   bf16 *__restrict__ ab) {
   BW_PDL();
   constexpr int LPK = DH / 8, KPW = 32 / LPK;
   __shared__ float red[BW_ATT_WARPS][2 + DH];
-  const int i = blockIdx.x / H, h = blockIdx.x % H, d = H * DH;
+  // row = s n + i: sequence i at position t = tb + s
+  const int row = blockIdx.x / H, h = blockIdx.x % H, d = H * DH, i = row % n;
+  const long t = tb + row / n;
+  // SWA: recorded positions max(0, t - W + 1) .. t (index pos - hist0);
+  // cross-attention: memory rows 0 .. t
+  const int j_lo = keys.swa ? (int)((t - Wm1 > 0 ? t - Wm1 : 0) - hist0) : 0;
+  const int j_hi = keys.swa ? (int)(t - hist0) : (int)t;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane / LPK, sl = lane % LPK;
   const T *K = keys.k(i, h), *V = keys.v(i, h);
   float qv[8], acc[8];
-  bw_ld8(q + (size_t)i * d + h * DH + sl * 8, qv);
+  bw_ld8(q + (size_t)row * d + h * DH + sl * 8, qv);
 #pragma unroll
   for (int e = 0; e < 8; e++) acc[e] = 0.f;
   float m = -INFINITY, l = 0.f;
@@ -514,10 +547,10 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
 #pragma unroll
     for (int e = 0; e < 8; e++) {
       const float v = acc[e] / l;
-      a[(size_t)i * d + h * DH + sl * 8 + e] = v;
-      if (ab) ab[(size_t)i * d + h * DH + sl * 8 + e] = __float2bfloat16_rn(v);
+      a[(size_t)row * d + h * DH + sl * 8 + e] = v;
+      if (ab) ab[(size_t)row * d + h * DH + sl * 8 + e] = __float2bfloat16_rn(v);
     }
-    if (sl == 0) lse[(size_t)i * H + h] = m + logf(l);
+    if (sl == 0) lse[(size_t)row * H + h] = m + logf(l);
   }
 }
 

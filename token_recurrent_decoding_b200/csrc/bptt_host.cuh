@@ -11,19 +11,29 @@
 // steps: 8 left the GEMMs' fixed cost a visible share of the step).
 constexpr int BW_GROUP = 32;
 
+// Steps whose forward the reverse traversal recomputes as one batch: a step's
+// recompute reads only recorded values (s_{t-1}, the recorded keys and
+// values, e_t), so up to BW_RECOMP steps of a group run their forward GEMMs
+// and attention as one launch over BW_RECOMP x n rows, before their backward
+// steps run one at a time.
+constexpr int BW_RECOMP = 8;
+
 // Workspace of one rlt_backward call: n rows, NS steps. Offsets in bytes.
 struct BwLayout {
   size_t s_hist, kv_hist, step, dring, xq, xda, xlse, xD, dmem, e32, de, total;
-  size_t wt, xb, grp, gg, n_dev;  // tensor-core operands; gain-gradient rows
-  size_t trl;                      // the list of the per-step transposes
-  size_t dmb, eT, wtm, rows_pad;   // memory-projection operands (bf16 models)
+  size_t wt, xf, xb, grp, gg, n_dev;  // tensor-core operands; gain-gradient rows
+  size_t trl;                          // the lists of the operand transposes
+  size_t dmb, eT, wtm, rows_pad;       // memory-projection operands (bf16 models)
   size_t step_floats, grp_layer_rows;
   int P;      // recorded positions t0 - (W-1) .. t1 - 1
-  int n_pad;  // rows of the bf16 operands (a multiple of 64)
+  int n_pad;  // rows of the bf16 gradient operands (a multiple of 64)
 };
 
-// Pointers into one step's region; every buffer starts on a 256-byte
-// boundary (the tensor-core epilogues store float2 / float4 vectors).
+// Pointers into the step region; every buffer starts on a 256-byte boundary
+// (the tensor-core epilogues store float2 / float4 vectors). The forward
+// values hold BW_RECOMP x n rows (row s n + i: batch step s, sequence i),
+// every per-layer block at a pitch of BW_RECOMP x n rows; the gradients of
+// the step being differentiated hold n rows.
 struct BwStep {
   float *cat, *gpre, *gs, *h, *u, *q1, *a1, *qx, *a2, *z, *zb, *act, *qkv, *ulast;
   float *r, *lse1, *lse2;
@@ -32,28 +42,30 @@ struct BwStep {
   static size_t floats(const rlt_config &c, int n) { return BwStep(nullptr, c, n).used; }
   BwStep(float *base, const rlt_config &c, int n) {
     const size_t d = c.d, F = c.ffn_dim, H = c.n_heads, L = c.n_dec_layers, N = n;
+    const size_t NR = N * BW_RECOMP;
+    const bool tc = c.dtype == RLT_BF16, sw = c.ffn_kind == RLT_SWIGLU;
     auto take = [&](size_t cnt) {
-      float *o = base ? base + used : nullptr;
+      float *o = base && cnt ? base + used : nullptr;
       used += (cnt + 63) / 64 * 64;
       return o;
     };
-    cat = take(N * 2 * d);
-    gpre = take(N * d);
-    gs = take(N * d);
-    h = take((3 * L + 1) * N * d);  // per layer: h1, h2, h3; then the final residual
-    u = take(3 * L * N * d);
-    q1 = take(L * N * d);
-    a1 = take(L * N * d);
-    qx = take(L * N * d);
-    a2 = take(L * N * d);
-    z = take(L * N * F);
-    zb = take(L * N * F);
-    act = take(L * N * F);
-    qkv = take(N * 3 * d);
-    ulast = take(N * d);
-    r = take((3 * L + 1) * N);
-    lse1 = take(L * N * H);
-    lse2 = take(L * N * H);
+    cat = take(NR * 2 * d);
+    gpre = take(NR * d);
+    gs = take(NR * d);
+    h = take((3 * L + 1) * NR * d);  // per layer: h1, h2, h3; then the final residual
+    u = take(tc ? 0 : 3 * L * NR * d);  // fp32 GEMM inputs (fp32 models)
+    q1 = take(L * NR * d);
+    a1 = take(L * NR * d);
+    qx = take(L * NR * d);
+    a2 = take(L * NR * d);
+    z = take(L * NR * F);
+    zb = take(sw ? L * NR * F : 0);
+    act = take(tc ? 0 : L * NR * F);
+    qkv = take(NR * 3 * d);
+    ulast = take(NR * d);
+    r = take((3 * L + 1) * NR);
+    lse1 = take(L * NR * H);
+    lse2 = take(L * NR * H);
     dh = take(N * d);
     dtmp = take(N * std::max(std::max(3 * d, F), 2 * d));
     dz = take(N * F);
@@ -66,13 +78,17 @@ struct BwStep {
   }
 };
 
-// Rows of one layer's group buffer: the transposed activations (u1, a1, u2,
-// a2, u3: d each; act: F) and output gradients (dqkv: 3d; dh at the SWA, the
+// Rows of one layer's bf16 forward operands (u1, a1, u2, a2, u3: d each;
+// act: F) and gradient operands (dqkv: 3d; dh at the SWA, the
 // cross-attention and the FFN outputs, dq of the cross-attention: d each;
-// dz, and dzb for SwiGLU: F).
-size_t bw_grp_layer_rows(const rlt_config &c) {
+// dz, and dzb for SwiGLU: F). A layer's group buffer holds both, transposed.
+size_t bw_fwd_layer_rows(const rlt_config &c) { return 5 * (size_t)c.d + c.ffn_dim; }
+size_t bw_grad_layer_rows(const rlt_config &c) {
   const size_t d = c.d, F = c.ffn_dim;
-  return 5 * d + F + 3 * d + 4 * d + F + (c.ffn_kind == RLT_SWIGLU ? F : 0);
+  return 3 * d + 4 * d + F + (c.ffn_kind == RLT_SWIGLU ? F : 0);
+}
+size_t bw_grp_layer_rows(const rlt_config &c) {
+  return bw_fwd_layer_rows(c) + bw_grad_layer_rows(c);
 }
 
 size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
@@ -94,21 +110,23 @@ size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
   B->xda = take(L * S * N * d * 4);
   B->xlse = take(L * S * N * H * 4);
   B->xD = take(L * S * N * H * 4);
-  // bf16 models: transposed weights, the row-major bf16 operand, the group
-  // buffers of the weight-gradient products
+  // bf16 models: transposed weights, the row-major bf16 operands (forward:
+  // BW_RECOMP x n rows; gradients: n_pad rows), the group buffers of the
+  // weight-gradient products
   const bool tc = c.dtype == RLT_BF16;
   const size_t NP = (N + 63) / 64 * 64;
   const size_t ffn_mats = c.ffn_kind == RLT_SWIGLU ? 3 : 2;
   B->n_pad = (int)NP;
   B->grp_layer_rows = bw_grp_layer_rows(c);
   B->wt = take(tc ? (L * (6 * d * d + ffn_mats * d * F) + 2 * d * d) * 2 : 0);
-  B->xb = take(tc ? (L * B->grp_layer_rows + 3 * d) * NP * 2 : 0);  // row-major operands
+  B->xf = take(tc ? (L * bw_fwd_layer_rows(c) + 2 * d) * N * BW_RECOMP * 2 : 0);
+  B->xb = take(tc ? (L * bw_grad_layer_rows(c) + d) * NP * 2 : 0);
   B->trl = take((13 * L + 2) * sizeof(BwTr));
   B->grp = take(tc ? (L * B->grp_layer_rows + 3 * d) * BW_GROUP * NP * 2 : 0);
   // per group: rows of the gain gradients (ln1..ln3 per layer, lnf) and of
   // the gate bias (dgpre)
   B->gg = take((3 * L + 2) * BW_GROUP * N * d * 4);
-  B->n_dev = take(4);
+  B->n_dev = take(4 * (BW_RECOMP + 1));
   const size_t G = c.mem_groups, RP = (N * c.max_len + 63) / 64 * 64;
   B->rows_pad = RP;
   B->dmem = take(tc ? 0 : G * N * c.max_len * 2 * d * 4);
@@ -176,74 +194,97 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   const float2 *rope = M->at<float2>(L.rope);
   const size_t nd = (size_t)n * d;
   const int n_pad = B.n_pad;
+  constexpr int R = BW_RECOMP;
+  // n_dev[r] = r n: the row count of an r-step batch, read by the decode GEMMs
   int *n_dev = reinterpret_cast<int *>(base + B.n_dev);
-  RLT_TRY(cudaMemcpyAsync(n_dev, &n, 4, cudaMemcpyHostToDevice, st));  // pageable: staged
+  {
+    int rows_of[R + 1];
+    for (int r = 0; r <= R; r++) rows_of[r] = r * n;
+    RLT_TRY(cudaMemcpyAsync(n_dev, rows_of, sizeof rows_of, cudaMemcpyHostToDevice, st));
+  }
 
   // ---- the bf16 operands of the tensor-core GEMMs, per layer: row-major
-  // as their producers write them (the decode GEMMs' A), and transposed into
-  // the group buffers at the end of each step (the weight gradients' A and B)
+  // as their producers write them (the GEMMs' A: forward operands for a
+  // batch of steps, gradient operands for one step), and transposed into the
+  // group buffers (the weight gradients' A and B)
   struct Ops {
     bf16 *u1, *a1, *u2, *a2, *u3, *act, *dqkv, *dhs, *dhx, *dqx, *dhf, *dz, *dzb;
   };
   std::vector<Ops> rb(LD, Ops{}), grp(LD, Ops{});
   bf16 *rb_cat = nullptr, *rb_dg = nullptr, *grp_cat = nullptr, *grp_dgpre = nullptr;
-  std::vector<BwTr> trl;
+  std::vector<BwTr> trf, trg;  // forward operands (per batch); gradients (per step)
   if (TC) {
-    auto carve = [&](bf16 *p, size_t blk, std::vector<Ops> &v, bf16 **cat, bf16 **dg) {
+    auto carve_fwd = [&](bf16 *&p, size_t blk, Ops &q) {
       auto take = [&](int rows) {
         bf16 *o = p;
         p += (size_t)rows * blk;
         return o;
       };
-      for (int l = 0; l < LD; l++) {
-        Ops &q = v[l];
-        q.u1 = take(d);
-        q.a1 = take(d);
-        q.u2 = take(d);
-        q.a2 = take(d);
-        q.u3 = take(d);
-        q.act = take(F);
-        q.dqkv = take(3 * d);
-        q.dhs = take(d);
-        q.dhx = take(d);
-        q.dqx = take(d);
-        q.dhf = take(d);
-        q.dz = take(F);
-        q.dzb = swiglu ? take(F) : nullptr;
-      }
-      *cat = take(2 * d);
-      *dg = take(d);
+      q.u1 = take(d);
+      q.a1 = take(d);
+      q.u2 = take(d);
+      q.a2 = take(d);
+      q.u3 = take(d);
+      q.act = take(F);
     };
-    bf16 *rbase = reinterpret_cast<bf16 *>(base + B.xb);
-    carve(rbase, (size_t)n_pad, rb, &rb_cat, &rb_dg);
-    carve(reinterpret_cast<bf16 *>(base + B.grp), (size_t)BW_GROUP * n_pad, grp, &grp_cat,
-          &grp_dgpre);
-    // padding rows of the row-major operands stay zero
-    RLT_TRY(cudaMemsetAsync(rbase, 0, (LD * B.grp_layer_rows + 3 * d) * (size_t)n_pad * 2, st));
+    auto carve_grad = [&](bf16 *&p, size_t blk, Ops &q) {
+      auto take = [&](int rows) {
+        bf16 *o = p;
+        p += (size_t)rows * blk;
+        return o;
+      };
+      q.dqkv = take(3 * d);
+      q.dhs = take(d);
+      q.dhx = take(d);
+      q.dqx = take(d);
+      q.dhf = take(d);
+      q.dz = take(F);
+      q.dzb = swiglu ? take(F) : nullptr;
+    };
+    const size_t fblk = (size_t)R * n, gblk = (size_t)BW_GROUP * n_pad;
+    bf16 *pf = reinterpret_cast<bf16 *>(base + B.xf), *pg = reinterpret_cast<bf16 *>(base + B.xb);
+    bf16 *pgrp = reinterpret_cast<bf16 *>(base + B.grp);
+    for (int l = 0; l < LD; l++) {
+      carve_fwd(pf, fblk, rb[l]);
+      carve_grad(pg, (size_t)n_pad, rb[l]);
+      carve_fwd(pgrp, gblk, grp[l]);
+      carve_grad(pgrp, gblk, grp[l]);
+    }
+    rb_cat = pf;
+    rb_dg = pg;
+    grp_cat = pgrp;
+    grp_dgpre = pgrp + (size_t)2 * d * gblk;
+    // padding rows of the gradient operands stay zero (the forward operands'
+    // tensor maps end at the batch's last row and read zeros past it)
+    RLT_TRY(cudaMemsetAsync(base + B.xb, 0, (LD * bw_grad_layer_rows(c) + d) * (size_t)n_pad * 2,
+                            st));
     for (int l = 0; l < LD; l++) {
       const Ops &a = rb[l], &b = grp[l];
-      trl.push_back({a.u1, b.u1, d});
-      trl.push_back({a.a1, b.a1, d});
-      trl.push_back({a.u2, b.u2, d});
-      trl.push_back({a.a2, b.a2, d});
-      trl.push_back({a.u3, b.u3, d});
-      trl.push_back({a.act, b.act, F});
-      trl.push_back({a.dqkv, b.dqkv, 3 * d});
-      trl.push_back({a.dhs, b.dhs, d});
-      trl.push_back({a.dhx, b.dhx, d});
-      trl.push_back({a.dqx, b.dqx, d});
-      trl.push_back({a.dhf, b.dhf, d});
-      trl.push_back({a.dz, b.dz, F});
-      if (swiglu) trl.push_back({a.dzb, b.dzb, F});
+      trf.push_back({a.u1, b.u1, d});
+      trf.push_back({a.a1, b.a1, d});
+      trf.push_back({a.u2, b.u2, d});
+      trf.push_back({a.a2, b.a2, d});
+      trf.push_back({a.u3, b.u3, d});
+      trf.push_back({a.act, b.act, F});
+      trg.push_back({a.dqkv, b.dqkv, 3 * d});
+      trg.push_back({a.dhs, b.dhs, d});
+      trg.push_back({a.dhx, b.dhx, d});
+      trg.push_back({a.dqx, b.dqx, d});
+      trg.push_back({a.dhf, b.dhf, d});
+      trg.push_back({a.dz, b.dz, F});
+      if (swiglu) trg.push_back({a.dzb, b.dzb, F});
     }
     if (c.alpha != 0.0f) {
-      trl.push_back({rb_cat, grp_cat, 2 * d});
-      trl.push_back({rb_dg, grp_dgpre, d});
+      trf.push_back({rb_cat, grp_cat, 2 * d});
+      trg.push_back({rb_dg, grp_dgpre, d});
     }
-    RLT_TRY(cudaMemcpyAsync(base + B.trl, trl.data(), trl.size() * sizeof(BwTr),
+    std::vector<BwTr> all(trf);
+    all.insert(all.end(), trg.begin(), trg.end());
+    RLT_TRY(cudaMemcpyAsync(base + B.trl, all.data(), all.size() * sizeof(BwTr),
                             cudaMemcpyHostToDevice, st));  // pageable: staged
   }
-  const BwTr *trl_dev = reinterpret_cast<const BwTr *>(base + B.trl);
+  const BwTr *trf_dev = reinterpret_cast<const BwTr *>(base + B.trl);
+  const BwTr *trg_dev = trf_dev + trf.size();
   // gain-gradient rows of a group: ln1, ln2, ln3 of layer l at 3l .. 3l+2,
   // lnf at 3L, the gate bias at 3L + 1; row block `slot` within each
   auto ggbuf = [&](int which, int slot_) {
@@ -278,23 +319,30 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     RLT_TRY(cudaGetLastError());
   }
 
-  // The group being filled: `cnt` steps, this step's column block `slot`.
+  // The group being filled: `cnt` steps, the next step's column block `slot`.
   int cnt = 0, slot = 0;
-  // out [n][N] = X [n][K] Wm^T (+ base_): bf16 models read the producer's
-  // bf16 copy Xb, fp32 models X
-  auto fwd = [&](const float *X, const bf16 *Xb, int K, const T *Wm, int N, float *out,
+  // out [rb n][N] = X [rb n][K] Wm^T (+ base_) over an rb-step batch: bf16
+  // models read the producer's bf16 copy Xb (tile GEMMs from 1024 rows, the
+  // decode GEMMs below), fp32 models X
+  auto fwd = [&](int rbs, const float *X, const bf16 *Xb, int K, const T *Wm, int N, float *out,
                  const float *base_) -> cudaError_t {
+    const int rows = rbs * n;
     if constexpr (TC) {
       (void)X;
+      if (rows >= 1024) {
+        if (base_) return gemm_tc(M, rows, rows, 0, N, K, Xb, Wm, EpiAddF32{base_, out, N}, st);
+        return gemm_tc(M, rows, rows, 0, N, K, Xb, Wm, EpiStoreF32{out, N}, st);
+      }
+      const int mg = (rows + 63) / 64 * 64;
       if (base_)
-        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, Xb, Wm,
+        return launch_dec<32>(M, mg, n_dev + rbs, rows, 0, N, K, Xb, Wm,
                               EpiAddF32Dec{{}, base_, out, N}, st);
-      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, N, K, Xb, Wm, EpiF32Dec{{}, out, N}, st);
+      return launch_dec<32>(M, mg, n_dev + rbs, rows, 0, N, K, Xb, Wm, EpiF32Dec{{}, out, N}, st);
     } else {
       (void)Xb;
       if (base_)
-        RLT_TRY(cudaMemcpyAsync(out, base_, (size_t)n * N * 4, cudaMemcpyDeviceToDevice, st));
-      return bw_gemm<true, true>(n, N, K, X, K, Wm, K, out, N, base_ != nullptr, st);
+        RLT_TRY(cudaMemcpyAsync(out, base_, (size_t)rows * N * 4, cudaMemcpyDeviceToDevice, st));
+      return bw_gemm<true, true>(rows, N, K, X, K, Wm, K, out, N, base_ != nullptr, st);
     }
   };
   // out [n][K] (=|+=) dY [n][N] Wm (Wm [N][K], WTm its transpose), and the
@@ -308,10 +356,10 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
       (void)ldx;
       (void)dW;
       if (acc)
-        return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, dYb, WTm,
+        return launch_dec<32>(M, n_pad, n_dev + 1, n_pad, 0, K, N, dYb, WTm,
                               EpiAccF32Dec{{}, out, K}, st);
-      return launch_dec<32>(M, n_pad, n_dev, n_pad, 0, K, N, dYb, WTm, EpiF32Dec{{}, out, K},
-                            st);
+      return launch_dec<32>(M, n_pad, n_dev + 1, n_pad, 0, K, N, dYb, WTm,
+                            EpiF32Dec{{}, out, K}, st);
     } else {
       (void)WTm;
       (void)dYb;
@@ -376,81 +424,91 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
         n, LD, H, DH, W, t1, const_cast<float *>(carry_in), S.dcarry, dring, 0);
     RLT_TRY(cudaGetLastError());
   }
-  const int attn_blocks = n * H;  // one CTA of BW_ATT_WARPS warps per (row, head)
-  auto hbuf = [&](int l, int which) { return S.h + ((size_t)3 * l + which) * nd; };
-  auto ubuf = [&](int l, int which) { return S.u + ((size_t)3 * l + which) * nd; };
-  auto rbuf = [&](int l, int which) { return S.r + ((size_t)3 * l + which) * n; };
-  // groups in processing order (t descending), the partial one first, so a
-  // group's column pitch is known when it starts
+  // forward values of batch step s (R x n rows per block, step s at row s n)
+  const size_t Rnd = (size_t)R * nd;
+  auto hbuf = [&](int l, int which, int s) { return S.h + ((size_t)3 * l + which) * Rnd + s * nd; };
+  auto ubuf = [&](int l, int which, int s) {
+    return TC ? nullptr : S.u + ((size_t)3 * l + which) * Rnd + s * nd;
+  };
+  auto rbuf = [&](int l, int which, int s) {
+    return S.r + ((size_t)3 * l + which) * R * n + (size_t)s * n;
+  };
+  auto lay = [&](float *p, int l, int s) { return p + l * Rnd + s * nd; };  // q1, a1, qx, a2
+  auto layF = [&](float *p, int l, int s) {                                // z, zb, act
+    return p ? p + ((size_t)l * R + s) * n * F : nullptr;
+  };
+  auto layH = [&](float *p, int l, int s) { return p + ((size_t)l * R + s) * n * H; };
   auto nb = [&](bf16 *p) { return TC ? p : nullptr; };  // bf16 outputs only for bf16 models
-  for (int k = NS - 1; k >= 0; k--) {
-    if (slot == cnt) {
-      const int done = NS - 1 - k;
-      cnt = done == 0 && NS % BW_GROUP ? NS % BW_GROUP : BW_GROUP;
-      slot = 0;
-    }
-    const long t = t0 + k;
-    const float *s_prev = s_hist + (size_t)k * nd;
-    // recompute the forward of step t
-    RLT_TRY(launch_k(k_bw_gate_cat<T>, bw_blocks(2 * (long)nd), 256, 0, st, n, d, ready, e,
-                     c.max_len, t, s_prev, S.cat, nb(rb_cat)));
+  const long hist0 = t0 - Wm1;  // position of recorded key row 0
+
+  // Forward of steps k_lo .. k_lo + rbs - 1 (positions tb ..), every layer,
+  // as one batch of rbs x n rows.
+  auto recompute = [&](int k_lo, int rbs) -> cudaError_t {
+    const long tb = t0 + k_lo;
+    const int rows = rbs * n;
+    const long rd = (long)rows * d;
+    RLT_TRY(launch_k(k_bw_gate_cat<T>, bw_blocks(2 * rd), 256, 0, st, rows, n, d, ready, e,
+                     c.max_len, tb, s_hist + (size_t)k_lo * nd, S.cat, nb(rb_cat)));
     if (c.alpha != 0.0f)
-      RLT_TRY(fwd(S.cat, rb_cat, 2 * d, (const T *)M->w.gate_w, d, S.gpre, nullptr));
+      RLT_TRY(fwd(rbs, S.cat, rb_cat, 2 * d, (const T *)M->w.gate_w, d, S.gpre, nullptr));
     else
-      RLT_TRY(cudaMemsetAsync(S.gpre, 0, nd * 4, st));
-    RLT_TRY(launch_k(k_bw_gate_fwd, bw_blocks(nd), 256, 0, st, n, d, S.gpre,
-                     (const float *)M->w.gate_b, S.cat, c.alpha, S.gs, hbuf(0, 0)));
+      RLT_TRY(cudaMemsetAsync(S.gpre, 0, rd * 4, st));
+    RLT_TRY(launch_k(k_bw_gate_fwd, bw_blocks(rd), 256, 0, st, rows, d, S.gpre,
+                     (const float *)M->w.gate_b, S.cat, c.alpha, S.gs, hbuf(0, 0, 0)));
     for (int l = 0; l < LD; l++) {
       const int g = G == 1 ? 0 : l;
-      float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2), *hn = hbuf(l + 1, 0);
-      // fp32 copies of the GEMM inputs only for fp32 models
-      float *u1 = TC ? nullptr : ubuf(l, 0), *u2 = TC ? nullptr : ubuf(l, 1),
-            *u3 = TC ? nullptr : ubuf(l, 2);
-      float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
-      float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
-            *act = TC ? nullptr : S.act + (size_t)l * n * F;
+      float *h1 = hbuf(l, 0, 0), *h2 = hbuf(l, 1, 0), *h3 = hbuf(l, 2, 0), *hn = hbuf(l + 1, 0, 0);
+      float *u1 = ubuf(l, 0, 0), *u2 = ubuf(l, 1, 0), *u3 = ubuf(l, 2, 0);
+      float *q1 = lay(S.q1, l, 0), *a1 = lay(S.a1, l, 0), *qx = lay(S.qx, l, 0),
+            *a2 = lay(S.a2, l, 0);
+      float *z = layF(S.z, l, 0), *zb = layF(S.zb, l, 0), *act = layF(S.act, l, 0);
       const Ops &o = rb[l];
-      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h1,
-                       (const float *)M->w.dec_ln1[l], u1, rbuf(l, 0), nb(o.u1)));
-      RLT_TRY(fwd(u1, o.u1, d, W_<T>::qkv(M, l), 3 * d, S.qkv, nullptr));
-      RLT_TRY(launch_k(k_bw_rope_q, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, t, rope,
+      RLT_TRY(launch_k(k_bw_rms_fwd, rows, 256, 0, st, d, c.rms_eps, h1,
+                       (const float *)M->w.dec_ln1[l], u1, rbuf(l, 0, 0), nb(o.u1)));
+      RLT_TRY(fwd(rbs, u1, o.u1, d, W_<T>::qkv(M, l), 3 * d, S.qkv, nullptr));
+      RLT_TRY(launch_k(k_bw_rope_q, bw_blocks(rd / 2), 256, 0, st, rows, n, H, DH, tb, rope,
                        S.qkv, q1));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
-      const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
-      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
-                       p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H, nb(o.a1)));
-      RLT_TRY(fwd(a1, o.a1, d, W_<T>::o(M, l), d, h2, h1));
-      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h2,
-                       (const float *)M->w.dec_ln2[l], u2, rbuf(l, 1), nb(o.u2)));
-      RLT_TRY(fwd(u2, o.u2, d, (const T *)M->w.dec_wqx[l], d, qx, nullptr));
+      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, rows * H, 32 * BW_ATT_WARPS, 0, st, n, H, swa, tb,
+                       hist0, Wm1, scale, q1, a1, layH(S.lse1, l, 0), nb(o.a1)));
+      RLT_TRY(fwd(rbs, a1, o.a1, d, W_<T>::o(M, l), d, h2, h1));
+      RLT_TRY(launch_k(k_bw_rms_fwd, rows, 256, 0, st, d, c.rms_eps, h2,
+                       (const float *)M->w.dec_ln2[l], u2, rbuf(l, 1, 0), nb(o.u2)));
+      RLT_TRY(fwd(rbs, u2, o.u2, d, (const T *)M->w.dec_wqx[l], d, qx, nullptr));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
-      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, xk, 0,
-                       (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, nb(o.a2)));
-      RLT_TRY(fwd(a2, o.a2, d, (const T *)M->w.dec_wox[l], d, h3, h2));
-      RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, h3,
-                       (const float *)M->w.dec_ln3[l], u3, rbuf(l, 2), nb(o.u3)));
-      RLT_TRY(fwd(u3, o.u3, d, W_<T>::w1(M, l), F, z, nullptr));
-      if (swiglu) RLT_TRY(fwd(u3, o.u3, d, W_<T>::wb(M, l), F, zb, nullptr));
-      RLT_TRY(launch_k(k_bw_act_fwd, bw_blocks((long)n * F), 256, 0, st, (long)n * F, swiglu, z,
-                       zb, act, nb(o.act)));
-      RLT_TRY(fwd(act, o.act, F, W_<T>::w2(M, l), d, hn, h3));
+      RLT_TRY(launch_k(k_bw_attn_fwd<T, DH>, rows * H, 32 * BW_ATT_WARPS, 0, st, n, H, xk, tb,
+                       0L, Wm1, scale, qx, a2, layH(S.lse2, l, 0), nb(o.a2)));
+      RLT_TRY(fwd(rbs, a2, o.a2, d, (const T *)M->w.dec_wox[l], d, h3, h2));
+      RLT_TRY(launch_k(k_bw_rms_fwd, rows, 256, 0, st, d, c.rms_eps, h3,
+                       (const float *)M->w.dec_ln3[l], u3, rbuf(l, 2, 0), nb(o.u3)));
+      RLT_TRY(fwd(rbs, u3, o.u3, d, W_<T>::w1(M, l), F, z, nullptr));
+      if (swiglu) RLT_TRY(fwd(rbs, u3, o.u3, d, W_<T>::wb(M, l), F, zb, nullptr));
+      RLT_TRY(launch_k(k_bw_act_fwd, bw_blocks((long)rows * F), 256, 0, st, (long)rows * F,
+                       swiglu, z, zb, act, nb(o.act)));
+      RLT_TRY(fwd(rbs, act, o.act, F, W_<T>::w2(M, l), d, hn, h3));
     }
-    float *rf = S.r + (size_t)3 * LD * n;
-    RLT_TRY(launch_k(k_bw_rms_fwd, n, 256, 0, st, d, c.rms_eps, hbuf(LD, 0),
-                     (const float *)M->w.dec_lnf, S.ulast, rf, (bf16 *)nullptr));
+    RLT_TRY(launch_k(k_bw_rms_fwd, rows, 256, 0, st, d, c.rms_eps, hbuf(LD, 0, 0),
+                     (const float *)M->w.dec_lnf, S.ulast, rbuf(LD, 0, 0), (bf16 *)nullptr));
+    return cudaSuccess;
+  };
 
+  // Backward of step k, batch step s; its gradient operands transposed into
+  // the group's column block `slot`.
+  auto backward = [&](int k, int s) -> cudaError_t {
+    const long t = t0 + k;
+    float *rf = rbuf(LD, 0, s);
     // differentiate step t: s_t = RMSNorm_f(h_L)
     RLT_TRY(launch_k(k_bw_ds_total, bw_blocks(nd), 256, 0, st, n, d, NS, k, sgrad, S.dcarry,
                      S.ds));
-    RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, hbuf(LD, 0), rf,
+    RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, hbuf(LD, 0, s), rf,
                      (const float *)M->w.dec_lnf, S.ds, S.dh, 1, ggbuf(3 * LD, slot),
                      nb(rb[LD - 1].dhf)));
     for (int l = LD - 1; l >= 0; l--) {
-      float *h1 = hbuf(l, 0), *h2 = hbuf(l, 1), *h3 = hbuf(l, 2);
-      float *u1 = ubuf(l, 0), *u2 = ubuf(l, 1), *u3 = ubuf(l, 2);
-      float *q1 = S.q1 + l * nd, *a1 = S.a1 + l * nd, *qx = S.qx + l * nd, *a2 = S.a2 + l * nd;
-      float *z = S.z + (size_t)l * n * F, *zb = S.zb + (size_t)l * n * F,
-            *act = S.act + (size_t)l * n * F;
+      float *h1 = hbuf(l, 0, s), *h2 = hbuf(l, 1, s), *h3 = hbuf(l, 2, s);
+      float *u1 = ubuf(l, 0, s), *u2 = ubuf(l, 1, s), *u3 = ubuf(l, 2, s);
+      float *q1 = lay(S.q1, l, s), *a1 = lay(S.a1, l, s), *qx = lay(S.qx, l, s),
+            *a2 = lay(S.a2, l, s);
+      float *z = layF(S.z, l, s), *zb = layF(S.zb, l, s), *act = layF(S.act, l, s);
       const Ops &o = rb[l];
       // FFN: h_out = h3 + W2 act(W1 u3)
       RLT_TRY(bwd(S.dh, o.dhf, d, W_<T>::w2(M, l), wt[l].w2, F, S.dtmp, false, act, F,
@@ -462,7 +520,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
       if (swiglu)
         RLT_TRY(bwd(S.dzb, o.dzb, F, W_<T>::wb(M, l), wt[l].wb, d, S.du, true, u3, d,
                     gr->dec_wb[l]));
-      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h3, rbuf(l, 2),
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h3, rbuf(l, 2, s),
                        (const float *)M->w.dec_ln3[l], S.du, S.dh, 0, ggbuf(3 * l + 2, slot),
                        nb(o.dhx)));
       // cross-attention: h3 = h2 + W_ox attn(W_qx u2, M<=t)
@@ -471,48 +529,70 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
                   gr->dec_wox[l]));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
       const size_t xo = ((size_t)l * NS + k) * nd, xs = ((size_t)l * NS + k) * n * H;
-      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, xk, 0,
-                       (int)t, scale, qx, a2, S.lse2 + (size_t)l * n * H, S.dtmp, S.dq,
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, n * H, 32 * BW_ATT_WARPS, 0, st, n, H, xk, 0,
+                       (int)t, scale, qx, a2, layH(S.lse2, l, s), S.dtmp, S.dq,
                        (float *)nullptr, W, 0L, xq + xo, xda + xo, xlse + xs, xD + xs,
                        nb(o.dqx)));
       RLT_TRY(bwd(S.dq, o.dqx, d, (const T *)M->w.dec_wqx[l], wt[l].qx, d, S.du, false, u2, d,
                   gr->dec_wqx[l]));
-      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h2, rbuf(l, 1),
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h2, rbuf(l, 1, s),
                        (const float *)M->w.dec_ln2[l], S.du, S.dh, 0, ggbuf(3 * l + 1, slot),
                        nb(o.dhs)));
       // SWA: h2 = h1 + W_o attn(q_t over the window); k_t, v_t enter the cache
       RLT_TRY(bwd(S.dh, o.dhs, d, W_<T>::o(M, l), wt[l].o, d, S.dtmp, false, a1, d,
                   gr->dec_wo[l]));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
-      const int p_lo = (int)(std::max(0L, t - Wm1) - (t0 - Wm1)), p_hi = (int)(t - (t0 - Wm1));
-      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, attn_blocks, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
-                       p_lo, p_hi, scale, q1, a1, S.lse1 + (size_t)l * n * H, S.dtmp, S.dq,
-                       dring, W, (long)(t0 - Wm1), (float *)nullptr, (float *)nullptr,
+      const int p_lo = (int)(std::max(0L, t - Wm1) - hist0), p_hi = (int)(t - hist0);
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, n * H, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
+                       p_lo, p_hi, scale, q1, a1, layH(S.lse1, l, s), S.dtmp, S.dq,
+                       dring, W, hist0, (float *)nullptr, (float *)nullptr,
                        (float *)nullptr, (float *)nullptr, (bf16 *)nullptr));
       RLT_TRY(launch_k(k_bw_qkv_grad, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, W, t,
                        rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv, nb(o.dqkv)));
       RLT_TRY(bwd(S.dqkv, o.dqkv, 3 * d, W_<T>::qkv(M, l), wt[l].qkv, d, S.du, false, u1, d,
                   gr->dec_wqkv[l]));
-      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h1, rbuf(l, 0),
+      RLT_TRY(launch_k(k_bw_rms_bwd, n, 256, 0, st, d, h1, rbuf(l, 0, s),
                        (const float *)M->w.dec_ln1[l], S.du, S.dh, 0, ggbuf(3 * l, slot),
                        l > 0 ? nb(rb[l - 1].dhf) : (bf16 *)nullptr));
     }
     // gated merge: x = e_t + alpha sigmoid(W_g [e_t; s_{t-1}] + b_g) s_{t-1}
     float *dgpre = ggbuf(3 * LD + 1, slot);
-    RLT_TRY(launch_k(k_bw_gate_bwd, bw_blocks(nd), 256, 0, st, n, d, c.alpha, S.dh, S.cat, S.gs,
-                     dgpre, S.dcarry, egrad, c.max_len, t,
+    float *cat = S.cat + (size_t)s * 2 * nd;
+    RLT_TRY(launch_k(k_bw_gate_bwd, bw_blocks(nd), 256, 0, st, n, d, c.alpha, S.dh, cat,
+                     S.gs + s * nd, dgpre, S.dcarry, egrad, c.max_len, t,
                      c.alpha != 0.0f ? nb(rb_dg) : (bf16 *)nullptr));
     if (c.alpha != 0.0f) {
-      RLT_TRY(bwd(dgpre, rb_dg, d, (const T *)M->w.gate_w, wt_gate, 2 * d, S.dtmp, false, S.cat,
+      RLT_TRY(bwd(dgpre, rb_dg, d, (const T *)M->w.gate_w, wt_gate, 2 * d, S.dtmp, false, cat,
                   2 * d, gr->gate_w));
       RLT_TRY(launch_k(k_bw_gate_bwd2, bw_blocks(nd), 256, 0, st, n, d, S.dtmp, S.dcarry, egrad,
                        c.max_len, t));
     }
-    // this step's operands, transposed into the group's column block
     if (TC)
-      RLT_TRY(launch_k(k_bw_grp_transpose, dim3(64, (unsigned)trl.size()), dim3(32, 8), 0, st,
-                       trl_dev, n, n_pad, (long)cnt * n_pad, (long)slot * n_pad));
-    if (++slot == cnt) RLT_TRY(flush());
+      RLT_TRY(launch_k(k_bw_grp_transpose, dim3(64, (unsigned)trg.size()), dim3(32, 8), 0, st,
+                       trg_dev, n, n_pad, 1, (long)cnt * n_pad, (long)slot));
+    return cudaSuccess;
+  };
+
+  // Groups in processing order (t descending), the partial one first so a
+  // group's column pitch is known when it starts; each group in batches of
+  // up to R steps, recomputed together, then differentiated one by one.
+  for (int k = NS - 1; k >= 0;) {
+    const int done = NS - 1 - k;
+    cnt = done == 0 && NS % BW_GROUP ? NS % BW_GROUP : BW_GROUP;
+    slot = 0;
+    while (slot < cnt) {
+      const int rbs = std::min(R, cnt - slot), k_lo = k - rbs + 1;
+      RLT_TRY(recompute(k_lo, rbs));
+      // the batch's forward operands into column blocks slot .. slot+rbs-1
+      // (step k_lo + s into block slot + rbs - 1 - s, the order it is
+      // differentiated in)
+      if (TC)
+        RLT_TRY(launch_k(k_bw_grp_transpose, dim3(32 * rbs, (unsigned)trf.size()), dim3(32, 8),
+                         0, st, trf_dev, n, n_pad, rbs, (long)cnt * n_pad, (long)slot));
+      for (int s = rbs - 1; s >= 0; s--, slot++) RLT_TRY(backward(k_lo + s, s));
+      k = k_lo - 1;
+    }
+    RLT_TRY(flush());
   }
   // the state entering the chunk
   if (carry_out) {
