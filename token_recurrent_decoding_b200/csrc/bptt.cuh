@@ -558,19 +558,25 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
 // Attention backward of one query per (row, head) over key rows
 // j_lo .. j_hi, with the lane layout of k_bw_attn_fwd: P_j = exp(scale q.k_j
 // - lse), dS_j = P_j (da.v_j - da.a), dq = scale sum_j dS_j k_j (lane-group
-// partial sums merged in a fixed order). SWA (dring != null): also
-// dk_j += scale dS_j q and dv_j += P_j da into the gradient ring slot of
-// position pos0 + j (each key is owned by one lane group). Cross-attention
-// (xq != null): q, da, lse and D = da.a are saved for the memory-gradient
-// pass.
-template <typename T, int DH>
-__global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
+// partial sums merged in a fixed order). q, da, lse and D = da.a are saved
+// (xq, xda, xlse, xD): the cross-attention's for the memory-gradient pass,
+// the SWA's for k_bw_swa_dkv. SWA (RING): keys at positions pos0 + j >=
+// p_rmw (those of the batch being differentiated) also take dk_j += scale
+// dS_j q and dv_j += P_j da in their gradient ring slot (each key is owned by
+// one lane group); older keys take this step's terms later, from the saved
+// values. The two forms are separate instantiations so the
+// cross-attention's loop, the long one, carries no ring registers.
+#ifndef BW_XU
+#define BW_XU 2  // keys per lane group in flight in the cross-attention backward
+#endif
+template <typename T, int DH, bool RING>
+__global__ void __launch_bounds__(32 * BW_ATT_WARPS, RING || BW_XU > 2 ? 6 : 8)
     k_bw_attn_bwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
                   const float *__restrict__ q, const float *__restrict__ a,
                   const float *__restrict__ lse, const float *__restrict__ da,
                   float *__restrict__ dq, float *__restrict__ dring, int W, long pos0,
-                  float *__restrict__ xq, float *__restrict__ xda, float *__restrict__ xlse,
-                  float *__restrict__ xD, bf16 *__restrict__ dqb) {
+                  long p_rmw, float *__restrict__ xq, float *__restrict__ xda,
+                  float *__restrict__ xlse, float *__restrict__ xD, bf16 *__restrict__ dqb) {
   BW_PDL();
   constexpr int LPK = DH / 8, KPW = 32 / LPK;
   __shared__ float red[BW_ATT_WARPS][DH];
@@ -590,25 +596,27 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
   }
   const float D = bw_group_sum<LPK>(Dp);
   const float L = lse[(size_t)i * H + h];
-  float *dk_ring = dring ? dring + ((((size_t)keys.l_or_g * n + i) * H + h) * 2 + 0) * W * DH
-                         : nullptr;
-  float *dv_ring = dring ? dk_ring + (size_t)W * DH : nullptr;
-  constexpr int S = BW_ATT_WARPS * KPW;  // keys per CTA pass; two passes per iteration
-  for (int base = j_lo + warp * KPW; base <= j_hi; base += 2 * S) {
-    BwRaw8<T> kv2[2], vv2[2];
-    float dot2[2] = {0.f, 0.f}, dp2[2] = {0.f, 0.f};
-    bool ok2[2];
+  float *dk_ring = RING ? dring + ((((size_t)keys.l_or_g * n + i) * H + h) * 2 + 0) * W * DH
+                        : nullptr;
+  float *dv_ring = RING ? dk_ring + (size_t)W * DH : nullptr;
+  constexpr int S = BW_ATT_WARPS * KPW;  // keys per CTA pass
+  constexpr int U = RING ? 2 : BW_XU;     // passes per iteration (loads in flight)
+  for (int base = j_lo + warp * KPW; base <= j_hi; base += U * S) {
+    BwRaw8<T> kv2[U], vv2[U];
+    float dot2[U], dp2[U];
+    bool ok2[U];
 #pragma unroll
-    for (int u = 0; u < 2; u++) {
+    for (int u = 0; u < U; u++) {
       const int j = base + grp + u * S;
       ok2[u] = j <= j_hi;
+      dot2[u] = dp2[u] = 0.f;
       if (ok2[u]) {
         kv2[u].load(K + (size_t)j * DH + sl * 8);
         vv2[u].load(V + (size_t)j * DH + sl * 8);
       }
     }
 #pragma unroll
-    for (int u = 0; u < 2; u++) {
+    for (int u = 0; u < U; u++) {
       if (ok2[u])
 #pragma unroll
         for (int e = 0; e < 8; e++) {
@@ -619,14 +627,14 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
       dp2[u] = bw_group_sum<LPK>(dp2[u]);
     }
 #pragma unroll
-    for (int u = 0; u < 2; u++) {
+    for (int u = 0; u < U; u++) {
       if (!ok2[u]) continue;
       const int j = base + grp + u * S;
       const float p = expf(dot2[u] * scale - L);
       const float ds = p * (dp2[u] - D);
 #pragma unroll
       for (int e = 0; e < 8; e++) dqv[e] += scale * ds * kv2[u].at(e);
-      if (dk_ring) {
+      if (RING && pos0 + j >= p_rmw) {
         const size_t slot = (size_t)((pos0 + j) % W) * DH + sl * 8;
         float4 *pk = reinterpret_cast<float4 *>(dk_ring + slot);
         float4 *pv = reinterpret_cast<float4 *>(dv_ring + slot);
@@ -663,15 +671,131 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
     for (int e = 0; e < 8; e++) {
       dq[off + e] = dqv[e];
       if (dqb) dqb[off + e] = __float2bfloat16_rn(dqv[e]);
-      if (xq) {
-        xq[off + e] = qv[e];
-        xda[off + e] = dav[e];
-      }
+      xq[off + e] = qv[e];
+      xda[off + e] = dav[e];
     }
-    if (xq && sl == 0) {
+    if (sl == 0) {
       xlse[(size_t)i * H + h] = L;
       xD[(size_t)i * H + h] = D;
     }
+  }
+}
+
+// The SWA keys' and values' gradient terms of already differentiated steps:
+// for each position p in [p_lo, p_hi] and each step t in [max(p, t_lo),
+// min(p + W - 1, t_hi)] (the steps whose window holds p), from the values
+// k_bw_attn_bwd saved at step t (record slot t mod Dr): P = exp(scale
+// q_t.k_p - lse_t), dS = P (da_t.v_p - D_t); dk_p += scale dS q_t and
+// dv_p += P da_t, added to the gradient ring slot p mod W. One CTA per
+// (layer, row, head); the steps' records pass through shared memory TS at a
+// time, each warp owns two positions (eight per pass) and its lane groups
+// split the steps, merged in a fixed order.
+template <typename T, int DH>
+__global__ void __launch_bounds__(128, 4)
+    k_bw_swa_dkv(int n, int H, int W, int Dr, long p_lo, long p_hi, long t_lo, long t_hi,
+                 long hist0, int P_hist, const T *__restrict__ kv_hist,
+                 const float *__restrict__ rq, const float *__restrict__ rda,
+                 const float *__restrict__ rlse, const float *__restrict__ rD, float scale,
+                 float *__restrict__ dring) {
+  BW_PDL();
+  constexpr int LPK = DH / 8, KPW = 32 / LPK, NW = 4, PPW = 2, TS = 16;
+  __shared__ __align__(16) float sq[TS][DH];
+  __shared__ __align__(16) float sda[TS][DH];
+  __shared__ float slse[TS], sD[TS];
+  const int h = blockIdx.x % H, i = (blockIdx.x / H) % n, l = blockIdx.x / H / n, d = H * DH;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane / LPK, sl = lane % LPK;
+  const size_t kvh = (((size_t)l * n + i) * H + h) * 2;
+  const T *Kb = kv_hist + kvh * P_hist * DH, *Vb = Kb + (size_t)P_hist * DH;
+  float *dkr = dring + kvh * W * DH, *dvr = dkr + (size_t)W * DH;
+  for (long pc = p_lo; pc <= p_hi; pc += NW * PPW) {
+    const long p0 = pc + warp * PPW;
+    float kk[PPW][8], vv[PPW][8], dk[PPW][8], dv[PPW][8];
+#pragma unroll
+    for (int u = 0; u < PPW; u++) {
+      const long p = p0 + u;
+#pragma unroll
+      for (int e = 0; e < 8; e++) kk[u][e] = vv[u][e] = dk[u][e] = dv[u][e] = 0.f;
+      if (p <= p_hi) {
+        bw_ld8(Kb + (size_t)(p - hist0) * DH + sl * 8, kk[u]);
+        bw_ld8(Vb + (size_t)(p - hist0) * DH + sl * 8, vv[u]);
+      }
+    }
+    const long pe = pc + NW * PPW - 1 < p_hi ? pc + NW * PPW - 1 : p_hi;
+    const long ts_lo = t_lo > pc ? t_lo : pc, ts_hi = t_hi < pe + W - 1 ? t_hi : pe + W - 1;
+    for (long tt = ts_lo; tt <= ts_hi; tt += TS) {
+      __syncthreads();
+      for (int x = threadIdx.x; x < TS * DH / 4; x += blockDim.x) {
+        const int s = x / (DH / 4), c = (x % (DH / 4)) * 4;
+        const long t = tt + s;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+        if (t <= ts_hi) {
+          const size_t ro = (((size_t)l * Dr + t % Dr) * n + i) * d + h * DH + c;
+          a = *reinterpret_cast<const float4 *>(rq + ro);
+          b = *reinterpret_cast<const float4 *>(rda + ro);
+        }
+        *reinterpret_cast<float4 *>(&sq[s][c]) = a;
+        *reinterpret_cast<float4 *>(&sda[s][c]) = b;
+      }
+      if (threadIdx.x < TS) {
+        const long t = tt + threadIdx.x;
+        const size_t ro = (((size_t)l * Dr + t % Dr) * n + i) * H + h;
+        slse[threadIdx.x] = t <= ts_hi ? rlse[ro] : 0.f;
+        sD[threadIdx.x] = t <= ts_hi ? rD[ro] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int s0 = 0; s0 < TS; s0 += KPW) {
+        const int s = s0 + grp;
+        const long t = tt + s;
+        float qs[8], das[8];
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+          qs[e] = sq[s][sl * 8 + e];
+          das[e] = sda[s][sl * 8 + e];
+        }
+#pragma unroll
+        for (int u = 0; u < PPW; u++) {
+          const long p = p0 + u;
+          float dot = 0.f, dp = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; e++) {
+            dot += qs[e] * kk[u][e];
+            dp += das[e] * vv[u][e];
+          }
+          dot = bw_group_sum<LPK>(dot);
+          dp = bw_group_sum<LPK>(dp);
+          if (p <= p_hi && t <= ts_hi && t >= p && t <= p + W - 1) {
+            const float P = expf(dot * scale - slse[s]), ds = P * (dp - sD[s]);
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+              dk[u][e] += scale * ds * qs[e];
+              dv[u][e] += P * das[e];
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = LPK; o < 32; o <<= 1)
+#pragma unroll
+      for (int u = 0; u < PPW; u++)
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+          dk[u][e] += __shfl_xor_sync(FULL_MASK, dk[u][e], o);
+          dv[u][e] += __shfl_xor_sync(FULL_MASK, dv[u][e], o);
+        }
+    if (grp == 0)
+#pragma unroll
+      for (int u = 0; u < PPW; u++) {
+        const long p = p0 + u;
+        if (p > p_hi) continue;
+        float *k = dkr + (size_t)(p % W) * DH + sl * 8, *v = dvr + (size_t)(p % W) * DH + sl * 8;
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+          k[e] += dk[u][e];
+          v[e] += dv[u][e];
+        }
+      }
   }
 }
 

@@ -21,12 +21,14 @@ constexpr int BW_RECOMP = 8;
 // Workspace of one rlt_backward call: n rows, NS steps. Offsets in bytes.
 struct BwLayout {
   size_t s_hist, kv_hist, step, dring, xq, xda, xlse, xD, dmem, e32, de, total;
+  size_t rec;  // the SWA's saved q, da, lse, D of the last Dr steps (slot t mod Dr)
   size_t wt, xf, xb, grp, gg, n_dev;  // tensor-core operands; gain-gradient rows
   size_t trl;                          // the lists of the operand transposes
   size_t dmb, eT, wtm, rows_pad;       // memory-projection operands (bf16 models)
   size_t step_floats, grp_layer_rows;
   int P;      // recorded positions t0 - (W-1) .. t1 - 1
   int n_pad;  // rows of the bf16 gradient operands (a multiple of 64)
+  int Dr;     // record slots: BW_RECOMP + W
 };
 
 // Pointers into the step region; every buffer starts on a 256-byte boundary
@@ -110,6 +112,8 @@ size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
   B->xda = take(L * S * N * d * 4);
   B->xlse = take(L * S * N * H * 4);
   B->xD = take(L * S * N * H * 4);
+  B->Dr = BW_RECOMP + (int)W;
+  B->rec = take(L * B->Dr * N * (2 * d + 2 * H) * 4);
   // bf16 models: transposed weights, the row-major bf16 operands (forward:
   // BW_RECOMP x n rows; gradients: n_pad rows), the group buffers of the
   // weight-gradient products
@@ -187,6 +191,10 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   float *dmem = reinterpret_cast<float *>(base + B.dmem);
   float *e32 = reinterpret_cast<float *>(base + B.e32), *de = reinterpret_cast<float *>(base + B.de);
   float *gg = reinterpret_cast<float *>(base + B.gg);
+  const int Dr = B.Dr;
+  float *rq = reinterpret_cast<float *>(base + B.rec);
+  float *rda = rq + (size_t)LD * Dr * n * d, *rlse = rda + (size_t)LD * Dr * n * d;
+  float *rD = rlse + (size_t)LD * Dr * n * H;
   BwStep S(reinterpret_cast<float *>(base + B.step), c, n);
   const int *ready = M->at<int>(L.ready);
   const T *ring = M->at<T>(L.ring), *mem = M->at<T>(L.mem), *e = M->at<T>(L.e);
@@ -492,8 +500,21 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     return cudaSuccess;
   };
 
-  // Backward of step k, batch step s; its gradient operands transposed into
-  // the group's column block `slot`.
+  // Gradient terms of the SWA keys at positions p_lo .. p_hi from the saved
+  // values of steps t_lo .. t_hi (already differentiated), every layer.
+  auto swa_dkv = [&](long p_lo, long p_hi, long t_lo, long t_hi) -> cudaError_t {
+    if (p_lo < 0) p_lo = 0;
+    if (p_lo < t_lo - Wm1) p_lo = t_lo - Wm1;
+    if (p_lo > p_hi || t_lo > t_hi) return cudaSuccess;
+    return launch_k(k_bw_swa_dkv<T, DH>, LD * n * H, 128, 0, st, n, H, W, Dr, p_lo, p_hi, t_lo,
+                    t_hi, hist0, B.P, (const T *)kv_hist, (const float *)rq,
+                    (const float *)rda, (const float *)rlse, (const float *)rD, scale, dring);
+  };
+
+  // Backward of step k, batch step s, in the batch whose first step is
+  // k_batch; its gradient operands transposed into the group's column block
+  // `slot`.
+  int k_batch = 0;
   auto backward = [&](int k, int s) -> cudaError_t {
     const long t = t0 + k;
     float *rf = rbuf(LD, 0, s);
@@ -529,9 +550,9 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
                   gr->dec_wox[l]));
       BwKeys<T> xk{mem, ready, g, n, H, DH, 0, c.max_seqs, c.max_len, false};
       const size_t xo = ((size_t)l * NS + k) * nd, xs = ((size_t)l * NS + k) * n * H;
-      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, n * H, 32 * BW_ATT_WARPS, 0, st, n, H, xk, 0,
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH, false>, n * H, 32 * BW_ATT_WARPS, 0, st, n, H, xk, 0,
                        (int)t, scale, qx, a2, layH(S.lse2, l, s), S.dtmp, S.dq,
-                       (float *)nullptr, W, 0L, xq + xo, xda + xo, xlse + xs, xD + xs,
+                       (float *)nullptr, W, 0L, 0L, xq + xo, xda + xo, xlse + xs, xD + xs,
                        nb(o.dqx)));
       RLT_TRY(bwd(S.dq, o.dqx, d, (const T *)M->w.dec_wqx[l], wt[l].qx, d, S.du, false, u2, d,
                   gr->dec_wqx[l]));
@@ -543,10 +564,11 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
                   gr->dec_wo[l]));
       BwKeys<T> swa{kv_hist, ready, l, n, H, DH, B.P, c.max_seqs, c.max_len, true};
       const int p_lo = (int)(std::max(0L, t - Wm1) - hist0), p_hi = (int)(t - hist0);
-      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH>, n * H, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
+      const size_t ro = ((size_t)l * Dr + t % Dr) * nd, rs = ((size_t)l * Dr + t % Dr) * n * H;
+      RLT_TRY(launch_k(k_bw_attn_bwd<T, DH, true>, n * H, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
                        p_lo, p_hi, scale, q1, a1, layH(S.lse1, l, s), S.dtmp, S.dq,
-                       dring, W, hist0, (float *)nullptr, (float *)nullptr,
-                       (float *)nullptr, (float *)nullptr, (bf16 *)nullptr));
+                       dring, W, hist0, t0 + k_batch, rq + ro, rda + ro, rlse + rs, rD + rs,
+                       (bf16 *)nullptr));
       RLT_TRY(launch_k(k_bw_qkv_grad, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, W, t,
                        rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv, nb(o.dqkv)));
       RLT_TRY(bwd(S.dqkv, o.dqkv, 3 * d, W_<T>::qkv(M, l), wt[l].qkv, d, S.du, false, u1, d,
@@ -583,6 +605,9 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     while (slot < cnt) {
       const int rbs = std::min(R, cnt - slot), k_lo = k - rbs + 1;
       RLT_TRY(recompute(k_lo, rbs));
+      // the batch's SWA keys take the terms of the steps after it
+      RLT_TRY(swa_dkv(t0 + k_lo, t0 + k, t0 + k + 1, t1 - 1));
+      k_batch = k_lo;
       // the batch's forward operands into column blocks slot .. slot+rbs-1
       // (step k_lo + s into block slot + rbs - 1 - s, the order it is
       // differentiated in)
@@ -594,8 +619,10 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
     }
     RLT_TRY(flush());
   }
-  // the state entering the chunk
+  // the state entering the chunk (the window's keys before t0 take the
+  // terms of the chunk's steps first)
   if (carry_out) {
+    RLT_TRY(swa_dkv(t0 - Wm1, t0 - 1, t0, t1 - 1));
     k_bw_carry<<<bw_blocks((long)n * d * (1 + 2L * LD * Wm1)), 256, 0, st>>>(
         n, LD, H, DH, W, t0, carry_out, S.dcarry, dring, 1);
     RLT_TRY(cudaGetLastError());
