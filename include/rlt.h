@@ -397,9 +397,11 @@ typedef struct rlt_grads {
 
 /* Host only. Device workspace bytes of rlt_backward for n rows and n_steps
  * positions (0 if the configuration is invalid). It holds the recorded s_t
- * and keys/values of the chunk, one step's activations, the saved
- * cross-attention terms and the memory-row gradients: about
- * n * n_steps * L_D * d * 8 + G * n * max_len * d * 8 bytes. */
+ * and keys/values of the chunk, the activations of a batch of up to eight
+ * recomputed steps, the saved cross-attention terms, the saved SWA terms of
+ * the last 8 + W steps and the memory-row gradients: about
+ * n * n_steps * L_D * d * 8 + G * n * max_len * d * 8 bytes plus a term
+ * independent of n_steps. */
 RLT_API size_t rlt_backward_workspace_bytes(const rlt_config *cfg, int n, int n_steps);
 
 /* One chunk of backpropagation through time for the listed sequences, all
@@ -408,9 +410,10 @@ RLT_API size_t rlt_backward_workspace_bytes(const rlt_config *cfg, int n, int n_
  *      model's own step kernels, exactly as rlt_run_sequence, recording s_t
  *      and every layer's (k_t, v_t) in the workspace; the sequences end at
  *      t_dec = t1 as after rlt_run_sequence.
- *   2. Reverse traversal t = t1-1 .. t0: the step's forward is recomputed
- *      from the recorded state and differentiated layer by layer; a key or
- *      value entry's gradient accumulates over the steps that read it.
+ *   2. Reverse traversal t = t1-1 .. t0: the forward is recomputed from
+ *      the recorded state (up to eight steps at once) and each step is
+ *      differentiated layer by layer; a key or value entry's gradient
+ *      accumulates over the steps that read it.
  *   3. The gradient of the memory rows M<=t1-1 is pushed through the memory
  *      projection into e and the mem_wk / mem_wv gradients.
  * The loss is L = sum_t <d_sgrad[i][t-t0], s_t> (+ <d_carry_in, H_{t1-1}>):

@@ -690,6 +690,12 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, RING || BW_XU > 2 ? 6 : 8)
 // (layer, row, head); the steps' records pass through shared memory TS at a
 // time, each warp owns two positions (eight per pass) and its lane groups
 // split the steps, merged in a fixed order.
+// 4-byte asynchronous copy into shared memory (zero-filled when src_bytes is 0).
+__device__ __forceinline__ void bw_cp4(uint32_t dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes));
+}
+
 template <typename T, int DH>
 __global__ void __launch_bounds__(128, 4)
     k_bw_swa_dkv(int n, int H, int W, int Dr, long p_lo, long p_hi, long t_lo, long t_hi,
@@ -698,15 +704,35 @@ __global__ void __launch_bounds__(128, 4)
                  const float *__restrict__ rlse, const float *__restrict__ rD, float scale,
                  float *__restrict__ dring) {
   BW_PDL();
-  constexpr int LPK = DH / 8, KPW = 32 / LPK, NW = 4, PPW = 2, TS = 16;
-  __shared__ __align__(16) float sq[TS][DH];
-  __shared__ __align__(16) float sda[TS][DH];
-  __shared__ float slse[TS], sD[TS];
+  constexpr int LPK = DH / 8, KPW = 32 / LPK, NW = 4, PPW = 2, TS = DH >= 128 ? 16 : 32;
+  // two buffers: the records of the next TS steps load while these are used
+  __shared__ __align__(16) float sq[2][TS][DH];
+  __shared__ __align__(16) float sda[2][TS][DH];
+  __shared__ float slse[2][TS], sD[2][TS];
   const int h = blockIdx.x % H, i = (blockIdx.x / H) % n, l = blockIdx.x / H / n, d = H * DH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane / LPK, sl = lane % LPK;
   const size_t kvh = (((size_t)l * n + i) * H + h) * 2;
   const T *Kb = kv_hist + kvh * P_hist * DH, *Vb = Kb + (size_t)P_hist * DH;
   float *dkr = dring + kvh * W * DH, *dvr = dkr + (size_t)W * DH;
+  // the records of steps tt .. tt + TS - 1 (zeros past ts_hi) into buffer b
+  auto load_tile = [&](int b, long tt, long ts_hi) {
+    for (int x = threadIdx.x; x < TS * DH / 4; x += blockDim.x) {
+      const int s = x / (DH / 4), c = (x % (DH / 4)) * 4;
+      const long t = tt + s;
+      const bool ok = t <= ts_hi;
+      const size_t ro = ok ? (((size_t)l * Dr + t % Dr) * n + i) * d + h * DH + c : 0;
+      cp_async16(smem_u32(&sq[b][s][c]), rq + ro, ok ? 16 : 0);
+      cp_async16(smem_u32(&sda[b][s][c]), rda + ro, ok ? 16 : 0);
+    }
+    if (threadIdx.x < TS) {
+      const long t = tt + threadIdx.x;
+      const bool ok = t <= ts_hi;
+      const size_t ro = ok ? (((size_t)l * Dr + t % Dr) * n + i) * H + h : 0;
+      bw_cp4(smem_u32(&slse[b][threadIdx.x]), rlse + ro, ok ? 4 : 0);
+      bw_cp4(smem_u32(&sD[b][threadIdx.x]), rD + ro, ok ? 4 : 0);
+    }
+    cp_async_commit();
+  };
   for (long pc = p_lo; pc <= p_hi; pc += NW * PPW) {
     const long p0 = pc + warp * PPW;
     float kk[PPW][8], vv[PPW][8], dk[PPW][8], dv[PPW][8];
@@ -722,25 +748,17 @@ __global__ void __launch_bounds__(128, 4)
     }
     const long pe = pc + NW * PPW - 1 < p_hi ? pc + NW * PPW - 1 : p_hi;
     const long ts_lo = t_lo > pc ? t_lo : pc, ts_hi = t_hi < pe + W - 1 ? t_hi : pe + W - 1;
-    for (long tt = ts_lo; tt <= ts_hi; tt += TS) {
-      __syncthreads();
-      for (int x = threadIdx.x; x < TS * DH / 4; x += blockDim.x) {
-        const int s = x / (DH / 4), c = (x % (DH / 4)) * 4;
-        const long t = tt + s;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-        if (t <= ts_hi) {
-          const size_t ro = (((size_t)l * Dr + t % Dr) * n + i) * d + h * DH + c;
-          a = *reinterpret_cast<const float4 *>(rq + ro);
-          b = *reinterpret_cast<const float4 *>(rda + ro);
-        }
-        *reinterpret_cast<float4 *>(&sq[s][c]) = a;
-        *reinterpret_cast<float4 *>(&sda[s][c]) = b;
-      }
-      if (threadIdx.x < TS) {
-        const long t = tt + threadIdx.x;
-        const size_t ro = (((size_t)l * Dr + t % Dr) * n + i) * H + h;
-        slse[threadIdx.x] = t <= ts_hi ? rlse[ro] : 0.f;
-        sD[threadIdx.x] = t <= ts_hi ? rD[ro] : 0.f;
+    const int ntile = ts_lo <= ts_hi ? (int)((ts_hi - ts_lo) / TS + 1) : 0;
+    __syncthreads();  // the previous pass's readers are done with both buffers
+    if (ntile > 0) load_tile(0, ts_lo, ts_hi);
+    for (int tk = 0; tk < ntile; tk++) {
+      const int b = tk & 1;
+      const long tt = ts_lo + (long)tk * TS;
+      if (tk + 1 < ntile) {
+        load_tile(b ^ 1, tt + TS, ts_hi);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
       }
       __syncthreads();
 #pragma unroll
@@ -750,8 +768,8 @@ __global__ void __launch_bounds__(128, 4)
         float qs[8], das[8];
 #pragma unroll
         for (int e = 0; e < 8; e++) {
-          qs[e] = sq[s][sl * 8 + e];
-          das[e] = sda[s][sl * 8 + e];
+          qs[e] = sq[b][s][sl * 8 + e];
+          das[e] = sda[b][s][sl * 8 + e];
         }
 #pragma unroll
         for (int u = 0; u < PPW; u++) {
@@ -765,7 +783,7 @@ __global__ void __launch_bounds__(128, 4)
           dot = bw_group_sum<LPK>(dot);
           dp = bw_group_sum<LPK>(dp);
           if (p <= p_hi && t <= ts_hi && t >= p && t <= p + W - 1) {
-            const float P = expf(dot * scale - slse[s]), ds = P * (dp - sD[s]);
+            const float P = expf(dot * scale - slse[b][s]), ds = P * (dp - sD[b][s]);
 #pragma unroll
             for (int e = 0; e < 8; e++) {
               dk[u][e] += scale * ds * qs[e];
@@ -774,6 +792,7 @@ __global__ void __launch_bounds__(128, 4)
           }
         }
       }
+      __syncthreads();  // buffer b is free for the tile after next
     }
 #pragma unroll
     for (int o = LPK; o < 32; o <<= 1)
