@@ -4,19 +4,19 @@
 // encoder outputs, memory and rotary table.
 #pragma once
 
+// The traversal's schedule (groups, batches, SWA ranges) is bptt_plan.h's.
 // Steps whose weight gradients one GEMM reduces (bf16 models): each step's
 // bf16 operands of the weight-gradient products (activations and output
 // gradients, transposed) land in column block `slot` of a group buffer, and
 // one tile GEMM per weight and group reduces over group x batch rows (32
 // steps: 8 left the GEMMs' fixed cost a visible share of the step).
-constexpr int BW_GROUP = 32;
+constexpr int BW_GROUP = rlt_bw::GROUP;
 
-// Steps whose forward the reverse traversal recomputes as one batch: a step's
-// recompute reads only recorded values (s_{t-1}, the recorded keys and
-// values, e_t), so up to BW_RECOMP steps of a group run their forward GEMMs
-// and attention as one launch over BW_RECOMP x n rows, before their backward
-// steps run one at a time.
-constexpr int BW_RECOMP = 8;
+// Steps whose forward the reverse traversal recomputes as one batch: up to
+// BW_RECOMP steps of a group run their forward GEMMs and attention as one
+// launch over BW_RECOMP x n rows, before their backward steps run one at a
+// time.
+constexpr int BW_RECOMP = rlt_bw::RECOMP;
 
 // Workspace of one rlt_backward call: n rows, NS steps. Offsets in bytes.
 struct BwLayout {
@@ -112,7 +112,7 @@ size_t bw_layout(const rlt_config &c, int n, int NS, BwLayout *B) {
   B->xda = take(L * S * N * d * 4);
   B->xlse = take(L * S * N * H * 4);
   B->xD = take(L * S * N * H * 4);
-  B->Dr = BW_RECOMP + (int)W;
+  B->Dr = rlt_bw::record_slots((int)W);
   B->rec = take(L * B->Dr * N * (2 * d + 2 * H) * 4);
   // bf16 models: transposed weights, the row-major bf16 operands (forward:
   // BW_RECOMP x n rows; gradients: n_pad rows), the group buffers of the
@@ -502,19 +502,17 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
 
   // Gradient terms of the SWA keys at positions p_lo .. p_hi from the saved
   // values of steps t_lo .. t_hi (already differentiated), every layer.
-  auto swa_dkv = [&](long p_lo, long p_hi, long t_lo, long t_hi) -> cudaError_t {
-    if (p_lo < 0) p_lo = 0;
-    if (p_lo < t_lo - Wm1) p_lo = t_lo - Wm1;
-    if (p_lo > p_hi || t_lo > t_hi) return cudaSuccess;
-    return launch_k(k_bw_swa_dkv<T, DH>, LD * n * H, 128, 0, st, n, H, W, Dr, p_lo, p_hi, t_lo,
-                    t_hi, hist0, B.P, (const T *)kv_hist, (const float *)rq,
+  auto swa_dkv = [&](const rlt_bw::Range &r) -> cudaError_t {
+    if (r.empty()) return cudaSuccess;
+    return launch_k(k_bw_swa_dkv<T, DH>, LD * n * H, 128, 0, st, n, H, W, Dr, r.p_lo, r.p_hi,
+                    r.t_lo, r.t_hi, hist0, B.P, (const T *)kv_hist, (const float *)rq,
                     (const float *)rda, (const float *)rlse, (const float *)rD, scale, dring);
   };
 
-  // Backward of step k, batch step s, in the batch whose first step is
-  // k_batch; its gradient operands transposed into the group's column block
-  // `slot`.
-  int k_batch = 0;
+  // Backward of step k, batch step s; the SWA's direct key terms go to
+  // positions >= p_direct (the batch's); its gradient operands are
+  // transposed into the group's column block `slot`.
+  long p_direct = t0;
   auto backward = [&](int k, int s) -> cudaError_t {
     const long t = t0 + k;
     float *rf = rbuf(LD, 0, s);
@@ -567,7 +565,7 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
       const size_t ro = ((size_t)l * Dr + t % Dr) * nd, rs = ((size_t)l * Dr + t % Dr) * n * H;
       RLT_TRY(launch_k(k_bw_attn_bwd<T, DH, true>, n * H, 32 * BW_ATT_WARPS, 0, st, n, H, swa,
                        p_lo, p_hi, scale, q1, a1, layH(S.lse1, l, s), S.dtmp, S.dq,
-                       dring, W, hist0, t0 + k_batch, rq + ro, rda + ro, rlse + rs, rD + rs,
+                       dring, W, hist0, p_direct, rq + ro, rda + ro, rlse + rs, rD + rs,
                        (bf16 *)nullptr));
       RLT_TRY(launch_k(k_bw_qkv_grad, bw_blocks((long)n * d / 2), 256, 0, st, n, H, DH, W, t,
                        rope, S.dq, dring + (size_t)l * n * 2 * d * W, S.dqkv, nb(o.dqkv)));
@@ -596,33 +594,28 @@ cudaError_t bw_impl(rlt_model *M, const int32_t *ids, int n, int NS, const float
   };
 
   // Groups in processing order (t descending), the partial one first so a
-  // group's column pitch is known when it starts; each group in batches of
-  // up to R steps, recomputed together, then differentiated one by one.
-  for (int k = NS - 1; k >= 0;) {
-    const int done = NS - 1 - k;
-    cnt = done == 0 && NS % BW_GROUP ? NS % BW_GROUP : BW_GROUP;
-    slot = 0;
-    while (slot < cnt) {
-      const int rbs = std::min(R, cnt - slot), k_lo = k - rbs + 1;
-      RLT_TRY(recompute(k_lo, rbs));
-      // the batch's SWA keys take the terms of the steps after it
-      RLT_TRY(swa_dkv(t0 + k_lo, t0 + k, t0 + k + 1, t1 - 1));
-      k_batch = k_lo;
-      // the batch's forward operands into column blocks slot .. slot+rbs-1
-      // (step k_lo + s into block slot + rbs - 1 - s, the order it is
-      // differentiated in)
-      if (TC)
-        RLT_TRY(launch_k(k_bw_grp_transpose, dim3(32 * rbs, (unsigned)trf.size()), dim3(32, 8),
-                         0, st, trf_dev, n, n_pad, rbs, (long)cnt * n_pad, (long)slot));
-      for (int s = rbs - 1; s >= 0; s--, slot++) RLT_TRY(backward(k_lo + s, s));
-      k = k_lo - 1;
-    }
-    RLT_TRY(flush());
+  // group's column pitch is known when it starts; each group in batches,
+  // recomputed together, then differentiated one by one.
+  for (const rlt_bw::Batch &bt : rlt_bw::batches(NS)) {
+    cnt = bt.cnt;
+    slot = bt.slot0;
+    RLT_TRY(recompute(bt.k_lo, bt.rbs));
+    // the batch's SWA keys take the terms of the steps after it
+    RLT_TRY(swa_dkv(rlt_bw::batch_range(t0, t1, bt, W)));
+    p_direct = rlt_bw::direct_from(t0, bt);
+    // the batch's forward operands into column blocks slot0 .. slot0+rbs-1
+    // (step k_lo + s into block slot0 + rbs - 1 - s, the order it is
+    // differentiated in)
+    if (TC)
+      RLT_TRY(launch_k(k_bw_grp_transpose, dim3(32 * bt.rbs, (unsigned)trf.size()), dim3(32, 8),
+                       0, st, trf_dev, n, n_pad, bt.rbs, (long)cnt * n_pad, (long)slot));
+    for (int s = bt.rbs - 1; s >= 0; s--, slot++) RLT_TRY(backward(bt.k_lo + s, s));
+    if (bt.last_of_group) RLT_TRY(flush());
   }
   // the state entering the chunk (the window's keys before t0 take the
   // terms of the chunk's steps first)
   if (carry_out) {
-    RLT_TRY(swa_dkv(t0 - Wm1, t0 - 1, t0, t1 - 1));
+    RLT_TRY(swa_dkv(rlt_bw::final_range(t0, t1, W)));
     k_bw_carry<<<bw_blocks((long)n * d * (1 + 2L * LD * Wm1)), 256, 0, st>>>(
         n, LD, H, DH, W, t0, carry_out, S.dcarry, dring, 1);
     RLT_TRY(cudaGetLastError());

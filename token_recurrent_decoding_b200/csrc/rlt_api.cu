@@ -29,6 +29,7 @@
 #include "gemm_dec.cuh"
 #include "step_fused.cuh"
 #include "bptt.cuh"
+#include "bptt_plan.h"
 
 using namespace rlt;
 
