@@ -566,11 +566,8 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, 8)
 // one lane group); older keys take this step's terms later, from the saved
 // values. The two forms are separate instantiations so the
 // cross-attention's loop, the long one, carries no ring registers.
-#ifndef BW_XU
-#define BW_XU 2  // keys per lane group in flight in the cross-attention backward
-#endif
 template <typename T, int DH, bool RING>
-__global__ void __launch_bounds__(32 * BW_ATT_WARPS, RING || BW_XU > 2 ? 6 : 8)
+__global__ void __launch_bounds__(32 * BW_ATT_WARPS, RING ? 6 : 8)
     k_bw_attn_bwd(int n, int H, BwKeys<T> keys, int j_lo, int j_hi, float scale,
                   const float *__restrict__ q, const float *__restrict__ a,
                   const float *__restrict__ lse, const float *__restrict__ da,
@@ -600,7 +597,7 @@ __global__ void __launch_bounds__(32 * BW_ATT_WARPS, RING || BW_XU > 2 ? 6 : 8)
                         : nullptr;
   float *dv_ring = RING ? dk_ring + (size_t)W * DH : nullptr;
   constexpr int S = BW_ATT_WARPS * KPW;  // keys per CTA pass
-  constexpr int U = RING ? 2 : BW_XU;     // passes per iteration (loads in flight)
+  constexpr int U = 2;                    // passes per iteration (loads in flight)
   for (int base = j_lo + warp * KPW; base <= j_hi; base += U * S) {
     BwRaw8<T> kv2[U], vv2[U];
     float dot2[U], dp2[U];
