@@ -21,7 +21,7 @@ SMALL = {
                                        vocab=512, window=8),
 }
 
-# Tolerances (north-star): step-wise max|err| / RMS(s), trajectory rel-L2 of s.
+# Parity tolerances: step-wise max|err| / RMS(s), trajectory rel-L2 of s.
 STEP_TOL = {configs.F32: 1e-5, configs.BF16: 2e-2}
 TRAJ_TOL = {configs.F32: 1e-4, configs.BF16: 5e-2}
 # newest K/V entries written by one step (bf16: one storage rounding on top)

@@ -4,7 +4,7 @@ pinned by finite differences of the C oracle).
 
 The oracle is fed the GPU's own encoder output e (so the encoder's rounding
 is not charged to the backward) and the same upstream gradients. Per
-gradient tensor the bar is the spec trajectory tolerance, as a
+gradient tensor the bar is the trajectory tolerance of the forward parity, as a
 relative L2 error: the gradient is a smooth function of the trajectory, and
 the GPU's trajectory is the product forward's (bf16 storage of K/V, memory
 and GEMM inputs for bf16 models), within that tolerance of the oracle's.
