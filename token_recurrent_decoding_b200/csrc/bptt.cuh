@@ -11,22 +11,26 @@
 //
 // Reverse traversal over a chunk of positions t0 .. t1-1: the forward of the
 // chunk runs first on the product step kernels while s_t and every layer's
-// (k_t, v_t) are recorded; then for t = t1-1 down to t0 one step's forward is
-// recomputed from (s_{t-1}, the recorded keys and values, e_t, M<=t) keeping
-// its activations, and the step is differentiated layer by layer in reverse.
-// The gradient of a key/value entry accumulates in a ring of W slots per
-// (layer, row, head) and is complete once step t has run (steps t .. t+W-1
-// read it); the cross-attention's gradient into the memory rows does not
-// feed back into the recurrence, so it is formed after the traversal from
-// the saved queries, output gradients and softmax statistics, as the
-// key/value half of a causal attention backward, then pushed through the
-// memory projection into e.
+// (k_t, v_t) are recorded; then for t = t1-1 down to t0 (in batches of up to
+// eight steps, bptt_plan.h) the forward is recomputed from (s_{t-1}, the
+// recorded keys and values, e_t, M<=t) keeping the activations, and each
+// step is differentiated layer by layer in reverse. The gradient of a
+// key/value entry collects in a ring of W slots per (layer, row, head) and
+// is complete once step t has run (steps t .. t+W-1 attend to it): a step
+// adds its terms directly to the keys of its batch, and k_bw_swa_dkv adds
+// the other keys' terms from the values each step saves. The
+// cross-attention's gradient into the memory rows does not feed back into
+// the recurrence, so it is formed after the traversal from the saved
+// queries, output gradients and softmax statistics, as the key/value half of
+// a causal attention backward, then pushed through the memory projection
+// into e.
 //
 // Arithmetic: the projections of bf16 models run on the tcgen05 tensor cores
-// (decode GEMMs for the recomputed forward and the activation gradients, with
-// the weights transposed once per call; tile GEMMs for the weight gradients,
-// reduced over the batch rows), their operands rounded to bf16 and fp32
-// accumulation, as the forward does; fp32 models use the SIMT GEMM below.
+// (the recomputed forward's GEMMs over a batch's rows, decode GEMMs for the
+// activation gradients with the weights transposed once per call; tile GEMMs
+// for the weight gradients, reduced over the batch rows), their operands
+// rounded to bf16 and fp32 accumulation, as the forward does; fp32 models
+// use the SIMT GEMM below.
 // Attention, norms, activations and every accumulation are fp32.
 #pragma once
 
